@@ -1,0 +1,67 @@
+"""Pins for the oracle's top-k search and the memory arithmetic (CPU only)."""
+import numpy as np
+import pytest
+
+import synth
+from conftest import read_golden
+from oracle import codec, memory, rotation as ro, search
+
+
+def test_topk_ties_go_to_lower_id():
+    s = np.array([[1.0, 3.0, 3.0, 2.0, 3.0, 0.5]])
+    vals, ids = search.topk_desc(s, 4)
+    np.testing.assert_array_equal(ids[0], [1, 2, 4, 3])
+    np.testing.assert_array_equal(vals[0], [3, 3, 3, 2])
+
+
+def test_topk_matches_full_sort():
+    s = np.random.default_rng(0).standard_normal((7, 500))
+    vals, ids = search.topk_desc(s, 10)
+    for i in range(7):
+        order = sorted(range(500), key=lambda j: (-s[i, j], j))[:10]
+        np.testing.assert_array_equal(ids[i], order)
+
+
+def test_recall_definition():
+    assert search.recall_at_k(np.array([[1, 2, 3], [4, 5, 6]]), np.array([[3, 2, 9], [7, 8, 9]])) == pytest.approx((2 / 3 + 0) / 2)
+
+
+def test_search_recall_rises_with_bits():
+    d, N, nq = 96, 3000, 30
+    U = synth.haar_basis(d, 77)
+    db = synth.anisotropic(N, d, 77, basis=U)
+    qs = synth.anisotropic(nq, d, 78, basis=U)
+    _, exact = search.exact_mips_topk(qs, db, 10)
+    rec = []
+    for bits in (1, 3):
+        rot = ro.build_rotation(d, bits, synth.rotation_randomness(d, 5, dense=True), "dense")
+        e = codec.encode(rot, db)
+        codes = codec.pack_planes(e["codes"], bits)
+        signs = codec.pack_bits(e["signs"])
+        norms = np.stack([e["norm"], e["rnorm"]], 1)
+        sc = search.search_scores(rot, qs, codes, signs, norms)
+        _, ids = search.topk_desc(sc, 10)
+        rec.append(search.recall_at_k(ids, exact))
+    assert rec[0] < rec[1]
+    assert rec[1] > 0.5
+
+
+def test_esm2_fp32_cache_is_330_mib():
+    g = {r[0]: float(r[1]) for r in read_golden("turboesm_memory.txt")}
+    L, H, d, T = int(g["layers"]), int(g["heads"]), int(g["head_dim"]), int(g["tokens"])
+    fp32_bytes = L * H * T * d * 2 * 4
+    assert fp32_bytes == 346_030_080
+    assert fp32_bytes / 2 ** 20 == pytest.approx(g["baseline_MB"])
+
+
+def test_packed_layout_ratio():
+    # this layout at d = 64, 2-bit codes + 1-bit QJL: 16 + 8 + 8 = 32 bytes per
+    # vector against 256 bytes of float32 -> 8.0x (the page quotes 7.1x and
+    # 3.125 bits/element; the three are not mutually consistent)
+    assert memory.record_bytes(64, 2) == 32
+    packed = memory.cache_bytes(33, 20, 1024, 64, 2)
+    assert packed == 43_253_760
+    assert 346_030_080 / packed == pytest.approx(8.0)
+    g = {r[0]: float(r[1]) for r in read_golden("turboesm_memory.txt")}
+    # the printed MB figures are rounded (47 MB: 46.5..47.5 -> 6.95..7.10x)
+    assert g["baseline_MB"] / g["packed_MB"] == pytest.approx(g["ratio"], abs=0.1)
