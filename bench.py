@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""Decode-attention throughput over a packed 3-bit (2+1) KV cache.
+
+Workload (default): Llama-3.1-8B-shaped GQA decode - 32 layers, batch 16,
+32 query heads over 8 KV heads, head_dim 128, 32768 cached tokens per
+sequence, bf16 heavy-tailed K/V (N(0,1) + 4 outlier channels x20 per
+(layer, kv-head)), 2-bit Lloyd-Max codes + 1-bit QJL (m = 128).
+
+One step = one decode step of the whole model's attention: for every layer,
+quantize the new token's K and V into slot T-1 of each sequence
+(tq_quantize_kv) and score the query against all T cached tokens
+(tq_decode_attention: q-prep, split-KV kernel, merge).  The packed cache
+(15 GB) is far larger than L2, so no flush is needed between steps.
+
+Metric: cached tokens scored per second, one unit = one (layer, sequence,
+kv-head, token) K+V record pair scored for all 4 query heads of its group.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+workload (the path shards by sequence with no exchange: weak scaling), the
+elapsed device time is the max over ranks and rank 0 prints the JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+WORKLOAD = "llama31_8b_gqa_decode"
+METRIC = "cached tokens scored/s (decode attn, 3-bit KV); % of B200 HBM roofline"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--bits", type=int, default=2, help="Lloyd-Max code bits (QJL adds 1)")
+    ap.add_argument("--layers", type=int, default=None, help="override layer count (testing only)")
+    ap.add_argument("--context", type=int, default=None, help="override context length (testing only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def shape(args):
+    c = dict(__import__("synth").CONFIGS[WORKLOAD])
+    if args.layers:
+        c["layers"] = args.layers
+    if args.context:
+        c["tokens"] = args.context
+    return c
+
+
+def config_json(c, args, world):
+    return {"workload": WORKLOAD, "layers": c["layers"], "batch": c["batch"], "q_heads": c["q_heads"],
+            "kv_heads": c["kv_heads"], "head_dim": c["head_dim"], "context": c["tokens"],
+            "bits": f"{args.bits}+1", "qjl_m": c["head_dim"], "kv_dtype_in": "bf16",
+            "cache_bytes_per_step": c["layers"] * c["batch"] * c["kv_heads"] * c["tokens"] * 2 * rec_bytes(c, args),
+            "l2": "inputs larger than L2 (packed cache per layer >> 126 MB); no flush",
+            "parallelism": f"replicas x{world} (weak)" if world > 1 else "single GPU"}
+
+
+def rec_bytes(c, args):
+    d = c["head_dim"]
+    return args.bits * d // 8 + d // 8 + 8
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- oracle baseline
+def oracle_baseline(c, args, budget_s=12.0, max_steps=None):
+    """Time the oracle decode on a bounded sample: one (layer, sequence,
+    kv-head) slice of the workload per step, on the host cores."""
+    import synth
+    from oracle import attention as at
+    from oracle import codec, rotation as ro
+    d, T, G = c["head_dim"], c["tokens"], c["q_heads"] // c["kv_heads"]
+    rk = ro.build_rotation(d, args.bits, synth.rotation_randomness(d, c["seed"]), rope_base=c["rope_base"])
+    rv = ro.build_rotation(d, args.bits, synth.rotation_randomness(d, c["seed"] + 7777))
+    k = synth.heavy_tailed((1, 1, T, d), [c["seed"], 1]).reshape(T, d)
+    v = synth.heavy_tailed((1, 1, T, d), [c["seed"], 2]).reshape(T, d)
+    q = synth.heavy_tailed((1, G, d), [c["seed"], 3])
+
+    def packed(rot, x, pos):
+        e = codec.encode(rot, x, pos)
+        return (codec.pack_planes(e["codes"], rot.bits)[None, None], codec.pack_bits(e["signs"])[None, None],
+                np.stack([e["norm"], e["rnorm"]], 1).astype(np.float32)[None, None])
+
+    kc, vc = packed(rk, k, np.arange(T)), packed(rv, v, None)
+    times = []
+    t_start = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        at.decode_attention(rk, rv, q, [T - 1], kc, vc, 1 / np.sqrt(d))
+        times.append(time.perf_counter() - t0)
+        if (max_steps and len(times) >= max_steps) or (not max_steps and time.perf_counter() - t_start > budget_s):
+            break
+    per = float(np.mean(times[1:] if len(times) > 1 else times))
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    return {"value": T / per, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"1 layer x 1 sequence x 1 kv-head ({T} tokens, {G} query heads) per step, "
+                      f"{len(times)} steps, {per:.3f} s/step; float64 NumPy"}, len(times), per
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    c = shape(args)
+    steps, warm = args.steps, args.warmup
+    base, n, per = oracle_baseline(c, args, max_steps=steps + warm)
+    line = {"metric": METRIC, "value": base["value"], "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": warm, "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": config_json(c, args, world), "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    c = shape(args)
+    L, B, Hq, Hkv, d, T = c["layers"], c["batch"], c["q_heads"], c["kv_heads"], c["head_dim"], c["tokens"]
+    seed = c["seed"] + 100 * rank
+    bits = args.bits
+    # ---- build: per-layer handles and packed caches ------------------------
+    rks, rvs, kcs, vcs, qs, nks, nvs = [], [], [], [], [], [], []
+    qpos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    for layer in range(L):
+        rk = tq.Rotation(d, bits, synth.rotation_randomness(d, [seed, layer, 1]), rope_base=c["rope_base"],
+                         rope_max_pos=T)
+        rv = tq.Rotation(d, bits, synth.rotation_randomness(d, [seed, layer, 2]))
+        kc = tq.empty_records(rk, (B, Hkv, T), dev)
+        vc = tq.empty_records(rv, (B, Hkv, T), dev)
+        x = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, layer, 3], dev)
+        tq.quantize_kv(rk, x, apply_rope=True, pos_period=T, out=kc)
+        del x
+        x = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, layer, 4], dev)
+        tq.quantize_kv(rv, x, out=vc)
+        del x
+        rks.append(rk)
+        rvs.append(rv)
+        kcs.append(kc)
+        vcs.append(vc)
+        qs.append(synth.heavy_tailed_torch((B, Hq, d), [seed, layer, 5], dev))
+        nks.append(synth.heavy_tailed_torch((B, Hkv, 1, d), [seed, layer, 6], dev).view(B * Hkv, d))
+        nvs.append(synth.heavy_tailed_torch((B, Hkv, 1, d), [seed, layer, 7], dev).view(B * Hkv, d))
+    ws = tq.alloc_workspace(tq.decode_workspace_size(rks[0], rvs[0], B, Hq, Hkv, T), dev)
+    outs = [torch.empty((B, Hq, d), dtype=torch.float32, device=dev) for _ in range(L)]
+    torch.cuda.synchronize()
+
+    def slot(cache):
+        return tuple(a[:, :, T - 1] for a in cache)
+
+    def step(prof=None, src=None):
+        for layer in range(L):
+            nk = nks[layer] if src is None else src[0][layer]
+            nv = nvs[layer] if src is None else src[1][layer]
+            q = qs[layer] if src is None else src[2][layer]
+            tq.quantize_kv(rks[layer], nk, apply_rope=True, pos_period=1, pos_offset=T - 1,
+                           out=slot(kcs[layer]), out_stride=T)
+            tq.quantize_kv(rvs[layer], nv, out=slot(vcs[layer]), out_stride=T)
+            if prof is not None:
+                tq.profile_next_decode(*prof[layer])
+            tq.decode_attention(rks[layer], rvs[layer], q, qpos, kcs[layer], vcs[layer], T, out=outs[layer],
+                                workspace=ws)
+
+    launches_per_step = L * (2 + 3)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- device-timed region -------------------------------------------------
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    prof = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+            for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(args.steps):
+        step(prof[s])
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = e0.elapsed_time(e1)
+    split_ms = [a.elapsed_time(b) for row in prof for (a, b) in row]
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    tokens_per_step = L * B * Hkv * T
+    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+
+    # ---- end-to-end through the public API with host buffers ----------------
+    host_in = ([torch.empty_like(x, device="cpu").pin_memory().copy_(x.cpu()) for x in nks],
+               [torch.empty_like(x, device="cpu").pin_memory().copy_(x.cpu()) for x in nvs],
+               [torch.empty_like(x, device="cpu").pin_memory().copy_(x.cpu()) for x in qs])
+    host_out = [torch.empty((B, Hq, d), dtype=torch.float32).pin_memory() for _ in range(L)]
+    dev_in = ([torch.empty_like(x) for x in nks], [torch.empty_like(x) for x in nvs], [torch.empty_like(x) for x in qs])
+    h2d = sum(x.numel() * x.element_size() for group in host_in for x in group)
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        for g in range(3):
+            for a, b in zip(dev_in[g], host_in[g]):
+                a.copy_(b, non_blocking=True)
+        step(src=dev_in)
+        for a, b in zip(host_out, outs):
+            a.copy_(b, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = f0.elapsed_time(f1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * tokens_per_step * args.steps / (e2e_ms / 1e3)
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peaks()
+    bytes_per_launch = B * Hkv * T * 2 * rec_bytes(c, args)
+    split_avg_s = float(np.mean(split_ms)) / 1e3
+    achieved = bytes_per_launch / split_avg_s / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "decode_split_kernel (one launch per layer)",
+                "algorithmic_bytes_per_launch": bytes_per_launch, "peak_source": peak_kind,
+                "launch_ms_avg": round(split_avg_s * 1e3, 4)}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_json(c, args, world),
+            "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "clocks": clk}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(c, args)[0]
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+/*
+ * tq.h - C ABI of the B200 rotation + Lloyd-Max + QJL vector codec.
+ *
+ * The codec (TurboQuant-style; sources named per entry point):
+ *   encode:  RoPE (keys only) -> rotation Pi -> per-coordinate b-bit
+ *            Lloyd-Max code + vector norm -> 1-bit QJL sketch sign(S r) of
+ *            the residual r plus ||r||, bit-packed;
+ *   decode:  attention scored straight from the packed cache, one pass.
+ *
+ * Conventions for every entry point:
+ *   - All pointers named "device" are CUDA device pointers on the device the
+ *     handle was built on; "host" pointers are ordinary host memory.
+ *   - The caller owns every buffer it passes.  The library allocates device
+ *     memory only inside tq_build_rotation (owned by the handle, released by
+ *     tq_free_rotation).
+ *   - Calls that launch kernels are asynchronous on `stream` (a cudaStream_t
+ *     passed as void*; NULL = legacy default stream).  Arguments are checked
+ *     on the host before anything is launched; a rejected call launches
+ *     nothing and returns a negative status.  Launch failures return
+ *     TQ_ECUDA; faults inside a kernel surface at the caller's next
+ *     synchronisation, as with any CUDA call.
+ *   - Nothing is thrown across the ABI.  Handles are immutable after build
+ *     and may be shared between threads and streams.
+ *
+ * Packed record of one vector (bits b, dimension d, sketch size m):
+ *   codes  b*d/8 bytes: b bit-planes of d bits, plane k holds bit k of every
+ *          code; coordinate i at byte i/8, bit i%8; planes in order k=0..b-1.
+ *          Codes number the Lloyd-Max levels in ascending order.
+ *   signs  m/8 bytes: bit j = 1 iff (S r)_j >= 0, same bit order.
+ *   norms  two float32: ||x|| (after RoPE) and ||r||.
+ * Codes, signs and norms live in three separate arrays indexed by record.
+ *
+ * Sources (pages, cited by title and section):
+ *   [TurboESM]   "TurboESM: Ultra-Efficient 3-Bit KV Cache Quantization for
+ *                Protein Language Models with Orthogonal Rotation and QJL
+ *                Correction", Résumé technique §2.A-§2.E.
+ *   [TurboQuant] TurboQuant digest (news.hada.io 27867): "Principe de
+ *                fonctionnement" (Étape 1, Étape 2), "QJL", "Expériences et
+ *                résultats".
+ *   [NSNQuant]   "NSNQuant: ...", Résumé Technique, Méthodologie §2.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define TQ_OK            0
+#define TQ_EINVAL       -1   /* bad argument (null pointer, size, alignment) */
+#define TQ_EUNSUPPORTED -2   /* valid but not implemented (d, bits, heads)   */
+#define TQ_EWORKSPACE   -3   /* workspace missing or too small               */
+#define TQ_ECUDA        -4   /* a CUDA runtime call or launch failed         */
+#define TQ_ENOMEM       -5   /* device allocation failed                     */
+
+/* ---- enumerations ------------------------------------------------------ */
+#define TQ_ROT_HADAMARD  0   /* Pi = H_d diag(D) / sqrt(d), d a power of two */
+#define TQ_ROT_DENSE     1   /* Pi = Q diag(sign(diag R)), G = QR, any d     */
+
+#define TQ_F32           0   /* float32 elements */
+#define TQ_BF16          1   /* bfloat16 elements */
+
+typedef struct tq_rotation tq_rotation;
+
+/* Human-readable text for a status code (static storage). */
+const char* tq_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int tq_version(void);
+
+/*
+ * tq_lloyd_max - host only; the scalar codebook the codec uses.
+ * [TurboQuant] "Principe", Étape 1 and comments: after a random rotation a
+ * standard quantizer, its boundaries and levels optimised by Lloyd-Max, is
+ * applied to each coordinate.  The law quantized is the exact density of one
+ * coordinate of a uniform point on S^{d-1}, f(t) ~ (1-t^2)^((d-3)/2).
+ *   d           dimension, 3 <= d <= 65536
+ *   bits        1..8
+ *   levels      host out [2^bits] ascending reconstruction levels (float64)
+ *   thresholds  host out [2^bits - 1], thresholds[j] = (levels[j]+levels[j+1])/2
+ * Returns TQ_OK or TQ_EINVAL.  Pure host computation; needs no GPU.
+ */
+int tq_lloyd_max(int d, int bits, double* levels, double* thresholds);
+
+/*
+ * tq_build_rotation - build a codec handle on the current CUDA device.
+ * [TurboQuant] Étape 1 (data-oblivious random rotation), [NSNQuant] §2
+ * (randomized Hadamard), [TurboQuant] "QJL" (Gaussian projection S),
+ * [TurboESM] §2.A (RoPE before the rotation).
+ *   d          vector dimension; TQ_ROT_HADAMARD needs d in {64, 128};
+ *              TQ_ROT_DENSE takes any multiple of 32 up to 4096.
+ *   code_bits  Lloyd-Max code bits per coordinate, 1..3.
+ *   kind       TQ_ROT_HADAMARD or TQ_ROT_DENSE.
+ *   signs      host [d] int8 of +1/-1 (the Hadamard sign diagonal D);
+ *              required for TQ_ROT_HADAMARD, ignored otherwise.
+ *   gauss_pi   host [d*d] float64 row-major Gaussian draws whose QR factor
+ *              (sign-fixed) is Pi; required for TQ_ROT_DENSE, else ignored.
+ *   gauss_s    host [m*d] float32 row-major N(0,1) draws; each is rounded to
+ *              the nearest bf16-representable value to form S.
+ *   m          QJL sketch size; must equal d.
+ *   rope_base  RoPE base (e.g. 10000); 0 disables RoPE for this handle.
+ *   rope_max_pos  positions 0..rope_max_pos-1 are supported (ignored when
+ *              rope_base is 0); at most 2^31.
+ *   out        receives the handle.
+ * The random draws are inputs so that every generator stays outside the
+ * library.  Builds the codebook (tq_lloyd_max), Pi, S and two-level RoPE
+ * tables on the host in float64 and uploads them.  Synchronous.
+ * Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM or TQ_ECUDA.
+ */
+int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
+                      const double* gauss_pi, const float* gauss_s, int m,
+                      double rope_base, int64_t rope_max_pos, tq_rotation** out);
+
+/* Release a handle and its device memory (NULL is accepted). */
+int tq_free_rotation(tq_rotation* h);
+
+/*
+ * tq_rotation_export - copy the handle's tables to the host (for checks).
+ *   pi          host out [d*d] float32 row-major Pi (y = Pi u), or NULL
+ *   s           host out [m*d] float32 row-major S, or NULL
+ *   levels      host out [2^bits] float64, or NULL
+ *   thresholds  host out [2^bits - 1] float64, or NULL
+ * Synchronous.  Returns TQ_OK, TQ_EINVAL or TQ_ECUDA.
+ */
+int tq_rotation_export(const tq_rotation* h, float* pi, float* s,
+                       double* levels, double* thresholds);
+
+/* Record geometry of a handle: d, m, bits and bytes of codes / signs. */
+int tq_rotation_dims(const tq_rotation* h, int* d, int* m, int* bits,
+                     int64_t* code_bytes, int64_t* sign_bytes);
+
+/*
+ * tq_quantize_kv - encode n vectors into packed records.
+ * [TurboESM] §2.A (RoPE first), [TurboQuant] Étape 1 (rotate, quantize each
+ * coordinate, keep the norm) and Étape 2 + "QJL" (sign bits of S r and ||r||),
+ * [TurboESM] §2.D (residual r = x - x_hat), §3 (quantize + pack at prefill).
+ *   h           handle (d, bits, Pi, S, codebook, RoPE tables)
+ *   x           device [n, ld] elements of `dtype` (TQ_F32 or TQ_BF16); row i
+ *               is the vector; ld >= d, ld % 8 == 0 for bf16, % 4 for f32
+ *   n           number of vectors (0 is a no-op)
+ *   pos         device [n] int64 positions, or NULL
+ *   pos_period, pos_offset   with pos == NULL, row i sits at position
+ *               pos_offset + (i mod pos_period)
+ *   apply_rope  nonzero: rotate by RoPE at the row's position before Pi
+ *               (needs a handle built with rope_base > 0 and every position
+ *               in [0, rope_max_pos))
+ *   codes, signs, norms  device outputs; row i is written to record
+ *               i * out_stride of each array (records of code_bytes,
+ *               sign_bytes and 2 floats); codes and signs 4-byte aligned,
+ *               norms 8-byte aligned
+ *   out_stride  records between consecutive output rows (>= 1)
+ * Positions out of range write NaN norms for that row (a host-given
+ * pos_period/pos_offset out of range is rejected with TQ_EINVAL instead).
+ */
+int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, int64_t n,
+                   int64_t ld, const int64_t* pos, int64_t pos_period,
+                   int64_t pos_offset, int apply_rope, uint8_t* codes,
+                   uint8_t* signs, float* norms, int64_t out_stride,
+                   void* stream);
+
+/*
+ * tq_decode_attention - one decode step of attention over packed K/V caches.
+ * [TurboESM] §2.E: dequantization, residual correction, inverse rotation
+ * Pi^T and an online softmax fused in one pass over the cache;
+ * [TurboQuant] "QJL": score <q, x_hat> + ||r|| sqrt(pi/2)/m <S q, sign(S r)>.
+ *   hk, hv      handles of the K and V caches (d = 128 for both; hk carries
+ *               RoPE, hv must not apply RoPE to V - its rope base is unused)
+ *   q           device [B, Hq, d] elements of q_dtype
+ *   q_pos       device [B] int64 query positions (used when hk has RoPE)
+ *   k_codes, k_signs, k_norms, v_codes, v_signs, v_norms
+ *               device caches; sequence (b, kv-head j) occupies records
+ *               (b*Hkv + j)*cache_stride .. + T-1; all 16-byte aligned
+ *   cache_stride  records between consecutive sequences (>= T, even)
+ *   B, Hq, Hkv  batch, query heads, KV heads; Hq % Hkv == 0 and
+ *               Hq/Hkv in {1, 2, 4, 8}
+ *   T           cached tokens per sequence (0 gives an all-zero output)
+ *   scale       softmax scale (typically 1/sqrt(d))
+ *   out         device [B, Hq, d] float32
+ *   workspace   device scratch of at least tq_decode_workspace_size(...)
+ *               bytes, 256-byte aligned; contents need no initialisation
+ * Query head h reads KV head h / (Hq/Hkv).  Returns TQ_OK, TQ_EINVAL,
+ * TQ_EUNSUPPORTED, TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
+                        const void* q, int q_dtype, const int64_t* q_pos,
+                        const uint8_t* k_codes, const uint8_t* k_signs,
+                        const float* k_norms, const uint8_t* v_codes,
+                        const uint8_t* v_signs, const float* v_norms,
+                        int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
+                        float scale, float* out, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Workspace bytes tq_decode_attention needs for these sizes (0 if invalid). */
+size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
+                                int B, int Hq, int Hkv, int64_t T);
+
+/*
+ * tq_profile_next_decode - instrumentation for benchmarks.  The next
+ * tq_decode_attention call made by this host thread records `ev_begin`
+ * immediately before and `ev_end` immediately after its split-KV kernel, on
+ * that call's stream, so the caller can time the dominant kernel alone with
+ * cudaEventElapsedTime.  Both are cudaEvent_t passed as void* (created by the
+ * caller, on the handle's device); NULL, NULL cancels.  One-shot: consumed by
+ * the next call (also when that call fails).  Returns TQ_OK or TQ_EINVAL.
+ */
+int tq_profile_next_decode(void* ev_begin, void* ev_end);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

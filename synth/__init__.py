@@ -73,7 +73,7 @@ def rotation_randomness(d: int, seed: int, dense: bool = False, m: int | None = 
         is the dense rotation), else None.
     """
     m = d if m is None else m
-    g = _rng([seed, 0x5107])
+    g = _rng([*np.atleast_1d(seed).tolist(), 0x5107])
     signs = np.where(g.random(d) < 0.5, -1, 1).astype(np.int8)
     gauss_s = g.standard_normal((m, d), dtype=np.float32)
     gauss_pi = g.standard_normal((d, d)) if dense else None

@@ -1,0 +1,68 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry
+point, and its host-only codebook agrees with the oracle."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+from oracle import codebook as cb
+
+HEADER = os.path.join(ROOT, "include", "tq.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    from vector_quantization_b200 import tq
+    lib = ctypes.CDLL(tq.LIB_PATH)
+    names = _declared()
+    assert len(names) >= 10
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    from vector_quantization_b200 import tq
+    assert tq.version() >= 100
+    for code in (0, -1, -2, -3, -4, -5):
+        assert tq._lib.tq_status_string(code)
+
+
+@pytest.mark.parametrize("d,bits", [(3, 2), (64, 1), (64, 2), (128, 2), (128, 3), (1536, 1), (1536, 3)])
+def test_library_codebook_matches_oracle(d, bits):
+    from vector_quantization_b200 import tq
+    lv, th = tq.lloyd_max(d, bits)
+    olv, oth = cb.lloyd_max(d, bits)
+    # Two independent fixed-point iterations (incomplete beta by continued
+    # fraction vs scipy) stop a few 1e-12 apart: Lloyd-Max converges linearly.
+    # Thresholds that close move a code only inside the 1e-5 flag band.
+    np.testing.assert_allclose(lv, olv, rtol=1e-10, atol=1e-15)
+    np.testing.assert_allclose(th, oth, rtol=1e-10, atol=1e-15)
+
+
+def test_bad_arguments_are_rejected_on_host():
+    from vector_quantization_b200 import tq
+    lv = np.zeros(4)
+    assert tq._lib.tq_lloyd_max(2, 2, lv.ctypes.data, lv.ctypes.data) == tq.TQ_EINVAL
+    assert tq._lib.tq_lloyd_max(64, 9, lv.ctypes.data, lv.ctypes.data) == tq.TQ_EINVAL
+    h = ctypes.c_void_p()
+    g = np.zeros((64, 64), np.float32)
+    s = np.ones(64, np.int8)
+    # m != d, bits out of range, bad kind, bad signs: all rejected before any device call
+    assert tq._lib.tq_build_rotation(64, 2, 0, s.ctypes.data, None, g.ctypes.data, 32, 0.0, 0, ctypes.byref(h)) == tq.TQ_EINVAL
+    assert tq._lib.tq_build_rotation(64, 4, 0, s.ctypes.data, None, g.ctypes.data, 64, 0.0, 0, ctypes.byref(h)) == tq.TQ_EINVAL
+    assert tq._lib.tq_build_rotation(64, 2, 7, s.ctypes.data, None, g.ctypes.data, 64, 0.0, 0, ctypes.byref(h)) == tq.TQ_EINVAL
+    bad = s.copy()
+    bad[3] = 0
+    assert tq._lib.tq_build_rotation(64, 2, 0, bad.ctypes.data, None, g.ctypes.data, 64, 0.0, 0, ctypes.byref(h)) == tq.TQ_EINVAL
+    assert tq._lib.tq_build_rotation(96, 2, 0, np.ones(96, np.int8).ctypes.data, None, np.zeros((96, 96), np.float32).ctypes.data,
+                                     96, 0.0, 0, ctypes.byref(h)) == tq.TQ_EUNSUPPORTED
+    assert tq._lib.tq_decode_workspace_size(None, None, 1, 1, 1, 10) == 0
+    assert tq._lib.tq_quantize_kv(None, None, 0, 1, 64, None, 1, 0, 0, None, None, None, 1, None) == tq.TQ_EINVAL

@@ -1,0 +1,108 @@
+"""GPU parity of the handle tables and of tq_quantize_kv against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import compare_records, oracle_records, oracle_rotation
+from oracle import rotation as ro
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_rot(d, bits, seed, rope=0.0, kind="hadamard"):
+    from vector_quantization_b200 import tq
+    rnd = synth.rotation_randomness(d, seed, dense=(kind == "dense"))
+    return tq.Rotation(d, bits, rnd, kind, rope_base=rope, rope_max_pos=(1 << 20) + 8)
+
+
+@pytest.mark.parametrize("d,bits", [(64, 2), (128, 1), (128, 2), (128, 3)])
+def test_export_matches_oracle(cuda_device, d, bits):
+    g = _gpu_rot(d, bits, 21)
+    o, _ = oracle_rotation(d, bits, 21)
+    ex = g.export()
+    np.testing.assert_allclose(ex["pi"], o.pi, rtol=0, atol=1e-7)
+    np.testing.assert_array_equal(ex["s"], o.s.astype(np.float32))
+    np.testing.assert_allclose(ex["levels"], o.levels, rtol=1e-10)
+    np.testing.assert_allclose(ex["thresholds"], o.thresholds, rtol=1e-10, atol=1e-15)
+
+
+def _run_encode(d, bits, n, dtype, rope, seed, period=None, offset=0, pos_array=False, out_stride=1, scale=1.0):
+    from vector_quantization_b200 import tq
+    g = _gpu_rot(d, bits, seed, rope=10000.0 if rope else 0.0)
+    o, _ = oracle_rotation(d, bits, seed, rope=10000.0 if rope else 0.0)
+    x = synth.heavy_tailed((n, d), seed + 1) * np.float32(scale)
+    xt = torch.from_numpy(x).to(cuda_device_of()).to(dtype)
+    x_used = xt.float().cpu().numpy()
+    period = period or n
+    pos = (np.arange(n) % period + offset).astype(np.int64)
+    kw = dict(apply_rope=rope)
+    if rope:
+        if pos_array:
+            kw["pos"] = torch.from_numpy(pos).to(xt.device)
+        else:
+            kw.update(pos_period=period, pos_offset=offset)
+    if out_stride > 1:
+        out = tq.empty_records(g, (n * out_stride,), xt.device)
+        for t in out:
+            t.fill_(0)
+        tq.quantize_kv(g, xt, out=out, out_stride=out_stride, **kw)
+        gpu = tuple(t[::out_stride].cpu().numpy() for t in out)
+    else:
+        gpu = tuple(t.cpu().numpy() for t in tq.quantize_kv(g, xt, **kw))
+    torch.cuda.synchronize()
+    _, _, _, enc = oracle_records(o, x_used, pos if rope else None)
+    return compare_records(o, gpu, enc)
+
+
+def cuda_device_of():
+    return torch.device("cuda:0")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_encode_parity(cuda_device, d, bits, dtype):
+    _run_encode(d, bits, 1031, dtype, rope=True, seed=100 + bits)
+
+
+@pytest.mark.parametrize("n", [1, 7, 33, 4099])
+def test_encode_ragged_counts_no_rope(cuda_device, n):
+    _run_encode(128, 2, n, torch.float32, rope=False, seed=7)
+
+
+def test_encode_positions_period_offset_and_array(cuda_device):
+    _run_encode(128, 2, 600, torch.bfloat16, rope=True, seed=8, period=256, offset=(1 << 20) - 300)
+    _run_encode(128, 3, 600, torch.float32, rope=True, seed=9, period=600, offset=12345, pos_array=True)
+
+
+def test_encode_strided_output(cuda_device):
+    _run_encode(128, 2, 300, torch.float32, rope=True, seed=10, out_stride=3)
+
+
+@pytest.mark.parametrize("scale", [1e-10, 1e10])
+def test_encode_scale_range(cuda_device, scale):
+    _run_encode(128, 2, 200, torch.float32, rope=True, seed=11, scale=scale)
+
+
+def test_encode_zero_vectors(cuda_device):
+    from vector_quantization_b200 import tq
+    g = _gpu_rot(128, 2, 12, rope=10000.0)
+    x = torch.zeros((5, 128), device=cuda_device)
+    codes, signs, norms = tq.quantize_kv(g, x, apply_rope=True, pos_period=5)
+    torch.cuda.synchronize()
+    assert torch.all(norms == 0)
+    # every code = 2 (upper-middle): plane 0 all zero, plane 1 all ones
+    assert torch.all(codes[:, :16] == 0) and torch.all(codes[:, 16:] == 0xFF)
+    assert torch.all(signs == 0xFF)
+
+
+def test_encode_rejects_bad_arguments(cuda_device):
+    from vector_quantization_b200 import tq
+    g = _gpu_rot(128, 2, 13, rope=10000.0)
+    x = torch.zeros((4, 128), device=cuda_device)
+    with pytest.raises(tq.TQError):  # position beyond the RoPE table
+        tq.quantize_kv(g, x, apply_rope=True, pos_period=4, pos_offset=(1 << 21))
+    g2 = _gpu_rot(128, 2, 13)
+    with pytest.raises(tq.TQError):  # RoPE asked of a handle without RoPE
+        tq.quantize_kv(g2, x, apply_rope=True, pos_period=4)

@@ -1,0 +1,123 @@
+"""GPU parity of tq_decode_attention against the oracle.
+
+The caches are packed by the oracle, so both sides score the same bytes; the
+tolerance is the benchmark spec's bound |gpu - ref| <= 1e-3 + 2e-3 |ref|."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import assert_close, oracle_records, oracle_rotation
+from oracle import attention as at
+
+pytestmark = pytest.mark.gpu
+D = 128
+
+
+def _gpu_rot(bits, seed, rope):
+    from vector_quantization_b200 import tq
+    rnd = synth.rotation_randomness(D, seed)
+    return tq.Rotation(D, bits, rnd, "hadamard", rope_base=rope, rope_max_pos=(1 << 20) + 8)
+
+
+def _packed_cache(orot, x, cap, pos=None, poison=True):
+    """Oracle-packed cache [B, H, cap, ...]; records past T poisoned (0xFF
+    bytes, NaN norms) so that any read past T shows up as NaN."""
+    B, H, T, d = x.shape
+    codes, signs, norms, _ = oracle_records(orot, x.reshape(-1, d), None if pos is None else np.tile(pos, B * H))
+    def place(a, fill):
+        out = np.full((B, H, cap) + a.shape[1:], fill, dtype=a.dtype)
+        out[:, :, :T] = a.reshape(B, H, T, -1)
+        return out
+    nan = np.float32(np.nan) if poison else np.float32(0)
+    return (place(codes, 0xFF if poison else 0), place(signs, 0xFF if poison else 0), place(norms, nan))
+
+
+def _to_dev(cache, dev):
+    return tuple(torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in cache)
+
+
+def run_decode(bits, G, T, B=2, Hkv=2, q_dtype=torch.float32, seed=0, cap_pad=6, rope=10000.0):
+    from vector_quantization_b200 import tq
+    dev = torch.device("cuda:0")
+    Hq = G * Hkv
+    cap = T + cap_pad + ((T + cap_pad) & 1)   # cache_stride must be even
+    rk_o, _ = oracle_rotation(D, bits, 500 + seed, rope=rope)
+    rv_o, _ = oracle_rotation(D, bits, 600 + seed)
+    rk, rv = _gpu_rot(bits, 500 + seed, rope), _gpu_rot(bits, 600 + seed, 0.0)
+    k = synth.heavy_tailed((B, Hkv, T, D), 700 + seed)
+    v = synth.heavy_tailed((B, Hkv, T, D), 800 + seed)
+    kc = _packed_cache(rk_o, k, cap, np.arange(T))
+    vc = _packed_cache(rv_o, v, cap)
+    q = torch.from_numpy(synth.heavy_tailed((B, Hq, D), 900 + seed)).to(dev).to(q_dtype)
+    q_pos = torch.full((B,), max(T - 1, 0), dtype=torch.int64, device=dev)
+    out = tq.decode_attention(rk, rv, q, q_pos, _to_dev(kc, dev), _to_dev(vc, dev), T)
+    torch.cuda.synchronize()
+    ref = at.decode_attention(rk_o, rv_o, q.float().cpu().numpy(), [max(T - 1, 0)] * B,
+                              tuple(a[:, :, :T] for a in kc), tuple(a[:, :, :T] for a in vc), 1 / np.sqrt(D))
+    return out.cpu().numpy(), ref
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 3])
+def test_decode_parity_heads_bits(cuda_device, G, bits):
+    gpu, ref = run_decode(bits, G, 300, seed=G * 10 + bits)
+    assert_close(gpu, ref, what=f"G={G} bits={bits}")
+
+
+@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 63, 64, 65, 1000, 5000])
+def test_decode_parity_lengths(cuda_device, T):
+    gpu, ref = run_decode(2, 4, T, seed=T)
+    assert_close(gpu, ref, what=f"T={T}")
+
+
+def test_decode_bf16_query(cuda_device):
+    gpu, ref = run_decode(2, 4, 777, q_dtype=torch.bfloat16, seed=3)
+    assert_close(gpu, ref)
+
+
+def test_decode_no_rope(cuda_device):
+    gpu, ref = run_decode(3, 2, 200, seed=4, rope=0.0)
+    assert_close(gpu, ref)
+
+
+def test_decode_empty_cache(cuda_device):
+    from vector_quantization_b200 import tq
+    dev = torch.device("cuda:0")
+    rk, rv = _gpu_rot(2, 1, 10000.0), _gpu_rot(2, 2, 0.0)
+    q = torch.randn(1, 4, D, device=dev)
+    z = tq.empty_records(rk, (1, 1, 2), dev)
+    out = tq.decode_attention(rk, rv, q, torch.zeros(1, dtype=torch.int64, device=dev), z, z, 0)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+
+
+def test_tiny_workload_end_to_end(cuda_device):
+    """1 head, d 128, 1024 fp32 tokens (N(0,1) + 4 outlier channels x20),
+    RoPE base 10000 on K, 2-bit codes + 1-bit QJL (m 128), one fp32 query:
+    GPU encode + GPU decode against oracle encode + oracle decode."""
+    from vector_quantization_b200 import tq
+    dev = torch.device("cuda:0")
+    T = 1024
+    cfg = synth.CONFIGS["tiny_d128_t1024"]
+    seed = cfg["seed"]
+    rk_o, _ = oracle_rotation(D, 2, seed, rope=10000.0)
+    rv_o, _ = oracle_rotation(D, 2, seed + 50)
+    rk, rv = _gpu_rot(2, seed, 10000.0), _gpu_rot(2, seed + 50, 0.0)
+    k = synth.heavy_tailed((1, 1, T, D), seed + 1)
+    v = synth.heavy_tailed((1, 1, T, D), seed + 2)
+    q = synth.heavy_tailed((1, 1, D), seed + 3)
+    kt, vt = torch.from_numpy(k).to(dev), torch.from_numpy(v).to(dev)
+    kcache = tq.quantize_kv(rk, kt, apply_rope=True, pos_period=T)
+    vcache = tq.quantize_kv(rv, vt)
+    out = tq.decode_attention(rk, rv, torch.from_numpy(q).to(dev), torch.tensor([T - 1], device=dev), kcache,
+                              vcache, T)
+    torch.cuda.synchronize()
+    kco = _packed_cache(rk_o, k, T, np.arange(T), poison=False)
+    vco = _packed_cache(rv_o, v, T, poison=False)
+    ref = at.decode_attention(rk_o, rv_o, q, [T - 1], kco, vco, 1 / np.sqrt(D))
+    # code parity first (identical except flagged coordinates)
+    from helpers import compare_records
+    _, _, _, ek = oracle_records(rk_o, k.reshape(-1, D), np.arange(T))
+    compare_records(rk_o, tuple(t.cpu().numpy() for t in kcache), ek)
+    assert_close(out.cpu().numpy(), ref, what="tiny end-to-end")

@@ -1,0 +1,699 @@
+// Decode attention scored straight from the packed K/V cache.
+//
+// [TurboESM] §2.E: dequantization, residual correction, inverse rotation
+// Pi^T and an online softmax fused into one pass over the cache, with no
+// dequantized intermediate in memory.  [TurboQuant] "QJL": the score of a
+// key is <q~, ||k|| c[idx]> + ||r|| sqrt(pi/2)/m <S q~, sign(S r)>, q~ = Pi q.
+//
+// Three launches per call:
+//  1. qprep   - per query head: RoPE, q~ = Pi q (fast Walsh-Hadamard),
+//               s = S q~; both written as bf16 hi/lo pairs directly in the
+//               register order of the main kernel's MMA B operand.
+//  2. split   - per (sequence, token chunk): streams the packed records
+//               through shared memory (cp.async, 4-stage ring per warp),
+//               scores 16 tokens at a time and accumulates the values.
+//  3. merge   - per query head: log-sum-exp merge of the chunk partials, the
+//               QJL value correction S^T acc_s, and Pi^T.
+//
+// The contraction trick.  A b-bit code is rewritten in Walsh form,
+//   c[idx] = sum_p w_p s_p(idx),  s_p a product of the code's bits as +-1,
+// (b = 2: s_1, s_0; b = 3: s_2, s_1, s_0, s_0 s_1 s_2), and the QJL bits are
+// +-1 as they stand.  Every term of the score and of the value sum is then a
+// product of an exact +-1 matrix (built from the packed bits with one shift
+// and one LOP3 per pair of elements) and a bf16 hi/lo split of q~, S q~ or
+// the softmax weights, so the per-token dot products run on the tensor pipe
+// (mma.sync m16n8k16, fp32 accumulate) without dequantizing anything.
+//   K side:  C[token][head,piece] = sum_dim s_p[token][dim] * q~hi/lo[dim]
+//   V side:  O[dim][head,piece]   = sum_tok s_p[tok][dim] * (w_p p ||v||)hi/lo
+// All G query heads of a KV head share each streamed record (GQA).
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "tq_internal.h"
+
+namespace {
+
+constexpr int kD = 128;        // head dimension handled here
+constexpr int kWarps = 4;      // warps per CTA
+constexpr int kTile = 16;      // tokens per MMA tile
+constexpr int kStages = 4;     // cp.async ring depth per warp
+constexpr float kLazyRescale = 8.0f;  // log2 units of headroom before rescaling
+
+struct DecodeParams {
+  const uint8_t* k_codes;
+  const uint8_t* k_signs;
+  const float2* k_norms;
+  const uint8_t* v_codes;
+  const uint8_t* v_signs;
+  const float2* v_norms;
+  int64_t cache_stride;
+  int64_t T;
+  int64_t chunk;           // tokens per split (multiple of kTile)
+  int n_splits;
+  const uint32_t* qfrag;   // [BH][2][NT][8][32][2]
+  float* partial;          // [BH][n_splits][G][2 + 2 kD]
+  float score_scale;       // softmax scale * log2(e)
+  float qjl;               // sqrt(pi/2) / m
+  float walsh_k[4];
+  float walsh_v[4];
+};
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, int src_bytes) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gsrc), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two bf16 values +-1 from bits x (low half) and x+16 (high half) of w:
+// bit = 1 -> +1.0, bit = 0 -> -1.0.
+__device__ __forceinline__ uint32_t pm1_pair(uint32_t w, int x) {
+  const uint32_t t = w << (15 - x);
+  return (~t & 0x80008000u) | 0x3F803F80u;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return l | (h << 16);
+}
+
+// Piece `piece` (0 = hi, 1 = lo) of the two-term bf16 split of v.
+__device__ __forceinline__ float bf16_piece(float v, int piece) {
+  const float hi = __bfloat162float(__float2bfloat16_rn(v));
+  return piece ? v - hi : hi;
+}
+
+template <int BITS>
+struct Planes {
+  static constexpr int P = BITS == 1 ? 1 : (BITS == 2 ? 2 : 4);
+  // Walsh planes from raw bit-plane words (same element layout in all words).
+  __device__ static __forceinline__ void make(const uint32_t (&raw)[BITS], uint32_t (&out)[P]) {
+    if constexpr (BITS == 1) {
+      out[0] = raw[0];
+    } else if constexpr (BITS == 2) {
+      out[0] = raw[1];
+      out[1] = raw[0];
+    } else {
+      out[0] = raw[2];
+      out[1] = raw[1];
+      out[2] = raw[0];
+      out[3] = raw[0] ^ raw[1] ^ raw[2];  // s0 s1 s2 = +1 iff an odd number of bits are 1
+    }
+  }
+};
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams p) {
+  constexpr int NT = (2 * G + 7) / 8;
+  constexpr int P = Planes<BITS>::P;
+  constexpr int CB = BITS * kD / 8;                 // code bytes per token
+  constexpr int SB = kD / 8;                        // sign bytes per token
+  constexpr int HALF = kTile * (CB + SB + 8);       // K (or V) part of a stage
+  constexpr int STAGE = 2 * HALF;
+  extern __shared__ __align__(16) uint8_t smem[];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int bh = blockIdx.y;
+  const int split = blockIdx.x;
+  const int64_t t_begin = static_cast<int64_t>(split) * p.chunk;
+  const int64_t t_end = min(p.T, t_begin + p.chunk);
+  const int n_tiles = t_end > t_begin ? static_cast<int>((t_end - t_begin + kTile - 1) / kTile) : 0;
+  const int my_count = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
+  const int64_t seq = static_cast<int64_t>(bh) * p.cache_stride;
+
+  uint8_t* my_stages = smem + warp * kStages * STAGE;
+
+  // Loads of one tile (16 tokens) into stage `st`; records past t_end are zero-filled.
+  auto issue = [&](int i) {
+    if (i < my_count) {
+      const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
+      const int nv = static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
+      uint8_t* stg = my_stages + (i % kStages) * STAGE;
+      constexpr int CCH = kTile * CB / 16, SCH = kTile * SB / 16, NCH = kTile * 8 / 16;
+      constexpr int HCH = CCH + SCH + NCH;
+      for (int c = lane; c < 2 * HCH; c += 32) {
+        const int side = c >= HCH;
+        const int cc = c - side * HCH;
+        const uint8_t* codes = side ? p.v_codes : p.k_codes;
+        const uint8_t* signs = side ? p.v_signs : p.k_signs;
+        const float2* norms = side ? p.v_norms : p.k_norms;
+        uint8_t* dst = stg + side * HALF;
+        const void* src;
+        int bytes;
+        if (cc < CCH) {
+          const int tok = cc / (CB / 16), part = cc % (CB / 16);
+          bytes = tok < nv ? 16 : 0;
+          src = bytes ? codes + (seq + t0 + tok) * CB + part * 16 : codes;
+          dst += cc * 16;
+        } else if (cc < CCH + SCH) {
+          const int tok = (cc - CCH) / (SB / 16), part = (cc - CCH) % (SB / 16);
+          bytes = tok < nv ? 16 : 0;
+          src = bytes ? signs + (seq + t0 + tok) * SB + part * 16 : signs;
+          dst += kTile * CB + (cc - CCH) * 16;
+        } else {
+          const int tok = 2 * (cc - CCH - SCH);
+          bytes = max(0, min(2, nv - tok)) * 8;
+          src = bytes ? static_cast<const void*>(norms + seq + t0 + tok) : static_cast<const void*>(norms);
+          dst += kTile * (CB + SB) + (cc - CCH - SCH) * 16;
+        }
+        cp_async16(dst, src, bytes);
+      }
+    }
+    cp_async_commit();
+  };
+
+  // B fragments of q~ (type 0) and S q~ (type 1), register order of mma B.
+  uint32_t qf[2][NT][8][2];
+  {
+    const uint32_t* src = p.qfrag + static_cast<size_t>(bh) * (2 * NT * 8 * 32 * 2);
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) {
+          const uint2 v = *reinterpret_cast<const uint2*>(src + (((t * NT + nt) * 8 + kb) * 32 + lane) * 2);
+          qf[t][nt][kb][0] = v.x;
+          qf[t][nt][kb][1] = v.y;
+        }
+  }
+
+  float accC[NT][8][4], accZ[NT][8][4];
+  float m_run[NT], l_run[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    m_run[nt] = -INFINITY;
+    l_run[nt] = 0.f;
+#pragma unroll
+    for (int rb = 0; rb < 8; ++rb)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) accC[nt][rb][r] = accZ[nt][rb][r] = 0.f;
+  }
+
+#pragma unroll 1
+  for (int i = 0; i < kStages - 1; ++i) issue(i);
+
+#pragma unroll 1
+  for (int i = 0; i < my_count; ++i) {
+    cp_async_wait<kStages - 2>();
+    __syncwarp();
+    const uint8_t* stg = my_stages + (i % kStages) * STAGE;
+    const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
+    const int nv = static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
+
+    // ---------------- K side: scores of tokens gid and gid + 8 -------------
+    float logit[NT][2];
+    {
+      const uint8_t* kc = stg;
+      const uint32_t* ks = reinterpret_cast<const uint32_t*>(stg + kTile * CB);
+      const float2* kn = reinterpret_cast<const float2*>(stg + kTile * (CB + SB));
+      uint32_t wk[2][P], wz[2];
+      float2 knorm[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int tok = gid + 8 * e;
+        uint32_t raw[BITS];
+#pragma unroll
+        for (int k = 0; k < BITS; ++k) raw[k] = reinterpret_cast<const uint32_t*>(kc + tok * CB + k * (kD / 8))[tig];
+        Planes<BITS>::make(raw, wk[e]);
+        wz[e] = ks[tok * (SB / 4) + tig];
+        knorm[e] = kn[tok];
+      }
+      float code[NT][2], zs[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) code[nt][0] = code[nt][1] = 0.f;
+#pragma unroll
+      for (int pl = 0; pl <= P; ++pl) {
+        float c[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
+        const uint32_t w0 = pl < P ? wk[0][pl < P ? pl : 0] : wz[0];
+        const uint32_t w1 = pl < P ? wk[1][pl < P ? pl : 0] : wz[1];
+        const int type = pl < P ? 0 : 1;
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) {
+          const uint32_t a[4] = {pm1_pair(w0, 2 * kb), pm1_pair(w1, 2 * kb), pm1_pair(w0, 2 * kb + 1),
+                                 pm1_pair(w1, 2 * kb + 1)};
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_bf16(c[nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float s0 = c[nt][0] + c[nt][1], s1 = c[nt][2] + c[nt][3];
+          if (pl < P) {
+            code[nt][0] = fmaf(p.walsh_k[pl < P ? pl : 0], s0, code[nt][0]);
+            code[nt][1] = fmaf(p.walsh_k[pl < P ? pl : 0], s1, code[nt][1]);
+          } else {
+            zs[nt][0] = s0;
+            zs[nt][1] = s1;
+          }
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float s = fmaf(knorm[e].x, code[nt][e], knorm[e].y * p.qjl * zs[nt][e]) * p.score_scale;
+          logit[nt][e] = (gid + 8 * e) < nv ? s : -INFINITY;
+        }
+    }
+
+    // ---------------- online softmax (head tig + 4 nt per thread) ----------
+    float prob[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float mx = fmaxf(logit[nt][0], logit[nt][1]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      if (mx > m_run[nt] + kLazyRescale) {
+        const float alpha = exp2f(m_run[nt] - mx);
+        l_run[nt] *= alpha;
+#pragma unroll
+        for (int rb = 0; rb < 8; ++rb)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            accC[nt][rb][r] *= alpha;
+            accZ[nt][rb][r] *= alpha;
+          }
+        m_run[nt] = mx;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) prob[nt][e] = logit[nt][e] == -INFINITY ? 0.f : exp2f(logit[nt][e] - m_run[nt]);
+      l_run[nt] += prob[nt][0] + prob[nt][1];
+    }
+
+    // ---------------- V side -------------------------------------------------
+    {
+      const uint8_t* vc = stg + HALF;
+      const uint8_t* vs = vc + kTile * CB;
+      const float2* vn = reinterpret_cast<const float2*>(vc + kTile * (CB + SB));
+      const int tk[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+      uint32_t x01[P], x23[P], z01, z23;
+      {
+        uint32_t r01[BITS], r23[BITS];
+#pragma unroll
+        for (int k = 0; k < BITS; ++k) {
+          const uint32_t h0 = reinterpret_cast<const uint16_t*>(vc + tk[0] * CB + k * (kD / 8))[gid];
+          const uint32_t h1 = reinterpret_cast<const uint16_t*>(vc + tk[1] * CB + k * (kD / 8))[gid];
+          const uint32_t h2 = reinterpret_cast<const uint16_t*>(vc + tk[2] * CB + k * (kD / 8))[gid];
+          const uint32_t h3 = reinterpret_cast<const uint16_t*>(vc + tk[3] * CB + k * (kD / 8))[gid];
+          r01[k] = h0 | (h1 << 16);
+          r23[k] = h2 | (h3 << 16);
+        }
+        Planes<BITS>::make(r01, x01);
+        Planes<BITS>::make(r23, x23);
+        const uint32_t g0 = reinterpret_cast<const uint16_t*>(vs + tk[0] * SB)[gid];
+        const uint32_t g1 = reinterpret_cast<const uint16_t*>(vs + tk[1] * SB)[gid];
+        const uint32_t g2 = reinterpret_cast<const uint16_t*>(vs + tk[2] * SB)[gid];
+        const uint32_t g3 = reinterpret_cast<const uint16_t*>(vs + tk[3] * SB)[gid];
+        z01 = g0 | (g1 << 16);
+        z23 = g2 | (g3 << 16);
+      }
+      float2 vnorm[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) vnorm[j] = vn[tk[j]];
+      const int piece = gid & 1;
+      const int srcA = (2 * tig) * 4 + (gid >> 1);
+      const int srcB = (2 * tig + 1) * 4 + (gid >> 1);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float pt[4];
+        pt[0] = __shfl_sync(0xffffffffu, prob[nt][0], srcA);
+        pt[2] = __shfl_sync(0xffffffffu, prob[nt][1], srcA);
+        pt[1] = __shfl_sync(0xffffffffu, prob[nt][0], srcB);
+        pt[3] = __shfl_sync(0xffffffffu, prob[nt][1], srcB);
+        uint32_t bc[P][2], bz[2];
+#pragma unroll
+        for (int pl = 0; pl < P; ++pl) {
+          float w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w[j] = bf16_piece(p.walsh_v[pl] * pt[j] * vnorm[j].x, piece);
+          bc[pl][0] = pack_bf16(w[0], w[1]);
+          bc[pl][1] = pack_bf16(w[2], w[3]);
+        }
+        {
+          float w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w[j] = bf16_piece(pt[j] * vnorm[j].y, piece);
+          bz[0] = pack_bf16(w[0], w[1]);
+          bz[1] = pack_bf16(w[2], w[3]);
+        }
+#pragma unroll
+        for (int rb = 0; rb < 8; ++rb) {
+#pragma unroll
+          for (int pl = 0; pl < P; ++pl) {
+            const uint32_t a[4] = {pm1_pair(x01[pl], 2 * rb), pm1_pair(x01[pl], 2 * rb + 1), pm1_pair(x23[pl], 2 * rb),
+                                   pm1_pair(x23[pl], 2 * rb + 1)};
+            mma_bf16(accC[nt][rb], a, bc[pl][0], bc[pl][1]);
+          }
+          const uint32_t a[4] = {pm1_pair(z01, 2 * rb), pm1_pair(z01, 2 * rb + 1), pm1_pair(z23, 2 * rb),
+                                 pm1_pair(z23, 2 * rb + 1)};
+          mma_bf16(accZ[nt][rb], a, bz[0], bz[1]);
+        }
+      }
+    }
+    __syncwarp();
+    issue(i + kStages - 1);
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // ---------------- merge the 4 warps of this CTA ---------------------------
+  // merge buffer per warp: [G][2 + 2 kD]  (m, l, O_code[kD], O_z[kD])
+  constexpr int REC = 2 + 2 * kD;
+  float* mbuf = reinterpret_cast<float*>(smem);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int h = tig + 4 * nt;
+    float l = l_run[nt];
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    l += __shfl_xor_sync(0xffffffffu, l, 8);
+    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    if (h < G) {
+      float* dst = mbuf + (warp * G + h) * REC;
+      if (gid == 0) {
+        dst[0] = m_run[nt];
+        dst[1] = l;
+      }
+#pragma unroll
+      for (int rb = 0; rb < 8; ++rb) {
+        const int d0 = 16 * gid + 2 * rb;  // rows gid / gid + 8 of row block rb
+        dst[2 + d0] = accC[nt][rb][0] + accC[nt][rb][1];
+        dst[2 + d0 + 1] = accC[nt][rb][2] + accC[nt][rb][3];
+        dst[2 + kD + d0] = accZ[nt][rb][0] + accZ[nt][rb][1];
+        dst[2 + kD + d0 + 1] = accZ[nt][rb][2] + accZ[nt][rb][3];
+      }
+    }
+  }
+  __syncthreads();
+  float* out = p.partial + (static_cast<size_t>(bh) * p.n_splits + split) * G * REC;
+  for (int idx = threadIdx.x; idx < G * REC; idx += blockDim.x) {
+    const int h = idx / REC, k = idx % REC;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mbuf[(w * G + h) * REC]);
+    float acc = 0.f;
+    if (k == 0) {
+      acc = M;
+    } else if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = mbuf[(w * G + h) * REC];
+        if (mw != -INFINITY) acc = fmaf(exp2f(mw - M), mbuf[(w * G + h) * REC + k], acc);
+      }
+    }
+    out[idx] = acc;
+  }
+}
+
+// One block of kD threads per (b, query head).
+template <typename T>
+__global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ q, const int64_t* __restrict__ q_pos,
+                                                          int Hq, int G, int NT, const float* __restrict__ dsigns,
+                                                          const float* __restrict__ st, const float2* __restrict__ rope_hi,
+                                                          const float2* __restrict__ rope_lo, int64_t rope_max_pos,
+                                                          int rope, uint16_t* __restrict__ qfrag) {
+  __shared__ float buf[kD];
+  const int i = threadIdx.x;
+  const int bq = blockIdx.x;           // b * Hq + hq
+  const int b = bq / Hq, hq = bq % Hq;
+  float v;
+  if constexpr (sizeof(T) == 4) v = q[static_cast<size_t>(bq) * kD + i];
+  else v = __bfloat162float(q[static_cast<size_t>(bq) * kD + i]);
+  if (rope) {
+    const int64_t pos = q_pos[b];
+    buf[i] = v;
+    __syncthreads();
+    if (pos < 0 || pos >= rope_max_pos) {
+      v = __int_as_float(0x7fc00000);
+    } else {
+      const int j = i & (kD / 2 - 1);
+      const float2 a = rope_hi[(pos >> kRopeLoBits) * (kD / 2) + j];
+      const float2 c = rope_lo[(pos & (kRopeLoRows - 1)) * (kD / 2) + j];
+      const float cs = a.x * c.x - a.y * c.y, sn = a.y * c.x + a.x * c.y;
+      const float x1 = buf[j], x2 = buf[j + kD / 2];
+      v = i < kD / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
+    }
+    __syncthreads();
+  }
+  // q~ = H (D q) / sqrt(d)
+  buf[i] = v * dsigns[i];
+  __syncthreads();
+#pragma unroll
+  for (int bit = 1; bit < kD; bit <<= 1) {
+    const float a = buf[i], o = buf[i ^ bit];
+    __syncthreads();
+    buf[i] = (i & bit) ? o - a : a + o;
+    __syncthreads();
+  }
+  const float qt = buf[i] * rsqrtf(static_cast<float>(kD));
+  __syncthreads();
+  buf[i] = qt;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < kD; ++k) s = fmaf(st[k * kD + i], buf[k], s);
+
+  // scatter the bf16 hi/lo pieces into the B-fragment layout
+  const int kv = hq / G, hl = hq % G;
+  const int bh = b * (Hq / G) + kv;
+  const int tg = i >> 5, x = i & 31, e = x >> 4, reg = x & 1, kb = (x & 15) >> 1;
+  const int nt = hl >> 2;
+#pragma unroll
+  for (int type = 0; type < 2; ++type) {
+    const float val = type == 0 ? qt : s;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(val);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
+#pragma unroll
+    for (int piece = 0; piece < 2; ++piece) {
+      const int n = 2 * (hl & 3) + piece;
+      const int ln = 4 * n + tg;
+      const size_t idx = ((((static_cast<size_t>(bh) * 2 + type) * NT + nt) * 8 + kb) * 32 + ln) * 4 + reg * 2 + e;
+      qfrag[idx] = __bfloat16_as_ushort(piece ? lo : hi);
+    }
+  }
+}
+
+// One block of kD threads per (b, query head).
+__global__ void __launch_bounds__(kD) decode_merge_kernel(const float* __restrict__ partial, int Hq, int G, int n_splits,
+                                                         const float* __restrict__ s_mat, const float* __restrict__ dsigns,
+                                                         float qjl, float* __restrict__ out) {
+  __shared__ float oz[kD];
+  __shared__ float buf[kD];
+  const int i = threadIdx.x;
+  const int bq = blockIdx.x;
+  const int b = bq / Hq, hq = bq % Hq;
+  const int Hkv = Hq / G;
+  const int bh = b * Hkv + hq / G, hl = hq % G;
+  constexpr int REC = 2 + 2 * kD;
+  const float* base = partial + static_cast<size_t>(bh) * n_splits * G * REC + hl * REC;
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, base[static_cast<size_t>(s) * G * REC]);
+  float L = 0.f, oc = 0.f, ozi = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < n_splits; ++s) {
+      const float* rec = base + static_cast<size_t>(s) * G * REC;
+      const float ms = rec[0];
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M);
+      L = fmaf(f, rec[1], L);
+      oc = fmaf(f, rec[2 + i], oc);
+      ozi = fmaf(f, rec[2 + kD + i], ozi);
+    }
+  }
+  oz[i] = ozi;
+  __syncthreads();
+  // rotated-space value: O_code + sqrt(pi/2)/m S^T O_z
+  float corr = 0.f;
+#pragma unroll 8
+  for (int j = 0; j < kD; ++j) corr = fmaf(s_mat[j * kD + i], oz[j], corr);
+  const float y = L > 0.f ? (oc + qjl * corr) / L : 0.f;
+  // Pi^T y = D H y / sqrt(d)
+  buf[i] = y;
+  __syncthreads();
+#pragma unroll
+  for (int bit = 1; bit < kD; bit <<= 1) {
+    const float a = buf[i], o = buf[i ^ bit];
+    __syncthreads();
+    buf[i] = (i & bit) ? o - a : a + o;
+    __syncthreads();
+  }
+  out[static_cast<size_t>(bq) * kD + i] = buf[i] * dsigns[i] * rsqrtf(static_cast<float>(kD));
+}
+
+thread_local cudaEvent_t g_prof_begin = nullptr;
+thread_local cudaEvent_t g_prof_end = nullptr;
+
+struct SplitPlan {
+  int n_splits;
+  int64_t chunk;
+};
+
+SplitPlan plan_splits(int BH, int64_t T) {
+  SplitPlan sp{1, kTile * kWarps};
+  if (T <= 0) return sp;
+  const int target = 148 * 8;
+  int64_t ns = (target + BH - 1) / BH;
+  const int64_t max_ns = (T + 255) / 256;
+  if (ns > max_ns) ns = max_ns;
+  if (ns < 1) ns = 1;
+  int64_t chunk = (T + ns - 1) / ns;
+  chunk = (chunk + kTile * kWarps - 1) / (kTile * kWarps) * (kTile * kWarps);
+  sp.chunk = chunk;
+  sp.n_splits = static_cast<int>((T + chunk - 1) / chunk);
+  return sp;
+}
+
+int num_tiles_n(int G) { return (2 * G + 7) / 8; }
+
+size_t frag_bytes(int BH, int G) { return static_cast<size_t>(BH) * 2 * num_tiles_n(G) * 8 * 32 * 2 * 4; }
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+size_t workspace_for(int B, int Hq, int Hkv, int64_t T) {
+  const int G = Hq / Hkv;
+  const int BH = B * Hkv;
+  const SplitPlan sp = plan_splits(BH, T);
+  return align256(frag_bytes(BH, G)) +
+         align256(static_cast<size_t>(BH) * sp.n_splits * G * (2 + 2 * kD) * sizeof(float));
+}
+
+template <int BITS, int G>
+int launch_split(const DecodeParams& p, int BH, cudaStream_t s) {
+  constexpr int CB = BITS * kD / 8, SB = kD / 8;
+  constexpr int STAGE = 2 * kTile * (CB + SB + 8);
+  const size_t stage_bytes = static_cast<size_t>(kWarps) * kStages * STAGE;
+  const size_t merge_bytes = static_cast<size_t>(kWarps) * G * (2 + 2 * kD) * sizeof(float);
+  const size_t smem = stage_bytes > merge_bytes ? stage_bytes : merge_bytes;
+  auto kern = decode_split_kernel<BITS, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return TQ_ECUDA;
+  dim3 grid(p.n_splits, BH);
+  kern<<<grid, kWarps * 32, smem, s>>>(p);
+  return tq::launch_status();
+}
+
+template <int BITS>
+int dispatch_g(int G, const DecodeParams& p, int BH, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_split<BITS, 1>(p, BH, s);
+    case 2: return launch_split<BITS, 2>(p, BH, s);
+    case 4: return launch_split<BITS, 4>(p, BH, s);
+    case 8: return launch_split<BITS, 8>(p, BH, s);
+  }
+  return TQ_EUNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" int tq_profile_next_decode(void* ev_begin, void* ev_end) {
+  if ((ev_begin == nullptr) != (ev_end == nullptr)) return TQ_EINVAL;
+  g_prof_begin = static_cast<cudaEvent_t>(ev_begin);
+  g_prof_end = static_cast<cudaEvent_t>(ev_end);
+  return TQ_OK;
+}
+
+extern "C" size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv, int B, int Hq, int Hkv,
+                                           int64_t T) {
+  if (!hk || !hv || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0) return 0;
+  return workspace_for(B, Hq, Hkv, T);
+}
+
+extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
+                                   const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
+                                   const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
+                                   const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
+                                   float scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
+  g_prof_begin = g_prof_end = nullptr;
+  if (!hk || !hv || !q || !out) return TQ_EINVAL;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || !std::isfinite(scale)) return TQ_EINVAL;
+  if (hk->d != hv->d || hk->m != hv->m) return TQ_EINVAL;
+  if (hk->d != kD || hk->m != kD) return TQ_EUNSUPPORTED;
+  if (hk->kind != TQ_ROT_HADAMARD || hv->kind != TQ_ROT_HADAMARD) return TQ_EUNSUPPORTED;
+  if (hk->bits != hv->bits) return TQ_EUNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_EUNSUPPORTED;
+  if (T > 0) {
+    if (!k_codes || !k_signs || !k_norms || !v_codes || !v_signs || !v_norms) return TQ_EINVAL;
+    if (cache_stride < T || (cache_stride & 1)) return TQ_EINVAL;
+    const void* ptrs[6] = {k_codes, k_signs, k_norms, v_codes, v_signs, v_norms};
+    for (const void* ptr : ptrs)
+      if (!tq::aligned16(ptr)) return TQ_EINVAL;
+  }
+  if (hk->rope_base > 0.0 && !q_pos) return TQ_EINVAL;
+  const int BH = B * Hkv;
+  const size_t need = workspace_for(B, Hq, Hkv, T);
+  if (!workspace || workspace_bytes < need) return TQ_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TQ_EINVAL;
+  if (!tq::on_handle_device(hk) || !tq::on_handle_device(hv)) return TQ_EINVAL;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const SplitPlan sp = plan_splits(BH, T);
+  const int NT = num_tiles_n(G);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws);
+  float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)));
+
+  if (2 * G < 8 * NT) {
+    if (cudaMemsetAsync(qfrag, 0, frag_bytes(BH, G), s) != cudaSuccess) return TQ_ECUDA;
+  }
+  const int rope = hk->rope_base > 0.0 ? 1 : 0;
+  if (q_dtype == TQ_F32)
+    decode_qprep_kernel<float><<<B * Hq, kD, 0, s>>>(static_cast<const float*>(q), q_pos, Hq, G, NT, hk->d_signs,
+                                                       hk->d_st, hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope,
+                                                       reinterpret_cast<uint16_t*>(qfrag));
+  else
+    decode_qprep_kernel<__nv_bfloat16><<<B * Hq, kD, 0, s>>>(static_cast<const __nv_bfloat16*>(q), q_pos, Hq, G, NT,
+                                                               hk->d_signs, hk->d_st, hk->d_rope_hi, hk->d_rope_lo,
+                                                               hk->rope_max_pos, rope,
+                                                               reinterpret_cast<uint16_t*>(qfrag));
+  int st = tq::launch_status();
+  if (st != TQ_OK) return st;
+
+  DecodeParams p{};
+  p.k_codes = k_codes;
+  p.k_signs = k_signs;
+  p.k_norms = reinterpret_cast<const float2*>(k_norms);
+  p.v_codes = v_codes;
+  p.v_signs = v_signs;
+  p.v_norms = reinterpret_cast<const float2*>(v_norms);
+  p.cache_stride = cache_stride;
+  p.T = T;
+  p.chunk = sp.chunk;
+  p.n_splits = sp.n_splits;
+  p.qfrag = qfrag;
+  p.partial = partial;
+  p.score_scale = scale * 1.4426950408889634f;
+  p.qjl = static_cast<float>(kQjlConst / hk->m);
+  for (int i = 0; i < 4; ++i) {
+    p.walsh_k[i] = static_cast<float>(hk->walsh[i]);
+    p.walsh_v[i] = static_cast<float>(hv->walsh[i]);
+  }
+  if (prof_begin && cudaEventRecord(prof_begin, s) != cudaSuccess) return TQ_ECUDA;
+  switch (hk->bits) {
+    case 1: st = dispatch_g<1>(G, p, BH, s); break;
+    case 2: st = dispatch_g<2>(G, p, BH, s); break;
+    case 3: st = dispatch_g<3>(G, p, BH, s); break;
+    default: st = TQ_EUNSUPPORTED;
+  }
+  if (st != TQ_OK) return st;
+  if (prof_end && cudaEventRecord(prof_end, s) != cudaSuccess) return TQ_ECUDA;
+  decode_merge_kernel<<<B * Hq, kD, 0, s>>>(partial, Hq, G, sp.n_splits, hv->d_s, hv->d_signs,
+                                            static_cast<float>(kQjlConst / hv->m), out);
+  return tq::launch_status();
+}

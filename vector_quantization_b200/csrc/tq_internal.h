@@ -1,0 +1,60 @@
+// Private declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/tq.h"
+
+// Codec handle.  Host copies keep what the host-side launch code needs;
+// device copies are what the kernels read.  Immutable after build.
+struct tq_rotation {
+  int device = 0;
+  int d = 0, m = 0, bits = 0, kind = 0;
+  double rope_base = 0.0;
+  int64_t rope_max_pos = 0;
+  int rope_hi_rows = 0;                 // rows of the coarse RoPE table
+
+  std::vector<double> levels;           // [2^bits] ascending
+  std::vector<double> thresholds;       // [2^bits - 1]
+  // Walsh form of the codebook: level(idx) = sum_p walsh[p] * s_p(idx),
+  // s_p the +-1 value of the p-th plane product (see plane_products()).
+  double walsh[4] = {0, 0, 0, 0};
+  int n_planes = 0;                     // 1, 2 or 4 for bits 1, 2, 3
+
+  // device
+  float* d_levels = nullptr;            // [2^bits]
+  float* d_thresholds = nullptr;        // [2^bits - 1]
+  float* d_signs = nullptr;             // [d] +-1 (Hadamard kind)
+  float* d_pi = nullptr;                // [d*d] row-major (dense kind)
+  float* d_s = nullptr;                 // [m*d] row-major S (bf16-exact values)
+  float* d_st = nullptr;                // [d*m] S transposed
+  float2* d_rope_hi = nullptr;          // [rope_hi_rows][d/2] (cos, sin) of h*1024*theta_i
+  float2* d_rope_lo = nullptr;          // [1024][d/2]           (cos, sin) of l*theta_i
+};
+
+// Number of low position bits resolved by the fine RoPE table.
+constexpr int kRopeLoBits = 10;
+constexpr int kRopeLoRows = 1 << kRopeLoBits;
+
+// sqrt(pi/2): the QJL estimator constant (divided by m at use).
+constexpr double kQjlConst = 1.2533141373155002512078826424055226;
+
+namespace tq {
+
+// Checks that the current device is the handle's device.
+bool on_handle_device(const tq_rotation* h);
+
+// Uniform launch-error check after a kernel launch.
+inline int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TQ_OK : TQ_ECUDA;
+}
+
+inline bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+}  // namespace tq

@@ -1,0 +1,224 @@
+"""Thin ctypes binding of ``libtq.so`` (argument marshalling only).
+
+Every function here checks shapes and dtypes of torch tensors, passes raw
+device pointers and sizes to the C ABI declared in ``include/tq.h`` and raises
+:class:`TQError` on a non-zero status.  All arithmetic runs in the library's
+CUDA kernels; there is no fallback of any kind: if ``libtq.so`` is missing or
+fails to load, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EWORKSPACE, TQ_ECUDA, TQ_ENOMEM = 0, -1, -2, -3, -4, -5
+TQ_ROT_HADAMARD, TQ_ROT_DENSE = 0, 1
+TQ_F32, TQ_BF16 = 0, 1
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.tq_status_string(status).decode()} ({status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m vector_quantization_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    c_i, c_i64, c_sz, c_p, c_d, c_f = (ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p,
+                                       ctypes.c_double, ctypes.c_float)
+    sig = {
+        "tq_status_string": (ctypes.c_char_p, [c_i]),
+        "tq_version": (c_i, []),
+        "tq_lloyd_max": (c_i, [c_i, c_i, c_p, c_p]),
+        "tq_build_rotation": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_i, c_d, c_i64, ctypes.POINTER(c_p)]),
+        "tq_free_rotation": (c_i, [c_p]),
+        "tq_rotation_export": (c_i, [c_p, c_p, c_p, c_p, c_p]),
+        "tq_rotation_dims": (c_i, [c_p, c_p, c_p, c_p, c_p, c_p]),
+        "tq_quantize_kv": (c_i, [c_p, c_p, c_i, c_i64, c_i64, c_p, c_i64, c_i64, c_i, c_p, c_p, c_p, c_i64, c_p]),
+        "tq_decode_attention": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
+                                      c_i64, c_f, c_p, c_p, c_sz, c_p]),
+        "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
+        "tq_profile_next_decode": (c_i, [c_p, c_p]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int, where: str):
+    if status != TQ_OK:
+        raise TQError(status, where)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream) -> int | None:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return TQ_F32
+    if t.dtype == torch.bfloat16:
+        return TQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def version() -> int:
+    return _lib.tq_version()
+
+
+def lloyd_max(d: int, bits: int):
+    """Host-only Lloyd-Max codebook of the library: (levels, thresholds) float64."""
+    lv = np.zeros(1 << bits)
+    th = np.zeros((1 << bits) - 1)
+    _check(_lib.tq_lloyd_max(d, bits, lv.ctypes.data, th.ctypes.data), "tq_lloyd_max")
+    return lv, th
+
+
+class Rotation:
+    """A codec handle (rotation, QJL matrix, codebook, RoPE tables) on the
+    current CUDA device.  ``randomness`` holds the seeded draws
+    (``signs``, ``gauss_s`` and, for ``kind='dense'``, ``gauss_pi``)."""
+
+    def __init__(self, d: int, bits: int, randomness: dict, kind: str = "hadamard",
+                 rope_base: float = 0.0, rope_max_pos: int = 1 << 21):
+        kind_code = {"hadamard": TQ_ROT_HADAMARD, "dense": TQ_ROT_DENSE}[kind]
+        signs = np.ascontiguousarray(randomness["signs"], dtype=np.int8)
+        gs = np.ascontiguousarray(randomness["gauss_s"], dtype=np.float32)
+        gp = randomness.get("gauss_pi")
+        gp = None if gp is None else np.ascontiguousarray(gp, dtype=np.float64)
+        h = ctypes.c_void_p()
+        _check(_lib.tq_build_rotation(d, bits, kind_code, signs.ctypes.data,
+                                      None if gp is None else gp.ctypes.data, gs.ctypes.data, gs.shape[0],
+                                      float(rope_base), int(rope_max_pos), ctypes.byref(h)), "tq_build_rotation")
+        self._h = h
+        dd, mm, bb = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        cb, sb = ctypes.c_int64(), ctypes.c_int64()
+        _check(_lib.tq_rotation_dims(h, ctypes.byref(dd), ctypes.byref(mm), ctypes.byref(bb), ctypes.byref(cb),
+                                     ctypes.byref(sb)), "tq_rotation_dims")
+        self.d, self.m, self.bits = dd.value, mm.value, bb.value
+        self.code_bytes, self.sign_bytes = cb.value, sb.value
+        self.kind = kind
+        self.rope_base = rope_base
+
+    @property
+    def handle(self):
+        return self._h
+
+    def export(self) -> dict:
+        d, m, n = self.d, self.m, 1 << self.bits
+        pi = np.zeros((d, d), np.float32)
+        s = np.zeros((m, d), np.float32)
+        lv = np.zeros(n)
+        th = np.zeros(n - 1)
+        _check(_lib.tq_rotation_export(self._h, pi.ctypes.data, s.ctypes.data, lv.ctypes.data, th.ctypes.data),
+               "tq_rotation_export")
+        return {"pi": pi, "s": s, "levels": lv, "thresholds": th}
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.tq_free_rotation(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def empty_records(rot: Rotation, shape, device):
+    """Allocate (codes, signs, norms) arrays for ``shape`` records."""
+    import torch
+    shape = tuple(shape)
+    codes = torch.empty(shape + (rot.code_bytes,), dtype=torch.uint8, device=device)
+    signs = torch.empty(shape + (rot.sign_bytes,), dtype=torch.uint8, device=device)
+    norms = torch.empty(shape + (2,), dtype=torch.float32, device=device)
+    return codes, signs, norms
+
+
+def quantize_kv(rot: Rotation, x, *, pos=None, pos_period: int | None = None, pos_offset: int = 0,
+                apply_rope: bool = False, out=None, out_stride: int = 1, stream=None):
+    """Encode the rows of ``x`` ([n, d] or [..., d], float32/bfloat16, CUDA).
+
+    Returns (codes, signs, norms).  With ``out`` the records are written into
+    the given arrays (row i at record i * out_stride of each)."""
+    d = x.shape[-1]
+    x2 = x.reshape(-1, d)
+    if x2.stride(-1) != 1:
+        raise ValueError("x rows must be contiguous")
+    n = x2.shape[0]
+    ld = x2.stride(0) if n > 1 else d
+    if out is None:
+        out = empty_records(rot, x.shape[:-1], x.device)
+    codes, signs, norms = out
+    if pos is not None and pos.dtype.is_floating_point:
+        raise TypeError("pos must be int64")
+    period = pos_period if pos_period is not None else max(n, 1)
+    _check(_lib.tq_quantize_kv(rot.handle, _ptr(x2), _dtype_code(x2), n, ld, _ptr(pos), period, pos_offset,
+                               1 if apply_rope else 0, _ptr(codes), _ptr(signs), _ptr(norms), out_stride,
+                               _stream_ptr(stream)), "tq_quantize_kv")
+    return codes, signs, norms
+
+
+def profile_next_decode(ev_begin, ev_end):
+    """Have the next decode_attention call (this thread) record the two
+    torch.cuda.Event objects around its split-KV kernel."""
+    _check(_lib.tq_profile_next_decode(ev_begin.cuda_event if ev_begin is not None else None,
+                                       ev_end.cuda_event if ev_end is not None else None), "tq_profile_next_decode")
+
+
+def decode_workspace_size(rot_k: Rotation, rot_v: Rotation, B: int, Hq: int, Hkv: int, T: int) -> int:
+    return _lib.tq_decode_workspace_size(rot_k.handle, rot_v.handle, B, Hq, Hkv, T)
+
+
+def alloc_workspace(nbytes: int, device):
+    import torch
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, T: int, *, scale: float | None = None,
+                     out=None, workspace=None, stream=None):
+    """One decode step: q [B, Hq, d] against caches (codes, signs, norms) of
+    shape [B, Hkv, cap, ...]; attends to the first T records of each
+    sequence.  Returns out [B, Hq, d] float32."""
+    import torch
+    B, Hq, d = q.shape
+    kc, ks, kn = k_cache
+    vc, vs, vn = v_cache
+    Hkv, cap = kc.shape[1], kc.shape[2]
+    for t in (kc, ks, kn, vc, vs, vn):
+        if not t.is_contiguous():
+            raise ValueError("cache arrays must be contiguous")
+    q = q.contiguous()
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(rot_k, rot_v, B, Hq, Hkv, T)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    _check(_lib.tq_decode_attention(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos), _ptr(kc),
+                                    _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, T,
+                                    float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                    _stream_ptr(stream)), "tq_decode_attention")
+    return out
