@@ -265,10 +265,12 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("bench_timed")
     e0.record()
     for s in range(args.steps):
         step(prof[s])
     e1.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()

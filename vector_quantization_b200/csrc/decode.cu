@@ -52,6 +52,7 @@ struct DecodeParams {
   int64_t chunk;           // tokens per split (multiple of kTile)
   int n_splits;
   const uint32_t* qfrag;   // [BH][2][NT][8][32][2]
+  const float* kconst;     // [BH][2][8]
   float* partial;          // [BH][n_splits][G][2 + 2 kD]
   float score_scale;       // softmax scale * log2(e)
   float qjl;               // sqrt(pi/2) / m
@@ -82,17 +83,27 @@ __device__ __forceinline__ uint32_t pm1_pair(uint32_t w, int x) {
   return (~t & 0x80008000u) | 0x3F803F80u;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
-  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
-  return l | (h << 16);
+// Bit j (and j + 16) of a plane word as a pair of bf16 values, one LOP3.
+// The kept bit lands at half-word position p = j + 8 (from w << 8) for j < 8,
+// or p = j for j >= 8: an exponent bit (p = 8..14) or the sign bit (p = 15)
+// of a bf16 whose other bits are the fixed pattern pos_base(p).  The
+// value is then v0 or v1 (kPosV0/kPosV1) - affine in the bit, and exact.
+// With s = 2 bit - 1 it is mu_p + sigma_p s; sigma_p is divided out of the
+// matching B entries and sum mu_p B subtracted once per head (q-prep).
+__host__ __device__ constexpr uint32_t pos_base(int p) {
+  return p == 8 ? 0x3E80u : p == 9 ? 0x3D80u : p == 10 ? 0x3B80u : p == 11 ? 0x3780u
+       : p == 12 ? 0x2F80u : p == 13 ? 0x1F80u : p == 14 ? 0x0000u : 0x3F80u;
 }
-
-// Piece `piece` (0 = hi, 1 = lo) of the two-term bf16 split of v.
-__device__ __forceinline__ float bf16_piece(float v, int piece) {
-  const float hi = __bfloat162float(__float2bfloat16_rn(v));
-  return piece ? v - hi : hi;
+__device__ __forceinline__ uint32_t bit_pair(uint32_t w, uint32_t w_shl8, int j) {
+  const int p = j < 8 ? j + 8 : j;
+  const uint32_t mask = (1u << p) | (1u << (p + 16));
+  return ((j < 8 ? w_shl8 : w) & mask) | (pos_base(p) * 0x10001u);
 }
+__device__ __forceinline__ float pos_v0(int p) {
+  return p == 8 ? 0.25f : p == 9 ? 0.0625f : p == 10 ? 0.00390625f : p == 11 ? 1.52587890625e-05f
+       : p == 12 ? 2.3283064365386963e-10f : p == 13 ? 5.421010862427522e-20f : p == 14 ? 0.f : 1.f;
+}
+__device__ __forceinline__ float pos_v1(int p) { return p == 14 ? 2.f : p == 15 ? -1.f : 1.f; }
 
 template <int BITS>
 struct Planes {
@@ -113,6 +124,15 @@ struct Planes {
   }
 };
 
+// Shared-memory position of the 16-byte chunk `part` of token `tok`'s codes.
+// With 2-bit codes (two chunks per token) the chunks of tokens 4..7 (mod 8)
+// are swapped so that the fragment reads below are free of bank conflicts.
+template <int BITS>
+__device__ __forceinline__ int code_chunk(int tok, int part) {
+  if constexpr (BITS == 2) return tok * 2 + (part ^ ((tok >> 2) & 1));
+  else return tok * BITS + part;
+}
+
 template <int BITS, int G>
 __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams p) {
   constexpr int NT = (2 * G + 7) / 8;
@@ -121,6 +141,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
   constexpr int SB = kD / 8;                        // sign bytes per token
   constexpr int HALF = kTile * (CB + SB + 8);       // K (or V) part of a stage
   constexpr int STAGE = 2 * HALF;
+  constexpr int CCH = kTile * CB / 16;              // 16-byte chunks of codes per side
   extern __shared__ __align__(16) uint8_t smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,59 +156,59 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
 
   uint8_t* my_stages = smem + warp * kStages * STAGE;
 
-  // Loads of one tile (16 tokens) into stage `st`; records past t_end are zero-filled.
+  // Per-lane roles in the tile copy: code chunks (both sides), then sign
+  // chunks (lanes 0-15 K, 16-31 V), then norm chunks (lanes 0-7 K, 8-15 V).
+  // A tile's records are contiguous in every array, so a chunk's source is
+  // the tile base plus 16 bytes per chunk.
+  const int sg_side = lane >> 4, sg_c = lane & 15;
+  const int nm_side = (lane >> 3) & 1, nm_c = lane & 7;
   auto issue = [&](int i) {
     if (i < my_count) {
-      const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
-      const int nv = static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
+      const int64_t t0 = seq + t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
+      const int nv = static_cast<int>(t_end - (t0 - seq) < kTile ? t_end - (t0 - seq) : kTile);
       uint8_t* stg = my_stages + (i % kStages) * STAGE;
-      constexpr int CCH = kTile * CB / 16, SCH = kTile * SB / 16, NCH = kTile * 8 / 16;
-      constexpr int HCH = CCH + SCH + NCH;
-      for (int c = lane; c < 2 * HCH; c += 32) {
-        const int side = c >= HCH;
-        const int cc = c - side * HCH;
-        const uint8_t* codes = side ? p.v_codes : p.k_codes;
-        const uint8_t* signs = side ? p.v_signs : p.k_signs;
-        const float2* norms = side ? p.v_norms : p.k_norms;
-        uint8_t* dst = stg + side * HALF;
-        const void* src;
-        int bytes;
-        if (cc < CCH) {
-          const int tok = cc / (CB / 16), part = cc % (CB / 16);
-          bytes = tok < nv ? 16 : 0;
-          src = bytes ? codes + (seq + t0 + tok) * CB + part * 16 : codes;
-          dst += cc * 16;
-        } else if (cc < CCH + SCH) {
-          const int tok = (cc - CCH) / (SB / 16), part = (cc - CCH) % (SB / 16);
-          bytes = tok < nv ? 16 : 0;
-          src = bytes ? signs + (seq + t0 + tok) * SB + part * 16 : signs;
-          dst += kTile * CB + (cc - CCH) * 16;
-        } else {
-          const int tok = 2 * (cc - CCH - SCH);
-          bytes = max(0, min(2, nv - tok)) * 8;
-          src = bytes ? static_cast<const void*>(norms + seq + t0 + tok) : static_cast<const void*>(norms);
-          dst += kTile * (CB + SB) + (cc - CCH - SCH) * 16;
+#pragma unroll
+      for (int side = 0; side < 2; ++side) {
+        const uint8_t* src = (side ? p.v_codes : p.k_codes) + t0 * CB;
+#pragma unroll
+        for (int c = lane; c < CCH; c += 32) {
+          const int tok = c / BITS, part = c % BITS;
+          cp_async16(stg + side * HALF + code_chunk<BITS>(tok, part) * 16, tok < nv ? src + c * 16 : src,
+                     tok < nv ? 16 : 0);
         }
-        cp_async16(dst, src, bytes);
+      }
+      {
+        const uint8_t* src = (sg_side ? p.v_signs : p.k_signs) + t0 * SB;
+        cp_async16(stg + sg_side * HALF + kTile * CB + sg_c * 16, sg_c < nv ? src + sg_c * 16 : src, sg_c < nv ? 16 : 0);
+      }
+      if (lane < 16) {
+        const float2* src = (nm_side ? p.v_norms : p.k_norms) + t0;
+        const int bytes = max(0, min(16, (nv - 2 * nm_c) * 8));
+        cp_async16(stg + nm_side * HALF + kTile * (CB + SB) + nm_c * 16, bytes ? src + 2 * nm_c : src, bytes);
       }
     }
     cp_async_commit();
   };
 
-  // B fragments of q~ (type 0) and S q~ (type 1), register order of mma B.
+  // B fragments of q~ (type 0) and S q~ (type 1), register order of mma B,
+  // already divided by sigma_p; kc[type][nt] = sum_k mu_k B_k of this head.
   uint32_t qf[2][NT][8][2];
+  float kc[2][NT];
   {
     const uint32_t* src = p.qfrag + static_cast<size_t>(bh) * (2 * NT * 8 * 32 * 2);
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb) {
           const uint2 v = *reinterpret_cast<const uint2*>(src + (((t * NT + nt) * 8 + kb) * 32 + lane) * 2);
           qf[t][nt][kb][0] = v.x;
           qf[t][nt][kb][1] = v.y;
         }
+        const int h = tig + 4 * nt;
+        kc[t][nt] = h < G ? p.kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] : 0.f;
+      }
   }
 
   float accC[NT][8][4], accZ[NT][8][4];
@@ -201,6 +222,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
 #pragma unroll
       for (int r = 0; r < 4; ++r) accC[nt][rb][r] = accZ[nt][rb][r] = 0.f;
   }
+  const uint32_t piece_mask = (gid & 1) ? 0xFFFF0000u : 0u;   // V-side B piece of this lane
+  const uint32_t half_sel = (gid & 1) ? 0x7632u : 0x5410u;
 
 #pragma unroll 1
   for (int i = 0; i < kStages - 1; ++i) issue(i);
@@ -216,48 +239,56 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
     // ---------------- K side: scores of tokens gid and gid + 8 -------------
     float logit[NT][2];
     {
-      const uint8_t* kc = stg;
+      const uint8_t* kcd = stg;
       const uint32_t* ks = reinterpret_cast<const uint32_t*>(stg + kTile * CB);
       const float2* kn = reinterpret_cast<const float2*>(stg + kTile * (CB + SB));
-      uint32_t wk[2][P], wz[2];
+      uint32_t wk[2][P + 1];
       float2 knorm[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int tok = gid + 8 * e;
         uint32_t raw[BITS];
 #pragma unroll
-        for (int k = 0; k < BITS; ++k) raw[k] = reinterpret_cast<const uint32_t*>(kc + tok * CB + k * (kD / 8))[tig];
-        Planes<BITS>::make(raw, wk[e]);
-        wz[e] = ks[tok * (SB / 4) + tig];
+        for (int k = 0; k < BITS; ++k)
+          raw[k] = reinterpret_cast<const uint32_t*>(kcd + code_chunk<BITS>(tok, k) * 16)[tig];
+        uint32_t pl[P];
+        Planes<BITS>::make(raw, pl);
+#pragma unroll
+        for (int q = 0; q < P; ++q) wk[e][q] = pl[q];
+        wk[e][P] = ks[tok * (SB / 4) + tig];
         knorm[e] = kn[tok];
       }
       float code[NT][2], zs[NT][2];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) code[nt][0] = code[nt][1] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) code[nt][0] = code[nt][1] = zs[nt][0] = zs[nt][1] = 0.f;
 #pragma unroll
       for (int pl = 0; pl <= P; ++pl) {
-        float c[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
-        const uint32_t w0 = pl < P ? wk[0][pl < P ? pl : 0] : wz[0];
-        const uint32_t w1 = pl < P ? wk[1][pl < P ? pl : 0] : wz[1];
         const int type = pl < P ? 0 : 1;
+        float c[2][NT][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) c[u][nt][0] = c[u][nt][1] = c[u][nt][2] = c[u][nt][3] = 0.f;
+        const uint32_t w0 = wk[0][pl], w1 = wk[1][pl];
+        const uint32_t s0 = w0 << 8, s1 = w1 << 8;
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb) {
-          const uint32_t a[4] = {pm1_pair(w0, 2 * kb), pm1_pair(w1, 2 * kb), pm1_pair(w0, 2 * kb + 1),
-                                 pm1_pair(w1, 2 * kb + 1)};
+          const uint32_t a[4] = {bit_pair(w0, s0, 2 * kb), bit_pair(w1, s1, 2 * kb), bit_pair(w0, s0, 2 * kb + 1),
+                                 bit_pair(w1, s1, 2 * kb + 1)};
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_bf16(c[nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
+          for (int nt = 0; nt < NT; ++nt) mma_bf16(c[kb & 1][nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const float s0 = c[nt][0] + c[nt][1], s1 = c[nt][2] + c[nt][3];
+          const float s0v = (c[0][nt][0] + c[0][nt][1]) + (c[1][nt][0] + c[1][nt][1]) - kc[type][nt];
+          const float s1v = (c[0][nt][2] + c[0][nt][3]) + (c[1][nt][2] + c[1][nt][3]) - kc[type][nt];
           if (pl < P) {
-            code[nt][0] = fmaf(p.walsh_k[pl < P ? pl : 0], s0, code[nt][0]);
-            code[nt][1] = fmaf(p.walsh_k[pl < P ? pl : 0], s1, code[nt][1]);
+            const float wgt = p.walsh_k[pl < P ? pl : 0];
+            code[nt][0] = fmaf(wgt, s0v, code[nt][0]);
+            code[nt][1] = fmaf(wgt, s1v, code[nt][1]);
           } else {
-            zs[nt][0] = s0;
-            zs[nt][1] = s1;
+            zs[nt][0] = s0v;
+            zs[nt][1] = s1v;
           }
         }
       }
@@ -297,35 +328,35 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
 
     // ---------------- V side -------------------------------------------------
     {
-      const uint8_t* vc = stg + HALF;
-      const uint8_t* vs = vc + kTile * CB;
-      const float2* vn = reinterpret_cast<const float2*>(vc + kTile * (CB + SB));
+      const uint8_t* vcd = stg + HALF;
+      const uint8_t* vs = vcd + kTile * CB;
+      const float2* vn = reinterpret_cast<const float2*>(vcd + kTile * (CB + SB));
       const int tk[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
       uint32_t x01[P], x23[P], z01, z23;
       {
+        // half-word gid of each plane: dims 16 gid .. 16 gid + 15
         uint32_t r01[BITS], r23[BITS];
 #pragma unroll
         for (int k = 0; k < BITS; ++k) {
-          const uint32_t h0 = reinterpret_cast<const uint16_t*>(vc + tk[0] * CB + k * (kD / 8))[gid];
-          const uint32_t h1 = reinterpret_cast<const uint16_t*>(vc + tk[1] * CB + k * (kD / 8))[gid];
-          const uint32_t h2 = reinterpret_cast<const uint16_t*>(vc + tk[2] * CB + k * (kD / 8))[gid];
-          const uint32_t h3 = reinterpret_cast<const uint16_t*>(vc + tk[3] * CB + k * (kD / 8))[gid];
-          r01[k] = h0 | (h1 << 16);
-          r23[k] = h2 | (h3 << 16);
+          const uint32_t h0 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[0], k) * 16)[gid >> 1];
+          const uint32_t h1 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[1], k) * 16)[gid >> 1];
+          const uint32_t h2 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[2], k) * 16)[gid >> 1];
+          const uint32_t h3 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[3], k) * 16)[gid >> 1];
+          r01[k] = __byte_perm(h0, h1, half_sel);
+          r23[k] = __byte_perm(h2, h3, half_sel);
         }
         Planes<BITS>::make(r01, x01);
         Planes<BITS>::make(r23, x23);
-        const uint32_t g0 = reinterpret_cast<const uint16_t*>(vs + tk[0] * SB)[gid];
-        const uint32_t g1 = reinterpret_cast<const uint16_t*>(vs + tk[1] * SB)[gid];
-        const uint32_t g2 = reinterpret_cast<const uint16_t*>(vs + tk[2] * SB)[gid];
-        const uint32_t g3 = reinterpret_cast<const uint16_t*>(vs + tk[3] * SB)[gid];
-        z01 = g0 | (g1 << 16);
-        z23 = g2 | (g3 << 16);
+        const uint32_t g0 = reinterpret_cast<const uint32_t*>(vs + tk[0] * SB)[gid >> 1];
+        const uint32_t g1 = reinterpret_cast<const uint32_t*>(vs + tk[1] * SB)[gid >> 1];
+        const uint32_t g2 = reinterpret_cast<const uint32_t*>(vs + tk[2] * SB)[gid >> 1];
+        const uint32_t g3 = reinterpret_cast<const uint32_t*>(vs + tk[3] * SB)[gid >> 1];
+        z01 = __byte_perm(g0, g1, half_sel);
+        z23 = __byte_perm(g2, g3, half_sel);
       }
       float2 vnorm[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) vnorm[j] = vn[tk[j]];
-      const int piece = gid & 1;
       const int srcA = (2 * tig) * 4 + (gid >> 1);
       const int srcB = (2 * tig + 1) * 4 + (gid >> 1);
 #pragma unroll
@@ -335,21 +366,30 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         pt[2] = __shfl_sync(0xffffffffu, prob[nt][1], srcA);
         pt[1] = __shfl_sync(0xffffffffu, prob[nt][0], srcB);
         pt[3] = __shfl_sync(0xffffffffu, prob[nt][1], srcB);
+        // B = two-term bf16 split of the weight; this lane carries one term:
+        // hi = w truncated to bf16, lo = w - hi (exact) truncated to bf16.
         uint32_t bc[P][2], bz[2];
+        float wv[4], wr[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          wv[j] = pt[j] * vnorm[j].x;
+          wr[j] = pt[j] * vnorm[j].y;
+        }
+        auto piece = [&](float w) { return w - __uint_as_float(__float_as_uint(w) & piece_mask); };
 #pragma unroll
         for (int pl = 0; pl < P; ++pl) {
-          float w[4];
+          float t[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) w[j] = bf16_piece(p.walsh_v[pl] * pt[j] * vnorm[j].x, piece);
-          bc[pl][0] = pack_bf16(w[0], w[1]);
-          bc[pl][1] = pack_bf16(w[2], w[3]);
+          for (int j = 0; j < 4; ++j) t[j] = piece(p.walsh_v[pl] * wv[j]);
+          bc[pl][0] = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[1]), 0x7632);
+          bc[pl][1] = __byte_perm(__float_as_uint(t[2]), __float_as_uint(t[3]), 0x7632);
         }
         {
-          float w[4];
+          float t[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) w[j] = bf16_piece(pt[j] * vnorm[j].y, piece);
-          bz[0] = pack_bf16(w[0], w[1]);
-          bz[1] = pack_bf16(w[2], w[3]);
+          for (int j = 0; j < 4; ++j) t[j] = piece(wr[j]);
+          bz[0] = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[1]), 0x7632);
+          bz[1] = __byte_perm(__float_as_uint(t[2]), __float_as_uint(t[3]), 0x7632);
         }
 #pragma unroll
         for (int rb = 0; rb < 8; ++rb) {
@@ -425,8 +465,10 @@ __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ 
                                                           int Hq, int G, int NT, const float* __restrict__ dsigns,
                                                           const float* __restrict__ st, const float2* __restrict__ rope_hi,
                                                           const float2* __restrict__ rope_lo, int64_t rope_max_pos,
-                                                          int rope, uint16_t* __restrict__ qfrag) {
+                                                          int rope, uint16_t* __restrict__ qfrag,
+                                                          float* __restrict__ kconst) {
   __shared__ float buf[kD];
+  __shared__ float red[2][kD / 32];
   const int i = threadIdx.x;
   const int bq = blockIdx.x;           // b * Hq + hq
   const int b = bq / Hq, hq = bq % Hq;
@@ -467,14 +509,20 @@ __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ 
 #pragma unroll 8
   for (int k = 0; k < kD; ++k) s = fmaf(st[k * kD + i], buf[k], s);
 
-  // scatter the bf16 hi/lo pieces into the B-fragment layout
+  // Scatter into the B-fragment layout of the split kernel.  Dim i sits in
+  // slot j = i & 15 of the word of lane-column tg = i / 32 (the bit_pair
+  // position p of that slot fixes sigma_p, mu_p); hi/lo bf16 pieces go to
+  // columns n = 2 (head % 4) + piece of n-tile head / 4.
   const int kv = hq / G, hl = hq % G;
   const int bh = b * (Hq / G) + kv;
-  const int tg = i >> 5, x = i & 31, e = x >> 4, reg = x & 1, kb = (x & 15) >> 1;
+  const int tg = i >> 5, x = i & 31, e = x >> 4, j = x & 15, reg = j & 1, kb = j >> 1;
+  const int pp = j < 8 ? j + 8 : j;
+  const float v0 = pos_v0(pp), v1 = pos_v1(pp);
+  const float mu = 0.5f * (v0 + v1), sigma = 0.5f * (v1 - v0);
   const int nt = hl >> 2;
 #pragma unroll
   for (int type = 0; type < 2; ++type) {
-    const float val = type == 0 ? qt : s;
+    const float val = (type == 0 ? qt : s) / sigma;
     const __nv_bfloat16 hi = __float2bfloat16_rn(val);
     const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
 #pragma unroll
@@ -484,6 +532,18 @@ __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ 
       const size_t idx = ((((static_cast<size_t>(bh) * 2 + type) * NT + nt) * 8 + kb) * 32 + ln) * 4 + reg * 2 + e;
       qfrag[idx] = __bfloat16_as_ushort(piece ? lo : hi);
     }
+    // sum over dims of mu_p (hi + lo)
+    float c = mu * (__bfloat162float(hi) + __bfloat162float(lo));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if ((i & 31) == 0) red[type][i >> 5] = c;
+  }
+  __syncthreads();
+  if (i < 2) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kD / 32; ++w) t += red[i][w];
+    kconst[(static_cast<size_t>(bh) * 2 + i) * 8 + hl] = t;
   }
 }
 
@@ -563,11 +623,13 @@ size_t frag_bytes(int BH, int G) { return static_cast<size_t>(BH) * 2 * num_tile
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
+size_t kconst_bytes(int BH) { return static_cast<size_t>(BH) * 2 * 8 * sizeof(float); }
+
 size_t workspace_for(int B, int Hq, int Hkv, int64_t T) {
   const int G = Hq / Hkv;
   const int BH = B * Hkv;
   const SplitPlan sp = plan_splits(BH, T);
-  return align256(frag_bytes(BH, G)) +
+  return align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)) +
          align256(static_cast<size_t>(BH) * sp.n_splits * G * (2 + 2 * kD) * sizeof(float));
 }
 
@@ -647,7 +709,8 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   const int NT = num_tiles_n(G);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws);
-  float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)));
+  float* kconst = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)));
+  float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
 
   if (2 * G < 8 * NT) {
     if (cudaMemsetAsync(qfrag, 0, frag_bytes(BH, G), s) != cudaSuccess) return TQ_ECUDA;
@@ -656,12 +719,12 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   if (q_dtype == TQ_F32)
     decode_qprep_kernel<float><<<B * Hq, kD, 0, s>>>(static_cast<const float*>(q), q_pos, Hq, G, NT, hk->d_signs,
                                                        hk->d_st, hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope,
-                                                       reinterpret_cast<uint16_t*>(qfrag));
+                                                       reinterpret_cast<uint16_t*>(qfrag), kconst);
   else
     decode_qprep_kernel<__nv_bfloat16><<<B * Hq, kD, 0, s>>>(static_cast<const __nv_bfloat16*>(q), q_pos, Hq, G, NT,
                                                                hk->d_signs, hk->d_st, hk->d_rope_hi, hk->d_rope_lo,
                                                                hk->rope_max_pos, rope,
-                                                               reinterpret_cast<uint16_t*>(qfrag));
+                                                               reinterpret_cast<uint16_t*>(qfrag), kconst);
   int st = tq::launch_status();
   if (st != TQ_OK) return st;
 
@@ -677,6 +740,7 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   p.chunk = sp.chunk;
   p.n_splits = sp.n_splits;
   p.qfrag = qfrag;
+  p.kconst = kconst;
   p.partial = partial;
   p.score_scale = scale * 1.4426950408889634f;
   p.qjl = static_cast<float>(kQjlConst / hk->m);

@@ -183,6 +183,9 @@ def quantize_kv(rot: Rotation, x, *, pos=None, pos_period: int | None = None, po
 def profile_next_decode(ev_begin, ev_end):
     """Have the next decode_attention call (this thread) record the two
     torch.cuda.Event objects around its split-KV kernel."""
+    for ev in (ev_begin, ev_end):
+        if ev is not None and not ev.cuda_event:
+            ev.record()  # torch creates the underlying cudaEvent lazily, on first record
     _check(_lib.tq_profile_next_decode(ev_begin.cuda_event if ev_begin is not None else None,
                                        ev_end.cuda_event if ev_end is not None else None), "tq_profile_next_decode")
 
