@@ -199,6 +199,38 @@ size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
                                 int B, int Hq, int Hkv, int64_t T);
 
 /*
+ * tq_decode_attention_noalloc - tq_decode_attention for callers that cannot
+ * allocate device memory.  The pages have no counterpart; this entry point
+ * is a deployment convenience.
+ * Callers such as serving runtimes that fix their device memory budget up
+ * front and forbid cudaMalloc afterwards, or plugin hosts that give the
+ * library no allocator, cannot supply the `workspace` of
+ * tq_decode_attention.  This variant takes the same arguments minus the
+ * workspace and uses instead a fixed 16 MiB scratch array compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  It calls no allocating routine.
+ *   - Sizes whose tq_decode_workspace_size(...) exceeds 16 MiB are rejected
+ *     with TQ_EWORKSPACE before anything is launched (e.g. batch 16 x 8 KV
+ *     heads x 32768 tokens with 4 query heads per KV head needs ~6 MB).
+ *   - The first call on each device looks up that device's copy of the
+ *     scratch array (cudaGetSymbolAddress) with that device current; make
+ *     that first call before any stream capture on the device.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents (every call rewrites what it reads, and clears what
+ *     must start at zero).  Calls whose kernels may overlap on the GPU -
+ *     concurrent streams, or host threads racing on one device - race on
+ *     the scratch: serialise them.
+ * Returns the statuses of tq_decode_attention.
+ */
+int tq_decode_attention_noalloc(const tq_rotation* hk, const tq_rotation* hv,
+                                const void* q, int q_dtype, const int64_t* q_pos,
+                                const uint8_t* k_codes, const uint8_t* k_signs,
+                                const float* k_norms, const uint8_t* v_codes,
+                                const uint8_t* v_signs, const float* v_norms,
+                                int64_t cache_stride, int B, int Hq, int Hkv,
+                                int64_t T, float scale, float* out, void* stream);
+
+/*
  * tq_profile_next_decode - instrumentation for benchmarks.  The next
  * tq_decode_attention call made by this host thread records `ev_begin`
  * immediately before and `ev_end` immediately after its split-KV kernel, on

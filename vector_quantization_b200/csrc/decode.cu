@@ -29,6 +29,7 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <mutex>
 
 #include "tq_internal.h"
 
@@ -760,4 +761,53 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   decode_merge_kernel<<<B * Hq, kD, 0, s>>>(partial, Hq, G, sp.n_splits, hv->d_s, hv->d_signs,
                                             static_cast<float>(kQjlConst / hv->m), out);
   return tq::launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Decode attention without any allocation (tq_decode_attention_noalloc).
+//
+// Some callers cannot call cudaMalloc: runtimes that own the device memory
+// budget and forbid allocation once serving starts, hosts that hand the
+// library no allocator, or paths that must never block on or fail in an
+// allocation.  For them the scratch of tq_decode_attention (query operand
+// fragments, per-head constants, split partials) lives in the fixed array
+// below, which every device that loads this library holds until exit.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB per device
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_scratch_addr[kNoAllocMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+extern "C" int tq_decode_attention_noalloc(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
+                                           const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
+                                           const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
+                                           const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv,
+                                           int64_t T, float scale, float* out, void* stream) {
+  if (!hk || !hv) return TQ_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0) return TQ_EINVAL;
+  if (workspace_for(B, Hq, Hkv, T) > kNoAllocScratchBytes) return TQ_EWORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return TQ_ECUDA;
+  void* scratch = nullptr;
+  {
+    // First call on a device: look up this device's copy of the array.  The
+    // host-side name of a __device__ variable is only a stand-in, never a
+    // device address, so the address must come from the runtime.
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_scratch_addr[dev]) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) {
+        cudaGetLastError();
+        return TQ_ECUDA;
+      }
+      g_noalloc_scratch_addr[dev] = addr;
+    }
+    scratch = g_noalloc_scratch_addr[dev];
+  }
+  return tq_decode_attention(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms,
+                             cache_stride, B, Hq, Hkv, T, scale, out, scratch, kNoAllocScratchBytes, stream);
 }
