@@ -199,6 +199,39 @@ size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
                                 int B, int Hq, int Hkv, int64_t T);
 
 /*
+ * tq_encoder_attention - bidirectional attention of S queries per head over
+ * a packed K/V cache (prefill / encoder use).
+ * [TurboESM] §2.A (RoPE before the rotation, so (Pi R_i q)^T (Pi R_j k) keeps
+ * the attention score), §2.E (dequantization, residual correction, Pi^T and
+ * the softmax fused); [TurboQuant] "QJL" (the score estimator).
+ *   hk, hv      handles of K and V (same d in {64, 128}, same bits, Hadamard)
+ *   q           device [B, Hq, S, d] of q_dtype; query s sits at position
+ *               q_pos_offset + s (RoPE when hk has a RoPE base; every such
+ *               position must be below rope_max_pos)
+ *   caches      as in tq_decode_attention: sequence (b, j) at records
+ *               (b*Hkv + j)*cache_stride .. + T-1, 16-byte aligned arrays
+ *   B, Hq, Hkv  Hq % Hkv == 0 (query head h reads KV head h / (Hq/Hkv))
+ *   S, T        queries per head (>= 1) and cached keys per sequence (>= 0)
+ *   scale       softmax scale
+ *   out         device [B, Hq, S, d] float32
+ *   workspace   device scratch of tq_encoder_workspace_size(...) bytes,
+ *               256-byte aligned
+ * No mask: every query sees all T keys.  Returns TQ_OK, TQ_EINVAL,
+ * TQ_EUNSUPPORTED, TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_encoder_attention(const tq_rotation* hk, const tq_rotation* hv,
+                         const void* q, int q_dtype, int64_t q_pos_offset,
+                         const uint8_t* k_codes, const uint8_t* k_signs,
+                         const float* k_norms, const uint8_t* v_codes,
+                         const uint8_t* v_signs, const float* v_norms,
+                         int64_t cache_stride, int B, int Hq, int Hkv, int S,
+                         int64_t T, float scale, float* out, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Workspace bytes tq_encoder_attention needs (0 if invalid). */
+size_t tq_encoder_workspace_size(const tq_rotation* hk, int B, int Hq, int S);
+
+/*
  * tq_decode_attention_noalloc - tq_decode_attention for callers that cannot
  * allocate device memory.  The pages have no counterpart; this entry point
  * is a deployment convenience.

@@ -7,7 +7,8 @@ package resolve lazily so that ``python -m vector_quantization_b200.build``
 can run before the library exists.
 """
 _EXPORTS = ("Rotation", "TQError", "alloc_workspace", "decode_attention", "decode_workspace_size",
-            "empty_records", "lloyd_max", "quantize_kv", "version", "profile_next_decode")
+            "empty_records", "lloyd_max", "quantize_kv", "version", "profile_next_decode",
+            "encoder_attention")
 
 
 def __getattr__(name):

@@ -1,0 +1,114 @@
+// Device helpers shared by the attention kernels: async copies, warp-level
+// MMA wrappers, and the construction of exact tensor-core operands from
+// packed code / sign bit-planes.
+//
+// A b-bit Lloyd-Max code is used in Walsh form,
+//   c[idx] = sum_p w_p s_p(idx),  s_p a product of the code's bits as +-1
+// (b = 1: s_0; b = 2: s_1, s_0; b = 3: s_2, s_1, s_0, s_0 s_1 s_2), so every
+// contraction with dequantized keys or values becomes a sum of contractions
+// with exact +-1 matrices built directly from the packed bits.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+namespace tqdev {
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, int src_bytes) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gsrc), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// D += A B, m16n8k16, bf16 operands, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D += A B, m16n8k16, fp16 operands, fp32 accumulate.
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two bf16 values +-1 from bits x (low half) and x+16 (high half) of w:
+// bit = 1 -> +1.0, bit = 0 -> -1.0 (one shift and one LOP3).
+__device__ __forceinline__ uint32_t pm1_pair(uint32_t w, int x) {
+  const uint32_t t = w << (15 - x);
+  return (~t & 0x80008000u) | 0x3F803F80u;
+}
+
+// Bits j and j+16 of a plane word as a pair of fp16 values in ONE LOP3.
+// The kept bit sits at half-word position p = j + 8 (taken from w << 8) for
+// j < 8, or p = j for j >= 8, inside a fixed fp16 pattern pos_base_h(p):
+// positions 8-9 are mantissa bits of 1.0, 10-14 exponent bits, 15 the sign.
+// The pair element is then v0(p) (bit 0) or v1(p) (bit 1), both exact, so
+// with s = 2 bit - 1 it equals mu_p + sigma_p s.  Callers divide sigma_p
+// out of the other operand and subtract sum_k mu_k B_k once per row/column.
+__host__ __device__ constexpr uint32_t pos_base_h(int p) {
+  return p == 8 ? 0x3C00u : p == 9 ? 0x3C00u : p == 10 ? 0x3800u : p == 11 ? 0x3400u
+       : p == 12 ? 0x2C00u : p == 13 ? 0x1C00u : p == 14 ? 0x0000u : 0x3C00u;
+}
+__device__ __forceinline__ uint32_t bit_pair_h(uint32_t w, uint32_t w_shl8, int j) {
+  const int p = j < 8 ? j + 8 : j;
+  const uint32_t mask = (1u << p) | (1u << (p + 16));
+  return ((j < 8 ? w_shl8 : w) & mask) | (pos_base_h(p) * 0x10001u);
+}
+__host__ __device__ constexpr float pos_v0_h(int p) {
+  return p == 8 ? 1.f : p == 9 ? 1.f : p == 10 ? 0.5f : p == 11 ? 0.25f : p == 12 ? 0.0625f
+       : p == 13 ? 0.00390625f : p == 14 ? 0.f : 1.f;
+}
+__host__ __device__ constexpr float pos_v1_h(int p) {
+  return p == 8 ? 1.25f : p == 9 ? 1.5f : p == 14 ? 2.f : p == 15 ? -1.f : 1.f;
+}
+// Position of pair slot j (see bit_pair_h).
+__host__ __device__ constexpr int slot_pos(int j) { return j < 8 ? j + 8 : j; }
+
+// fp32 bits rounded to the nearest bf16 (ties away from zero), low half zero.
+__device__ __forceinline__ uint32_t bf16_round_bits(float w) { return (__float_as_uint(w) + 0x8000u) & 0xFFFF0000u; }
+
+// Power-of-two factor bringing max |x| to [2^13, 2^14) (1 for x = 0), so
+// that fp16 pieces of scaled values never overflow.
+__device__ __forceinline__ float fp16_range_scale(float max_abs) {
+  if (!(max_abs > 0.f) || !isfinite(max_abs)) return 1.f;
+  int e;
+  frexpf(max_abs, &e);           // max_abs in [2^(e-1), 2^e)
+  return ldexpf(1.f, 14 - e);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
+         (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);
+}
+
+template <int BITS>
+struct Planes {
+  static constexpr int P = BITS == 1 ? 1 : (BITS == 2 ? 2 : 4);
+  // Walsh planes from raw bit-plane words (same element layout in all words).
+  __device__ static __forceinline__ void make(const uint32_t (&raw)[BITS], uint32_t (&out)[P]) {
+    if constexpr (BITS == 1) {
+      out[0] = raw[0];
+    } else if constexpr (BITS == 2) {
+      out[0] = raw[1];
+      out[1] = raw[0];
+    } else {
+      out[0] = raw[2];
+      out[1] = raw[1];
+      out[2] = raw[0];
+      out[3] = raw[0] ^ raw[1] ^ raw[2];  // s0 s1 s2 = +1 iff an odd number of bits are 1
+    }
+  }
+};
+
+}  // namespace tqdev

@@ -31,9 +31,12 @@
 #include <cmath>
 #include <mutex>
 
+#include "bitplane.cuh"
 #include "tq_internal.h"
 
 namespace {
+
+using namespace tqdev;
 
 constexpr int kD = 128;        // head dimension handled here
 constexpr int kWarps = 4;      // warps per CTA
@@ -53,76 +56,12 @@ struct DecodeParams {
   int64_t chunk;           // tokens per split (multiple of kTile)
   int n_splits;
   const uint32_t* qfrag;   // [BH][2][NT][8][32][2]
-  const float* kconst;     // [BH][2][8]
+  const float2* kconst;    // [BH][2][8]: (sum_k mu_k B_k, 1 / fp16 range scale)
   float* partial;          // [BH][n_splits][G][2 + 2 kD]
   float score_scale;       // softmax scale * log2(e)
   float qjl;               // sqrt(pi/2) / m
   float walsh_k[4];
   float walsh_v[4];
-};
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, int src_bytes) {
-  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gsrc), "r"(src_bytes));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Two bf16 values +-1 from bits x (low half) and x+16 (high half) of w:
-// bit = 1 -> +1.0, bit = 0 -> -1.0.
-__device__ __forceinline__ uint32_t pm1_pair(uint32_t w, int x) {
-  const uint32_t t = w << (15 - x);
-  return (~t & 0x80008000u) | 0x3F803F80u;
-}
-
-// Bit j (and j + 16) of a plane word as a pair of bf16 values, one LOP3.
-// The kept bit lands at half-word position p = j + 8 (from w << 8) for j < 8,
-// or p = j for j >= 8: an exponent bit (p = 8..14) or the sign bit (p = 15)
-// of a bf16 whose other bits are the fixed pattern pos_base(p).  The
-// value is then v0 or v1 (kPosV0/kPosV1) - affine in the bit, and exact.
-// With s = 2 bit - 1 it is mu_p + sigma_p s; sigma_p is divided out of the
-// matching B entries and sum mu_p B subtracted once per head (q-prep).
-__host__ __device__ constexpr uint32_t pos_base(int p) {
-  return p == 8 ? 0x3E80u : p == 9 ? 0x3D80u : p == 10 ? 0x3B80u : p == 11 ? 0x3780u
-       : p == 12 ? 0x2F80u : p == 13 ? 0x1F80u : p == 14 ? 0x0000u : 0x3F80u;
-}
-__device__ __forceinline__ uint32_t bit_pair(uint32_t w, uint32_t w_shl8, int j) {
-  const int p = j < 8 ? j + 8 : j;
-  const uint32_t mask = (1u << p) | (1u << (p + 16));
-  return ((j < 8 ? w_shl8 : w) & mask) | (pos_base(p) * 0x10001u);
-}
-__device__ __forceinline__ float pos_v0(int p) {
-  return p == 8 ? 0.25f : p == 9 ? 0.0625f : p == 10 ? 0.00390625f : p == 11 ? 1.52587890625e-05f
-       : p == 12 ? 2.3283064365386963e-10f : p == 13 ? 5.421010862427522e-20f : p == 14 ? 0.f : 1.f;
-}
-__device__ __forceinline__ float pos_v1(int p) { return p == 14 ? 2.f : p == 15 ? -1.f : 1.f; }
-
-template <int BITS>
-struct Planes {
-  static constexpr int P = BITS == 1 ? 1 : (BITS == 2 ? 2 : 4);
-  // Walsh planes from raw bit-plane words (same element layout in all words).
-  __device__ static __forceinline__ void make(const uint32_t (&raw)[BITS], uint32_t (&out)[P]) {
-    if constexpr (BITS == 1) {
-      out[0] = raw[0];
-    } else if constexpr (BITS == 2) {
-      out[0] = raw[1];
-      out[1] = raw[0];
-    } else {
-      out[0] = raw[2];
-      out[1] = raw[1];
-      out[2] = raw[0];
-      out[3] = raw[0] ^ raw[1] ^ raw[2];  // s0 s1 s2 = +1 iff an odd number of bits are 1
-    }
-  }
 };
 
 // Shared-memory position of the 16-byte chunk `part` of token `tok`'s codes.
@@ -191,10 +130,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
     cp_async_commit();
   };
 
-  // B fragments of q~ (type 0) and S q~ (type 1), register order of mma B,
-  // already divided by sigma_p; kc[type][nt] = sum_k mu_k B_k of this head.
+  // fp16 B fragments of q~ (type 0) and S q~ (type 1), register order of mma
+  // B, divided by sigma_p and scaled into fp16 range; kc[type][nt] =
+  // (sum_k mu_k B_k, 1 / scale) of this lane's head.
   uint32_t qf[2][NT][8][2];
-  float kc[2][NT];
+  float2 kc[2][NT];
   {
     const uint32_t* src = p.qfrag + static_cast<size_t>(bh) * (2 * NT * 8 * 32 * 2);
 #pragma unroll
@@ -208,7 +148,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
           qf[t][nt][kb][1] = v.y;
         }
         const int h = tig + 4 * nt;
-        kc[t][nt] = h < G ? p.kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] : 0.f;
+        kc[t][nt] = h < G ? p.kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] : make_float2(0.f, 0.f);
       }
   }
 
@@ -274,15 +214,15 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         const uint32_t s0 = w0 << 8, s1 = w1 << 8;
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb) {
-          const uint32_t a[4] = {bit_pair(w0, s0, 2 * kb), bit_pair(w1, s1, 2 * kb), bit_pair(w0, s0, 2 * kb + 1),
-                                 bit_pair(w1, s1, 2 * kb + 1)};
+          const uint32_t a[4] = {bit_pair_h(w0, s0, 2 * kb), bit_pair_h(w1, s1, 2 * kb),
+                                 bit_pair_h(w0, s0, 2 * kb + 1), bit_pair_h(w1, s1, 2 * kb + 1)};
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_bf16(c[kb & 1][nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
+          for (int nt = 0; nt < NT; ++nt) mma_f16(c[kb & 1][nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const float s0v = (c[0][nt][0] + c[0][nt][1]) + (c[1][nt][0] + c[1][nt][1]) - kc[type][nt];
-          const float s1v = (c[0][nt][2] + c[0][nt][3]) + (c[1][nt][2] + c[1][nt][3]) - kc[type][nt];
+          const float s0v = ((c[0][nt][0] + c[0][nt][1]) + (c[1][nt][0] + c[1][nt][1]) - kc[type][nt].x) * kc[type][nt].y;
+          const float s1v = ((c[0][nt][2] + c[0][nt][3]) + (c[1][nt][2] + c[1][nt][3]) - kc[type][nt].x) * kc[type][nt].y;
           if (pl < P) {
             const float wgt = p.walsh_k[pl < P ? pl : 0];
             code[nt][0] = fmaf(wgt, s0v, code[nt][0]);
@@ -368,7 +308,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         pt[1] = __shfl_sync(0xffffffffu, prob[nt][0], srcB);
         pt[3] = __shfl_sync(0xffffffffu, prob[nt][1], srcB);
         // B = two-term bf16 split of the weight; this lane carries one term:
-        // hi = w truncated to bf16, lo = w - hi (exact) truncated to bf16.
+        // hi = w rounded to bf16, lo = (w - hi) rounded: |w - hi - lo| <= 2^-17 |w|.
         uint32_t bc[P][2], bz[2];
         float wv[4], wr[4];
 #pragma unroll
@@ -376,7 +316,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
           wv[j] = pt[j] * vnorm[j].x;
           wr[j] = pt[j] * vnorm[j].y;
         }
-        auto piece = [&](float w) { return w - __uint_as_float(__float_as_uint(w) & piece_mask); };
+        auto piece = [&](float w) {
+          const uint32_t hi = (__float_as_uint(w) + 0x8000u) & 0xFFFF0000u;
+          const float lo = w - __uint_as_float(hi);
+          return __uint_as_float(((__float_as_uint(lo) + 0x8000u) & piece_mask) | (hi & ~piece_mask));
+        };
 #pragma unroll
         for (int pl = 0; pl < P; ++pl) {
           float t[4];
@@ -467,7 +411,7 @@ __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ 
                                                           const float* __restrict__ st, const float2* __restrict__ rope_hi,
                                                           const float2* __restrict__ rope_lo, int64_t rope_max_pos,
                                                           int rope, uint16_t* __restrict__ qfrag,
-                                                          float* __restrict__ kconst) {
+                                                          float2* __restrict__ kconst) {
   __shared__ float buf[kD];
   __shared__ float red[2][kD / 32];
   const int i = threadIdx.x;
@@ -511,40 +455,51 @@ __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ 
   for (int k = 0; k < kD; ++k) s = fmaf(st[k * kD + i], buf[k], s);
 
   // Scatter into the B-fragment layout of the split kernel.  Dim i sits in
-  // slot j = i & 15 of the word of lane-column tg = i / 32 (the bit_pair
-  // position p of that slot fixes sigma_p, mu_p); hi/lo bf16 pieces go to
-  // columns n = 2 (head % 4) + piece of n-tile head / 4.
+  // pair slot j = i & 15 of the word of lane-column tg = i / 32; that slot's
+  // half-word position fixes (mu_p, sigma_p) of the fp16 bit operand.  The
+  // value x / sigma_p is scaled by a per-head power of two into fp16 range
+  // and split into hi/lo fp16 pieces (columns n = 2 (head % 4) + piece of
+  // n-tile head / 4).
   const int kv = hq / G, hl = hq % G;
   const int bh = b * (Hq / G) + kv;
   const int tg = i >> 5, x = i & 31, e = x >> 4, j = x & 15, reg = j & 1, kb = j >> 1;
-  const int pp = j < 8 ? j + 8 : j;
-  const float v0 = pos_v0(pp), v1 = pos_v1(pp);
-  const float mu = 0.5f * (v0 + v1), sigma = 0.5f * (v1 - v0);
+  const int pp = slot_pos(j);
+  const float mu = 0.5f * (pos_v0_h(pp) + pos_v1_h(pp)), sigma = 0.5f * (pos_v1_h(pp) - pos_v0_h(pp));
   const int nt = hl >> 2;
 #pragma unroll
   for (int type = 0; type < 2; ++type) {
     const float val = (type == 0 ? qt : s) / sigma;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(val);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
+    float mx = fabsf(val);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((i & 31) == 0) red[type][i >> 5] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(red[type][0], red[type][1]), fmaxf(red[type][2], red[type][3]));
+    __syncthreads();
+    const float lam = fp16_range_scale(mx);
+    const float sv = val * lam;
+    const __half hi = __float2half_rn(sv);
+    const __half lo = __float2half_rn(sv - __half2float(hi));
 #pragma unroll
     for (int piece = 0; piece < 2; ++piece) {
       const int n = 2 * (hl & 3) + piece;
       const int ln = 4 * n + tg;
       const size_t idx = ((((static_cast<size_t>(bh) * 2 + type) * NT + nt) * 8 + kb) * 32 + ln) * 4 + reg * 2 + e;
-      qfrag[idx] = __bfloat16_as_ushort(piece ? lo : hi);
+      qfrag[idx] = __half_as_ushort(piece ? lo : hi);
     }
     // sum over dims of mu_p (hi + lo)
-    float c = mu * (__bfloat162float(hi) + __bfloat162float(lo));
+    float c = mu * (__half2float(hi) + __half2float(lo));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    __syncthreads();
     if ((i & 31) == 0) red[type][i >> 5] = c;
-  }
-  __syncthreads();
-  if (i < 2) {
-    float t = 0.f;
+    __syncthreads();
+    if (i == 0) {
+      float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < kD / 32; ++w) t += red[i][w];
-    kconst[(static_cast<size_t>(bh) * 2 + i) * 8 + hl] = t;
+      for (int w = 0; w < kD / 32; ++w) t += red[type][w];
+      kconst[(static_cast<size_t>(bh) * 2 + type) * 8 + hl] = make_float2(t, 1.0f / lam);
+    }
   }
 }
 
@@ -624,7 +579,7 @@ size_t frag_bytes(int BH, int G) { return static_cast<size_t>(BH) * 2 * num_tile
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
-size_t kconst_bytes(int BH) { return static_cast<size_t>(BH) * 2 * 8 * sizeof(float); }
+size_t kconst_bytes(int BH) { return static_cast<size_t>(BH) * 2 * 8 * sizeof(float2); }
 
 size_t workspace_for(int B, int Hq, int Hkv, int64_t T) {
   const int G = Hq / Hkv;
@@ -710,7 +665,7 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   const int NT = num_tiles_n(G);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws);
-  float* kconst = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)));
+  float2* kconst = reinterpret_cast<float2*>(ws + align256(frag_bytes(BH, G)));
   float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
 
   if (2 * G < 8 * NT) {

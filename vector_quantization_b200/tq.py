@@ -46,6 +46,9 @@ def _load():
                                       c_i64, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
         "tq_profile_next_decode": (c_i, [c_p, c_p]),
+        "tq_encoder_attention": (c_i, [c_p, c_p, c_p, c_i, c_i64, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i,
+                                       c_i, c_i, c_i64, c_f, c_p, c_p, c_sz, c_p]),
+        "tq_encoder_workspace_size": (c_sz, [c_p, c_i, c_i, c_i]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -224,4 +227,27 @@ def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cach
                                     _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, T,
                                     float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream_ptr(stream)), "tq_decode_attention")
+    return out
+
+
+def encoder_attention(rot_k: Rotation, rot_v: Rotation, q, k_cache, v_cache, T: int, *, q_pos_offset: int = 0,
+                      scale: float | None = None, out=None, workspace=None, stream=None):
+    """Bidirectional attention: q [B, Hq, S, d] against caches [B, Hkv, cap, ...]
+    (first T records of each sequence).  Returns out [B, Hq, S, d] float32."""
+    import torch
+    B, Hq, S, d = q.shape
+    kc, ks, kn = k_cache
+    vc, vs, vn = v_cache
+    Hkv, cap = kc.shape[1], kc.shape[2]
+    q = q.contiguous()
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((B, Hq, S, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(_lib.tq_encoder_workspace_size(rot_k.handle, B, Hq, S), q.device)
+    _check(_lib.tq_encoder_attention(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), q_pos_offset, _ptr(kc),
+                                     _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, S, T,
+                                     float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                     _stream_ptr(stream)), "tq_encoder_attention")
     return out
