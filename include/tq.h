@@ -163,6 +163,51 @@ int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, int64_t n,
                    void* stream);
 
 /*
+ * tq_quantize_dense - encode n vectors with a dense-rotation handle
+ * (TQ_ROT_DENSE).  Same steps and record format as tq_quantize_kv, without
+ * RoPE; y = Pi x and S r are dense contractions here, computed as fp32 GEMMs
+ * over chunks of vectors.  [TurboQuant] "Principe", Étape 1 / Étape 2, "QJL".
+ *   x           device [n, ld] float32, ld >= d, ld % 4 == 0, 16-byte aligned
+ *   codes, signs, norms  device outputs, records 0..n-1 (contiguous)
+ *   workspace   device scratch, 16-byte aligned; any size of at least
+ *               (d + m) * 4 bytes works - vectors are processed in chunks of
+ *               workspace_bytes / ((d + m) * 4); tq_quantize_dense_workspace_size
+ *               gives a size that processes up to 32768 vectors per chunk
+ * Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED (not a dense handle),
+ * TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_quantize_dense(const tq_rotation* h, const float* x, int64_t n,
+                      int64_t ld, uint8_t* codes, uint8_t* signs, float* norms,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Suggested workspace bytes for tq_quantize_dense of n vectors (0 if invalid). */
+size_t tq_quantize_dense_workspace_size(const tq_rotation* h, int64_t n);
+
+/*
+ * tq_search_topk - brute-force maximum-inner-product top-k from packed codes.
+ * [TurboQuant] "Expériences et résultats", "Performances en recherche
+ * vectorielle" (search without large codebooks) and "QJL" (the estimator):
+ *   score(q, n) = ||x_n|| <Pi q, c[idx_n]> + ||r_n|| sqrt(pi/2)/m <S Pi q, sign(S r_n)>
+ *   h           dense-rotation handle (d % 128 == 0)
+ *   queries     device [nq, d] float32 (16-byte aligned), nq >= 1
+ *   codes, signs, norms  device packed database, records 0..N-1
+ *   k           1..32
+ *   scores, ids device [nq, k] outputs: best first; ties go to the lower id;
+ *               when N < k the tail holds -inf and id -1
+ *   workspace   device scratch of tq_search_workspace_size(...) bytes,
+ *               256-byte aligned
+ * Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_search_topk(const tq_rotation* h, const float* queries, int nq,
+                   const uint8_t* codes, const uint8_t* signs,
+                   const float* norms, int64_t N, int k, float* scores,
+                   int64_t* ids, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/* Workspace bytes tq_search_topk needs (0 if invalid). */
+size_t tq_search_workspace_size(const tq_rotation* h, int nq, int64_t N, int k);
+
+/*
  * tq_decode_attention - one decode step of attention over packed K/V caches.
  * [TurboESM] §2.E: dequantization, residual correction, inverse rotation
  * Pi^T and an online softmax fused in one pass over the cache;

@@ -8,7 +8,7 @@ can run before the library exists.
 """
 _EXPORTS = ("Rotation", "TQError", "alloc_workspace", "decode_attention", "decode_workspace_size",
             "empty_records", "lloyd_max", "quantize_kv", "version", "profile_next_decode",
-            "encoder_attention")
+            "encoder_attention", "quantize_dense", "search_topk", "search_workspace_size")
 
 
 def __getattr__(name):

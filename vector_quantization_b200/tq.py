@@ -49,6 +49,10 @@ def _load():
         "tq_encoder_attention": (c_i, [c_p, c_p, c_p, c_i, c_i64, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i,
                                        c_i, c_i, c_i64, c_f, c_p, c_p, c_sz, c_p]),
         "tq_encoder_workspace_size": (c_sz, [c_p, c_i, c_i, c_i]),
+        "tq_quantize_dense": (c_i, [c_p, c_p, c_i64, c_i64, c_p, c_p, c_p, c_p, c_sz, c_p]),
+        "tq_quantize_dense_workspace_size": (c_sz, [c_p, c_i64]),
+        "tq_search_topk": (c_i, [c_p, c_p, c_i, c_p, c_p, c_p, c_i64, c_i, c_p, c_p, c_p, c_sz, c_p]),
+        "tq_search_workspace_size": (c_sz, [c_p, c_i, c_i64, c_i]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -251,3 +255,43 @@ def encoder_attention(rot_k: Rotation, rot_v: Rotation, q, k_cache, v_cache, T: 
                                      float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                      _stream_ptr(stream)), "tq_encoder_attention")
     return out
+
+
+def quantize_dense(rot: Rotation, x, *, out=None, workspace=None, stream=None):
+    """Encode rows of x ([n, d] float32, CUDA) with a dense-rotation handle.
+    Returns (codes, signs, norms)."""
+    import torch
+    if x.dtype != torch.float32:
+        raise TypeError("quantize_dense takes float32 input")
+    x2 = x.reshape(-1, x.shape[-1])
+    n = x2.shape[0]
+    ld = x2.stride(0) if n > 1 else x2.shape[1]
+    if out is None:
+        out = empty_records(rot, (n,), x.device)
+    codes, signs, norms = out
+    if workspace is None:
+        workspace = alloc_workspace(_lib.tq_quantize_dense_workspace_size(rot.handle, n), x.device)
+    _check(_lib.tq_quantize_dense(rot.handle, _ptr(x2), n, ld, _ptr(codes), _ptr(signs), _ptr(norms),
+                                  _ptr(workspace), workspace.numel(), _stream_ptr(stream)), "tq_quantize_dense")
+    return codes, signs, norms
+
+
+def search_workspace_size(rot: Rotation, nq: int, N: int, k: int) -> int:
+    return _lib.tq_search_workspace_size(rot.handle, nq, N, k)
+
+
+def search_topk(rot: Rotation, queries, db, k: int = 10, *, workspace=None, stream=None):
+    """Top-k inner products of queries ([nq, d] float32) against the packed
+    database db = (codes, signs, norms).  Returns (scores [nq, k], ids [nq, k])."""
+    import torch
+    q = queries.contiguous()
+    nq = q.shape[0]
+    codes, signs, norms = db
+    N = codes.shape[0]
+    scores = torch.empty((nq, k), dtype=torch.float32, device=q.device)
+    ids = torch.empty((nq, k), dtype=torch.int64, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(search_workspace_size(rot, nq, N, k), q.device)
+    _check(_lib.tq_search_topk(rot.handle, _ptr(q), nq, _ptr(codes), _ptr(signs), _ptr(norms), N, k, _ptr(scores),
+                               _ptr(ids), _ptr(workspace), workspace.numel(), _stream_ptr(stream)), "tq_search_topk")
+    return scores, ids
