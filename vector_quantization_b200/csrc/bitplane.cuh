@@ -75,6 +75,23 @@ __host__ __device__ constexpr float pos_v1_h(int p) {
 // Position of pair slot j (see bit_pair_h).
 __host__ __device__ constexpr int slot_pos(int j) { return j < 8 ? j + 8 : j; }
 
+// The same construction for bf16 operands: kept bit at position p = 8..14
+// (bf16 exponent bits) or 15 (sign) inside the pattern pos_base_b(p).
+__host__ __device__ constexpr uint32_t pos_base_b(int p) {
+  return p == 8 ? 0x3E80u : p == 9 ? 0x3D80u : p == 10 ? 0x3B80u : p == 11 ? 0x3780u
+       : p == 12 ? 0x2F80u : p == 13 ? 0x1F80u : p == 14 ? 0x0000u : 0x3F80u;
+}
+__device__ __forceinline__ uint32_t bit_pair_b(uint32_t w, uint32_t w_shl8, int j) {
+  const int p = j < 8 ? j + 8 : j;
+  const uint32_t mask = (1u << p) | (1u << (p + 16));
+  return ((j < 8 ? w_shl8 : w) & mask) | (pos_base_b(p) * 0x10001u);
+}
+__host__ __device__ constexpr float pos_v0_b(int p) {
+  return p == 8 ? 0.25f : p == 9 ? 0.0625f : p == 10 ? 0.00390625f : p == 11 ? 1.52587890625e-05f
+       : p == 12 ? 2.3283064365386963e-10f : p == 13 ? 5.421010862427522e-20f : p == 14 ? 0.f : 1.f;
+}
+__host__ __device__ constexpr float pos_v1_b(int p) { return p == 14 ? 2.f : p == 15 ? -1.f : 1.f; }
+
 // fp32 bits rounded to the nearest bf16 (ties away from zero), low half zero.
 __device__ __forceinline__ uint32_t bf16_round_bits(float w) { return (__float_as_uint(w) + 0x8000u) & 0xFFFF0000u; }
 

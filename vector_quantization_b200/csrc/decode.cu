@@ -154,10 +154,14 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
 
   float accC[NT][8][4], accZ[NT][8][4];
   float m_run[NT], l_run[NT];
+  // Sums of the V-side B values this lane feeds (column n = gid): the value
+  // operand's bit pairs carry an offset mu_p that the epilogue removes.
+  float sbc[NT], sbz[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     m_run[nt] = -INFINITY;
     l_run[nt] = 0.f;
+    sbc[nt] = sbz[nt] = 0.f;
 #pragma unroll
     for (int rb = 0; rb < 8; ++rb)
 #pragma unroll
@@ -250,9 +254,15 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      if (mx > m_run[nt] + kLazyRescale) {
-        const float alpha = exp2f(m_run[nt] - mx);
+      const bool need = mx > m_run[nt] + kLazyRescale;
+      if (__any_sync(0xffffffffu, need)) {
+        // alpha of head tig (accumulators) and of head gid/2 (fed-B sums,
+        // held by lane gid/2 whose tig is gid/2)
+        const float alpha = need ? exp2f(m_run[nt] - mx) : 1.f;
+        const float alpha_b = __shfl_sync(0xffffffffu, alpha, gid >> 1);
         l_run[nt] *= alpha;
+        sbc[nt] *= alpha_b;
+        sbz[nt] *= alpha_b;
 #pragma unroll
         for (int rb = 0; rb < 8; ++rb)
 #pragma unroll
@@ -260,7 +270,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
             accC[nt][rb][r] *= alpha;
             accZ[nt][rb][r] *= alpha;
           }
-        m_run[nt] = mx;
+        if (need) m_run[nt] = mx;
       }
 #pragma unroll
       for (int e = 0; e < 2; ++e) prob[nt][e] = logit[nt][e] == -INFINITY ? 0.f : exp2f(logit[nt][e] - m_run[nt]);
@@ -295,6 +305,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         z01 = __byte_perm(g0, g1, half_sel);
         z23 = __byte_perm(g2, g3, half_sel);
       }
+      uint32_t xs01[P], xs23[P];
+#pragma unroll
+      for (int q = 0; q < P; ++q) {
+        xs01[q] = x01[q] << 8;
+        xs23[q] = x23[q] << 8;
+      }
+      const uint32_t zs01 = z01 << 8, zs23 = z23 << 8;
       float2 vnorm[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) vnorm[j] = vn[tk[j]];
@@ -326,6 +343,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
           float t[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) t[j] = piece(p.walsh_v[pl] * wv[j]);
+          sbc[nt] += (t[0] + t[1]) + (t[2] + t[3]);
           bc[pl][0] = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[1]), 0x7632);
           bc[pl][1] = __byte_perm(__float_as_uint(t[2]), __float_as_uint(t[3]), 0x7632);
         }
@@ -333,19 +351,23 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
           float t[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) t[j] = piece(wr[j]);
+          sbz[nt] += (t[0] + t[1]) + (t[2] + t[3]);
           bz[0] = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[1]), 0x7632);
           bz[1] = __byte_perm(__float_as_uint(t[2]), __float_as_uint(t[3]), 0x7632);
         }
+        // A: bit j of the half-word (dim 16 gid + j) for tokens T0/T1 (x01) and
+        // T2/T3 (x23) as a bf16 pair in one LOP3 (bit_pair_b): row gid takes
+        // j = 2 rb, row gid + 8 takes j = 2 rb + 1.
 #pragma unroll
         for (int rb = 0; rb < 8; ++rb) {
 #pragma unroll
           for (int pl = 0; pl < P; ++pl) {
-            const uint32_t a[4] = {pm1_pair(x01[pl], 2 * rb), pm1_pair(x01[pl], 2 * rb + 1), pm1_pair(x23[pl], 2 * rb),
-                                   pm1_pair(x23[pl], 2 * rb + 1)};
+            const uint32_t a[4] = {bit_pair_b(x01[pl], xs01[pl], 2 * rb), bit_pair_b(x01[pl], xs01[pl], 2 * rb + 1),
+                                   bit_pair_b(x23[pl], xs23[pl], 2 * rb), bit_pair_b(x23[pl], xs23[pl], 2 * rb + 1)};
             mma_bf16(accC[nt][rb], a, bc[pl][0], bc[pl][1]);
           }
-          const uint32_t a[4] = {pm1_pair(z01, 2 * rb), pm1_pair(z01, 2 * rb + 1), pm1_pair(z23, 2 * rb),
-                                 pm1_pair(z23, 2 * rb + 1)};
+          const uint32_t a[4] = {bit_pair_b(z01, zs01, 2 * rb), bit_pair_b(z01, zs01, 2 * rb + 1),
+                                 bit_pair_b(z23, zs23, 2 * rb), bit_pair_b(z23, zs23, 2 * rb + 1)};
           mma_bf16(accZ[nt][rb], a, bz[0], bz[1]);
         }
       }
@@ -367,6 +389,14 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
     l += __shfl_xor_sync(0xffffffffu, l, 4);
     l += __shfl_xor_sync(0xffffffffu, l, 8);
     l += __shfl_xor_sync(0xffffffffu, l, 16);
+    // sum of fed B over the lane's two columns (head tig: hi col 2 tig, lo col 2 tig + 1)
+    float bc_sum = sbc[nt], bz_sum = sbz[nt];
+    bc_sum += __shfl_xor_sync(0xffffffffu, bc_sum, 1);
+    bc_sum += __shfl_xor_sync(0xffffffffu, bc_sum, 2);
+    bz_sum += __shfl_xor_sync(0xffffffffu, bz_sum, 1);
+    bz_sum += __shfl_xor_sync(0xffffffffu, bz_sum, 2);
+    const float SBc = __shfl_sync(0xffffffffu, bc_sum, 8 * tig) + __shfl_sync(0xffffffffu, bc_sum, 8 * tig + 4);
+    const float SBz = __shfl_sync(0xffffffffu, bz_sum, 8 * tig) + __shfl_sync(0xffffffffu, bz_sum, 8 * tig + 4);
     if (h < G) {
       float* dst = mbuf + (warp * G + h) * REC;
       if (gid == 0) {
@@ -376,10 +406,14 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
 #pragma unroll
       for (int rb = 0; rb < 8; ++rb) {
         const int d0 = 16 * gid + 2 * rb;  // rows gid / gid + 8 of row block rb
-        dst[2 + d0] = accC[nt][rb][0] + accC[nt][rb][1];
-        dst[2 + d0 + 1] = accC[nt][rb][2] + accC[nt][rb][3];
-        dst[2 + kD + d0] = accZ[nt][rb][0] + accZ[nt][rb][1];
-        dst[2 + kD + d0 + 1] = accZ[nt][rb][2] + accZ[nt][rb][3];
+        // remove the operand offset: O = (acc - mu_p sum B) / sigma_p
+        const int p0 = slot_pos(2 * rb), p1 = slot_pos(2 * rb + 1);
+        const float mu0 = 0.5f * (pos_v0_b(p0) + pos_v1_b(p0)), is0 = 2.f / (pos_v1_b(p0) - pos_v0_b(p0));
+        const float mu1 = 0.5f * (pos_v0_b(p1) + pos_v1_b(p1)), is1 = 2.f / (pos_v1_b(p1) - pos_v0_b(p1));
+        dst[2 + d0] = (accC[nt][rb][0] + accC[nt][rb][1] - mu0 * SBc) * is0;
+        dst[2 + d0 + 1] = (accC[nt][rb][2] + accC[nt][rb][3] - mu1 * SBc) * is1;
+        dst[2 + kD + d0] = (accZ[nt][rb][0] + accZ[nt][rb][1] - mu0 * SBz) * is0;
+        dst[2 + kD + d0 + 1] = (accZ[nt][rb][2] + accZ[nt][rb][3] - mu1 * SBz) * is1;
       }
     }
   }
