@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--layers", type=int, default=None, help="override layer count (testing only)")
     ap.add_argument("--context", type=int, default=None, help="override context length (testing only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the secondary workload measurements")
     return ap.parse_args()
 
 
@@ -174,6 +175,93 @@ def oracle_baseline(c, args, budget_s=12.0, max_steps=None):
             "sample": f"1 layer x 1 sequence x 1 kv-head ({T} tokens, {G} query heads) per step, "
                       f"{len(times)} steps, {per:.3f} s/step; float64 NumPy"}, len(times), per
 
+
+
+# --------------------------------------------------------------------------- secondary workloads
+def _time_ms(fn, reps=3, warm=2):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_extras(dev, peak_gbs):
+    """Device-timed measurements of the other rows of the path, each on its
+    own workload: encode and decode on the Llama-3.1-70B-shaped 1M-token
+    slice, one ESM-2-650M encoder layer, and 1M-vector d=1536 search."""
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    out = {}
+    # 70B-shaped slice: 1 layer, 8 KV heads, 64 query heads, 2^20 tokens, 2+1 bits
+    c = synth.CONFIGS["llama31_70b_long_slice"]
+    Hkv, Hq, d, T, seed = c["kv_heads"], c["q_heads"], c["head_dim"], c["tokens"], c["seed"]
+    rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 2]))
+    k = synth.heavy_tailed_torch((1, Hkv, T, d), [seed, 3], dev)
+    v = synth.heavy_tailed_torch((1, Hkv, T, d), [seed, 4], dev)
+    kc, vc = tq.empty_records(rk, (1, Hkv, T), dev), tq.empty_records(rv, (1, Hkv, T), dev)
+    def enc():
+        tq.quantize_kv(rk, k, apply_rope=True, pos_period=T, out=kc)
+        tq.quantize_kv(rv, v, out=vc)
+    ms = _time_ms(enc)
+    nvec = 2 * Hkv * T
+    byts = nvec * (2 * d + rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)))
+    out["encode_70b_slice"] = {"vectors": nvec, "ms": round(ms, 4), "vectors_per_s": nvec / ms * 1e3,
+                               "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
+                               "algorithmic_bytes": byts, "note": "bf16 in (256 B) + packed record out (56 B) per vector"}
+    del k, v
+    q = synth.heavy_tailed_torch((1, Hq, d), [seed, 5], dev)
+    qpos = torch.full((1,), T - 1, dtype=torch.int64, device=dev)
+    ws = tq.alloc_workspace(tq.decode_workspace_size(rk, rv, 1, Hq, Hkv, T), dev)
+    o = torch.empty((1, Hq, d), dtype=torch.float32, device=dev)
+    ms = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws), reps=10)
+    byts = Hkv * T * 2 * rec_bytes({"head_dim": d}, argparse.Namespace(bits=2))
+    out["decode_70b_slice"] = {"tokens_per_s": Hkv * T / ms * 1e3, "ms": round(ms, 4),
+                               "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
+                               "note": "G = 8 query heads per KV head; all three launches timed"}
+    del kc, vc
+    # ESM-2-650M encoder layer: [8, 20, 1024, 64] bf16, 2+1 bits, bidirectional attention
+    c = synth.CONFIGS["esm2_650m_encoder"]
+    B, H, T, d, seed = c["batch"], c["heads"], c["tokens"], c["head_dim"], c["seed"]
+    rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 2]))
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    mk = lambda: torch.randn((B, H, T, d), generator=g, device=dev).to(torch.bfloat16)
+    k, v, q = mk(), mk(), mk()
+    kc, vc = tq.quantize_kv(rk, k, apply_rope=True, pos_period=T), tq.quantize_kv(rv, v)
+    o = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+    ws = tq.alloc_workspace(tq._lib.tq_encoder_workspace_size(rk.handle, B, H, T), dev)
+    ms = _time_ms(lambda: tq.encoder_attention(rk, rv, q, kc, vc, T, out=o, workspace=ws))
+    flops = 2 * B * H * T * T * 2 * (d + d)
+    out["encoder_esm2_layer"] = {"ms": round(ms, 4), "TFLOP_s": round(flops / ms / 1e9, 1), "algorithmic_flops": flops,
+                                 "note": "2 B H S T (d + m) MACs for scores and for values; mma.sync tensor pipe"}
+    del k, v, q, kc, vc
+    # vector search: 1M x 1536 fp32, 1000 queries, top-10, 1+1 bits
+    c = synth.CONFIGS["vector_search_d1536"]
+    N, d, nq, kk, seed = c["n_db"], c["dim"], c["n_queries"], c["top_k"], c["seed"]
+    g.manual_seed(seed)
+    lam = (torch.arange(1, d + 1, device=dev, dtype=torch.float32) ** -0.4)
+    db = torch.randn((N, d), generator=g, device=dev) * lam
+    qs = torch.randn((nq, d), generator=g, device=dev) * lam
+    rot = tq.Rotation(d, 1, synth.rotation_randomness(d, [seed, 1], dense=True), kind="dense")
+    wsd = tq.alloc_workspace(tq._lib.tq_quantize_dense_workspace_size(rot.handle, N), dev)
+    packed = tq.empty_records(rot, (N,), dev)
+    ms_enc = _time_ms(lambda: tq.quantize_dense(rot, db, out=packed, workspace=wsd), reps=1, warm=1)
+    wss = tq.alloc_workspace(tq.search_workspace_size(rot, nq, N, kk), dev)
+    ms = _time_ms(lambda: tq.search_topk(rot, qs, packed, kk, workspace=wss), reps=2, warm=1)
+    flops = 2 * nq * N * (d + d)
+    out["search_1m_d1536"] = {"queries_per_s": nq / ms * 1e3, "ms": round(ms, 3), "TFLOP_s": round(flops / ms / 1e9, 1),
+                              "encode_ms": round(ms_enc, 3), "note": "1+1 bits, top-10; data isotropic-in-basis stand-in"}
+    return out
 
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
@@ -332,6 +420,10 @@ def run_ours(args, rank, world, local_rank):
             "clocks": clk}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_baseline(c, args)[0]
+    if world == 1 and not args.no_extras:
+        del kcs, vcs
+        torch.cuda.empty_cache()
+        line["extras"] = run_extras(dev, peak)
     print(json.dumps(line), flush=True)
 
 

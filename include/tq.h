@@ -129,6 +129,18 @@ int tq_free_rotation(tq_rotation* h);
 int tq_rotation_export(const tq_rotation* h, float* pi, float* s,
                        double* levels, double* thresholds);
 
+/*
+ * tq_tensor_core_selftest - diagnostic: runs one 128 x 128 x 128 bf16 product
+ * through the 5th-generation tensor-core path (tcgen05 with operands in
+ * swizzled shared memory and the accumulator in tensor memory) on the
+ * current device, with exactly representable small-integer operands, and
+ * stores in *mismatches the number of result elements that differ from the
+ * exact integer product (0 on a working device).  Synchronous; allocates
+ * and frees its own 64 KB of device memory.  Returns TQ_OK, TQ_EINVAL,
+ * TQ_ENOMEM or TQ_ECUDA.
+ */
+int tq_tensor_core_selftest(int64_t* mismatches);
+
 /* Record geometry of a handle: d, m, bits and bytes of codes / signs. */
 int tq_rotation_dims(const tq_rotation* h, int* d, int* m, int* bits,
                      int64_t* code_bytes, int64_t* sign_bytes);

@@ -106,3 +106,8 @@ def test_encode_rejects_bad_arguments(cuda_device):
     g2 = _gpu_rot(128, 2, 13)
     with pytest.raises(tq.TQError):  # RoPE asked of a handle without RoPE
         tq.quantize_kv(g2, x, apply_rope=True, pos_period=4)
+
+
+def test_tensor_core_selftest(cuda_device):
+    from vector_quantization_b200 import tq
+    assert tq.tensor_core_selftest() == 0

@@ -53,6 +53,7 @@ def _load():
         "tq_quantize_dense_workspace_size": (c_sz, [c_p, c_i64]),
         "tq_search_topk": (c_i, [c_p, c_p, c_i, c_p, c_p, c_p, c_i64, c_i, c_p, c_p, c_p, c_sz, c_p]),
         "tq_search_workspace_size": (c_sz, [c_p, c_i, c_i64, c_i]),
+        "tq_tensor_core_selftest": (c_i, [c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -91,6 +92,14 @@ def _dtype_code(t) -> int:
 
 def version() -> int:
     return _lib.tq_version()
+
+
+def tensor_core_selftest() -> int:
+    """Run the device self-test of the tcgen05 path; returns the number of
+    wrong elements of a 128^3 exact product (0 when working)."""
+    bad = ctypes.c_int64()
+    _check(_lib.tq_tensor_core_selftest(ctypes.byref(bad)), "tq_tensor_core_selftest")
+    return bad.value
 
 
 def lloyd_max(d: int, bits: int):
