@@ -43,6 +43,14 @@ METRIC = "cached tokens scored/s (decode attn, 3-bit KV); % of B200 HBM roofline
 UNIT = "tokens/s"
 
 
+# ncu dram__bytes_read.sum + dram__bytes_write.sum of decode_split_kernel<2,4>
+# per cached token (235,449,600 + 6,678,272 B over 16*8*16384 tokens), or None
+# when the kernel has changed since that capture.
+SPLIT_TRAFFIC_PER_TOKEN = (235_449_600 + 6_678_272) / (16 * 8 * 16384)
+
+EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536")
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -54,6 +62,10 @@ def parse():
     ap.add_argument("--context", type=int, default=None, help="override context length (testing only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary workload measurements")
+    ap.add_argument("--extra", action="append", choices=EXTRAS, default=None,
+                    help="run only this secondary workload (repeatable) and print its measurement")
+    ap.add_argument("--slice-tokens", type=int, default=None,
+                    help="context of the 70B-shaped slice for --extra runs (default 2^20)")
     return ap.parse_args()
 
 
@@ -192,17 +204,36 @@ def _time_ms(fn, reps=3, warm=2):
     return a.elapsed_time(b) / reps
 
 
-def run_extras(dev, peak_gbs):
+def run_extras(dev, peak_gbs, select=None, slice_tokens=None):
     """Device-timed measurements of the other rows of the path, each on its
     own workload: encode and decode on the Llama-3.1-70B-shaped 1M-token
-    slice, one ESM-2-650M encoder layer, and 1M-vector d=1536 search."""
+    slice, one ESM-2-650M encoder layer, and 1M-vector d=1536 search.
+    `select` restricts the run to some of them; `slice_tokens` shrinks the
+    70B-shaped slice (profiling runs)."""
     import torch
     import synth
     from vector_quantization_b200 import tq
     out = {}
+    select = set(select or EXTRAS)
+    g = torch.Generator(device=dev)
     # 70B-shaped slice: 1 layer, 8 KV heads, 64 query heads, 2^20 tokens, 2+1 bits
     c = synth.CONFIGS["llama31_70b_long_slice"]
     Hkv, Hq, d, T, seed = c["kv_heads"], c["q_heads"], c["head_dim"], c["tokens"], c["seed"]
+    T = slice_tokens or T
+    if select & {"encode_70b_slice", "decode_70b_slice"}:
+        out.update(_extras_70b(dev, peak_gbs, select, Hkv, Hq, d, T, seed, c))
+    if "encoder_esm2_layer" in select:
+        out.update(_extra_encoder(dev, g))
+    if "search_1m_d1536" in select:
+        out.update(_extra_search(dev, g))
+    return out
+
+
+def _extras_70b(dev, peak_gbs, select, Hkv, Hq, d, T, seed, c):
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    out = {}
     rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 1]), rope_base=c["rope_base"], rope_max_pos=T)
     rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 2]))
     k = synth.heavy_tailed_torch((1, Hkv, T, d), [seed, 3], dev)
@@ -214,10 +245,14 @@ def run_extras(dev, peak_gbs):
     ms = _time_ms(enc)
     nvec = 2 * Hkv * T
     byts = nvec * (2 * d + rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)))
-    out["encode_70b_slice"] = {"vectors": nvec, "ms": round(ms, 4), "vectors_per_s": nvec / ms * 1e3,
-                               "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
-                               "algorithmic_bytes": byts, "note": "bf16 in (256 B) + packed record out (56 B) per vector"}
+    if "encode_70b_slice" in select:
+        out["encode_70b_slice"] = {"vectors": nvec, "ms": round(ms, 4), "vectors_per_s": nvec / ms * 1e3,
+                                   "GB_s": round(byts / ms / 1e6, 1),
+                                   "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4), "algorithmic_bytes": byts,
+                                   "note": "bf16 in (256 B) + packed record out (56 B) per vector"}
     del k, v
+    if "decode_70b_slice" not in select:
+        return out
     q = synth.heavy_tailed_torch((1, Hq, d), [seed, 5], dev)
     qpos = torch.full((1,), T - 1, dtype=torch.int64, device=dev)
     ws = tq.alloc_workspace(tq.decode_workspace_size(rk, rv, 1, Hq, Hkv, T), dev)
@@ -227,13 +262,19 @@ def run_extras(dev, peak_gbs):
     out["decode_70b_slice"] = {"tokens_per_s": Hkv * T / ms * 1e3, "ms": round(ms, 4),
                                "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
                                "note": "G = 8 query heads per KV head; all three launches timed"}
-    del kc, vc
+    return out
+
+
+def _extra_encoder(dev, g):
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    out = {}
     # ESM-2-650M encoder layer: [8, 20, 1024, 64] bf16, 2+1 bits, bidirectional attention
     c = synth.CONFIGS["esm2_650m_encoder"]
     B, H, T, d, seed = c["batch"], c["heads"], c["tokens"], c["head_dim"], c["seed"]
     rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 1]), rope_base=c["rope_base"], rope_max_pos=T)
     rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 2]))
-    g = torch.Generator(device=dev)
     g.manual_seed(seed)
     mk = lambda: torch.randn((B, H, T, d), generator=g, device=dev).to(torch.bfloat16)
     k, v, q = mk(), mk(), mk()
@@ -244,7 +285,14 @@ def run_extras(dev, peak_gbs):
     flops = 2 * B * H * T * T * 2 * (d + d)
     out["encoder_esm2_layer"] = {"ms": round(ms, 4), "TFLOP_s": round(flops / ms / 1e9, 1), "algorithmic_flops": flops,
                                  "note": "2 B H S T (d + m) MACs for scores and for values; mma.sync tensor pipe"}
-    del k, v, q, kc, vc
+    return out
+
+
+def _extra_search(dev, g):
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    out = {}
     # vector search: 1M x 1536 fp32, 1000 queries, top-10, 1+1 bits
     c = synth.CONFIGS["vector_search_d1536"]
     N, d, nq, kk, seed = c["n_db"], c["dim"], c["n_queries"], c["top_k"], c["seed"]
@@ -406,8 +454,13 @@ def run_ours(args, rank, world, local_rank):
     bytes_per_launch = B * Hkv * T * 2 * rec_bytes(c, args)
     split_avg_s = float(np.mean(split_ms)) / 1e3
     achieved = bytes_per_launch / split_avg_s / 1e9
+    # DRAM bytes per launch of the split kernel, from one ncu capture of the
+    # T = 16384 case (read + write = 242.13 MB), scaled by the token count to
+    # the launch timed here; traffic grows in proportion to the tokens streamed.
+    # Must be reset to None whenever decode_split_kernel changes.
+    traffic = SPLIT_TRAFFIC_PER_TOKEN * B * Hkv * T if SPLIT_TRAFFIC_PER_TOKEN and args.bits == 2 else None
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": traffic,
                 "kernel": "decode_split_kernel (one launch per layer)",
                 "algorithmic_bytes_per_launch": bytes_per_launch, "peak_source": peak_kind,
                 "launch_ms_avg": round(split_avg_s * 1e3, 4)}
@@ -434,6 +487,12 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.extra:
+        import torch
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"extras": run_extras(dev, measured_peaks()[0], args.extra, args.slice_tokens)}), flush=True)
         return
     if world > 1:
         import datetime

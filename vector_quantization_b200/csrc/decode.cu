@@ -438,150 +438,240 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
   }
 }
 
-// One block of kD threads per (b, query head).
-template <typename T>
+// Fast Walsh-Hadamard transform (Sylvester order, unnormalised) of G
+// vectors of kD values, thread i holding coordinate i of each: five stages
+// by warp shuffles, the two across warps through shared memory `buf`.
+template <int G>
+__device__ __forceinline__ void fwht_block(float (&v)[G], float (*buf)[kD]) {
+  const int i = threadIdx.x, lane = i & 31;
+#pragma unroll
+  for (int bit = 1; bit < 32; bit <<= 1) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[h], bit);
+      v[h] = (lane & bit) ? o - v[h] : v[h] + o;
+    }
+  }
+#pragma unroll
+  for (int bit = 32; bit < kD; bit <<= 1) {
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < G; ++h) buf[h][i] = v[h];
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float o = buf[h][i ^ bit];
+      v[h] = (i & bit) ? o - v[h] : v[h] + o;
+    }
+  }
+}
+
+// sum_k col[k] x[h][k] for the G vectors staged in shared memory.
+template <int G>
+__device__ __forceinline__ void matvec_col(const float (&col)[kD], const float (*x)[kD], float (&acc)[G]) {
+#pragma unroll
+  for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll
+  for (int k = 0; k < kD; k += 4) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float4 xv = *reinterpret_cast<const float4*>(&x[h][k]);
+      acc[h] = fmaf(col[k], xv.x, acc[h]);
+      acc[h] = fmaf(col[k + 1], xv.y, acc[h]);
+      acc[h] = fmaf(col[k + 2], xv.z, acc[h]);
+      acc[h] = fmaf(col[k + 3], xv.w, acc[h]);
+    }
+  }
+}
+
+// One block of kD threads per (sequence b, KV head), covering the G query
+// heads of the group: RoPE, q~ = Pi q, s = S q~, then the fp16 B fragments
+// of the split kernel.  Thread i owns coordinate i and loads column i of S^T
+// (row i of S) once for all G heads, at the start, so the loads overlap the
+// rotation.
+template <typename T, int G>
 __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ q, const int64_t* __restrict__ q_pos,
-                                                          int Hq, int G, int NT, const float* __restrict__ dsigns,
+                                                          int Hkv, const float* __restrict__ dsigns,
                                                           const float* __restrict__ st, const float2* __restrict__ rope_hi,
                                                           const float2* __restrict__ rope_lo, int64_t rope_max_pos,
                                                           int rope, uint16_t* __restrict__ qfrag,
                                                           float2* __restrict__ kconst) {
-  __shared__ float buf[kD];
-  __shared__ float red[2][kD / 32];
-  const int i = threadIdx.x;
-  const int bq = blockIdx.x;           // b * Hq + hq
-  const int b = bq / Hq, hq = bq % Hq;
-  float v;
-  if constexpr (sizeof(T) == 4) v = q[static_cast<size_t>(bq) * kD + i];
-  else v = __bfloat162float(q[static_cast<size_t>(bq) * kD + i]);
+  constexpr int NT = (2 * G + 7) / 8;
+  __shared__ __align__(16) float buf[G][kD];
+  __shared__ float red[2][G][2][kD / 32];
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int bh = blockIdx.x;   // b * Hkv + kv; query head h of the group is row bh * G + h of q
+  const int b = bh / Hkv;
+  float scol[kD];
+#pragma unroll
+  for (int k = 0; k < kD; ++k) scol[k] = __ldg(st + k * kD + i);
+  float v[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const size_t at = (static_cast<size_t>(bh) * G + h) * kD + i;
+    if constexpr (sizeof(T) == 4) v[h] = q[at];
+    else v[h] = __bfloat162float(q[at]);
+  }
   if (rope) {
     const int64_t pos = q_pos[b];
-    buf[i] = v;
+#pragma unroll
+    for (int h = 0; h < G; ++h) buf[h][i] = v[h];
     __syncthreads();
     if (pos < 0 || pos >= rope_max_pos) {
-      v = __int_as_float(0x7fc00000);
+#pragma unroll
+      for (int h = 0; h < G; ++h) v[h] = __int_as_float(0x7fc00000);
     } else {
       const int j = i & (kD / 2 - 1);
       const float2 a = rope_hi[(pos >> kRopeLoBits) * (kD / 2) + j];
       const float2 c = rope_lo[(pos & (kRopeLoRows - 1)) * (kD / 2) + j];
       const float cs = a.x * c.x - a.y * c.y, sn = a.y * c.x + a.x * c.y;
-      const float x1 = buf[j], x2 = buf[j + kD / 2];
-      v = i < kD / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float x1 = buf[h][j], x2 = buf[h][j + kD / 2];
+        v[h] = i < kD / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
+      }
     }
-    __syncthreads();
   }
   // q~ = H (D q) / sqrt(d)
-  buf[i] = v * dsigns[i];
+  const float ds = dsigns[i];
+#pragma unroll
+  for (int h = 0; h < G; ++h) v[h] *= ds;
+  fwht_block<G>(v, buf);
+  const float inv_sqrt_d = rsqrtf(static_cast<float>(kD));
   __syncthreads();
 #pragma unroll
-  for (int bit = 1; bit < kD; bit <<= 1) {
-    const float a = buf[i], o = buf[i ^ bit];
-    __syncthreads();
-    buf[i] = (i & bit) ? o - a : a + o;
-    __syncthreads();
+  for (int h = 0; h < G; ++h) {
+    v[h] *= inv_sqrt_d;
+    buf[h][i] = v[h];
   }
-  const float qt = buf[i] * rsqrtf(static_cast<float>(kD));
   __syncthreads();
-  buf[i] = qt;
-  __syncthreads();
-  float s = 0.f;
-#pragma unroll 8
-  for (int k = 0; k < kD; ++k) s = fmaf(st[k * kD + i], buf[k], s);
+  float sv[G];
+  matvec_col<G>(scol, buf, sv);
 
   // Scatter into the B-fragment layout of the split kernel.  Dim i sits in
   // pair slot j = i & 15 of the word of lane-column tg = i / 32; that slot's
   // half-word position fixes (mu_p, sigma_p) of the fp16 bit operand.  The
   // value x / sigma_p is scaled by a per-head power of two into fp16 range
   // and split into hi/lo fp16 pieces (columns n = 2 (head % 4) + piece of
-  // n-tile head / 4).
-  const int kv = hq / G, hl = hq % G;
-  const int bh = b * (Hq / G) + kv;
+  // n-tile head / 4).  Columns of absent heads (G < 4) are zero.
   const int tg = i >> 5, x = i & 31, e = x >> 4, j = x & 15, reg = j & 1, kb = j >> 1;
   const int pp = slot_pos(j);
-  const float mu = 0.5f * (pos_v0_h(pp) + pos_v1_h(pp)), sigma = 0.5f * (pos_v1_h(pp) - pos_v0_h(pp));
-  const int nt = hl >> 2;
+  const float mu = 0.5f * (pos_v0_h(pp) + pos_v1_h(pp)), inv_sigma = 2.f / (pos_v1_h(pp) - pos_v0_h(pp));
+  auto frag_at = [&](int type, int nt, int n) {
+    return ((((static_cast<size_t>(bh) * 2 + type) * NT + nt) * 8 + kb) * 32 + 4 * n + tg) * 4 + reg * 2 + e;
+  };
+  float val[G][2];
 #pragma unroll
-  for (int type = 0; type < 2; ++type) {
-    const float val = (type == 0 ? qt : s) / sigma;
-    float mx = fabsf(val);
+  for (int h = 0; h < G; ++h) {
+    val[h][0] = v[h] * inv_sigma;
+    val[h][1] = sv[h] * inv_sigma;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if ((i & 31) == 0) red[type][i >> 5] = mx;
-    __syncthreads();
-    mx = fmaxf(fmaxf(red[type][0], red[type][1]), fmaxf(red[type][2], red[type][3]));
-    __syncthreads();
-    const float lam = fp16_range_scale(mx);
-    const float sv = val * lam;
-    const __half hi = __float2half_rn(sv);
-    const __half lo = __float2half_rn(sv - __half2float(hi));
+    for (int t = 0; t < 2; ++t) {
+      float mx = fabsf(val[h][t]);
 #pragma unroll
-    for (int piece = 0; piece < 2; ++piece) {
-      const int n = 2 * (hl & 3) + piece;
-      const int ln = 4 * n + tg;
-      const size_t idx = ((((static_cast<size_t>(bh) * 2 + type) * NT + nt) * 8 + kb) * 32 + ln) * 4 + reg * 2 + e;
-      qfrag[idx] = __half_as_ushort(piece ? lo : hi);
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) red[0][h][t][warp] = mx;
     }
-    // sum over dims of mu_p (hi + lo)
-    float c = mu * (__half2float(hi) + __half2float(lo));
+  }
+  __syncthreads();
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    __syncthreads();
-    if ((i & 31) == 0) red[type][i >> 5] = c;
-    __syncthreads();
-    if (i == 0) {
-      float t = 0.f;
+  for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int w = 0; w < kD / 32; ++w) t += red[type][w];
-      kconst[(static_cast<size_t>(bh) * 2 + type) * 8 + hl] = make_float2(t, 1.0f / lam);
+    for (int t = 0; t < 2; ++t) {
+      const float mx = fmaxf(fmaxf(red[0][h][t][0], red[0][h][t][1]), fmaxf(red[0][h][t][2], red[0][h][t][3]));
+      const float lam = fp16_range_scale(mx);
+      const float x2 = val[h][t] * lam;
+      const __half hi = __float2half_rn(x2);
+      const __half lo = __float2half_rn(x2 - __half2float(hi));
+      const int n = 2 * (h & 3);
+      qfrag[frag_at(t, h >> 2, n)] = __half_as_ushort(hi);
+      qfrag[frag_at(t, h >> 2, n + 1)] = __half_as_ushort(lo);
+      float c = mu * (__half2float(hi) + __half2float(lo));   // sum over dims of mu_p (hi + lo)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+      if (lane == 0) red[1][h][t][warp] = c;
+      val[h][t] = lam;
     }
+  if constexpr (2 * G < 8) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      for (int n = 2 * G; n < 8; ++n) qfrag[frag_at(t, 0, n)] = 0;
+  }
+  __syncthreads();
+  if (i < 2 * G) {
+    const int h = i >> 1, t = i & 1;
+    const float c = (red[1][h][t][0] + red[1][h][t][1]) + (red[1][h][t][2] + red[1][h][t][3]);
+    kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] = make_float2(c, 1.0f / val[h][t]);
   }
 }
 
-// One block of kD threads per (b, query head).
-__global__ void __launch_bounds__(kD) decode_merge_kernel(const float* __restrict__ partial, int Hq, int G, int n_splits,
+// One block of kD threads per (sequence b, KV head), covering its G query
+// heads: log-sum-exp merge of the split partials, the QJL value correction
+// sqrt(pi/2)/m S^T O_z, and Pi^T.  Column i of S is loaded once, at the
+// start, for all G heads.  The split weights f_s = 2^(m_s - M) of each head
+// are formed by the lanes of one warp in parallel and staged in shared
+// memory (dynamic, n_splits * G floats), so that each thread's sums over
+// splits are plain independent loads.
+template <int G>
+__global__ void __launch_bounds__(kD) decode_merge_kernel(const float* __restrict__ partial, int n_splits,
                                                          const float* __restrict__ s_mat, const float* __restrict__ dsigns,
                                                          float qjl, float* __restrict__ out) {
-  __shared__ float oz[kD];
-  __shared__ float buf[kD];
-  const int i = threadIdx.x;
-  const int bq = blockIdx.x;
-  const int b = bq / Hq, hq = bq % Hq;
-  const int Hkv = Hq / G;
-  const int bh = b * Hkv + hq / G, hl = hq % G;
   constexpr int REC = 2 + 2 * kD;
-  const float* base = partial + static_cast<size_t>(bh) * n_splits * G * REC + hl * REC;
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, base[static_cast<size_t>(s) * G * REC]);
-  float L = 0.f, oc = 0.f, ozi = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < n_splits; ++s) {
-      const float* rec = base + static_cast<size_t>(s) * G * REC;
+  constexpr int W = kD / 32;
+  __shared__ __align__(16) float oz[G][kD];
+  __shared__ __align__(16) float buf[G][kD];
+  __shared__ float Ls[G];
+  extern __shared__ float fs[];   // [n_splits][G]
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int bh = blockIdx.x;
+  float scol[kD];
+#pragma unroll
+  for (int j = 0; j < kD; ++j) scol[j] = __ldg(s_mat + j * kD + i);
+  const float* base = partial + static_cast<size_t>(bh) * n_splits * G * REC;
+  for (int h = warp; h < G; h += W) {
+    float M = -INFINITY;
+    for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, base[(static_cast<size_t>(s) * G + h) * REC]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float l = 0.f;
+    for (int s = lane; s < n_splits; s += 32) {
+      const float* rec = base + (static_cast<size_t>(s) * G + h) * REC;
       const float ms = rec[0];
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M);
-      L = fmaf(f, rec[1], L);
-      oc = fmaf(f, rec[2 + i], oc);
-      ozi = fmaf(f, rec[2 + kD + i], ozi);
+      const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
+      fs[s * G + h] = f;
+      l = fmaf(f, rec[1], l);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) Ls[h] = l;
   }
-  oz[i] = ozi;
+  __syncthreads();
+  float oc[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float c = 0.f, z = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < n_splits; ++s) {
+      const float f = fs[s * G + h];
+      const float* rec = base + (static_cast<size_t>(s) * G + h) * REC;
+      c = fmaf(f, rec[2 + i], c);
+      z = fmaf(f, rec[2 + kD + i], z);
+    }
+    oc[h] = c;
+    oz[h][i] = z;
+  }
   __syncthreads();
   // rotated-space value: O_code + sqrt(pi/2)/m S^T O_z
-  float corr = 0.f;
-#pragma unroll 8
-  for (int j = 0; j < kD; ++j) corr = fmaf(s_mat[j * kD + i], oz[j], corr);
-  const float y = L > 0.f ? (oc + qjl * corr) / L : 0.f;
-  // Pi^T y = D H y / sqrt(d)
-  buf[i] = y;
-  __syncthreads();
+  float corr[G];
+  matvec_col<G>(scol, oz, corr);
+  float y[G];
 #pragma unroll
-  for (int bit = 1; bit < kD; bit <<= 1) {
-    const float a = buf[i], o = buf[i ^ bit];
-    __syncthreads();
-    buf[i] = (i & bit) ? o - a : a + o;
-    __syncthreads();
-  }
-  out[static_cast<size_t>(bq) * kD + i] = buf[i] * dsigns[i] * rsqrtf(static_cast<float>(kD));
+  for (int h = 0; h < G; ++h) y[h] = Ls[h] > 0.f ? (oc[h] + qjl * corr[h]) / Ls[h] : 0.f;
+  // Pi^T y = D H y / sqrt(d)
+  fwht_block<G>(y, buf);
+  const float f = dsigns[i] * rsqrtf(static_cast<float>(kD));
+#pragma unroll
+  for (int h = 0; h < G; ++h) out[(static_cast<size_t>(bh) * G + h) * kD + i] = y[h] * f;
 }
 
 thread_local cudaEvent_t g_prof_begin = nullptr;
@@ -635,6 +725,43 @@ int launch_split(const DecodeParams& p, int BH, cudaStream_t s) {
     return TQ_ECUDA;
   dim3 grid(p.n_splits, BH);
   kern<<<grid, kWarps * 32, smem, s>>>(p);
+  return tq::launch_status();
+}
+
+template <typename T>
+void qprep_g(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope, uint16_t* qfrag,
+             float2* kconst, cudaStream_t s) {
+#define TQ_QPREP(GG)                                                                                        \
+  decode_qprep_kernel<T, GG><<<BH, kD, 0, s>>>(q, q_pos, Hkv, hk->d_signs, hk->d_st, hk->d_rope_hi, hk->d_rope_lo, \
+                                               hk->rope_max_pos, rope, qfrag, kconst)
+  switch (G) {
+    case 1: TQ_QPREP(1); break;
+    case 2: TQ_QPREP(2); break;
+    case 4: TQ_QPREP(4); break;
+    case 8: TQ_QPREP(8); break;
+  }
+#undef TQ_QPREP
+}
+
+int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
+                 uint16_t* qfrag, float2* kconst, cudaStream_t s) {
+  if (q_dtype == TQ_F32)
+    qprep_g<float>(G, BH, Hkv, static_cast<const float*>(q), q_pos, hk, rope, qfrag, kconst, s);
+  else
+    qprep_g<__nv_bfloat16>(G, BH, Hkv, static_cast<const __nv_bfloat16*>(q), q_pos, hk, rope, qfrag, kconst, s);
+  return TQ_OK;
+}
+
+int launch_merge(int G, int BH, const float* partial, int n_splits, const tq_rotation* hv, float* out, cudaStream_t s) {
+  const float qjl = static_cast<float>(kQjlConst / hv->m);
+  const size_t fsb = static_cast<size_t>(n_splits) * G * sizeof(float);   // <= 1184 * 8 * 4 bytes
+  switch (G) {
+    case 1: decode_merge_kernel<1><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
+    case 2: decode_merge_kernel<2><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
+    case 4: decode_merge_kernel<4><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
+    case 8: decode_merge_kernel<8><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
+    default: return TQ_EUNSUPPORTED;
+  }
   return tq::launch_status();
 }
 
@@ -702,20 +829,10 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   float2* kconst = reinterpret_cast<float2*>(ws + align256(frag_bytes(BH, G)));
   float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
 
-  if (2 * G < 8 * NT) {
-    if (cudaMemsetAsync(qfrag, 0, frag_bytes(BH, G), s) != cudaSuccess) return TQ_ECUDA;
-  }
   const int rope = hk->rope_base > 0.0 ? 1 : 0;
-  if (q_dtype == TQ_F32)
-    decode_qprep_kernel<float><<<B * Hq, kD, 0, s>>>(static_cast<const float*>(q), q_pos, Hq, G, NT, hk->d_signs,
-                                                       hk->d_st, hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope,
-                                                       reinterpret_cast<uint16_t*>(qfrag), kconst);
-  else
-    decode_qprep_kernel<__nv_bfloat16><<<B * Hq, kD, 0, s>>>(static_cast<const __nv_bfloat16*>(q), q_pos, Hq, G, NT,
-                                                               hk->d_signs, hk->d_st, hk->d_rope_hi, hk->d_rope_lo,
-                                                               hk->rope_max_pos, rope,
-                                                               reinterpret_cast<uint16_t*>(qfrag), kconst);
-  int st = tq::launch_status();
+  int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, reinterpret_cast<uint16_t*>(qfrag), kconst, s);
+  if (st != TQ_OK) return st;
+  st = tq::launch_status();
   if (st != TQ_OK) return st;
 
   DecodeParams p{};
@@ -747,9 +864,7 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   }
   if (st != TQ_OK) return st;
   if (prof_end && cudaEventRecord(prof_end, s) != cudaSuccess) return TQ_ECUDA;
-  decode_merge_kernel<<<B * Hq, kD, 0, s>>>(partial, Hq, G, sp.n_splits, hv->d_s, hv->d_signs,
-                                            static_cast<float>(kQjlConst / hv->m), out);
-  return tq::launch_status();
+  return launch_merge(G, BH, partial, sp.n_splits, hv, out, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -7,7 +7,8 @@
 // "QJL" (one sign bit per Johnson-Lindenstrauss projection of the residual);
 // [NSNQuant] §2 (randomized Hadamard transform, H D / sqrt(d)).
 //
-// A CTA encodes tiles of 128 vectors.  Per-vector work runs one warp per
+// A CTA encodes tiles of R vectors (R = 8..128, chosen per call so that
+// small batches still spread over many SMs).  Per-vector work runs one warp per
 // vector: lane l holds coordinates l + 32 j (j < D/32), so the fast
 // Walsh-Hadamard transform needs 5 shuffle stages plus log2(D/32) in-register
 // stages, and a warp ballot over one register yields one 32-bit word of a
@@ -15,12 +16,14 @@
 // advances its cos/sin by one position with an angle-addition step and reads
 // the two-level tables only where positions jump.  The QJL projection S r of
 // the whole tile is a dense product and runs on the 5th-generation tensor
-// core (tcgen05): r is written as bf16 hi/lo pieces into a 128-byte swizzled
-// shared-memory operand, S (bf16-exact) stays resident in shared memory, the
-// fp32 result lands in tensor memory and each thread reads back its vector's
-// row to form the sign bits.
+// core (tcgen05, M = 128 rows; rows past R stay zero): r is written as bf16
+// hi/lo pieces into a 128-byte swizzled shared-memory operand, S (bf16-exact,
+// stored by the handle already in operand layout) stays resident in shared
+// memory, the fp32 result lands in tensor memory and each thread reads back
+// its vector's row to form the sign bits.
 #include <cuda_bf16.h>
 
+#include "bitplane.cuh"
 #include "tcgen05.cuh"
 #include "tq_internal.h"
 
@@ -37,7 +40,8 @@ struct EncodeParams {
   float2* norms;        // record = (||x||, ||r||)
   int64_t out_stride;
   const float* dsigns;  // [D]
-  const float* st;      // [D][D] S transposed (st[i*D + j] = S[j][i])
+  const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
+  int rows;             // vectors per tile, R in {8, 16, 32, 64, 128}
   const float* thresholds;
   const float* levels;
   const float2* rope_hi;
@@ -65,7 +69,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
   constexpr int NT = (1 << BITS) - 1;
   constexpr int OPB = kTileVec * D * 2;           // bytes of one bf16 [128 x D] operand
   constexpr int SB = D * D * 2;                   // bytes of S [m x d] bf16
-  constexpr int RUN = kTileVec / (kEncThreads / 32);   // vectors per warp per tile (contiguous run)
+  const int R = p.rows;                           // vectors per tile
+  const int RUN = R / (kEncThreads / 32);         // vectors per warp per tile (contiguous run)
   extern __shared__ uint8_t raw[];
   __shared__ uint64_t mbar;
   __shared__ uint32_t tmem_slot;
@@ -77,14 +82,17 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
   uint8_t* r_lo = base + SB + OPB;    // residual tile, lo bf16 piece
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < D * D; i += blockDim.x) {
-    const int j = i / D, k = i % D;   // S[j][k] = st[k * D + j]
-    *reinterpret_cast<__nv_bfloat16*>(s_op + tqtc::sw128_offset(j, k, D)) = __float2bfloat16_rn(p.st[k * D + j]);
+  for (int c = tid; c < SB / 16; c += blockDim.x) tqdev::cp_async16(s_op + 16 * c, p.s_op + 8 * c, 16);
+  tqdev::cp_async_commit();
+  if (R < kTileVec) {
+    // rows R..127 of the residual operand are never written: keep them zero
+    for (int c = tid; c < 2 * OPB / 16; c += blockDim.x) reinterpret_cast<uint4*>(r_hi)[c] = make_uint4(0, 0, 0, 0);
   }
   if (tid < NT) thr_s[tid] = p.thresholds[tid];
   if (tid < (1 << BITS)) lev_s[tid] = p.levels[tid];
   if (tid == 0) tqtc::mbar_init(&mbar, 1);
   if (warp == 0) tqtc::tmem_alloc(&tmem_slot, D < 32 ? 32 : D);
+  tqdev::cp_async_wait<0>();
   tqtc::fence_before_sync();
   __syncthreads();
   tqtc::fence_after_sync();
@@ -101,10 +109,10 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
     for (int j = 0; j < NJ / 2; ++j) step[j] = p.rope_lo[(D / 2) + lane + 32 * j];
   }
   uint32_t phase = 0;
-  const int64_t n_tiles = (p.n + kTileVec - 1) / kTileVec;
+  const int64_t n_tiles = (p.n + R - 1) / R;
 
   for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    const int64_t row0 = tile * kTileVec;
+    const int64_t row0 = tile * R;
     // ---------------- per-vector work: warp owns a run of RUN vectors ---------
     float2 cs[NJ / 2 > 0 ? NJ / 2 : 1];
     int64_t prev_pos = -2;
@@ -243,7 +251,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
     {
       const int quad = warp & 3, half = warp >> 2;
       const int v = quad * 32 + lane;
-      const int64_t row = row0 + v;
+      const int64_t row = v < R ? row0 + v : p.n;
       constexpr int COLS = D / 2;
       uint32_t words[COLS / 32];
 #pragma unroll
@@ -278,9 +286,14 @@ int launch_encode(const EncodeParams& p, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (p.n + kTileVec - 1) / kTileVec;
+  // smallest tile (>= 8 rows, one per warp) that still gives each CTA slot work
+  int rows = 8;
+  while (rows < kTileVec && (p.n + rows - 1) / rows > 2LL * sms) rows *= 2;
+  EncodeParams q = p;
+  q.rows = rows;
+  const int64_t tiles = (p.n + rows - 1) / rows;
   const int blocks = static_cast<int>(tiles < sms * 2LL ? tiles : sms * 2LL);
-  kern<<<blocks, kEncThreads, smem, stream>>>(p);
+  kern<<<blocks, kEncThreads, smem, stream>>>(q);
   return tq::launch_status();
 }
 
@@ -332,7 +345,7 @@ extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, in
   p.norms = reinterpret_cast<float2*>(norms);
   p.out_stride = out_stride;
   p.dsigns = h->d_signs;
-  p.st = h->d_st;
+  p.s_op = h->d_s_op;
   p.thresholds = h->d_thresholds;
   p.levels = h->d_levels;
   p.rope_hi = h->d_rope_hi;

@@ -227,6 +227,7 @@ void release(tq_rotation* h) {
   cudaFree(h->d_pi);
   cudaFree(h->d_s);
   cudaFree(h->d_st);
+  cudaFree(h->d_s_op);
   cudaFree(h->d_rope_hi);
   cudaFree(h->d_rope_lo);
   delete h;
@@ -341,6 +342,22 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
       }
     if ((st = upload(&h->d_s, s.data(), s.size())) != TQ_OK) { release(h); return st; }
     if ((st = upload(&h->d_st, stt.data(), stt.size())) != TQ_OK) { release(h); return st; }
+    if (kind == TQ_ROT_HADAMARD) {
+      // K-major bf16 operand with a 128-byte swizzle: K/64 blocks of m rows x
+      // 64 elements; row r of a block at (r/8)*1024 + (r%8)*128 bytes, its
+      // 16-byte chunk c stored at chunk position c ^ (r%8).  S is
+      // bf16-exact, so the upper half of each float is the bf16 value.
+      std::vector<uint16_t> op(static_cast<size_t>(m) * d);
+      for (int j = 0; j < m; ++j)
+        for (int k = 0; k < d; ++k) {
+          const size_t off = static_cast<size_t>(k >> 6) * (static_cast<size_t>(m) * 128) + (j >> 3) * 1024 +
+                             (j & 7) * 128 + ((((k & 63) >> 3) ^ (j & 7)) << 4) + ((k & 7) << 1);
+          uint32_t bits;
+          std::memcpy(&bits, &s[static_cast<size_t>(j) * d + k], 4);
+          op[off / 2] = static_cast<uint16_t>(bits >> 16);
+        }
+      if ((st = upload(&h->d_s_op, op.data(), op.size())) != TQ_OK) { release(h); return st; }
+    }
   }
   if (rope_base > 0.0) {
     const int half = d / 2;

@@ -31,6 +31,9 @@ struct tq_rotation {
   float* d_pi = nullptr;                // [d*d] row-major (dense kind)
   float* d_s = nullptr;                 // [m*d] row-major S (bf16-exact values)
   float* d_st = nullptr;                // [d*m] S transposed
+  // S as bf16 in the tensor-core operand layout (K-major, 128-byte swizzle,
+  // rows = sketch index, K = coordinate); Hadamard kind only.
+  uint16_t* d_s_op = nullptr;
   float2* d_rope_hi = nullptr;          // [rope_hi_rows][d/2] (cos, sin) of h*1024*theta_i
   float2* d_rope_lo = nullptr;          // [1024][d/2]           (cos, sin) of l*theta_i
 };
