@@ -56,14 +56,30 @@ __device__ __forceinline__ uint32_t pm1_pair(uint32_t w, int x) {
 // The pair element is then v0(p) (bit 0) or v1(p) (bit 1), both exact, so
 // with s = 2 bit - 1 it equals mu_p + sigma_p s.  Callers divide sigma_p
 // out of the other operand and subtract sum_k mu_k B_k once per row/column.
+//
+// Every pattern except p = 14 is 1.0 with bit p cleared, so the pair is a
+// bit-select of w under the mask and the register constant `one` = 1.0 in
+// both halves: (w & M) | (one & ~M), one LOP3 with the mask as immediate
+// and a single register shared by all slots (p = 14 is w & M).  `one` must
+// reach the kernel as a runtime value (a kernel parameter), so the compiler
+// cannot fold it into a second immediate.
 __host__ __device__ constexpr uint32_t pos_base_h(int p) {
   return p == 8 ? 0x3C00u : p == 9 ? 0x3C00u : p == 10 ? 0x3800u : p == 11 ? 0x3400u
        : p == 12 ? 0x2C00u : p == 13 ? 0x1C00u : p == 14 ? 0x0000u : 0x3C00u;
 }
-__device__ __forceinline__ uint32_t bit_pair_h(uint32_t w, uint32_t w_shl8, int j) {
-  const int p = j < 8 ? j + 8 : j;
+constexpr uint32_t kOneH2 = 0x3C003C00u;   // fp16 1.0 in both halves
+constexpr uint32_t kOneB2 = 0x3F803F80u;   // bf16 1.0 in both halves
+
+__device__ __forceinline__ uint32_t bit_select(uint32_t w, int p, uint32_t one) {
   const uint32_t mask = (1u << p) | (1u << (p + 16));
-  return ((j < 8 ? w_shl8 : w) & mask) | (pos_base_h(p) * 0x10001u);
+  uint32_t d;
+  if (p == 14) asm("lop3.b32 %0, %1, %2, %3, 0xC0;" : "=r"(d) : "r"(w), "r"(mask), "r"(one));
+  else asm("lop3.b32 %0, %1, %2, %3, 0xE2;" : "=r"(d) : "r"(w), "r"(mask), "r"(one));
+  return d;
+}
+// one_h must hold kOneH2.
+__device__ __forceinline__ uint32_t bit_pair_h(uint32_t w, uint32_t w_shl8, int j, uint32_t one_h) {
+  return bit_select(j < 8 ? w_shl8 : w, j < 8 ? j + 8 : j, one_h);
 }
 __host__ __device__ constexpr float pos_v0_h(int p) {
   return p == 8 ? 1.f : p == 9 ? 1.f : p == 10 ? 0.5f : p == 11 ? 0.25f : p == 12 ? 0.0625f
@@ -76,21 +92,32 @@ __host__ __device__ constexpr float pos_v1_h(int p) {
 __host__ __device__ constexpr int slot_pos(int j) { return j < 8 ? j + 8 : j; }
 
 // The same construction for bf16 operands: kept bit at position p = 8..14
-// (bf16 exponent bits) or 15 (sign) inside the pattern pos_base_b(p).
+// (bf16 exponent bits) or 15 (sign) inside the pattern pos_base_b(p), again
+// 1.0 with bit p cleared except p = 14; one_b must hold kOneB2.
 __host__ __device__ constexpr uint32_t pos_base_b(int p) {
   return p == 8 ? 0x3E80u : p == 9 ? 0x3D80u : p == 10 ? 0x3B80u : p == 11 ? 0x3780u
        : p == 12 ? 0x2F80u : p == 13 ? 0x1F80u : p == 14 ? 0x0000u : 0x3F80u;
 }
-__device__ __forceinline__ uint32_t bit_pair_b(uint32_t w, uint32_t w_shl8, int j) {
-  const int p = j < 8 ? j + 8 : j;
-  const uint32_t mask = (1u << p) | (1u << (p + 16));
-  return ((j < 8 ? w_shl8 : w) & mask) | (pos_base_b(p) * 0x10001u);
+__device__ __forceinline__ uint32_t bit_pair_b(uint32_t w, uint32_t w_shl8, int j, uint32_t one_b) {
+  return bit_select(j < 8 ? w_shl8 : w, j < 8 ? j + 8 : j, one_b);
 }
 __host__ __device__ constexpr float pos_v0_b(int p) {
   return p == 8 ? 0.25f : p == 9 ? 0.0625f : p == 10 ? 0.00390625f : p == 11 ? 1.52587890625e-05f
        : p == 12 ? 2.3283064365386963e-10f : p == 13 ? 5.421010862427522e-20f : p == 14 ? 0.f : 1.f;
 }
 __host__ __device__ constexpr float pos_v1_b(int p) { return p == 14 ? 2.f : p == 15 ? -1.f : 1.f; }
+
+constexpr bool bases_are_one_minus_bit() {
+  for (int p = 8; p < 16; ++p) {
+    if (p == 14) {
+      if (pos_base_h(p) != 0 || pos_base_b(p) != 0) return false;
+    } else if (pos_base_h(p) != (0x3C00u & ~(1u << p)) || pos_base_b(p) != (0x3F80u & ~(1u << p))) {
+      return false;
+    }
+  }
+  return true;
+}
+static_assert(bases_are_one_minus_bit(), "bit_select relies on the patterns being 1.0 with bit p cleared");
 
 // fp32 bits rounded to the nearest bf16 (ties away from zero), low half zero.
 __device__ __forceinline__ uint32_t bf16_round_bits(float w) { return (__float_as_uint(w) + 0x8000u) & 0xFFFF0000u; }

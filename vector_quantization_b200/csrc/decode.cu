@@ -62,6 +62,7 @@ struct DecodeParams {
   float qjl;               // sqrt(pi/2) / m
   float walsh_k[4];
   float walsh_v[4];
+  uint32_t one_h, one_b;   // kOneH2 / kOneB2, passed at run time (see bit_select)
 };
 
 // Shared-memory position of the 16-byte chunk `part` of token `tok`'s codes.
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
   const int gid = lane >> 2, tig = lane & 3;
   const int bh = blockIdx.y;
   const int split = blockIdx.x;
+  const uint32_t one_h = p.one_h, one_b = p.one_b;
   const int64_t t_begin = static_cast<int64_t>(split) * p.chunk;
   const int64_t t_end = min(p.T, t_begin + p.chunk);
   const int n_tiles = t_end > t_begin ? static_cast<int>((t_end - t_begin + kTile - 1) / kTile) : 0;
@@ -218,8 +220,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         const uint32_t s0 = w0 << 8, s1 = w1 << 8;
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb) {
-          const uint32_t a[4] = {bit_pair_h(w0, s0, 2 * kb), bit_pair_h(w1, s1, 2 * kb),
-                                 bit_pair_h(w0, s0, 2 * kb + 1), bit_pair_h(w1, s1, 2 * kb + 1)};
+          const uint32_t a[4] = {bit_pair_h(w0, s0, 2 * kb, one_h), bit_pair_h(w1, s1, 2 * kb, one_h),
+                                 bit_pair_h(w0, s0, 2 * kb + 1, one_h), bit_pair_h(w1, s1, 2 * kb + 1, one_h)};
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) mma_f16(c[kb & 1][nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
         }
@@ -362,12 +364,14 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         for (int rb = 0; rb < 8; ++rb) {
 #pragma unroll
           for (int pl = 0; pl < P; ++pl) {
-            const uint32_t a[4] = {bit_pair_b(x01[pl], xs01[pl], 2 * rb), bit_pair_b(x01[pl], xs01[pl], 2 * rb + 1),
-                                   bit_pair_b(x23[pl], xs23[pl], 2 * rb), bit_pair_b(x23[pl], xs23[pl], 2 * rb + 1)};
+            const uint32_t a[4] = {bit_pair_b(x01[pl], xs01[pl], 2 * rb, one_b),
+                                   bit_pair_b(x01[pl], xs01[pl], 2 * rb + 1, one_b),
+                                   bit_pair_b(x23[pl], xs23[pl], 2 * rb, one_b),
+                                   bit_pair_b(x23[pl], xs23[pl], 2 * rb + 1, one_b)};
             mma_bf16(accC[nt][rb], a, bc[pl][0], bc[pl][1]);
           }
-          const uint32_t a[4] = {bit_pair_b(z01, zs01, 2 * rb), bit_pair_b(z01, zs01, 2 * rb + 1),
-                                 bit_pair_b(z23, zs23, 2 * rb), bit_pair_b(z23, zs23, 2 * rb + 1)};
+          const uint32_t a[4] = {bit_pair_b(z01, zs01, 2 * rb, one_b), bit_pair_b(z01, zs01, 2 * rb + 1, one_b),
+                                 bit_pair_b(z23, zs23, 2 * rb, one_b), bit_pair_b(z23, zs23, 2 * rb + 1, one_b)};
           mma_bf16(accZ[nt][rb], a, bz[0], bz[1]);
         }
       }
@@ -850,6 +854,8 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   p.kconst = kconst;
   p.partial = partial;
   p.score_scale = scale * 1.4426950408889634f;
+  p.one_h = kOneH2;
+  p.one_b = kOneB2;
   p.qjl = static_cast<float>(kQjlConst / hk->m);
   for (int i = 0; i < 4; ++i) {
     p.walsh_k[i] = static_cast<float>(hk->walsh[i]);

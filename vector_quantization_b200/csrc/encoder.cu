@@ -49,6 +49,7 @@ struct EncParams {
   float qjl_k, qjl_v;      // sqrt(pi/2) / m of the K and V handles
   float walsh_k[4];
   float walsh_v[4];
+  uint32_t one_h, one_b;   // kOneH2 / kOneB2, passed at run time (see bit_select)
   const float* v_s;        // [D][D] S_V row-major
   const float* v_signs_d;  // [D] Hadamard signs of the V handle
   float* out;              // [B*Hq][S][D]
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(kWarps * 32) encoder_attention_kernel(EncParam
           const uint32_t w = wk[nt][pl], ws = w << 8;
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb)
-            mma_f16(cc[nt], qa[type][kb], bit_pair_h(w, ws, 2 * kb), bit_pair_h(w, ws, 2 * kb + 1));
+            mma_f16(cc[nt], qa[type][kb], bit_pair_h(w, ws, 2 * kb, p.one_h), bit_pair_h(w, ws, 2 * kb + 1, p.one_h));
         }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
@@ -575,6 +576,8 @@ extern "C" int tq_encoder_attention(const tq_rotation* hk, const tq_rotation* hv
   p.G = Hq / Hkv;
   p.score_scale = scale * 1.4426950408889634f;
   p.qjl_k = static_cast<float>(kQjlConst / hk->m);
+  p.one_h = kOneH2;
+  p.one_b = kOneB2;
   p.qjl_v = static_cast<float>(kQjlConst / hv->m);
   for (int i = 0; i < 4; ++i) {
     p.walsh_k[i] = static_cast<float>(hk->walsh[i]);

@@ -52,6 +52,7 @@ struct SearchParams {
   const float4* qconst;       // [nq_pad]: (K_q, 1/lam_q, K_s, 1/lam_s)
   float qjl;
   float walsh[4];
+  uint32_t one_h;             // kOneH2, passed at run time (see bit_select)
   float* cand_score;          // [n_ranges][nq][k]
   int64_t* cand_id;
 };
@@ -169,8 +170,9 @@ __global__ void __launch_bounds__(kSWarps * 32) search_score_kernel(SearchParams
             bq[t][nt] = *reinterpret_cast<const uint2*>(bb + (((t * 8 + kb) * 2 + nt) * 32 + lane) * 2);
 #pragma unroll
         for (int q = 0; q <= P; ++q) {
-          const uint32_t a[4] = {bit_pair_h(w0[q], ws0[q], 2 * kb), bit_pair_h(w1[q], ws1[q], 2 * kb),
-                                 bit_pair_h(w0[q], ws0[q], 2 * kb + 1), bit_pair_h(w1[q], ws1[q], 2 * kb + 1)};
+          const uint32_t a[4] = {bit_pair_h(w0[q], ws0[q], 2 * kb, p.one_h), bit_pair_h(w1[q], ws1[q], 2 * kb, p.one_h),
+                                 bit_pair_h(w0[q], ws0[q], 2 * kb + 1, p.one_h),
+                                 bit_pair_h(w1[q], ws1[q], 2 * kb + 1, p.one_h)};
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             if (q < P) mma_f16(cacc[q < P ? q : 0][nt], a, bq[0][nt].x, bq[0][nt].y);
@@ -416,6 +418,7 @@ extern "C" int tq_search_topk(const tq_rotation* h, const float* queries, int nq
   p.qconst = reinterpret_cast<const float4*>(ws + L.qconst);
   p.qjl = static_cast<float>(kQjlConst / m);
   for (int i = 0; i < 4; ++i) p.walsh[i] = static_cast<float>(h->walsh[i]);
+  p.one_h = kOneH2;
   p.cand_score = reinterpret_cast<float*>(ws + L.cs);
   p.cand_id = reinterpret_cast<int64_t*>(ws + L.ci);
   switch (h->bits) {
