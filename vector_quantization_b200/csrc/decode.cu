@@ -11,7 +11,11 @@
 //               register order of the main kernel's MMA B operand.
 //  2. split   - per (sequence, token chunk): streams the packed records
 //               through shared memory (cp.async, 4-stage ring per warp),
-//               scores 16 tokens at a time and accumulates the values.
+//               scores 16 tokens at a time and accumulates the values.  The
+//               loop is software-pipelined: the key-side products of tile i
+//               and the value-side products of tile i-1 sit in one loop body,
+//               so the two tensor-core streams overlap; the online-softmax
+//               rescale runs after both, which keeps it exact.
 //  3. merge   - per query head: log-sum-exp merge of the chunk partials, the
 //               QJL value correction S^T acc_s, and Pi^T.
 //
@@ -75,14 +79,14 @@ __device__ __forceinline__ int code_chunk(int tok, int part) {
 }
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kernel(DecodeParams p) {
   constexpr int NT = (2 * G + 7) / 8;
   constexpr int P = Planes<BITS>::P;
-  constexpr int CB = BITS * kD / 8;                 // code bytes per token
-  constexpr int SB = kD / 8;                        // sign bytes per token
-  constexpr int HALF = kTile * (CB + SB + 8);       // K (or V) part of a stage
+  constexpr int CB = BITS * kD / 8;
+  constexpr int SB = kD / 8;
+  constexpr int HALF = kTile * (CB + SB + 8);
   constexpr int STAGE = 2 * HALF;
-  constexpr int CCH = kTile * CB / 16;              // 16-byte chunks of codes per side
+  constexpr int CCH = kTile * CB / 16;
   extern __shared__ __align__(16) uint8_t smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -95,13 +99,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
   const int n_tiles = t_end > t_begin ? static_cast<int>((t_end - t_begin + kTile - 1) / kTile) : 0;
   const int my_count = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
   const int64_t seq = static_cast<int64_t>(bh) * p.cache_stride;
-
   uint8_t* my_stages = smem + warp * kStages * STAGE;
 
-  // Per-lane roles in the tile copy: code chunks (both sides), then sign
-  // chunks (lanes 0-15 K, 16-31 V), then norm chunks (lanes 0-7 K, 8-15 V).
-  // A tile's records are contiguous in every array, so a chunk's source is
-  // the tile base plus 16 bytes per chunk.
   const int sg_side = lane >> 4, sg_c = lane & 15;
   const int nm_side = (lane >> 3) & 1, nm_c = lane & 7;
   auto issue = [&](int i) {
@@ -132,9 +131,6 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
     cp_async_commit();
   };
 
-  // fp16 B fragments of q~ (type 0) and S q~ (type 1), register order of mma
-  // B, divided by sigma_p and scaled into fp16 range; kc[type][nt] =
-  // (sum_k mu_k B_k, 1 / scale) of this lane's head.
   uint32_t qf[2][NT][8][2];
   float2 kc[2][NT];
   {
@@ -153,11 +149,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         kc[t][nt] = h < G ? p.kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] : make_float2(0.f, 0.f);
       }
   }
-
   float accC[NT][8][4], accZ[NT][8][4];
   float m_run[NT], l_run[NT];
-  // Sums of the V-side B values this lane feeds (column n = gid): the value
-  // operand's bit pairs carry an offset mu_p that the epilogue removes.
   float sbc[NT], sbz[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -169,87 +162,107 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
 #pragma unroll
       for (int r = 0; r < 4; ++r) accC[nt][rb][r] = accZ[nt][rb][r] = 0.f;
   }
-  const uint32_t piece_mask = (gid & 1) ? 0xFFFF0000u : 0u;   // V-side B piece of this lane
+  const float piece_m = (gid & 1) ? 1.f : 0.f;   // this lane feeds the hi (0) or lo (1) piece
   const uint32_t half_sel = (gid & 1) ? 0x7632u : 0x5410u;
-
-#pragma unroll 1
-  for (int i = 0; i < kStages - 1; ++i) issue(i);
-
-#pragma unroll 1
-  for (int i = 0; i < my_count; ++i) {
-    cp_async_wait<kStages - 2>();
-    __syncwarp();
-    const uint8_t* stg = my_stages + (i % kStages) * STAGE;
-    const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
-    const int nv = static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
-
-    // ---------------- K side: scores of tokens gid and gid + 8 -------------
-    float logit[NT][2];
-    {
-      const uint8_t* kcd = stg;
-      const uint32_t* ks = reinterpret_cast<const uint32_t*>(stg + kTile * CB);
-      const float2* kn = reinterpret_cast<const float2*>(stg + kTile * (CB + SB));
-      uint32_t wk[2][P + 1];
-      float2 knorm[2];
+  // ---- K side of one tile: logits of tokens gid, gid + 8 for head tig + 4 nt
+  auto k_side = [&](const uint8_t* stg, int nv, float (&logit)[NT][2]) {
+    const uint8_t* kcd = stg;
+    const uint32_t* ks = reinterpret_cast<const uint32_t*>(stg + kTile * CB);
+    const float2* kn = reinterpret_cast<const float2*>(stg + kTile * (CB + SB));
+    uint32_t wk[2][P + 1], ws[2][P + 1];
+    float2 knorm[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tok = gid + 8 * e;
-        uint32_t raw[BITS];
+    for (int e = 0; e < 2; ++e) {
+      const int tok = gid + 8 * e;
+      uint32_t raw[BITS];
 #pragma unroll
-        for (int k = 0; k < BITS; ++k)
-          raw[k] = reinterpret_cast<const uint32_t*>(kcd + code_chunk<BITS>(tok, k) * 16)[tig];
-        uint32_t pl[P];
-        Planes<BITS>::make(raw, pl);
+      for (int k = 0; k < BITS; ++k)
+        raw[k] = reinterpret_cast<const uint32_t*>(kcd + code_chunk<BITS>(tok, k) * 16)[tig];
+      uint32_t pl[P];
+      Planes<BITS>::make(raw, pl);
 #pragma unroll
-        for (int q = 0; q < P; ++q) wk[e][q] = pl[q];
-        wk[e][P] = ks[tok * (SB / 4) + tig];
-        knorm[e] = kn[tok];
+      for (int q = 0; q < P; ++q) wk[e][q] = pl[q];
+      wk[e][P] = ks[tok * (SB / 4) + tig];
+      knorm[e] = kn[tok];
+#pragma unroll
+      for (int q = 0; q <= P; ++q) ws[e][q] = wk[e][q] << 8;
+    }
+    float code[NT][2], zsc[NT][2];
+    if constexpr (NT == 1) {
+      // one accumulator per plane; planes interleaved per k-block (three
+      // independent tensor-core chains)
+      float c[P + 1][NT][4];
+#pragma unroll
+      for (int pl = 0; pl <= P; ++pl)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) c[pl][nt][0] = c[pl][nt][1] = c[pl][nt][2] = c[pl][nt][3] = 0.f;
+#pragma unroll
+      for (int kb = 0; kb < 8; ++kb) {
+#pragma unroll
+        for (int pl = 0; pl <= P; ++pl) {
+          const int type = pl < P ? 0 : 1;
+          const uint32_t a[4] = {bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb, one_h),
+                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb, one_h),
+                                 bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb + 1, one_h),
+                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb + 1, one_h)};
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_f16(c[pl][nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
+        }
       }
-      float code[NT][2], zs[NT][2];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) code[nt][0] = code[nt][1] = zs[nt][0] = zs[nt][1] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) {
+        code[nt][0] = code[nt][1] = 0.f;
+#pragma unroll
+        for (int pl = 0; pl < P; ++pl) {
+          code[nt][0] = fmaf(p.walsh_k[pl], (c[pl][nt][0] + c[pl][nt][1] - kc[0][nt].x) * kc[0][nt].y, code[nt][0]);
+          code[nt][1] = fmaf(p.walsh_k[pl], (c[pl][nt][2] + c[pl][nt][3] - kc[0][nt].x) * kc[0][nt].y, code[nt][1]);
+        }
+        zsc[nt][0] = (c[P][nt][0] + c[P][nt][1] - kc[1][nt].x) * kc[1][nt].y;
+        zsc[nt][1] = (c[P][nt][2] + c[P][nt][3] - kc[1][nt].x) * kc[1][nt].y;
+      }
+    } else {
+      // two n-tiles (G = 8): planes one after the other, one accumulator set
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) code[nt][0] = code[nt][1] = 0.f;
 #pragma unroll
       for (int pl = 0; pl <= P; ++pl) {
         const int type = pl < P ? 0 : 1;
-        float c[2][NT][4];
+        float c[NT][4];
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) c[u][nt][0] = c[u][nt][1] = c[u][nt][2] = c[u][nt][3] = 0.f;
-        const uint32_t w0 = wk[0][pl], w1 = wk[1][pl];
-        const uint32_t s0 = w0 << 8, s1 = w1 << 8;
+        for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
 #pragma unroll
         for (int kb = 0; kb < 8; ++kb) {
-          const uint32_t a[4] = {bit_pair_h(w0, s0, 2 * kb, one_h), bit_pair_h(w1, s1, 2 * kb, one_h),
-                                 bit_pair_h(w0, s0, 2 * kb + 1, one_h), bit_pair_h(w1, s1, 2 * kb + 1, one_h)};
+          const uint32_t a[4] = {bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb, one_h),
+                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb, one_h),
+                                 bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb + 1, one_h),
+                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb + 1, one_h)};
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16(c[kb & 1][nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
+          for (int nt = 0; nt < NT; ++nt) mma_f16(c[nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const float s0v = ((c[0][nt][0] + c[0][nt][1]) + (c[1][nt][0] + c[1][nt][1]) - kc[type][nt].x) * kc[type][nt].y;
-          const float s1v = ((c[0][nt][2] + c[0][nt][3]) + (c[1][nt][2] + c[1][nt][3]) - kc[type][nt].x) * kc[type][nt].y;
+          const float s0v = (c[nt][0] + c[nt][1] - kc[type][nt].x) * kc[type][nt].y;
+          const float s1v = (c[nt][2] + c[nt][3] - kc[type][nt].x) * kc[type][nt].y;
           if (pl < P) {
-            const float wgt = p.walsh_k[pl < P ? pl : 0];
-            code[nt][0] = fmaf(wgt, s0v, code[nt][0]);
-            code[nt][1] = fmaf(wgt, s1v, code[nt][1]);
+            code[nt][0] = fmaf(p.walsh_k[pl < P ? pl : 0], s0v, code[nt][0]);
+            code[nt][1] = fmaf(p.walsh_k[pl < P ? pl : 0], s1v, code[nt][1]);
           } else {
-            zs[nt][0] = s0v;
-            zs[nt][1] = s1v;
+            zsc[nt][0] = s0v;
+            zsc[nt][1] = s1v;
           }
         }
       }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float s = fmaf(knorm[e].x, code[nt][e], knorm[e].y * p.qjl * zs[nt][e]) * p.score_scale;
-          logit[nt][e] = (gid + 8 * e) < nv ? s : -INFINITY;
-        }
     }
-
-    // ---------------- online softmax (head tig + 4 nt per thread) ----------
-    float prob[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float l0 = fmaf(knorm[0].x, code[nt][0], knorm[0].y * p.qjl * zsc[nt][0]) * p.score_scale;
+      const float l1 = fmaf(knorm[1].x, code[nt][1], knorm[1].y * p.qjl * zsc[nt][1]) * p.score_scale;
+      logit[nt][0] = gid < nv ? l0 : -INFINITY;
+      logit[nt][1] = gid + 8 < nv ? l1 : -INFINITY;
+    }
+  };
+  // ---- online softmax: new running max (rescaling what is accumulated) and p
+  auto softmax = [&](const float (&logit)[NT][2], float (&prob)[NT][2]) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float mx = fmaxf(logit[nt][0], logit[nt][1]);
@@ -258,8 +271,6 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const bool need = mx > m_run[nt] + kLazyRescale;
       if (__any_sync(0xffffffffu, need)) {
-        // alpha of head tig (accumulators) and of head gid/2 (fed-B sums,
-        // held by lane gid/2 whose tig is gid/2)
         const float alpha = need ? exp2f(m_run[nt] - mx) : 1.f;
         const float alpha_b = __shfl_sync(0xffffffffu, alpha, gid >> 1);
         l_run[nt] *= alpha;
@@ -275,115 +286,154 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
         if (need) m_run[nt] = mx;
       }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) prob[nt][e] = logit[nt][e] == -INFINITY ? 0.f : exp2f(logit[nt][e] - m_run[nt]);
+      for (int e = 0; e < 2; ++e) prob[nt][e] = exp2f(logit[nt][e] - m_run[nt]);
       l_run[nt] += prob[nt][0] + prob[nt][1];
     }
+  };
 
-    // ---------------- V side -------------------------------------------------
+  // ---- V side of one tile with its probabilities
+  auto v_side = [&](const uint8_t* stg, const float (&prob)[NT][2]) {
+    const uint8_t* vcd = stg + HALF;
+    const uint8_t* vs = vcd + kTile * CB;
+    const float2* vn = reinterpret_cast<const float2*>(vcd + kTile * (CB + SB));
+    const int tk[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+    uint32_t x01[P], x23[P], z01, z23;
     {
-      const uint8_t* vcd = stg + HALF;
-      const uint8_t* vs = vcd + kTile * CB;
-      const float2* vn = reinterpret_cast<const float2*>(vcd + kTile * (CB + SB));
-      const int tk[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
-      uint32_t x01[P], x23[P], z01, z23;
-      {
-        // half-word gid of each plane: dims 16 gid .. 16 gid + 15
-        uint32_t r01[BITS], r23[BITS];
+      uint32_t r01[BITS], r23[BITS];
 #pragma unroll
-        for (int k = 0; k < BITS; ++k) {
-          const uint32_t h0 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[0], k) * 16)[gid >> 1];
-          const uint32_t h1 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[1], k) * 16)[gid >> 1];
-          const uint32_t h2 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[2], k) * 16)[gid >> 1];
-          const uint32_t h3 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[3], k) * 16)[gid >> 1];
-          r01[k] = __byte_perm(h0, h1, half_sel);
-          r23[k] = __byte_perm(h2, h3, half_sel);
-        }
-        Planes<BITS>::make(r01, x01);
-        Planes<BITS>::make(r23, x23);
-        const uint32_t g0 = reinterpret_cast<const uint32_t*>(vs + tk[0] * SB)[gid >> 1];
-        const uint32_t g1 = reinterpret_cast<const uint32_t*>(vs + tk[1] * SB)[gid >> 1];
-        const uint32_t g2 = reinterpret_cast<const uint32_t*>(vs + tk[2] * SB)[gid >> 1];
-        const uint32_t g3 = reinterpret_cast<const uint32_t*>(vs + tk[3] * SB)[gid >> 1];
-        z01 = __byte_perm(g0, g1, half_sel);
-        z23 = __byte_perm(g2, g3, half_sel);
+      for (int k = 0; k < BITS; ++k) {
+        const uint32_t h0 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[0], k) * 16)[gid >> 1];
+        const uint32_t h1 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[1], k) * 16)[gid >> 1];
+        const uint32_t h2 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[2], k) * 16)[gid >> 1];
+        const uint32_t h3 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[3], k) * 16)[gid >> 1];
+        r01[k] = __byte_perm(h0, h1, half_sel);
+        r23[k] = __byte_perm(h2, h3, half_sel);
       }
-      uint32_t xs01[P], xs23[P];
+      Planes<BITS>::make(r01, x01);
+      Planes<BITS>::make(r23, x23);
+      const uint32_t g0 = reinterpret_cast<const uint32_t*>(vs + tk[0] * SB)[gid >> 1];
+      const uint32_t g1 = reinterpret_cast<const uint32_t*>(vs + tk[1] * SB)[gid >> 1];
+      const uint32_t g2 = reinterpret_cast<const uint32_t*>(vs + tk[2] * SB)[gid >> 1];
+      const uint32_t g3 = reinterpret_cast<const uint32_t*>(vs + tk[3] * SB)[gid >> 1];
+      z01 = __byte_perm(g0, g1, half_sel);
+      z23 = __byte_perm(g2, g3, half_sel);
+    }
+    uint32_t xs01[P], xs23[P];
 #pragma unroll
-      for (int q = 0; q < P; ++q) {
-        xs01[q] = x01[q] << 8;
-        xs23[q] = x23[q] << 8;
+    for (int q = 0; q < P; ++q) {
+      xs01[q] = x01[q] << 8;
+      xs23[q] = x23[q] << 8;
+    }
+    const uint32_t zs01 = z01 << 8, zs23 = z23 << 8;
+    float2 vnorm[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) vnorm[j] = vn[tk[j]];
+    const int srcA = (2 * tig) * 4 + (gid >> 1);
+    const int srcB = (2 * tig + 1) * 4 + (gid >> 1);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float pt[4];
+      pt[0] = __shfl_sync(0xffffffffu, prob[nt][0], srcA);
+      pt[2] = __shfl_sync(0xffffffffu, prob[nt][1], srcA);
+      pt[1] = __shfl_sync(0xffffffffu, prob[nt][0], srcB);
+      pt[3] = __shfl_sync(0xffffffffu, prob[nt][1], srcB);
+      uint32_t bc[P][2], bz[2];
+      float wv[4], wr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        wv[j] = pt[j] * vnorm[j].x;
+        wr[j] = pt[j] * vnorm[j].y;
       }
-      const uint32_t zs01 = z01 << 8, zs23 = z23 << 8;
-      float2 vnorm[4];
+      // B operand: lanes of even gid feed RN(w), odd gid RN(w - RN(w)), both
+      // as bf16 pairs: one paired conversion, an FFMA by piece_m in {0, 1},
+      // one paired conversion out (|w - hi - lo| <= 2^-17 |w|).
+      auto pair2 = [&](float a, float b) -> uint32_t {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        const uint32_t hb = *reinterpret_cast<uint32_t*>(&h);
+        const float ha = __uint_as_float(hb << 16), hbf = __uint_as_float(hb & 0xFFFF0000u);
+        __nv_bfloat162 r = __floats2bfloat162_rn(fmaf(-piece_m, ha, a), fmaf(-piece_m, hbf, b));
+        return *reinterpret_cast<uint32_t*>(&r);
+      };
 #pragma unroll
-      for (int j = 0; j < 4; ++j) vnorm[j] = vn[tk[j]];
-      const int srcA = (2 * tig) * 4 + (gid >> 1);
-      const int srcB = (2 * tig + 1) * 4 + (gid >> 1);
+      for (int pl = 0; pl < P; ++pl) {
+        bc[pl][0] = pair2(p.walsh_v[pl] * wv[0], p.walsh_v[pl] * wv[1]);
+        bc[pl][1] = pair2(p.walsh_v[pl] * wv[2], p.walsh_v[pl] * wv[3]);
+      }
+      bz[0] = pair2(wr[0], wr[1]);
+      bz[1] = pair2(wr[2], wr[3]);
+      // unrounded weight sums for the offset mu_p sum B (hi + lo differ from
+      // w by at most 2^-17 |w|, far inside the output tolerance)
+      sbc[nt] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
+      sbz[nt] += (wr[0] + wr[1]) + (wr[2] + wr[3]);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float pt[4];
-        pt[0] = __shfl_sync(0xffffffffu, prob[nt][0], srcA);
-        pt[2] = __shfl_sync(0xffffffffu, prob[nt][1], srcA);
-        pt[1] = __shfl_sync(0xffffffffu, prob[nt][0], srcB);
-        pt[3] = __shfl_sync(0xffffffffu, prob[nt][1], srcB);
-        // B = two-term bf16 split of the weight; this lane carries one term:
-        // hi = w rounded to bf16, lo = (w - hi) rounded: |w - hi - lo| <= 2^-17 |w|.
-        uint32_t bc[P][2], bz[2];
-        float wv[4], wr[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          wv[j] = pt[j] * vnorm[j].x;
-          wr[j] = pt[j] * vnorm[j].y;
-        }
-        auto piece = [&](float w) {
-          const uint32_t hi = (__float_as_uint(w) + 0x8000u) & 0xFFFF0000u;
-          const float lo = w - __uint_as_float(hi);
-          return __uint_as_float(((__float_as_uint(lo) + 0x8000u) & piece_mask) | (hi & ~piece_mask));
-        };
+      for (int rb = 0; rb < 8; ++rb) {
 #pragma unroll
         for (int pl = 0; pl < P; ++pl) {
-          float t[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) t[j] = piece(p.walsh_v[pl] * wv[j]);
-          sbc[nt] += (t[0] + t[1]) + (t[2] + t[3]);
-          bc[pl][0] = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[1]), 0x7632);
-          bc[pl][1] = __byte_perm(__float_as_uint(t[2]), __float_as_uint(t[3]), 0x7632);
+          const uint32_t a[4] = {bit_pair_b(x01[pl], xs01[pl], 2 * rb, one_b),
+                                 bit_pair_b(x01[pl], xs01[pl], 2 * rb + 1, one_b),
+                                 bit_pair_b(x23[pl], xs23[pl], 2 * rb, one_b),
+                                 bit_pair_b(x23[pl], xs23[pl], 2 * rb + 1, one_b)};
+          mma_bf16(accC[nt][rb], a, bc[pl][0], bc[pl][1]);
         }
-        {
-          float t[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) t[j] = piece(wr[j]);
-          sbz[nt] += (t[0] + t[1]) + (t[2] + t[3]);
-          bz[0] = __byte_perm(__float_as_uint(t[0]), __float_as_uint(t[1]), 0x7632);
-          bz[1] = __byte_perm(__float_as_uint(t[2]), __float_as_uint(t[3]), 0x7632);
-        }
-        // A: bit j of the half-word (dim 16 gid + j) for tokens T0/T1 (x01) and
-        // T2/T3 (x23) as a bf16 pair in one LOP3 (bit_pair_b): row gid takes
-        // j = 2 rb, row gid + 8 takes j = 2 rb + 1.
-#pragma unroll
-        for (int rb = 0; rb < 8; ++rb) {
-#pragma unroll
-          for (int pl = 0; pl < P; ++pl) {
-            const uint32_t a[4] = {bit_pair_b(x01[pl], xs01[pl], 2 * rb, one_b),
-                                   bit_pair_b(x01[pl], xs01[pl], 2 * rb + 1, one_b),
-                                   bit_pair_b(x23[pl], xs23[pl], 2 * rb, one_b),
-                                   bit_pair_b(x23[pl], xs23[pl], 2 * rb + 1, one_b)};
-            mma_bf16(accC[nt][rb], a, bc[pl][0], bc[pl][1]);
-          }
-          const uint32_t a[4] = {bit_pair_b(z01, zs01, 2 * rb, one_b), bit_pair_b(z01, zs01, 2 * rb + 1, one_b),
-                                 bit_pair_b(z23, zs23, 2 * rb, one_b), bit_pair_b(z23, zs23, 2 * rb + 1, one_b)};
-          mma_bf16(accZ[nt][rb], a, bz[0], bz[1]);
-        }
+        const uint32_t a[4] = {bit_pair_b(z01, zs01, 2 * rb, one_b), bit_pair_b(z01, zs01, 2 * rb + 1, one_b),
+                               bit_pair_b(z23, zs23, 2 * rb, one_b), bit_pair_b(z23, zs23, 2 * rb + 1, one_b)};
+        mma_bf16(accZ[nt][rb], a, bz[0], bz[1]);
       }
     }
-    __syncwarp();
-    issue(i + kStages - 1);
+  };
+  auto tile_nv = [&](int i) {
+    const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
+    return static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
+  };
+
+#pragma unroll 1
+  for (int i = 0; i < kStages - 1; ++i) issue(i);
+
+  // Pipelined order for G <= 4; with G = 8 the two tiles' live values would
+  // not fit the register file, so tiles run one after the other.
+  constexpr bool kPipe = G <= 4;
+  if constexpr (kPipe) {
+    float prob_prev[NT][2];
+    const uint8_t* stg_prev = my_stages;
+    if (my_count > 0) {
+      cp_async_wait<kStages - 2>();
+      __syncwarp();
+      float logit[NT][2];
+      k_side(my_stages, tile_nv(0), logit);
+      softmax(logit, prob_prev);
+      issue(kStages - 1);   // stage kStages-1 is still unused
+    }
+#pragma unroll 1
+    for (int i = 1; i < my_count; ++i) {
+      cp_async_wait<kStages - 2>();
+      __syncwarp();
+      const uint8_t* stg = my_stages + (i % kStages) * STAGE;
+      float logit[NT][2];
+      k_side(stg, tile_nv(i), logit);   // independent of the V side below
+      v_side(stg_prev, prob_prev);
+      softmax(logit, prob_prev);
+      stg_prev = stg;
+      __syncwarp();
+      issue(i + kStages - 1);           // into the stage of tile i - 1
+    }
+    if (my_count > 0) v_side(stg_prev, prob_prev);
+  } else {
+#pragma unroll 1
+    for (int i = 0; i < my_count; ++i) {
+      cp_async_wait<kStages - 2>();
+      __syncwarp();
+      const uint8_t* stg = my_stages + (i % kStages) * STAGE;
+      float logit[NT][2], prob[NT][2];
+      k_side(stg, tile_nv(i), logit);
+      softmax(logit, prob);
+      v_side(stg, prob);
+      __syncwarp();
+      issue(i + kStages - 1);           // into the stage of tile i - 1
+    }
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // ---------------- merge the 4 warps of this CTA ---------------------------
-  // merge buffer per warp: [G][2 + 2 kD]  (m, l, O_code[kD], O_z[kD])
   constexpr int REC = 2 + 2 * kD;
   float* mbuf = reinterpret_cast<float*>(smem);
 #pragma unroll
@@ -393,14 +443,19 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
     l += __shfl_xor_sync(0xffffffffu, l, 4);
     l += __shfl_xor_sync(0xffffffffu, l, 8);
     l += __shfl_xor_sync(0xffffffffu, l, 16);
-    // sum of fed B over the lane's two columns (head tig: hi col 2 tig, lo col 2 tig + 1)
     float bc_sum = sbc[nt], bz_sum = sbz[nt];
     bc_sum += __shfl_xor_sync(0xffffffffu, bc_sum, 1);
     bc_sum += __shfl_xor_sync(0xffffffffu, bc_sum, 2);
     bz_sum += __shfl_xor_sync(0xffffffffu, bz_sum, 1);
     bz_sum += __shfl_xor_sync(0xffffffffu, bz_sum, 2);
-    const float SBc = __shfl_sync(0xffffffffu, bc_sum, 8 * tig) + __shfl_sync(0xffffffffu, bc_sum, 8 * tig + 4);
-    const float SBz = __shfl_sync(0xffffffffu, bz_sum, 8 * tig) + __shfl_sync(0xffffffffu, bz_sum, 8 * tig + 4);
+    // column sums of the fed B over the split: every lane holds the full
+    // weights of its tokens, so one lane of the head's (hi, lo) pair suffices;
+    // the code operand of plane p carried walsh_v[p] w
+    float wsum = 0.f;
+#pragma unroll
+    for (int pl = 0; pl < P; ++pl) wsum += p.walsh_v[pl];
+    const float SBc = __shfl_sync(0xffffffffu, bc_sum, 8 * tig) * wsum;
+    const float SBz = __shfl_sync(0xffffffffu, bz_sum, 8 * tig);
     if (h < G) {
       float* dst = mbuf + (warp * G + h) * REC;
       if (gid == 0) {
@@ -409,8 +464,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(DecodeParams 
       }
 #pragma unroll
       for (int rb = 0; rb < 8; ++rb) {
-        const int d0 = 16 * gid + 2 * rb;  // rows gid / gid + 8 of row block rb
-        // remove the operand offset: O = (acc - mu_p sum B) / sigma_p
+        const int d0 = 16 * gid + 2 * rb;
         const int p0 = slot_pos(2 * rb), p1 = slot_pos(2 * rb + 1);
         const float mu0 = 0.5f * (pos_v0_b(p0) + pos_v1_b(p0)), is0 = 2.f / (pos_v1_b(p0) - pos_v0_b(p0));
         const float mu1 = 0.5f * (pos_v0_b(p1) + pos_v1_b(p1)), is1 = 2.f / (pos_v1_b(p1) - pos_v0_b(p1));
