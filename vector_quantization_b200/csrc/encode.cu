@@ -12,9 +12,9 @@
 // vector: lane l holds coordinates l + 32 j (j < D/32), so the fast
 // Walsh-Hadamard transform needs 5 shuffle stages plus log2(D/32) in-register
 // stages, and a warp ballot over one register yields one 32-bit word of a
-// bit-plane directly.  Each warp takes a run of consecutive rows, so RoPE
-// advances its cos/sin by one position with an angle-addition step and reads
-// the two-level tables only where positions jump.  The QJL projection S r of
+// bit-plane directly.  A warp works on two vectors at a time as independent
+// chains; RoPE takes cos/sin of each row's position from the two-level tables
+// (angle addition of a coarse and a fine angle).  The QJL projection S r of
 // the whole tile is a dense product and runs on the 5th-generation tensor
 // core (tcgen05, M = 128 rows; rows past R stay zero): r is written as bf16
 // hi/lo pieces into a 128-byte swizzled shared-memory operand, S (bf16-exact,
@@ -61,6 +61,7 @@ __device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
 constexpr int kTileVec = 128;
 constexpr int kEncThreads = 256;
+constexpr int kEncWarps = kEncThreads / 32;
 constexpr int kWaitLimit = 1 << 22;
 
 template <int D, int BITS, typename T>
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
   constexpr int OPB = kTileVec * D * 2;           // bytes of one bf16 [128 x D] operand
   constexpr int SB = D * D * 2;                   // bytes of S [m x d] bf16
   const int R = p.rows;                           // vectors per tile
-  const int RUN = R / (kEncThreads / 32);         // vectors per warp per tile (contiguous run)
+  const int RUN = R >= kEncWarps ? R / kEncWarps : 1;   // vectors per warp per tile (contiguous run)
   extern __shared__ uint8_t raw[];
   __shared__ uint64_t mbar;
   __shared__ uint32_t tmem_slot;
@@ -102,130 +103,153 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
   float dsg[NJ];
 #pragma unroll
   for (int j = 0; j < NJ; ++j) dsg[j] = p.dsigns[lane + 32 * j];
-  // rotation by one position of the frequencies this lane owns (i = lane + 32 j, j < NJ/2)
-  float2 step[NJ / 2 > 0 ? NJ / 2 : 1];
-  if (p.rope) {
+  float thr[NT];
 #pragma unroll
-    for (int j = 0; j < NJ / 2; ++j) step[j] = p.rope_lo[(D / 2) + lane + 32 * j];
-  }
+  for (int t = 0; t < NT; ++t) thr[t] = thr_s[t];
   uint32_t phase = 0;
   const int64_t n_tiles = (p.n + R - 1) / R;
 
   for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
     const int64_t row0 = tile * R;
+    bool ok = true;
     // ---------------- per-vector work: warp owns a run of RUN vectors ---------
-    float2 cs[NJ / 2 > 0 ? NJ / 2 : 1];
-    int64_t prev_pos = -2;
-    for (int q = 0; q < RUN; ++q) {
-      const int v = warp * RUN + q;
-      const int64_t row = row0 + v;
-      float r[NJ];
-      bool valid = row < p.n;
-      if (valid) {
-        const T* xr = static_cast<const T*>(p.x) + row * p.ld;
-        float x[NJ];
+    // Two vectors per step as independent chains, so their shuffle and
+    // load latencies overlap.  The Walsh-Hadamard transform runs on the
+    // unnormalised vector (it is linear), so the norm reduction overlaps it.
+    int64_t pos_base = 0;   // position of the run's first row when pos == NULL
+    if (p.rope && !p.pos) {
+      const int64_t r0w = row0 + static_cast<int64_t>(warp) * RUN;
+      pos_base = r0w < p.n ? r0w % p.pos_period : 0;
+    }
+    for (int q0 = 0; q0 < RUN; q0 += 2) {
+      float x[2][NJ];
+      bool valid[2], pos_ok[2];
+      int64_t row[2];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) x[j] = load_elem<T>(xr + lane + 32 * j);
-        const int64_t rec = row * p.out_stride;
-        if (p.rope) {
-          const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
-          if (pos < 0 || pos >= p.rope_max_pos) {
-            if (lane == 0) p.norms[rec] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-            valid = false;
+      for (int c = 0; c < 2; ++c) {
+        const int q = q0 + c;
+        const int vl = warp * RUN + q;
+        row[c] = row0 + vl;
+        valid[c] = q < RUN && vl < R && row[c] < p.n;
+        pos_ok[c] = true;
+        const T* xr = static_cast<const T*>(p.x) + (valid[c] ? row[c] : 0) * p.ld;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) x[c][j] = load_elem<T>(xr + lane + 32 * j);
+      }
+      if (p.rope) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          int64_t pos;
+          if (p.pos) {
+            pos = valid[c] ? p.pos[row[c]] : 0;
           } else {
-            if (pos != prev_pos + 1) {
-              // seed cos/sin(pos theta_i) from the two-level tables (angle addition)
-              const float2* hi = p.rope_hi + (pos >> kRopeLoBits) * (D / 2);
-              const float2* lo = p.rope_lo + (pos & (kRopeLoRows - 1)) * (D / 2);
+            int64_t m = pos_base + q0 + c;
+            if (m >= p.pos_period) m %= p.pos_period;
+            pos = p.pos_offset + m;
+          }
+          pos_ok[c] = pos >= 0 && pos < p.rope_max_pos;
+          const int64_t pc = pos_ok[c] ? pos : 0;
+          // cos/sin(pos theta_i) from the two-level tables (angle addition)
+          const float2* hi = p.rope_hi + (pc >> kRopeLoBits) * (D / 2);
+          const float2* lo = p.rope_lo + (pc & (kRopeLoRows - 1)) * (D / 2);
 #pragma unroll
-              for (int j = 0; j < NJ / 2; ++j) {
-                const float2 a = hi[lane + 32 * j], b = lo[lane + 32 * j];
-                cs[j] = make_float2(a.x * b.x - a.y * b.y, a.y * b.x + a.x * b.y);
-              }
-            } else {
-              // advance one position: (c, s) <- rotation by theta_i
-#pragma unroll
-              for (int j = 0; j < NJ / 2; ++j)
-                cs[j] = make_float2(cs[j].x * step[j].x - cs[j].y * step[j].y, cs[j].y * step[j].x + cs[j].x * step[j].y);
-            }
-            prev_pos = pos;
-#pragma unroll
-            for (int j = 0; j < NJ / 2; ++j) {
-              const float x1 = x[j], x2 = x[j + NJ / 2];
-              x[j] = x1 * cs[j].x - x2 * cs[j].y;
-              x[j + NJ / 2] = x2 * cs[j].x + x1 * cs[j].y;
-            }
+          for (int j = 0; j < NJ / 2; ++j) {
+            const float2 a = hi[lane + 32 * j], b = lo[lane + 32 * j];
+            const float cs = a.x * b.x - a.y * b.y, sn = a.y * b.x + a.x * b.y;
+            const float x1 = x[c][j], x2 = x[c][j + NJ / 2];
+            x[c][j] = x1 * cs - x2 * sn;
+            x[c][j + NJ / 2] = x2 * cs + x1 * sn;
           }
         }
-        if (valid) {
-          float ss = 0.f;
+      }
+      // u = H D x (unnormalised, Sylvester order); lane l holds u[l + 32 j]
+      float u[2][NJ], ss[2];
 #pragma unroll
-          for (int j = 0; j < NJ; ++j) ss = fmaf(x[j], x[j], ss);
+      for (int c = 0; c < 2; ++c) {
+        ss[c] = 0.f;
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          const float norm = sqrtf(ss);
-          const float inv = norm > 0.f ? 1.0f / norm : 0.f;
-          // y = H (D x / ||x||) / sqrt(d), Sylvester order; lane l holds y[l + 32 j]
-          float u[NJ];
+        for (int j = 0; j < NJ; ++j) {
+          ss[c] = fmaf(x[c][j], x[c][j], ss[c]);
+          u[c][j] = x[c][j] * dsg[j];
+        }
+      }
 #pragma unroll
-          for (int j = 0; j < NJ; ++j) u[j] = x[j] * inv * dsg[j];
+      for (int st = 0; st < 5; ++st) {
+        const bool upper = (lane >> st) & 1;
 #pragma unroll
-          for (int s = 0; s < 5; ++s) {
-            const bool upper = (lane >> s) & 1;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-              const float o = __shfl_xor_sync(0xffffffffu, u[j], 1 << s);
-              u[j] = upper ? o - u[j] : u[j] + o;
-            }
-          }
-#pragma unroll
-          for (int b = 1; b < NJ; b <<= 1) {
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-              if (j & b) continue;
-              const float a0 = u[j], a1 = u[j | b];
-              u[j] = a0 + a1;
-              u[j | b] = a0 - a1;
-            }
-          }
-          int idx[NJ];
-          float rr = 0.f;
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
           for (int j = 0; j < NJ; ++j) {
-            const float y = u[j] * inv_sqrt_d;
-            int c = 0;
-#pragma unroll
-            for (int t = 0; t < NT; ++t) c += (y >= thr_s[t]) ? 1 : 0;
-            idx[j] = c;
-            r[j] = norm * (y - lev_s[c]);
-            rr = fmaf(r[j], r[j], rr);
+            const float o = __shfl_xor_sync(0xffffffffu, u[c][j], 1 << st);
+            u[c][j] = upper ? o - u[c][j] : u[c][j] + o;
           }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
-          uint32_t* crec = p.codes + rec * (BITS * NJ);
-#pragma unroll
-          for (int k = 0; k < BITS; ++k) {
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-              const uint32_t w = __ballot_sync(0xffffffffu, (idx[j] >> k) & 1);
-              if (lane == k * NJ + j) crec[k * NJ + j] = w;
-            }
-          }
-          if (lane == 0) p.norms[rec] = make_float2(norm, sqrtf(rr));
+          ss[c] += __shfl_xor_sync(0xffffffffu, ss[c], 16 >> st);
         }
       }
-      if (!valid) {
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) r[j] = 0.f;
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int bb = 1; bb < NJ; bb <<= 1)
+#pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            if (j & bb) continue;
+            const float a0 = u[c][j], a1 = u[c][j | bb];
+            u[c][j] = a0 + a1;
+            u[c][j | bb] = a0 - a1;
+          }
+      float r[2][NJ], rr[2], nrm[2];
+      int idx[2][NJ];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        nrm[c] = sqrtf(ss[c]);
+        const float scale = (nrm[c] > 0.f ? 1.0f / nrm[c] : 0.f) * inv_sqrt_d;
+        const bool keep = valid[c] && pos_ok[c];
+        rr[c] = 0.f;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const float y = u[c][j] * scale;   // coordinate of the unit vector
+          int ci = 0;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) ci += (y >= thr[t]) ? 1 : 0;
+          idx[c][j] = ci;
+          r[c][j] = keep ? nrm[c] * (y - lev_s[ci]) : 0.f;
+          rr[c] = fmaf(r[c][j], r[c][j], rr[c]);
+        }
       }
-      // residual as two bf16 pieces, row v of the A operand of S r
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const __nv_bfloat16 h = __float2bfloat16_rn(r[j]);
-        const __nv_bfloat16 l = __float2bfloat16_rn(r[j] - __bfloat162float(h));
-        const uint32_t off = tqtc::sw128_offset(v, lane + 32 * j, kTileVec);
-        *reinterpret_cast<__nv_bfloat16*>(r_hi + off) = h;
-        *reinterpret_cast<__nv_bfloat16*>(r_lo + off) = l;
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) rr[c] += __shfl_xor_sync(0xffffffffu, rr[c], o);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (q0 + c >= RUN || warp * RUN + q0 + c >= R) break;
+        if (valid[c]) {
+          const int64_t rec = row[c] * p.out_stride;
+          if (pos_ok[c]) {
+            uint32_t* crec = p.codes + rec * (BITS * NJ);
+#pragma unroll
+            for (int k = 0; k < BITS; ++k) {
+#pragma unroll
+              for (int j = 0; j < NJ; ++j) {
+                const uint32_t w = __ballot_sync(0xffffffffu, (idx[c][j] >> k) & 1);
+                if (lane == k * NJ + j) crec[k * NJ + j] = w;
+              }
+            }
+            if (lane == 0) p.norms[rec] = make_float2(nrm[c], sqrtf(rr[c]));
+          } else if (lane == 0) {
+            p.norms[rec] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+          }
+        }
+        // residual as two bf16 pieces, row v of the A operand of S r
+        const int v = warp * RUN + q0 + c;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(r[c][j]);
+          const __nv_bfloat16 l = __float2bfloat16_rn(r[c][j] - __bfloat162float(h));
+          const uint32_t off = tqtc::sw128_offset(v, lane + 32 * j, kTileVec);
+          *reinterpret_cast<__nv_bfloat16*>(r_hi + off) = h;
+          *reinterpret_cast<__nv_bfloat16*>(r_lo + off) = l;
+        }
       }
     }
     // ---------------- S r on the tensor core: D[v][j] = sum_k R[v][k] S[j][k] --
@@ -244,7 +268,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
                           tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, true);
       tqtc::mma_commit(&mbar);
     }
-    const bool ok = tqtc::mbar_wait(&mbar, phase, kWaitLimit);
+    ok = tqtc::mbar_wait(&mbar, phase, kWaitLimit) && ok;
     phase ^= 1;
     tqtc::fence_after_sync();
     // ---------------- sign bits: warp w reads lanes 32 (w % 4).., half the columns
@@ -286,6 +310,7 @@ int launch_encode(const EncodeParams& p, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // smallest tile (>= 8 rows, one per warp) that still gives each CTA slot work
   // smallest tile (>= 8 rows, one per warp) that still gives each CTA slot work
   int rows = 8;
   while (rows < kTileVec && (p.n + rows - 1) / rows > 2LL * sms) rows *= 2;
