@@ -66,6 +66,20 @@ def test_encode_parity(cuda_device, d, bits, dtype):
     _run_encode(d, bits, 1031, dtype, rope=True, seed=100 + bits)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_encode_parity_large_batch(cuda_device, d, bits, dtype):
+    """Batches of 16384 or more vectors take the thread-per-vector kernel:
+    several 128-row tiles per CTA group and a ragged last tile."""
+    _run_encode(d, bits, 16384 + 1031, dtype, rope=True, seed=200 + bits)
+
+
+def test_encode_large_batch_positions_array_strided(cuda_device):
+    _run_encode(128, 2, 16384 + 77, torch.bfloat16, rope=True, seed=210, period=5000, offset=3,
+                pos_array=True, out_stride=2)
+
+
 @pytest.mark.parametrize("n", [1, 7, 33, 4099])
 def test_encode_ragged_counts_no_rope(cuda_device, n):
     _run_encode(128, 2, n, torch.float32, rope=False, seed=7)

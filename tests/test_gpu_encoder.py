@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import synth
-from helpers import assert_close, oracle_records, oracle_rotation
+from helpers import assert_close, compare_records, oracle_records, oracle_rotation
 from oracle import attention as at
 
 pytestmark = pytest.mark.gpu
@@ -107,6 +107,16 @@ def test_esm2_layer_full_size_sampled(cuda_device):
         gpu_same = tq.encoder_attention(rk, rv, q[b:b + 1, h:h + 1].contiguous(), to(ko), to(vo), T)
         torch.cuda.synchronize()
         assert_close(gpu_same[0, 0].cpu().numpy(), ref, what=f"head ({b},{h}) oracle-packed")
-        # full-size launch output (GPU-packed cache): codes may differ only at
-        # boundary-flagged coordinates, which moves outputs far less than the tolerance
-        assert_close(out[b, h].cpu().numpy(), ref, what=f"head ({b},{h}) full launch")
+        # full-size launch: the GPU records of this head equal the oracle's
+        # encoding except at boundary-flagged coordinates (a flipped code is
+        # a legitimate outcome there, and with x15 outlier channels it moves a
+        # logit by more than the output tolerance), and the launch's output
+        # equals the oracle's attention over those same GPU records
+        gk = tuple(a[b:b + 1, h:h + 1].cpu().numpy() for a in kc)
+        gv = tuple(a[b:b + 1, h:h + 1].cpu().numpy() for a in vc)
+        _, _, _, enc_k = oracle_records(rk_o, kk.reshape(-1, d), np.arange(T))
+        _, _, _, enc_v = oracle_records(rv_o, vv.reshape(-1, d))
+        compare_records(rk_o, tuple(x.reshape(T, -1) for x in gk), enc_k)
+        compare_records(rv_o, tuple(x.reshape(T, -1) for x in gv), enc_v)
+        ref_gpu = at.encoder_attention(rk_o, rv_o, qq, gk, gv, 1 / np.sqrt(d))[0, 0]
+        assert_close(out[b, h].cpu().numpy(), ref_gpu, what=f"head ({b},{h}) full launch")

@@ -7,20 +7,9 @@
 // "QJL" (one sign bit per Johnson-Lindenstrauss projection of the residual);
 // [NSNQuant] §2 (randomized Hadamard transform, H D / sqrt(d)).
 //
-// A CTA encodes tiles of R vectors (R = 8..128, chosen per call so that
-// small batches still spread over many SMs).  Per-vector work runs one warp per
-// vector: lane l holds coordinates l + 32 j (j < D/32), so the fast
-// Walsh-Hadamard transform needs 5 shuffle stages plus log2(D/32) in-register
-// stages, and a warp ballot over one register yields one 32-bit word of a
-// bit-plane directly.  A warp works on two vectors at a time as independent
-// chains; RoPE takes cos/sin of each row's position from the two-level tables
-// (angle addition of a coarse and a fine angle).  The QJL projection S r of
-// the whole tile is a dense product and runs on the 5th-generation tensor
-// core (tcgen05, M = 128 rows; rows past R stay zero): r is written as bf16
-// hi/lo pieces into a 128-byte swizzled shared-memory operand, S (bf16-exact,
-// stored by the handle already in operand layout) stays resident in shared
-// memory, the fp32 result lands in tensor memory and each thread reads back
-// its vector's row to form the sign bits.
+// The kernel (encode_rows_kernel, below) gives each thread one whole vector
+// in registers; the QJL projection S r of each 128-vector tile is a dense
+// product and runs on the 5th-generation tensor core (tcgen05).
 #include <cuda_bf16.h>
 
 #include "bitplane.cuh"
@@ -41,13 +30,32 @@ struct EncodeParams {
   int64_t out_stride;
   const float* dsigns;  // [D]
   const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
-  int rows;             // vectors per tile, R in {8, 16, 32, 64, 128}
+  int rows;             // warp-per-vector kernel: vectors per tile, R in {8, 16, ..., 128}
   const float* thresholds;
   const float* levels;
   const float2* rope_hi;
   const float2* rope_lo;
   int64_t rope_max_pos;
+  // thread-per-vector kernel: sign diagonal and the positive half of the
+  // (symmetric) codebook, read straight from the parameter space
+  float dsg[128];
+  float tpos[4];        // thresholds above 0, ascending (2^(b-1) - 1 of them)
+  float lpos[4];        // levels above 0, ascending (2^(b-1) of them)
 };
+
+// Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
+constexpr int kTileVec = 128;
+constexpr int kWaitLimit = 1 << 22;
+
+// ===========================================================================
+// Warp-per-vector encode, for small batches (a decode step's new keys and
+// values): lane l of a warp holds coordinates l + 32 j, the Walsh-Hadamard
+// transform takes 5 shuffle stages plus log2(d/32) in-register stages, and a
+// ballot over one register yields a bit-plane word.  Its per-vector latency
+// is far below the thread-per-vector kernel's, which wins on throughput.
+// ===========================================================================
+constexpr int kEncThreads = 256;
+constexpr int kEncWarps = kEncThreads / 32;
 
 template <typename T>
 __device__ __forceinline__ float load_elem(const T* p);
@@ -59,10 +67,6 @@ __device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p
 }
 
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
-constexpr int kTileVec = 128;
-constexpr int kEncThreads = 256;
-constexpr int kEncWarps = kEncThreads / 32;
-constexpr int kWaitLimit = 1 << 22;
 
 template <int D, int BITS, typename T>
 __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodeParams p) {
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
 }
 
 template <int D, int BITS, typename T>
-int launch_encode(const EncodeParams& p, cudaStream_t stream) {
+int launch_encode_warp(const EncodeParams& p, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(D) * D * 2 + 2 * static_cast<size_t>(kTileVec) * D * 2 + 1024;
   auto kern = encode_hadamard_kernel<D, BITS, T>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
@@ -320,6 +324,336 @@ int launch_encode(const EncodeParams& p, cudaStream_t stream) {
   const int blocks = static_cast<int>(tiles < sms * 2LL ? tiles : sms * 2LL);
   kern<<<blocks, kEncThreads, smem, stream>>>(q);
   return tq::launch_status();
+}
+
+// ===========================================================================
+// Thread-per-vector encode.  Each thread holds one whole vector in registers,
+// so RoPE, the norm, the Walsh-Hadamard transform (log2 d in-register
+// butterfly stages) and the quantizer need no cross-lane traffic, and each
+// bit-plane word is assembled in the thread.  A CTA is two groups of four
+// warps; a group owns one 128-row tile (thread t = row t = tensor-memory lane
+// t), its own residual operand and accumulator, and synchronises with a named
+// barrier, so one group's tensor-core product and read-back overlap the other
+// group's per-vector work.  S (shared by both groups) is resident in shared
+// memory in operand layout.
+// ===========================================================================
+constexpr int kRowThreads = 256;    // two groups
+constexpr int kGroupThreads = 128;  // one tile row per thread
+
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(1 + g), "r"(kGroupThreads) : "memory");
+}
+
+// Row of D elements (16-byte aligned) into fp32 registers.
+template <int D, typename T>
+__device__ __forceinline__ void load_row(const T* xr, float (&u)[D]) {
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr) + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        u[8 * c + 2 * q] = __uint_as_float(w[q] << 16);
+        u[8 * c + 2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(xr) + c);
+      u[4 * c] = v.x;
+      u[4 * c + 1] = v.y;
+      u[4 * c + 2] = v.z;
+      u[4 * c + 3] = v.w;
+    }
+  }
+}
+
+// Unnormalised Sylvester-order Walsh-Hadamard transform in registers.
+template <int D>
+__device__ __forceinline__ void fwht_regs(float (&u)[D]) {
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < D; ++i)
+      if (!(i & h)) {
+        const float a = u[i], b = u[i | h];
+        u[i] = a + b;
+        u[i | h] = a - b;
+      }
+}
+
+// Codes of 32 coordinates y[i] (unit-vector coordinates, never -0), as BITS
+// plane words, and their residuals norm * (y - level) written over y.  The
+// codebook is symmetric: the sign picks the half and |y| against the positive
+// thresholds t_k picks the level m within it, idx = pos ? 2^(b-1) + m :
+// 2^(b-1) - 1 - m.  Every plane bit is then an XNOR of sign bits: s_y (y < 0)
+// and s_k (|y| - t_k < 0, exact in fp32): bit b-1 = !s_y, bit b-2 = s_y == s_1
+// (b = 2: s_0), bit 0 (b = 3) = s_y == s_0 ^ s_1 ^ s_2.  Bits are shifted in
+// with one funnel shift each and the words complemented at the end.
+// nl[k] = norm * lpos[k].  Returns the sum of squared residuals.
+template <int BITS>
+__device__ __forceinline__ float quantize32(float* y, const float (&tp)[4], const float (&nl)[4], float norm,
+                                            uint32_t (&w)[BITS]) {
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) w[k] = 0;
+  float rr = 0.f;
+#pragma unroll
+  for (int i = 31; i >= 0; --i) {
+    const float v = y[i];
+    const uint32_t sy = __float_as_uint(v);
+    const float a = fabsf(v);
+    float nmag;
+    if constexpr (BITS == 1) {
+      w[0] = __funnelshift_l(sy, w[0], 1);
+      nmag = nl[0];
+    } else if constexpr (BITS == 2) {
+      const uint32_t s0 = __float_as_uint(a - tp[0]);
+      w[1] = __funnelshift_l(sy, w[1], 1);
+      w[0] = __funnelshift_l(sy ^ s0, w[0], 1);
+      nmag = a >= tp[0] ? nl[1] : nl[0];
+    } else {
+      const uint32_t s0 = __float_as_uint(a - tp[0]), s1 = __float_as_uint(a - tp[1]),
+                     s2 = __float_as_uint(a - tp[2]);
+      w[2] = __funnelshift_l(sy, w[2], 1);
+      w[1] = __funnelshift_l(sy ^ s1, w[1], 1);
+      w[0] = __funnelshift_l(sy ^ s0 ^ s1 ^ s2, w[0], 1);
+      nmag = a >= tp[2] ? nl[3] : (a >= tp[1] ? nl[2] : (a >= tp[0] ? nl[1] : nl[0]));
+    }
+    const float r = fmaf(norm, v, -copysignf(nmag, v));
+    y[i] = r;
+    rr = fmaf(r, r, rr);
+  }
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) w[k] = ~w[k];
+  return rr;
+}
+template <int D, int BITS, typename T>
+__global__ void __launch_bounds__(kRowThreads, 1) encode_rows_kernel(EncodeParams p) {
+  constexpr int NJ = D / 32;
+  constexpr int OPB = kTileVec * D * 2;           // bytes of one bf16 [128 x D] operand
+  constexpr int SB = D * D * 2;                   // bytes of S [m x d] bf16
+  extern __shared__ uint8_t raw[];
+  __shared__ uint64_t mbar[2];
+  __shared__ uint32_t tmem_slot;
+  uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
+  uint8_t* s_op = base;                           // S, K-major SW128 (rows = sketch index)
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int g = tid >> 7, t = tid & (kGroupThreads - 1);   // group, row in the tile
+  uint8_t* r_hi = base + SB + g * 2 * OPB;       // this group's residual tile, hi bf16 piece
+  uint8_t* r_lo = r_hi + OPB;                     // lo bf16 piece
+  // bf16 inputs: each thread prefetches its row of the group's next tile
+  // into shared memory (16-byte cp.async, chunk c stored at c ^ (t & 15) so
+  // the row reads spread over the banks)
+  constexpr bool kStage = sizeof(T) == 2;
+  constexpr int RB = D * static_cast<int>(sizeof(T));   // bytes per row
+  uint8_t* xstage = base + SB + 4 * OPB + g * kTileVec * RB + t * RB;
+  auto prefetch_row = [&](int64_t tile) {
+    if constexpr (kStage) {
+      const int64_t r = tile * kTileVec + t;
+      if (tile < (p.n + kTileVec - 1) / kTileVec && r < p.n) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(static_cast<const T*>(p.x) + r * p.ld);
+#pragma unroll
+        for (int c = 0; c < RB / 16; ++c) tqdev::cp_async16(xstage + 16 * (c ^ (t & (RB / 16 - 1))), src + 16 * c, 16);
+      }
+      tqdev::cp_async_commit();
+    }
+  };
+
+  for (int c = tid; c < SB / 16; c += blockDim.x) tqdev::cp_async16(s_op + 16 * c, p.s_op + 8 * c, 16);
+  tqdev::cp_async_commit();
+  if (tid < 2) tqtc::mbar_init(&mbar[tid], 1);
+  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, 2 * D);
+  tqdev::cp_async_wait<0>();
+  tqtc::fence_before_sync();
+  __syncthreads();
+  tqtc::fence_after_sync();
+  const uint32_t tmem = tmem_slot + g * D + (static_cast<uint32_t>(t & ~31) << 16);   // lane block of this warp
+  const uint32_t idesc = tqtc::idesc_bf16_f32(kTileVec, D);
+  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  float tp[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tp[k] = p.tpos[k];
+  const int64_t n_tiles = (p.n + kTileVec - 1) / kTileVec;
+  // swizzled row base of this thread's row in the residual operands
+  const uint32_t rowbase = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
+  const uint32_t vx = t & 7;
+  uint32_t phase = 0;
+
+  prefetch_row(2 * static_cast<int64_t>(blockIdx.x) + g);
+  for (int64_t tile = 2 * static_cast<int64_t>(blockIdx.x) + g; tile < n_tiles; tile += 2 * gridDim.x) {
+    const int64_t row = tile * kTileVec + t;
+    bool valid = row < p.n;
+    float u[D];
+    float nrm = 0.f, rr = 0.f;
+    if constexpr (kStage) {
+      // this thread's row (its own cp.async group), then the next tile's row
+      tqdev::cp_async_wait<0>();
+      if (valid) {
+#pragma unroll
+        for (int c = 0; c < RB / 16; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xstage + 16 * (c ^ (t & (RB / 16 - 1))));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            u[8 * c + 2 * q] = __uint_as_float(w[q] << 16);
+            u[8 * c + 2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+          }
+        }
+      }
+      prefetch_row(tile + 2 * gridDim.x);
+    }
+    if (valid) {
+      if constexpr (!kStage) load_row<D, T>(static_cast<const T*>(p.x) + row * p.ld, u);
+      if (p.rope) {
+        const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
+        if (pos < 0 || pos >= p.rope_max_pos) {
+          valid = false;
+          p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+        } else {
+          // cos/sin(pos theta_i) from the two-level tables (angle addition)
+          const float4* hi = reinterpret_cast<const float4*>(p.rope_hi + (pos >> kRopeLoBits) * (D / 2));
+          const float4* lo = reinterpret_cast<const float4*>(p.rope_lo + (pos & (kRopeLoRows - 1)) * (D / 2));
+#pragma unroll
+          for (int c = 0; c < D / 4; ++c) {
+            if ((c & 7) == 0) asm volatile("" ::: "memory");   // bound the loads in flight (registers)
+            const float4 a = __ldg(hi + c), b = __ldg(lo + c);
+            const float c0 = a.x * b.x - a.y * b.y, s0 = a.y * b.x + a.x * b.y;
+            const float c1 = a.z * b.z - a.w * b.w, s1 = a.w * b.z + a.z * b.w;
+            const int i0 = 2 * c, i1 = 2 * c + 1;
+            const float x0 = u[i0], y0 = u[i0 + D / 2], x1 = u[i1], y1 = u[i1 + D / 2];
+            u[i0] = x0 * c0 - y0 * s0;
+            u[i0 + D / 2] = y0 * c0 + x0 * s0;
+            u[i1] = x1 * c1 - y1 * s1;
+            u[i1 + D / 2] = y1 * c1 + x1 * s1;
+          }
+        }
+      }
+    }
+    if (valid) {
+      float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < D; ++i) {
+        ss[i & 3] = fmaf(u[i], u[i], ss[i & 3]);
+        u[i] *= p.dsg[i];
+      }
+      nrm = sqrtf((ss[0] + ss[1]) + (ss[2] + ss[3]));
+      fwht_regs<D>(u);
+      const float scale = (nrm > 0.f ? 1.0f / nrm : 0.f) * inv_sqrt_d;
+#pragma unroll
+      for (int i = 0; i < D; ++i) u[i] = fmaf(u[i], scale, 0.f);   // unit-vector coordinates, -0 -> +0
+      float nl[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) nl[k] = nrm * p.lpos[k];
+      uint32_t words[BITS][NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        uint32_t w[BITS];
+        rr += quantize32<BITS>(u + 32 * j, tp, nl, nrm, w);
+#pragma unroll
+        for (int k = 0; k < BITS; ++k) words[k][j] = w[k];
+      }
+      uint32_t* crec = p.codes + row * p.out_stride * (BITS * NJ);   // 4-byte aligned records
+#pragma unroll
+      for (int k = 0; k < BITS; ++k)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) crec[k * NJ + j] = words[k][j];
+      p.norms[row * p.out_stride] = make_float2(nrm, sqrtf(rr));
+    } else {
+#pragma unroll
+      for (int i = 0; i < D; ++i) u[i] = 0.f;
+    }
+    // residual as bf16 hi + lo, row t of this group's A operand (16-byte chunks)
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      uint32_t h[4], l[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = u[8 * c + 2 * q], b = u[8 * c + 2 * q + 1];
+        __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
+        const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb);
+        __nv_bfloat162 lb =
+            __floats2bfloat162_rn(a - __uint_as_float(hbits << 16), b - __uint_as_float(hbits & 0xFFFF0000u));
+        h[q] = hbits;
+        l[q] = *reinterpret_cast<uint32_t*>(&lb);
+      }
+      const uint32_t off = (c >> 3) * (kTileVec * 128) + rowbase + ((((c & 7) ^ vx)) << 4);
+      *reinterpret_cast<uint4*>(r_hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+      *reinterpret_cast<uint4*>(r_lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+    // ---- S r of the tile on the tensor core (one thread of the group issues)
+    tqtc::fence_smem_to_async();
+    tqtc::fence_before_sync();
+    group_sync(g);
+    if (t == 0) {
+      tqtc::fence_after_sync();
+      const uint32_t dacc = tmem_slot + g * D;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(tqtc::smem_u32(r_hi), ks, kTileVec),
+                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(tqtc::smem_u32(r_lo), ks, kTileVec),
+                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, true);
+      tqtc::mma_commit(&mbar[g]);
+    }
+    const bool ok = tqtc::mbar_wait(&mbar[g], phase, kWaitLimit);
+    phase ^= 1;
+    tqtc::fence_after_sync();
+    // ---- sign bits of row t: lane t of the accumulator
+    uint32_t sw[NJ];
+#pragma unroll
+    for (int c = 0; c < NJ; ++c) {
+      float val[32];
+      tqtc::tmem_ld32(tmem + 32 * c, val);
+      uint32_t w = 0;
+#pragma unroll
+      for (int b = 31; b >= 0; --b) w = (w << 1) | (val[b] >= 0.f ? 1u : 0u);
+      sw[c] = ok ? w : 0u;
+    }
+    if (row < p.n) {
+      uint32_t* srec = p.signs + row * p.out_stride * NJ;
+#pragma unroll
+      for (int c = 0; c < NJ; ++c) srec[c] = sw[c];
+      if (!ok) p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    }
+    tqtc::fence_before_sync();
+    group_sync(g);
+  }
+  tqtc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tqtc::tmem_free(tmem_slot, 2 * D);
+}
+
+template <int D, int BITS, typename T>
+int launch_encode_rows(const EncodeParams& p, cudaStream_t stream) {
+  // S + two groups x (hi, lo) residual tiles + (bf16) two staged input tiles:
+  // 225 KB at d = 128
+  const size_t stage = sizeof(T) == 2 ? 2 * static_cast<size_t>(kTileVec) * D * sizeof(T) : 0;
+  const size_t smem = static_cast<size_t>(D) * D * 2 + 4 * static_cast<size_t>(kTileVec) * D * 2 + stage + 1024;
+  auto kern = encode_rows_kernel<D, BITS, T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return TQ_ECUDA;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = (p.n + kTileVec - 1) / kTileVec;
+  const int64_t pairs = (tiles + 1) / 2;
+  const int blocks = static_cast<int>(pairs < sms ? pairs : sms);
+  kern<<<blocks, kRowThreads, smem, stream>>>(p);
+  return tq::launch_status();
+}
+
+// Batches below this many vectors take the low-latency warp-per-vector kernel.
+constexpr int64_t kRowsKernelMinN = 16384;
+
+template <int D, int BITS, typename T>
+int launch_encode(const EncodeParams& p, cudaStream_t stream) {
+  if (p.n < kRowsKernelMinN) return launch_encode_warp<D, BITS, T>(p, stream);
+  return launch_encode_rows<D, BITS, T>(p, stream);
 }
 
 template <int D, typename T>
@@ -371,6 +705,14 @@ extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, in
   p.out_stride = out_stride;
   p.dsigns = h->d_signs;
   p.s_op = h->d_s_op;
+  {
+    const int half = 1 << (h->bits - 1);
+    for (int i = 0; i < h->d && i < 128; ++i) p.dsg[i] = h->signs[i];
+    for (int k = 0; k < 4; ++k) {
+      p.lpos[k] = k < half ? static_cast<float>(h->levels[half + k]) : 0.f;
+      p.tpos[k] = k < half - 1 ? static_cast<float>(h->thresholds[half + k]) : 0.f;
+    }
+  }
   p.thresholds = h->d_thresholds;
   p.levels = h->d_levels;
   p.rope_hi = h->d_rope_hi;

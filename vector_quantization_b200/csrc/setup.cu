@@ -326,6 +326,7 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
     std::vector<float> sg(d);
     for (int i = 0; i < d; ++i) sg[i] = static_cast<float>(signs[i]);
     if ((st = upload(&h->d_signs, sg.data(), sg.size())) != TQ_OK) { release(h); return st; }
+    h->signs = sg;
   } else {
     std::vector<double> pi;
     haar_from_gaussian(gauss_pi, d, &pi);

@@ -19,6 +19,7 @@ struct tq_rotation {
 
   std::vector<double> levels;           // [2^bits] ascending
   std::vector<double> thresholds;       // [2^bits - 1]
+  std::vector<float> signs;             // [d] +-1 (Hadamard kind)
   // Walsh form of the codebook: level(idx) = sum_p walsh[p] * s_p(idx),
   // s_p the +-1 value of the p-th plane product (see plane_products()).
   double walsh[4] = {0, 0, 0, 0};
