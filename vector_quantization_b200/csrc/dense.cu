@@ -5,14 +5,19 @@
 // quantizer per coordinate with the vector norm kept; Étape 2 / "QJL": sign
 // bits of the Johnson-Lindenstrauss projection of the residual plus ||r||.
 // With a dense rotation both y = Pi x and S r are genuine dense
-// contractions, run here as fp32 GEMMs over a chunk of vectors:
-//   1. Y = X Pi^T          (sgemm_nt, fp32 FFMA, 128x128 tiles)
-//   2. per row: ||x||, y = Y / ||x||, codes (bit-planes by warp ballot),
-//      R = ||x|| (y - c[idx]) written over Y, ||r||
-//   3. P = R S^T           (sgemm_nt)
-//   4. per row: sign bits of P by warp ballot
-// fp32 keeps the rotated unit coordinates within ~1e-8 of the exact values,
-// far inside the 1e-5 boundary band that decides code parity.
+// contractions; they run on the tensor core (tc_gemm.cu) over a chunk of
+// vectors, with fp32 operands split into bf16 hi + lo pieces:
+//   1. X -> X_hi, X_lo (bf16)
+//   2. Y = X Pi^T          (X_hi Pi_hi + X_hi Pi_lo + X_lo Pi_hi, fp32 accumulate)
+//   3. per row: ||x||, y = Y / ||x||, codes (bit-planes by warp ballot),
+//      r = ||x|| (y - c[idx]) written as bf16 hi + lo over X_hi, X_lo, ||r||
+//   4. P = R S^T           (R_hi S + R_lo S; S is bf16-exact)
+//   5. per row: sign bits of P by warp ballot
+// The split keeps each product within ~2^-16 relative, so rotated unit
+// coordinates stay ~1e-7 from the exact values (sum of d products of random
+// sign), far inside the 1e-5 boundary band that decides code parity.
+#include <cuda_bf16.h>
+
 #include <cmath>
 
 #include "tq_internal.h"
@@ -104,7 +109,9 @@ __global__ void __launch_bounds__(256) sgemm_nt_kernel(int M, int N, int K, cons
 // One warp per row: norms, codes (bit-planes), residual written over Y.
 template <int BITS>
 __global__ void __launch_bounds__(256) dense_quantize_rows_kernel(const float* __restrict__ x, int64_t ld, int64_t n,
-                                                                  int d, float* __restrict__ yr,
+                                                                  int d, const float* __restrict__ yr,
+                                                                  __nv_bfloat16* __restrict__ rh,
+                                                                  __nv_bfloat16* __restrict__ rl,
                                                                   const float* __restrict__ thresholds,
                                                                   const float* __restrict__ levels,
                                                                   uint32_t* __restrict__ codes, float2* __restrict__ norms) {
@@ -124,7 +131,7 @@ __global__ void __launch_bounds__(256) dense_quantize_rows_kernel(const float* _
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float norm = sqrtf(ss);
   const float inv = norm > 0.f ? 1.0f / norm : 0.f;
-  float* y = yr + row * d;
+  const float* y = yr + row * d;
   const int words = d / 32;
   uint32_t* crec = codes + row * (BITS * words);
   float rr = 0.f;
@@ -134,7 +141,9 @@ __global__ void __launch_bounds__(256) dense_quantize_rows_kernel(const float* _
 #pragma unroll
     for (int t = 0; t < NT; ++t) c += (yv >= thr[t]) ? 1 : 0;
     const float r = norm * (yv - lev[c]);
-    y[32 * w + lane] = r;
+    const __nv_bfloat16 h = __float2bfloat16_rn(r);
+    rh[row * d + 32 * w + lane] = h;
+    rl[row * d + 32 * w + lane] = __float2bfloat16_rn(r - __bfloat162float(h));
     rr = fmaf(r, r, rr);
 #pragma unroll
     for (int k = 0; k < BITS; ++k) {
@@ -173,8 +182,9 @@ int sgemm_nt(int M, int N, int K, const float* A, int64_t lda, const float* B, i
   return launch_status();
 }
 
-// Bytes of dense-encode scratch per vector of a chunk (Y/R and P rows).
-size_t dense_bytes_per_row(const tq_rotation* h) { return static_cast<size_t>(h->d + h->m) * sizeof(float); }
+// Bytes of dense-encode scratch per vector of a chunk: X (then R) as bf16
+// hi + lo, and Y (then P) as fp32 (m = d).
+size_t dense_bytes_per_row(const tq_rotation* h) { return static_cast<size_t>(h->d) * 4 + static_cast<size_t>(h->m) * 4; }
 
 }  // namespace tq
 
@@ -199,25 +209,32 @@ extern "C" int tq_quantize_dense(const tq_rotation* h, const float* x, int64_t n
   if (!tq::on_handle_device(h)) return TQ_EINVAL;
   const int d = h->d, m = h->m;
   const int64_t chunk = static_cast<int64_t>(workspace_bytes / per_row);
-  float* yr = static_cast<float*>(workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t cbytes = static_cast<int64_t>(h->bits) * d / 8, sbytes = m / 8;
   for (int64_t r0 = 0; r0 < n; r0 += chunk) {
     const int64_t rows = n - r0 < chunk ? n - r0 : chunk;
-    float* proj = yr + rows * d;
-    int st = tq::sgemm_nt(static_cast<int>(rows), d, d, x + r0 * ld, ld, h->d_pi, d, yr, d, s);
+    // scratch of the chunk: X (later R) as bf16 hi, lo; Y (later P) as fp32
+    uint16_t* xh = static_cast<uint16_t*>(workspace);
+    uint16_t* xl = xh + rows * d;
+    float* yr = reinterpret_cast<float*>(xl + rows * d);
+    int st = tq::split_bf16(x + r0 * ld, ld, rows, d, xh, xl, d, s);
     if (st != TQ_OK) return st;
+    if ((st = tq::tc_gemm_split(static_cast<int>(rows), d, d, xh, xl, d, h->d_pi_hi, h->d_pi_lo, d, yr, d, s)) != TQ_OK)
+      return st;
     const int blocks = static_cast<int>((rows + 7) / 8);
     uint32_t* cw = reinterpret_cast<uint32_t*>(codes + r0 * cbytes);
     float2* nw = reinterpret_cast<float2*>(norms) + r0;
+    __nv_bfloat16* rh = reinterpret_cast<__nv_bfloat16*>(xh);
+    __nv_bfloat16* rl = reinterpret_cast<__nv_bfloat16*>(xl);
     switch (h->bits) {
-      case 1: dense_quantize_rows_kernel<1><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, h->d_thresholds, h->d_levels, cw, nw); break;
-      case 2: dense_quantize_rows_kernel<2><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, h->d_thresholds, h->d_levels, cw, nw); break;
-      default: dense_quantize_rows_kernel<3><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, h->d_thresholds, h->d_levels, cw, nw); break;
+      case 1: dense_quantize_rows_kernel<1><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw); break;
+      case 2: dense_quantize_rows_kernel<2><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw); break;
+      default: dense_quantize_rows_kernel<3><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw); break;
     }
     if ((st = tq::launch_status()) != TQ_OK) return st;
-    if ((st = tq::sgemm_nt(static_cast<int>(rows), m, d, yr, d, h->d_s, d, proj, m, s)) != TQ_OK) return st;
-    dense_sign_rows_kernel<<<blocks, 256, 0, s>>>(proj, rows, m, reinterpret_cast<uint32_t*>(signs + r0 * sbytes));
+    if ((st = tq::tc_gemm_split(static_cast<int>(rows), m, d, xh, xl, d, h->d_s_bf16, nullptr, d, yr, m, s)) != TQ_OK)
+      return st;
+    dense_sign_rows_kernel<<<blocks, 256, 0, s>>>(yr, rows, m, reinterpret_cast<uint32_t*>(signs + r0 * sbytes));
     if ((st = tq::launch_status()) != TQ_OK) return st;
   }
   return TQ_OK;

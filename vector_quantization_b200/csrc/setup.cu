@@ -228,6 +228,9 @@ void release(tq_rotation* h) {
   cudaFree(h->d_s);
   cudaFree(h->d_st);
   cudaFree(h->d_s_op);
+  cudaFree(h->d_pi_hi);
+  cudaFree(h->d_pi_lo);
+  cudaFree(h->d_s_bf16);
   cudaFree(h->d_rope_hi);
   cudaFree(h->d_rope_lo);
   delete h;
@@ -332,6 +335,19 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
     haar_from_gaussian(gauss_pi, d, &pi);
     std::vector<float> pf(pi.begin(), pi.end());
     if ((st = upload(&h->d_pi, pf.data(), pf.size())) != TQ_OK) { release(h); return st; }
+    // bf16 hi + lo pieces of Pi (each rounded to nearest)
+    std::vector<uint16_t> ph(pf.size()), pl(pf.size());
+    for (size_t i = 0; i < pf.size(); ++i) {
+      const float hv = round_to_bf16(pf[i]);
+      const float lv = round_to_bf16(pf[i] - hv);
+      uint32_t hb, lb;
+      std::memcpy(&hb, &hv, 4);
+      std::memcpy(&lb, &lv, 4);
+      ph[i] = static_cast<uint16_t>(hb >> 16);
+      pl[i] = static_cast<uint16_t>(lb >> 16);
+    }
+    if ((st = upload(&h->d_pi_hi, ph.data(), ph.size())) != TQ_OK) { release(h); return st; }
+    if ((st = upload(&h->d_pi_lo, pl.data(), pl.size())) != TQ_OK) { release(h); return st; }
   }
   {
     std::vector<float> s(static_cast<size_t>(m) * d), stt(static_cast<size_t>(d) * m);
@@ -343,6 +359,15 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
       }
     if ((st = upload(&h->d_s, s.data(), s.size())) != TQ_OK) { release(h); return st; }
     if ((st = upload(&h->d_st, stt.data(), stt.size())) != TQ_OK) { release(h); return st; }
+    if (kind == TQ_ROT_DENSE) {
+      std::vector<uint16_t> sb(s.size());
+      for (size_t i = 0; i < s.size(); ++i) {
+        uint32_t bits;
+        std::memcpy(&bits, &s[i], 4);
+        sb[i] = static_cast<uint16_t>(bits >> 16);   // S is bf16-exact
+      }
+      if ((st = upload(&h->d_s_bf16, sb.data(), sb.size())) != TQ_OK) { release(h); return st; }
+    }
     if (kind == TQ_ROT_HADAMARD) {
       // K-major bf16 operand with a 128-byte swizzle: K/64 blocks of m rows x
       // 64 elements; row r of a block at (r/8)*1024 + (r%8)*128 bytes, its

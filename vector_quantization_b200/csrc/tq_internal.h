@@ -35,6 +35,11 @@ struct tq_rotation {
   // S as bf16 in the tensor-core operand layout (K-major, 128-byte swizzle,
   // rows = sketch index, K = coordinate); Hadamard kind only.
   uint16_t* d_s_op = nullptr;
+  // Dense kind: Pi as bf16 hi + lo pieces and S as bf16, row-major, for the
+  // split tensor-core contractions.
+  uint16_t* d_pi_hi = nullptr;
+  uint16_t* d_pi_lo = nullptr;
+  uint16_t* d_s_bf16 = nullptr;
   float2* d_rope_hi = nullptr;          // [rope_hi_rows][d/2] (cos, sin) of h*1024*theta_i
   float2* d_rope_lo = nullptr;          // [1024][d/2]           (cos, sin) of l*theta_i
 };
@@ -60,5 +65,13 @@ inline int launch_status() {
 inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
+
+// fp32 -> bf16 hi + lo pieces of a row-major matrix (cols % 4 == 0).
+int split_bf16(const float* x, int64_t ldx, int64_t rows, int cols, uint16_t* hi, uint16_t* lo, int64_t ldo,
+               cudaStream_t s);
+// C[M][N] = A[M][K] B[N][K]^T from bf16 pieces on the tensor core
+// (A_hi B_hi + A_hi B_lo + A_lo B_hi; bl == nullptr drops the B_lo term).
+int tc_gemm_split(int M, int N, int K, const uint16_t* ah, const uint16_t* al, int64_t lda, const uint16_t* bh,
+                  const uint16_t* bl, int64_t ldb, float* C, int64_t ldc, cudaStream_t s);
 
 }  // namespace tq
