@@ -44,9 +44,9 @@ UNIT = "tokens/s"
 
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of decode_split_kernel<2,4>
-# per cached token (235,449,600 + 6,678,272 B over 16*8*16384 tokens), or None
+# per cached token (235,454,976 + 6,258,176 B over 16*8*16384 tokens), or None
 # when the kernel has changed since that capture.
-SPLIT_TRAFFIC_PER_TOKEN = None   # kernel changed since the last capture
+SPLIT_TRAFFIC_PER_TOKEN = (235_454_976 + 6_258_176) / (16 * 8 * 16384)
 
 EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536")
 
@@ -66,6 +66,8 @@ def parse():
                     help="run only this secondary workload (repeatable) and print its measurement")
     ap.add_argument("--slice-tokens", type=int, default=None,
                     help="context of the 70B-shaped slice for --extra runs (default 2^20)")
+    ap.add_argument("--search-rows", type=int, default=None,
+                    help="database rows of the search workload for --extra runs (default 10^6)")
     return ap.parse_args()
 
 
@@ -204,7 +206,7 @@ def _time_ms(fn, reps=3, warm=2):
     return a.elapsed_time(b) / reps
 
 
-def run_extras(dev, peak_gbs, select=None, slice_tokens=None):
+def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None):
     """Device-timed measurements of the other rows of the path, each on its
     own workload: encode and decode on the Llama-3.1-70B-shaped 1M-token
     slice, one ESM-2-650M encoder layer, and 1M-vector d=1536 search.
@@ -225,7 +227,7 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None):
     if "encoder_esm2_layer" in select:
         out.update(_extra_encoder(dev, g))
     if "search_1m_d1536" in select:
-        out.update(_extra_search(dev, g))
+        out.update(_extra_search(dev, g, search_rows))
     return out
 
 
@@ -288,7 +290,7 @@ def _extra_encoder(dev, g):
     return out
 
 
-def _extra_search(dev, g):
+def _extra_search(dev, g, rows=None):
     import torch
     import synth
     from vector_quantization_b200 import tq
@@ -296,6 +298,7 @@ def _extra_search(dev, g):
     # vector search: 1M x 1536 fp32, 1000 queries, top-10, 1+1 bits
     c = synth.CONFIGS["vector_search_d1536"]
     N, d, nq, kk, seed = c["n_db"], c["dim"], c["n_queries"], c["top_k"], c["seed"]
+    N = rows or N
     g.manual_seed(seed)
     lam = (torch.arange(1, d + 1, device=dev, dtype=torch.float32) ** -0.4)
     db = torch.randn((N, d), generator=g, device=dev) * lam
@@ -455,7 +458,7 @@ def run_ours(args, rank, world, local_rank):
     split_avg_s = float(np.mean(split_ms)) / 1e3
     achieved = bytes_per_launch / split_avg_s / 1e9
     # DRAM bytes per launch of the split kernel, from one ncu capture of the
-    # T = 16384 case (read + write = 242.13 MB), scaled by the token count to
+    # T = 16384 case (read + write = 241.71 MB), scaled by the token count to
     # the launch timed here; traffic grows in proportion to the tokens streamed.
     # Must be reset to None whenever decode_split_kernel changes.
     traffic = SPLIT_TRAFFIC_PER_TOKEN * B * Hkv * T if SPLIT_TRAFFIC_PER_TOKEN and args.bits == 2 else None
@@ -492,7 +495,8 @@ def main():
         import torch
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
-        print(json.dumps({"extras": run_extras(dev, measured_peaks()[0], args.extra, args.slice_tokens)}), flush=True)
+        print(json.dumps({"extras": run_extras(dev, measured_peaks()[0], args.extra, args.slice_tokens,
+                                               args.search_rows)}), flush=True)
         return
     if world > 1:
         import datetime
