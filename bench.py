@@ -48,7 +48,7 @@ UNIT = "tokens/s"
 # when the kernel has changed since that capture.
 SPLIT_TRAFFIC_PER_TOKEN = (235_454_976 + 6_258_176) / (16 * 8 * 16384)
 
-EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536")
+EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1")
 
 
 def parse():
@@ -228,6 +228,8 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None):
         out.update(_extra_encoder(dev, g))
     if "search_1m_d1536" in select:
         out.update(_extra_search(dev, g, search_rows))
+    if "decode_llama8b_layer_3p1" in select:
+        out.update(_extra_decode_3p1(dev, peak_gbs))
     return out
 
 
@@ -303,16 +305,55 @@ def _extra_search(dev, g, rows=None):
     lam = (torch.arange(1, d + 1, device=dev, dtype=torch.float32) ** -0.4)
     db = torch.randn((N, d), generator=g, device=dev) * lam
     qs = torch.randn((nq, d), generator=g, device=dev) * lam
-    rot = tq.Rotation(d, 1, synth.rotation_randomness(d, [seed, 1], dense=True), kind="dense")
-    wsd = tq.alloc_workspace(tq._lib.tq_quantize_dense_workspace_size(rot.handle, N), dev)
-    packed = tq.empty_records(rot, (N,), dev)
-    ms_enc = _time_ms(lambda: tq.quantize_dense(rot, db, out=packed, workspace=wsd), reps=1, warm=1)
-    wss = tq.alloc_workspace(tq.search_workspace_size(rot, nq, N, kk), dev)
-    ms = _time_ms(lambda: tq.search_topk(rot, qs, packed, kk, workspace=wss), reps=2, warm=1)
-    flops = 2 * nq * N * (d + d)
-    out["search_1m_d1536"] = {"queries_per_s": nq / ms * 1e3, "ms": round(ms, 3), "TFLOP_s": round(flops / ms / 1e9, 1),
-                              "encode_ms": round(ms_enc, 3), "note": "1+1 bits, top-10; data isotropic-in-basis stand-in"}
+    wsd = None
+    for bits, key in ((1, "search_1m_d1536"), (3, "search_1m_d1536_3p1")):
+        rot = tq.Rotation(d, bits, synth.rotation_randomness(d, [seed, bits], dense=True), kind="dense")
+        if wsd is None:
+            wsd = tq.alloc_workspace(tq._lib.tq_quantize_dense_workspace_size(rot.handle, N), dev)
+        packed = tq.empty_records(rot, (N,), dev)
+        ms_enc = _time_ms(lambda: tq.quantize_dense(rot, db, out=packed, workspace=wsd), reps=1, warm=1)
+        wss = tq.alloc_workspace(tq.search_workspace_size(rot, nq, N, kk), dev)
+        ms = _time_ms(lambda: tq.search_topk(rot, qs, packed, kk, workspace=wss), reps=2, warm=1)
+        flops = 2 * nq * N * (d + d)
+        gemm_flops = 2 * N * d * d * 2   # y = Pi x and S r, one fp32 product each
+        out[key] = {"queries_per_s": nq / ms * 1e3, "ms": round(ms, 3), "TFLOP_s": round(flops / ms / 1e9, 1),
+                    "encode_ms": round(ms_enc, 3), "encode_TFLOP_s": round(gemm_flops / ms_enc / 1e9, 1),
+                    "note": f"{bits}+1 bits, top-10; data isotropic-in-basis stand-in"}
+        del packed, wss
     return out
+
+
+def _extra_decode_3p1(dev, peak_gbs):
+    """One layer of the Llama-3.1-8B-shaped decode (B16, Hq32, Hkv8, T32768)
+    at 4-bit (3+1): the split kernel's time and bandwidth."""
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["llama31_8b_gqa_decode"]
+    B, Hq, Hkv, d, T, seed = c["batch"], c["q_heads"], c["kv_heads"], c["head_dim"], c["tokens"], c["seed"]
+    rk = tq.Rotation(d, 3, synth.rotation_randomness(d, [seed, 7, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(d, 3, synth.rotation_randomness(d, [seed, 7, 2]))
+    kc, vc = tq.empty_records(rk, (B, Hkv, T), dev), tq.empty_records(rv, (B, Hkv, T), dev)
+    x = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, 7, 3], dev)
+    tq.quantize_kv(rk, x, apply_rope=True, pos_period=T, out=kc)
+    x = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, 7, 4], dev)
+    tq.quantize_kv(rv, x, out=vc)
+    del x
+    q = synth.heavy_tailed_torch((B, Hq, d), [seed, 7, 5], dev)
+    qpos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    ws = tq.alloc_workspace(tq.decode_workspace_size(rk, rv, B, Hq, Hkv, T), dev)
+    o = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(8)]
+    for i in range(11):
+        if i >= 3:
+            tq.profile_next_decode(*ev[i - 3])
+        tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws)
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    byts = B * Hkv * T * 2 * rec_bytes({"head_dim": d}, argparse.Namespace(bits=3))
+    return {"decode_llama8b_layer_3p1": {"split_ms": round(ms, 4), "GB_s": round(byts / ms / 1e6, 1),
+                                         "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
+                                         "algorithmic_bytes": byts, "note": "one layer, 144 B per token pair"}}
 
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):

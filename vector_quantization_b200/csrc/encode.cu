@@ -628,6 +628,222 @@ __global__ void __launch_bounds__(kRowThreads, 1) encode_rows_kernel(EncodeParam
   if (warp == 0) tqtc::tmem_free(tmem_slot, 2 * D);
 }
 
+// ===========================================================================
+// Two threads per vector (d = 128): thread h of a pair (lanes l and l ^ 16)
+// holds the coordinates whose bit 5 equals h, {32h + i, 64 + 32h + i : i < 32},
+// so RoPE pairs (i, i + 64) and six of the seven Walsh-Hadamard stages stay in
+// the thread and one stage (bit 5) crosses lanes; each thread assembles two
+// whole plane words (coordinates 32h.., 64 + 32h..).  A CTA of 8 warps owns
+// one 128-row tile at a time; with half the registers of the one-thread
+// kernel two CTAs share an SM, so one CTA's tensor-core product and read-back
+// overlap the other's per-vector work.
+// ===========================================================================
+constexpr int kPairThreads = 256;
+
+template <int BITS, typename T>
+__global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodeParams p) {
+  constexpr int D = 128, NJ = 4;
+  constexpr int OPB = kTileVec * D * 2;           // bytes of one bf16 [128 x D] operand
+  constexpr int SB = D * D * 2;                   // bytes of S [m x d] bf16
+  extern __shared__ uint8_t raw[];
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ __align__(16) float dsg_s[D];
+  uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
+  uint8_t* s_op = base;
+  uint8_t* r_hi = base + SB;
+  uint8_t* r_lo = r_hi + OPB;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = lane >> 4;                                            // half of the vector
+  const int t = 32 * (warp & 3) + 16 * (warp >> 2) + (lane & 15);    // row in the tile
+  for (int c = tid; c < SB / 16; c += blockDim.x) tqdev::cp_async16(s_op + 16 * c, p.s_op + 8 * c, 16);
+  tqdev::cp_async_commit();
+  if (tid < D) dsg_s[tid] = p.dsg[tid];
+  if (tid == 0) tqtc::mbar_init(&mbar, 1);
+  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, D);
+  tqdev::cp_async_wait<0>();
+  tqtc::fence_before_sync();
+  __syncthreads();
+  tqtc::fence_after_sync();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t idesc = tqtc::idesc_bf16_f32(kTileVec, D);
+  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  float tp[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tp[k] = p.tpos[k];
+  const int64_t n_tiles = (p.n + kTileVec - 1) / kTileVec;
+  const uint32_t rowbase = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
+  const uint32_t vx = t & 7;
+  uint32_t phase = 0;
+
+  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+    const int64_t row = tile * kTileVec + t;
+    bool valid = row < p.n;
+    float u[64];   // u[32 s + i] = coordinate 64 s + 32 h + i
+    float nrm = 0.f, rr = 0.f;
+    if (valid) {
+      const T* xr = static_cast<const T*>(p.x) + row * p.ld;
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr) + 8 * sh + 4 * h + q);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              u[32 * sh + 8 * q + 2 * e] = __uint_as_float(w[e] << 16);
+              u[32 * sh + 8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+            }
+          }
+      } else {
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(xr) + 16 * sh + 8 * h + q);
+            u[32 * sh + 4 * q] = v.x;
+            u[32 * sh + 4 * q + 1] = v.y;
+            u[32 * sh + 4 * q + 2] = v.z;
+            u[32 * sh + 4 * q + 3] = v.w;
+          }
+      }
+      if (p.rope) {
+        const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
+        if (pos < 0 || pos >= p.rope_max_pos) {
+          valid = false;
+          if (h == 0) p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+        } else {
+          // frequencies 32h + i of the pairs (u[i], u[32 + i])
+          const float4* hi = reinterpret_cast<const float4*>(p.rope_hi + (pos >> kRopeLoBits) * (D / 2)) + 16 * h;
+          const float4* lo = reinterpret_cast<const float4*>(p.rope_lo + (pos & (kRopeLoRows - 1)) * (D / 2)) + 16 * h;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float4 a = __ldg(hi + c), b = __ldg(lo + c);
+            const float c0 = a.x * b.x - a.y * b.y, s0 = a.y * b.x + a.x * b.y;
+            const float c1 = a.z * b.z - a.w * b.w, s1 = a.w * b.z + a.z * b.w;
+            const float x0 = u[2 * c], y0 = u[32 + 2 * c], x1 = u[2 * c + 1], y1 = u[33 + 2 * c];
+            u[2 * c] = x0 * c0 - y0 * s0;
+            u[32 + 2 * c] = y0 * c0 + x0 * s0;
+            u[2 * c + 1] = x1 * c1 - y1 * s1;
+            u[33 + 2 * c] = y1 * c1 + x1 * s1;
+          }
+        }
+      }
+    }
+    // every lane runs the transform (shuffles need the whole warp); rows
+    // that are absent or out of RoPE range carry zeros and store nothing
+    if (!valid) {
+#pragma unroll
+      for (int e = 0; e < 64; ++e) u[e] = 0.f;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 dv = *reinterpret_cast<const float4*>(dsg_s + 64 * sh + 32 * h + 4 * q);
+        const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float& x = u[32 * sh + 4 * q + e];
+          ss = fmaf(x, x, ss);
+          x *= dd[e];
+        }
+      }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+    nrm = sqrtf(ss);
+    fwht_regs<64>(u);                                   // coordinate bits 0-4 and 6
+    const float sgn = h ? -1.f : 1.f;                   // coordinate bit 5: across the lane pair
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, u[e], 16);
+      u[e] = fmaf(sgn, u[e], o);
+    }
+    const float scale = (nrm > 0.f ? 1.0f / nrm : 0.f) * inv_sqrt_d;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) u[e] = fmaf(u[e], scale, 0.f);   // unit-vector coordinates, -0 -> +0
+    float nl[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) nl[k] = nrm * p.lpos[k];
+    uint32_t w0[BITS], w1[BITS];
+    rr = quantize32<BITS>(u, tp, nl, nrm, w0);          // coordinates 32h .. 32h + 31: word h
+    rr += quantize32<BITS>(u + 32, tp, nl, nrm, w1);    // 64 + 32h ..: word 2 + h
+    rr += __shfl_xor_sync(0xffffffffu, rr, 16);
+    if (valid) {
+      uint32_t* crec = p.codes + row * p.out_stride * (BITS * NJ);   // 4-byte aligned records
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) {
+        crec[k * NJ + h] = w0[k];
+        crec[k * NJ + 2 + h] = w1[k];
+      }
+      if (h == 0) p.norms[row * p.out_stride] = make_float2(nrm, sqrtf(rr));
+    }
+    // residual as bf16 hi + lo into row t of the A operand (16-byte chunks)
+#pragma unroll
+    for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hv[4], lv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = valid ? u[32 * sh + 8 * q + 2 * e] : 0.f, b = valid ? u[32 * sh + 8 * q + 2 * e + 1] : 0.f;
+          __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
+          const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb);
+          __nv_bfloat162 lb =
+              __floats2bfloat162_rn(a - __uint_as_float(hbits << 16), b - __uint_as_float(hbits & 0xFFFF0000u));
+          hv[e] = hbits;
+          lv[e] = *reinterpret_cast<uint32_t*>(&lb);
+        }
+        const int c = 8 * sh + 4 * h + q;   // 16-byte chunk of the row
+        const uint32_t off = (c >> 3) * (kTileVec * 128) + rowbase + ((((c & 7) ^ vx)) << 4);
+        *reinterpret_cast<uint4*>(r_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(r_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+      }
+    // ---- S r of the tile on the tensor core
+    tqtc::fence_smem_to_async();
+    tqtc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      tqtc::fence_after_sync();
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tqtc::mma_bf16_ss(tmem, tqtc::sw128_desc_kstep(tqtc::smem_u32(r_hi), ks, kTileVec),
+                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tqtc::mma_bf16_ss(tmem, tqtc::sw128_desc_kstep(tqtc::smem_u32(r_lo), ks, kTileVec),
+                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, true);
+      tqtc::mma_commit(&mbar);
+    }
+    const bool ok = tqtc::mbar_wait(&mbar, phase, kWaitLimit);
+    phase ^= 1;
+    tqtc::fence_after_sync();
+    // ---- sign bits: warp w reads lanes 32 (w % 4) + lane, columns 64 (w / 4) ..
+    {
+      const int quad = warp & 3, part = warp >> 2;
+      const int64_t srow = tile * kTileVec + quad * 32 + lane;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float val[32];
+        tqtc::tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 64 * part + 32 * c, val);
+        uint32_t w = 0;
+#pragma unroll
+        for (int b = 31; b >= 0; --b) w = (w << 1) | (val[b] >= 0.f ? 1u : 0u);
+        if (srow < p.n) p.signs[srow * p.out_stride * NJ + 2 * part + c] = ok ? w : 0u;
+      }
+      if (!ok && part == 0 && srow < p.n)
+        p.norms[srow * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    }
+    tqtc::fence_before_sync();
+    __syncthreads();
+  }
+  tqtc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tqtc::tmem_free(tmem_slot, D);
+}
+
 template <int D, int BITS, typename T>
 int launch_encode_rows(const EncodeParams& p, cudaStream_t stream) {
   // S + two groups x (hi, lo) residual tiles + (bf16) two staged input tiles:
@@ -650,9 +866,25 @@ int launch_encode_rows(const EncodeParams& p, cudaStream_t stream) {
 // Batches below this many vectors take the low-latency warp-per-vector kernel.
 constexpr int64_t kRowsKernelMinN = 16384;
 
+template <int BITS, typename T>
+int launch_encode_pairs(const EncodeParams& p, cudaStream_t stream) {
+  const size_t smem = 128 * 128 * 2 + 2 * static_cast<size_t>(kTileVec) * 128 * 2 + 1024;   // 97 KB: 2 CTAs / SM
+  auto kern = encode_pairs_kernel<BITS, T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return TQ_ECUDA;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = (p.n + kTileVec - 1) / kTileVec;
+  const int blocks = static_cast<int>(tiles < 2LL * sms ? tiles : 2LL * sms);
+  kern<<<blocks, kPairThreads, smem, stream>>>(p);
+  return tq::launch_status();
+}
+
 template <int D, int BITS, typename T>
 int launch_encode(const EncodeParams& p, cudaStream_t stream) {
   if (p.n < kRowsKernelMinN) return launch_encode_warp<D, BITS, T>(p, stream);
+  if constexpr (D == 128) return launch_encode_pairs<BITS, T>(p, stream);
   return launch_encode_rows<D, BITS, T>(p, stream);
 }
 
