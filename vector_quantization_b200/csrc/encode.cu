@@ -680,6 +680,15 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodePar
   for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
     const int64_t row = tile * kTileVec + t;
     bool valid = row < p.n;
+    {
+      // pull this row of the CTA's next tile toward L2 (thread h: the row's
+      // 128-byte line h for bf16) so its loads need not wait on DRAM
+      const int64_t nrow = row + static_cast<int64_t>(gridDim.x) * kTileVec;
+      if (nrow < p.n) {
+        const char* np = reinterpret_cast<const char*>(static_cast<const T*>(p.x) + nrow * p.ld) + h * 64 * sizeof(T);
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(np));
+      }
+    }
     float u[64];   // u[32 s + i] = coordinate 64 s + 32 h + i
     float nrm = 0.f, rr = 0.f;
     if (valid) {
