@@ -75,6 +75,19 @@ def test_encode_parity_large_batch(cuda_device, d, bits, dtype):
     _run_encode(d, bits, 16384 + 1031, dtype, rope=True, seed=200 + bits)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_encode_parity_small_batch(cuda_device, d, bits, dtype):
+    """Batches of at most 256 vectors (a decode step's appended keys and
+    values) take the block-per-vector kernel."""
+    _run_encode(d, bits, 256, dtype, rope=True, seed=220 + bits, period=100, offset=(1 << 20) - 150)
+
+
+def test_encode_small_batch_positions_array_strided(cuda_device):
+    _run_encode(128, 3, 128, torch.bfloat16, rope=True, seed=230, offset=77, pos_array=True, out_stride=5)
+
+
 def test_encode_large_batch_positions_array_strided(cuda_device):
     _run_encode(128, 2, 16384 + 77, torch.bfloat16, rope=True, seed=210, period=5000, offset=3,
                 pos_array=True, out_stride=2)

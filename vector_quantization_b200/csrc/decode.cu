@@ -131,6 +131,13 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
     cp_async_commit();
   };
 
+  // The first tiles of the cache do not depend on the q-prep launch: start
+  // their copies, then wait for q-prep's outputs (programmatic dependent
+  // launch; a no-op when launched without it).
+#pragma unroll 1
+  for (int i = 0; i < kStages - 1; ++i) issue(i);
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+
   uint32_t qf[2][NT][8][2];
   float2 kc[2][NT];
   {
@@ -386,9 +393,6 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
     return static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
   };
 
-#pragma unroll 1
-  for (int i = 0; i < kStages - 1; ++i) issue(i);
-
   // Pipelined order for G <= 4; with G = 8 the two tiles' live values would
   // not fit the register file, so tiles run one after the other.
   constexpr bool kPipe = G <= 4;
@@ -563,6 +567,8 @@ __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ 
   float scol[kD];
 #pragma unroll
   for (int k = 0; k < kD; ++k) scol[k] = __ldg(st + k * kD + i);
+  // S belongs to the handle; q may come from the previous launch
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   float v[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -685,6 +691,7 @@ __global__ void __launch_bounds__(kD) decode_merge_kernel(const float* __restric
   float scol[kD];
 #pragma unroll
   for (int j = 0; j < kD; ++j) scol[j] = __ldg(s_mat + j * kD + i);
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the split kernel's partials
   const float* base = partial + static_cast<size_t>(bh) * n_splits * G * REC;
   for (int h = warp; h < G; h += W) {
     float M = -INFINITY;
@@ -771,6 +778,24 @@ size_t workspace_for(int B, int Hq, int Hkv, int64_t T) {
          align256(static_cast<size_t>(BH) * sp.n_splits * G * (2 + 2 * kD) * sizeof(float));
 }
 
+// Launch that may overlap the tail of the previous kernel on the stream
+// (programmatic dependent launch); the kernel waits for it with
+// griddepcontrol.wait before touching that kernel's outputs.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? TQ_OK : TQ_ECUDA;
+}
+
 template <int BITS, int G>
 int launch_split(const DecodeParams& p, int BH, cudaStream_t s) {
   constexpr int CB = BITS * kD / 8, SB = kD / 8;
@@ -782,16 +807,15 @@ int launch_split(const DecodeParams& p, int BH, cudaStream_t s) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return TQ_ECUDA;
   dim3 grid(p.n_splits, BH);
-  kern<<<grid, kWarps * 32, smem, s>>>(p);
-  return tq::launch_status();
+  return launch_pdl(kern, grid, dim3(kWarps * 32), smem, s, p);
 }
 
 template <typename T>
 void qprep_g(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope, uint16_t* qfrag,
              float2* kconst, cudaStream_t s) {
-#define TQ_QPREP(GG)                                                                                        \
-  decode_qprep_kernel<T, GG><<<BH, kD, 0, s>>>(q, q_pos, Hkv, hk->d_signs, hk->d_st, hk->d_rope_hi, hk->d_rope_lo, \
-                                               hk->rope_max_pos, rope, qfrag, kconst)
+#define TQ_QPREP(GG)                                                                                       \
+  launch_pdl(decode_qprep_kernel<T, GG>, dim3(BH), dim3(kD), 0, s, q, q_pos, Hkv, hk->d_signs, hk->d_st,        \
+             hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope, qfrag, kconst)
   switch (G) {
     case 1: TQ_QPREP(1); break;
     case 2: TQ_QPREP(2); break;
@@ -814,10 +838,10 @@ int launch_merge(int G, int BH, const float* partial, int n_splits, const tq_rot
   const float qjl = static_cast<float>(kQjlConst / hv->m);
   const size_t fsb = static_cast<size_t>(n_splits) * G * sizeof(float);   // <= 1184 * 8 * 4 bytes
   switch (G) {
-    case 1: decode_merge_kernel<1><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
-    case 2: decode_merge_kernel<2><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
-    case 4: decode_merge_kernel<4><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
-    case 8: decode_merge_kernel<8><<<BH, kD, fsb, s>>>(partial, n_splits, hv->d_s, hv->d_signs, qjl, out); break;
+    case 1: return launch_pdl(decode_merge_kernel<1>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 2: return launch_pdl(decode_merge_kernel<2>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 4: return launch_pdl(decode_merge_kernel<4>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 8: return launch_pdl(decode_merge_kernel<8>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
     default: return TQ_EUNSUPPORTED;
   }
   return tq::launch_status();

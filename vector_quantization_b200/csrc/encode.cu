@@ -30,6 +30,7 @@ struct EncodeParams {
   int64_t out_stride;
   const float* dsigns;  // [D]
   const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
+  const float* st;      // S transposed, fp32: st[k * d + j] = S[j][k]
   int rows;             // warp-per-vector kernel: vectors per tile, R in {8, 16, ..., 128}
   const float* thresholds;
   const float* levels;
@@ -46,6 +47,129 @@ struct EncodeParams {
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
 constexpr int kTileVec = 128;
 constexpr int kWaitLimit = 1 << 22;
+
+// ===========================================================================
+// Block-per-vector encode, for the few vectors a decode step appends: thread
+// i owns coordinate i; RoPE pairs meet through shared memory, the norm and
+// ||r|| are block reductions, the Walsh-Hadamard transform takes five
+// shuffle stages and log2(d/32) shared-memory stages, a warp ballot yields a
+// plane word, and S r is a matrix-vector product on the CUDA cores with row i
+// of S loaded into registers at the start (so its loads overlap the rest).
+// ===========================================================================
+template <int D, int BITS, typename T>
+__global__ void __launch_bounds__(D) encode_vec_kernel(EncodeParams p) {
+  constexpr int NW = D / 32;
+  __shared__ __align__(16) float buf[D];
+  __shared__ float red[2][NW];
+  const int i = threadIdx.x, lane = i & 31, w = i >> 5;
+  const int64_t row = blockIdx.x;
+  float scol[D];   // row i of S
+#pragma unroll
+  for (int k = 0; k < D; ++k) scol[k] = __ldg(p.st + k * D + i);
+  // S belongs to the handle; everything below may depend on the previous
+  // launch on the stream (programmatic dependent launch)
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  const T* xr = static_cast<const T*>(p.x) + row * p.ld;
+  float x;
+  if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(xr) + i);
+  else x = __bfloat162float(xr[i]);
+  const int64_t rec = row * p.out_stride;
+  if (p.rope) {
+    const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
+    if (pos < 0 || pos >= p.rope_max_pos) {   // uniform over the block
+      if (i == 0) p.norms[rec] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+      return;
+    }
+    buf[i] = x;
+    __syncthreads();
+    const int j = i & (D / 2 - 1);
+    const float2 a = p.rope_hi[(pos >> kRopeLoBits) * (D / 2) + j];
+    const float2 b = p.rope_lo[(pos & (kRopeLoRows - 1)) * (D / 2) + j];
+    const float cs = a.x * b.x - a.y * b.y, sn = a.y * b.x + a.x * b.y;
+    const float x1 = buf[j], x2 = buf[j + D / 2];
+    x = i < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
+  }
+  // ||x|| and u = H D x (unnormalised, Sylvester order)
+  float ss = x * x;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  float u = x * p.dsg[i];
+#pragma unroll
+  for (int bit = 1; bit < 32; bit <<= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, u, bit);
+    u = (lane & bit) ? o - u : u + o;
+  }
+  if (lane == 0) red[0][w] = ss;
+#pragma unroll
+  for (int bit = 32; bit < D; bit <<= 1) {
+    __syncthreads();
+    buf[i] = u;
+    __syncthreads();
+    const float o = buf[i ^ bit];
+    u = (i & bit) ? o - u : u + o;
+  }
+  __syncthreads();
+  ss = 0.f;
+#pragma unroll
+  for (int q = 0; q < NW; ++q) ss += red[0][q];
+  const float nrm = sqrtf(ss);
+  const float y = fmaf(u, (nrm > 0.f ? 1.0f / nrm : 0.f) * rsqrtf(static_cast<float>(D)), 0.f);   // -0 -> +0
+  // symmetric codebook: sign picks the half, |y| against the positive thresholds the level
+  const bool pos = y >= 0.f;
+  const float a = fabsf(y);
+  uint32_t bits[BITS];
+  float mag;
+  if constexpr (BITS == 1) {
+    bits[0] = pos;
+    mag = p.lpos[0];
+  } else if constexpr (BITS == 2) {
+    const bool o = a >= p.tpos[0];
+    bits[1] = pos;
+    bits[0] = pos == o;
+    mag = o ? p.lpos[1] : p.lpos[0];
+  } else {
+    const bool m1 = a >= p.tpos[0], m2 = a >= p.tpos[1], m3 = a >= p.tpos[2];
+    bits[2] = pos;
+    bits[1] = pos == m2;
+    bits[0] = pos == (m1 != (m2 != m3));
+    mag = m3 ? p.lpos[3] : (m2 ? p.lpos[2] : (m1 ? p.lpos[1] : p.lpos[0]));
+  }
+  const float r = nrm * (y - copysignf(mag, y));
+  uint32_t* crec = p.codes + rec * (BITS * NW);
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) {
+    const uint32_t word = __ballot_sync(0xffffffffu, bits[k]);
+    if (lane == 0) crec[k * NW + w] = word;
+  }
+  float rr = r * r;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
+  if (lane == 0) red[1][w] = rr;
+  buf[i] = r;
+  __syncthreads();
+  // (S r)_i
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < D; k += 4) {
+    const float4 rv = *reinterpret_cast<const float4*>(buf + k);
+    acc[0] = fmaf(scol[k], rv.x, acc[0]);
+    acc[1] = fmaf(scol[k + 1], rv.y, acc[1]);
+    acc[2] = fmaf(scol[k + 2], rv.z, acc[2]);
+    acc[3] = fmaf(scol[k + 3], rv.w, acc[3]);
+  }
+  const float proj = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  const uint32_t sword = __ballot_sync(0xffffffffu, proj >= 0.f);
+  if (lane == 0) p.signs[rec * NW + w] = sword;
+  if (i == 0) {
+    rr = 0.f;
+#pragma unroll
+    for (int q = 0; q < NW; ++q) rr += red[1][q];
+    p.norms[rec] = make_float2(nrm, sqrtf(rr));
+  }
+}
+
+// Batches up to this many vectors take the block-per-vector kernel.
+constexpr int64_t kVecKernelMaxN = 256;
 
 // ===========================================================================
 // Warp-per-vector encode, for small batches (a decode step's new keys and
@@ -892,6 +1016,18 @@ int launch_encode_pairs(const EncodeParams& p, cudaStream_t stream) {
 
 template <int D, int BITS, typename T>
 int launch_encode(const EncodeParams& p, cudaStream_t stream) {
+  if (p.n <= kVecKernelMaxN) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.n));
+    cfg.blockDim = dim3(D);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, encode_vec_kernel<D, BITS, T>, p) == cudaSuccess ? TQ_OK : TQ_ECUDA;
+  }
   if (p.n < kRowsKernelMinN) return launch_encode_warp<D, BITS, T>(p, stream);
   if constexpr (D == 128) return launch_encode_pairs<BITS, T>(p, stream);
   return launch_encode_rows<D, BITS, T>(p, stream);
@@ -946,6 +1082,7 @@ extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, in
   p.out_stride = out_stride;
   p.dsigns = h->d_signs;
   p.s_op = h->d_s_op;
+  p.st = h->d_st;
   {
     const int half = 1 << (h->bits - 1);
     for (int i = 0; i < h->d && i < 128; ++i) p.dsg[i] = h->signs[i];
