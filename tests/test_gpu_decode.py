@@ -121,3 +121,33 @@ def test_tiny_workload_end_to_end(cuda_device):
     _, _, _, ek = oracle_records(rk_o, k.reshape(-1, D), np.arange(T))
     compare_records(rk_o, tuple(t.cpu().numpy() for t in kcache), ek)
     assert_close(out.cpu().numpy(), ref, what="tiny end-to-end")
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_decode_full_size_sampled(cuda_device, bits):
+    """The Llama-3.1-8B-shaped decode layer at full size (batch 16, 32 query
+    heads over 8 KV heads, 32768 cached tokens, heavy-tailed bf16 K/V, RoPE)
+    in the launch configuration the bench times: GPU-encoded caches, one
+    decode launch; sampled (sequence, KV head) pairs checked against the
+    oracle's attention over the very same packed records."""
+    from vector_quantization_b200 import tq
+    dev = torch.device("cuda:0")
+    cfg = synth.CONFIGS["llama31_8b_gqa_decode"]
+    B, Hq, Hkv, T, seed = cfg["batch"], cfg["q_heads"], cfg["kv_heads"], cfg["tokens"], cfg["seed"]
+    G = Hq // Hkv
+    rk = tq.Rotation(D, bits, synth.rotation_randomness(D, [seed, 11]), rope_base=10000.0, rope_max_pos=T)
+    rv = tq.Rotation(D, bits, synth.rotation_randomness(D, [seed, 12]))
+    rk_o, _ = oracle_rotation(D, bits, [seed, 11], rope=10000.0)
+    rv_o, _ = oracle_rotation(D, bits, [seed, 12])
+    kc = tq.quantize_kv(rk, synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 13], dev), apply_rope=True, pos_period=T)
+    vc = tq.quantize_kv(rv, synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 14], dev))
+    q = synth.heavy_tailed_torch((B, Hq, D), [seed, 15], dev)
+    q_pos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    out = tq.decode_attention(rk, rv, q, q_pos, kc, vc, T)
+    torch.cuda.synchronize()
+    for b, j in [(0, 0), (B - 1, Hkv - 1), (7, 3)]:
+        kk = tuple(a[b:b + 1, j:j + 1].cpu().numpy() for a in kc)
+        vv = tuple(a[b:b + 1, j:j + 1].cpu().numpy() for a in vc)
+        qq = q[b:b + 1, j * G:(j + 1) * G].float().cpu().numpy()
+        ref = at.decode_attention(rk_o, rv_o, qq, [T - 1], kk, vv, 1 / np.sqrt(D))
+        assert_close(out[b:b + 1, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"bits {bits} seq {b} kv-head {j}")
