@@ -29,7 +29,7 @@ namespace {
 
 using namespace tqdev;
 
-constexpr int kWarps = 8;          // warps per CTA, 8 queries each
+constexpr int kWarps = 4;          // warps per CTA, 8 queries each (3 CTAs per SM at d = 64)
 constexpr int kQPerWarp = 8;
 constexpr int kChunk = 128;        // keys staged per shared-memory chunk
 constexpr float kLazyRescale = 8.0f;
@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256) encoder_qprep_kernel(const T* __restrict_
 }
 
 template <int D, int BITS>
-__global__ void __launch_bounds__(kWarps * 32) encoder_attention_kernel(EncParams p) {
+__global__ void __launch_bounds__(kWarps * 32, D == 64 ? 3 : 1) encoder_attention_kernel(EncParams p) {
   constexpr int P = Planes<BITS>::P;
   constexpr int CB = BITS * D / 8, SB = D / 8;
   constexpr int KB = D / 16;             // k-blocks of the score MMA
