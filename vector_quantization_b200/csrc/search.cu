@@ -13,13 +13,13 @@
 // scoring kernel, and a merge of the per-range candidate lists.
 //
 // Scoring kernel: one CTA = 16 queries x a range of database rows.  The
-// queries' B fragments (all d dims) stay resident in shared memory; 4 warps
-// take 16 database rows each per 64-row tile and build the A operand of
+// queries' B fragments (all d dims) stay resident in shared memory; 8 warps
+// take 16 database rows each per 128-row tile and build the A operand of
 // mma.sync m16n8k16 (fp16, fp32 accumulate) straight from the packed code and
 // sign bit-planes with one LOP3 per register (bitplane.cuh).  Code planes are
 // in Walsh form, so they are exact; the query side is a single fp16 piece
 // (2^-12 relative), well inside the score tolerance for this workload.  Each
-// warp keeps the running top-k of 4 queries in registers (lane i = rank i),
+// warp keeps the running top-k of 2 queries in registers (lane i = rank i),
 // inserting candidates warp-parallel.
 #include <cmath>
 
@@ -37,8 +37,9 @@ using namespace tqdev;
 
 constexpr int kQT = 16;          // queries per CTA
 constexpr int kRowsPerWarp = 16;
-constexpr int kSWarps = 4;
-constexpr int kTileRows = kSWarps * kRowsPerWarp;   // 64 database rows per tile
+constexpr int kSWarps = 8;
+constexpr int kTileRows = kSWarps * kRowsPerWarp;   // 128 database rows per tile
+constexpr int kQPW = kQT / kSWarps;                 // queries whose top-k one warp keeps
 constexpr int kMaxK = 32;
 
 struct SearchParams {
@@ -103,11 +104,11 @@ __global__ void __launch_bounds__(kSWarps * 32) search_score_kernel(SearchParams
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
     for (int e = 0; e < 2; ++e) qc[nt][e] = p.qconst[qtile * kQT + 8 * nt + 2 * tig + e];
-  // this warp's running top-k of queries 4 warp .. 4 warp + 3 (lane = rank)
-  float ls[4];
-  int64_t li[4];
+  // this warp's running top-k of queries kQPW warp .. (lane = rank)
+  float ls[kQPW];
+  int64_t li[kQPW];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < kQPW; ++j) {
     ls[j] = -INFINITY;
     li[j] = INT64_MAX;
   }
@@ -131,14 +132,26 @@ __global__ void __launch_bounds__(kSWarps * 32) search_score_kernel(SearchParams
 #pragma unroll
         for (int r = 0; r < 4; ++r) cacc[pl][nt][r] = 0.f;
     }
+    // word tig of 128-dim block blk of every plane (and of the signs), rows
+    // gid and gid + 8; the next block's words are loaded one block ahead
+    uint32_t nx0[BITS + 1], nx1[BITS + 1];
+    auto load_words = [&](int blk) {
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) {
+        nx0[k] = __ldg(reinterpret_cast<const uint32_t*>(c0 + k * (p.d / 8)) + 4 * blk + tig);
+        nx1[k] = __ldg(reinterpret_cast<const uint32_t*>(c1 + k * (p.d / 8)) + 4 * blk + tig);
+      }
+      nx0[BITS] = __ldg(reinterpret_cast<const uint32_t*>(s0p) + 4 * blk + tig);
+      nx1[BITS] = __ldg(reinterpret_cast<const uint32_t*>(s1p) + 4 * blk + tig);
+    };
+    load_words(0);
 #pragma unroll 1
     for (int blk = 0; blk < p.nblk; ++blk) {
-      // word tig of 128-dim block blk of every plane, rows gid and gid + 8
       uint32_t raw0[BITS], raw1[BITS];
 #pragma unroll
       for (int k = 0; k < BITS; ++k) {
-        raw0[k] = __ldg(reinterpret_cast<const uint32_t*>(c0 + k * (p.d / 8)) + 4 * blk + tig);
-        raw1[k] = __ldg(reinterpret_cast<const uint32_t*>(c1 + k * (p.d / 8)) + 4 * blk + tig);
+        raw0[k] = nx0[k];
+        raw1[k] = nx1[k];
       }
       uint32_t w0[P + 1], w1[P + 1];
       {
@@ -150,9 +163,10 @@ __global__ void __launch_bounds__(kSWarps * 32) search_score_kernel(SearchParams
           w0[q] = pl0[q];
           w1[q] = pl1[q];
         }
-        w0[P] = __ldg(reinterpret_cast<const uint32_t*>(s0p) + 4 * blk + tig);
-        w1[P] = __ldg(reinterpret_cast<const uint32_t*>(s1p) + 4 * blk + tig);
+        w0[P] = nx0[BITS];
+        w1[P] = nx1[BITS];
       }
+      if (blk + 1 < p.nblk) load_words(blk + 1);
       uint32_t ws0[P + 1], ws1[P + 1];
 #pragma unroll
       for (int q = 0; q <= P; ++q) {
@@ -201,14 +215,14 @@ __global__ void __launch_bounds__(kSWarps * 32) search_score_kernel(SearchParams
         sc[qq * kTileRows + warp * kRowsPerWarp + gid + 8] = v1 ? fmaf(n1.x, code1, n1.y * p.qjl * z1) : -INFINITY;
       }
     __syncthreads();
-    // ---- top-k update: warp w owns queries 4w .. 4w+3 -------------------------
+    // ---- top-k update: warp w owns queries kQPW w .. kQPW w + kQPW - 1 ---------
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int qq = 4 * warp + j;
+    for (int j = 0; j < kQPW; ++j) {
+      const int qq = kQPW * warp + j;
       const float thr = __shfl_sync(0xffffffffu, ls[j], p.k - 1);
       const int64_t thr_id = __shfl_sync(0xffffffffu, li[j], p.k - 1);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < kTileRows / 32; ++half) {
         const int rr = half * 32 + lane;
         const float s = sc[qq * kTileRows + rr];
         const int64_t id = t0 + rr;
@@ -225,8 +239,8 @@ __global__ void __launch_bounds__(kSWarps * 32) search_score_kernel(SearchParams
   }
   // ---- write this range's candidates ---------------------------------------
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int q = qtile * kQT + 4 * warp + j;
+  for (int j = 0; j < kQPW; ++j) {
+    const int q = qtile * kQT + kQPW * warp + j;
     if (q < p.nq && lane < p.k) {
       const size_t o = (static_cast<size_t>(range) * p.nq + q) * p.k + lane;
       p.cand_score[o] = ls[j];
