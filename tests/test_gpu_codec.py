@@ -10,10 +10,10 @@ from oracle import rotation as ro
 pytestmark = pytest.mark.gpu
 
 
-def _gpu_rot(d, bits, seed, rope=0.0, kind="hadamard"):
+def _gpu_rot(d, bits, seed, rope=0.0, kind="hadamard", max_pos=(1 << 20) + 8):
     from vector_quantization_b200 import tq
     rnd = synth.rotation_randomness(d, seed, dense=(kind == "dense"))
-    return tq.Rotation(d, bits, rnd, kind, rope_base=rope, rope_max_pos=(1 << 20) + 8)
+    return tq.Rotation(d, bits, rnd, kind, rope_base=rope, rope_max_pos=max_pos)
 
 
 @pytest.mark.parametrize("d,bits", [(64, 2), (128, 1), (128, 2), (128, 3)])
@@ -27,9 +27,10 @@ def test_export_matches_oracle(cuda_device, d, bits):
     np.testing.assert_allclose(ex["thresholds"], o.thresholds, rtol=1e-10, atol=1e-15)
 
 
-def _run_encode(d, bits, n, dtype, rope, seed, period=None, offset=0, pos_array=False, out_stride=1, scale=1.0):
+def _run_encode(d, bits, n, dtype, rope, seed, period=None, offset=0, pos_array=False, out_stride=1, scale=1.0,
+                max_pos=(1 << 20) + 8):
     from vector_quantization_b200 import tq
-    g = _gpu_rot(d, bits, seed, rope=10000.0 if rope else 0.0)
+    g = _gpu_rot(d, bits, seed, rope=10000.0 if rope else 0.0, max_pos=max_pos)
     o, _ = oracle_rotation(d, bits, seed, rope=10000.0 if rope else 0.0)
     x = synth.heavy_tailed((n, d), seed + 1) * np.float32(scale)
     xt = torch.from_numpy(x).to(cuda_device_of()).to(dtype)
@@ -86,6 +87,21 @@ def test_encode_parity_small_batch(cuda_device, d, bits, dtype):
 
 def test_encode_small_batch_positions_array_strided(cuda_device):
     _run_encode(128, 3, 128, torch.bfloat16, rope=True, seed=230, offset=77, pos_array=True, out_stride=5)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_encode_large_batch_far_positions(cuda_device, dtype):
+    """Two-thread kernel at the top of its RoPE range: positions up to
+    2^22 - 1, where pos * theta_0 needs the widest reduction by 2 pi."""
+    n = 16384 + 259
+    _run_encode(128, 2, n, dtype, rope=True, seed=240, offset=(1 << 22) - n, max_pos=1 << 22)
+
+
+def test_encode_large_batch_positions_past_reduction_range(cuda_device):
+    """A handle whose positions may pass 2^22 takes the table-driven kernel."""
+    n = 16384 + 3
+    _run_encode(128, 3, n, torch.bfloat16, rope=True, seed=241, offset=(1 << 22) + 100,
+                max_pos=(1 << 22) + 100 + n)
 
 
 def test_encode_large_batch_positions_array_strided(cuda_device):

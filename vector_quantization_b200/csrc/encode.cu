@@ -42,6 +42,7 @@ struct EncodeParams {
   float dsg[128];
   float tpos[4];        // thresholds above 0, ascending (2^(b-1) - 1 of them)
   float lpos[4];        // levels above 0, ascending (2^(b-1) of them)
+  float2 theta[64];     // two-thread kernel: RoPE frequency i as (hi, lo) float pieces
 };
 
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
@@ -764,27 +765,57 @@ __global__ void __launch_bounds__(kRowThreads, 1) encode_rows_kernel(EncodeParam
 // ===========================================================================
 constexpr int kPairThreads = 256;
 
+// 2 pi = 6 + kC2 + kC3 (kC2 + kC3 within about 1e-17 of 2 pi - 6): with
+// k < 2^22, k * 6 is exact and the three-term reduction of a RoPE angle
+// (Cody and Waite's method) keeps its error near 2^-22.
+constexpr double kTwoPiMinus6 = 0.28318530717958647692528676655900576839433879875021;
+constexpr float kC2 = static_cast<float>(kTwoPiMinus6);
+constexpr float kC3 = static_cast<float>(kTwoPiMinus6 - static_cast<double>(kC2));
+constexpr float kInvTwoPi = 0.15915494309189533577f;
+// Largest RoPE position the two-thread kernel takes: positions are exact as
+// float and k = rint(angle / 2 pi) < 2^22 for every frequency (theta <= 1).
+constexpr int64_t kPairsMaxRopePos = int64_t(1) << 22;
+
 template <int BITS, typename T>
-__global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodeParams p) {
-  constexpr int D = 128, NJ = 4;
+__global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                      EncodeParams p) {
+  constexpr int D = 128;
   constexpr int OPB = kTileVec * D * 2;           // bytes of one bf16 [128 x D] operand
   constexpr int SB = D * D * 2;                   // bytes of S [m x d] bf16
+  constexpr int kBoxCols = 128 / static_cast<int>(sizeof(T));   // one 128-byte swizzled box column
+  constexpr int kBoxes = D / kBoxCols;                            // 2 (bf16) or 4 (fp32)
+  constexpr uint32_t kXBytes = kTileVec * D * sizeof(T);         // one input tile: 32 or 64 KB
   extern __shared__ uint8_t raw[];
-  __shared__ uint64_t mbar;
+  __shared__ uint64_t mbar, mbar_x;
   __shared__ uint32_t tmem_slot;
+  __shared__ int s_fail;   // a bounded wait ran out: every later tile is marked, none waits
   __shared__ __align__(16) float dsg_s[D];
+  __shared__ __align__(16) float2 th_s[D / 2];
   uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
   uint8_t* s_op = base;
   uint8_t* r_hi = base + SB;
   uint8_t* r_lo = r_hi + OPB;
-
+  uint8_t* xs = r_hi;   // input tile (TMA, 128-byte swizzle), staged where the residual operand goes
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = lane >> 4;                                            // half of the vector
   const int t = 32 * (warp & 3) + 16 * (warp >> 2) + (lane & 15);    // row in the tile
+  const int64_t n_tiles = (p.n + kTileVec - 1) / kTileVec;
+  auto issue_x = [&](int64_t tl) {
+    tqtc::mbar_arrive_expect_tx(&mbar_x, kXBytes);
+#pragma unroll
+    for (int b = 0; b < kBoxes; ++b)
+      tqtc::tma_load_2d(xs + b * (kTileVec * 128), &xmap, b * kBoxCols, static_cast<int>(tl * kTileVec), &mbar_x);
+  };
   for (int c = tid; c < SB / 16; c += blockDim.x) tqdev::cp_async16(s_op + 16 * c, p.s_op + 8 * c, 16);
   tqdev::cp_async_commit();
   if (tid < D) dsg_s[tid] = p.dsg[tid];
-  if (tid == 0) tqtc::mbar_init(&mbar, 1);
+  if (tid < D / 2) th_s[tid] = p.theta[tid];
+  if (tid == 0) {
+    s_fail = 0;
+    tqtc::mbar_init(&mbar, 1);
+    tqtc::mbar_init(&mbar_x, 1);
+    if (blockIdx.x < n_tiles) issue_x(blockIdx.x);
+  }
   if (warp == 0) tqtc::tmem_alloc(&tmem_slot, D);
   tqdev::cp_async_wait<0>();
   tqtc::fence_before_sync();
@@ -796,72 +827,82 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodePar
   float tp[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) tp[k] = p.tpos[k];
-  const int64_t n_tiles = (p.n + kTileVec - 1) / kTileVec;
   const uint32_t rowbase = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
   const uint32_t vx = t & 7;
-  uint32_t phase = 0;
+  uint32_t phase = 0, phase_x = 0;
 
   for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
     const int64_t row = tile * kTileVec + t;
     bool valid = row < p.n;
-    {
-      // pull this row of the CTA's next tile toward L2 (thread h: the row's
-      // 128-byte line h for bf16) so its loads need not wait on DRAM
-      const int64_t nrow = row + static_cast<int64_t>(gridDim.x) * kTileVec;
-      if (nrow < p.n) {
-        const char* np = reinterpret_cast<const char*>(static_cast<const T*>(p.x) + nrow * p.ld) + h * 64 * sizeof(T);
-        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(np));
-      }
-    }
+    const bool failed = s_fail != 0;   // written before the previous iteration's last barrier
+    const bool ok_x = !failed && tqtc::mbar_wait(&mbar_x, phase_x, kWaitLimit);
+    phase_x ^= 1;
     float u[64];   // u[32 s + i] = coordinate 64 s + 32 h + i
-    float nrm = 0.f, rr = 0.f;
-    if (valid) {
-      const T* xr = static_cast<const T*>(p.x) + row * p.ld;
-      if constexpr (sizeof(T) == 2) {
+    // this thread's half row from the staged tile (rows past n are zero-filled)
+    if constexpr (sizeof(T) == 2) {
 #pragma unroll
-        for (int sh = 0; sh < 2; ++sh)
+      for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr) + 8 * sh + 4 * h + q);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        for (int q = 0; q < 4; ++q) {
+          const int j = 4 * h + q;   // 16-byte chunk of box sh (coordinates 64 sh ..)
+          const uint4 v = *reinterpret_cast<const uint4*>(xs + sh * (kTileVec * 128) + t * 128 + ((j ^ (t & 7)) << 4));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              u[32 * sh + 8 * q + 2 * e] = __uint_as_float(w[e] << 16);
-              u[32 * sh + 8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-            }
+          for (int e = 0; e < 4; ++e) {
+            u[32 * sh + 8 * q + 2 * e] = __uint_as_float(w[e] << 16);
+            u[32 * sh + 8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
           }
+        }
+    } else {
+#pragma unroll
+      for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int b = 2 * sh + h;   // box of coordinates 32 b ..
+          const float4 v = *reinterpret_cast<const float4*>(xs + b * (kTileVec * 128) + t * 128 + ((q ^ (t & 7)) << 4));
+          u[32 * sh + 4 * q] = v.x;
+          u[32 * sh + 4 * q + 1] = v.y;
+          u[32 * sh + 4 * q + 2] = v.z;
+          u[32 * sh + 4 * q + 3] = v.w;
+        }
+    }
+    __syncthreads();   // the tile is in registers: its buffer may take the residual
+    if (!ok_x) {
+      valid = false;
+      if (row < p.n && h == 0)
+        p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+    }
+    // ||x|| before RoPE (a rotation: the norm is unchanged by it)
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) ss = fmaf(u[e], u[e], ss);
+    if (valid && p.rope) {
+      const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
+      if (pos < 0 || pos >= p.rope_max_pos) {
+        valid = false;
+        if (h == 0) p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
       } else {
+        // pairs (u[i], u[32 + i]) turn by pos * theta_j, j = 32 h + i; the
+        // angle is pos theta_hi + pos theta_lo (error term of the first
+        // product by FMA), reduced by 2 pi in three terms, then sin / cos on
+        // [-pi, pi]
+        const float pf = static_cast<float>(pos);   // exact: pos < 2^22
 #pragma unroll
-        for (int sh = 0; sh < 2; ++sh)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(xr) + 16 * sh + 8 * h + q);
-            u[32 * sh + 4 * q] = v.x;
-            u[32 * sh + 4 * q + 1] = v.y;
-            u[32 * sh + 4 * q + 2] = v.z;
-            u[32 * sh + 4 * q + 3] = v.w;
-          }
-      }
-      if (p.rope) {
-        const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
-        if (pos < 0 || pos >= p.rope_max_pos) {
-          valid = false;
-          if (h == 0) p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-        } else {
-          // frequencies 32h + i of the pairs (u[i], u[32 + i])
-          const float4* hi = reinterpret_cast<const float4*>(p.rope_hi + (pos >> kRopeLoBits) * (D / 2)) + 16 * h;
-          const float4* lo = reinterpret_cast<const float4*>(p.rope_lo + (pos & (kRopeLoRows - 1)) * (D / 2)) + 16 * h;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float4 a = __ldg(hi + c), b = __ldg(lo + c);
-            const float c0 = a.x * b.x - a.y * b.y, s0 = a.y * b.x + a.x * b.y;
-            const float c1 = a.z * b.z - a.w * b.w, s1 = a.w * b.z + a.z * b.w;
-            const float x0 = u[2 * c], y0 = u[32 + 2 * c], x1 = u[2 * c + 1], y1 = u[33 + 2 * c];
-            u[2 * c] = x0 * c0 - y0 * s0;
-            u[32 + 2 * c] = y0 * c0 + x0 * s0;
-            u[2 * c + 1] = x1 * c1 - y1 * s1;
-            u[33 + 2 * c] = y1 * c1 + x1 * s1;
-          }
+        for (int i = 0; i < 32; ++i) {
+          if ((i & 7) == 0) asm volatile("" ::: "memory");   // bound the loads in flight (registers)
+          const float2 th = th_s[32 * h + i];
+          const float ah = pf * th.x;
+          const float al = fmaf(pf, th.y, fmaf(pf, th.x, -ah));
+          const float k = rintf(ah * kInvTwoPi);
+          float r = fmaf(-k, 6.0f, ah);
+          r = fmaf(-k, kC2, r);
+          r = fmaf(-k, kC3, r);
+          r += al;
+          float sn, cs;
+          __sincosf(r, &sn, &cs);
+          const float x0 = u[i], y0 = u[32 + i];
+          u[i] = x0 * cs - y0 * sn;
+          u[32 + i] = y0 * cs + x0 * sn;
         }
       }
     }
@@ -871,7 +912,6 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodePar
 #pragma unroll
       for (int e = 0; e < 64; ++e) u[e] = 0.f;
     }
-    float ss = 0.f;
 #pragma unroll
     for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
@@ -879,14 +919,10 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodePar
         const float4 dv = *reinterpret_cast<const float4*>(dsg_s + 64 * sh + 32 * h + 4 * q);
         const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float& x = u[32 * sh + 4 * q + e];
-          ss = fmaf(x, x, ss);
-          x *= dd[e];
-        }
+        for (int e = 0; e < 4; ++e) u[32 * sh + 4 * q + e] *= dd[e];
       }
     ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-    nrm = sqrtf(ss);
+    const float nrm = valid ? sqrtf(ss) : 0.f;
     fwht_regs<64>(u);                                   // coordinate bits 0-4 and 6
     const float sgn = h ? -1.f : 1.f;                   // coordinate bit 5: across the lane pair
 #pragma unroll
@@ -901,10 +937,11 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodePar
 #pragma unroll
     for (int k = 0; k < 4; ++k) nl[k] = nrm * p.lpos[k];
     uint32_t w0[BITS], w1[BITS];
-    rr = quantize32<BITS>(u, tp, nl, nrm, w0);          // coordinates 32h .. 32h + 31: word h
+    float rr = quantize32<BITS>(u, tp, nl, nrm, w0);    // coordinates 32h .. 32h + 31: word h
     rr += quantize32<BITS>(u + 32, tp, nl, nrm, w1);    // 64 + 32h ..: word 2 + h
     rr += __shfl_xor_sync(0xffffffffu, rr, 16);
     if (valid) {
+      constexpr int NJ = 4;
       uint32_t* crec = p.codes + row * p.out_stride * (BITS * NJ);   // 4-byte aligned records
 #pragma unroll
       for (int k = 0; k < BITS; ++k) {
@@ -938,7 +975,7 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodePar
     tqtc::fence_smem_to_async();
     tqtc::fence_before_sync();
     __syncthreads();
-    if (tid == 0) {
+    if (tid == 0 && !failed) {
       tqtc::fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
@@ -950,11 +987,15 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(EncodePar
                           tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, true);
       tqtc::mma_commit(&mbar);
     }
-    const bool ok = tqtc::mbar_wait(&mbar, phase, kWaitLimit);
+    const bool ok = !failed && ok_x && tqtc::mbar_wait(&mbar, phase, kWaitLimit);
     phase ^= 1;
     tqtc::fence_after_sync();
+    if (!ok) s_fail = 1;
+    // the products have read the residual: its buffer takes the next input tile
+    if (tid == 0 && ok && tile + gridDim.x < n_tiles) issue_x(tile + gridDim.x);
     // ---- sign bits: warp w reads lanes 32 (w % 4) + lane, columns 64 (w / 4) ..
     {
+      constexpr int NJ = 4;
       const int quad = warp & 3, part = warp >> 2;
       const int64_t srow = tile * kTileVec + quad * 32 + lane;
 #pragma unroll
@@ -1001,6 +1042,14 @@ constexpr int64_t kRowsKernelMinN = 16384;
 
 template <int BITS, typename T>
 int launch_encode_pairs(const EncodeParams& p, cudaStream_t stream) {
+  // Positions past 2^22 (the in-kernel angle reduction's range) or more rows
+  // than a TMA coordinate holds go to the table-driven one-thread kernel.
+  if ((p.rope && p.rope_max_pos > kPairsMaxRopePos) || p.n >= (int64_t(1) << 31))
+    return launch_encode_rows<128, BITS, T>(p, stream);
+  CUtensorMap xmap;
+  if (!tq::make_tmap_2d(&xmap, p.x, static_cast<int>(sizeof(T)), p.n, 128, p.ld, 128 / static_cast<int>(sizeof(T)),
+                        kTileVec))
+    return launch_encode_rows<128, BITS, T>(p, stream);
   const size_t smem = 128 * 128 * 2 + 2 * static_cast<size_t>(kTileVec) * 128 * 2 + 1024;   // 97 KB: 2 CTAs / SM
   auto kern = encode_pairs_kernel<BITS, T>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
@@ -1010,7 +1059,7 @@ int launch_encode_pairs(const EncodeParams& p, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = (p.n + kTileVec - 1) / kTileVec;
   const int blocks = static_cast<int>(tiles < 2LL * sms ? tiles : 2LL * sms);
-  kern<<<blocks, kPairThreads, smem, stream>>>(p);
+  kern<<<blocks, kPairThreads, smem, stream>>>(xmap, p);
   return tq::launch_status();
 }
 
@@ -1096,6 +1145,7 @@ extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, in
   p.rope_hi = h->d_rope_hi;
   p.rope_lo = h->d_rope_lo;
   p.rope_max_pos = h->rope_max_pos;
+  for (int i = 0; i < 64; ++i) p.theta[i] = make_float2(h->rope_th_hi[i], h->rope_th_lo[i]);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (h->d == 128)
     return dtype == TQ_F32 ? dispatch_bits<128, float>(h->bits, p, s) : dispatch_bits<128, __nv_bfloat16>(h->bits, p, s);

@@ -390,6 +390,10 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
     h->rope_hi_rows = static_cast<int>((rope_max_pos + kRopeLoRows - 1) / kRopeLoRows);
     std::vector<double> theta(half);
     for (int i = 0; i < half; ++i) theta[i] = std::pow(rope_base, -2.0 * i / d);
+    for (int i = 0; i < half && i < 64; ++i) {
+      h->rope_th_hi[i] = static_cast<float>(theta[i]);
+      h->rope_th_lo[i] = static_cast<float>(theta[i] - static_cast<double>(h->rope_th_hi[i]));
+    }
     std::vector<float2> hi(static_cast<size_t>(h->rope_hi_rows) * half), lo(static_cast<size_t>(kRopeLoRows) * half);
     for (int r = 0; r < h->rope_hi_rows; ++r)
       for (int i = 0; i < half; ++i) {

@@ -37,14 +37,6 @@ constexpr int kGWaitLimit = 1 << 24;
 constexpr int kATileBytes = kGM * kGK * 2;   // 16 KB
 constexpr int kBTileBytes = kGN * kGK * 2;   // 16 KB
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* mbar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
-          "r"(tqtc::smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(tqtc::smem_u32(mbar))
-      : "memory");
-}
-
 template <bool BLO>
 __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap mAh,
                                                          const __grid_constant__ CUtensorMap mAl,
@@ -85,10 +77,10 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
       if (!ok) break;
       uint8_t* st = stage_ptr(s);
       tqtc::mbar_arrive_expect_tx(&full[s], STAGE);
-      tma_load_2d(st, &mAh, kt * kGK, m0, &full[s]);
-      tma_load_2d(st + kATileBytes, &mAl, kt * kGK, m0, &full[s]);
-      tma_load_2d(st + 2 * kATileBytes, &mBh, kt * kGK, n0, &full[s]);
-      if constexpr (BLO) tma_load_2d(st + 2 * kATileBytes + kBTileBytes, &mBl, kt * kGK, n0, &full[s]);
+      tqtc::tma_load_2d(st, &mAh, kt * kGK, m0, &full[s]);
+      tqtc::tma_load_2d(st + kATileBytes, &mAl, kt * kGK, m0, &full[s]);
+      tqtc::tma_load_2d(st + 2 * kATileBytes, &mBh, kt * kGK, n0, &full[s]);
+      if constexpr (BLO) tqtc::tma_load_2d(st + 2 * kATileBytes + kBTileBytes, &mBl, kt * kGK, n0, &full[s]);
     }
     if (!ok) failed = 1;
   } else if (tid == 32) {
@@ -200,20 +192,26 @@ EncodeTiledFn encode_tiled() {
 // Tensor map of a row-major bf16 matrix [rows][cols] (ld elements per row)
 // read in boxes of 64 columns x box_rows rows with a 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
-  EncodeTiledFn fn = encode_tiled();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGK), static_cast<cuuint32_t>(box_rows)};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return tq::make_tmap_2d(map, ptr, 2, rows, cols, ld, kGK, box_rows);
 }
 
 }  // namespace
 
 namespace tq {
+
+bool make_tmap_2d(CUtensorMap* map, const void* ptr, int elem_bytes, int64_t rows, int64_t cols, int64_t ld,
+                  int box_cols, int box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn || (elem_bytes != 2 && elem_bytes != 4)) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * elem_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  return fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int split_bf16(const float* x, int64_t ldx, int64_t rows, int cols, uint16_t* hi, uint16_t* lo, int64_t ldo,
                cudaStream_t s) {

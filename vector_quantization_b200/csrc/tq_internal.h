@@ -1,6 +1,7 @@
 // Private declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -16,6 +17,9 @@ struct tq_rotation {
   double rope_base = 0.0;
   int64_t rope_max_pos = 0;
   int rope_hi_rows = 0;                 // rows of the coarse RoPE table
+  // RoPE frequencies theta_i = base^(-2i/d), i < d/2, as float hi + lo pieces
+  // (theta_i - hi - lo within about 2^-48 theta_i)
+  float rope_th_hi[64] = {}, rope_th_lo[64] = {};
 
   std::vector<double> levels;           // [2^bits] ascending
   std::vector<double> thresholds;       // [2^bits - 1]
@@ -65,6 +69,14 @@ inline int launch_status() {
 inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
+
+// Tensor map (2-D, 128-byte swizzle, zero fill past the edges) of a row-major
+// matrix [rows][cols] of bf16 (elem_bytes 2) or fp32 (4) elements with ld
+// elements per row, read in boxes of box_cols x box_rows; false when the
+// driver entry point is missing or the arguments break the TMA rules (base
+// 16-byte aligned, ld * elem_bytes a multiple of 16).
+bool make_tmap_2d(CUtensorMap* map, const void* ptr, int elem_bytes, int64_t rows, int64_t cols, int64_t ld,
+                  int box_cols, int box_rows);
 
 // fp32 -> bf16 hi + lo pieces of a row-major matrix (cols % 4 == 0).
 int split_bf16(const float* x, int64_t ldx, int64_t rows, int cols, uint16_t* hi, uint16_t* lo, int64_t ldo,
