@@ -753,15 +753,66 @@ __global__ void __launch_bounds__(kRowThreads, 1) encode_rows_kernel(EncodeParam
   if (warp == 0) tqtc::tmem_free(tmem_slot, 2 * D);
 }
 
+// Codes of the 32 coordinates held as y[m] = (c 2m, c 2m+1) (unit-vector
+// coordinates, never -0): as quantize32, with the residual and its square
+// sum formed two at a time (fp32x2).  Returns the sum of squared residuals.
+template <int BITS>
+__device__ __forceinline__ float quantize32_x2(float2* y, const float (&tp)[4], const float (&nl)[4], float norm,
+                                               uint32_t (&w)[BITS]) {
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) w[k] = 0;
+  const float2 norm2 = make_float2(norm, norm);
+  float2 rr = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int m = 15; m >= 0; --m) {
+    float c[2];
+#pragma unroll
+    for (int e = 1; e >= 0; --e) {
+      const float v = e ? y[m].y : y[m].x;
+      const uint32_t sy = __float_as_uint(v);
+      const float a = fabsf(v);
+      float nmag;
+      if constexpr (BITS == 1) {
+        w[0] = __funnelshift_l(sy, w[0], 1);
+        nmag = nl[0];
+      } else if constexpr (BITS == 2) {
+        const uint32_t s0 = __float_as_uint(a - tp[0]);
+        w[1] = __funnelshift_l(sy, w[1], 1);
+        w[0] = __funnelshift_l(sy ^ s0, w[0], 1);
+        nmag = a >= tp[0] ? nl[1] : nl[0];
+      } else {
+        const uint32_t s0 = __float_as_uint(a - tp[0]), s1 = __float_as_uint(a - tp[1]),
+                       s2 = __float_as_uint(a - tp[2]);
+        w[2] = __funnelshift_l(sy, w[2], 1);
+        w[1] = __funnelshift_l(sy ^ s1, w[1], 1);
+        w[0] = __funnelshift_l(sy ^ s0 ^ s1 ^ s2, w[0], 1);
+        nmag = a >= tp[2] ? nl[3] : (a >= tp[1] ? nl[2] : (a >= tp[0] ? nl[1] : nl[0]));
+      }
+      c[e] = -copysignf(nmag, v);
+    }
+    const float2 r = __ffma2_rn(norm2, y[m], make_float2(c[0], c[1]));
+    y[m] = r;
+    rr = __ffma2_rn(r, r, rr);
+  }
+#pragma unroll
+  for (int k = 0; k < BITS; ++k) w[k] = ~w[k];
+  return rr.x + rr.y;
+}
+
 // ===========================================================================
 // Two threads per vector (d = 128): thread h of a pair (lanes l and l ^ 16)
 // holds the coordinates whose bit 5 equals h, {32h + i, 64 + 32h + i : i < 32},
-// so RoPE pairs (i, i + 64) and six of the seven Walsh-Hadamard stages stay in
-// the thread and one stage (bit 5) crosses lanes; each thread assembles two
-// whole plane words (coordinates 32h.., 64 + 32h..).  A CTA of 8 warps owns
-// one 128-row tile at a time; with half the registers of the one-thread
-// kernel two CTAs share an SM, so one CTA's tensor-core product and read-back
-// overlap the other's per-vector work.
+// as 32 fp32 pairs v[16 s + m] = (64 s + 32 h + 2m, + 1), so RoPE pairs
+// (i, i + 64) and six of the seven Walsh-Hadamard stages stay in the thread
+// and one stage (bit 5) crosses lanes; each thread assembles two whole plane
+// words (coordinates 32h.., 64 + 32h..).  The elementwise arithmetic runs on
+// fp32x2 instructions (two coordinates, or two RoPE frequencies, per
+// instruction) except the butterfly inside a pair.  A CTA of 8 warps owns one
+// 128-row tile at a time; the tile arrives by 2-D TMA (128-byte swizzle) one
+// tile ahead, into the residual operand's buffer, which the previous tile's
+// tensor-core product has finished reading.  With half the registers of the
+// one-thread kernel two CTAs share an SM, so one CTA's tensor-core product
+// and read-back overlap the other's per-vector work.
 // ===========================================================================
 constexpr int kPairThreads = 256;
 
@@ -789,8 +840,9 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
   __shared__ uint64_t mbar, mbar_x;
   __shared__ uint32_t tmem_slot;
   __shared__ int s_fail;   // a bounded wait ran out: every later tile is marked, none waits
-  __shared__ __align__(16) float dsg_s[D];
-  __shared__ __align__(16) float2 th_s[D / 2];
+  __shared__ __align__(16) float2 dsg_s[D / 2];   // sign diagonal, coordinate pairs
+  __shared__ __align__(16) float2 thh_s[D / 4];   // RoPE theta hi pieces, frequency pairs
+  __shared__ __align__(16) float2 thl_s[D / 4];   // and lo pieces
   uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
   uint8_t* s_op = base;
   uint8_t* r_hi = base + SB;
@@ -808,8 +860,11 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
   };
   for (int c = tid; c < SB / 16; c += blockDim.x) tqdev::cp_async16(s_op + 16 * c, p.s_op + 8 * c, 16);
   tqdev::cp_async_commit();
-  if (tid < D) dsg_s[tid] = p.dsg[tid];
-  if (tid < D / 2) th_s[tid] = p.theta[tid];
+  if (tid < D / 2) dsg_s[tid] = make_float2(p.dsg[2 * tid], p.dsg[2 * tid + 1]);
+  if (tid < D / 4) {
+    thh_s[tid] = make_float2(p.theta[2 * tid].x, p.theta[2 * tid + 1].x);
+    thl_s[tid] = make_float2(p.theta[2 * tid].y, p.theta[2 * tid + 1].y);
+  }
   if (tid == 0) {
     s_fail = 0;
     tqtc::mbar_init(&mbar, 1);
@@ -824,6 +879,7 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
   const uint32_t tmem = tmem_slot;
   const uint32_t idesc = tqtc::idesc_bf16_f32(kTileVec, D);
   const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  const float2 m1 = make_float2(-1.f, -1.f);
   float tp[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) tp[k] = p.tpos[k];
@@ -837,7 +893,7 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
     const bool failed = s_fail != 0;   // written before the previous iteration's last barrier
     const bool ok_x = !failed && tqtc::mbar_wait(&mbar_x, phase_x, kWaitLimit);
     phase_x ^= 1;
-    float u[64];   // u[32 s + i] = coordinate 64 s + 32 h + i
+    float2 v[32];   // v[16 s + m] = coordinates (64 s + 32 h + 2m, + 1)
     // this thread's half row from the staged tile (rows past n are zero-filled)
     if constexpr (sizeof(T) == 2) {
 #pragma unroll
@@ -845,13 +901,11 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int j = 4 * h + q;   // 16-byte chunk of box sh (coordinates 64 sh ..)
-          const uint4 v = *reinterpret_cast<const uint4*>(xs + sh * (kTileVec * 128) + t * 128 + ((j ^ (t & 7)) << 4));
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          const uint4 w4 = *reinterpret_cast<const uint4*>(xs + sh * (kTileVec * 128) + t * 128 + ((j ^ (t & 7)) << 4));
+          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            u[32 * sh + 8 * q + 2 * e] = __uint_as_float(w[e] << 16);
-            u[32 * sh + 8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-          }
+          for (int e = 0; e < 4; ++e)
+            v[16 * sh + 4 * q + e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
         }
     } else {
 #pragma unroll
@@ -859,11 +913,9 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const int b = 2 * sh + h;   // box of coordinates 32 b ..
-          const float4 v = *reinterpret_cast<const float4*>(xs + b * (kTileVec * 128) + t * 128 + ((q ^ (t & 7)) << 4));
-          u[32 * sh + 4 * q] = v.x;
-          u[32 * sh + 4 * q + 1] = v.y;
-          u[32 * sh + 4 * q + 2] = v.z;
-          u[32 * sh + 4 * q + 3] = v.w;
+          const float4 f = *reinterpret_cast<const float4*>(xs + b * (kTileVec * 128) + t * 128 + ((q ^ (t & 7)) << 4));
+          v[16 * sh + 2 * q] = make_float2(f.x, f.y);
+          v[16 * sh + 2 * q + 1] = make_float2(f.z, f.w);
         }
     }
     __syncthreads();   // the tile is in registers: its buffer may take the residual
@@ -873,36 +925,47 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
         p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
     }
     // ||x|| before RoPE (a rotation: the norm is unchanged by it)
-    float ss = 0.f;
+    float ss;
+    {
+      float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int e = 0; e < 64; ++e) ss = fmaf(u[e], u[e], ss);
+      for (int m = 0; m < 32; ++m) a2 = __ffma2_rn(v[m], v[m], a2);
+      ss = a2.x + a2.y;
+    }
     if (valid && p.rope) {
       const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
       if (pos < 0 || pos >= p.rope_max_pos) {
         valid = false;
         if (h == 0) p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
       } else {
-        // pairs (u[i], u[32 + i]) turn by pos * theta_j, j = 32 h + i; the
-        // angle is pos theta_hi + pos theta_lo (error term of the first
-        // product by FMA), reduced by 2 pi in three terms, then sin / cos on
-        // [-pi, pi]
+        // pairs (v[m], v[16 + m]) turn by pos * theta_j, j = 32 h + 2m (+1);
+        // the angle is pos theta_hi + pos theta_lo (error term of the first
+        // product by FMA), reduced by 2 pi in three terms (with k negated:
+        // rint is odd), then sin / cos on [-pi, pi]
         const float pf = static_cast<float>(pos);   // exact: pos < 2^22
+        const float2 pf2 = make_float2(pf, pf), npf2 = make_float2(-pf, -pf);
+        const float2 q2c = make_float2(-kInvTwoPi, -kInvTwoPi), six2 = make_float2(6.f, 6.f);
+        const float2 c2c = make_float2(kC2, kC2), c3c = make_float2(kC3, kC3);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if ((i & 7) == 0) asm volatile("" ::: "memory");   // bound the loads in flight (registers)
-          const float2 th = th_s[32 * h + i];
-          const float ah = pf * th.x;
-          const float al = fmaf(pf, th.y, fmaf(pf, th.x, -ah));
-          const float k = rintf(ah * kInvTwoPi);
-          float r = fmaf(-k, 6.0f, ah);
-          r = fmaf(-k, kC2, r);
-          r = fmaf(-k, kC3, r);
-          r += al;
-          float sn, cs;
-          __sincosf(r, &sn, &cs);
-          const float x0 = u[i], y0 = u[32 + i];
-          u[i] = x0 * cs - y0 * sn;
-          u[32 + i] = y0 * cs + x0 * sn;
+        for (int m = 0; m < 16; ++m) {
+          if ((m & 3) == 0) asm volatile("" ::: "memory");   // bound the loads in flight (registers)
+          const float2 thh = thh_s[16 * h + m], thl = thl_s[16 * h + m];
+          const float2 ah = __fmul2_rn(pf2, thh);
+          const float2 e = __ffma2_rn(npf2, thh, ah);        // -(pf theta_hi - ah), exact
+          const float2 nal = __ffma2_rn(npf2, thl, e);       // -(low part of the angle)
+          const float2 q = __fmul2_rn(ah, q2c);
+          const float2 kn = make_float2(rintf(q.x), rintf(q.y));   // -k
+          float2 r = __ffma2_rn(kn, six2, ah);
+          r = __ffma2_rn(kn, c2c, r);
+          r = __ffma2_rn(kn, c3c, r);
+          r = __ffma2_rn(nal, m1, r);
+          float s0, c0, s1, c1;
+          __sincosf(r.x, &s0, &c0);
+          __sincosf(r.y, &s1, &c1);
+          const float2 sn = make_float2(s0, s1), cs = make_float2(c0, c1);
+          const float2 x = v[m], y = v[16 + m];
+          v[m] = __ffma2_rn(y, __fmul2_rn(sn, m1), __fmul2_rn(x, cs));   // x cos - y sin
+          v[16 + m] = __ffma2_rn(x, sn, __fmul2_rn(y, cs));              // y cos + x sin
         }
       }
     }
@@ -910,35 +973,50 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
     // that are absent or out of RoPE range carry zeros and store nothing
     if (!valid) {
 #pragma unroll
-      for (int e = 0; e < 64; ++e) u[e] = 0.f;
+      for (int m = 0; m < 32; ++m) v[m] = make_float2(0.f, 0.f);
     }
+    // D x, then the Walsh-Hadamard stages on coordinate bits 0-4 and 6
 #pragma unroll
     for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 dv = *reinterpret_cast<const float4*>(dsg_s + 64 * sh + 32 * h + 4 * q);
-        const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
+      for (int m = 0; m < 16; ++m) v[16 * sh + m] = __fmul2_rn(v[16 * sh + m], dsg_s[32 * sh + 16 * h + m]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) u[32 * sh + 4 * q + e] *= dd[e];
-      }
+    for (int m = 0; m < 32; ++m) {   // bit 0: inside a pair
+      const float a = v[m].x, b = v[m].y;
+      v[m] = make_float2(a + b, a - b);
+    }
+#pragma unroll
+    for (int hb = 1; hb < 32; hb <<= 1)   // bits 1-4 and 6 (pair index bits 0-4)
+#pragma unroll
+      for (int m = 0; m < 32; ++m)
+        if (!(m & hb)) {
+          const float2 a = v[m], b = v[m | hb];
+          v[m] = __fadd2_rn(a, b);
+          v[m | hb] = __ffma2_rn(b, m1, a);
+        }
     ss += __shfl_xor_sync(0xffffffffu, ss, 16);
     const float nrm = valid ? sqrtf(ss) : 0.f;
-    fwht_regs<64>(u);                                   // coordinate bits 0-4 and 6
-    const float sgn = h ? -1.f : 1.f;                   // coordinate bit 5: across the lane pair
+    {
+      const float sgn = h ? -1.f : 1.f;                 // coordinate bit 5: across the lane pair
+      const float2 sgn2 = make_float2(sgn, sgn);
 #pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      const float o = __shfl_xor_sync(0xffffffffu, u[e], 16);
-      u[e] = fmaf(sgn, u[e], o);
+      for (int m = 0; m < 32; ++m) {
+        const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[m].x, 16), __shfl_xor_sync(0xffffffffu, v[m].y, 16));
+        v[m] = __ffma2_rn(sgn2, v[m], o);
+      }
     }
-    const float scale = (nrm > 0.f ? 1.0f / nrm : 0.f) * inv_sqrt_d;
+    {
+      const float scale = (nrm > 0.f ? 1.0f / nrm : 0.f) * inv_sqrt_d;
+      const float2 sc2 = make_float2(scale, scale), z2 = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int e = 0; e < 64; ++e) u[e] = fmaf(u[e], scale, 0.f);   // unit-vector coordinates, -0 -> +0
+      for (int m = 0; m < 32; ++m) v[m] = __ffma2_rn(v[m], sc2, z2);   // unit-vector coordinates, -0 -> +0
+    }
     float nl[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) nl[k] = nrm * p.lpos[k];
     uint32_t w0[BITS], w1[BITS];
-    float rr = quantize32<BITS>(u, tp, nl, nrm, w0);    // coordinates 32h .. 32h + 31: word h
-    rr += quantize32<BITS>(u + 32, tp, nl, nrm, w1);    // 64 + 32h ..: word 2 + h
+    float rr = quantize32_x2<BITS>(v, tp, nl, nrm, w0);        // coordinates 32h .. 32h + 31: word h
+    rr += quantize32_x2<BITS>(v + 16, tp, nl, nrm, w1);        // 64 + 32h ..: word 2 + h
     rr += __shfl_xor_sync(0xffffffffu, rr, 16);
     if (valid) {
       constexpr int NJ = 4;
@@ -950,7 +1028,8 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
       }
       if (h == 0) p.norms[row * p.out_stride] = make_float2(nrm, sqrtf(rr));
     }
-    // residual as bf16 hi + lo into row t of the A operand (16-byte chunks)
+    // residual (zero on absent rows) as bf16 hi + lo into row t of the A
+    // operand (16-byte chunks)
 #pragma unroll
     for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
@@ -958,11 +1037,12 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
         uint32_t hv[4], lv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = valid ? u[32 * sh + 8 * q + 2 * e] : 0.f, b = valid ? u[32 * sh + 8 * q + 2 * e + 1] : 0.f;
-          __nv_bfloat162 hb = __floats2bfloat162_rn(a, b);
-          const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb);
-          __nv_bfloat162 lb =
-              __floats2bfloat162_rn(a - __uint_as_float(hbits << 16), b - __uint_as_float(hbits & 0xFFFF0000u));
+          const float2 r = v[16 * sh + 4 * q + e];
+          __nv_bfloat162 hb2 = __floats2bfloat162_rn(r.x, r.y);
+          const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb2);
+          const float2 lo = __ffma2_rn(make_float2(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u)),
+                                       m1, r);
+          __nv_bfloat162 lb = __floats2bfloat162_rn(lo.x, lo.y);
           hv[e] = hbits;
           lv[e] = *reinterpret_cast<uint32_t*>(&lb);
         }
@@ -994,6 +1074,9 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
     // the products have read the residual: its buffer takes the next input tile
     if (tid == 0 && ok && tile + gridDim.x < n_tiles) issue_x(tile + gridDim.x);
     // ---- sign bits: warp w reads lanes 32 (w % 4) + lane, columns 64 (w / 4) ..
+    // Each bit is the complemented fp32 sign bit, shifted in by one funnel
+    // shift: 1 for +0 and positive projections, 0 for negative ones and -0
+    // (an exact zero projection is within any sign tolerance).
     {
       constexpr int NJ = 4;
       const int quad = warp & 3, part = warp >> 2;
@@ -1004,8 +1087,8 @@ __global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __g
         tqtc::tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 64 * part + 32 * c, val);
         uint32_t w = 0;
 #pragma unroll
-        for (int b = 31; b >= 0; --b) w = (w << 1) | (val[b] >= 0.f ? 1u : 0u);
-        if (srow < p.n) p.signs[srow * p.out_stride * NJ + 2 * part + c] = ok ? w : 0u;
+        for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[b]), w, 1);
+        if (srow < p.n) p.signs[srow * p.out_stride * NJ + 2 * part + c] = ok ? ~w : 0u;
       }
       if (!ok && part == 0 && srow < p.n)
         p.norms[srow * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
