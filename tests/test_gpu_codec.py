@@ -89,6 +89,14 @@ def test_encode_small_batch_positions_array_strided(cuda_device):
     _run_encode(128, 3, 128, torch.bfloat16, rope=True, seed=230, offset=77, pos_array=True, out_stride=5)
 
 
+@pytest.mark.parametrize("bits", [1, 2, 3])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_encode_parity_large_batch_no_rope(cuda_device, bits, dtype):
+    """Large batches without RoPE: bf16 rows go to the tensor core as they
+    are staged, fp32 rows through the fp16 hi/lo split."""
+    _run_encode(128, bits, 2 * 16384 + 389, dtype, rope=False, seed=250 + bits)
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_encode_large_batch_far_positions(cuda_device, dtype):
     """Two-thread kernel at the top of its RoPE range: positions up to

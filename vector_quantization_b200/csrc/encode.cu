@@ -30,6 +30,7 @@ struct EncodeParams {
   int64_t out_stride;
   const float* dsigns;  // [D]
   const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
+  const uint16_t* hd_op; // tensor-core encode: H D in the same layout (fp16 bits when split, else bf16)
   const float* st;      // S transposed, fp32: st[k * d + j] = S[j][k]
   int rows;             // warp-per-vector kernel: vectors per tile, R in {8, 16, ..., 128}
   const float* thresholds;
@@ -42,7 +43,7 @@ struct EncodeParams {
   float dsg[128];
   float tpos[4];        // thresholds above 0, ascending (2^(b-1) - 1 of them)
   float lpos[4];        // levels above 0, ascending (2^(b-1) of them)
-  float2 theta[64];     // two-thread kernel: RoPE frequency i as (hi, lo) float pieces
+  float2 theta[64];     // tensor-core encode: RoPE frequency i as (hi, lo) float pieces
 };
 
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
@@ -799,23 +800,6 @@ __device__ __forceinline__ float quantize32_x2(float2* y, const float (&tp)[4], 
   return rr.x + rr.y;
 }
 
-// ===========================================================================
-// Two threads per vector (d = 128): thread h of a pair (lanes l and l ^ 16)
-// holds the coordinates whose bit 5 equals h, {32h + i, 64 + 32h + i : i < 32},
-// as 32 fp32 pairs v[16 s + m] = (64 s + 32 h + 2m, + 1), so RoPE pairs
-// (i, i + 64) and six of the seven Walsh-Hadamard stages stay in the thread
-// and one stage (bit 5) crosses lanes; each thread assembles two whole plane
-// words (coordinates 32h.., 64 + 32h..).  The elementwise arithmetic runs on
-// fp32x2 instructions (two coordinates, or two RoPE frequencies, per
-// instruction) except the butterfly inside a pair.  A CTA of 8 warps owns one
-// 128-row tile at a time; the tile arrives by 2-D TMA (128-byte swizzle) one
-// tile ahead, into the residual operand's buffer, which the previous tile's
-// tensor-core product has finished reading.  With half the registers of the
-// one-thread kernel two CTAs share an SM, so one CTA's tensor-core product
-// and read-back overlap the other's per-vector work.
-// ===========================================================================
-constexpr int kPairThreads = 256;
-
 // 2 pi = 6 + kC2 + kC3 (kC2 + kC3 within about 1e-17 of 2 pi - 6): with
 // k < 2^22, k * 6 is exact and the three-term reduction of a RoPE angle
 // (Cody and Waite's method) keeps its error near 2^-22.
@@ -823,282 +807,371 @@ constexpr double kTwoPiMinus6 = 0.2831853071795864769252867665590057683943387987
 constexpr float kC2 = static_cast<float>(kTwoPiMinus6);
 constexpr float kC3 = static_cast<float>(kTwoPiMinus6 - static_cast<double>(kC2));
 constexpr float kInvTwoPi = 0.15915494309189533577f;
-// Largest RoPE position the two-thread kernel takes: positions are exact as
+// Largest RoPE position the tensor-core encode takes: positions are exact as
 // float and k = rint(angle / 2 pi) < 2^22 for every frequency (theta <= 1).
 constexpr int64_t kPairsMaxRopePos = int64_t(1) << 22;
 
-template <int BITS, typename T>
-__global__ void __launch_bounds__(kPairThreads, 2) encode_pairs_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                                      EncodeParams p) {
+// ===========================================================================
+// Rotation on the tensor core (d = 128, large batches).  y = H D x is a
+// dense 128 x 128 contraction with exact +-1 entries, so each 128-row tile
+// is rotated by tcgen05 MMAs against H D resident in shared memory, and the
+// CUDA cores keep only RoPE, the codes, the residual and the sign bits.
+//
+// One CTA per SM runs two groups of 8 warps; each group owns a tile at a
+// time (its own staging / operand buffers, tensor-memory columns, mbarriers
+// and named barrier), so one group's tensor-core work and waits overlap the
+// other's CUDA-core work.  S and H D are shared.  Per tile:
+//  1. the input tile arrives by 2-D TMA (128-byte swizzle) into the group's
+//     operand buffer, requested one tile ahead;
+//  2. SPLIT (RoPE or fp32 input): thread pairs (row t, half h) load the row,
+//     take ||x|| (before RoPE: a rotation keeps it), apply RoPE, scale by a
+//     power of two near 1 / ||x|| and write fp16 hi + lo pieces (22 bits;
+//     bf16 pieces, 2^-17, would move ||r|| by up to ~8e-6 ||x||) as the A
+//     operand; otherwise (bf16 without RoPE) the staged tile is the A
+//     operand as it stands (against bf16 H D, exact products);
+//  3. y = A (H D)^T into tensor memory (fp32);
+//  4. thread pairs (TMEM lane = row, column half) read y, form the unit
+//     coordinates y / (||x|| sqrt d), the codes and the residual (fp32x2),
+//     and write the residual as bf16 hi + lo over the A operand;
+//  5. S r into the same tensor-memory columns; the sign bits are read back.
+// ===========================================================================
+constexpr int kTcThreads = 512;   // two groups of 8 warps
+
+template <int BITS, typename T, bool SPLIT>
+__global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                 EncodeParams p) {
+  static_assert(SPLIT || sizeof(T) == 2, "fp32 input needs the split path");
   constexpr int D = 128;
-  constexpr int OPB = kTileVec * D * 2;           // bytes of one bf16 [128 x D] operand
-  constexpr int SB = D * D * 2;                   // bytes of S [m x d] bf16
-  constexpr int kBoxCols = 128 / static_cast<int>(sizeof(T));   // one 128-byte swizzled box column
-  constexpr int kBoxes = D / kBoxCols;                            // 2 (bf16) or 4 (fp32)
-  constexpr uint32_t kXBytes = kTileVec * D * sizeof(T);         // one input tile: 32 or 64 KB
+  constexpr int OPB = kTileVec * D * 2;           // 32 KB: one 16-bit [128 x 128] operand
+  constexpr int kBoxCols = 128 / static_cast<int>(sizeof(T));
+  constexpr int kBoxes = D / kBoxCols;
+  constexpr uint32_t kXBytes = kTileVec * D * sizeof(T);
   extern __shared__ uint8_t raw[];
-  __shared__ uint64_t mbar, mbar_x;
+  __shared__ uint64_t mb_x[2], mb_y[2], mb_s[2];
   __shared__ uint32_t tmem_slot;
-  __shared__ int s_fail;   // a bounded wait ran out: every later tile is marked, none waits
-  __shared__ __align__(16) float2 dsg_s[D / 2];   // sign diagonal, coordinate pairs
-  __shared__ __align__(16) float2 thh_s[D / 4];   // RoPE theta hi pieces, frequency pairs
-  __shared__ __align__(16) float2 thl_s[D / 4];   // and lo pieces
+  __shared__ int s_fail[2];
+  __shared__ __align__(16) float2 thh_s[D / 4];
+  __shared__ __align__(16) float2 thl_s[D / 4];
+  __shared__ float xnrm[2][2][kTileVec];          // per group: ||x|| (SPLIT) or partial sums of squares
+  __shared__ float xrr[2][2][kTileVec];           // per group: partial sums of squared residuals
   uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
   uint8_t* s_op = base;
-  uint8_t* r_hi = base + SB;
-  uint8_t* r_lo = r_hi + OPB;
-  uint8_t* xs = r_hi;   // input tile (TMA, 128-byte swizzle), staged where the residual operand goes
+  uint8_t* hd_op = base + OPB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = lane >> 4;                                            // half of the vector
-  const int t = 32 * (warp & 3) + 16 * (warp >> 2) + (lane & 15);    // row in the tile
+  const int g = warp >> 3, gw = warp & 7, gt = tid & 255;
+  uint8_t* a_hi = base + 2 * OPB + g * 2 * OPB;
+  uint8_t* a_lo = a_hi + OPB;
+  uint8_t* xs = a_hi;   // staged input tile (bf16: a_hi; fp32: a_hi and a_lo)
   const int64_t n_tiles = (p.n + kTileVec - 1) / kTileVec;
+  const int64_t tstep = 2 * static_cast<int64_t>(gridDim.x);
+  auto gsync = [&]() { asm volatile("bar.sync %0, 256;\n" ::"r"(1 + g) : "memory"); };
   auto issue_x = [&](int64_t tl) {
-    tqtc::mbar_arrive_expect_tx(&mbar_x, kXBytes);
+    tqtc::mbar_arrive_expect_tx(&mb_x[g], kXBytes);
 #pragma unroll
     for (int b = 0; b < kBoxes; ++b)
-      tqtc::tma_load_2d(xs + b * (kTileVec * 128), &xmap, b * kBoxCols, static_cast<int>(tl * kTileVec), &mbar_x);
+      tqtc::tma_load_2d(xs + b * (kTileVec * 128), &xmap, b * kBoxCols, static_cast<int>(tl * kTileVec), &mb_x[g]);
   };
-  for (int c = tid; c < SB / 16; c += blockDim.x) tqdev::cp_async16(s_op + 16 * c, p.s_op + 8 * c, 16);
+  for (int c = tid; c < 2 * OPB / 16; c += blockDim.x)
+    tqdev::cp_async16(base + 16 * c, c < OPB / 16 ? p.s_op + 8 * c : p.hd_op + 8 * (c - OPB / 16), 16);
   tqdev::cp_async_commit();
-  if (tid < D / 2) dsg_s[tid] = make_float2(p.dsg[2 * tid], p.dsg[2 * tid + 1]);
   if (tid < D / 4) {
     thh_s[tid] = make_float2(p.theta[2 * tid].x, p.theta[2 * tid + 1].x);
     thl_s[tid] = make_float2(p.theta[2 * tid].y, p.theta[2 * tid + 1].y);
   }
   if (tid == 0) {
-    s_fail = 0;
-    tqtc::mbar_init(&mbar, 1);
-    tqtc::mbar_init(&mbar_x, 1);
-    if (blockIdx.x < n_tiles) issue_x(blockIdx.x);
+    s_fail[0] = s_fail[1] = 0;
+    for (int i = 0; i < 2; ++i) {
+      tqtc::mbar_init(&mb_x[i], 1);
+      tqtc::mbar_init(&mb_y[i], 1);
+      tqtc::mbar_init(&mb_s[i], 1);
+    }
   }
-  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, D);
+  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, 256);
   tqdev::cp_async_wait<0>();
+  tqtc::fence_smem_to_async();
   tqtc::fence_before_sync();
   __syncthreads();
   tqtc::fence_after_sync();
-  const uint32_t tmem = tmem_slot;
-  const uint32_t idesc = tqtc::idesc_bf16_f32(kTileVec, D);
+  int64_t tile = 2 * static_cast<int64_t>(blockIdx.x) + g;
+  if (gt == 0 && tile < n_tiles) issue_x(tile);
+  const uint32_t tm = tmem_slot + 128 * g;                  // y, then S r: 128 columns per group
+  const uint32_t tm_lane = static_cast<uint32_t>(32 * (gw & 3)) << 16;
+  constexpr uint32_t idy = SPLIT ? tqtc::idesc_f16_f32(kTileVec, D) : tqtc::idesc_bf16_f32(kTileVec, D);
+  constexpr uint32_t ids = tqtc::idesc_bf16_f32(kTileVec, D);
   const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
   const float2 m1 = make_float2(-1.f, -1.f);
   float tp[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) tp[k] = p.tpos[k];
-  const uint32_t rowbase = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
-  const uint32_t vx = t & 7;
-  uint32_t phase = 0, phase_x = 0;
+  // phase-2 mapping (SPLIT): row t2 of the tile, coordinates {32 h2 + i, 64 + 32 h2 + i}
+  const int t2 = 32 * (gw & 3) + 16 * (gw >> 2) + (lane & 15), h2 = lane >> 4;
+  const uint32_t rowbase2 = static_cast<uint32_t>((t2 >> 3) * 1024 + (t2 & 7) * 128);
+  // phase-4 mapping: row r4 = tensor-memory lane, coordinates 64 c4 .. 64 c4 + 63
+  const int r4 = 32 * (gw & 3) + lane, c4 = gw >> 2;
+  const uint32_t rowbase4 = static_cast<uint32_t>((r4 >> 3) * 1024 + (r4 & 7) * 128);
+  uint32_t ph_x = 0, ph_y = 0, ph_s = 0;
+  const float qnan = __int_as_float(0x7fc00000);
 
-  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    const int64_t row = tile * kTileVec + t;
-    bool valid = row < p.n;
-    const bool failed = s_fail != 0;   // written before the previous iteration's last barrier
-    const bool ok_x = !failed && tqtc::mbar_wait(&mbar_x, phase_x, kWaitLimit);
-    phase_x ^= 1;
-    float2 v[32];   // v[16 s + m] = coordinates (64 s + 32 h + 2m, + 1)
-    // this thread's half row from the staged tile (rows past n are zero-filled)
-    if constexpr (sizeof(T) == 2) {
+  for (; tile < n_tiles; tile += tstep) {
+    const bool failed = s_fail[g] != 0;   // written before the previous iteration's last barrier
+    const bool ok_x = !failed && tqtc::mbar_wait(&mb_x[g], ph_x, kWaitLimit);
+    ph_x ^= 1;
+    if constexpr (SPLIT) {
+      // ---- 2. row t2 into registers, ||x||, RoPE, fp16 hi + lo A operand
+      const int64_t row = tile * kTileVec + t2;
+      bool valid = row < p.n && ok_x;
+      float2 v[32];   // v[16 s + m] = coordinates (64 s + 32 h2 + 2m, + 1)
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int j = 4 * h2 + q;
+            const uint4 w4 = *reinterpret_cast<const uint4*>(xs + sh * (kTileVec * 128) + t2 * 128 + ((j ^ (t2 & 7)) << 4));
+            const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              v[16 * sh + 4 * q + e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+          }
+      } else {
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int b = 2 * sh + h2;
+            const float4 f = *reinterpret_cast<const float4*>(xs + b * (kTileVec * 128) + t2 * 128 + ((q ^ (t2 & 7)) << 4));
+            v[16 * sh + 2 * q] = make_float2(f.x, f.y);
+            v[16 * sh + 2 * q + 1] = make_float2(f.z, f.w);
+          }
+      }
+      float ss;
+      {
+        float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 32; ++m) a2 = __ffma2_rn(v[m], v[m], a2);
+        ss = a2.x + a2.y;
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+      if (valid && p.rope) {
+        const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
+        if (pos < 0 || pos >= p.rope_max_pos) {
+          valid = false;
+        } else {
+          // pairs (v[m], v[16 + m]) turn by pos * theta_j, j = 32 h2 + 2m (+1):
+          // angle pos theta_hi + pos theta_lo, reduced by 2 pi in three terms
+          // (k negated: rint is odd), then sin / cos on [-pi, pi]
+          const float pf = static_cast<float>(pos);   // exact: pos < 2^22
+          const float2 pf2 = make_float2(pf, pf), npf2 = make_float2(-pf, -pf);
+          const float2 q2c = make_float2(-kInvTwoPi, -kInvTwoPi), six2 = make_float2(6.f, 6.f);
+          const float2 c2c = make_float2(kC2, kC2), c3c = make_float2(kC3, kC3);
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            if ((m & 3) == 0) asm volatile("" ::: "memory");   // bound the loads in flight (registers)
+            const float2 thh = thh_s[16 * h2 + m], thl = thl_s[16 * h2 + m];
+            const float2 ah = __fmul2_rn(pf2, thh);
+            const float2 e = __ffma2_rn(npf2, thh, ah);
+            const float2 nal = __ffma2_rn(npf2, thl, e);
+            const float2 q = __fmul2_rn(ah, q2c);
+            const float2 kn = make_float2(rintf(q.x), rintf(q.y));
+            float2 r = __ffma2_rn(kn, six2, ah);
+            r = __ffma2_rn(kn, c2c, r);
+            r = __ffma2_rn(kn, c3c, r);
+            r = __ffma2_rn(nal, m1, r);
+            float s0, c0, s1, c1;
+            __sincosf(r.x, &s0, &c0);
+            __sincosf(r.y, &s1, &c1);
+            const float2 sn = make_float2(s0, s1), cs = make_float2(c0, c1);
+            const float2 x = v[m], y = v[16 + m];
+            v[m] = __ffma2_rn(y, __fmul2_rn(sn, m1), __fmul2_rn(x, cs));
+            v[16 + m] = __ffma2_rn(x, sn, __fmul2_rn(y, cs));
+          }
+        }
+      }
+      const float nrm = sqrtf(ss);
+      // a power of two near 1 / ||x|| keeps the fp16 pieces in range (exact scaling)
+      float sc = 0.f;
+      if (valid && nrm > 0.f) {
+        int e;
+        frexpf(nrm, &e);
+        sc = ldexpf(1.f, -e);
+      }
+      if (h2 == 0) xnrm[g][0][t2] = valid ? nrm : qnan;
+      if (!valid && row < p.n && h2 == 0) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
+      const float2 sc2 = make_float2(sc, sc);
+      gsync();   // every row is in registers: the staging buffer takes the A operand
 #pragma unroll
       for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int j = 4 * h + q;   // 16-byte chunk of box sh (coordinates 64 sh ..)
-          const uint4 w4 = *reinterpret_cast<const uint4*>(xs + sh * (kTileVec * 128) + t * 128 + ((j ^ (t & 7)) << 4));
-          const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+          uint32_t hv[4], lv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            v[16 * sh + 4 * q + e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+          for (int e = 0; e < 4; ++e) {
+            const float2 x = __fmul2_rn(v[16 * sh + 4 * q + e], sc2);
+            const __half2 hh = __floats2half2_rn(x.x, x.y);
+            const float2 lo = __ffma2_rn(__half22float2(hh), m1, x);
+            const __half2 lh = __floats2half2_rn(lo.x, lo.y);
+            hv[e] = *reinterpret_cast<const uint32_t*>(&hh);
+            lv[e] = *reinterpret_cast<const uint32_t*>(&lh);
+          }
+          const int c = 8 * sh + 4 * h2 + q;
+          const uint32_t off = (c >> 3) * (kTileVec * 128) + rowbase2 + ((((c & 7) ^ (t2 & 7))) << 4);
+          *reinterpret_cast<uint4*>(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          *reinterpret_cast<uint4*>(a_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
         }
-    } else {
-#pragma unroll
-      for (int sh = 0; sh < 2; ++sh)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int b = 2 * sh + h;   // box of coordinates 32 b ..
-          const float4 f = *reinterpret_cast<const float4*>(xs + b * (kTileVec * 128) + t * 128 + ((q ^ (t & 7)) << 4));
-          v[16 * sh + 2 * q] = make_float2(f.x, f.y);
-          v[16 * sh + 2 * q + 1] = make_float2(f.z, f.w);
-        }
+      tqtc::fence_smem_to_async();
     }
-    __syncthreads();   // the tile is in registers: its buffer may take the residual
-    if (!ok_x) {
-      valid = false;
-      if (row < p.n && h == 0)
-        p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-    }
-    // ||x|| before RoPE (a rotation: the norm is unchanged by it)
-    float ss;
-    {
+    const int64_t row = tile * kTileVec + r4;
+    if constexpr (!SPLIT) {
+      // ||x||^2 of row r4, this thread's 64 coordinates (box c4 of the staged bf16 tile)
       float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int m = 0; m < 32; ++m) a2 = __ffma2_rn(v[m], v[m], a2);
-      ss = a2.x + a2.y;
-    }
-    if (valid && p.rope) {
-      const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
-      if (pos < 0 || pos >= p.rope_max_pos) {
-        valid = false;
-        if (h == 0) p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-      } else {
-        // pairs (v[m], v[16 + m]) turn by pos * theta_j, j = 32 h + 2m (+1);
-        // the angle is pos theta_hi + pos theta_lo (error term of the first
-        // product by FMA), reduced by 2 pi in three terms (with k negated:
-        // rint is odd), then sin / cos on [-pi, pi]
-        const float pf = static_cast<float>(pos);   // exact: pos < 2^22
-        const float2 pf2 = make_float2(pf, pf), npf2 = make_float2(-pf, -pf);
-        const float2 q2c = make_float2(-kInvTwoPi, -kInvTwoPi), six2 = make_float2(6.f, 6.f);
-        const float2 c2c = make_float2(kC2, kC2), c3c = make_float2(kC3, kC3);
+      for (int j = 0; j < 8; ++j) {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(xs + c4 * (kTileVec * 128) + rowbase4 + ((j ^ (r4 & 7)) << 4));
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          if ((m & 3) == 0) asm volatile("" ::: "memory");   // bound the loads in flight (registers)
-          const float2 thh = thh_s[16 * h + m], thl = thl_s[16 * h + m];
-          const float2 ah = __fmul2_rn(pf2, thh);
-          const float2 e = __ffma2_rn(npf2, thh, ah);        // -(pf theta_hi - ah), exact
-          const float2 nal = __ffma2_rn(npf2, thl, e);       // -(low part of the angle)
-          const float2 q = __fmul2_rn(ah, q2c);
-          const float2 kn = make_float2(rintf(q.x), rintf(q.y));   // -k
-          float2 r = __ffma2_rn(kn, six2, ah);
-          r = __ffma2_rn(kn, c2c, r);
-          r = __ffma2_rn(kn, c3c, r);
-          r = __ffma2_rn(nal, m1, r);
-          float s0, c0, s1, c1;
-          __sincosf(r.x, &s0, &c0);
-          __sincosf(r.y, &s1, &c1);
-          const float2 sn = make_float2(s0, s1), cs = make_float2(c0, c1);
-          const float2 x = v[m], y = v[16 + m];
-          v[m] = __ffma2_rn(y, __fmul2_rn(sn, m1), __fmul2_rn(x, cs));   // x cos - y sin
-          v[16 + m] = __ffma2_rn(x, sn, __fmul2_rn(y, cs));              // y cos + x sin
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+          a2 = __ffma2_rn(x, x, a2);
         }
       }
+      xnrm[g][c4][r4] = a2.x + a2.y;
     }
-    // every lane runs the transform (shuffles need the whole warp); rows
-    // that are absent or out of RoPE range carry zeros and store nothing
-    if (!valid) {
+    // ---- 3. y = A (H D)^T
+    tqtc::fence_before_sync();
+    gsync();
+    if (gt == 0 && !failed) {
+      tqtc::fence_after_sync();
 #pragma unroll
-      for (int m = 0; m < 32; ++m) v[m] = make_float2(0.f, 0.f);
-    }
-    // D x, then the Walsh-Hadamard stages on coordinate bits 0-4 and 6
+      for (int ks = 0; ks < D / 16; ++ks)
+        tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_hi), ks, kTileVec),
+                          tqtc::sw128_desc_kstep(tqtc::smem_u32(hd_op), ks, D), idy, ks > 0);
+      if constexpr (SPLIT) {
 #pragma unroll
-    for (int sh = 0; sh < 2; ++sh)
-#pragma unroll
-      for (int m = 0; m < 16; ++m) v[16 * sh + m] = __fmul2_rn(v[16 * sh + m], dsg_s[32 * sh + 16 * h + m]);
-#pragma unroll
-    for (int m = 0; m < 32; ++m) {   // bit 0: inside a pair
-      const float a = v[m].x, b = v[m].y;
-      v[m] = make_float2(a + b, a - b);
-    }
-#pragma unroll
-    for (int hb = 1; hb < 32; hb <<= 1)   // bits 1-4 and 6 (pair index bits 0-4)
-#pragma unroll
-      for (int m = 0; m < 32; ++m)
-        if (!(m & hb)) {
-          const float2 a = v[m], b = v[m | hb];
-          v[m] = __fadd2_rn(a, b);
-          v[m | hb] = __ffma2_rn(b, m1, a);
-        }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-    const float nrm = valid ? sqrtf(ss) : 0.f;
-    {
-      const float sgn = h ? -1.f : 1.f;                 // coordinate bit 5: across the lane pair
-      const float2 sgn2 = make_float2(sgn, sgn);
-#pragma unroll
-      for (int m = 0; m < 32; ++m) {
-        const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[m].x, 16), __shfl_xor_sync(0xffffffffu, v[m].y, 16));
-        v[m] = __ffma2_rn(sgn2, v[m], o);
+        for (int ks = 0; ks < D / 16; ++ks)
+          tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_lo), ks, kTileVec),
+                            tqtc::sw128_desc_kstep(tqtc::smem_u32(hd_op), ks, D), idy, true);
       }
+      tqtc::mma_commit(&mb_y[g]);
+    }
+    // ---- 4. codes and residual of row r4, coordinates 64 c4 ..
+    float nrm, scale;
+    bool valid;
+    if constexpr (SPLIT) {
+      nrm = xnrm[g][0][r4];
+      valid = row < p.n && !isnan(nrm);
+      float sc = 0.f;
+      if (valid && nrm > 0.f) {
+        int e;
+        frexpf(nrm, &e);
+        sc = ldexpf(1.f, -e);
+      }
+      // y holds H D (sc x): the unit coordinates are y / (sc ||x|| sqrt d)
+      scale = valid && nrm > 0.f ? 1.f / (sc * nrm) * inv_sqrt_d : 0.f;
+    } else {
+      nrm = sqrtf(xnrm[g][0][r4] + xnrm[g][1][r4]);
+      valid = row < p.n && ok_x;
+      scale = valid && nrm > 0.f ? 1.f / nrm * inv_sqrt_d : 0.f;
+      if (!valid && row < p.n && c4 == 0) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
+    }
+    const bool ok_y = !failed && tqtc::mbar_wait(&mb_y[g], ph_y, kWaitLimit);
+    ph_y ^= 1;
+    tqtc::fence_after_sync();
+    float2 u[32];   // u[m] = coordinates (64 c4 + 2m, + 1)
+    {
+      float y[32];
+      tqtc::tmem_ld32(tm + tm_lane + 64 * c4, y);
+#pragma unroll
+      for (int m = 0; m < 16; ++m) u[m] = make_float2(y[2 * m], y[2 * m + 1]);
+      tqtc::tmem_ld32(tm + tm_lane + 64 * c4 + 32, y);
+#pragma unroll
+      for (int m = 0; m < 16; ++m) u[16 + m] = make_float2(y[2 * m], y[2 * m + 1]);
     }
     {
-      const float scale = (nrm > 0.f ? 1.0f / nrm : 0.f) * inv_sqrt_d;
       const float2 sc2 = make_float2(scale, scale), z2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int m = 0; m < 32; ++m) v[m] = __ffma2_rn(v[m], sc2, z2);   // unit-vector coordinates, -0 -> +0
+      for (int m = 0; m < 32; ++m) u[m] = __ffma2_rn(u[m], sc2, z2);   // unit-vector coordinates, -0 -> +0
     }
+    const float nv = valid ? nrm : 0.f;
     float nl[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) nl[k] = nrm * p.lpos[k];
+    for (int k = 0; k < 4; ++k) nl[k] = nv * p.lpos[k];
     uint32_t w0[BITS], w1[BITS];
-    float rr = quantize32_x2<BITS>(v, tp, nl, nrm, w0);        // coordinates 32h .. 32h + 31: word h
-    rr += quantize32_x2<BITS>(v + 16, tp, nl, nrm, w1);        // 64 + 32h ..: word 2 + h
-    rr += __shfl_xor_sync(0xffffffffu, rr, 16);
-    if (valid) {
+    float rr = quantize32_x2<BITS>(u, tp, nl, nv, w0);        // coordinates 64 c4 .. + 31: word 2 c4
+    rr += quantize32_x2<BITS>(u + 16, tp, nl, nv, w1);        // 64 c4 + 32 ..: word 2 c4 + 1
+    xrr[g][c4][r4] = rr;
+    if (valid && ok_y) {
       constexpr int NJ = 4;
       uint32_t* crec = p.codes + row * p.out_stride * (BITS * NJ);   // 4-byte aligned records
 #pragma unroll
       for (int k = 0; k < BITS; ++k) {
-        crec[k * NJ + h] = w0[k];
-        crec[k * NJ + 2 + h] = w1[k];
+        crec[k * NJ + 2 * c4] = w0[k];
+        crec[k * NJ + 2 * c4 + 1] = w1[k];
       }
-      if (h == 0) p.norms[row * p.out_stride] = make_float2(nrm, sqrtf(rr));
     }
-    // residual (zero on absent rows) as bf16 hi + lo into row t of the A
-    // operand (16-byte chunks)
+    // residual (zero on absent rows) as bf16 hi + lo over the A operand, row r4
+    // (the staged tile was read before the barrier ahead of the products)
 #pragma unroll
-    for (int sh = 0; sh < 2; ++sh)
+    for (int j = 0; j < 8; ++j) {
+      uint32_t hv[4], lv[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t hv[4], lv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 r = v[16 * sh + 4 * q + e];
-          __nv_bfloat162 hb2 = __floats2bfloat162_rn(r.x, r.y);
-          const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb2);
-          const float2 lo = __ffma2_rn(make_float2(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u)),
-                                       m1, r);
-          __nv_bfloat162 lb = __floats2bfloat162_rn(lo.x, lo.y);
-          hv[e] = hbits;
-          lv[e] = *reinterpret_cast<uint32_t*>(&lb);
-        }
-        const int c = 8 * sh + 4 * h + q;   // 16-byte chunk of the row
-        const uint32_t off = (c >> 3) * (kTileVec * 128) + rowbase + ((((c & 7) ^ vx)) << 4);
-        *reinterpret_cast<uint4*>(r_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        *reinterpret_cast<uint4*>(r_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+      for (int e = 0; e < 4; ++e) {
+        const float2 r = u[4 * j + e];
+        __nv_bfloat162 hb2 = __floats2bfloat162_rn(r.x, r.y);
+        const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb2);
+        const float2 lo =
+            __ffma2_rn(make_float2(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u)), m1, r);
+        __nv_bfloat162 lb = __floats2bfloat162_rn(lo.x, lo.y);
+        hv[e] = hbits;
+        lv[e] = *reinterpret_cast<uint32_t*>(&lb);
       }
-    // ---- S r of the tile on the tensor core
+      const uint32_t off = c4 * (kTileVec * 128) + rowbase4 + ((j ^ (r4 & 7)) << 4);
+      *reinterpret_cast<uint4*>(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      *reinterpret_cast<uint4*>(a_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+    }
+    // ---- 5. S r of the tile, into the columns y has left
     tqtc::fence_smem_to_async();
     tqtc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0 && !failed) {
+    gsync();
+    if (gt == 0 && !failed) {
       tqtc::fence_after_sync();
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
-        tqtc::mma_bf16_ss(tmem, tqtc::sw128_desc_kstep(tqtc::smem_u32(r_hi), ks, kTileVec),
-                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, ks > 0);
+        tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_hi), ks, kTileVec),
+                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), ids, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks)
-        tqtc::mma_bf16_ss(tmem, tqtc::sw128_desc_kstep(tqtc::smem_u32(r_lo), ks, kTileVec),
-                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), idesc, true);
-      tqtc::mma_commit(&mbar);
+        tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_lo), ks, kTileVec),
+                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), ids, true);
+      tqtc::mma_commit(&mb_s[g]);
     }
-    const bool ok = !failed && ok_x && tqtc::mbar_wait(&mbar, phase, kWaitLimit);
-    phase ^= 1;
+    if (valid && ok_y && c4 == 0) p.norms[row * p.out_stride] = make_float2(nrm, sqrtf(rr + xrr[g][1][r4]));
+    const bool ok = ok_y && tqtc::mbar_wait(&mb_s[g], ph_s, kWaitLimit);
+    ph_s ^= 1;
     tqtc::fence_after_sync();
-    if (!ok) s_fail = 1;
-    // the products have read the residual: its buffer takes the next input tile
-    if (tid == 0 && ok && tile + gridDim.x < n_tiles) issue_x(tile + gridDim.x);
-    // ---- sign bits: warp w reads lanes 32 (w % 4) + lane, columns 64 (w / 4) ..
-    // Each bit is the complemented fp32 sign bit, shifted in by one funnel
-    // shift: 1 for +0 and positive projections, 0 for negative ones and -0
-    // (an exact zero projection is within any sign tolerance).
+    if (!ok || !ok_x) s_fail[g] = 1;
+    // the products have read the operand buffer: it takes the group's next tile
+    if (gt == 0 && ok && tile + tstep < n_tiles) issue_x(tile + tstep);
+    // sign bits of S r: complemented fp32 sign bits, one funnel shift each
+    // (an exact -0 projection reads as negative, within the sign tolerance)
     {
       constexpr int NJ = 4;
-      const int quad = warp & 3, part = warp >> 2;
-      const int64_t srow = tile * kTileVec + quad * 32 + lane;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float val[32];
-        tqtc::tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 64 * part + 32 * c, val);
+        tqtc::tmem_ld32(tm + tm_lane + 64 * c4 + 32 * c, val);
         uint32_t w = 0;
 #pragma unroll
         for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[b]), w, 1);
-        if (srow < p.n) p.signs[srow * p.out_stride * NJ + 2 * part + c] = ok ? ~w : 0u;
+        if (row < p.n) p.signs[row * p.out_stride * NJ + 2 * c4 + c] = ok ? ~w : 0u;
       }
-      if (!ok && part == 0 && srow < p.n)
-        p.norms[srow * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+      if (!ok && c4 == 0 && row < p.n) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
     }
     tqtc::fence_before_sync();
-    __syncthreads();
+    gsync();
   }
   tqtc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tqtc::tmem_free(tmem_slot, D);
+  if (warp == 0) tqtc::tmem_free(tmem_slot, 256);
 }
 
 template <int D, int BITS, typename T>
@@ -1123,27 +1196,36 @@ int launch_encode_rows(const EncodeParams& p, cudaStream_t stream) {
 // Batches below this many vectors take the low-latency warp-per-vector kernel.
 constexpr int64_t kRowsKernelMinN = 16384;
 
-template <int BITS, typename T>
-int launch_encode_pairs(const EncodeParams& p, cudaStream_t stream) {
-  // Positions past 2^22 (the in-kernel angle reduction's range) or more rows
-  // than a TMA coordinate holds go to the table-driven one-thread kernel.
-  if ((p.rope && p.rope_max_pos > kPairsMaxRopePos) || p.n >= (int64_t(1) << 31))
-    return launch_encode_rows<128, BITS, T>(p, stream);
-  CUtensorMap xmap;
-  if (!tq::make_tmap_2d(&xmap, p.x, static_cast<int>(sizeof(T)), p.n, 128, p.ld, 128 / static_cast<int>(sizeof(T)),
-                        kTileVec))
-    return launch_encode_rows<128, BITS, T>(p, stream);
-  const size_t smem = 128 * 128 * 2 + 2 * static_cast<size_t>(kTileVec) * 128 * 2 + 1024;   // 97 KB: 2 CTAs / SM
-  auto kern = encode_pairs_kernel<BITS, T>;
+template <int BITS, typename T, bool SPLIT>
+int launch_encode_tc(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_t stream) {
+  const size_t smem = 6 * static_cast<size_t>(kTileVec) * 128 * 2 + 1024;   // S, H D, 2 x (hi, lo): 193 KB
+  auto kern = encode_tc_kernel<BITS, T, SPLIT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return TQ_ECUDA;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = (p.n + kTileVec - 1) / kTileVec;
-  const int blocks = static_cast<int>(tiles < 2LL * sms ? tiles : 2LL * sms);
-  kern<<<blocks, kPairThreads, smem, stream>>>(xmap, p);
+  const int64_t pairs = (tiles + 1) / 2;
+  const int blocks = static_cast<int>(pairs < sms ? pairs : sms);
+  kern<<<blocks, kTcThreads, smem, stream>>>(xmap, p);
   return tq::launch_status();
+}
+
+template <int BITS, typename T>
+int launch_encode_d128(const EncodeParams& p, cudaStream_t stream) {
+  // Positions past 2^22 (the in-kernel angle reduction's range) or more rows
+  // than a TMA coordinate holds go to the table-driven one-thread kernel.
+  if ((p.rope && p.rope_max_pos > kPairsMaxRopePos) || p.n >= (int64_t(1) << 31) || !p.hd_op)
+    return launch_encode_rows<128, BITS, T>(p, stream);
+  CUtensorMap xmap;
+  if (!tq::make_tmap_2d(&xmap, p.x, static_cast<int>(sizeof(T)), p.n, 128, p.ld, 128 / static_cast<int>(sizeof(T)),
+                        kTileVec))
+    return launch_encode_rows<128, BITS, T>(p, stream);
+  if constexpr (sizeof(T) == 2) {
+    if (!p.rope) return launch_encode_tc<BITS, T, false>(p, xmap, stream);
+  }
+  return launch_encode_tc<BITS, T, true>(p, xmap, stream);
 }
 
 template <int D, int BITS, typename T>
@@ -1161,7 +1243,7 @@ int launch_encode(const EncodeParams& p, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, encode_vec_kernel<D, BITS, T>, p) == cudaSuccess ? TQ_OK : TQ_ECUDA;
   }
   if (p.n < kRowsKernelMinN) return launch_encode_warp<D, BITS, T>(p, stream);
-  if constexpr (D == 128) return launch_encode_pairs<BITS, T>(p, stream);
+  if constexpr (D == 128) return launch_encode_d128<BITS, T>(p, stream);
   return launch_encode_rows<D, BITS, T>(p, stream);
 }
 
@@ -1214,6 +1296,8 @@ extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, in
   p.out_stride = out_stride;
   p.dsigns = h->d_signs;
   p.s_op = h->d_s_op;
+  // H D for the tensor-core encode: fp16 when the rows are split (RoPE or fp32 input), else bf16
+  p.hd_op = (apply_rope || dtype == TQ_F32) ? h->d_hd_f16 : h->d_hd_bf16;
   p.st = h->d_st;
   {
     const int half = 1 << (h->bits - 1);

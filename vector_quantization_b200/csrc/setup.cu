@@ -228,6 +228,8 @@ void release(tq_rotation* h) {
   cudaFree(h->d_s);
   cudaFree(h->d_st);
   cudaFree(h->d_s_op);
+  cudaFree(h->d_hd_f16);
+  cudaFree(h->d_hd_bf16);
   cudaFree(h->d_pi_hi);
   cudaFree(h->d_pi_lo);
   cudaFree(h->d_s_bf16);
@@ -383,6 +385,21 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
           op[off / 2] = static_cast<uint16_t>(bits >> 16);
         }
       if ((st = upload(&h->d_s_op, op.data(), op.size())) != TQ_OK) { release(h); return st; }
+      if (d == 128) {
+        // H D with H[j][k] = (-1)^popcount(j & k): rows j (output coordinate),
+        // K = k, entries +-1 exact in fp16 (0x3C00) and bf16 (0x3F80)
+        std::vector<uint16_t> hf(static_cast<size_t>(d) * d), hb(static_cast<size_t>(d) * d);
+        for (int j = 0; j < d; ++j)
+          for (int k = 0; k < d; ++k) {
+            const size_t off = static_cast<size_t>(k >> 6) * (static_cast<size_t>(d) * 128) + (j >> 3) * 1024 +
+                               (j & 7) * 128 + ((((k & 63) >> 3) ^ (j & 7)) << 4) + ((k & 7) << 1);
+            const bool neg = (__builtin_popcount(static_cast<unsigned>(j & k)) & 1) != (h->signs[k] < 0.f);
+            hf[off / 2] = neg ? 0xBC00u : 0x3C00u;
+            hb[off / 2] = neg ? 0xBF80u : 0x3F80u;
+          }
+        if ((st = upload(&h->d_hd_f16, hf.data(), hf.size())) != TQ_OK) { release(h); return st; }
+        if ((st = upload(&h->d_hd_bf16, hb.data(), hb.size())) != TQ_OK) { release(h); return st; }
+      }
     }
   }
   if (rope_base > 0.0) {

@@ -42,6 +42,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor: fp16 x fp16 -> fp32, both K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Descriptor of the k-th 16-element K step of an operand with R rows.
 __device__ __forceinline__ uint64_t sw128_desc_kstep(uint32_t base, int kstep, int R) {
   const uint32_t addr = base + static_cast<uint32_t>((kstep >> 2) * (R * 128) + (kstep & 3) * 32);

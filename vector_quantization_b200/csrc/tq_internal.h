@@ -39,6 +39,11 @@ struct tq_rotation {
   // S as bf16 in the tensor-core operand layout (K-major, 128-byte swizzle,
   // rows = sketch index, K = coordinate); Hadamard kind only.
   uint16_t* d_s_op = nullptr;
+  // H D (the unnormalised Hadamard times the sign diagonal, entries +-1) in
+  // the same operand layout, rows = output coordinate, as fp16 and as bf16
+  // bits; Hadamard kind, d = 128 only.
+  uint16_t* d_hd_f16 = nullptr;
+  uint16_t* d_hd_bf16 = nullptr;
   // Dense kind: Pi as bf16 hi + lo pieces and S as bf16, row-major, for the
   // split tensor-core contractions.
   uint16_t* d_pi_hi = nullptr;
