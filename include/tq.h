@@ -141,6 +141,18 @@ int tq_rotation_export(const tq_rotation* h, float* pi, float* s,
  */
 int tq_tensor_core_selftest(int64_t* mismatches);
 
+/*
+ * tq_wait_selftest - diagnostic of the bounded waits every tensor-core and
+ * TMA wait in the kernels uses: one thread initialises an mbarrier that
+ * expects one arrival and waits for its first phase with a limit of 2^16
+ * polls.  arrive != 0: the thread arrives first, and *completed = 1 when the
+ * wait saw the phase complete.  arrive == 0: nothing completes the phase;
+ * the wait gives up after its limit and *completed = 0 (the context stays
+ * usable; no trap, no fault).  Synchronous; allocates and frees 4 bytes of
+ * device memory.  Returns TQ_OK, TQ_EINVAL, TQ_ENOMEM or TQ_ECUDA.
+ */
+int tq_wait_selftest(int arrive, int* completed);
+
 /* Record geometry of a handle: d, m, bits and bytes of codes / signs. */
 int tq_rotation_dims(const tq_rotation* h, int* d, int* m, int* bits,
                      int64_t* code_bytes, int64_t* sign_bytes);

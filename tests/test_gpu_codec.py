@@ -159,6 +159,15 @@ def test_encode_rejects_bad_arguments(cuda_device):
         tq.quantize_kv(g2, x, apply_rope=True, pos_period=4)
 
 
+def test_bounded_wait_gives_up_and_context_stays_usable(cuda_device):
+    """A wait on an mbarrier phase that nothing completes returns after its
+    poll limit with a status the host reads; the context keeps working."""
+    from vector_quantization_b200 import tq
+    assert tq.wait_selftest(arrive=False) == 0
+    assert tq.wait_selftest(arrive=True) == 1
+    assert tq.tensor_core_selftest() == 0
+
+
 def test_tensor_core_selftest(cuda_device):
     from vector_quantization_b200 import tq
     assert tq.tensor_core_selftest() == 0

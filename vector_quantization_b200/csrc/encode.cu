@@ -48,7 +48,7 @@ struct EncodeParams {
 
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
 constexpr int kTileVec = 128;
-constexpr int kWaitLimit = 1 << 22;
+constexpr int kWaitLimit = 1 << 17;   // polls of about 9 us each: a wait gives up after about a second
 
 // ===========================================================================
 // Block-per-vector encode, for the few vectors a decode step appends: thread

@@ -33,7 +33,7 @@ namespace {
 constexpr int kGM = 128, kGN = 128, kGK = 64;
 constexpr int kGStages = 3;
 constexpr int kGAcc = 4;                     // tensor-memory accumulators (kGAcc * kGN = 512 columns)
-constexpr int kGWaitLimit = 1 << 24;
+constexpr int kGWaitLimit = 1 << 17;   // polls of about 9 us each: a wait gives up after about a second
 constexpr int kATileBytes = kGM * kGK * 2;   // 16 KB
 constexpr int kBTileBytes = kGN * kGK * 2;   // 16 KB
 

@@ -14,7 +14,7 @@
 namespace {
 
 constexpr int kN = 128;
-constexpr int kWaitLimit = 1 << 22;
+constexpr int kWaitLimit = 1 << 17;   // polls of about 9 us each: a wait gives up after about a second
 
 __device__ __host__ inline int sel_a(int r, int k) { return (r * 7 + k * 3) % 11 - 5; }
 __device__ __host__ inline int sel_b(int n, int k) { return (n * 5 + k) % 9 - 4; }
@@ -62,7 +62,40 @@ __global__ void __launch_bounds__(128) tc_selftest_kernel(float* __restrict__ ou
   if (warp == 0) tqtc::tmem_free(tmem, kN);
 }
 
+// Bounded-wait check: thread 0 inits an mbarrier expecting one arrival.
+// With `arrive` it arrives first and the wait must see the phase complete;
+// without, nothing ever completes the phase and the wait must give up after
+// `limit` polls.  status[0] = 1 if the wait saw completion, 0 if it gave up.
+__global__ void wait_selftest_kernel(int arrive, int limit, int* __restrict__ status) {
+  __shared__ uint64_t mbar;
+  if (threadIdx.x != 0) return;
+  tqtc::mbar_init(&mbar, 1);
+  if (arrive) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(tqtc::smem_u32(&mbar)) : "memory");
+  status[0] = tqtc::mbar_wait(&mbar, 0, limit) ? 1 : 0;
+}
+
 }  // namespace
+
+extern "C" int tq_wait_selftest(int arrive, int* completed) {
+  if (!completed) return TQ_EINVAL;
+  *completed = -1;
+  int* d_status = nullptr;
+  if (cudaMalloc(&d_status, sizeof(int)) != cudaSuccess) return TQ_ENOMEM;
+  int st = TQ_OK;
+  int h = -1;
+  if (cudaMemset(d_status, 0xFF, sizeof(int)) != cudaSuccess) {
+    st = TQ_ECUDA;
+  } else {
+    wait_selftest_kernel<<<1, 32>>>(arrive ? 1 : 0, 1 << 16, d_status);
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(&h, d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+      st = TQ_ECUDA;
+    else
+      *completed = h;
+  }
+  cudaFree(d_status);
+  return st;
+}
 
 extern "C" int tq_tensor_core_selftest(int64_t* mismatches) {
   if (!mismatches) return TQ_EINVAL;

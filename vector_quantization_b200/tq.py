@@ -54,6 +54,7 @@ def _load():
         "tq_search_topk": (c_i, [c_p, c_p, c_i, c_p, c_p, c_p, c_i64, c_i, c_p, c_p, c_p, c_sz, c_p]),
         "tq_search_workspace_size": (c_sz, [c_p, c_i, c_i64, c_i]),
         "tq_tensor_core_selftest": (c_i, [c_p]),
+        "tq_wait_selftest": (c_i, [c_i, c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -92,6 +93,13 @@ def _dtype_code(t) -> int:
 
 def version() -> int:
     return _lib.tq_version()
+
+
+def wait_selftest(arrive: bool) -> int:
+    """1 if a bounded mbarrier wait saw its phase complete, 0 if it gave up."""
+    done = ctypes.c_int(-1)
+    _check(_lib.tq_wait_selftest(1 if arrive else 0, ctypes.byref(done)), "tq_wait_selftest")
+    return done.value
 
 
 def tensor_core_selftest() -> int:
