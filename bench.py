@@ -370,6 +370,24 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- rank plumbing
+def max_over_ranks(value, dist, device):
+    """The largest `value` over all ranks (every rank receives it); the
+    value itself with a single process (dist None)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, units_per_step_per_rank, steps, slowest_ms):
+    """Units all ranks processed per second, timed by the slowest rank
+    (weak scaling: every rank processes the same number of units)."""
+    return world * units_per_step_per_rank * steps / (slowest_ms / 1e3)
+
+
 # --------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -456,12 +474,9 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     elapsed_ms = e0.elapsed_time(e1)
     split_ms = [a.elapsed_time(b) for row in prof for (a, b) in row]
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     tokens_per_step = L * B * Hkv * T
-    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    value = whole_job_rate(world, tokens_per_step, args.steps, elapsed_ms)
 
     # ---- end-to-end through the public API with host buffers ----------------
     host_in = ([torch.empty_like(x, device="cpu").pin_memory().copy_(x.cpu()) for x in nks],
@@ -486,11 +501,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = f0.elapsed_time(f1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * tokens_per_step * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = whole_job_rate(world, tokens_per_step, args.steps, e2e_ms)
 
     if rank != 0:
         return

@@ -1,0 +1,68 @@
+"""Multi-process host logic of bench.py on CPU (gloo, world size 2): the
+device time is taken as the maximum over ranks, every rank sees the same
+value, the whole-job rate counts all ranks' units, and the reference arm does
+its work on rank 0 only."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        mine = 10.0 + 5.0 * rank                   # rank 1 is the slower one
+        slowest = bench.max_over_ranks(mine, dist, torch.device("cpu"))
+        rate = bench.whole_job_rate(world, 1000, 4, slowest)
+        dist.barrier()
+        out.put((rank, slowest, rate))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_rate_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [g[0] for g in got] == [0, 1]
+    for _, slowest, rate in got:
+        assert slowest == 15.0                     # max over ranks, on every rank
+        assert rate == pytest.approx(2 * 1000 * 4 / 0.015)
+
+
+def test_single_process_aggregation_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5, None, None) == 3.5
+    assert bench.whole_job_rate(1, 100, 10, 1000.0) == pytest.approx(1000.0)
+
+
+def test_reference_arm_other_ranks_do_no_work(capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+    bench.run_reference(None, 1, 2)                # args unused on rank != 0: returns at once
+    assert capsys.readouterr().out == ""
