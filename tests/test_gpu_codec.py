@@ -171,3 +171,35 @@ def test_bounded_wait_gives_up_and_context_stays_usable(cuda_device):
 def test_tensor_core_selftest(cuda_device):
     from vector_quantization_b200 import tq
     assert tq.tensor_core_selftest() == 0
+
+
+def test_encode_70b_slice_full_size_sampled(cuda_device):
+    """The bench's encode workload at full size: 8 KV heads x 2^20 tokens,
+    d = 128, bf16, 2+1 bits, keys with RoPE (position = token index) and
+    values without, each as one launch like the bench.  Sampled rows (tile
+    edges, the last rows, and a seeded random set) against the oracle over the
+    same bf16 inputs."""
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["llama31_70b_long_slice"]
+    Hkv, d, T, seed = c["kv_heads"], c["head_dim"], c["tokens"], c["seed"]
+    dev = cuda_device_of()
+    n = Hkv * T
+    rng = np.random.default_rng([seed, 77])
+    rows = np.unique(np.concatenate([
+        np.array([0, 1, 127, 128, 129, 255, 256, T - 1, T, T + 1, n - 129, n - 128, n - 2, n - 1]),
+        rng.integers(0, n, size=1500)]))
+    for apply_rope, tag in ((True, 3), (False, 4)):
+        rnd = synth.rotation_randomness(d, [seed, 1 if apply_rope else 2])
+        g = tq.Rotation(d, 2, rnd, rope_base=c["rope_base"] if apply_rope else 0.0, rope_max_pos=T)
+        o = ro.build_rotation(d, 2, rnd, rope_base=c["rope_base"] if apply_rope else 0.0)
+        x = synth.heavy_tailed_torch((1, Hkv, T, d), [seed, tag], dev)
+        out = tq.empty_records(g, (1, Hkv, T), dev)
+        kw = dict(apply_rope=True, pos_period=T) if apply_rope else {}
+        tq.quantize_kv(g, x, out=out, **kw)
+        torch.cuda.synchronize()
+        idx = torch.from_numpy(rows).to(dev)
+        xs = x.reshape(n, d).index_select(0, idx).float().cpu().numpy()
+        gpu = tuple(t.reshape(n, -1).index_select(0, idx).cpu().numpy() for t in out)
+        _, _, _, enc = oracle_records(o, xs, (rows % T).astype(np.int64) if apply_rope else None)
+        compare_records(o, gpu, enc)
+        del x, out
