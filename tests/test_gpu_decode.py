@@ -151,3 +151,32 @@ def test_decode_full_size_sampled(cuda_device, bits):
         qq = q[b:b + 1, j * G:(j + 1) * G].float().cpu().numpy()
         ref = at.decode_attention(rk_o, rv_o, qq, [T - 1], kk, vv, 1 / np.sqrt(D))
         assert_close(out[b:b + 1, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"bits {bits} seq {b} kv-head {j}")
+
+
+def test_decode_70b_slice_full_size_sampled(cuda_device):
+    """The Llama-3.1-70B-shaped long-context slice at full size (one
+    sequence, 64 query heads over 8 KV heads: G = 8, 2^20 cached tokens,
+    2+1 bits) in the launch configuration the bench times; one KV head's 8
+    query heads checked against the oracle's attention over the same packed
+    records."""
+    from vector_quantization_b200 import tq
+    dev = torch.device("cuda:0")
+    c = synth.CONFIGS["llama31_70b_long_slice"]
+    Hq, Hkv, T, seed = c["q_heads"], c["kv_heads"], c["tokens"], c["seed"]
+    G = Hq // Hkv
+    rk = tq.Rotation(D, 2, synth.rotation_randomness(D, [seed, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(D, 2, synth.rotation_randomness(D, [seed, 2]))
+    rk_o, _ = oracle_rotation(D, 2, [seed, 1], rope=c["rope_base"])
+    rv_o, _ = oracle_rotation(D, 2, [seed, 2])
+    kc = tq.quantize_kv(rk, synth.heavy_tailed_torch((1, Hkv, T, D), [seed, 3], dev), apply_rope=True, pos_period=T)
+    vc = tq.quantize_kv(rv, synth.heavy_tailed_torch((1, Hkv, T, D), [seed, 4], dev))
+    q = synth.heavy_tailed_torch((1, Hq, D), [seed, 5], dev)
+    q_pos = torch.full((1,), T - 1, dtype=torch.int64, device=dev)
+    out = tq.decode_attention(rk, rv, q, q_pos, kc, vc, T)
+    torch.cuda.synchronize()
+    j = Hkv - 1
+    kk = tuple(a[:, j:j + 1].cpu().numpy() for a in kc)
+    vv = tuple(a[:, j:j + 1].cpu().numpy() for a in vc)
+    qq = q[:, j * G:(j + 1) * G].float().cpu().numpy()
+    ref = at.decode_attention(rk_o, rv_o, qq, [T - 1], kk, vv, 1 / np.sqrt(D))
+    assert_close(out[:, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"70B slice kv-head {j}")
