@@ -9,11 +9,12 @@
 // dense Pi ([TurboQuant] "Principe", Étape 1) and the sketch S r ([TurboQuant]
 // "QJL") - where d is not a power of two and no fast transform exists.
 //
-// Kernel: one CTA per 128 x 128 output tile, 128 threads.  Operand tiles of
-// 64 K-elements are loaded by TMA (2-D tensor maps, 128-byte swizzle, zero
-// fill past the matrix edges) into a 3-stage ring; thread 0 issues the loads,
-// thread 32 the MMAs (M = 128, N = 128, K = 16 each), completion of a stage's
-// MMAs frees it through tcgen05.commit on an mbarrier.  K tiles go round-robin
+// Kernel: persistent, one CTA per SM over 128 x 128 output tiles.  Operand
+// tiles of 64 K-elements are loaded by TMA (2-D tensor maps, 128-byte
+// swizzle, zero fill past the matrix edges) into a 3- or 4-stage ring (192
+// KB); one thread issues the loads, one the MMAs (M = 128, N = 128, K = 16
+// each), completion of a stage's MMAs frees it through tcgen05.commit on an
+// mbarrier, and four epilogue warps drain each tile.  K tiles go round-robin
 // to four fp32 accumulators in tensor memory (all 512 columns), summed in
 // fp32 by the CUDA cores at the end: the tensor core's accumulation rounds
 // toward zero, and with d = 1536 a single accumulator shrank the rotated
@@ -31,34 +32,49 @@
 namespace {
 
 constexpr int kGM = 128, kGN = 128, kGK = 64;
-constexpr int kGStages = 3;
 constexpr int kGAcc = 4;                     // tensor-memory accumulators (kGAcc * kGN = 512 columns)
 constexpr int kGWaitLimit = 1 << 17;   // polls of about 9 us each: a wait gives up after about a second
 constexpr int kATileBytes = kGM * kGK * 2;   // 16 KB
 constexpr int kBTileBytes = kGN * kGK * 2;   // 16 KB
 
+// Persistent form of the split-bf16 GEMM: one CTA per SM walks the output
+// tiles (stride gridDim.x).  Warp 0 (one thread) streams every tile's K tiles
+// through the TMA ring; warp 1 (one thread) issues the MMAs, and before each
+// new tile waits until the epilogue has taken the previous tile's four
+// accumulators out of tensor memory; warps 2-5 (tensor-memory lane quadrants
+// warp % 4) wait for a tile's last MMA, sum its accumulators into registers,
+// release tensor memory (128 arrivals on an mbarrier) and only then store,
+// so the stores and the next tile's loads overlap the next tile's MMAs.
+// Every wait is bounded; once one runs out, later tiles are written as NaN
+// without waiting.
+constexpr int kPThreads = 6 * 32;
+
 template <bool BLO>
-__global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap mAh,
-                                                         const __grid_constant__ CUtensorMap mAl,
-                                                         const __grid_constant__ CUtensorMap mBh,
-                                                         const __grid_constant__ CUtensorMap mBl, int M, int N, int K,
-                                                         float* __restrict__ C, int64_t ldc) {
+__global__ void __launch_bounds__(kPThreads, 1) tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap mAh,
+                                                                         const __grid_constant__ CUtensorMap mAl,
+                                                                         const __grid_constant__ CUtensorMap mBh,
+                                                                         const __grid_constant__ CUtensorMap mBl,
+                                                                         int M, int N, int K, float* __restrict__ C,
+                                                                         int64_t ldc) {
+  constexpr int STAGES = BLO ? 3 : 4;
   constexpr int STAGE = 2 * kATileBytes + (BLO ? 2 : 1) * kBTileBytes;
   extern __shared__ uint8_t raw[];
-  __shared__ uint64_t full[kGStages], empty[kGStages], done;
+  __shared__ uint64_t full[STAGES], empty[STAGES], acc_full, acc_empty;
   __shared__ uint32_t tmem_slot;
-  __shared__ int failed;
+  __shared__ volatile int failed;
   uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int m0 = blockIdx.y * kGM, n0 = blockIdx.x * kGN;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tiles_n = (N + kGN - 1) / kGN;
+  const int n_tiles = ((M + kGM - 1) / kGM) * tiles_n;
   const int KT = (K + kGK - 1) / kGK;
 
   if (tid == 0) {
-    for (int s = 0; s < kGStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       tqtc::mbar_init(&full[s], 1);
       tqtc::mbar_init(&empty[s], 1);
     }
-    tqtc::mbar_init(&done, 1);
+    tqtc::mbar_init(&acc_full, 1);
+    tqtc::mbar_init(&acc_empty, 128);
     failed = 0;
   }
   if (warp == 0) tqtc::tmem_alloc(&tmem_slot, kGAcc * kGN);
@@ -66,85 +82,120 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
   __syncthreads();
   tqtc::fence_after_sync();
   const uint32_t tmem = tmem_slot;
-
   auto stage_ptr = [&](int s) { return base + s * STAGE; };
-  if (tid == 0) {
-    // producer: TMA loads of the K tiles into the ring
-    bool ok = true;
-    for (int kt = 0; kt < KT && ok; ++kt) {
-      const int s = kt % kGStages;
-      if (kt >= kGStages) ok = tqtc::mbar_wait(&empty[s], ((kt / kGStages) - 1) & 1, kGWaitLimit);
-      if (!ok) break;
-      uint8_t* st = stage_ptr(s);
-      tqtc::mbar_arrive_expect_tx(&full[s], STAGE);
-      tqtc::tma_load_2d(st, &mAh, kt * kGK, m0, &full[s]);
-      tqtc::tma_load_2d(st + kATileBytes, &mAl, kt * kGK, m0, &full[s]);
-      tqtc::tma_load_2d(st + 2 * kATileBytes, &mBh, kt * kGK, n0, &full[s]);
-      if constexpr (BLO) tqtc::tma_load_2d(st + 2 * kATileBytes + kBTileBytes, &mBl, kt * kGK, n0, &full[s]);
-    }
-    if (!ok) failed = 1;
-  } else if (tid == 32) {
-    // MMA issuer
-    const uint32_t idesc = tqtc::idesc_bf16_f32(kGM, kGN);
-    bool ok = true;
-    for (int kt = 0; kt < KT && ok; ++kt) {
-      const int s = kt % kGStages;
-      ok = tqtc::mbar_wait(&full[s], (kt / kGStages) & 1, kGWaitLimit);
-      if (!ok) break;
-      tqtc::fence_after_sync();
-      const uint32_t a_hi = tqtc::smem_u32(stage_ptr(s)), a_lo = a_hi + kATileBytes;
-      const uint32_t b_hi = a_hi + 2 * kATileBytes, b_lo = b_hi + kBTileBytes;
-      const uint32_t dacc = tmem + (kt % kGAcc) * kGN;
-#pragma unroll
-      for (int ks = 0; ks < kGK / 16; ++ks) {
-        const bool acc = kt >= kGAcc || ks > 0;
-        tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(a_hi, ks, kGM), tqtc::sw128_desc_kstep(b_hi, ks, kGN), idesc, acc);
-        if constexpr (BLO)
-          tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(a_hi, ks, kGM), tqtc::sw128_desc_kstep(b_lo, ks, kGN), idesc,
-                            true);
-        tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(a_lo, ks, kGM), tqtc::sw128_desc_kstep(b_hi, ks, kGN), idesc, true);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer: TMA loads of every tile's K tiles into the ring
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile / tiles_n) * kGM, n0 = (tile % tiles_n) * kGN;
+        for (int kt = 0; kt < KT; ++kt, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES) ok = tqtc::mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, kGWaitLimit);
+          if (!ok || failed) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = stage_ptr(s);
+          tqtc::mbar_arrive_expect_tx(&full[s], STAGE);
+          tqtc::tma_load_2d(st, &mAh, kt * kGK, m0, &full[s]);
+          tqtc::tma_load_2d(st + kATileBytes, &mAl, kt * kGK, m0, &full[s]);
+          tqtc::tma_load_2d(st + 2 * kATileBytes, &mBh, kt * kGK, n0, &full[s]);
+          if constexpr (BLO) tqtc::tma_load_2d(st + 2 * kATileBytes + kBTileBytes, &mBl, kt * kGK, n0, &full[s]);
+        }
       }
-      tqtc::mma_commit(&empty[s]);
+      if (!ok) failed = 1;
     }
-    if (!ok) failed = 1;
-    tqtc::mma_commit(&done);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer
+      const uint32_t idesc = tqtc::idesc_bf16_f32(kGM, kGN);
+      int it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tc) {
+        if (tc > 0) ok = tqtc::mbar_wait(&acc_empty, (tc - 1) & 1, kGWaitLimit);   // previous tile taken out
+        if (!ok || failed) {
+          ok = false;
+          break;
+        }
+        tqtc::fence_after_sync();
+        for (int kt = 0; kt < KT; ++kt, ++it) {
+          const int s = it % STAGES;
+          ok = tqtc::mbar_wait(&full[s], (it / STAGES) & 1, kGWaitLimit);
+          if (!ok || failed) {
+            ok = false;
+            break;
+          }
+          tqtc::fence_after_sync();
+          const uint32_t a_hi = tqtc::smem_u32(stage_ptr(s)), a_lo = a_hi + kATileBytes;
+          const uint32_t b_hi = a_hi + 2 * kATileBytes, b_lo = b_hi + kBTileBytes;
+          const uint32_t dacc = tmem + (kt % kGAcc) * kGN;
+#pragma unroll
+          for (int ks = 0; ks < kGK / 16; ++ks) {
+            const bool acc = kt >= kGAcc || ks > 0;
+            tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(a_hi, ks, kGM), tqtc::sw128_desc_kstep(b_hi, ks, kGN), idesc,
+                              acc);
+            if constexpr (BLO)
+              tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(a_hi, ks, kGM), tqtc::sw128_desc_kstep(b_lo, ks, kGN),
+                                idesc, true);
+            tqtc::mma_bf16_ss(dacc, tqtc::sw128_desc_kstep(a_lo, ks, kGM), tqtc::sw128_desc_kstep(b_hi, ks, kGN), idesc,
+                              true);
+          }
+          tqtc::mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tqtc::mma_commit(&acc_full);   // arrives once this tile's MMAs have completed
+      }
+      if (!ok) failed = 1;
+    }
+  } else {
+    // ---- epilogue: thread = tensor-memory lane = row 32 (warp % 4) + lane of the tile
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const int n_acc = KT < kGAcc ? KT : kGAcc;
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tc) {
+      const int m0 = (tile / tiles_n) * kGM, n0 = (tile % tiles_n) * kGN;
+      // warp-uniform: the tensor-memory loads below are .sync.aligned
+      const bool ok = __all_sync(0xffffffffu, !failed && tqtc::mbar_wait(&acc_full, tc & 1, kGWaitLimit));
+      tqtc::fence_after_sync();
+      float v[kGN];
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < kGN / 32; ++c) {
+          float w[32];
+          tqtc::tmem_ld32(tl + 32 * c, w);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[32 * c + q] = w[q];
+          for (int a = 1; a < n_acc; ++a) {
+            tqtc::tmem_ld32(tl + a * kGN + 32 * c, w);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[32 * c + q] += w[q];
+          }
+        }
+      }
+      tqtc::fence_before_sync();
+      tqtc::mbar_arrive(&acc_empty);   // this lane's accumulators are in registers
+      if (!ok) failed = 1;
+      const int row = m0 + r;
+      if (row < M) {
+        float* dst = C + static_cast<int64_t>(row) * ldc + n0;
+        if (n0 + kGN <= N && (ldc & 3) == 0) {
+#pragma unroll
+          for (int q = 0; q < kGN / 4; ++q)
+            reinterpret_cast<float4*>(dst)[q] =
+                ok ? make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]) : make_float4(NAN, NAN, NAN, NAN);
+        } else {
+#pragma unroll
+          for (int q = 0; q < kGN; ++q)
+            if (n0 + q < N) dst[q] = ok ? v[q] : NAN;
+        }
+      }
+    }
   }
   __syncwarp();
-  const bool ok = tqtc::mbar_wait(&done, 0, kGWaitLimit);
-  tqtc::fence_after_sync();
-  __syncthreads();
-  const bool good = ok && !failed;
-  // epilogue: thread t holds row m0 + t (tensor-memory lane t)
-  const int row = m0 + tid;
-  const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-#pragma unroll 1
-  const int n_acc = KT < kGAcc ? KT : kGAcc;
-  for (int c = 0; c < kGN / 32; ++c) {
-    float v[32];
-    tqtc::tmem_ld32(tl + 32 * c, v);
-    for (int a = 1; a < n_acc; ++a) {
-      float w[32];
-      tqtc::tmem_ld32(tl + a * kGN + 32 * c, w);
-#pragma unroll
-      for (int q = 0; q < 32; ++q) v[q] += w[q];
-    }
-    const int col = n0 + 32 * c;
-    if (row < M && col < N) {
-      float* dst = C + static_cast<int64_t>(row) * ldc + col;
-      if (col + 32 <= N && (ldc & 3) == 0) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 o = good ? make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3])
-                                : make_float4(NAN, NAN, NAN, NAN);
-          reinterpret_cast<float4*>(dst)[q] = o;
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (col + q < N) dst[q] = good ? v[q] : NAN;
-      }
-    }
-  }
   tqtc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tqtc::tmem_free(tmem, kGAcc * kGN);
@@ -234,19 +285,23 @@ int tc_gemm_split(int M, int N, int K, const uint16_t* ah, const uint16_t* al, i
   if (!make_map(&mah, ah, M, K, lda, kGM) || !make_map(&mal, al, M, K, lda, kGM) ||
       !make_map(&mbh, bh, N, K, ldb, kGN) || !make_map(&mbl, bl ? bl : bh, N, K, ldb, kGN))
     return TQ_ECUDA;
-  const dim3 grid((N + kGN - 1) / kGN, (M + kGM - 1) / kGM);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t n_tiles = static_cast<int64_t>((M + kGM - 1) / kGM) * ((N + kGN - 1) / kGN);
+  const dim3 grid(static_cast<unsigned>(n_tiles < sms ? n_tiles : sms));
   if (bl) {
-    const size_t smem = kGStages * (2 * kATileBytes + 2 * kBTileBytes) + 1024;
-    if (cudaFuncSetAttribute(tc_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-        cudaSuccess)
-      return TQ_ECUDA;
-    tc_gemm_kernel<true><<<grid, 128, smem, s>>>(mah, mal, mbh, mbl, M, N, K, C, ldc);
-  } else {
-    const size_t smem = kGStages * (2 * kATileBytes + kBTileBytes) + 1024;
-    if (cudaFuncSetAttribute(tc_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const size_t smem = 3 * (2 * kATileBytes + 2 * kBTileBytes) + 1024;
+    if (cudaFuncSetAttribute(tc_gemm_persistent_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return TQ_ECUDA;
-    tc_gemm_kernel<false><<<grid, 128, smem, s>>>(mah, mal, mbh, mbl, M, N, K, C, ldc);
+    tc_gemm_persistent_kernel<true><<<grid, kPThreads, smem, s>>>(mah, mal, mbh, mbl, M, N, K, C, ldc);
+  } else {
+    const size_t smem = 4 * (2 * kATileBytes + kBTileBytes) + 1024;
+    if (cudaFuncSetAttribute(tc_gemm_persistent_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return TQ_ECUDA;
+    tc_gemm_persistent_kernel<false><<<grid, kPThreads, smem, s>>>(mah, mal, mbh, mbl, M, N, K, C, ldc);
   }
   return launch_status();
 }

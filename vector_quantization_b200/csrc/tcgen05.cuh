@@ -109,6 +109,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity, int m
   return false;
 }
 
+// Arrive once on `mbar` (release).
+__device__ __forceinline__ void mbar_arrive(uint64_t* mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(mbar)) : "memory");
+}
+
 // Expect `bytes` of asynchronous copies on `mbar` and arrive once.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(bytes)
