@@ -500,117 +500,95 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   }
 }
 
-// Fast Walsh-Hadamard transform (Sylvester order, unnormalised) of G
-// vectors of kD values, thread i holding coordinate i of each: five stages
-// by warp shuffles, the two across warps through shared memory `buf`.
-template <int G>
-__device__ __forceinline__ void fwht_block(float (&v)[G], float (*buf)[kD]) {
-  const int i = threadIdx.x, lane = i & 31;
+// Fast Walsh-Hadamard transform (Sylvester order, unnormalised) of one kD
+// vector per group of kD threads, thread i of the group holding coordinate i:
+// five stages by warp shuffles, the two across warps through the group's row
+// of shared memory `buf`.  All groups of the block run it together.
+__device__ __forceinline__ void fwht_group(float& v, int i, float* buf) {
+  const int lane = i & 31;
 #pragma unroll
   for (int bit = 1; bit < 32; bit <<= 1) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float o = __shfl_xor_sync(0xffffffffu, v[h], bit);
-      v[h] = (lane & bit) ? o - v[h] : v[h] + o;
-    }
+    const float o = __shfl_xor_sync(0xffffffffu, v, bit);
+    v = (lane & bit) ? o - v : v + o;
   }
 #pragma unroll
   for (int bit = 32; bit < kD; bit <<= 1) {
     __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h) buf[h][i] = v[h];
+    buf[i] = v;
     __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float o = buf[h][i ^ bit];
-      v[h] = (i & bit) ? o - v[h] : v[h] + o;
-    }
+    const float o = buf[i ^ bit];
+    v = (i & bit) ? o - v : v + o;
   }
 }
 
-// sum_k col[k] x[h][k] for the G vectors staged in shared memory.
-template <int G>
-__device__ __forceinline__ void matvec_col(const float (&col)[kD], const float (*x)[kD], float (&acc)[G]) {
-#pragma unroll
-  for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll
-  for (int k = 0; k < kD; k += 4) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float4 xv = *reinterpret_cast<const float4*>(&x[h][k]);
-      acc[h] = fmaf(col[k], xv.x, acc[h]);
-      acc[h] = fmaf(col[k + 1], xv.y, acc[h]);
-      acc[h] = fmaf(col[k + 2], xv.z, acc[h]);
-      acc[h] = fmaf(col[k + 3], xv.w, acc[h]);
-    }
-  }
-}
-
-// One block of kD threads per (sequence b, KV head), covering the G query
-// heads of the group: RoPE, q~ = Pi q, s = S q~, then the fp16 B fragments
-// of the split kernel.  Thread i owns coordinate i and loads column i of S^T
-// (row i of S) once for all G heads, at the start, so the loads overlap the
-// rotation.
+// One block of G groups of kD threads per (sequence b, KV head); group h is
+// query head h of the group, thread i of it coordinate i: RoPE, q~ = Pi q,
+// s = S q~, then the fp16 B fragments of the split kernel.  The product S q~
+// is split by columns of S instead of by heads: group g holds columns
+// [g kD/G, (g + 1) kD/G) of row i of S in registers (loaded before the wait
+// for q, so the loads overlap the previous launch) and forms the partial sums
+// of all G heads over them; the G partials meet in shared memory.
 template <typename T, int G>
-__global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ q, const int64_t* __restrict__ q_pos,
-                                                          int Hkv, const float* __restrict__ dsigns,
-                                                          const float* __restrict__ st, const float2* __restrict__ rope_hi,
-                                                          const float2* __restrict__ rope_lo, int64_t rope_max_pos,
-                                                          int rope, uint16_t* __restrict__ qfrag,
-                                                          float2* __restrict__ kconst) {
+__global__ void __launch_bounds__(kD * G) decode_qprep_kernel(const T* __restrict__ q, const int64_t* __restrict__ q_pos,
+                                                             int Hkv, const float* __restrict__ dsigns,
+                                                             const float* __restrict__ st,
+                                                             const float2* __restrict__ rope_hi,
+                                                             const float2* __restrict__ rope_lo, int64_t rope_max_pos,
+                                                             int rope, uint16_t* __restrict__ qfrag,
+                                                             float2* __restrict__ kconst) {
   constexpr int NT = (2 * G + 7) / 8;
+  constexpr int KS = kD / G;   // columns of S per group
   __shared__ __align__(16) float buf[G][kD];
+  __shared__ __align__(16) float part[G][G][kD];   // [column group][head][i]
   __shared__ float red[2][G][2][kD / 32];
-  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int tid = threadIdx.x, h = tid / kD, i = tid % kD, lane = tid & 31, wg = i >> 5;
   const int bh = blockIdx.x;   // b * Hkv + kv; query head h of the group is row bh * G + h of q
   const int b = bh / Hkv;
-  float scol[kD];
+  float scol[KS];
 #pragma unroll
-  for (int k = 0; k < kD; ++k) scol[k] = __ldg(st + k * kD + i);
+  for (int k = 0; k < KS; ++k) scol[k] = __ldg(st + (h * KS + k) * kD + i);
   // S belongs to the handle; q may come from the previous launch
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  float v[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
+  float v;
+  {
     const size_t at = (static_cast<size_t>(bh) * G + h) * kD + i;
-    if constexpr (sizeof(T) == 4) v[h] = q[at];
-    else v[h] = __bfloat162float(q[at]);
+    if constexpr (sizeof(T) == 4) v = q[at];
+    else v = __bfloat162float(q[at]);
   }
   if (rope) {
     const int64_t pos = q_pos[b];
-#pragma unroll
-    for (int h = 0; h < G; ++h) buf[h][i] = v[h];
+    buf[h][i] = v;
     __syncthreads();
     if (pos < 0 || pos >= rope_max_pos) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) v[h] = __int_as_float(0x7fc00000);
+      v = __int_as_float(0x7fc00000);
     } else {
       const int j = i & (kD / 2 - 1);
       const float2 a = rope_hi[(pos >> kRopeLoBits) * (kD / 2) + j];
       const float2 c = rope_lo[(pos & (kRopeLoRows - 1)) * (kD / 2) + j];
       const float cs = a.x * c.x - a.y * c.y, sn = a.y * c.x + a.x * c.y;
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float x1 = buf[h][j], x2 = buf[h][j + kD / 2];
-        v[h] = i < kD / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
-      }
+      const float x1 = buf[h][j], x2 = buf[h][j + kD / 2];
+      v = i < kD / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
     }
   }
   // q~ = H (D q) / sqrt(d)
-  const float ds = dsigns[i];
-#pragma unroll
-  for (int h = 0; h < G; ++h) v[h] *= ds;
-  fwht_block<G>(v, buf);
-  const float inv_sqrt_d = rsqrtf(static_cast<float>(kD));
+  v *= dsigns[i];
+  fwht_group(v, i, buf[h]);
+  v *= rsqrtf(static_cast<float>(kD));
   __syncthreads();
+  buf[h][i] = v;
+  __syncthreads();
+  // partial S q~ of every head over this group's columns of S
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    v[h] *= inv_sqrt_d;
-    buf[h][i] = v[h];
+  for (int hh = 0; hh < G; ++hh) {
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) acc = fmaf(scol[k], buf[hh][h * KS + k], acc);
+    part[h][hh][i] = acc;
   }
   __syncthreads();
-  float sv[G];
-  matvec_col<G>(scol, buf, sv);
+  float sv = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) sv += part[g][h][i];
 
   // Scatter into the B-fragment layout of the split kernel.  Dim i sits in
   // pair slot j = i & 15 of the word of lane-column tg = i / 32; that slot's
@@ -624,76 +602,76 @@ __global__ void __launch_bounds__(kD) decode_qprep_kernel(const T* __restrict__ 
   auto frag_at = [&](int type, int nt, int n) {
     return ((((static_cast<size_t>(bh) * 2 + type) * NT + nt) * 8 + kb) * 32 + 4 * n + tg) * 4 + reg * 2 + e;
   };
-  float val[G][2];
+  const float val[2] = {v * inv_sigma, sv * inv_sigma};
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    val[h][0] = v[h] * inv_sigma;
-    val[h][1] = sv[h] * inv_sigma;
+  for (int t = 0; t < 2; ++t) {
+    float mx = fabsf(val[t]);
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      float mx = fabsf(val[h][t]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (lane == 0) red[0][h][t][warp] = mx;
-    }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[0][h][t][wg] = mx;
   }
   __syncthreads();
+  float lam[2];
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+  for (int t = 0; t < 2; ++t) {
+    const float mx = fmaxf(fmaxf(red[0][h][t][0], red[0][h][t][1]), fmaxf(red[0][h][t][2], red[0][h][t][3]));
+    lam[t] = fp16_range_scale(mx);
+    const float x2 = val[t] * lam[t];
+    const __half hi = __float2half_rn(x2);
+    const __half lo = __float2half_rn(x2 - __half2float(hi));
+    const int n = 2 * (h & 3);
+    qfrag[frag_at(t, h >> 2, n)] = __half_as_ushort(hi);
+    qfrag[frag_at(t, h >> 2, n + 1)] = __half_as_ushort(lo);
+    float c = mu * (__half2float(hi) + __half2float(lo));   // sum over dims of mu_p (hi + lo)
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const float mx = fmaxf(fmaxf(red[0][h][t][0], red[0][h][t][1]), fmaxf(red[0][h][t][2], red[0][h][t][3]));
-      const float lam = fp16_range_scale(mx);
-      const float x2 = val[h][t] * lam;
-      const __half hi = __float2half_rn(x2);
-      const __half lo = __float2half_rn(x2 - __half2float(hi));
-      const int n = 2 * (h & 3);
-      qfrag[frag_at(t, h >> 2, n)] = __half_as_ushort(hi);
-      qfrag[frag_at(t, h >> 2, n + 1)] = __half_as_ushort(lo);
-      float c = mu * (__half2float(hi) + __half2float(lo));   // sum over dims of mu_p (hi + lo)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-      if (lane == 0) red[1][h][t][warp] = c;
-      val[h][t] = lam;
-    }
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) red[1][h][t][wg] = c;
+  }
   if constexpr (2 * G < 8) {
+    if (h == 0) {
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
-      for (int n = 2 * G; n < 8; ++n) qfrag[frag_at(t, 0, n)] = 0;
+      for (int t = 0; t < 2; ++t)
+        for (int n = 2 * G; n < 8; ++n) qfrag[frag_at(t, 0, n)] = 0;
+    }
   }
   __syncthreads();
-  if (i < 2 * G) {
-    const int h = i >> 1, t = i & 1;
+  if (i < 2) {
+    const int t = i;
     const float c = (red[1][h][t][0] + red[1][h][t][1]) + (red[1][h][t][2] + red[1][h][t][3]);
-    kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] = make_float2(c, 1.0f / val[h][t]);
+    kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] = make_float2(c, 1.0f / lam[t]);
   }
 }
 
-// One block of kD threads per (sequence b, KV head), covering its G query
-// heads: log-sum-exp merge of the split partials, the QJL value correction
-// sqrt(pi/2)/m S^T O_z, and Pi^T.  Column i of S is loaded once, at the
-// start, for all G heads.  The split weights f_s = 2^(m_s - M) of each head
-// are formed by the lanes of one warp in parallel and staged in shared
-// memory (dynamic, n_splits * G floats), so that each thread's sums over
-// splits are plain independent loads.
+// One block of G groups of kD threads per (sequence b, KV head); group h is
+// query head h of the KV head, thread i of it coordinate i: log-sum-exp merge
+// of the split partials, the QJL value correction sqrt(pi/2)/m S^T O_z, and
+// Pi^T.  The product S^T O_z is split by rows of S instead of by heads: group
+// g holds rows [g kD/G, (g + 1) kD/G) of column i of S in registers (loaded
+// before the wait for the split kernel, so the loads overlap its tail) and
+// forms the partial sums of all G heads over them; the G partials meet in
+// shared memory.  The split weights f_s = 2^(m_s - M) of each head are formed
+// by the first warp of its group and staged in shared memory (dynamic,
+// n_splits * G floats), so each thread's sums over splits are plain loads.
 template <int G>
-__global__ void __launch_bounds__(kD) decode_merge_kernel(const float* __restrict__ partial, int n_splits,
-                                                         const float* __restrict__ s_mat, const float* __restrict__ dsigns,
-                                                         float qjl, float* __restrict__ out) {
+__global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __restrict__ partial, int n_splits,
+                                                             const float* __restrict__ s_mat,
+                                                             const float* __restrict__ dsigns, float qjl,
+                                                             float* __restrict__ out) {
   constexpr int REC = 2 + 2 * kD;
-  constexpr int W = kD / 32;
+  constexpr int KS = kD / G;   // rows of S per group
   __shared__ __align__(16) float oz[G][kD];
+  __shared__ __align__(16) float part[G][G][kD];   // [row group][head][i]
   __shared__ __align__(16) float buf[G][kD];
   __shared__ float Ls[G];
   extern __shared__ float fs[];   // [n_splits][G]
-  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int tid = threadIdx.x, h = tid / kD, i = tid % kD, lane = tid & 31;
   const int bh = blockIdx.x;
-  float scol[kD];
+  float scol[KS];
 #pragma unroll
-  for (int j = 0; j < kD; ++j) scol[j] = __ldg(s_mat + j * kD + i);
+  for (int j = 0; j < KS; ++j) scol[j] = __ldg(s_mat + (h * KS + j) * kD + i);
   asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the split kernel's partials
   const float* base = partial + static_cast<size_t>(bh) * n_splits * G * REC;
-  for (int h = warp; h < G; h += W) {
+  if (i < 32) {
     float M = -INFINITY;
     for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, base[(static_cast<size_t>(s) * G + h) * REC]);
 #pragma unroll
@@ -711,32 +689,32 @@ __global__ void __launch_bounds__(kD) decode_merge_kernel(const float* __restric
     if (lane == 0) Ls[h] = l;
   }
   __syncthreads();
-  float oc[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float c = 0.f, z = 0.f;
+  float c = 0.f, z = 0.f;
 #pragma unroll 4
-    for (int s = 0; s < n_splits; ++s) {
-      const float f = fs[s * G + h];
-      const float* rec = base + (static_cast<size_t>(s) * G + h) * REC;
-      c = fmaf(f, rec[2 + i], c);
-      z = fmaf(f, rec[2 + kD + i], z);
-    }
-    oc[h] = c;
-    oz[h][i] = z;
+  for (int s = 0; s < n_splits; ++s) {
+    const float f = fs[s * G + h];
+    const float* rec = base + (static_cast<size_t>(s) * G + h) * REC;
+    c = fmaf(f, rec[2 + i], c);
+    z = fmaf(f, rec[2 + kD + i], z);
+  }
+  oz[h][i] = z;
+  __syncthreads();
+  // partial S^T O_z of every head over this group's rows of S
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < KS; ++j) acc = fmaf(scol[j], oz[hh][h * KS + j], acc);
+    part[h][hh][i] = acc;
   }
   __syncthreads();
-  // rotated-space value: O_code + sqrt(pi/2)/m S^T O_z
-  float corr[G];
-  matvec_col<G>(scol, oz, corr);
-  float y[G];
+  float corr = 0.f;
 #pragma unroll
-  for (int h = 0; h < G; ++h) y[h] = Ls[h] > 0.f ? (oc[h] + qjl * corr[h]) / Ls[h] : 0.f;
-  // Pi^T y = D H y / sqrt(d)
-  fwht_block<G>(y, buf);
-  const float f = dsigns[i] * rsqrtf(static_cast<float>(kD));
-#pragma unroll
-  for (int h = 0; h < G; ++h) out[(static_cast<size_t>(bh) * G + h) * kD + i] = y[h] * f;
+  for (int g = 0; g < G; ++g) corr += part[g][h][i];
+  // rotated-space value: O_code + sqrt(pi/2)/m S^T O_z, then Pi^T y = D H y / sqrt(d)
+  float y = Ls[h] > 0.f ? (c + qjl * corr) / Ls[h] : 0.f;
+  fwht_group(y, i, buf[h]);
+  out[(static_cast<size_t>(bh) * G + h) * kD + i] = y * (dsigns[i] * rsqrtf(static_cast<float>(kD)));
 }
 
 thread_local cudaEvent_t g_prof_begin = nullptr;
@@ -814,7 +792,7 @@ template <typename T>
 void qprep_g(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope, uint16_t* qfrag,
              float2* kconst, cudaStream_t s) {
 #define TQ_QPREP(GG)                                                                                       \
-  launch_pdl(decode_qprep_kernel<T, GG>, dim3(BH), dim3(kD), 0, s, q, q_pos, Hkv, hk->d_signs, hk->d_st,        \
+  launch_pdl(decode_qprep_kernel<T, GG>, dim3(BH), dim3(kD * GG), 0, s, q, q_pos, Hkv, hk->d_signs, hk->d_st,        \
              hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope, qfrag, kconst)
   switch (G) {
     case 1: TQ_QPREP(1); break;
@@ -838,10 +816,10 @@ int launch_merge(int G, int BH, const float* partial, int n_splits, const tq_rot
   const float qjl = static_cast<float>(kQjlConst / hv->m);
   const size_t fsb = static_cast<size_t>(n_splits) * G * sizeof(float);   // <= 1184 * 8 * 4 bytes
   switch (G) {
-    case 1: return launch_pdl(decode_merge_kernel<1>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
-    case 2: return launch_pdl(decode_merge_kernel<2>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
-    case 4: return launch_pdl(decode_merge_kernel<4>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
-    case 8: return launch_pdl(decode_merge_kernel<8>, dim3(BH), dim3(kD), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 1: return launch_pdl(decode_merge_kernel<1>, dim3(BH), dim3(kD * 1), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 2: return launch_pdl(decode_merge_kernel<2>, dim3(BH), dim3(kD * 2), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 4: return launch_pdl(decode_merge_kernel<4>, dim3(BH), dim3(kD * 4), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 8: return launch_pdl(decode_merge_kernel<8>, dim3(BH), dim3(kD * 8), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
     default: return TQ_EUNSUPPORTED;
   }
   return tq::launch_status();
