@@ -434,15 +434,14 @@ def run_ours(args, rank, world, local_rank):
             nk = nks[layer] if src is None else src[0][layer]
             nv = nvs[layer] if src is None else src[1][layer]
             q = qs[layer] if src is None else src[2][layer]
-            tq.quantize_kv(rks[layer], nk, apply_rope=True, pos_period=1, pos_offset=T - 1,
-                           out=slot(kcs[layer]), out_stride=T)
-            tq.quantize_kv(rvs[layer], nv, out=slot(vcs[layer]), out_stride=T)
+            tq.quantize_kv_pair(rks[layer], nk, rvs[layer], nv, apply_rope=True, pos_period=1, pos_offset=T - 1,
+                                out_k=slot(kcs[layer]), out_v=slot(vcs[layer]), out_stride=T)
             if prof is not None:
                 tq.profile_next_decode(*prof[layer])
             tq.decode_attention(rks[layer], rvs[layer], q, qpos, kcs[layer], vcs[layer], T, out=outs[layer],
                                 workspace=ws)
 
-    launches_per_step = L * (2 + 3)
+    launches_per_step = L * (1 + 3)
     dist = None
     if world > 1:
         import torch.distributed as dist

@@ -187,6 +187,23 @@ int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, int64_t n,
                    void* stream);
 
 /*
+ * tq_quantize_kv_pair - the keys and values one decode step appends, in one
+ * call: n rows of xk with handle hk (RoPE as in tq_quantize_kv, with pos /
+ * pos_period / pos_offset / apply_rope) and n rows of xv with handle hv
+ * (never RoPE), both of `dtype` with row stride ld, written to record
+ * i * out_stride of the K and V arrays.  Records are identical to two
+ * tq_quantize_kv calls.  For n <= 256 with equal d and bits both sets are
+ * encoded by one launch; otherwise the two calls run in order.
+ * Returns TQ_OK, TQ_EINVAL or TQ_EUNSUPPORTED as tq_quantize_kv.
+ */
+int tq_quantize_kv_pair(const tq_rotation* hk, const void* xk, const tq_rotation* hv,
+                        const void* xv, int dtype, int64_t n, int64_t ld,
+                        const int64_t* pos, int64_t pos_period, int64_t pos_offset,
+                        int apply_rope, uint8_t* k_codes, uint8_t* k_signs,
+                        float* k_norms, uint8_t* v_codes, uint8_t* v_signs,
+                        float* v_norms, int64_t out_stride, void* stream);
+
+/*
  * tq_quantize_dense - encode n vectors with a dense-rotation handle
  * (TQ_ROT_DENSE).  Same steps and record format as tq_quantize_kv, without
  * RoPE; y = Pi x and S r are dense contractions here, computed as fp32 GEMMs

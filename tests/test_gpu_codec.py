@@ -203,3 +203,28 @@ def test_encode_70b_slice_full_size_sampled(cuda_device):
         _, _, _, enc = oracle_records(o, xs, (rows % T).astype(np.int64) if apply_rope else None)
         compare_records(o, gpu, enc)
         del x, out
+
+
+@pytest.mark.parametrize("n", [1, 128, 256, 300])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_kv_pair_equals_two_calls(cuda_device, n, dtype):
+    """The decode-step append call (keys with RoPE, values without, one launch
+    up to 256 rows) writes the same records as two tq_quantize_kv calls."""
+    from vector_quantization_b200 import tq
+    dev = cuda_device_of()
+    rk = _gpu_rot(128, 2, 260, rope=10000.0)
+    rv = _gpu_rot(128, 2, 261)
+    k = torch.from_numpy(synth.heavy_tailed((n, 128), 262)).to(dev).to(dtype)
+    v = torch.from_numpy(synth.heavy_tailed((n, 128), 263)).to(dev).to(dtype)
+    stride = 3
+    kw = dict(apply_rope=True, pos_period=n, pos_offset=(1 << 20) - n)
+    pk, pv = tq.empty_records(rk, (n * stride,), dev), tq.empty_records(rv, (n * stride,), dev)
+    sk, sv = tq.empty_records(rk, (n * stride,), dev), tq.empty_records(rv, (n * stride,), dev)
+    for t in (*pk, *pv, *sk, *sv):
+        t.zero_()
+    tq.quantize_kv_pair(rk, k, rv, v, out_k=pk, out_v=pv, out_stride=stride, **kw)
+    tq.quantize_kv(rk, k, out=sk, out_stride=stride, **kw)
+    tq.quantize_kv(rv, v, out=sv, out_stride=stride)
+    torch.cuda.synchronize()
+    for a, b in zip((*pk, *pv), (*sk, *sv)):
+        assert torch.equal(a, b)

@@ -59,7 +59,7 @@ constexpr int kWaitLimit = 1 << 17;   // polls of about 9 us each: a wait gives 
 // of S loaded into registers at the start (so its loads overlap the rest).
 // ===========================================================================
 template <int D, int BITS, typename T>
-__global__ void __launch_bounds__(D) encode_vec_kernel(EncodeParams p) {
+__device__ __forceinline__ void encode_vec_body(const EncodeParams& p) {
   constexpr int NW = D / 32;
   __shared__ __align__(16) float buf[D];
   __shared__ float red[2][NW];
@@ -168,6 +168,20 @@ __global__ void __launch_bounds__(D) encode_vec_kernel(EncodeParams p) {
     for (int q = 0; q < NW; ++q) rr += red[1][q];
     p.norms[rec] = make_float2(nrm, sqrtf(rr));
   }
+}
+
+template <int D, int BITS, typename T>
+__global__ void __launch_bounds__(D) encode_vec_kernel(const __grid_constant__ EncodeParams p) {
+  encode_vec_body<D, BITS, T>(p);
+}
+
+// The same for two row sets of equal count, d and bits in one launch (the
+// keys and values a decode step appends): blockIdx.y picks the set.
+template <int D, int BITS, typename T>
+__global__ void __launch_bounds__(D) encode_vec_pair_kernel(const __grid_constant__ EncodeParams pk,
+                                                           const __grid_constant__ EncodeParams pv) {
+  if (blockIdx.y == 0) encode_vec_body<D, BITS, T>(pk);
+  else encode_vec_body<D, BITS, T>(pv);
 }
 
 // Batches up to this many vectors take the block-per-vector kernel.
@@ -1247,6 +1261,30 @@ int launch_encode(const EncodeParams& p, cudaStream_t stream) {
   return launch_encode_rows<D, BITS, T>(p, stream);
 }
 
+template <int D, int BITS, typename T>
+int launch_encode_vec_pair(const EncodeParams& pk, const EncodeParams& pv, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pk.n), 2);
+  cfg.blockDim = dim3(D);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, encode_vec_pair_kernel<D, BITS, T>, pk, pv) == cudaSuccess ? TQ_OK : TQ_ECUDA;
+}
+
+template <int D, typename T>
+int dispatch_vec_pair(int bits, const EncodeParams& pk, const EncodeParams& pv, cudaStream_t s) {
+  switch (bits) {
+    case 1: return launch_encode_vec_pair<D, 1, T>(pk, pv, s);
+    case 2: return launch_encode_vec_pair<D, 2, T>(pk, pv, s);
+    case 3: return launch_encode_vec_pair<D, 3, T>(pk, pv, s);
+  }
+  return TQ_EUNSUPPORTED;
+}
+
 template <int D, typename T>
 int dispatch_bits(int bits, const EncodeParams& p, cudaStream_t s) {
   switch (bits) {
@@ -1259,13 +1297,14 @@ int dispatch_bits(int bits, const EncodeParams& p, cudaStream_t s) {
 
 }  // namespace
 
-extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, int64_t n, int64_t ld,
-                              const int64_t* pos, int64_t pos_period, int64_t pos_offset,
-                              int apply_rope, uint8_t* codes, uint8_t* signs, float* norms,
-                              int64_t out_stride, void* stream) {
+namespace {
+
+// Checks of one tq_quantize_kv call and its kernel parameters.
+int make_encode_params(const tq_rotation* h, const void* x, int dtype, int64_t n, int64_t ld, const int64_t* pos,
+                       int64_t pos_period, int64_t pos_offset, int apply_rope, uint8_t* codes, uint8_t* signs,
+                       float* norms, int64_t out_stride, EncodeParams* out) {
   if (!h) return TQ_EINVAL;
   if (n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_EINVAL;
-  if (n == 0) return TQ_OK;
   if (!x || !codes || !signs || !norms || out_stride < 1 || ld < h->d) return TQ_EINVAL;
   if ((reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(signs) & 3u) ||
       (reinterpret_cast<uintptr_t>(norms) & 7u))
@@ -1313,10 +1352,56 @@ extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, in
   p.rope_lo = h->d_rope_lo;
   p.rope_max_pos = h->rope_max_pos;
   for (int i = 0; i < 64; ++i) p.theta[i] = make_float2(h->rope_th_hi[i], h->rope_th_lo[i]);
+  *out = p;
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" int tq_quantize_kv(const tq_rotation* h, const void* x, int dtype, int64_t n, int64_t ld,
+                              const int64_t* pos, int64_t pos_period, int64_t pos_offset,
+                              int apply_rope, uint8_t* codes, uint8_t* signs, float* norms,
+                              int64_t out_stride, void* stream) {
+  if (!h) return TQ_EINVAL;
+  if (n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_EINVAL;
+  if (n == 0) return TQ_OK;
+  EncodeParams p{};
+  const int st = make_encode_params(h, x, dtype, n, ld, pos, pos_period, pos_offset, apply_rope, codes, signs, norms,
+                                    out_stride, &p);
+  if (st != TQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (h->d == 128)
     return dtype == TQ_F32 ? dispatch_bits<128, float>(h->bits, p, s) : dispatch_bits<128, __nv_bfloat16>(h->bits, p, s);
   if (h->d == 64)
     return dtype == TQ_F32 ? dispatch_bits<64, float>(h->bits, p, s) : dispatch_bits<64, __nv_bfloat16>(h->bits, p, s);
   return TQ_EUNSUPPORTED;
+}
+
+extern "C" int tq_quantize_kv_pair(const tq_rotation* hk, const void* xk, const tq_rotation* hv, const void* xv,
+                                   int dtype, int64_t n, int64_t ld, const int64_t* pos, int64_t pos_period,
+                                   int64_t pos_offset, int apply_rope, uint8_t* k_codes, uint8_t* k_signs,
+                                   float* k_norms, uint8_t* v_codes, uint8_t* v_signs, float* v_norms,
+                                   int64_t out_stride, void* stream) {
+  if (!hk || !hv) return TQ_EINVAL;
+  if (n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_EINVAL;
+  if (n == 0) return TQ_OK;
+  EncodeParams pk{}, pv{};
+  int st = make_encode_params(hk, xk, dtype, n, ld, pos, pos_period, pos_offset, apply_rope, k_codes, k_signs,
+                              k_norms, out_stride, &pk);
+  if (st != TQ_OK) return st;
+  if ((st = make_encode_params(hv, xv, dtype, n, ld, nullptr, 1, 0, 0, v_codes, v_signs, v_norms, out_stride, &pv)) !=
+      TQ_OK)
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n <= kVecKernelMaxN && hk->d == hv->d && hk->bits == hv->bits && (hk->d == 128 || hk->d == 64)) {
+    if (hk->d == 128)
+      return dtype == TQ_F32 ? dispatch_vec_pair<128, float>(hk->bits, pk, pv, s)
+                             : dispatch_vec_pair<128, __nv_bfloat16>(hk->bits, pk, pv, s);
+    return dtype == TQ_F32 ? dispatch_vec_pair<64, float>(hk->bits, pk, pv, s)
+                           : dispatch_vec_pair<64, __nv_bfloat16>(hk->bits, pk, pv, s);
+  }
+  st = tq_quantize_kv(hk, xk, dtype, n, ld, pos, pos_period, pos_offset, apply_rope, k_codes, k_signs, k_norms,
+                      out_stride, stream);
+  if (st != TQ_OK) return st;
+  return tq_quantize_kv(hv, xv, dtype, n, ld, nullptr, 1, 0, 0, v_codes, v_signs, v_norms, out_stride, stream);
 }

@@ -42,6 +42,8 @@ def _load():
         "tq_rotation_export": (c_i, [c_p, c_p, c_p, c_p, c_p]),
         "tq_rotation_dims": (c_i, [c_p, c_p, c_p, c_p, c_p, c_p]),
         "tq_quantize_kv": (c_i, [c_p, c_p, c_i, c_i64, c_i64, c_p, c_i64, c_i64, c_i, c_p, c_p, c_p, c_i64, c_p]),
+        "tq_quantize_kv_pair": (c_i, [c_p, c_p, c_p, c_p, c_i, c_i64, c_i64, c_p, c_i64, c_i64, c_i,
+                                      c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_p]),
         "tq_decode_attention": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
                                       c_i64, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
@@ -202,6 +204,34 @@ def quantize_kv(rot: Rotation, x, *, pos=None, pos_period: int | None = None, po
                                1 if apply_rope else 0, _ptr(codes), _ptr(signs), _ptr(norms), out_stride,
                                _stream_ptr(stream)), "tq_quantize_kv")
     return codes, signs, norms
+
+
+def quantize_kv_pair(rot_k: Rotation, xk, rot_v: Rotation, xv, *, pos=None, pos_period: int | None = None,
+                     pos_offset: int = 0, apply_rope: bool = False, out_k=None, out_v=None, out_stride: int = 1,
+                     stream=None):
+    """Encode the keys ``xk`` (RoPE as in :func:`quantize_kv`) and values
+    ``xv`` (no RoPE) a decode step appends, in one call; both [n, d] or
+    [..., d] of one dtype and row stride.  Returns ((k records), (v records))."""
+    d = xk.shape[-1]
+    k2, v2 = xk.reshape(-1, d), xv.reshape(-1, d)
+    if k2.stride(-1) != 1 or v2.stride(-1) != 1:
+        raise ValueError("x rows must be contiguous")
+    if k2.shape != v2.shape or k2.dtype != v2.dtype or k2.stride(0) != v2.stride(0):
+        raise ValueError("keys and values must share shape, dtype and row stride")
+    n = k2.shape[0]
+    ld = k2.stride(0) if n > 1 else d
+    if out_k is None:
+        out_k = empty_records(rot_k, xk.shape[:-1], xk.device)
+    if out_v is None:
+        out_v = empty_records(rot_v, xv.shape[:-1], xv.device)
+    if pos is not None and pos.dtype.is_floating_point:
+        raise TypeError("pos must be int64")
+    period = pos_period if pos_period is not None else max(n, 1)
+    _check(_lib.tq_quantize_kv_pair(rot_k.handle, _ptr(k2), rot_v.handle, _ptr(v2), _dtype_code(k2), n, ld, _ptr(pos),
+                                    period, pos_offset, 1 if apply_rope else 0, _ptr(out_k[0]), _ptr(out_k[1]),
+                                    _ptr(out_k[2]), _ptr(out_v[0]), _ptr(out_v[1]), _ptr(out_v[2]), out_stride,
+                                    _stream_ptr(stream)), "tq_quantize_kv_pair")
+    return out_k, out_v
 
 
 def profile_next_decode(ev_begin, ev_end):
