@@ -288,7 +288,7 @@ def _extra_encoder(dev, g):
     ms = _time_ms(lambda: tq.encoder_attention(rk, rv, q, kc, vc, T, out=o, workspace=ws))
     flops = 2 * B * H * T * T * 2 * (d + d)
     out["encoder_esm2_layer"] = {"ms": round(ms, 4), "TFLOP_s": round(flops / ms / 1e9, 1), "algorithmic_flops": flops,
-                                 "note": "2 B H S T (d + m) MACs for scores and for values; mma.sync tensor pipe"}
+                                 "note": "2 B H S T (d + m) MACs for scores and for values; tcgen05 tensor core (d = 64, 1-2 bit codes)"}
     return out
 
 

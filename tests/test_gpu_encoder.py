@@ -64,6 +64,14 @@ def test_encoder_gqa_bf16_offset(cuda_device):
     assert_close(gpu, ref)
 
 
+@pytest.mark.parametrize("bits", [1, 2])
+def test_encoder_gqa_d64_several_query_tiles(cuda_device, bits):
+    # d = 64: four query heads on two KV heads, 300 queries (three 128-query
+    # tiles, the last ragged) against 161 keys (an odd number of 32-key tiles)
+    gpu, ref = run(64, bits, 1, 4, 2, 300, 161, seed=11 + bits, q_dtype=torch.bfloat16, q_off=7)
+    assert_close(gpu, ref, what=f"bits={bits}")
+
+
 def test_encoder_empty_cache(cuda_device):
     from vector_quantization_b200 import tq
     dev = torch.device("cuda:0")

@@ -23,6 +23,7 @@
 #include <cmath>
 
 #include "bitplane.cuh"
+#include "tcgen05.cuh"
 #include "tq_internal.h"
 
 namespace {
@@ -471,6 +472,542 @@ __global__ void __launch_bounds__(kWarps * 32, D == 64 ? 3 : 1) encoder_attentio
   }
 }
 
+// ===========================================================================
+// Encoder attention on the tensor core (d = 64, 1- and 2-bit codes).
+//
+// Every key and value tile serves all 128 queries of a CTA, so its bit planes
+// are expanded once per tile into exact +-1 operands in shared memory and the
+// two products run as tcgen05 MMAs with fp32 accumulators in tensor memory:
+//   scores  D_p[q][key] = sum_slot  A[q][slot] * Kop_p[key][slot]
+//           (A = q~ for the code planes, S q~ for the sign plane, as fp16 hi
+//           and lo pieces of a per-row power-of-two scaling, both pieces
+//           accumulating into the same D; keys as fp16 +-1)
+//   values  O_code[q][slot] += sum_(p,key) (P ||v|| w_p)[q][(p,key)] * Vop_p[key][slot]
+//           O_z[q][slot]    += sum_key     (P ||r_v||)[q][key]        * Vop_z[key][slot]
+//           (bf16 hi and lo pieces of the weights against bf16 +-1 values)
+// One shift and one LOP3 put bits b and b + 16 of a plane word into one
+// 32-bit operand word, so slot k stands for coordinate
+// dim(k) = 32 (k / 32) + (k / 2) % 16 + 16 (k % 2) in the queries, keys,
+// values and output columns alike; the epilogue undoes it.  The key operand
+// (K-major, a row per key) and the value operand (MN-major, a row per key)
+// share one physical layout.
+//
+// A CTA owns 128 queries of one head.  16 worker warps, four threads per
+// query row (tensor-memory lane): warp w reads lane quarter w % 4 and keys
+// 8 (w / 4) .. + 7 of each 32-key tile; the quarters exchange their tile
+// maxima through shared memory.  A 17th warp only issues the MMAs: it waits
+// on mbarriers the workers arrive on (operands expanded, probabilities
+// written) and commits the products to mbarriers the workers wait on, so the
+// issue of the MMAs never holds up a worker barrier.  The loop is
+// software-pipelined over tiles: while the workers run the softmax of tile
+// i, the tensor core computes the scores of tile i + 1 (two score buffers in
+// tensor memory, two key and value operand buffers in shared memory), and
+// the packed records of tile i + 2 are in flight (cp.async).  Every wait is
+// bounded; the rows of a CTA whose wait ran out are written as NaN (after a
+// failed wait the MMA warp stops issuing but still commits, so no wait of
+// the workers is left without its arrival).
+// ===========================================================================
+constexpr int kTcQ = 128;               // queries per CTA
+constexpr int kTcKeys = 32;             // keys per tile
+constexpr int kTcWorkers = 512;         // 16 worker warps, four threads per query row
+constexpr int kTcThreads = kTcWorkers + 32;   // and the MMA warp
+constexpr int kTcWait = 1 << 17;        // polls of about 9 us each
+constexpr int kTcOpQ = kTcQ * 128;      // one [128 x 64] 16-bit operand: 16 KB
+constexpr int kTcOpK = kTcKeys * 128;   // one [32 x 64] 16-bit operand: 4 KB
+constexpr int kTcXStride = 129;         // floats per row of the epilogue buffer
+constexpr uint32_t kTcColO = 256;       // tensor-memory columns: scores 0..191 (two buffers), O 256..383
+
+template <int BITS>
+__host__ __device__ constexpr int tc_kv_bytes() {
+  return 2 * (Planes<BITS>::P + 1) * kTcOpK;   // key and value operands of one tile
+}
+template <int BITS>
+__host__ __device__ constexpr int tc_stage_bytes() {
+  return 2 * kTcKeys * (BITS * 8 + 8 + 8);   // K and V sides of one staged tile (d = 64)
+}
+template <int BITS>
+constexpr size_t tc_smem_bytes() {
+  return 1024 + 4 * kTcOpQ + 2 * tc_kv_bytes<BITS>() + 3 * kTcOpQ + 2 * tc_stage_bytes<BITS>();
+}
+
+// slot k of an operand row -> coordinate
+__host__ __device__ constexpr int tc_slot_dim(int k) { return 32 * (k >> 5) + ((k >> 1) & 15) + 16 * (k & 1); }
+
+// byte offset of 16-byte chunk j of row r in a 128-byte swizzled operand
+__device__ __forceinline__ uint32_t tc_chunk_off(int r, int j) {
+  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
+}
+
+// 8 consecutive slots as fp16 hi and lo pieces: hi = RN(x), lo = RN(x - hi)
+__device__ __forceinline__ void tc_split8_h(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __half2 hh = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
+    const float2 hf = __half22float2(hh);
+    const __half2 ll = __floats2half2_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
+    h[e] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[e] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// 8 consecutive slots as bf16 hi and lo pieces: hi = RN(x), lo = RN(x - hi)
+__device__ __forceinline__ void tc_split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+    h[e] = *reinterpret_cast<uint32_t*>(&hh);
+    const float2 d = __ffma2_rn(make_float2(__uint_as_float(h[e] << 16), __uint_as_float(h[e] & 0xFFFF0000u)),
+                                make_float2(-1.f, -1.f), make_float2(x[2 * e], x[2 * e + 1]));
+    __nv_bfloat162 ll = __floats2bfloat162_rn(d.x, d.y);
+    l[e] = *reinterpret_cast<uint32_t*>(&ll);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_constant__ EncParams p) {
+  constexpr int D = 64;
+  constexpr int P = Planes<BITS>::P;
+  constexpr int CB = BITS * D / 8, SB = D / 8;
+  constexpr int HALF = kTcKeys * (CB + SB + 8);
+  constexpr int STG = 2 * HALF;
+  constexpr int KV = tc_kv_bytes<BITS>();
+  static_assert(P <= 2, "code planes of at most 2 bits");
+  extern __shared__ uint8_t raw[];
+  __shared__ uint64_t mb_s[2], mb_pv, mb_kv, mb_p;   // products done; operands / probabilities ready
+  __shared__ uint32_t tmem_slot;
+  __shared__ int s_fail;
+  __shared__ float s_inv_lam[2][kTcQ];        // per query row: 1 / range scale of q~ (0) and S q~ (1)
+  __shared__ float s_mx[4][kTcQ];             // per key quarter, query row: tile maximum of the logits
+  __shared__ float2 s_kf[2][kTcKeys];         // per tile buffer, key: (||k||, ||r_k|| qjl_k) x score scale
+  __shared__ float4 s_vf[2][kTcKeys];         // per tile buffer, key: (||v|| w_0, ||v|| w_1, ||r_v||, 0)
+  uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kq = warp >> 2;                   // key quarter of this thread in the softmax
+  const int row = 32 * (warp & 3) + lane;     // query row = tensor-memory lane
+  uint8_t* aq_hi = base;                      // q~ pieces (rows = queries)
+  uint8_t* aq_lo = base + kTcOpQ;
+  uint8_t* as_hi = base + 2 * kTcOpQ;         // S q~ pieces
+  uint8_t* as_lo = base + 3 * kTcOpQ;
+  uint8_t* kvb = base + 4 * kTcOpQ;           // two buffers: key operand planes, then value operand rows
+  uint8_t* ac_hi = kvb + 2 * KV;              // rows = queries, slots (pl, key)
+  uint8_t* ac_lo = ac_hi + kTcOpQ;
+  uint8_t* az = ac_lo + kTcOpQ;               // slots key: hi piece, 32 + key: lo piece
+  uint8_t* stg = az + kTcOpQ;                 // two staged tiles
+
+  const int bq = blockIdx.y;
+  const int b = bq / p.Hq, h = bq % p.Hq;
+  const int bh = b * (p.Hq / p.G) + h / p.G;
+  const int q0 = blockIdx.x * kTcQ;
+  const int64_t seq = static_cast<int64_t>(bh) * p.cache_stride;
+  const int n_tiles = static_cast<int>((p.T + kTcKeys - 1) / kTcKeys);
+
+  const bool mma_warp = warp == kTcWorkers / 32;
+  if (tid == 0) {
+    tqtc::mbar_init(&mb_s[0], 1);
+    tqtc::mbar_init(&mb_s[1], 1);
+    tqtc::mbar_init(&mb_pv, 1);
+    tqtc::mbar_init(&mb_kv, kTcWorkers);
+    tqtc::mbar_init(&mb_p, kTcWorkers);
+    s_fail = 0;
+  }
+  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, 512);
+
+  auto issue = [&](int t) {   // stage tile t into buffer t & 1
+    if (t < n_tiles) {
+      const int64_t t0 = static_cast<int64_t>(t) * kTcKeys;
+      const int nv = static_cast<int>(p.T - t0 < kTcKeys ? p.T - t0 : kTcKeys);
+      uint8_t* dst = stg + (t & 1) * STG;
+      for (int c = tid; c < STG / 16; c += kTcWorkers) {
+        const int side = c >= STG / 32;
+        const int off = (c - side * (STG / 32)) * 16;   // byte offset inside this side
+        const uint8_t* src_base;
+        int rec, region;
+        if (off < kTcKeys * CB) {
+          src_base = side ? p.v_codes : p.k_codes;
+          rec = CB;
+          region = 0;
+        } else if (off < kTcKeys * (CB + SB)) {
+          src_base = side ? p.v_signs : p.k_signs;
+          rec = SB;
+          region = kTcKeys * CB;
+        } else {
+          src_base = reinterpret_cast<const uint8_t*>(side ? p.v_norms : p.k_norms);
+          rec = 8;
+          region = kTcKeys * (CB + SB);
+        }
+        const int inreg = off - region;
+        const int bytes = max(0, min(16, nv * rec - inreg));
+        const uint8_t* src = src_base + (seq + t0) * rec + inreg;
+        cp_async16(dst + side * HALF + off, bytes ? src : src_base, bytes);
+      }
+    }
+    cp_async_commit();
+  };
+  if (!mma_warp) {
+    issue(0);
+    issue(1);
+  }
+
+  // ---- query operands: thread (row, kq) writes slots 16 kq .. 16 kq + 15 of
+  // q~ (kq < 2) or S q~ (kq >= 2) as fp16 hi and lo pieces of x * lam, lam a
+  // power of two bringing the row's max |x| into [2^13, 2^14) (about 22
+  // significant bits); the key operand is fp16 too
+  if (!mma_warp) {
+    const int q = q0 + row, type = kq >> 1, half = kq & 1;
+    float v[32];   // coordinates 32 half .. 32 half + 31
+    float mx = 0.f;
+    if (q < p.S) {
+      const float4* src =
+          reinterpret_cast<const float4*>(p.qprep + ((static_cast<int64_t>(bq) * p.S + q) * 2 + type) * D);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 f = src[8 * half + i];
+        v[4 * i] = f.x;
+        v[4 * i + 1] = f.y;
+        v[4 * i + 2] = f.z;
+        v[4 * i + 3] = f.w;
+        const float4 o = src[8 * (1 - half) + i];
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(v[i]));
+    const float lam = fp16_range_scale(mx);
+    if (half == 0) s_inv_lam[type][row] = 1.f / lam;
+    uint8_t* dhi = type ? as_hi : aq_hi;
+    uint8_t* dlo = type ? as_lo : aq_lo;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float x[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = v[tc_slot_dim(8 * j + e)] * lam;   // slot 32 half + 8 j + e
+      uint4 hi, lo;
+      tc_split8_h(x, hi, lo);
+      *reinterpret_cast<uint4*>(dhi + tc_chunk_off(row, 4 * half + j)) = hi;
+      *reinterpret_cast<uint4*>(dlo + tc_chunk_off(row, 4 * half + j)) = lo;
+    }
+  }
+
+  // ---- expansion of tile t (staged in buffer t & 1) into operand buffer t & 1:
+  // thread -> key tid / 16, side (tid / 8) % 2, chunk tid % 8 of every plane
+  const int xkey = tid >> 4, xside = (tid >> 3) & 1, xj = tid & 7;
+  auto expand = [&](int t) {
+    const uint8_t* sd = stg + (t & 1) * STG + xside * HALF;
+    uint32_t rw[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) rw[k] = reinterpret_cast<const uint32_t*>(sd + xkey * CB + k * (D / 8))[xj >> 2];
+    uint32_t pw[P + 1];
+    {
+      uint32_t pl[P];
+      Planes<BITS>::make(rw, pl);
+#pragma unroll
+      for (int q = 0; q < P; ++q) pw[q] = pl[q];
+    }
+    pw[P] = reinterpret_cast<const uint32_t*>(sd + kTcKeys * CB + xkey * SB)[xj >> 2];
+    const uint32_t one = xside ? 0x3F803F80u : 0x3C003C00u;   // +1 in both halves: bf16 values, fp16 keys
+    uint8_t* dst = kvb + (t & 1) * KV + xside * (P + 1) * kTcOpK;
+#pragma unroll
+    for (int pl = 0; pl <= P; ++pl) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t s = pw[pl] << (15 - (4 * (xj & 3) + e));
+        w4[e] = (~s & 0x80008000u) | one;
+      }
+      *reinterpret_cast<uint4*>(dst + pl * kTcOpK + tc_chunk_off(xkey, xj)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    if (tid < kTcKeys) {
+      const uint8_t* s0 = stg + (t & 1) * STG;
+      const float2 kn = reinterpret_cast<const float2*>(s0 + kTcKeys * (CB + SB))[tid];
+      const float2 vn = reinterpret_cast<const float2*>(s0 + HALF + kTcKeys * (CB + SB))[tid];
+      s_kf[t & 1][tid] = make_float2(kn.x * p.score_scale, kn.y * p.qjl_k * p.score_scale);
+      s_vf[t & 1][tid] = make_float4(vn.x * p.walsh_v[0], vn.x * p.walsh_v[1], vn.y, 0.f);
+    }
+  };
+
+  tqtc::fence_smem_to_async();
+  tqtc::fence_before_sync();
+  __syncthreads();
+  tqtc::fence_after_sync();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);   // this warp's lanes
+  // descriptors (the leader issues): a k step adds 32 bytes along K (2 units),
+  // an MN-major k step 16 rows (2048 bytes, 128 units)
+  const uint64_t dq_hi = tqtc::sw128_desc(tqtc::smem_u32(aq_hi)), dq_lo = tqtc::sw128_desc(tqtc::smem_u32(aq_lo));
+  const uint64_t ds_hi = tqtc::sw128_desc(tqtc::smem_u32(as_hi)), ds_lo = tqtc::sw128_desc(tqtc::smem_u32(as_lo));
+  const uint64_t dkv = tqtc::sw128_desc(tqtc::smem_u32(kvb)), dkv_mn = tqtc::sw128_desc_mn(tqtc::smem_u32(kvb));
+  const uint64_t dc_hi = tqtc::sw128_desc(tqtc::smem_u32(ac_hi)), dc_lo = tqtc::sw128_desc(tqtc::smem_u32(ac_lo));
+  const uint64_t dz = tqtc::sw128_desc(tqtc::smem_u32(az));
+  auto issue_scores = [&](int t) {   // D[t & 1] = q pieces x key operand of tile t
+    constexpr uint32_t idesc = tqtc::idesc_f16_f32(kTcQ, kTcKeys);
+    const uint32_t dcol = tmem + 96 * (t & 1);
+    const uint64_t kb = dkv + static_cast<uint64_t>(((t & 1) * KV) >> 4);
+#pragma unroll
+    for (int pl = 0; pl <= P; ++pl) {
+      const uint64_t a_hi = pl < P ? dq_hi : ds_hi, a_lo = pl < P ? dq_lo : ds_lo;
+      const uint64_t bk = kb + static_cast<uint64_t>((pl * kTcOpK) >> 4);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) tqtc::mma_bf16_ss(dcol + 32 * pl, a_hi + 2 * ks, bk + 2 * ks, idesc, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) tqtc::mma_bf16_ss(dcol + 32 * pl, a_lo + 2 * ks, bk + 2 * ks, idesc, true);
+    }
+  };
+  auto issue_values = [&](int t) {   // O += probability operands x value operand of tile t
+    constexpr uint32_t idesc = tqtc::idesc_bf16_f32(kTcQ, D) | tqtc::kIdescBMajorMN;
+    const bool acc = t > 0;
+    const uint64_t vc = dkv_mn + static_cast<uint64_t>(((t & 1) * KV + (P + 1) * kTcOpK) >> 4);
+    const uint64_t vz = vc + static_cast<uint64_t>((P * kTcOpK) >> 4);
+    const uint32_t ocode = tmem + kTcColO, oz = tmem + kTcColO + 64;
+#pragma unroll
+    for (int ks = 0; ks < 2 * P; ++ks) tqtc::mma_bf16_ss(ocode, dc_hi + 2 * ks, vc + 128 * ks, idesc, acc || ks > 0);
+#pragma unroll
+    for (int ks = 0; ks < 2 * P; ++ks) tqtc::mma_bf16_ss(ocode, dc_lo + 2 * ks, vc + 128 * ks, idesc, true);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) tqtc::mma_bf16_ss(oz, dz + 2 * ks, vz + 128 * (ks & 1), idesc, acc || ks > 0);
+  };
+
+  if (mma_warp) {
+    // ---- MMA issue: scores of tile t + 1 as soon as its operands are
+    // expanded, values of tile t as soon as its probabilities are written
+    if (lane == 0) {
+      bool mok = true;
+      auto ready = [&](uint64_t* mb, int t) {
+        mok = mok && s_fail == 0 && tqtc::mbar_wait(mb, t & 1, kTcWait);
+        if (!mok) s_fail = 1;
+        tqtc::fence_after_sync();
+        return mok;
+      };
+      if (n_tiles > 0) {
+        if (ready(&mb_kv, 0)) issue_scores(0);
+        tqtc::mma_commit(&mb_s[0]);
+      }
+      for (int t = 0; t < n_tiles; ++t) {
+        if (t + 1 < n_tiles) {
+          if (ready(&mb_kv, t + 1)) issue_scores(t + 1);
+          tqtc::mma_commit(&mb_s[(t + 1) & 1]);
+        }
+        if (ready(&mb_p, t)) issue_values(t);
+        tqtc::mma_commit(&mb_pv);
+      }
+    }
+    __syncwarp();
+  } else {
+
+  auto work_sync = [&]() { asm volatile("bar.sync 1, %0;\n" ::"n"(kTcWorkers) : "memory"); };
+  // prologue: tile 0 expanded
+  bool ok = true;
+  if (n_tiles > 0) {
+    cp_async_wait<1>();
+    work_sync();
+    expand(0);
+    tqtc::fence_smem_to_async();
+    tqtc::fence_before_sync();
+    tqtc::mbar_arrive(&mb_kv);
+  }
+  float m_run = -INFINITY, l_run = 0.f;
+  uint32_t ph_s0 = 0, ph_s1 = 0, ph_pv = 0;
+  bool pv_pending = false;   // value products issued and not yet waited for (CTA-uniform)
+#pragma unroll 1
+  for (int it = 0; it < n_tiles; ++it) {
+    const bool has_next = it + 1 < n_tiles;
+    cp_async_wait<0>();
+    work_sync();   // tile it + 1 is staged; buffer it & 1 of the staging is free
+    issue(it + 2);
+    // the previous value products read the value operand and probability
+    // buffers that are rewritten below (the MMA warp commits even after a
+    // failure, so these waits always end)
+    if (pv_pending) {
+      ok = tqtc::mbar_wait(&mb_pv, ph_pv, kTcWait) && ok;
+      ph_pv ^= 1;
+      pv_pending = false;
+    }
+    // scores of tile it (issued one iteration earlier; waiting for them here
+    // also means the MMA warp has taken this tile's operand signal, so the
+    // next signal cannot complete a phase it has not yet waited for)
+    {
+      uint32_t& ph = (it & 1) ? ph_s1 : ph_s0;
+      ok = tqtc::mbar_wait(&mb_s[it & 1], ph, kTcWait) && ok;
+      ph ^= 1;
+    }
+    tqtc::fence_after_sync();
+    if (has_next) {
+      expand(it + 1);
+      tqtc::fence_smem_to_async();
+      tqtc::fence_before_sync();
+      tqtc::mbar_arrive(&mb_kv);
+    }
+    const bool failed = __any_sync(0xffffffffu, !ok || s_fail != 0);   // warp-uniform (tensor-memory access below)
+    const int64_t t0 = static_cast<int64_t>(it) * kTcKeys;
+    const int nv = static_cast<int>(p.T - t0 < kTcKeys ? p.T - t0 : kTcKeys);
+
+    // ---- logits of query `row` against keys 8 kq .. 8 kq + 7 of tile it
+    float lg[8];
+    {
+      float d0[8], d1[8], dzv[8];
+      const uint32_t dcol = tl + 96 * (it & 1) + 8 * kq;
+      tqtc::tmem_ld8x3(dcol, dcol + 32 * (P - 1), dcol + 32 * P, d0, d1, dzv);
+      const float iq = s_inv_lam[0][row], iz = s_inv_lam[1][row];
+      const float wq0 = p.walsh_k[0] * iq, wq1 = p.walsh_k[1] * iq;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float2 kf = s_kf[it & 1][8 * kq + k];
+        float c = wq0 * d0[k];
+        if constexpr (P == 2) c = fmaf(wq1, d1[k], c);
+        lg[k] = fmaf(kf.x, c, kf.y * iz * dzv[k]);
+      }
+    }
+    if (nv < kTcKeys) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) lg[k] = 8 * kq + k < nv ? lg[k] : -INFINITY;
+    }
+    float mloc = lg[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) mloc = fmaxf(mloc, lg[k]);
+    s_mx[kq][row] = mloc;
+    work_sync();
+    const float mx = fmaxf(fmaxf(s_mx[0][row], s_mx[1][row]), fmaxf(s_mx[2][row], s_mx[3][row]));
+    const bool need = mx > m_run + kLazyRescale;   // the same in the four threads of the row
+    if (__any_sync(0xffffffffu, need)) {
+      const float alpha = need ? exp2f(m_run - mx) : 1.f;
+      if (it > 0 && !failed) {
+        // this thread's quarter of O (columns 32 kq ..), rescaled in tensor
+        // memory (the previous value products are complete)
+        float o[32];
+        const uint32_t a = tl + kTcColO + 32 * kq;
+        tqtc::tmem_ld32(a, o);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o[k] *= alpha;
+        tqtc::tmem_st32(a, o);
+      }
+      l_run *= alpha;
+      if (need) m_run = mx;
+    }
+    // ---- probabilities -> value-product operands (row `row`, keys 8 kq .. + 7)
+    {
+      float xc[P][8], xz[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float pk = lg[k] == -INFINITY ? 0.f : exp2f(lg[k] - m_run);
+        l_run += pk;
+        const float4 vf = s_vf[it & 1][8 * kq + k];
+        xc[0][k] = pk * vf.x;
+        if constexpr (P == 2) xc[P - 1][k] = pk * vf.y;
+        xz[k] = pk * vf.z;
+      }
+      uint4 hi, lo;
+#pragma unroll
+      for (int pl = 0; pl < P; ++pl) {
+        tc_split8(xc[pl], hi, lo);
+        *reinterpret_cast<uint4*>(ac_hi + tc_chunk_off(row, 4 * pl + kq)) = hi;
+        *reinterpret_cast<uint4*>(ac_lo + tc_chunk_off(row, 4 * pl + kq)) = lo;
+      }
+      tc_split8(xz, hi, lo);
+      *reinterpret_cast<uint4*>(az + tc_chunk_off(row, kq)) = hi;
+      *reinterpret_cast<uint4*>(az + tc_chunk_off(row, 4 + kq)) = lo;
+    }
+    tqtc::fence_smem_to_async();
+    tqtc::fence_before_sync();
+    tqtc::mbar_arrive(&mb_p);
+    pv_pending = true;
+    if (!ok) s_fail = 1;
+  }
+  if (pv_pending) ok = tqtc::mbar_wait(&mb_pv, ph_pv, kTcWait) && ok;
+  tqtc::fence_after_sync();
+  if (!ok) s_fail = 1;
+  cp_async_wait<0>();
+  work_sync();   // the operand areas take the epilogue buffers
+
+  // ---- epilogue: y = (O_code + qjl S^T O_z) / l, out = Pi^T y.  Thread
+  // (row, kq) moves O columns 32 kq .. + 31 (O_code for kq < 2, O_z after) into
+  // the row's buffer by coordinate, then computes y for coordinates
+  // 16 kq .. 16 kq + 15, then the transform and its own 16 outputs.
+  float* xbuf = reinterpret_cast<float*>(kvb);      // [128][kTcXStride]: y (0..63), O_z (64..127)
+  float* lbuf = xbuf + kTcQ * kTcXStride;           // [4][128]: l of each quarter
+  float* smat = lbuf + 4 * kTcQ;                    // [64][64]: S of the value handle
+  float* xrow = xbuf + row * kTcXStride;
+  for (int i = tid; i < D * D / 4; i += kTcWorkers)
+    reinterpret_cast<float4*>(smat)[i] = reinterpret_cast<const float4*>(p.v_s)[i];
+  lbuf[kq * kTcQ + row] = n_tiles > 0 ? l_run : 0.f;
+  {
+    float o[32];
+    tqtc::tmem_ld32(tl + kTcColO + 32 * kq, o);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) xrow[32 * kq + tc_slot_dim(k)] = n_tiles > 0 ? o[k] : 0.f;
+  }
+  work_sync();
+  const float l = (lbuf[row] + lbuf[kTcQ + row]) + (lbuf[2 * kTcQ + row] + lbuf[3 * kTcQ + row]);
+  const float inv_l = l > 0.f ? 1.f / l : 0.f;
+  float y[16];   // coordinates 16 kq + i
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = xrow[16 * kq + i];
+  // (S^T O_z)_i = sum_j S[j][i] O_z[j] for this thread's coordinates
+#pragma unroll 2
+  for (int j = 0; j < D; ++j) {
+    const float zj = xrow[D + j] * p.qjl_v;
+    const float4* srow = reinterpret_cast<const float4*>(smat + j * D + 16 * kq);
+#pragma unroll
+    for (int i4 = 0; i4 < 4; ++i4) {
+      const float4 s4 = srow[i4];
+      y[4 * i4] = fmaf(s4.x, zj, y[4 * i4]);
+      y[4 * i4 + 1] = fmaf(s4.y, zj, y[4 * i4 + 1]);
+      y[4 * i4 + 2] = fmaf(s4.z, zj, y[4 * i4 + 2]);
+      y[4 * i4 + 3] = fmaf(s4.w, zj, y[4 * i4 + 3]);
+    }
+  }
+  work_sync();   // every thread has read the row's coordinates
+#pragma unroll
+  for (int i = 0; i < 16; ++i) xrow[16 * kq + i] = y[i] * inv_l;
+  work_sync();
+  // Pi^T y = D H y / sqrt(d), H in Sylvester order, on the whole row
+  float yy[D];
+#pragma unroll
+  for (int i = 0; i < D; ++i) yy[i] = xrow[i];
+#pragma unroll
+  for (int hb = 1; hb < D; hb <<= 1)
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      if (i & hb) continue;
+      const float a0 = yy[i], a1 = yy[i | hb];
+      yy[i] = a0 + a1;
+      yy[i | hb] = a0 - a1;
+    }
+  const int q = q0 + row;
+  if (q < p.S) {
+    const bool bad = s_fail != 0;
+    float4* o = reinterpret_cast<float4*>(p.out + (static_cast<int64_t>(bq) * p.S + q) * D + 16 * kq);
+    const float* sg = p.v_signs_d + 16 * kq;
+    const float inv_sqrt_d = 0.125f;
+#pragma unroll
+    for (int i4 = 0; i4 < 4; ++i4) {
+      float r[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * i4 + e;
+        // yy is indexed by compile-time coordinates: select this quarter's
+        float hv = 0.f;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+          if (qq == kq) hv = yy[16 * qq + i];
+        r[e] = bad ? NAN : hv * sg[i] * inv_sqrt_d;
+      }
+      o[i4] = make_float4(r[0], r[1], r[2], r[3]);
+    }
+  }
+  }   // workers
+  tqtc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tqtc::tmem_free(tmem, 512);
+}
+
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 size_t enc_workspace(int B, int Hq, int S, int d) {
@@ -488,6 +1025,18 @@ int launch_enc(const EncParams& p, int B, cudaStream_t s) {
     return TQ_ECUDA;
   dim3 grid((p.S + kWarps * kQPerWarp - 1) / (kWarps * kQPerWarp), B * p.Hq);
   kern<<<grid, kWarps * 32, smem, s>>>(p);
+  return tq::launch_status();
+}
+
+template <int BITS>
+int launch_enc_tc(const EncParams& p, int B, cudaStream_t s) {
+  constexpr size_t smem = tc_smem_bytes<BITS>();
+  static_assert(smem <= 227 * 1024, "shared memory of the tensor-core encoder kernel");
+  auto kern = encoder_tc_kernel<BITS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return TQ_ECUDA;
+  dim3 grid((p.S + kTcQ - 1) / kTcQ, B * p.Hq);
+  kern<<<grid, kTcThreads, smem, s>>>(p);
   return tq::launch_status();
 }
 
@@ -586,5 +1135,8 @@ extern "C" int tq_encoder_attention(const tq_rotation* hk, const tq_rotation* hv
   p.v_s = hv->d_s;
   p.v_signs_d = hv->d_signs;
   p.out = out;
+  // d = 64 with 1- or 2-bit codes and m = d: tensor-core kernel; otherwise the mma.sync kernel
+  if (d == 64 && hk->m == 64 && hk->bits <= 2 && tq::aligned16(out))
+    return hk->bits == 1 ? launch_enc_tc<1>(p, B, s) : launch_enc_tc<2>(p, B, s);
   return d == 64 ? dispatch_bits<64>(hk->bits, p, B, s) : dispatch_bits<128>(hk->bits, p, B, s);
 }
