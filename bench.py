@@ -8,9 +8,10 @@ sequence, bf16 heavy-tailed K/V (N(0,1) + 4 outlier channels x20 per
 
 One step = one decode step of the whole model's attention: for every layer,
 quantize the new token's K and V into slot T-1 of each sequence
-(tq_quantize_kv) and score the query against all T cached tokens
-(tq_decode_attention: q-prep, split-KV kernel, merge).  The packed cache
-(15 GB) is far larger than L2, so no flush is needed between steps.
+(tq_quantize_kv_pair: keys and values in one launch) and score the query
+against all T cached tokens (tq_decode_attention: q-prep, split-KV kernel,
+merge).  The packed cache (15 GB) is far larger than L2, so no flush is
+needed between steps.
 
 Metric: cached tokens scored per second, one unit = one (layer, sequence,
 kv-head, token) K+V record pair scored for all 4 query heads of its group.

@@ -502,7 +502,10 @@ __global__ void __launch_bounds__(kWarps * 32, D == 64 ? 3 : 1) encoder_attentio
 // software-pipelined over tiles: while the workers run the softmax of tile
 // i, the tensor core computes the scores of tile i + 1 (two score buffers in
 // tensor memory, two key and value operand buffers in shared memory), and
-// the packed records of tile i + 2 are in flight (cp.async).  Every wait is
+// the packed records of tile i + 2 are in flight (cp.async); the key and
+// value operands rotate through three buffers, so the value products of
+// tile i - 1 may still run while tile i + 1 is expanded, and the workers wait
+// for them only before they rewrite the probability operands.  Every wait is
 // bounded; the rows of a CTA whose wait ran out are written as NaN (after a
 // failed wait the MMA warp stops issuing but still commits, so no wait of
 // the workers is left without its arrival).
@@ -527,7 +530,7 @@ __host__ __device__ constexpr int tc_stage_bytes() {
 }
 template <int BITS>
 constexpr size_t tc_smem_bytes() {
-  return 1024 + 4 * kTcOpQ + 2 * tc_kv_bytes<BITS>() + 3 * kTcOpQ + 2 * tc_stage_bytes<BITS>();
+  return 1024 + 4 * kTcOpQ + 3 * tc_kv_bytes<BITS>() + 3 * kTcOpQ + 2 * tc_stage_bytes<BITS>();
 }
 
 // slot k of an operand row -> coordinate
@@ -594,8 +597,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
   uint8_t* aq_lo = base + kTcOpQ;
   uint8_t* as_hi = base + 2 * kTcOpQ;         // S q~ pieces
   uint8_t* as_lo = base + 3 * kTcOpQ;
-  uint8_t* kvb = base + 4 * kTcOpQ;           // two buffers: key operand planes, then value operand rows
-  uint8_t* ac_hi = kvb + 2 * KV;              // rows = queries, slots (pl, key)
+  uint8_t* kvb = base + 4 * kTcOpQ;           // three buffers: key operand planes, then value operand rows
+  uint8_t* ac_hi = kvb + 3 * KV;              // rows = queries, slots (pl, key)
   uint8_t* ac_lo = ac_hi + kTcOpQ;
   uint8_t* az = ac_lo + kTcOpQ;               // slots key: hi piece, 32 + key: lo piece
   uint8_t* stg = az + kTcOpQ;                 // two staged tiles
@@ -697,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     }
   }
 
-  // ---- expansion of tile t (staged in buffer t & 1) into operand buffer t & 1:
+  // ---- expansion of tile t (staged in buffer t & 1) into operand buffer t % 3:
   // thread -> key tid / 16, side (tid / 8) % 2, chunk tid % 8 of every plane
   const int xkey = tid >> 4, xside = (tid >> 3) & 1, xj = tid & 7;
   auto expand = [&](int t) {
@@ -714,7 +717,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     }
     pw[P] = reinterpret_cast<const uint32_t*>(sd + kTcKeys * CB + xkey * SB)[xj >> 2];
     const uint32_t one = xside ? 0x3F803F80u : 0x3C003C00u;   // +1 in both halves: bf16 values, fp16 keys
-    uint8_t* dst = kvb + (t & 1) * KV + xside * (P + 1) * kTcOpK;
+    uint8_t* dst = kvb + (t % 3) * KV + xside * (P + 1) * kTcOpK;
 #pragma unroll
     for (int pl = 0; pl <= P; ++pl) {
       uint32_t w4[4];
@@ -750,7 +753,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
   auto issue_scores = [&](int t) {   // D[t & 1] = q pieces x key operand of tile t
     constexpr uint32_t idesc = tqtc::idesc_f16_f32(kTcQ, kTcKeys);
     const uint32_t dcol = tmem + 96 * (t & 1);
-    const uint64_t kb = dkv + static_cast<uint64_t>(((t & 1) * KV) >> 4);
+    const uint64_t kb = dkv + static_cast<uint64_t>(((t % 3) * KV) >> 4);
 #pragma unroll
     for (int pl = 0; pl <= P; ++pl) {
       const uint64_t a_hi = pl < P ? dq_hi : ds_hi, a_lo = pl < P ? dq_lo : ds_lo;
@@ -764,7 +767,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
   auto issue_values = [&](int t) {   // O += probability operands x value operand of tile t
     constexpr uint32_t idesc = tqtc::idesc_bf16_f32(kTcQ, D) | tqtc::kIdescBMajorMN;
     const bool acc = t > 0;
-    const uint64_t vc = dkv_mn + static_cast<uint64_t>(((t & 1) * KV + (P + 1) * kTcOpK) >> 4);
+    const uint64_t vc = dkv_mn + static_cast<uint64_t>(((t % 3) * KV + (P + 1) * kTcOpK) >> 4);
     const uint64_t vz = vc + static_cast<uint64_t>((P * kTcOpK) >> 4);
     const uint32_t ocode = tmem + kTcColO, oz = tmem + kTcColO + 64;
 #pragma unroll
@@ -822,14 +825,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     cp_async_wait<0>();
     work_sync();   // tile it + 1 is staged; buffer it & 1 of the staging is free
     issue(it + 2);
-    // the previous value products read the value operand and probability
-    // buffers that are rewritten below (the MMA warp commits even after a
-    // failure, so these waits always end)
-    if (pv_pending) {
-      ok = tqtc::mbar_wait(&mb_pv, ph_pv, kTcWait) && ok;
-      ph_pv ^= 1;
-      pv_pending = false;
-    }
     // scores of tile it (issued one iteration earlier; waiting for them here
     // also means the MMA warp has taken this tile's operand signal, so the
     // next signal cannot complete a phase it has not yet waited for)
@@ -845,7 +840,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
       tqtc::fence_before_sync();
       tqtc::mbar_arrive(&mb_kv);
     }
-    const bool failed = __any_sync(0xffffffffu, !ok || s_fail != 0);   // warp-uniform (tensor-memory access below)
     const int64_t t0 = static_cast<int64_t>(it) * kTcKeys;
     const int nv = static_cast<int>(p.T - t0 < kTcKeys ? p.T - t0 : kTcKeys);
 
@@ -874,6 +868,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     for (int k = 1; k < 8; ++k) mloc = fmaxf(mloc, lg[k]);
     s_mx[kq][row] = mloc;
     work_sync();
+    // the previous value products read the probability operands rewritten
+    // below and accumulate the O rescaled below (the MMA warp commits even
+    // after a failure, so this wait always ends)
+    if (pv_pending) {
+      ok = tqtc::mbar_wait(&mb_pv, ph_pv, kTcWait) && ok;
+      ph_pv ^= 1;
+      pv_pending = false;
+    }
+    tqtc::fence_after_sync();
+    const bool failed = __any_sync(0xffffffffu, !ok || s_fail != 0);   // warp-uniform (tensor-memory access below)
     const float mx = fmaxf(fmaxf(s_mx[0][row], s_mx[1][row]), fmaxf(s_mx[2][row], s_mx[3][row]));
     const bool need = mx > m_run + kLazyRescale;   // the same in the four threads of the row
     if (__any_sync(0xffffffffu, need)) {
