@@ -806,6 +806,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
   } else {
 
   auto work_sync = [&]() { asm volatile("bar.sync 1, %0;\n" ::"n"(kTcWorkers) : "memory"); };
+  // one lane polls an mbarrier for the warp (all lanes polling the same word
+  // serialise in shared memory); the shuffle orders the other lanes after it
+  auto warp_wait = [&](uint64_t* mb, uint32_t parity) {
+    int done = 0;
+    if (lane == 0) done = tqtc::mbar_wait(mb, parity, kTcWait) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, done, 0) != 0;
+  };
   // prologue: tile 0 expanded
   bool ok = true;
   if (n_tiles > 0) {
@@ -830,7 +837,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     // next signal cannot complete a phase it has not yet waited for)
     {
       uint32_t& ph = (it & 1) ? ph_s1 : ph_s0;
-      ok = tqtc::mbar_wait(&mb_s[it & 1], ph, kTcWait) && ok;
+      ok = warp_wait(&mb_s[it & 1], ph) && ok;
       ph ^= 1;
     }
     tqtc::fence_after_sync();
@@ -872,7 +879,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     // below and accumulate the O rescaled below (the MMA warp commits even
     // after a failure, so this wait always ends)
     if (pv_pending) {
-      ok = tqtc::mbar_wait(&mb_pv, ph_pv, kTcWait) && ok;
+      ok = warp_wait(&mb_pv, ph_pv) && ok;
       ph_pv ^= 1;
       pv_pending = false;
     }
@@ -924,7 +931,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     pv_pending = true;
     if (!ok) s_fail = 1;
   }
-  if (pv_pending) ok = tqtc::mbar_wait(&mb_pv, ph_pv, kTcWait) && ok;
+  if (pv_pending) ok = warp_wait(&mb_pv, ph_pv) && ok;
   tqtc::fence_after_sync();
   if (!ok) s_fail = 1;
   cp_async_wait<0>();
