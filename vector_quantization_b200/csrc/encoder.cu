@@ -8,8 +8,10 @@
 // pass).  Queries sit at positions q_pos_offset + s.
 //
 // Two launches: a q-prep kernel (one warp per query: RoPE, fast
-// Walsh-Hadamard rotation, S q~) and the attention kernel.  The attention
-// kernel is flash-attention shaped on mma.sync m16n8k16 (bf16 in, fp32
+// Walsh-Hadamard rotation, S q~) and an attention kernel.  For d = 64 with 1-
+// or 2-bit codes that is the tensor-core kernel further down (tcgen05,
+// accumulators in tensor memory).  Otherwise it is the kernel below,
+// flash-attention shaped on mma.sync m16n8k16 (bf16 in, fp32
 // accumulate): a warp owns 8 queries, whose hi and lo bf16 pieces form the 16
 // rows of the A operand, so both pieces of one query land in the same thread
 // and are summed there.  Keys enter as the B operand straight from their bit

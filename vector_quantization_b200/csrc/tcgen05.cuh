@@ -2,8 +2,8 @@
 // (tcgen05.*): tensor-memory allocation, shared-memory matrix descriptors,
 // MMA issue, completion through an mbarrier, and tensor-memory loads.
 //
-// Operands are bf16 in shared memory, K-major, in the 128-byte swizzled
-// canonical layout: a matrix of R rows x K columns (K a multiple of 64) is
+// Operands are 16-bit (bf16 or fp16) in shared memory, K-major (one MN-major
+// form is below), in the 128-byte swizzled canonical layout: a matrix of R rows x K columns (K a multiple of 64) is
 // stored as K/64 column blocks of R x 64 elements; inside a block row r
 // occupies 128 bytes at (r/8)*1024 + (r%8)*128, and its 16-byte chunk c is
 // stored at chunk position c ^ (r % 8).  Blocks are 1024-byte aligned.  The
