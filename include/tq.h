@@ -131,13 +131,14 @@ int tq_rotation_export(const tq_rotation* h, float* pi, float* s,
 
 /*
  * tq_tensor_core_selftest - diagnostic: runs one 128 x 128 x 128 bf16 product
- * through the 5th-generation tensor-core path (tcgen05 with operands in
- * swizzled shared memory and the accumulator in tensor memory) on the
- * current device, with exactly representable small-integer operands, and
- * stores in *mismatches the number of result elements that differ from the
- * exact integer product (0 on a working device).  Synchronous; allocates
- * and frees its own 64 KB of device memory.  Returns TQ_OK, TQ_EINVAL,
- * TQ_ENOMEM or TQ_ECUDA.
+ * and two 128 x 64 x 64 products (second operand K-major, and MN-major as
+ * the encoder attention's value operand) through the 5th-generation
+ * tensor-core path (tcgen05 with operands in swizzled shared memory and the
+ * accumulator in tensor memory) on the current device, with exactly
+ * representable small-integer operands, and stores in *mismatches the
+ * number of result elements that differ from the exact integer products
+ * (0 on a working device).  Synchronous; allocates and frees its own 64 KB
+ * of device memory.  Returns TQ_OK, TQ_EINVAL, TQ_ENOMEM or TQ_ECUDA.
  */
 int tq_tensor_core_selftest(int64_t* mismatches);
 

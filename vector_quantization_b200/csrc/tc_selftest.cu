@@ -1,8 +1,9 @@
-// Device self-test of the tensor-core (tcgen05) path the encoder relies on:
-// one 128 x 128 x 128 bf16 product with exactly representable small-integer
-// operands, built in the 128-byte swizzled shared-memory layout, computed
-// into tensor memory and read back, compared element by element with the
-// exact integer result on the host.
+// Device self-test of the tensor-core (tcgen05) forms the kernels rely on:
+// one 128 x 128 x 128 bf16 product and two 128 x 64 x 64 products (B K-major,
+// and B MN-major as the value operand of the encoder attention kernel), with
+// exactly representable small-integer operands in the 128-byte swizzled
+// shared-memory layouts, computed into tensor memory and read back, compared
+// element by element with the exact integer results on the host.
 #include <cstdlib>
 #include <vector>
 
@@ -60,6 +61,65 @@ __global__ void __launch_bounds__(128) tc_selftest_kernel(float* __restrict__ ou
   tqtc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tqtc::tmem_free(tmem, kN);
+}
+
+// 128 x 64 x 64: D[m][n] = sum_k A[m][k] B[k][n], B stored K-major (row n,
+// column k) or MN-major (row k holding the 64 n of that k).
+constexpr int kM2 = 128, kN2 = 64, kK2 = 64;
+__device__ __host__ inline int sel_a2(int m, int k) { return (m * 7 + k * 3) % 11 - 5; }
+__device__ __host__ inline int sel_b2(int k, int n) { return (n * 5 + k * 13) % 9 - 4; }
+
+__global__ void __launch_bounds__(128) tc_selftest_n64_kernel(int mn_major, float* __restrict__ out,
+                                                              int* __restrict__ status) {
+  extern __shared__ uint8_t raw[];
+  __shared__ uint64_t mbar;
+  __shared__ uint32_t tmem_slot;
+  uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
+  uint8_t* A = base;
+  uint8_t* B = base + kM2 * kK2 * 2;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < kM2 * kK2; i += blockDim.x) {
+    const int m = i / kK2, k = i % kK2;
+    *reinterpret_cast<__nv_bfloat16*>(A + tqtc::sw128_offset(m, k, kM2)) =
+        __float2bfloat16_rn(static_cast<float>(sel_a2(m, k)));
+  }
+  for (int i = tid; i < kK2 * kN2; i += blockDim.x) {
+    const int k = i / kN2, n = i % kN2;
+    const uint32_t off = mn_major ? static_cast<uint32_t>((k >> 3) * 1024 + (k & 7) * 128 +
+                                                          (((n >> 3) ^ (k & 7)) << 4) + ((n & 7) << 1))
+                                  : tqtc::sw128_offset(n, k, kN2);
+    *reinterpret_cast<__nv_bfloat16*>(B + off) = __float2bfloat16_rn(static_cast<float>(sel_b2(k, n)));
+  }
+  if (tid == 0) tqtc::mbar_init(&mbar, 1);
+  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, kN2);
+  tqtc::fence_smem_to_async();
+  tqtc::fence_before_sync();
+  __syncthreads();
+  tqtc::fence_after_sync();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 0) {
+    const uint32_t idesc = tqtc::idesc_bf16_f32(kM2, kN2) | (mn_major ? tqtc::kIdescBMajorMN : 0u);
+    for (int ks = 0; ks < kK2 / 16; ++ks) {
+      const uint64_t bd = mn_major ? tqtc::sw128_desc_mn(tqtc::smem_u32(B) + ks * 2048)
+                                   : tqtc::sw128_desc_kstep(tqtc::smem_u32(B), ks, kN2);
+      tqtc::mma_bf16_ss(tmem, tqtc::sw128_desc_kstep(tqtc::smem_u32(A), ks, kM2), bd, idesc, ks > 0);
+    }
+    tqtc::mma_commit(&mbar);
+  }
+  const bool ok = tqtc::mbar_wait(&mbar, 0, kWaitLimit);
+  if (!ok && lane == 0) atomicExch(status, 1);
+  tqtc::fence_after_sync();
+  if (ok) {
+    const int row = warp * 32 + lane;
+    for (int c0 = 0; c0 < kN2; c0 += 32) {
+      float v[32];
+      tqtc::tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+      for (int j = 0; j < 32; ++j) out[row * kN2 + c0 + j] = v[j];
+    }
+  }
+  tqtc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tqtc::tmem_free(tmem, kN2);
 }
 
 // Bounded-wait check: thread 0 inits an mbarrier expecting one arrival.
@@ -130,6 +190,35 @@ extern "C" int tq_tensor_core_selftest(int64_t* mismatches) {
         }
       *mismatches = bad;
     }
+  }
+  // the two 128 x 64 x 64 forms
+  const int smem2 = kM2 * kK2 * 2 + kK2 * kN2 * 2 + 1024;
+  if (st == TQ_OK &&
+      cudaFuncSetAttribute(tc_selftest_n64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) != cudaSuccess)
+    st = TQ_ECUDA;
+  for (int mn = 0; mn < 2 && st == TQ_OK; ++mn) {
+    std::vector<float> out(kM2 * kN2);
+    int status = 0;
+    if (cudaMemset(d_status, 0, sizeof(int)) != cudaSuccess ||
+        cudaMemset(d_out, 0xFF, sizeof(float) * kM2 * kN2) != cudaSuccess) {
+      st = TQ_ECUDA;
+      break;
+    }
+    tc_selftest_n64_kernel<<<1, 128, smem2>>>(mn, d_out, d_status);
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(out.data(), d_out, sizeof(float) * kM2 * kN2, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(&status, d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+      st = TQ_ECUDA;
+      break;
+    }
+    int64_t bad = status ? kM2 * kN2 : 0;
+    for (int m = 0; m < kM2 && !status; ++m)
+      for (int n = 0; n < kN2; ++n) {
+        long ref = 0;
+        for (int k = 0; k < kK2; ++k) ref += static_cast<long>(sel_a2(m, k)) * sel_b2(k, n);
+        if (out[m * kN2 + n] != static_cast<float>(ref)) ++bad;
+      }
+    *mismatches += bad;
   }
   cudaFree(d_out);
   cudaFree(d_status);
