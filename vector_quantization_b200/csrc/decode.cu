@@ -138,23 +138,35 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   for (int i = 0; i < kStages - 1; ++i) issue(i);
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
-  uint32_t qf[2][NT][8][2];
+  // The query B fragments: in registers for one n-tile (G <= 4); in shared
+  // memory for two (G = 8), read at each MMA, which frees the registers the
+  // pipelined loop needs there.
+  uint32_t qf[2][1][8][2];   // used for NT == 1 only (the compiler drops it otherwise)
+  __shared__ uint2 s_qf[2][NT][8][NT == 1 ? 1 : 32];   // a stub for NT == 1
   float2 kc[2][NT];
   {
     const uint32_t* src = p.qfrag + static_cast<size_t>(bh) * (2 * NT * 8 * 32 * 2);
+    if constexpr (NT == 1) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int kb = 0; kb < 8; ++kb) {
+          const uint2 v = *reinterpret_cast<const uint2*>(src + ((t * 8 + kb) * 32 + lane) * 2);
+          qf[t][0][kb][0] = v.x;
+          qf[t][0][kb][1] = v.y;
+        }
+    } else {
+      for (int i = threadIdx.x; i < 2 * NT * 8 * 32; i += blockDim.x)
+        (&s_qf[0][0][0][0])[i] = reinterpret_cast<const uint2*>(src)[i];
+    }
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int kb = 0; kb < 8; ++kb) {
-          const uint2 v = *reinterpret_cast<const uint2*>(src + (((t * NT + nt) * 8 + kb) * 32 + lane) * 2);
-          qf[t][nt][kb][0] = v.x;
-          qf[t][nt][kb][1] = v.y;
-        }
         const int h = tig + 4 * nt;
         kc[t][nt] = h < G ? p.kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] : make_float2(0.f, 0.f);
       }
+    if constexpr (NT != 1) __syncthreads();
   }
   float accC[NT][8][4], accZ[NT][8][4];
   float m_run[NT], l_run[NT];
@@ -244,7 +256,10 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
                                  bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb + 1, one_h),
                                  bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb + 1, one_h)};
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16(c[nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint2 qb = s_qf[type][nt][kb][lane];
+            mma_f16(c[nt], a, qb.x, qb.y);
+          }
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -393,9 +408,9 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
     return static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
   };
 
-  // Pipelined order for G <= 4; with G = 8 the two tiles' live values would
-  // not fit the register file, so tiles run one after the other.
-  constexpr bool kPipe = G <= 4;
+  // Pipelined order (for G = 8 it fits the register file because the query
+  // fragments are in shared memory).
+  constexpr bool kPipe = true;
   if constexpr (kPipe) {
     float prob_prev[NT][2];
     const uint8_t* stg_prev = my_stages;
