@@ -55,6 +55,7 @@ struct EncParams {
   uint32_t one_h, one_b;   // kOneH2 / kOneB2, passed at run time (see bit_select)
   const float* v_s;        // [D][D] S_V row-major
   const float* v_signs_d;  // [D] Hadamard signs of the V handle
+  const uint16_t* epi;     // output-transform operands of the V handle (d = 64; tensor-core kernel)
   float* out;              // [B*Hq][S][D]
 };
 
@@ -519,7 +520,7 @@ constexpr int kTcThreads = kTcWorkers + 32;   // and the MMA warp
 constexpr int kTcWait = 1 << 17;        // polls of about 9 us each
 constexpr int kTcOpQ = kTcQ * 128;      // one [128 x 64] 16-bit operand: 16 KB
 constexpr int kTcOpK = kTcKeys * 128;   // one [32 x 64] 16-bit operand: 4 KB
-constexpr int kTcXStride = 129;         // floats per row of the epilogue buffer
+constexpr int kTcEpiB = 64 * 128;      // one [64 x 64] bf16 operand of the output transform: 8 KB
 constexpr uint32_t kTcColO = 256;       // tensor-memory columns: scores 0..191 (two buffers), O 256..383
 
 template <int BITS>
@@ -585,6 +586,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
   static_assert(P <= 2, "code planes of at most 2 bits");
   extern __shared__ uint8_t raw[];
   __shared__ uint64_t mb_s[2], mb_pv, mb_kv, mb_p;   // products done; operands / probabilities ready
+  __shared__ uint64_t mb_epi;                        // the output transform's products done
   __shared__ uint32_t tmem_slot;
   __shared__ int s_fail;
   __shared__ float s_inv_lam[2][kTcQ];        // per query row: 1 / range scale of q~ (0) and S q~ (1)
@@ -619,6 +621,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     tqtc::mbar_init(&mb_pv, 1);
     tqtc::mbar_init(&mb_kv, kTcWorkers);
     tqtc::mbar_init(&mb_p, kTcWorkers);
+    tqtc::mbar_init(&mb_epi, 1);
     s_fail = 0;
   }
   if (warp == 0) tqtc::tmem_alloc(&tmem_slot, 512);
@@ -939,81 +942,69 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
   cp_async_wait<0>();
   work_sync();   // the operand areas take the epilogue buffers
 
-  // ---- epilogue: y = (O_code + qjl S^T O_z) / l, out = Pi^T y.  Thread
-  // (row, kq) moves O columns 32 kq .. + 31 (O_code for kq < 2, O_z after) into
-  // the row's buffer by coordinate, then computes y for coordinates
-  // 16 kq .. 16 kq + 15, then the transform and its own 16 outputs.
-  float* xbuf = reinterpret_cast<float*>(kvb);      // [128][kTcXStride]: y (0..63), O_z (64..127)
-  float* lbuf = xbuf + kTcQ * kTcXStride;           // [4][128]: l of each quarter
-  float* smat = lbuf + 4 * kTcQ;                    // [64][64]: S of the value handle
-  float* xrow = xbuf + row * kTcXStride;
-  for (int i = tid; i < D * D / 4; i += kTcWorkers)
-    reinterpret_cast<float4*>(smat)[i] = reinterpret_cast<const float4*>(p.v_s)[i];
+  // ---- epilogue on the tensor core: out = D H (O_code + qjl S^T O_z) / (8 l)
+  // = (O_code B1^T + O_z B2^T) / l with B1 = D H / 8 and B2 = qjl D H S^T / 8
+  // in slot order (built with the value handle).  Thread (row, kq) writes O
+  // columns 32 kq .. + 31 (O_code for kq < 2, O_z after) as bf16 hi and lo
+  // operand rows, one thread issues the 20 MMAs into the first score buffer,
+  // and each thread scales and stores its 16 outputs.
+  uint8_t* eo = kvb;                            // O_code hi, lo, O_z hi, lo: 4 x [128 x 64] bf16
+  uint8_t* eb = kvb + 4 * kTcOpQ;               // B1, B2 hi, B2 lo: 3 x [64 x 64] bf16
+  float* lbuf = reinterpret_cast<float*>(eb + 3 * kTcEpiB);   // [4][128]: l of each quarter
+  for (int i = tid; i < 3 * kTcEpiB / 16; i += kTcWorkers)
+    cp_async16(eb + 16 * i, reinterpret_cast<const uint8_t*>(p.epi) + 16 * i, 16);
+  cp_async_commit();
   lbuf[kq * kTcQ + row] = n_tiles > 0 ? l_run : 0.f;
   {
     float o[32];
     tqtc::tmem_ld32(tl + kTcColO + 32 * kq, o);
+    uint8_t* ahi = eo + (kq >> 1) * 2 * kTcOpQ;
+    uint8_t* alo = ahi + kTcOpQ;
 #pragma unroll
-    for (int k = 0; k < 32; ++k) xrow[32 * kq + tc_slot_dim(k)] = n_tiles > 0 ? o[k] : 0.f;
+    for (int j = 0; j < 4; ++j) {
+      float x[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = n_tiles > 0 ? o[8 * j + e] : 0.f;
+      uint4 hi, lo;
+      tc_split8(x, hi, lo);
+      const int c = 4 * (kq & 1) + j;   // slots 32 (kq % 2) + 8 j .. + 7
+      *reinterpret_cast<uint4*>(ahi + tc_chunk_off(row, c)) = hi;
+      *reinterpret_cast<uint4*>(alo + tc_chunk_off(row, c)) = lo;
+    }
   }
+  cp_async_wait<0>();
+  tqtc::fence_smem_to_async();
+  tqtc::fence_before_sync();
   work_sync();
+  if (tid == 0) {
+    tqtc::fence_after_sync();
+    constexpr uint32_t idesc = tqtc::idesc_bf16_f32(kTcQ, D);
+    const uint64_t a0 = tqtc::sw128_desc(tqtc::smem_u32(eo)), b0 = tqtc::sw128_desc(tqtc::smem_u32(eb));
+    constexpr uint64_t at = kTcOpQ >> 4, bt = kTcEpiB >> 4;
+    // code hi x B1, code lo x B1, z hi x B2 hi, z hi x B2 lo, z lo x B2 hi
+    constexpr int pa[5] = {0, 1, 2, 2, 3}, pb[5] = {0, 0, 1, 2, 1};
+#pragma unroll
+    for (int pr = 0; pr < 5; ++pr)
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        tqtc::mma_bf16_ss(tmem, a0 + pa[pr] * at + 2 * ks, b0 + pb[pr] * bt + 2 * ks, idesc, pr > 0 || ks > 0);
+    tqtc::mma_commit(&mb_epi);
+  }
+  const bool eok = warp_wait(&mb_epi, 0);
+  tqtc::fence_after_sync();
   const float l = (lbuf[row] + lbuf[kTcQ + row]) + (lbuf[2 * kTcQ + row] + lbuf[3 * kTcQ + row]);
   const float inv_l = l > 0.f ? 1.f / l : 0.f;
-  float y[16];   // coordinates 16 kq + i
-#pragma unroll
-  for (int i = 0; i < 16; ++i) y[i] = xrow[16 * kq + i];
-  // (S^T O_z)_i = sum_j S[j][i] O_z[j] for this thread's coordinates
-#pragma unroll 2
-  for (int j = 0; j < D; ++j) {
-    const float zj = xrow[D + j] * p.qjl_v;
-    const float4* srow = reinterpret_cast<const float4*>(smat + j * D + 16 * kq);
-#pragma unroll
-    for (int i4 = 0; i4 < 4; ++i4) {
-      const float4 s4 = srow[i4];
-      y[4 * i4] = fmaf(s4.x, zj, y[4 * i4]);
-      y[4 * i4 + 1] = fmaf(s4.y, zj, y[4 * i4 + 1]);
-      y[4 * i4 + 2] = fmaf(s4.z, zj, y[4 * i4 + 2]);
-      y[4 * i4 + 3] = fmaf(s4.w, zj, y[4 * i4 + 3]);
-    }
-  }
-  work_sync();   // every thread has read the row's coordinates
-#pragma unroll
-  for (int i = 0; i < 16; ++i) xrow[16 * kq + i] = y[i] * inv_l;
-  work_sync();
-  // Pi^T y = D H y / sqrt(d), H in Sylvester order, on the whole row
-  float yy[D];
-#pragma unroll
-  for (int i = 0; i < D; ++i) yy[i] = xrow[i];
-#pragma unroll
-  for (int hb = 1; hb < D; hb <<= 1)
-#pragma unroll
-    for (int i = 0; i < D; ++i) {
-      if (i & hb) continue;
-      const float a0 = yy[i], a1 = yy[i | hb];
-      yy[i] = a0 + a1;
-      yy[i | hb] = a0 - a1;
-    }
+  float r0[16], r1[16], r2[16];
+  tqtc::tmem_ld16x3(tl + 16 * kq, tl + 16 * kq, tl + 16 * kq, r0, r1, r2);
   const int q = q0 + row;
   if (q < p.S) {
-    const bool bad = s_fail != 0;
+    const bool bad = s_fail != 0 || !eok;
     float4* o = reinterpret_cast<float4*>(p.out + (static_cast<int64_t>(bq) * p.S + q) * D + 16 * kq);
-    const float* sg = p.v_signs_d + 16 * kq;
-    const float inv_sqrt_d = 0.125f;
 #pragma unroll
-    for (int i4 = 0; i4 < 4; ++i4) {
-      float r[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * i4 + e;
-        // yy is indexed by compile-time coordinates: select this quarter's
-        float hv = 0.f;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq)
-          if (qq == kq) hv = yy[16 * qq + i];
-        r[e] = bad ? NAN : hv * sg[i] * inv_sqrt_d;
-      }
-      o[i4] = make_float4(r[0], r[1], r[2], r[3]);
-    }
+    for (int i4 = 0; i4 < 4; ++i4)
+      o[i4] = bad ? make_float4(NAN, NAN, NAN, NAN)
+                  : make_float4(r0[4 * i4] * inv_l, r0[4 * i4 + 1] * inv_l, r0[4 * i4 + 2] * inv_l,
+                                r0[4 * i4 + 3] * inv_l);
   }
   }   // workers
   tqtc::fence_before_sync();
@@ -1149,7 +1140,8 @@ extern "C" int tq_encoder_attention(const tq_rotation* hk, const tq_rotation* hv
   p.v_signs_d = hv->d_signs;
   p.out = out;
   // d = 64 with 1- or 2-bit codes and m = d: tensor-core kernel; otherwise the mma.sync kernel
-  if (d == 64 && hk->m == 64 && hk->bits <= 2 && tq::aligned16(out))
+  p.epi = hv->d_enc_epi;
+  if (d == 64 && hk->m == 64 && hk->bits <= 2 && hv->d_enc_epi && tq::aligned16(out))
     return hk->bits == 1 ? launch_enc_tc<1>(p, B, s) : launch_enc_tc<2>(p, B, s);
   return d == 64 ? dispatch_bits<64>(hk->bits, p, B, s) : dispatch_bits<128>(hk->bits, p, B, s);
 }

@@ -230,6 +230,7 @@ void release(tq_rotation* h) {
   cudaFree(h->d_s_op);
   cudaFree(h->d_hd_f16);
   cudaFree(h->d_hd_bf16);
+  cudaFree(h->d_enc_epi);
   cudaFree(h->d_pi_hi);
   cudaFree(h->d_pi_lo);
   cudaFree(h->d_s_bf16);
@@ -399,6 +400,34 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
           }
         if ((st = upload(&h->d_hd_f16, hf.data(), hf.size())) != TQ_OK) { release(h); return st; }
         if ((st = upload(&h->d_hd_bf16, hb.data(), hb.size())) != TQ_OK) { release(h); return st; }
+      }
+      if (d == 64 && m == 64) {
+        // output transform of the tensor-core encoder attention (see
+        // tq_internal.h): three [64 x 64] bf16 operands, rows i = output
+        // coordinate, K = slot k standing for coordinate dim(k)
+        auto slot_dim = [](int k) { return 32 * (k >> 5) + ((k >> 1) & 15) + 16 * (k & 1); };
+        auto had = [](int i, int j) { return (__builtin_popcount(static_cast<unsigned>(i & j)) & 1) ? -1.0 : 1.0; };
+        const double qjl = kQjlConst / m;
+        std::vector<uint16_t> ep(static_cast<size_t>(3) * d * d);
+        for (int i = 0; i < d; ++i)
+          for (int k = 0; k < d; ++k) {
+            const int dk = slot_dim(k);
+            const double sgn = h->signs[i] < 0.f ? -1.0 : 1.0;
+            double g = 0.0;   // sum_t H[i][t] S[dk][t]
+            for (int t = 0; t < d; ++t) g += had(i, t) * s[static_cast<size_t>(dk) * d + t];
+            const float b1 = static_cast<float>(sgn * had(i, dk) / 8.0);
+            const float b2 = static_cast<float>(sgn * qjl * g / 8.0);
+            const float b2h = round_to_bf16(b2), b2l = round_to_bf16(b2 - b2h);
+            const size_t off = static_cast<size_t>((i >> 3) * 1024 + (i & 7) * 128 + ((((k >> 3) ^ (i & 7))) << 4) +
+                                                   ((k & 7) << 1)) / 2;
+            const float vals[3] = {b1, b2h, b2l};
+            for (int t = 0; t < 3; ++t) {
+              uint32_t bits;
+              std::memcpy(&bits, &vals[t], 4);
+              ep[static_cast<size_t>(t) * d * d + off] = static_cast<uint16_t>(bits >> 16);
+            }
+          }
+        if ((st = upload(&h->d_enc_epi, ep.data(), ep.size())) != TQ_OK) { release(h); return st; }
       }
     }
   }

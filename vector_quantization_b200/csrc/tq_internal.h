@@ -44,6 +44,12 @@ struct tq_rotation {
   // bits; Hadamard kind, d = 128 only.
   uint16_t* d_hd_f16 = nullptr;
   uint16_t* d_hd_bf16 = nullptr;
+  // Hadamard kind, d = 64: the output transform of the tensor-core encoder
+  // attention, out = D H (O_code + qjl S^T O_z) / sqrt(d), as three bf16
+  // operands [64 output coordinates x 64 slots] in the same layout, columns
+  // in the kernel's slot order (slot k = coordinate 32 (k / 32) + (k / 2) % 16
+  // + 16 (k % 2)): D H / 8 (exact), then qjl D H S^T / 8 as hi and lo pieces.
+  uint16_t* d_enc_epi = nullptr;
   // Dense kind: Pi as bf16 hi + lo pieces and S as bf16, row-major, for the
   // split tensor-core contractions.
   uint16_t* d_pi_hi = nullptr;
