@@ -139,15 +139,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t b
                : "memory");
 }
 
-// Bulk asynchronous copy global -> shared of `bytes` (multiple of 16, both
-// addresses 16-byte aligned), completing its bytes on `mbar`.  No multicast.
-__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* mbar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(mbar))
-               : "memory");
-}
-
 // Tiled 2-D TMA load of one box at coordinates (c0 innermost, c1) of the
 // tensor map at `map` (a __grid_constant__ kernel parameter) into shared
 // memory, completing its bytes on `mbar`.  c0 times the element size must be a
