@@ -131,6 +131,15 @@ __device__ __forceinline__ float fp16_range_scale(float max_abs) {
   return ldexpf(1.f, 14 - e);
 }
 
+// 2^x by the hardware approximation (PTX ex2.approx: relative error near
+// 2^-22, subnormal results flushed to zero, 2^-inf = +0), for softmax
+// weights, which need no more.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return static_cast<uint32_t>(__half_as_ushort(__float2half_rn(lo))) |
          (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(hi))) << 16);

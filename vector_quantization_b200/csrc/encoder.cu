@@ -893,7 +893,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     const float mx = fmaxf(fmaxf(s_mx[0][row], s_mx[1][row]), fmaxf(s_mx[2][row], s_mx[3][row]));
     const bool need = mx > m_run + kLazyRescale;   // the same in the four threads of the row
     if (__any_sync(0xffffffffu, need)) {
-      const float alpha = need ? exp2f(m_run - mx) : 1.f;
+      const float alpha = need ? exp2_approx(m_run - mx) : 1.f;
       if (it > 0 && !failed) {
         // this thread's quarter of O (columns 32 kq ..), rescaled in tensor
         // memory (the previous value products are complete)
@@ -912,7 +912,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
       float xc[P][8], xz[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float pk = lg[k] == -INFINITY ? 0.f : exp2f(lg[k] - m_run);
+        const float pk = lg[k] == -INFINITY ? 0.f : exp2_approx(lg[k] - m_run);
         l_run += pk;
         const float4 vf = s_vf[it & 1][8 * kq + k];
         xc[0][k] = pk * vf.x;
