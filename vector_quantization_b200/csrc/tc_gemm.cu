@@ -20,7 +20,7 @@
 // toward zero, and with d = 1536 a single accumulator shrank the rotated
 // coordinates by ~5e-6 relative; a quarter of the accumulation steps per
 // accumulator keeps that bias near 1e-6.  Every wait is bounded; a tile whose
-// wait runs out is written as NaN.  No multicast.
+// wait runs out is written as NaN.  Each CTA loads its own tiles.
 #include <cuda.h>
 #include <cuda_bf16.h>
 

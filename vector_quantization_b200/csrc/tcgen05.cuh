@@ -142,7 +142,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t b
 // Tiled 2-D TMA load of one box at coordinates (c0 innermost, c1) of the
 // tensor map at `map` (a __grid_constant__ kernel parameter) into shared
 // memory, completing its bytes on `mbar`.  c0 times the element size must be a
-// multiple of 16 bytes.  No multicast.
+// multiple of 16 bytes.  The load fills this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int c0, int c1, uint64_t* mbar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
