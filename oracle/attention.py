@@ -22,6 +22,17 @@ q' with the fully dequantized key (two independent routes); T = 1 returns the
 dequantized value; q = 0 returns the mean value; token permutation
 invariance; convergence to exact attention as bits grow; the unquantized
 rotated path equals exact RoPE attention ([TurboESM] §2.A).
+
+Full-precision window ([NSNQuant] §4, "Résidus", after KIVI): the cache is a
+quantized part of T tokens plus a residual of the R most recent tokens kept
+as the model produced them; when the residual is full it is quantized and
+appended to the packed part.  Decode attends to both: window token i sits at
+position T + i, so its key gets RoPE there, and the softmax runs over the
+union.  Pins (tests/test_oracle_window.py): R = 0 equals decode_attention
+(whose scores take the other route, through the codes); T = 0 equals textbook
+softmax attention; one window token and no packed part returns its value; a
+shift of every position by the same amount leaves the output unchanged,
+which fails if the window keys are not placed after the packed part.
 """
 from __future__ import annotations
 
@@ -120,3 +131,48 @@ def exact_attention(q, k, v, scale: float, rope_base: float = 0.0, q_pos=None, k
     s = s - np.max(s, axis=1, keepdims=True)
     e = np.exp(s)
     return (e / np.sum(e, axis=1, keepdims=True)) @ v
+
+
+def decode_attention_window(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, k_window,
+                            v_window, scale: float) -> np.ndarray:
+    """One decode step over a packed cache plus a full-precision window
+    ([NSNQuant] §4, "Résidus").
+
+    q [B, Hq, d], q_pos [B]; packed caches (codes, signs, norms) of shape
+    [B, Hkv, T, ...] as in :func:`decode_attention`; k_window, v_window
+    [B, Hkv, R, d] the raw keys (before RoPE) and values of the R most recent
+    tokens, window token i at position T + i.  The keys are the dequantized
+    packed keys followed by RoPE(k_window); the values the dequantized packed
+    values followed by v_window; softmax attention over all T + R of them.
+    Returns out [B, Hq, d] float64."""
+    from .codec import dequantize
+    q = np.asarray(q, dtype=np.float64)
+    kw = np.asarray(k_window, dtype=np.float64)
+    vw = np.asarray(v_window, dtype=np.float64)
+    B, Hq, d = q.shape
+    kc, kz, kn, kr = _unpack_cache(rot_k, *k_cache)
+    vc, vz, vn, vr = _unpack_cache(rot_v, *v_cache)
+    Hkv, T = kc.shape[1], kc.shape[2]
+    R = kw.shape[2]
+    g = Hq // Hkv
+    out = np.zeros((B, Hq, rot_v.d))
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // g
+            keys = [dequantize(rot_k, kc[b, kv], kz[b, kv], kn[b, kv], kr[b, kv])]
+            vals = [dequantize(rot_v, vc[b, kv], vz[b, kv], vn[b, kv], vr[b, kv])]
+            kwin = kw[b, kv]
+            qh = q[b, h]
+            if rot_k.rope_base:
+                kwin = apply_rope(kwin, T + np.arange(R), rot_k.rope_base)
+                qh = apply_rope(qh, q_pos[b], rot_k.rope_base)
+            keys.append(kwin)
+            vals.append(vw[b, kv])
+            K = np.concatenate(keys, axis=0)
+            V = np.concatenate(vals, axis=0)
+            if K.shape[0] == 0:
+                continue
+            score = (K @ qh) * scale
+            e = np.exp(score - np.max(score))
+            out[b, h] = (e / np.sum(e)) @ V
+    return out
