@@ -49,7 +49,8 @@ UNIT = "tokens/s"
 # when the kernel has changed since that capture.
 SPLIT_TRAFFIC_PER_TOKEN = (235_454_464 + 6_769_152) / (16 * 8 * 16384)
 
-EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1")
+EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1",
+          "decode_llama8b_layer_window")
 
 
 def parse():
@@ -231,6 +232,8 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None):
         out.update(_extra_search(dev, g, search_rows))
     if "decode_llama8b_layer_3p1" in select:
         out.update(_extra_decode_3p1(dev, peak_gbs))
+    if "decode_llama8b_layer_window" in select:
+        out.update(_extra_decode_window(dev, peak_gbs))
     return out
 
 
@@ -355,6 +358,44 @@ def _extra_decode_3p1(dev, peak_gbs):
     return {"decode_llama8b_layer_3p1": {"split_ms": round(ms, 4), "GB_s": round(byts / ms / 1e6, 1),
                                          "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
                                          "algorithmic_bytes": byts, "note": "one layer, 144 B per token pair"}}
+
+def _extra_decode_window(dev, peak_gbs, R=128):
+    """One layer of the Llama-3.1-8B-shaped decode (B16, Hq32, Hkv8, 2+1 bits)
+    whose 32768 cached tokens are 32768 - R packed ones plus a bf16
+    full-precision window of the R most recent, against the same layer with
+    all 32768 packed.  Whole-call device time of both (four launches, and
+    five with the window); the cache (470 MB) is larger than L2."""
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["llama31_8b_gqa_decode"]
+    B, Hq, Hkv, d, T, seed = c["batch"], c["q_heads"], c["kv_heads"], c["head_dim"], c["tokens"], c["seed"]
+    rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 8, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 8, 2]))
+    kc, vc = tq.empty_records(rk, (B, Hkv, T), dev), tq.empty_records(rv, (B, Hkv, T), dev)
+    xk = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, 8, 3], dev)
+    tq.quantize_kv(rk, xk, apply_rope=True, pos_period=T, out=kc)
+    kw = xk[:, :, T - R:].to(torch.bfloat16).contiguous()
+    del xk
+    xv = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, 8, 4], dev)
+    tq.quantize_kv(rv, xv, out=vc)
+    vw = xv[:, :, T - R:].to(torch.bfloat16).contiguous()
+    del xv
+    q = synth.heavy_tailed_torch((B, Hq, d), [seed, 8, 5], dev)
+    qpos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    o = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ws = tq.alloc_workspace(tq.decode_window_workspace_size(rk, rv, B, Hq, Hkv, T - R, R), dev)
+    ws2 = tq.alloc_workspace(tq.decode_workspace_size(rk, rv, B, Hq, Hkv, T), dev)
+    ms_w = _time_ms(lambda: tq.decode_attention_window(rk, rv, q, qpos, kc, vc, T - R, kw, vw, R, out=o,
+                                                       workspace=ws), reps=20, warm=3)
+    ms_p = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws2), reps=20, warm=3)
+    byts = B * Hkv * (T - R) * 2 * rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)) + 2 * kw.numel() * 2
+    return {"decode_llama8b_layer_window": {"ms": round(ms_w, 4), "ms_all_packed": round(ms_p, 4),
+                                            "GB_s": round(byts / ms_w / 1e6, 1),
+                                            "frac_hbm": round(byts / ms_w / 1e6 / peak_gbs, 4),
+                                            "algorithmic_bytes": byts,
+                                            "note": f"{T - R} packed tokens (112 B per pair) + {R}-token bf16 window "
+                                                    "(512 B per pair); whole call, 5 launches"}}
 
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):

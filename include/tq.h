@@ -37,7 +37,8 @@
  *   [TurboQuant] TurboQuant digest (news.hada.io 27867): "Principe de
  *                fonctionnement" (Étape 1, Étape 2), "QJL", "Expériences et
  *                résultats".
- *   [NSNQuant]   "NSNQuant: ...", Résumé Technique, Méthodologie §2.
+ *   [NSNQuant]   "NSNQuant: ...", Résumé Technique, Méthodologie §2 and
+ *                §4 ("Résidus": the full-precision window).
  */
 #ifndef TQ_H_
 #define TQ_H_
@@ -284,6 +285,49 @@ int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
 /* Workspace bytes tq_decode_attention needs for these sizes (0 if invalid). */
 size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
                                 int B, int Hq, int Hkv, int64_t T);
+
+/*
+ * tq_decode_attention_window - tq_decode_attention over a packed cache plus
+ * a full-precision window of the most recent tokens.
+ * [NSNQuant] §4, "Résidus" (after KIVI): the cache is a quantized part and a
+ * residual kept in full precision; when the residual is full the caller
+ * flushes it (tq_quantize_kv / tq_quantize_kv_pair with positions T .. T+R-1
+ * into records T .. T+R-1) and empties the window.
+ *   hk ... cache_stride, B, Hq, Hkv, T, scale, out
+ *               as in tq_decode_attention (T packed tokens, possibly 0)
+ *   k_window, v_window
+ *               device [B*Hkv, window_stride, d] elements of window_dtype:
+ *               row (b*Hkv + j)*window_stride + i is token i of the window
+ *               of sequence b, KV head j - the key as the model produced it
+ *               (before RoPE) and its value; token i sits at position T + i,
+ *               where its key gets RoPE when hk has a RoPE base (T + R must
+ *               not exceed the handle's rope_max_pos)
+ *   window_dtype  TQ_F32 or TQ_BF16 (both pointers 16-byte aligned)
+ *   window_stride rows between consecutive sequences' windows (>= R)
+ *   R           window tokens, 0 .. 1024 (0 gives tq_decode_attention's
+ *               result exactly)
+ *   workspace   at least tq_decode_window_workspace_size(...) bytes
+ * The softmax runs over all T + R tokens: scores of window tokens are
+ * <RoPE(q, q_pos), RoPE(k_i, T + i)> * scale in fp32, their values enter
+ * unquantized.  Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED (R > 1024 or as
+ * tq_decode_attention), TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_decode_attention_window(const tq_rotation* hk, const tq_rotation* hv,
+                               const void* q, int q_dtype, const int64_t* q_pos,
+                               const uint8_t* k_codes, const uint8_t* k_signs,
+                               const float* k_norms, const uint8_t* v_codes,
+                               const uint8_t* v_signs, const float* v_norms,
+                               int64_t cache_stride, const void* k_window,
+                               const void* v_window, int window_dtype,
+                               int64_t window_stride, int R, int B, int Hq,
+                               int Hkv, int64_t T, float scale, float* out,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Workspace bytes tq_decode_attention_window needs (0 if invalid). */
+size_t tq_decode_window_workspace_size(const tq_rotation* hk,
+                                       const tq_rotation* hv, int B, int Hq,
+                                       int Hkv, int64_t T, int R);
 
 /*
  * tq_encoder_attention - bidirectional attention of S queries per head over

@@ -65,4 +65,5 @@ def test_bad_arguments_are_rejected_on_host():
     assert tq._lib.tq_build_rotation(96, 2, 0, np.ones(96, np.int8).ctypes.data, None, np.zeros((96, 96), np.float32).ctypes.data,
                                      96, 0.0, 0, ctypes.byref(h)) == tq.TQ_EUNSUPPORTED
     assert tq._lib.tq_decode_workspace_size(None, None, 1, 1, 1, 10) == 0
+    assert tq._lib.tq_decode_window_workspace_size(None, None, 1, 1, 1, 10, 4) == 0
     assert tq._lib.tq_quantize_kv(None, None, 0, 1, 64, None, 1, 0, 0, None, None, None, 1, None) == tq.TQ_EINVAL

@@ -59,9 +59,10 @@ struct DecodeParams {
   int64_t T;
   int64_t chunk;           // tokens per split (multiple of kTile)
   int n_splits;
+  int n_slots;             // partial records per head: n_splits, then one per window chunk
   const uint32_t* qfrag;   // [BH][2][NT][8][32][2]
   const float2* kconst;    // [BH][2][8]: (sum_k mu_k B_k, 1 / fp16 range scale)
-  float* partial;          // [BH][n_splits][G][2 + 2 kD]
+  float* partial;          // [BH][n_slots][G][2 + 2 kD]
   float score_scale;       // softmax scale * log2(e)
   float qjl;               // sqrt(pi/2) / m
   float walsh_k[4];
@@ -499,7 +500,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
     }
   }
   __syncthreads();
-  float* out = p.partial + (static_cast<size_t>(bh) * p.n_splits + split) * G * REC;
+  float* out = p.partial + (static_cast<size_t>(bh) * p.n_slots + split) * G * REC;
   for (int idx = threadIdx.x; idx < G * REC; idx += blockDim.x) {
     const int h = idx / REC, k = idx % REC;
     float M = -INFINITY;
@@ -736,6 +737,188 @@ __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __res
   out[(static_cast<size_t>(bh) * G + h) * kD + i] = y * (dsigns[i] * rsqrtf(static_cast<float>(kD)));
 }
 
+// (cos, sin) of pos * theta_j from the two RoPE tables: the angle of the
+// coarse row pos >> kRopeLoBits plus that of the fine row pos mod kRopeLoRows.
+__device__ __forceinline__ float2 rope_cs(const float2* __restrict__ rope_hi, const float2* __restrict__ rope_lo,
+                                          int64_t pos, int j) {
+  const float2 a = rope_hi[(pos >> kRopeLoBits) * (kD / 2) + j];
+  const float2 c = rope_lo[(pos & (kRopeLoRows - 1)) * (kD / 2) + j];
+  return make_float2(a.x * c.x - a.y * c.y, a.y * c.x + a.x * c.y);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x) {
+  if constexpr (sizeof(T) == 4) return x;
+  else return __bfloat162float(x);
+}
+
+constexpr int kWindowMax = 1024;   // tokens of a full-precision window
+constexpr int kWinChunk = 32;      // window tokens per block, one partial record each
+
+// The full-precision window ([NSNQuant] §4, "Résidus", after KIVI): the R most
+// recent tokens of each sequence, kept as the model produced them, scored and
+// summed exactly and written as split partials of their own, which the merge
+// combines with the packed cache's partials by the same log-sum-exp rule.
+// One block of four warps per (chunk of 32 window tokens, sequence b and KV
+// head), for all G query heads of the KV head:
+//  1. q' = RoPE(q, q_pos) in the original space (thread i: coordinate i).
+//  2. Logits: warp w takes tokens w + 4u; lane l holds coordinates l + 32c
+//     (c < 4), so both members of a RoPE pair (j, j + kD/2) sit in one lane;
+//     token t gets RoPE at position T + t (after the packed part).  The key
+//     rows of all of a warp's tokens are loaded before any is used.
+//  3. Softmax statistics of the chunk per head (max, then 2^(logit - max)
+//     and their sum), one warp per head, one lane per token.
+//  4. acc = sum_t w_t v_t in the original space: lane l of warp w sums
+//     coordinates 4l .. 4l + 3 over the warp's tokens (vector loads), the four
+//     warps' sums meet in shared memory; then y = Pi_V acc = H (D_V acc) /
+//     sqrt(d) with the value handle's signs D_V, the rotated space the merge
+//     applies Pi_V^T to.  The QJL half of the partial is zero.
+template <typename TW, int G>
+__global__ void __launch_bounds__(kD) decode_window_kernel(
+    const void* __restrict__ q, int q_f32, const int64_t* __restrict__ q_pos, int Hkv, const TW* __restrict__ k_win,
+    const TW* __restrict__ v_win, int64_t win_stride, int R, int64_t T, const float* __restrict__ v_dsigns,
+    const float2* __restrict__ rope_hi, const float2* __restrict__ rope_lo, int64_t rope_max_pos, int rope,
+    float score_scale, float* __restrict__ partial, int n_slots, int slot0) {
+  constexpr int REC = 2 + 2 * kD;
+  constexpr int TPW = kWinChunk / 4;   // tokens per warp
+  __shared__ __align__(16) float qs[G][kD];
+  __shared__ __align__(16) float red[4][G][kD];   // per-warp value sums (first: the raw query)
+  __shared__ float lg[G][kWinChunk];              // logits, then weights
+  __shared__ float stat[2][G];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.y, b = bh / Hkv, chunk = blockIdx.x;
+  const int t0 = chunk * kWinChunk;
+  const int n = min(kWinChunk, R - t0);   // >= 1: the host launches ceil(R / kWinChunk) chunks
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  float* qraw = &red[0][0][0];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const size_t at = (static_cast<size_t>(bh) * G + h) * kD + tid;
+    qraw[h * kD + tid] =
+        q_f32 ? static_cast<const float*>(q)[at] : __bfloat162float(static_cast<const __nv_bfloat16*>(q)[at]);
+  }
+  __syncthreads();
+  {
+    const int j = tid & (kD / 2 - 1);
+    float2 cs = make_float2(1.f, 0.f);
+    bool bad = false;
+    if (rope) {
+      const int64_t pos = q_pos[b];
+      bad = pos < 0 || pos >= rope_max_pos;
+      if (!bad) cs = rope_cs(rope_hi, rope_lo, pos, j);
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float v = qraw[h * kD + tid];
+      if (rope) {
+        const float x1 = qraw[h * kD + j], x2 = qraw[h * kD + j + kD / 2];
+        v = bad ? __int_as_float(0x7fc00000) : (tid < kD / 2 ? x1 * cs.x - x2 * cs.y : x2 * cs.x + x1 * cs.y);
+      }
+      qs[h][tid] = v;
+    }
+  }
+  __syncthreads();
+  const size_t row0 = static_cast<size_t>(bh) * win_stride + t0;
+  {
+    float x[TPW][4];
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+      const int t = warp + 4 * u;
+      const TW* kr = k_win + (row0 + (t < n ? t : 0)) * kD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) x[u][c] = to_f32(kr[lane + 32 * c]);
+    }
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+      const int t = warp + 4 * u;
+      if (rope) {
+        const int64_t pos = T + t0 + t;   // below rope_max_pos for t < n (checked by the host)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const float2 cs = t < n ? rope_cs(rope_hi, rope_lo, pos, lane + 32 * c) : make_float2(1.f, 0.f);
+          const float x1 = x[u][c], x2 = x[u][c + 2];
+          x[u][c] = x1 * cs.x - x2 * cs.y;
+          x[u][c + 2] = x2 * cs.x + x1 * cs.y;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) s = fmaf(qs[h][lane + 32 * c], x[u][c], s);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) lg[h][t] = t < n ? s * score_scale : -INFINITY;
+      }
+    }
+  }
+  __syncthreads();
+  for (int h = warp; h < G; h += 4) {
+    const float s = lg[h][lane];
+    float mx = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float e = exp2f(s - mx);
+    lg[h][lane] = e;
+    float l = e;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      stat[0][h] = mx;
+      stat[1][h] = l;
+    }
+  }
+  __syncthreads();
+  {
+    float vv[TPW][4];
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+      const int t = warp + 4 * u;
+      const TW* vr = v_win + (row0 + (t < n ? t : 0)) * kD + 4 * lane;
+      if constexpr (sizeof(TW) == 4) {
+        const float4 w = *reinterpret_cast<const float4*>(vr);
+        vv[u][0] = w.x, vv[u][1] = w.y, vv[u][2] = w.z, vv[u][3] = w.w;
+      } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(vr);
+        vv[u][0] = __uint_as_float(w.x << 16), vv[u][1] = __uint_as_float(w.x & 0xFFFF0000u);
+        vv[u][2] = __uint_as_float(w.y << 16), vv[u][3] = __uint_as_float(w.y & 0xFFFF0000u);
+      }
+    }
+    float acc[G][4];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+#pragma unroll
+    for (int u = 0; u < TPW; ++u) {
+      const int t = warp + 4 * u;
+      if (t < n) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float w = lg[h][t];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[h][c] = fmaf(w, vv[u][c], acc[h][c]);
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      *reinterpret_cast<float4*>(&red[warp][h][4 * lane]) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+  }
+  __syncthreads();
+  const float dsg = v_dsigns[tid];
+  for (int h = 0; h < G; ++h) {
+    float y = ((red[0][h][tid] + red[1][h][tid]) + (red[2][h][tid] + red[3][h][tid])) * dsg;
+    fwht_group(y, tid, qs[0]);
+    y *= rsqrtf(static_cast<float>(kD));
+    float* rec = partial + ((static_cast<size_t>(bh) * n_slots + slot0 + chunk) * G + h) * REC;
+    if (tid == 0) {
+      rec[0] = stat[0][h];
+      rec[1] = stat[1][h];
+    }
+    rec[2 + tid] = y;
+    rec[2 + kD + tid] = 0.f;
+  }
+}
+
 thread_local cudaEvent_t g_prof_begin = nullptr;
 thread_local cudaEvent_t g_prof_end = nullptr;
 
@@ -767,12 +950,13 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 size_t kconst_bytes(int BH) { return static_cast<size_t>(BH) * 2 * 8 * sizeof(float2); }
 
-size_t workspace_for(int B, int Hq, int Hkv, int64_t T) {
+size_t workspace_for(int B, int Hq, int Hkv, int64_t T, int R = 0) {
   const int G = Hq / Hkv;
   const int BH = B * Hkv;
   const SplitPlan sp = plan_splits(BH, T);
+  const int slots = sp.n_splits + (R + kWinChunk - 1) / kWinChunk;
   return align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)) +
-         align256(static_cast<size_t>(BH) * sp.n_splits * G * (2 + 2 * kD) * sizeof(float));
+         align256(static_cast<size_t>(BH) * slots * G * (2 + 2 * kD) * sizeof(float));
 }
 
 // Launch that may overlap the tail of the previous kernel on the stream
@@ -833,7 +1017,7 @@ int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64
 
 int launch_merge(int G, int BH, const float* partial, int n_splits, const tq_rotation* hv, float* out, cudaStream_t s) {
   const float qjl = static_cast<float>(kQjlConst / hv->m);
-  const size_t fsb = static_cast<size_t>(n_splits) * G * sizeof(float);   // <= 1184 * 8 * 4 bytes
+  const size_t fsb = static_cast<size_t>(n_splits) * G * sizeof(float);   // <= (1184 + 32) * 8 * 4 bytes
   switch (G) {
     case 1: return launch_pdl(decode_merge_kernel<1>, dim3(BH), dim3(kD * 1), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
     case 2: return launch_pdl(decode_merge_kernel<2>, dim3(BH), dim3(kD * 2), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
@@ -864,19 +1048,47 @@ extern "C" int tq_profile_next_decode(void* ev_begin, void* ev_end) {
   return TQ_OK;
 }
 
-extern "C" size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv, int B, int Hq, int Hkv,
-                                           int64_t T) {
-  if (!hk || !hv || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0) return 0;
-  return workspace_for(B, Hq, Hkv, T);
+namespace {
+
+int launch_window(int G, int win_dtype, int q_dtype, int BH, int Hkv, const void* q, const int64_t* q_pos,
+                  const tq_rotation* hk, const tq_rotation* hv, int rope, const void* k_win, const void* v_win,
+                  int64_t win_stride, int R, int64_t T, float score_scale, float* partial, int n_slots, int slot,
+                  cudaStream_t s) {
+  const int q_f32 = q_dtype == TQ_F32 ? 1 : 0;
+  const dim3 grid((R + kWinChunk - 1) / kWinChunk, BH);
+#define TQ_WINDOW(TW, GG)                                                                                            \
+  return launch_pdl(decode_window_kernel<TW, GG>, grid, dim3(kD), 0, s, q, q_f32, q_pos, Hkv,                         \
+                    static_cast<const TW*>(k_win), static_cast<const TW*>(v_win), win_stride, R, T, hv->d_signs,   \
+                    hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope, score_scale, partial, n_slots, slot)
+  if (win_dtype == TQ_F32) {
+    switch (G) {
+      case 1: TQ_WINDOW(float, 1);
+      case 2: TQ_WINDOW(float, 2);
+      case 4: TQ_WINDOW(float, 4);
+      case 8: TQ_WINDOW(float, 8);
+    }
+  } else {
+    switch (G) {
+      case 1: TQ_WINDOW(__nv_bfloat16, 1);
+      case 2: TQ_WINDOW(__nv_bfloat16, 2);
+      case 4: TQ_WINDOW(__nv_bfloat16, 4);
+      case 8: TQ_WINDOW(__nv_bfloat16, 8);
+    }
+  }
+#undef TQ_WINDOW
+  return TQ_EUNSUPPORTED;
 }
 
-extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
-                                   const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
-                                   const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
-                                   const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
-                                   float scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
-  const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
-  g_prof_begin = g_prof_end = nullptr;
+// One decode step over the packed cache and, when R > 0, a full-precision
+// window of the R tokens after it.  Launch order: q-prep, window, split,
+// merge; each waits (griddepcontrol.wait) for the launch before it, so the
+// chain orders all four.
+int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype, const int64_t* q_pos,
+                const uint8_t* k_codes, const uint8_t* k_signs, const float* k_norms, const uint8_t* v_codes,
+                const uint8_t* v_signs, const float* v_norms, int64_t cache_stride, const void* k_win,
+                const void* v_win, int win_dtype, int64_t win_stride, int R, int B, int Hq, int Hkv, int64_t T,
+                float scale, float* out, void* workspace, size_t workspace_bytes, cudaStream_t s,
+                cudaEvent_t prof_begin, cudaEvent_t prof_end) {
   if (!hk || !hv || !q || !out) return TQ_EINVAL;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_EINVAL;
   if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || !std::isfinite(scale)) return TQ_EINVAL;
@@ -893,26 +1105,39 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
     for (const void* ptr : ptrs)
       if (!tq::aligned16(ptr)) return TQ_EINVAL;
   }
-  if (hk->rope_base > 0.0 && !q_pos) return TQ_EINVAL;
+  const int rope = hk->rope_base > 0.0 ? 1 : 0;
+  if (R < 0) return TQ_EINVAL;
+  if (R > kWindowMax) return TQ_EUNSUPPORTED;
+  if (R > 0) {
+    if (!k_win || !v_win || win_stride < R) return TQ_EINVAL;
+    if (win_dtype != TQ_F32 && win_dtype != TQ_BF16) return TQ_EINVAL;
+    if (!tq::aligned16(k_win) || !tq::aligned16(v_win)) return TQ_EINVAL;   // rows are read as vectors
+    if (rope && T + R > hk->rope_max_pos) return TQ_EINVAL;
+  }
+  if (rope && !q_pos) return TQ_EINVAL;
   const int BH = B * Hkv;
-  const size_t need = workspace_for(B, Hq, Hkv, T);
+  const size_t need = workspace_for(B, Hq, Hkv, T, R);
   if (!workspace || workspace_bytes < need) return TQ_EWORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TQ_EINVAL;
   if (!tq::on_handle_device(hk) || !tq::on_handle_device(hv)) return TQ_EINVAL;
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const SplitPlan sp = plan_splits(BH, T);
-  const int NT = num_tiles_n(G);
+  const int n_slots = sp.n_splits + (R + kWinChunk - 1) / kWinChunk;   // window chunks after the splits
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws);
   float2* kconst = reinterpret_cast<float2*>(ws + align256(frag_bytes(BH, G)));
   float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
+  const float score_scale = scale * 1.4426950408889634f;
 
-  const int rope = hk->rope_base > 0.0 ? 1 : 0;
   int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, reinterpret_cast<uint16_t*>(qfrag), kconst, s);
   if (st != TQ_OK) return st;
   st = tq::launch_status();
   if (st != TQ_OK) return st;
+  if (R > 0) {
+    st = launch_window(G, win_dtype, q_dtype, BH, Hkv, q, q_pos, hk, hv, rope, k_win, v_win, win_stride, R, T, score_scale,
+                       partial, n_slots, sp.n_splits, s);
+    if (st != TQ_OK) return st;
+  }
 
   DecodeParams p{};
   p.k_codes = k_codes;
@@ -925,10 +1150,11 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   p.T = T;
   p.chunk = sp.chunk;
   p.n_splits = sp.n_splits;
+  p.n_slots = n_slots;
   p.qfrag = qfrag;
   p.kconst = kconst;
   p.partial = partial;
-  p.score_scale = scale * 1.4426950408889634f;
+  p.score_scale = score_scale;
   p.one_h = kOneH2;
   p.one_b = kOneB2;
   p.qjl = static_cast<float>(kQjlConst / hk->m);
@@ -945,7 +1171,47 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   }
   if (st != TQ_OK) return st;
   if (prof_end && cudaEventRecord(prof_end, s) != cudaSuccess) return TQ_ECUDA;
-  return launch_merge(G, BH, partial, sp.n_splits, hv, out, s);
+  return launch_merge(G, BH, partial, n_slots, hv, out, s);
+}
+
+}  // namespace
+
+extern "C" size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv, int B, int Hq, int Hkv,
+                                           int64_t T) {
+  if (!hk || !hv || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0) return 0;
+  return workspace_for(B, Hq, Hkv, T);
+}
+
+extern "C" size_t tq_decode_window_workspace_size(const tq_rotation* hk, const tq_rotation* hv, int B, int Hq,
+                                                  int Hkv, int64_t T, int R) {
+  if (!hk || !hv || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || R < 0 || R > kWindowMax) return 0;
+  return workspace_for(B, Hq, Hkv, T, R);
+}
+
+extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
+                                   const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
+                                   const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
+                                   const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
+                                   float scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
+  g_prof_begin = g_prof_end = nullptr;
+  return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
+                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, scale, out, workspace, workspace_bytes,
+                     static_cast<cudaStream_t>(stream), prof_begin, prof_end);
+}
+
+extern "C" int tq_decode_attention_window(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
+                                          const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
+                                          const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
+                                          const float* v_norms, int64_t cache_stride, const void* k_window,
+                                          const void* v_window, int window_dtype, int64_t window_stride, int R,
+                                          int B, int Hq, int Hkv, int64_t T, float scale, float* out,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
+  g_prof_begin = g_prof_end = nullptr;
+  return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
+                     k_window, v_window, window_dtype, window_stride, R, B, Hq, Hkv, T, scale, out, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end);
 }
 
 // ---------------------------------------------------------------------------

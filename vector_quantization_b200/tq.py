@@ -47,6 +47,9 @@ def _load():
         "tq_decode_attention": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
                                       c_i64, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
+        "tq_decode_attention_window": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_p, c_p,
+                                             c_i, c_i64, c_i, c_i, c_i, c_i, c_i64, c_f, c_p, c_p, c_sz, c_p]),
+        "tq_decode_window_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64, c_i]),
         "tq_profile_next_decode": (c_i, [c_p, c_p]),
         "tq_encoder_attention": (c_i, [c_p, c_p, c_p, c_i, c_i64, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i,
                                        c_i, c_i, c_i64, c_f, c_p, c_p, c_sz, c_p]),
@@ -278,6 +281,42 @@ def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cach
                                     _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, T,
                                     float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream_ptr(stream)), "tq_decode_attention")
+    return out
+
+
+def decode_window_workspace_size(rot_k: Rotation, rot_v: Rotation, B: int, Hq: int, Hkv: int, T: int,
+                                 R: int) -> int:
+    return _lib.tq_decode_window_workspace_size(rot_k.handle, rot_v.handle, B, Hq, Hkv, T, R)
+
+
+def decode_attention_window(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, T: int, k_window,
+                            v_window, R: int, *, scale: float | None = None, out=None, workspace=None, stream=None):
+    """One decode step over the first T records of the packed caches plus the
+    first R tokens of the full-precision windows k_window, v_window
+    ([B, Hkv, cap_w, d], float32 or bfloat16, keys before RoPE); window token
+    i sits at position T + i.  Returns out [B, Hq, d] float32."""
+    import torch
+    B, Hq, d = q.shape
+    kc, ks, kn = k_cache
+    vc, vs, vn = v_cache
+    Hkv, cap = kc.shape[1], kc.shape[2]
+    for t in (kc, ks, kn, vc, vs, vn, k_window, v_window):
+        if not t.is_contiguous():
+            raise ValueError("cache and window arrays must be contiguous")
+    if k_window.shape != v_window.shape or k_window.dtype != v_window.dtype:
+        raise ValueError("k_window and v_window must share shape and dtype")
+    q = q.contiguous()
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(decode_window_workspace_size(rot_k, rot_v, B, Hq, Hkv, T, R), q.device)
+    _check(_lib.tq_decode_attention_window(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos), _ptr(kc),
+                                           _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, _ptr(k_window),
+                                           _ptr(v_window), _dtype_code(k_window), k_window.shape[2], R, B, Hq, Hkv,
+                                           T, float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                           _stream_ptr(stream)), "tq_decode_attention_window")
     return out
 
 
