@@ -62,3 +62,27 @@ def compare_records(rot, gpu, enc, x_norm_scale=None):
     assert np.all(np.abs(g_norms[same, 1] - nr) <= 1e-6 * nr + 2e-6 * nx[same])
     return {"code_mismatch_flagged": int(diff.sum()), "flagged": int(enc["code_flags"].sum()),
             "vectors_all_codes_equal": int(same.sum())}
+
+
+def _oracle_slice(rot_o, x, pos=None):
+    """The oracle's own records of one (sequence, KV head) slice x [T, d] of
+    the synthetic input, as [1, 1, T, ...] arrays."""
+    codes, signs, norms, enc = oracle_records(rot_o, x, pos)
+    T = x.shape[0]
+    return tuple(a.reshape(1, 1, T, -1) for a in (codes, signs, norms)), enc
+
+
+def check_and_substitute(rot_o, cache, b, j, x, pos=None):
+    """GPU encode parity of the first T = len(x) records of slice (b, j) of a
+    device cache [B, H, cap, ...] (codes equal except boundary-flagged
+    coordinates), then those records are overwritten with the oracle's own
+    encoding of x, so that an attention launch over the cache and the oracle
+    read the same bytes without the oracle reading anything the GPU wrote.
+    Returns the oracle records as [1, 1, T, ...] arrays."""
+    rec, enc = _oracle_slice(rot_o, x, pos)
+    T = x.shape[0]
+    compare_records(rot_o, tuple(a[b, j, :T].cpu().numpy().reshape(T, -1) for a in cache), enc)
+    import torch
+    for a, r in zip(cache, rec):
+        a[b, j, :T] = torch.from_numpy(np.ascontiguousarray(r[0, 0])).to(a.device)
+    return rec

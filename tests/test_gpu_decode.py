@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import synth
-from helpers import assert_close, oracle_records, oracle_rotation
+from helpers import assert_close, check_and_substitute, oracle_records, oracle_rotation
 from oracle import attention as at
 
 pytestmark = pytest.mark.gpu
@@ -127,9 +127,11 @@ def test_tiny_workload_end_to_end(cuda_device):
 def test_decode_full_size_sampled(cuda_device, bits):
     """The Llama-3.1-8B-shaped decode layer at full size (batch 16, 32 query
     heads over 8 KV heads, 32768 cached tokens, heavy-tailed bf16 K/V, RoPE)
-    in the launch configuration the bench times: GPU-encoded caches, one
-    decode launch; sampled (sequence, KV head) pairs checked against the
-    oracle's attention over the very same packed records."""
+    in the launch configuration the bench times.  The caches are GPU-encoded;
+    sampled (sequence, KV head) slices are checked against the oracle's
+    encoding of the same inputs and replaced by the oracle's records; one
+    full-size decode launch; the sampled outputs against the oracle's
+    attention over its own records."""
     from vector_quantization_b200 import tq
     dev = torch.device("cuda:0")
     cfg = synth.CONFIGS["llama31_8b_gqa_decode"]
@@ -139,26 +141,34 @@ def test_decode_full_size_sampled(cuda_device, bits):
     rv = tq.Rotation(D, bits, synth.rotation_randomness(D, [seed, 12]))
     rk_o, _ = oracle_rotation(D, bits, [seed, 11], rope=10000.0)
     rv_o, _ = oracle_rotation(D, bits, [seed, 12])
-    kc = tq.quantize_kv(rk, synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 13], dev), apply_rope=True, pos_period=T)
-    vc = tq.quantize_kv(rv, synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 14], dev))
+    samples = [(0, 0), (B - 1, Hkv - 1), (7, 3)]
+    xk = synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 13], dev)
+    kc = tq.quantize_kv(rk, xk, apply_rope=True, pos_period=T)
+    xk_s = {bj: xk[bj].float().cpu().numpy() for bj in samples}
+    del xk
+    xv = synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 14], dev)
+    vc = tq.quantize_kv(rv, xv)
+    xv_s = {bj: xv[bj].float().cpu().numpy() for bj in samples}
+    del xv
+    torch.cuda.synchronize()
+    ko = {bj: check_and_substitute(rk_o, kc, *bj, xk_s[bj], np.arange(T)) for bj in samples}
+    vo = {bj: check_and_substitute(rv_o, vc, *bj, xv_s[bj]) for bj in samples}
     q = synth.heavy_tailed_torch((B, Hq, D), [seed, 15], dev)
     q_pos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
     out = tq.decode_attention(rk, rv, q, q_pos, kc, vc, T)
     torch.cuda.synchronize()
-    for b, j in [(0, 0), (B - 1, Hkv - 1), (7, 3)]:
-        kk = tuple(a[b:b + 1, j:j + 1].cpu().numpy() for a in kc)
-        vv = tuple(a[b:b + 1, j:j + 1].cpu().numpy() for a in vc)
+    for b, j in samples:
         qq = q[b:b + 1, j * G:(j + 1) * G].float().cpu().numpy()
-        ref = at.decode_attention(rk_o, rv_o, qq, [T - 1], kk, vv, 1 / np.sqrt(D))
+        ref = at.decode_attention(rk_o, rv_o, qq, [T - 1], ko[b, j], vo[b, j], 1 / np.sqrt(D))
         assert_close(out[b:b + 1, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"bits {bits} seq {b} kv-head {j}")
 
 
 def test_decode_70b_slice_full_size_sampled(cuda_device):
     """The Llama-3.1-70B-shaped long-context slice at full size (one
     sequence, 64 query heads over 8 KV heads: G = 8, 2^20 cached tokens,
-    2+1 bits) in the launch configuration the bench times; one KV head's 8
-    query heads checked against the oracle's attention over the same packed
-    records."""
+    2+1 bits) in the launch configuration the bench times; one KV head's
+    slice is checked against and replaced by the oracle's records, and its
+    8 query heads' outputs are checked against the oracle's attention."""
     from vector_quantization_b200 import tq
     dev = torch.device("cuda:0")
     c = synth.CONFIGS["llama31_70b_long_slice"]
@@ -168,15 +178,22 @@ def test_decode_70b_slice_full_size_sampled(cuda_device):
     rv = tq.Rotation(D, 2, synth.rotation_randomness(D, [seed, 2]))
     rk_o, _ = oracle_rotation(D, 2, [seed, 1], rope=c["rope_base"])
     rv_o, _ = oracle_rotation(D, 2, [seed, 2])
-    kc = tq.quantize_kv(rk, synth.heavy_tailed_torch((1, Hkv, T, D), [seed, 3], dev), apply_rope=True, pos_period=T)
-    vc = tq.quantize_kv(rv, synth.heavy_tailed_torch((1, Hkv, T, D), [seed, 4], dev))
+    j = Hkv - 1
+    xk = synth.heavy_tailed_torch((1, Hkv, T, D), [seed, 3], dev)
+    kc = tq.quantize_kv(rk, xk, apply_rope=True, pos_period=T)
+    xk_j = xk[0, j].float().cpu().numpy()
+    del xk
+    xv = synth.heavy_tailed_torch((1, Hkv, T, D), [seed, 4], dev)
+    vc = tq.quantize_kv(rv, xv)
+    xv_j = xv[0, j].float().cpu().numpy()
+    del xv
+    torch.cuda.synchronize()
+    kk = check_and_substitute(rk_o, kc, 0, j, xk_j, np.arange(T))
+    vv = check_and_substitute(rv_o, vc, 0, j, xv_j)
     q = synth.heavy_tailed_torch((1, Hq, D), [seed, 5], dev)
     q_pos = torch.full((1,), T - 1, dtype=torch.int64, device=dev)
     out = tq.decode_attention(rk, rv, q, q_pos, kc, vc, T)
     torch.cuda.synchronize()
-    j = Hkv - 1
-    kk = tuple(a[:, j:j + 1].cpu().numpy() for a in kc)
-    vv = tuple(a[:, j:j + 1].cpu().numpy() for a in vc)
     qq = q[:, j * G:(j + 1) * G].float().cpu().numpy()
     ref = at.decode_attention(rk_o, rv_o, qq, [T - 1], kk, vv, 1 / np.sqrt(D))
     assert_close(out[:, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"70B slice kv-head {j}")

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import synth
-from helpers import assert_close, compare_records, oracle_records, oracle_rotation
+from helpers import assert_close, check_and_substitute, compare_records, oracle_records, oracle_rotation
 from oracle import attention as at
 
 pytestmark = pytest.mark.gpu
@@ -190,3 +190,46 @@ def test_streaming_append_and_flush(cuda_device):
             _, _, _, enc = oracle_records(rk_o, k_all[:, :, rows].reshape(-1, D), np.tile(np.arange(T, T + W), B * Hkv))
             compare_records(rk_o, gpu_k, enc)
             T, R = T + W, 0
+
+
+def test_window_full_size_sampled(cuda_device):
+    """The bench's window workload at full size, in its launch configuration:
+    the Llama-3.1-8B-shaped layer (batch 16, 32 query heads over 8 KV heads,
+    2+1 bits) whose 32768 tokens are 32640 packed ones plus a bf16 window of
+    the last 128.  GPU-encoded caches; sampled slices checked against the
+    oracle's encoding and replaced by the oracle's records; one launch; the
+    sampled outputs against the oracle."""
+    from vector_quantization_b200 import tq
+    dev = torch.device("cuda:0")
+    c = synth.CONFIGS["llama31_8b_gqa_decode"]
+    B, Hq, Hkv, T, seed = c["batch"], c["q_heads"], c["kv_heads"], c["tokens"], c["seed"]
+    G, R = Hq // Hkv, 128
+    Tp = T - R
+    rk = tq.Rotation(D, 2, synth.rotation_randomness(D, [seed, 8, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(D, 2, synth.rotation_randomness(D, [seed, 8, 2]))
+    rk_o, _ = oracle_rotation(D, 2, [seed, 8, 1], rope=c["rope_base"])
+    rv_o, _ = oracle_rotation(D, 2, [seed, 8, 2])
+    samples = [(0, 0), (B - 1, Hkv - 1), (5, 6)]
+    xk = synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 8, 3], dev)
+    kc = tq.quantize_kv(rk, xk, apply_rope=True, pos_period=T)
+    kw = xk[:, :, Tp:].to(torch.bfloat16).contiguous()
+    xk_s = {bj: xk[bj][:Tp].float().cpu().numpy() for bj in samples}
+    del xk
+    xv = synth.heavy_tailed_torch((B, Hkv, T, D), [seed, 8, 4], dev)
+    vc = tq.quantize_kv(rv, xv)
+    vw = xv[:, :, Tp:].to(torch.bfloat16).contiguous()
+    xv_s = {bj: xv[bj][:Tp].float().cpu().numpy() for bj in samples}
+    del xv
+    torch.cuda.synchronize()
+    ko = {bj: check_and_substitute(rk_o, kc, *bj, xk_s[bj], np.arange(Tp)) for bj in samples}
+    vo = {bj: check_and_substitute(rv_o, vc, *bj, xv_s[bj]) for bj in samples}
+    q = synth.heavy_tailed_torch((B, Hq, D), [seed, 8, 5], dev)
+    qpos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    out = tq.decode_attention_window(rk, rv, q, qpos, kc, vc, Tp, kw, vw, R)
+    torch.cuda.synchronize()
+    for b, j in samples:
+        qq = q[b:b + 1, j * G:(j + 1) * G].float().cpu().numpy()
+        ref = at.decode_attention_window(rk_o, rv_o, qq, [T - 1], ko[b, j], vo[b, j],
+                                         kw[b:b + 1, j:j + 1].double().cpu().numpy(),
+                                         vw[b:b + 1, j:j + 1].double().cpu().numpy(), 1 / np.sqrt(D))
+        assert_close(out[b:b + 1, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"seq {b} kv-head {j}")
