@@ -193,6 +193,120 @@ def oracle_baseline(c, args, budget_s=12.0, max_steps=None):
 
 
 
+def _oracle_rate(fn, units, min_s=1.5):
+    """Units per second of fn on the host cores: at least one call and min_s."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_s:
+            return units * n / el, n, el / n
+
+
+def oracle_extra_baselines(select):
+    """The oracle as it stands timed beside each secondary line, on a bounded
+    sample of that line's workload (same laws and sizes per unit), in that
+    line's unit."""
+    import synth
+    from oracle import attention as at
+    from oracle import codec, rotation as ro
+    from oracle import search as osearch
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    out = {}
+
+    def base(value, unit, sample):
+        return {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample}
+
+    def packed(rot, x, pos):
+        e = codec.encode(rot, x, pos)
+        return (codec.pack_planes(e["codes"], rot.bits)[None, None], codec.pack_bits(e["signs"])[None, None],
+                np.stack([e["norm"], e["rnorm"]], 1).astype(np.float32)[None, None])
+
+    d = 128
+    if select & {"encode_70b_slice", "decode_70b_slice"}:
+        c = synth.CONFIGS["llama31_70b_long_slice"]
+        n = 8192
+        rk = ro.build_rotation(d, 2, synth.rotation_randomness(d, [c["seed"], 1]), rope_base=c["rope_base"])
+        rv = ro.build_rotation(d, 2, synth.rotation_randomness(d, [c["seed"], 2]))
+        k = synth.heavy_tailed((1, 1, n, d), [c["seed"], 91]).reshape(n, d)
+        v = synth.heavy_tailed((1, 1, n, d), [c["seed"], 92]).reshape(n, d)
+        if "encode_70b_slice" in select:
+            ne = 4096
+            r, calls, per = _oracle_rate(lambda: (codec.encode(rk, k[:ne], np.arange(ne)), codec.encode(rv, v[:ne])),
+                                         2 * ne)
+            out["encode_70b_slice"] = base(r, "vectors/s", f"{ne} keys (RoPE) + {ne} values, d 128, 2+1 bits; "
+                                                           f"{calls} calls, {per:.2f} s each")
+        if "decode_70b_slice" in select:
+            G = c["q_heads"] // c["kv_heads"]
+            kc, vc = packed(rk, k, np.arange(n)), packed(rv, v, None)
+            q = synth.heavy_tailed((1, G, d), [c["seed"], 93])
+            r, calls, per = _oracle_rate(lambda: at.decode_attention(rk, rv, q, [n - 1], kc, vc, 1 / np.sqrt(d)), n)
+            out["decode_70b_slice"] = base(r, "tokens/s", f"one KV head with its {G} query heads over {n} cached "
+                                                          f"tokens (the slice has 2^20; the oracle's time is linear "
+                                                          f"in tokens); {calls} calls, {per:.2f} s each")
+    if "encoder_esm2_layer" in select:
+        c = synth.CONFIGS["esm2_650m_encoder"]
+        T, de = c["tokens"], c["head_dim"]
+        rk = ro.build_rotation(de, 2, synth.rotation_randomness(de, [c["seed"], 1]), rope_base=c["rope_base"])
+        rv = ro.build_rotation(de, 2, synth.rotation_randomness(de, [c["seed"], 2]))
+        x = synth.lognormal_channels((1, 3, T, de), [c["seed"], 94])
+        kc, vc = packed(rk, x[0, 0], np.arange(T)), packed(rv, x[0, 1], None)
+        q = x[:, 2:3]
+        flops = 2 * T * T * 2 * (de + de)
+        r, calls, per = _oracle_rate(lambda: at.encoder_attention(rk, rv, q, kc, vc, 1 / np.sqrt(de)), flops / 1e12)
+        out["encoder_esm2_layer"] = base(r, "TFLOP/s", f"one head of the layer (S = T = {T}, d {de}, 2+1 bits; the "
+                                                       f"layer has {c['batch'] * c['heads']}); {calls} calls, "
+                                                       f"{per:.2f} s each")
+    for key, bits in (("search_1m_d1536", 1), ("search_1m_d1536_3p1", 3)):
+        if "search_1m_d1536" not in select:
+            break
+        c = synth.CONFIGS["vector_search_d1536"]
+        N, ds, nq = 4096, c["dim"], 4
+        rot = ro.build_rotation(ds, bits, synth.rotation_randomness(ds, c["seed"] + bits, dense=True), "dense")
+        basis = synth.haar_basis(ds, c["seed"])
+        db = synth.anisotropic(N, ds, [c["seed"], 95], basis)
+        qs = synth.anisotropic(nq, ds, [c["seed"], 96], basis)
+        e = codec.encode(rot, db)
+        codes, signs = e["codes"], e["signs"]
+        norms = np.stack([e["norm"], e["rnorm"]], 1)
+
+        def run():
+            sc = osearch.search_scores(rot, qs, codes, signs, norms)
+            for row in sc:
+                osearch.topk_desc(row, c["top_k"])
+        r, calls, per = _oracle_rate(run, nq * N / c["n_db"])
+        out[key] = base(r, "queries/s", f"{nq} queries over {N} of the {c['n_db']} database vectors, d {ds}, "
+                                        f"{bits}+1 bits, top-{c['top_k']}, scaled to the full database; "
+                                        f"{calls} calls, {per:.2f} s each")
+    if select & {"decode_llama8b_layer_3p1", "decode_llama8b_layer_window"}:
+        c = synth.CONFIGS["llama31_8b_gqa_decode"]
+        T, G = 8192, c["q_heads"] // c["kv_heads"]
+        for key, bits, R in (("decode_llama8b_layer_3p1", 3, 0), ("decode_llama8b_layer_window", 2, 128)):
+            if key not in select:
+                continue
+            rk = ro.build_rotation(d, bits, synth.rotation_randomness(d, [c["seed"], 97]), rope_base=c["rope_base"])
+            rv = ro.build_rotation(d, bits, synth.rotation_randomness(d, [c["seed"], 98]))
+            k = synth.heavy_tailed((1, 1, T, d), [c["seed"], 99]).reshape(T, d)
+            v = synth.heavy_tailed((1, 1, T, d), [c["seed"], 100]).reshape(T, d)
+            q = synth.heavy_tailed((1, G, d), [c["seed"], 101])
+            Tp = T - R
+            kc, vc = packed(rk, k[:Tp], np.arange(Tp)), packed(rv, v[:Tp], None)
+            if R:
+                kw, vw = k[None, None, Tp:], v[None, None, Tp:]
+                fn = lambda: at.decode_attention_window(rk, rv, q, [T - 1], kc, vc, kw, vw, 1 / np.sqrt(d))
+            else:
+                fn = lambda: at.decode_attention(rk, rv, q, [T - 1], kc, vc, 1 / np.sqrt(d))
+            r, calls, per = _oracle_rate(fn, T)
+            out[key] = base(r, "tokens/s", f"one (sequence, KV head), {T} of the layer's {c['tokens']} tokens"
+                                           f"{f' ({R} in the window)' if R else ''}, {G} query heads, {bits}+1 bits "
+                                           f"(the oracle's time is linear in tokens); {calls} calls, {per:.2f} s each")
+    return out
+
+
 # --------------------------------------------------------------------------- secondary workloads
 def _time_ms(fn, reps=3, warm=2):
     import torch
@@ -208,7 +322,7 @@ def _time_ms(fn, reps=3, warm=2):
     return a.elapsed_time(b) / reps
 
 
-def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None):
+def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, cpu=True):
     """Device-timed measurements of the other rows of the path, each on its
     own workload: encode and decode on the Llama-3.1-70B-shaped 1M-token
     slice, one ESM-2-650M encoder layer, and 1M-vector d=1536 search.
@@ -234,6 +348,10 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None):
         out.update(_extra_decode_3p1(dev, peak_gbs))
     if "decode_llama8b_layer_window" in select:
         out.update(_extra_decode_window(dev, peak_gbs))
+    if cpu and not slice_tokens:
+        for key, b in oracle_extra_baselines(select).items():
+            if key in out:
+                out[key]["cpu_baseline"] = b
     return out
 
 
@@ -573,7 +691,7 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_extras:
         del kcs, vcs
         torch.cuda.empty_cache()
-        line["extras"] = run_extras(dev, peak)
+        line["extras"] = run_extras(dev, peak, cpu=not args.no_cpu_baseline)
     print(json.dumps(line), flush=True)
 
 
@@ -590,7 +708,7 @@ def main():
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
         print(json.dumps({"extras": run_extras(dev, measured_peaks()[0], args.extra, args.slice_tokens,
-                                               args.search_rows)}), flush=True)
+                                               args.search_rows, cpu=not args.no_cpu_baseline)}), flush=True)
         return
     if world > 1:
         import datetime
