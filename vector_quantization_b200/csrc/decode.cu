@@ -765,7 +765,8 @@ constexpr int kWinChunk = 32;      // window tokens per block, one partial recor
 //  2. Logits: warp w takes tokens w + 4u; lane l holds coordinates l + 32c
 //     (c < 4), so both members of a RoPE pair (j, j + kD/2) sit in one lane;
 //     token t gets RoPE at position T + t (after the packed part).  The key
-//     rows of all of a warp's tokens are loaded before any is used.
+//     and value rows of all of a warp's tokens are loaded at the start,
+//     before the query is formed.
 //  3. Softmax statistics of the chunk per head (max, then 2^(logit - max)
 //     and their sum), one warp per head, one lane per token.
 //  4. acc = sum_t w_t v_t in the original space: lane l of warp w sums
@@ -790,6 +791,37 @@ __global__ void __launch_bounds__(kD) decode_window_kernel(
   const int t0 = chunk * kWinChunk;
   const int n = min(kWinChunk, R - t0);   // >= 1: the host launches ceil(R / kWinChunk) chunks
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  // The key and value rows of this warp's tokens do not depend on the query:
+  // their loads are issued first and overlap the query's RoPE below.
+  const size_t row0 = static_cast<size_t>(bh) * win_stride + t0;
+  float x[TPW][4], vv[TPW][4];
+#pragma unroll
+  for (int u = 0; u < TPW; ++u) {
+    const int t = warp + 4 * u;
+    const size_t row = row0 + (t < n ? t : 0);
+    const TW* kr = k_win + row * kD;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) x[u][c] = to_f32(kr[lane + 32 * c]);
+    const TW* vr = v_win + row * kD + 4 * lane;
+    if constexpr (sizeof(TW) == 4) {
+      const float4 w = *reinterpret_cast<const float4*>(vr);
+      vv[u][0] = w.x, vv[u][1] = w.y, vv[u][2] = w.z, vv[u][3] = w.w;
+    } else {
+      const uint2 w = *reinterpret_cast<const uint2*>(vr);
+      vv[u][0] = __uint_as_float(w.x << 16), vv[u][1] = __uint_as_float(w.x & 0xFFFF0000u);
+      vv[u][2] = __uint_as_float(w.y << 16), vv[u][3] = __uint_as_float(w.y & 0xFFFF0000u);
+    }
+  }
+  // (cos, sin) of the keys' RoPE pairs j = lane and lane + 32, at position
+  // T + t, below rope_max_pos for t < n (checked by the host)
+  float2 kcs[TPW][2];
+#pragma unroll
+  for (int u = 0; u < TPW; ++u) {
+    const int t = warp + 4 * u;
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      kcs[u][c] = rope && t < n ? rope_cs(rope_hi, rope_lo, T + t0 + t, lane + 32 * c) : make_float2(1.f, 0.f);
+  }
   float* qraw = &red[0][0][0];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -818,24 +850,14 @@ __global__ void __launch_bounds__(kD) decode_window_kernel(
     }
   }
   __syncthreads();
-  const size_t row0 = static_cast<size_t>(bh) * win_stride + t0;
   {
-    float x[TPW][4];
-#pragma unroll
-    for (int u = 0; u < TPW; ++u) {
-      const int t = warp + 4 * u;
-      const TW* kr = k_win + (row0 + (t < n ? t : 0)) * kD;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) x[u][c] = to_f32(kr[lane + 32 * c]);
-    }
 #pragma unroll
     for (int u = 0; u < TPW; ++u) {
       const int t = warp + 4 * u;
       if (rope) {
-        const int64_t pos = T + t0 + t;   // below rope_max_pos for t < n (checked by the host)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const float2 cs = t < n ? rope_cs(rope_hi, rope_lo, pos, lane + 32 * c) : make_float2(1.f, 0.f);
+          const float2 cs = kcs[u][c];
           const float x1 = x[u][c], x2 = x[u][c + 2];
           x[u][c] = x1 * cs.x - x2 * cs.y;
           x[u][c + 2] = x2 * cs.x + x1 * cs.y;
@@ -870,20 +892,6 @@ __global__ void __launch_bounds__(kD) decode_window_kernel(
   }
   __syncthreads();
   {
-    float vv[TPW][4];
-#pragma unroll
-    for (int u = 0; u < TPW; ++u) {
-      const int t = warp + 4 * u;
-      const TW* vr = v_win + (row0 + (t < n ? t : 0)) * kD + 4 * lane;
-      if constexpr (sizeof(TW) == 4) {
-        const float4 w = *reinterpret_cast<const float4*>(vr);
-        vv[u][0] = w.x, vv[u][1] = w.y, vv[u][2] = w.z, vv[u][3] = w.w;
-      } else {
-        const uint2 w = *reinterpret_cast<const uint2*>(vr);
-        vv[u][0] = __uint_as_float(w.x << 16), vv[u][1] = __uint_as_float(w.x & 0xFFFF0000u);
-        vv[u][2] = __uint_as_float(w.y << 16), vv[u][3] = __uint_as_float(w.y & 0xFFFF0000u);
-      }
-    }
     float acc[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
