@@ -67,3 +67,25 @@ def test_bad_arguments_are_rejected_on_host():
     assert tq._lib.tq_decode_workspace_size(None, None, 1, 1, 1, 10) == 0
     assert tq._lib.tq_decode_window_workspace_size(None, None, 1, 1, 1, 10, 4) == 0
     assert tq._lib.tq_quantize_kv(None, None, 0, 1, 64, None, 1, 0, 0, None, None, None, 1, None) == tq.TQ_EINVAL
+    # window decode: null handles rejected on the host, before any device call
+    assert tq._lib.tq_decode_attention_window(None, None, None, 0, None, None, None, None, None, None, None, 0,
+                                              None, None, 0, 0, 0, 1, 4, 1, 0, 0.125, None, None, 0,
+                                              None) == tq.TQ_EINVAL
+
+
+def test_window_binding_checks_shapes_before_any_call():
+    """The binding rejects window arrays of different shape or dtype, and
+    non-contiguous ones, before it reaches the library (no GPU needed)."""
+    import torch
+    from vector_quantization_b200 import tq
+    rec = (torch.zeros((1, 1, 4, 32), dtype=torch.uint8), torch.zeros((1, 1, 4, 16), dtype=torch.uint8),
+           torch.zeros((1, 1, 4, 2)))
+    q = torch.zeros((1, 4, 128))
+    qpos = torch.zeros(1, dtype=torch.int64)
+    kw = torch.zeros((1, 1, 8, 128))
+    with pytest.raises(ValueError, match="share shape and dtype"):
+        tq.decode_attention_window(None, None, q, qpos, rec, rec, 4, kw, torch.zeros((1, 1, 9, 128)), 2)
+    with pytest.raises(ValueError, match="share shape and dtype"):
+        tq.decode_attention_window(None, None, q, qpos, rec, rec, 4, kw, kw.to(torch.bfloat16), 2)
+    with pytest.raises(ValueError, match="contiguous"):
+        tq.decode_attention_window(None, None, q, qpos, rec, rec, 4, kw.transpose(2, 3), kw.transpose(2, 3), 2)
