@@ -139,3 +139,38 @@ def score_from_codes(rot: Rotation, q, codes, signs, norm, rnorm) -> np.ndarray:
     qjl = (sq @ z.T) * (QJL_CONST / rot.m) * np.asarray(rnorm, dtype=np.float64)[None, :]
     out = mse + qjl
     return out[0] if single else out
+
+
+# ---------------------------------------------------------------------------
+# Residual-correction variants, for comparison at equal bits (test
+# infrastructure; the CUDA path implements the QJL form above only).
+#
+# [TurboESM] §2.D keeps only the sign of the residual (1 bit) and rebuilds
+# x_tilde = x_hat + sign * e_bar, e_bar a mean residual magnitude the page
+# calibrates beforehand.  Calibration data is out of scope here, so e_bar is
+# read as the mean magnitude of this vector's own residual,
+# e_bar = ||r||_1 / d, stored in place of ||r|| (same bytes as the QJL form
+# with m = d: d code bits per plane, d sign bits, two floats).  Signs are of
+# the rotated residual, coordinate by coordinate (no projection).
+# The MSE-only form drops the residual term: x_tilde = Pi^T ||x|| c[idx].
+# ---------------------------------------------------------------------------
+def encode_sign_residual(rot: Rotation, x, pos=None) -> dict:
+    """Codes as :func:`encode`; sign bits z_i = [r_i >= 0] of the rotated
+    residual r = ||x|| (y - c[idx]) and e_bar = ||r||_1 / d per vector."""
+    e = encode(rot, x, pos)
+    r = e["norm"][:, None] * (e["y"] - rot.levels[e["codes"]])
+    return dict(codes=e["codes"], signs=r >= 0.0, norm=e["norm"], ebar=np.mean(np.abs(r), axis=1), r=r)
+
+
+def dequantize_sign_residual(rot: Rotation, codes, signs, norm, ebar, rotated: bool = False) -> np.ndarray:
+    """x_tilde = Pi^T (||x|| c[idx] + e_bar (2z - 1)) ([TurboESM] §2.D)."""
+    z = np.where(np.asarray(signs, dtype=bool), 1.0, -1.0)
+    xr = np.asarray(norm, dtype=np.float64)[:, None] * rot.levels[np.asarray(codes)] \
+        + np.asarray(ebar, dtype=np.float64)[:, None] * z
+    return xr if rotated else xr @ rot.pi
+
+
+def dequantize_mse_only(rot: Rotation, codes, norm, rotated: bool = False) -> np.ndarray:
+    """x_tilde = Pi^T ||x|| c[idx]: the codes alone, no residual term."""
+    xr = np.asarray(norm, dtype=np.float64)[:, None] * rot.levels[np.asarray(codes)]
+    return xr if rotated else xr @ rot.pi
