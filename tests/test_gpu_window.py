@@ -1,9 +1,11 @@
 """GPU parity of tq_decode_attention_window (packed cache plus a full-precision
 window of recent tokens, [NSNQuant] §4 "Résidus") against the oracle.
 
-The packed caches are written by the oracle, so both sides score the same
-bytes; window keys and values are the same float32 (or bf16-rounded) values on
-both sides.  Tolerance: |gpu - ref| <= 1e-3 + 2e-3 |ref|."""
+The packed caches of the small cases are written by the oracle, so both sides
+score the same bytes; the full-size case encodes on the GPU, checks the
+sampled slices against the oracle's encoding and replaces them by it.  Window
+keys and values are the same float32 (or bf16-rounded) values on both sides.
+Tolerance: |gpu - ref| <= 1e-3 + 2e-3 |ref|."""
 import numpy as np
 import pytest
 import torch
