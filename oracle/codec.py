@@ -174,3 +174,30 @@ def dequantize_mse_only(rot: Rotation, codes, norm, rotated: bool = False) -> np
     """x_tilde = Pi^T ||x|| c[idx]: the codes alone, no residual term."""
     xr = np.asarray(norm, dtype=np.float64)[:, None] * rot.levels[np.asarray(codes)]
     return xr if rotated else xr @ rot.pi
+
+
+# ---------------------------------------------------------------------------
+# Normalize-Shift-Normalize pre-transform ([NSNQuant] §1), for comparison
+# (test infrastructure; the CUDA path has no NSN step).  For a block of l
+# tokens x [l, d]:
+#   x1 = x sqrt(d) / ||x||           per token, s1 = ||x|| / sqrt(d)
+#   o  = mean over the block's tokens of x1, per channel
+#   x3 = (x1 - o) sqrt(d) / ||x1 - o||  per token, s2 = ||x1 - o|| / sqrt(d)
+# so that x = s1 (s2 x3 + o).  x3 then goes through the codec as any vector.
+# ---------------------------------------------------------------------------
+def nsn_forward(x):
+    """Returns (x3 [l, d], s1 [l], o [d], s2 [l]) of [NSNQuant] §1."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[1]
+    s1 = np.sqrt(np.sum(x * x, axis=1)) / math.sqrt(d)
+    x1 = x / np.where(s1 > 0, s1, 1.0)[:, None]
+    o = np.mean(x1, axis=0)
+    x2 = x1 - o
+    s2 = np.sqrt(np.sum(x2 * x2, axis=1)) / math.sqrt(d)
+    x3 = x2 / np.where(s2 > 0, s2, 1.0)[:, None]
+    return x3, s1, o, s2
+
+
+def nsn_inverse(x3, s1, o, s2):
+    """x = s1 (s2 x3 + o)."""
+    return np.asarray(s1)[:, None] * (np.asarray(s2)[:, None] * np.asarray(x3) + np.asarray(o)[None, :])

@@ -1,4 +1,5 @@
-"""Residual-correction variants at equal bits (CPU, oracle only).
+"""Residual-correction variants at equal bits, and the NSN pre-transform
+([NSNQuant] §1) ahead of the codec (CPU, oracle only).
 
 Three reconstructions of a d-dimensional vector at 3 bits per coordinate plus
 two floats:
@@ -118,3 +119,60 @@ def test_compare_at_equal_bits():
         # its error is (pi/2 - 1/d) times that of the codes alone
         ratio = rows["qjl 2+1"][0] / rows["mse 2 (2 bits only)"][0]
         assert abs(ratio - (np.pi / 2 - 1 / d)) < 0.05, ratio
+
+
+# ---------------------------------------------------------------------------
+# Normalize-Shift-Normalize ([NSNQuant] §1) ahead of the codec
+# ---------------------------------------------------------------------------
+def _offset_law(n, d, seed, n_offset=8, offset=4.0, n_outliers=4):
+    """heavy_tailed rows plus a fixed per-channel offset on n_offset seeded
+    channels (channels whose mean is far from zero in every token)."""
+    x = synth.heavy_tailed((1, 1, n, d), seed, n_outliers=n_outliers).reshape(n, d).astype(np.float64)
+    rng = np.random.default_rng(seed + 1)
+    ch = rng.choice(d, n_offset, replace=False)
+    x[:, ch] += offset * np.where(rng.random(n_offset) < 0.5, -1.0, 1.0)
+    return x
+
+
+def test_nsn_round_trip_and_invariants():
+    d = 128
+    x = _offset_law(300, d, 91)
+    x3, s1, o, s2 = codec.nsn_forward(x)
+    np.testing.assert_allclose(codec.nsn_inverse(x3, s1, o, s2), x, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(np.sum(x3 * x3, axis=1), d, rtol=1e-12)              # norm sqrt(d)
+    np.testing.assert_allclose(np.mean(x3 * s2[:, None], axis=0), 0.0, atol=1e-12)   # centred channels
+    np.testing.assert_allclose(np.sum((x / s1[:, None]) ** 2, axis=1), d, rtol=1e-12)
+
+
+def test_nsn_comparison():
+    """The codec (2+1 bits) on x directly and on NSN's x3, for rows with 8
+    channels offset by +-4 in every token, over heavy_tailed rows (with the
+    x20 outlier channels) and over N(0, 1) rows: unit MSE and attention
+    cosine against exact attention.  Printed; the NSN route must not lose on
+    the MSE of these laws, where the shift removes the offsets."""
+    d, n, nq = 128, 2048, 64
+    rot = _rot(d, 2, 106)
+
+    def direct(x):
+        e = codec.encode(rot, x)
+        return codec.dequantize(rot, e["codes"], e["signs"], e["norm"], e["rnorm"])
+
+    def nsn(x):
+        x3, s1, o, s2 = codec.nsn_forward(x)
+        return codec.nsn_inverse(direct(x3), s1, o, s2)
+
+    for n_outliers in (4, 0):
+        k = _offset_law(n, d, 101, n_outliers=n_outliers)
+        v = _offset_law(n, d, 103, n_outliers=n_outliers)
+        q = synth.heavy_tailed((1, 1, nq, d), 105, n_outliers=n_outliers).reshape(nq, d).astype(np.float64)
+        exact = _attention(q, k, v, 1 / np.sqrt(d))
+        res = {}
+        print(f"\noffsets +-4 on 8 channels, {'with 4 outlier channels x20' if n_outliers else 'N(0, 1) otherwise'}")
+        for name, f in (("codec on x", direct), ("codec on NSN(x)", nsn)):
+            kt, vt = f(k), f(v)
+            umse = float(np.mean(np.sum((k - kt) ** 2, axis=1) / np.sum(k * k, axis=1)))
+            out = _attention(q, kt, vt, 1 / np.sqrt(d))
+            cos = np.sum(out * exact, axis=1) / (np.linalg.norm(out, axis=1) * np.linalg.norm(exact, axis=1))
+            res[name] = (umse, float(np.mean(cos)))
+            print(f"{name:18s} unit MSE {umse:.5f}  attention cosine {np.mean(cos):.6f}")
+        assert res["codec on NSN(x)"][0] < res["codec on x"][0]
