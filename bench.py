@@ -50,7 +50,7 @@ UNIT = "tokens/s"
 SPLIT_TRAFFIC_PER_TOKEN = (235_454_464 + 6_769_152) / (16 * 8 * 16384)
 
 EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1",
-          "decode_llama8b_layer_window")
+          "decode_llama8b_layer_window", "tiny_d128_t1024", "encode_esm2_33_layers")
 
 
 def parse():
@@ -282,6 +282,32 @@ def oracle_extra_baselines(select):
         out[key] = base(r, "queries/s", f"{nq} queries over {N} of the {c['n_db']} database vectors, d {ds}, "
                                         f"{bits}+1 bits, top-{c['top_k']}, scaled to the full database; "
                                         f"{calls} calls, {per:.2f} s each")
+    if "tiny_d128_t1024" in select:
+        c = synth.CONFIGS["tiny_d128_t1024"]
+        T, seed = c["tokens"], c["seed"]
+        rk = ro.build_rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 1]), rope_base=c["rope_base"])
+        rv = ro.build_rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 2]))
+        k = synth.heavy_tailed((1, 1, T, d), [seed, 9, 3]).reshape(T, d)
+        v = synth.heavy_tailed((1, 1, T, d), [seed, 9, 4]).reshape(T, d)
+        q = synth.heavy_tailed((1, 1, d), [seed, 9, 5])
+        t0 = time.perf_counter()
+        kc, vc = packed(rk, k, np.arange(T)), packed(rv, v, None)
+        t_enc = time.perf_counter() - t0
+        _, calls, per = _oracle_rate(lambda: at.decode_attention(rk, rv, q, [T - 1], kc, vc, 1 / np.sqrt(d)), 1)
+        out["tiny_d128_t1024"] = {"value": per * 1e6, "unit": "decode us", "encode_us": t_enc * 1e6, "cores": cores,
+                                  "kind": "oracle",
+                                  "sample": f"the whole workload: encode of {T} keys + {T} values once, decode "
+                                            f"{calls} times ({per * 1e3:.1f} ms each)"}
+    if "encode_esm2_33_layers" in select:
+        c = synth.CONFIGS["esm2_650m_encoder"]
+        de, ne = c["head_dim"], 8192
+        rk = ro.build_rotation(de, 2, synth.rotation_randomness(de, [c["seed"], 9, 1]), rope_base=c["rope_base"])
+        rv = ro.build_rotation(de, 2, synth.rotation_randomness(de, [c["seed"], 9, 2]))
+        x = synth.lognormal_channels((1, 2, ne, de), [c["seed"], 9, 6])
+        pos = np.arange(ne) % c["tokens"]
+        r, calls, per = _oracle_rate(lambda: (codec.encode(rk, x[0, 0], pos), codec.encode(rv, x[0, 1])), 2 * ne)
+        out["encode_esm2_33_layers"] = base(r, "vectors/s", f"{ne} keys (RoPE) + {ne} values, d {de}, 2+1 bits; "
+                                                            f"{calls} calls, {per:.2f} s each")
     if select & {"decode_llama8b_layer_3p1", "decode_llama8b_layer_window"}:
         c = synth.CONFIGS["llama31_8b_gqa_decode"]
         T, G = 8192, c["q_heads"] // c["kv_heads"]
@@ -338,20 +364,29 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, 
     c = synth.CONFIGS["llama31_70b_long_slice"]
     Hkv, Hq, d, T, seed = c["kv_heads"], c["q_heads"], c["head_dim"], c["tokens"], c["seed"]
     T = slice_tokens or T
-    if select & {"encode_70b_slice", "decode_70b_slice"}:
-        out.update(_extras_70b(dev, peak_gbs, select, Hkv, Hq, d, T, seed, c))
-    if "encoder_esm2_layer" in select:
-        out.update(_extra_encoder(dev, g))
-    if "search_1m_d1536" in select:
-        out.update(_extra_search(dev, g, search_rows))
-    if "decode_llama8b_layer_3p1" in select:
-        out.update(_extra_decode_3p1(dev, peak_gbs))
-    if "decode_llama8b_layer_window" in select:
-        out.update(_extra_decode_window(dev, peak_gbs))
+    runs = [({"encode_70b_slice", "decode_70b_slice"},
+             lambda: _extras_70b(dev, peak_gbs, select, Hkv, Hq, d, T, seed, c)),
+            ({"encoder_esm2_layer"}, lambda: _extra_encoder(dev, g)),
+            ({"search_1m_d1536"}, lambda: _extra_search(dev, g, search_rows)),
+            ({"decode_llama8b_layer_3p1"}, lambda: _extra_decode_3p1(dev, peak_gbs)),
+            ({"decode_llama8b_layer_window"}, lambda: _extra_decode_window(dev, peak_gbs)),
+            ({"tiny_d128_t1024"}, lambda: _extra_tiny(dev)),
+            ({"encode_esm2_33_layers"}, lambda: _extra_encode_esm2(dev, peak_gbs, g))]
+    for names, run in runs:
+        if not names & select:
+            continue
+        try:   # one line failing leaves the others (and the headline) in place
+            out.update(run())
+        except Exception as exc:
+            out[sorted(names & select)[0]] = {"error": f"{type(exc).__name__}: {exc}"}
+        torch.cuda.empty_cache()
     if cpu and not slice_tokens:
-        for key, b in oracle_extra_baselines(select).items():
-            if key in out:
-                out[key]["cpu_baseline"] = b
+        try:
+            for key, b in oracle_extra_baselines(select).items():
+                if key in out and "error" not in out[key]:
+                    out[key]["cpu_baseline"] = b
+        except Exception as exc:
+            out["cpu_baseline_error"] = f"{type(exc).__name__}: {exc}"
     return out
 
 
@@ -514,6 +549,66 @@ def _extra_decode_window(dev, peak_gbs, R=128):
                                             "algorithmic_bytes": byts,
                                             "note": f"{T - R} packed tokens (112 B per pair) + {R}-token bf16 window "
                                                     "(512 B per pair); whole call, 5 launches"}}
+
+def _extra_tiny(dev):
+    """The tiny workload (1 head, d 128, 1024 fp32 tokens, heavy-tailed with
+    4 outlier channels x20, RoPE on K, 2+1 bits, one fp32 query): encode of
+    its K and V and one decode, as absolute latencies (the data fit in L2)."""
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["tiny_d128_t1024"]
+    T, d, seed = c["tokens"], c["head_dim"], c["seed"]
+    rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 2]))
+    k = torch.from_numpy(synth.heavy_tailed((1, 1, T, d), [seed, 9, 3])).to(dev)
+    v = torch.from_numpy(synth.heavy_tailed((1, 1, T, d), [seed, 9, 4])).to(dev)
+    q = torch.from_numpy(synth.heavy_tailed((1, 1, d), [seed, 9, 5])).to(dev)
+    kc, vc = tq.empty_records(rk, (1, 1, T), dev), tq.empty_records(rv, (1, 1, T), dev)
+
+    def enc():
+        tq.quantize_kv(rk, k, apply_rope=True, pos_period=T, out=kc)
+        tq.quantize_kv(rv, v, out=vc)
+    us_enc = _time_ms(enc, reps=50, warm=5) * 1e3
+    qpos = torch.full((1,), T - 1, dtype=torch.int64, device=dev)
+    ws = tq.alloc_workspace(tq.decode_workspace_size(rk, rv, 1, 1, 1, T), dev)
+    o = torch.empty((1, 1, d), dtype=torch.float32, device=dev)
+    us_dec = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws),
+                      reps=50, warm=5) * 1e3
+    return {"tiny_d128_t1024": {"encode_us": round(us_enc, 2), "decode_us": round(us_dec, 2),
+                                "note": "1024 keys (RoPE) + 1024 values encoded (two calls), then one decode of "
+                                        "one fp32 query; latency, inputs resident in L2"}}
+
+
+def _extra_encode_esm2(dev, peak_gbs, g):
+    """Encode of the whole ESM-2-650M-shaped cache: 33 layers x [8, 20, 1024,
+    64] bf16 keys (RoPE at positions 0..1023) and values, 2+1 bits, one call
+    each: 2 x 5.4M vectors.  N(0, 1) bf16 rows stand in for the log-normal
+    channel law (the encode does the same work whatever the values)."""
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["esm2_650m_encoder"]
+    L, B, H, T, d, seed = c["layers"], c["batch"], c["heads"], c["tokens"], c["head_dim"], c["seed"]
+    n = L * B * H * T
+    rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 2]))
+    g.manual_seed(seed + 9)
+    k = torch.randn((n, d), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((n, d), generator=g, device=dev).to(torch.bfloat16)
+    kc, vc = tq.empty_records(rk, (n,), dev), tq.empty_records(rv, (n,), dev)
+
+    def enc():
+        tq.quantize_kv(rk, k, apply_rope=True, pos_period=T, out=kc)
+        tq.quantize_kv(rv, v, out=vc)
+    ms = _time_ms(enc, reps=5, warm=2)
+    nvec = 2 * n
+    byts = nvec * (2 * d + rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)))
+    return {"encode_esm2_33_layers": {"vectors": nvec, "ms": round(ms, 4), "vectors_per_s": nvec / ms * 1e3,
+                                      "GB_s": round(byts / ms / 1e6, 1),
+                                      "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4), "algorithmic_bytes": byts,
+                                      "note": "bf16 in (128 B) + packed record out (32 B) per vector"}}
+
 
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
@@ -691,7 +786,10 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_extras:
         del kcs, vcs
         torch.cuda.empty_cache()
-        line["extras"] = run_extras(dev, peak, cpu=not args.no_cpu_baseline)
+        try:
+            line["extras"] = run_extras(dev, peak, cpu=not args.no_cpu_baseline)
+        except Exception as exc:   # the headline line is printed whatever a secondary line does
+            line["extras"] = {"error": f"{type(exc).__name__}: {exc}"}
     print(json.dumps(line), flush=True)
 
 
