@@ -66,3 +66,13 @@ def test_reference_arm_other_ranks_do_no_work(capsys):
     import bench
     bench.run_reference(None, 1, 2)                # args unused on rank != 0: returns at once
     assert capsys.readouterr().out == ""
+
+
+def test_oracle_baseline_of_a_secondary_line():
+    """The oracle leg beside a secondary bench line runs on the host alone and
+    returns a positive rate with its unit, core count and sample."""
+    import bench
+    out = bench.oracle_extra_baselines({"tiny_d128_t1024"})
+    b = out["tiny_d128_t1024"]
+    assert b["kind"] == "oracle" and b["value"] > 0 and b["cores"] >= 1
+    assert b["unit"] == "decode us" and "1024 keys" in b["sample"]
