@@ -263,8 +263,8 @@ size_t tq_search_workspace_size(const tq_rotation* h, int nq, int64_t N, int k);
  *               device caches; sequence (b, kv-head j) occupies records
  *               (b*Hkv + j)*cache_stride .. + T-1; all 16-byte aligned
  *   cache_stride  records between consecutive sequences (>= T, even)
- *   B, Hq, Hkv  batch, query heads, KV heads; Hq % Hkv == 0 and
- *               Hq/Hkv in {1, 2, 4, 8}
+ *   B, Hq, Hkv  batch, query heads, KV heads; Hq % Hkv == 0,
+ *               Hq/Hkv in {1, 2, 4, 8} and B*Hkv <= 65535
  *   T           cached tokens per sequence (0 gives an all-zero output)
  *   scale       softmax scale (typically 1/sqrt(d))
  *   out         device [B, Hq, d] float32
@@ -384,7 +384,9 @@ size_t tq_encoder_workspace_size(const tq_rotation* hk, int B, int Hq, int S);
  *     must start at zero).  Calls whose kernels may overlap on the GPU -
  *     concurrent streams, or host threads racing on one device - race on
  *     the scratch: serialise them.
- * Returns the statuses of tq_decode_attention.
+ * Returns the statuses of tq_decode_attention, in this order: the handle and
+ * size checks (TQ_EINVAL, TQ_EUNSUPPORTED), then TQ_EWORKSPACE for sizes
+ * beyond the scratch, then the pointer checks and launches.
  */
 int tq_decode_attention_noalloc(const tq_rotation* hk, const tq_rotation* hv,
                                 const void* q, int q_dtype, const int64_t* q_pos,

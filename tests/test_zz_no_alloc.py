@@ -69,11 +69,13 @@ def test_noalloc_rejects_requests_beyond_its_scratch(cuda_device):
     tq, fn = _bind()
     dev = cuda_device
     rk, rv, kc, vc, q, qpos = _case(tq, 4, 64, 1, 1, 91, dev)
-    out = torch.zeros_like(q, dtype=torch.float32)
-    # 4096 sequences of 2^20 tokens need far more than the fixed scratch
+    # 4096 sequences of 2^20 tokens need far more than the fixed scratch.
+    # The cache and output pointers are NULL: the size check must answer
+    # first, and were it ever to move behind the pointer checks the call would
+    # still return an error (TQ_EINVAL) instead of launching over buffers far
+    # smaller than the sizes claimed.
     B, Hkv, T = 512, 8, 1 << 20
     assert tq.decode_workspace_size(rk, rv, B, 4 * Hkv, Hkv, T) > (16 << 20)
-    st = fn(rk.handle, rv.handle, q.data_ptr(), 0, qpos.data_ptr(), kc[0].data_ptr(), kc[1].data_ptr(),
-            kc[2].data_ptr(), vc[0].data_ptr(), vc[1].data_ptr(), vc[2].data_ptr(), T, B, 4 * Hkv, Hkv, T,
-            0.088, out.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    st = fn(rk.handle, rv.handle, q.data_ptr(), 0, qpos.data_ptr(), None, None, None, None, None, None,
+            T, B, 4 * Hkv, Hkv, T, 0.088, None, torch.cuda.current_stream().cuda_stream)
     assert st == tq.TQ_EWORKSPACE

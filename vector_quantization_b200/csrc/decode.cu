@@ -958,6 +958,27 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 size_t kconst_bytes(int BH) { return static_cast<size_t>(BH) * 2 * 8 * sizeof(float2); }
 
+// Sequences (batch x KV heads) of one call: the split kernel's grid has one
+// row of blocks per sequence, and CUDA caps a grid's y extent at 65535.
+constexpr int64_t kMaxSequences = 65535;
+
+// Checks of the handles and sizes alone (no pointers), in the order the
+// entry points report them: TQ_EINVAL for malformed sizes, TQ_EUNSUPPORTED
+// for well-formed requests this library does not serve.
+int check_decode_sizes(const tq_rotation* hk, const tq_rotation* hv, int B, int Hq, int Hkv, int64_t T) {
+  if (!hk || !hv) return TQ_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0) return TQ_EINVAL;
+  if (hk->d != hv->d || hk->m != hv->m) return TQ_EINVAL;
+  if (static_cast<int64_t>(B) * Hkv > kMaxSequences) return TQ_EUNSUPPORTED;
+  if (hk->d != kD || hk->m != kD) return TQ_EUNSUPPORTED;
+  if (hk->kind != TQ_ROT_HADAMARD || hv->kind != TQ_ROT_HADAMARD) return TQ_EUNSUPPORTED;
+  if (hk->bits != hv->bits) return TQ_EUNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_EUNSUPPORTED;
+  return TQ_OK;
+}
+
+// Workspace bytes of one call; B * Hkv must already be within kMaxSequences.
 size_t workspace_for(int B, int Hq, int Hkv, int64_t T, int R = 0) {
   const int G = Hq / Hkv;
   const int BH = B * Hkv;
@@ -1097,15 +1118,14 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
                 const void* v_win, int win_dtype, int64_t win_stride, int R, int B, int Hq, int Hkv, int64_t T,
                 float scale, float* out, void* workspace, size_t workspace_bytes, cudaStream_t s,
                 cudaEvent_t prof_begin, cudaEvent_t prof_end) {
-  if (!hk || !hv || !q || !out) return TQ_EINVAL;
+  {
+    const int st = check_decode_sizes(hk, hv, B, Hq, Hkv, T);
+    if (st != TQ_OK) return st;
+  }
+  if (!q || !out) return TQ_EINVAL;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_EINVAL;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || !std::isfinite(scale)) return TQ_EINVAL;
-  if (hk->d != hv->d || hk->m != hv->m) return TQ_EINVAL;
-  if (hk->d != kD || hk->m != kD) return TQ_EUNSUPPORTED;
-  if (hk->kind != TQ_ROT_HADAMARD || hv->kind != TQ_ROT_HADAMARD) return TQ_EUNSUPPORTED;
-  if (hk->bits != hv->bits) return TQ_EUNSUPPORTED;
+  if (!std::isfinite(scale)) return TQ_EINVAL;
   const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_EUNSUPPORTED;
   if (T > 0) {
     if (!k_codes || !k_signs || !k_norms || !v_codes || !v_signs || !v_norms) return TQ_EINVAL;
     if (cache_stride < T || (cache_stride & 1)) return TQ_EINVAL;
@@ -1186,13 +1206,13 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
 
 extern "C" size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv, int B, int Hq, int Hkv,
                                            int64_t T) {
-  if (!hk || !hv || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0) return 0;
+  if (check_decode_sizes(hk, hv, B, Hq, Hkv, T) != TQ_OK) return 0;
   return workspace_for(B, Hq, Hkv, T);
 }
 
 extern "C" size_t tq_decode_window_workspace_size(const tq_rotation* hk, const tq_rotation* hv, int B, int Hq,
                                                   int Hkv, int64_t T, int R) {
-  if (!hk || !hv || B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0 || R < 0 || R > kWindowMax) return 0;
+  if (check_decode_sizes(hk, hv, B, Hq, Hkv, T) != TQ_OK || R < 0 || R > kWindowMax) return 0;
   return workspace_for(B, Hq, Hkv, T, R);
 }
 
@@ -1246,8 +1266,12 @@ extern "C" int tq_decode_attention_noalloc(const tq_rotation* hk, const tq_rotat
                                            const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
                                            const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv,
                                            int64_t T, float scale, float* out, void* stream) {
-  if (!hk || !hv) return TQ_EINVAL;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || T < 0) return TQ_EINVAL;
+  // the handle and size checks of tq_decode_attention come first, so a call
+  // this library cannot serve at all reports that rather than the cap below
+  {
+    const int st = check_decode_sizes(hk, hv, B, Hq, Hkv, T);
+    if (st != TQ_OK) return st;
+  }
   if (workspace_for(B, Hq, Hkv, T) > kNoAllocScratchBytes) return TQ_EWORKSPACE;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return TQ_ECUDA;
