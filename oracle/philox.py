@@ -25,8 +25,9 @@ sides):
 * counter = (i mod 2^32, i >> 32, stream, 0), with stream 0 for D, 1 for S and
   2 for the dense Gaussian;
 * D_i = -1 when the top bit of word 0 of block i is set, else +1;
-* Gaussians come in pairs: block p gives two 53-bit uniforms
-  u = ((w0 >> 5) 2^26 + (w1 >> 6) + 1/2) / 2^53 from words (0, 1) and (2, 3),
+* Gaussians come in pairs: block p gives two 52-bit uniforms
+  u = ((w0 >> 6) 2^26 + (w1 >> 6) + 1/2) / 2^52 from words (0, 1) and (2, 3)
+  (every step exact in float64, so u lies strictly inside (0, 1)),
   then Box-Muller: r = sqrt(-2 ln u1), z_{2p} = r cos(2 pi u2),
   z_{2p+1} = r sin(2 pi u2); the row-major element k of S (or of the dense
   Gaussian) is z_k.
@@ -91,19 +92,20 @@ def _blocks(seed: int, stream: int, n: int):
     return philox4x32(idx & np.uint64(MASK32), idx >> np.uint64(32), np.uint64(stream), np.uint64(0), k0, k1)
 
 
-def uniform53(wa, wb) -> np.ndarray:
-    """(0, 1) uniforms from two 32-bit words: 53 bits, centred on the grid."""
-    a = (np.asarray(wa, dtype=np.uint64) >> np.uint64(5)).astype(np.float64)
+def uniform52(wa, wb) -> np.ndarray:
+    """(0, 1) uniforms from two 32-bit words: 52 bits, centred on the grid.
+    The integer part is below 2^52, so adding 1/2 and scaling are exact."""
+    a = (np.asarray(wa, dtype=np.uint64) >> np.uint64(6)).astype(np.float64)
     b = (np.asarray(wb, dtype=np.uint64) >> np.uint64(6)).astype(np.float64)
-    return (a * 67108864.0 + b + 0.5) / 9007199254740992.0
+    return (a * 67108864.0 + b + 0.5) / 4503599627370496.0
 
 
 def gaussians(seed: int, stream: int, count: int) -> np.ndarray:
     """The first `count` N(0, 1) draws of a stream (Box-Muller pairs), float64."""
     n_pairs = (count + 1) // 2
     w0, w1, w2, w3 = _blocks(seed, stream, n_pairs)
-    u1 = uniform53(w0, w1)
-    u2 = uniform53(w2, w3)
+    u1 = uniform52(w0, w1)
+    u2 = uniform52(w2, w3)
     r = np.sqrt(-2.0 * np.log(u1))
     z = np.empty(2 * n_pairs, dtype=np.float64)
     z[0::2] = r * np.cos(2.0 * np.pi * u2)
@@ -119,10 +121,12 @@ def sign_diagonal(seed: int, d: int) -> np.ndarray:
 
 def rotation_draws(d: int, seed: int, dense: bool = False, m: int | None = None) -> dict:
     """All draws of a seeded handle, in the layout `build_rotation` takes:
-    signs int8 [d], gauss_s float64 [m, d], gauss_pi float64 [d, d] or None."""
+    signs int8 [d], gauss_s float32 [m, d] (the float64 draws rounded to
+    float32, the type in which a handle receives its QJL Gaussians),
+    gauss_pi float64 [d, d] or None."""
     m = d if m is None else m
     return {
         "signs": sign_diagonal(seed, d),
-        "gauss_s": gaussians(seed, STREAM_S, m * d).reshape(m, d),
+        "gauss_s": gaussians(seed, STREAM_S, m * d).reshape(m, d).astype(np.float32),
         "gauss_pi": gaussians(seed, STREAM_DENSE, d * d).reshape(d, d) if dense else None,
     }

@@ -3,7 +3,7 @@
 The generator is pinned to the published known-answer vectors of
 Philox4x32-10 (tests/golden/philox4x32_10_kat.txt), which a wrong multiplier,
 a swapped output word, a missing key bump or an off-by-one round count all
-fail.  The derived draws are pinned by their laws: 53-bit uniforms strictly
+fail.  The derived draws are pinned by their laws: 52-bit uniforms strictly
 inside (0, 1) with the moments of U(0, 1), Box-Muller normals with the
 moments of N(0, 1) and a Kolmogorov-Smirnov test, and +-1 signs with balanced
 frequencies."""
@@ -44,13 +44,14 @@ def test_vectorised_equals_scalar_on_many_counters():
 
 def test_uniforms_inside_unit_interval_with_uniform_moments():
     w = philox._blocks(12345, 7, 200000)
-    u = philox.uniform53(w[0], w[1])
+    u = philox.uniform52(w[0], w[1])
     assert u.min() > 0.0 and u.max() < 1.0
     assert abs(u.mean() - 0.5) < 5 * np.sqrt(1 / 12 / u.size)
     assert abs(u.var() - 1 / 12) < 0.002
     # the extreme grid points map strictly inside (0, 1)
-    assert philox.uniform53(np.uint64(0), np.uint64(0)) == 0.5 / 2**53
-    assert philox.uniform53(np.uint64(2**32 - 1), np.uint64(2**32 - 1)) == 1.0 - 0.5 / 2**53
+    assert philox.uniform52(np.uint64(0), np.uint64(0)) == 0.5 / 2**52
+    assert philox.uniform52(np.uint64(2**32 - 1), np.uint64(2**32 - 1)) == 1.0 - 0.5 / 2**52
+    assert 1.0 - 0.5 / 2**52 < 1.0
 
 
 def test_gaussians_have_the_standard_normal_law():
@@ -74,6 +75,7 @@ def test_signs_are_balanced_and_streams_and_seeds_differ():
     assert not np.allclose(a["gauss_s"], b["gauss_s"])
     # S and the dense Gaussian come from different streams of one seed
     assert not np.allclose(a["gauss_s"].ravel()[:1000], a["gauss_pi"].ravel()[:1000])
+    assert a["gauss_s"].dtype == np.float32 and a["gauss_pi"].dtype == np.float64
 
 
 @pytest.mark.parametrize("seed", [0, 2**63 + 12345])
