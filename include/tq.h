@@ -107,14 +107,51 @@ int tq_lloyd_max(int d, int bits, double* levels, double* thresholds);
  *   rope_max_pos  positions 0..rope_max_pos-1 are supported (ignored when
  *              rope_base is 0); at most 2^31.
  *   out        receives the handle.
- * The random draws are inputs so that every generator stays outside the
- * library.  Builds the codebook (tq_lloyd_max), Pi, S and two-level RoPE
- * tables on the host in float64 and uploads them.  Synchronous.
+ * The random draws are inputs here (tq_build_rotation_seeded draws them
+ * from a seed instead).  Builds the codebook (tq_lloyd_max), Pi, S and
+ * two-level RoPE tables on the host in float64 and uploads them.
+ * Synchronous.
  * Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ENOMEM or TQ_ECUDA.
  */
 int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
                       const double* gauss_pi, const float* gauss_s, int m,
                       double rope_base, int64_t rope_max_pos, tq_rotation** out);
+
+/*
+ * tq_rotation_draws - host only; the random draws a seeded handle is built
+ * from.  [TurboQuant] Étape 1 and "QJL" (a random rotation, a Gaussian
+ * projection S), [NSNQuant] §2 (random sign diagonal D), [TurboESM] §2.B (a
+ * rotation per layer and head, reproducible from its seed).  The pages name
+ * no generator; this library uses Philox4x32-10 (Salmon et al., "Parallel
+ * random numbers: as easy as 1, 2, 3", SC 2011) with key = (seed mod 2^32,
+ * seed >> 32) and counter = (i mod 2^32, i >> 32, stream, 0):
+ *   stream 0  D_i = -1 if the top bit of word 0 of block i is set, else +1;
+ *   stream 1  S, m*d Gaussians row-major; stream 2  the d*d Gaussian matrix
+ *             of a dense rotation, row-major.  Gaussians come in pairs from
+ *             block p: uniforms u = ((w0>>6)*2^26 + (w1>>6) + 1/2) / 2^52
+ *             from words (0,1) and (2,3), then Box-Muller z_2p = r cos(2 pi
+ *             u2), z_2p+1 = r sin(2 pi u2), r = sqrt(-2 ln u1), in float64.
+ *   d, m        1..4096
+ *   kind        TQ_ROT_HADAMARD or TQ_ROT_DENSE (gauss_pi is filled only
+ *               for TQ_ROT_DENSE)
+ *   signs       host out [d] int8 of +-1, or NULL
+ *   gauss_pi    host out [d*d] float64, or NULL
+ *   gauss_s     host out [m*d] float32 (each float64 draw rounded to the
+ *               nearest float32), or NULL
+ * Returns TQ_OK or TQ_EINVAL.  Pure host computation; needs no GPU.
+ */
+int tq_rotation_draws(int d, int kind, uint64_t seed, int m, int8_t* signs,
+                      double* gauss_pi, float* gauss_s);
+
+/*
+ * tq_build_rotation_seeded - tq_build_rotation from a 64-bit seed: the
+ * handle built from the draws tq_rotation_draws(d, kind, seed, m, ...)
+ * returns, identical to passing those draws to tq_build_rotation.  The other
+ * arguments and the statuses are those of tq_build_rotation.
+ */
+int tq_build_rotation_seeded(int d, int code_bits, int kind, uint64_t seed,
+                             int m, double rope_base, int64_t rope_max_pos,
+                             tq_rotation** out);
 
 /* Release a handle and its device memory (NULL is accepted). */
 int tq_free_rotation(tq_rotation* h);

@@ -89,3 +89,31 @@ def test_window_binding_checks_shapes_before_any_call():
         tq.decode_attention_window(None, None, q, qpos, rec, rec, 4, kw, kw.to(torch.bfloat16), 2)
     with pytest.raises(ValueError, match="contiguous"):
         tq.decode_attention_window(None, None, q, qpos, rec, rec, 4, kw.transpose(2, 3), kw.transpose(2, 3), 2)
+
+
+@pytest.mark.parametrize("d,kind,seed", [(128, "hadamard", 0), (64, "hadamard", 2**40 + 7), (96, "dense", 1234567)])
+def test_library_seeded_draws_match_oracle_generator(d, kind, seed):
+    """The library's Philox4x32-10 draws (host code, no GPU) against the
+    oracle's own implementation of the same published generator: signs and
+    the float32 QJL Gaussians bit for bit, the float64 dense Gaussians to a
+    few ulps (the two sides call different libm builds for log/cos/sin)."""
+    from vector_quantization_b200 import tq
+    from oracle import philox
+    lib = tq.rotation_draws(d, seed, kind)
+    ora = philox.rotation_draws(d, seed, dense=(kind == "dense"))
+    np.testing.assert_array_equal(lib["signs"], ora["signs"])
+    # float64 draws that differ in the last ulp may round to different
+    # float32 values only when they sit on a float32 rounding midpoint
+    np.testing.assert_allclose(lib["gauss_s"], ora["gauss_s"], rtol=2**-23, atol=0)
+    assert np.mean(lib["gauss_s"] == ora["gauss_s"]) > 0.999
+    if kind == "dense":
+        np.testing.assert_allclose(lib["gauss_pi"], ora["gauss_pi"], rtol=1e-14, atol=1e-300)
+    else:
+        assert lib["gauss_pi"] is None
+
+
+def test_library_seeded_draws_reject_bad_sizes():
+    from vector_quantization_b200 import tq
+    assert tq._lib.tq_rotation_draws(0, 0, 1, 128, None, None, None) == tq.TQ_EINVAL
+    assert tq._lib.tq_rotation_draws(128, 7, 1, 128, None, None, None) == tq.TQ_EINVAL
+    assert tq._lib.tq_rotation_draws(128, 0, 1, 128, None, None, None) == tq.TQ_OK

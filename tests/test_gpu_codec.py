@@ -228,3 +228,26 @@ def test_quantize_kv_pair_equals_two_calls(cuda_device, n, dtype):
     torch.cuda.synchronize()
     for a, b in zip((*pk, *pv), (*sk, *sv)):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("d,bits,kind,seed", [(128, 2, "hadamard", 7), (64, 3, "hadamard", 2**33 + 5),
+                                              (128, 1, "dense", 99)])
+def test_seeded_build_matches_oracle_from_its_own_generator(cuda_device, d, bits, kind, seed):
+    """tq_build_rotation_seeded draws D, S (and the Gaussian of a dense Pi)
+    with the library's Philox4x32-10; the oracle draws them with its own
+    implementation of that generator and builds its handle from them.  The
+    exported tables agree, and encoding with the seeded handle gives the
+    oracle's records."""
+    from vector_quantization_b200 import tq
+    from oracle import philox
+    g = tq.Rotation(d, bits, seed, kind)
+    o = ro.build_rotation(d, bits, philox.rotation_draws(d, seed, dense=(kind == "dense")), kind)
+    ex = g.export()
+    np.testing.assert_allclose(ex["pi"], o.pi, rtol=0, atol=2e-7)
+    np.testing.assert_array_equal(ex["s"], o.s.astype(np.float32))
+    np.testing.assert_allclose(ex["levels"], o.levels, rtol=1e-10)
+    if kind == "hadamard":
+        x = synth.heavy_tailed((300, d), seed % 1000 + 3)
+        gpu = tq.quantize_kv(g, torch.from_numpy(x).to(cuda_device))
+        codes, signs, norms, enc = oracle_records(o, x)
+        compare_records(o, tuple(a.cpu().numpy() for a in gpu), enc)

@@ -8,6 +8,7 @@
 // bits.  [NSNQuant] Méthodologie §2: randomized Hadamard transform.
 // [TurboESM] §2.A: RoPE applied before the rotation.
 #include <cmath>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <limits>
@@ -239,6 +240,69 @@ void release(tq_rotation* h) {
   delete h;
 }
 
+// ---------------------------------------------------------------------------
+// Seeded draws of a handle: the counter-based generator Philox4x32-10
+// (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3",
+// SC 2011).  Ten rounds; a round multiplies counter words 0 and 2 by two
+// fixed 32-bit constants, keeps the low halves as the new words 3 and 1, and
+// XORs the high halves with the other two words and the key; the key steps
+// by two Weyl constants between rounds.  How a handle uses it:
+//   key = (seed mod 2^32, seed >> 32); counter = (i mod 2^32, i >> 32,
+//   stream, 0), stream 0 for the sign diagonal D, 1 for the QJL matrix S,
+//   2 for the Gaussian matrix behind a dense rotation.
+//   D_i = -1 when the top bit of word 0 of block i is set, else +1.
+//   Gaussians in pairs: block p gives two uniforms
+//   u = ((w0 >> 6) 2^26 + (w1 >> 6) + 1/2) / 2^52 (words 0-1, then 2-3),
+//   exact in double and strictly inside (0, 1); then Box-Muller,
+//   r = sqrt(-2 ln u1), z_2p = r cos(2 pi u2), z_2p+1 = r sin(2 pi u2).
+// ---------------------------------------------------------------------------
+struct Philox4 {
+  uint32_t w[4];
+};
+
+Philox4 philox4x32_10(uint64_t index, uint32_t stream, uint64_t seed) {
+  uint32_t c0 = static_cast<uint32_t>(index), c1 = static_cast<uint32_t>(index >> 32), c2 = stream, c3 = 0;
+  uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t prod_a = static_cast<uint64_t>(0xD2511F53u) * c0;
+    const uint64_t prod_b = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+    const uint32_t n0 = static_cast<uint32_t>(prod_b >> 32) ^ c1 ^ k0;
+    const uint32_t n1 = static_cast<uint32_t>(prod_b);
+    const uint32_t n2 = static_cast<uint32_t>(prod_a >> 32) ^ c3 ^ k1;
+    const uint32_t n3 = static_cast<uint32_t>(prod_a);
+    c0 = n0;
+    c1 = n1;
+    c2 = n2;
+    c3 = n3;
+  }
+  return Philox4{{c0, c1, c2, c3}};
+}
+
+constexpr uint32_t kStreamSigns = 0, kStreamQjl = 1, kStreamDense = 2;
+
+double uniform_from_words(uint32_t hi, uint32_t lo) {
+  const double a = static_cast<double>(hi >> 6), b = static_cast<double>(lo >> 6);
+  return (a * 67108864.0 + b + 0.5) / 4503599627370496.0;
+}
+
+// The first `count` N(0, 1) draws of a stream, through `put(k, z)`.
+template <typename Put>
+void gaussian_stream(uint64_t seed, uint32_t stream, uint64_t count, Put put) {
+  const double two_pi = 6.283185307179586;   // nearest double to 2 pi
+  for (uint64_t p = 0; 2 * p < count; ++p) {
+    const Philox4 r = philox4x32_10(p, stream, seed);
+    const double u1 = uniform_from_words(r.w[0], r.w[1]);
+    const double u2 = uniform_from_words(r.w[2], r.w[3]);
+    const double rad = std::sqrt(-2.0 * std::log(u1));
+    put(2 * p, rad * std::cos(two_pi * u2));
+    if (2 * p + 1 < count) put(2 * p + 1, rad * std::sin(two_pi * u2));
+  }
+}
+
 }  // namespace
 
 namespace tq {
@@ -456,6 +520,37 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
   }
   *out = h;
   return TQ_OK;
+}
+
+int tq_rotation_draws(int d, int kind, uint64_t seed, int m, int8_t* signs, double* gauss_pi, float* gauss_s) {
+  if (d < 1 || d > 4096 || m < 1 || m > 4096) return TQ_EINVAL;
+  if (kind != TQ_ROT_HADAMARD && kind != TQ_ROT_DENSE) return TQ_EINVAL;
+  if (signs) {
+    for (int i = 0; i < d; ++i) signs[i] = (philox4x32_10(static_cast<uint64_t>(i), kStreamSigns, seed).w[0] >> 31) ? -1 : 1;
+  }
+  if (gauss_s) {
+    gaussian_stream(seed, kStreamQjl, static_cast<uint64_t>(m) * d,
+                    [&](uint64_t k, double z) { gauss_s[k] = static_cast<float>(z); });
+  }
+  if (gauss_pi && kind == TQ_ROT_DENSE) {
+    gaussian_stream(seed, kStreamDense, static_cast<uint64_t>(d) * d, [&](uint64_t k, double z) { gauss_pi[k] = z; });
+  }
+  return TQ_OK;
+}
+
+int tq_build_rotation_seeded(int d, int code_bits, int kind, uint64_t seed, int m, double rope_base,
+                             int64_t rope_max_pos, tq_rotation** out) {
+  if (!out) return TQ_EINVAL;
+  *out = nullptr;
+  if (d < 1 || d > 4096 || m != d) return TQ_EINVAL;
+  if (kind != TQ_ROT_HADAMARD && kind != TQ_ROT_DENSE) return TQ_EINVAL;
+  std::vector<int8_t> sg(d);
+  std::vector<float> gs(static_cast<size_t>(m) * d);
+  std::vector<double> gp(kind == TQ_ROT_DENSE ? static_cast<size_t>(d) * d : 0);
+  const int st = tq_rotation_draws(d, kind, seed, m, sg.data(), gp.empty() ? nullptr : gp.data(), gs.data());
+  if (st != TQ_OK) return st;
+  return tq_build_rotation(d, code_bits, kind, sg.data(), gp.empty() ? nullptr : gp.data(), gs.data(), m, rope_base,
+                           rope_max_pos, out);
 }
 
 int tq_free_rotation(tq_rotation* h) {

@@ -38,6 +38,8 @@ def _load():
         "tq_version": (c_i, []),
         "tq_lloyd_max": (c_i, [c_i, c_i, c_p, c_p]),
         "tq_build_rotation": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_i, c_d, c_i64, ctypes.POINTER(c_p)]),
+        "tq_build_rotation_seeded": (c_i, [c_i, c_i, c_i, ctypes.c_uint64, c_i, c_d, c_i64, ctypes.POINTER(c_p)]),
+        "tq_rotation_draws": (c_i, [c_i, c_i, ctypes.c_uint64, c_i, c_p, c_p, c_p]),
         "tq_free_rotation": (c_i, [c_p]),
         "tq_rotation_export": (c_i, [c_p, c_p, c_p, c_p, c_p]),
         "tq_rotation_dims": (c_i, [c_p, c_p, c_p, c_p, c_p, c_p]),
@@ -123,22 +125,43 @@ def lloyd_max(d: int, bits: int):
     return lv, th
 
 
+def rotation_draws(d: int, seed: int, kind: str = "hadamard", m: int | None = None) -> dict:
+    """Host-only: the draws a handle built from ``seed`` uses (the library's
+    Philox4x32-10 streams): signs int8 [d], gauss_s float32 [m, d] and, for
+    ``kind='dense'``, gauss_pi float64 [d, d]."""
+    m = d if m is None else m
+    kind_code = {"hadamard": TQ_ROT_HADAMARD, "dense": TQ_ROT_DENSE}[kind]
+    signs = np.zeros(d, np.int8)
+    gs = np.zeros((m, d), np.float32)
+    gp = np.zeros((d, d), np.float64) if kind == "dense" else None
+    _check(_lib.tq_rotation_draws(d, kind_code, int(seed) & (2**64 - 1), m, signs.ctypes.data,
+                                  None if gp is None else gp.ctypes.data, gs.ctypes.data), "tq_rotation_draws")
+    return {"signs": signs, "gauss_s": gs, "gauss_pi": gp}
+
+
 class Rotation:
     """A codec handle (rotation, QJL matrix, codebook, RoPE tables) on the
-    current CUDA device.  ``randomness`` holds the seeded draws
-    (``signs``, ``gauss_s`` and, for ``kind='dense'``, ``gauss_pi``)."""
+    current CUDA device.  ``randomness`` is either a dict of draws (``signs``,
+    ``gauss_s`` and, for ``kind='dense'``, ``gauss_pi``) or an integer seed,
+    from which the library draws them itself (tq_build_rotation_seeded)."""
 
-    def __init__(self, d: int, bits: int, randomness: dict, kind: str = "hadamard",
+    def __init__(self, d: int, bits: int, randomness, kind: str = "hadamard",
                  rope_base: float = 0.0, rope_max_pos: int = 1 << 21):
         kind_code = {"hadamard": TQ_ROT_HADAMARD, "dense": TQ_ROT_DENSE}[kind]
-        signs = np.ascontiguousarray(randomness["signs"], dtype=np.int8)
-        gs = np.ascontiguousarray(randomness["gauss_s"], dtype=np.float32)
-        gp = randomness.get("gauss_pi")
-        gp = None if gp is None else np.ascontiguousarray(gp, dtype=np.float64)
         h = ctypes.c_void_p()
-        _check(_lib.tq_build_rotation(d, bits, kind_code, signs.ctypes.data,
-                                      None if gp is None else gp.ctypes.data, gs.ctypes.data, gs.shape[0],
-                                      float(rope_base), int(rope_max_pos), ctypes.byref(h)), "tq_build_rotation")
+        if isinstance(randomness, (int, np.integer)):
+            _check(_lib.tq_build_rotation_seeded(d, bits, kind_code, int(randomness) & (2**64 - 1), d,
+                                                 float(rope_base), int(rope_max_pos), ctypes.byref(h)),
+                   "tq_build_rotation_seeded")
+        else:
+            signs = np.ascontiguousarray(randomness["signs"], dtype=np.int8)
+            gs = np.ascontiguousarray(randomness["gauss_s"], dtype=np.float32)
+            gp = randomness.get("gauss_pi")
+            gp = None if gp is None else np.ascontiguousarray(gp, dtype=np.float64)
+            _check(_lib.tq_build_rotation(d, bits, kind_code, signs.ctypes.data,
+                                          None if gp is None else gp.ctypes.data, gs.ctypes.data, gs.shape[0],
+                                          float(rope_base), int(rope_max_pos), ctypes.byref(h)),
+                   "tq_build_rotation")
         self._h = h
         dd, mm, bb = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
         cb, sb = ctypes.c_int64(), ctypes.c_int64()
