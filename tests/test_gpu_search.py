@@ -129,3 +129,45 @@ def test_search_full_size_sampled(cuda_device, bits):
     rec = osearch.recall_at_k(ids[:50], exact)
     print(f"recall@10 (bits {bits}+1, 50 queries): {rec:.3f}")
     assert rec > (0.3 if bits == 1 else 0.6)
+
+
+def _oracle_pack_chunked(o, db, chunk=16384):
+    parts = [oracle_records(o, db[s:s + chunk])[:3] for s in range(0, len(db), chunk)]
+    return tuple(np.concatenate([p[i] for p in parts]) for i in range(3))
+
+
+def _oracle_scores_chunked(o, q, codes, signs, norms, chunk=16384):
+    return np.concatenate([osearch.search_scores(o, q, codes[s:s + chunk], signs[s:s + chunk], norms[s:s + chunk])
+                           for s in range(0, len(codes), chunk)], axis=1)
+
+
+@pytest.mark.parametrize("bits", [1, 3])
+def test_search_top10_id_set_over_many_waves(cuda_device, bits):
+    """Top-10 id sets at scale, on the grid of the 1M x 1536 search workload:
+    1000 queries (63 query tiles of 16) over 262,144 database rows of d = 256
+    give 75 row ranges of 3,584 rows (28 tiles of 128) per query tile, the
+    same 63 x 75 = 4,725 CTAs (about 16 waves) as the full workload, and a
+    merge of 75 partial lists per query.  (d = 256 keeps the float64 oracle
+    encode of the whole database to seconds; the grid and the merge do not
+    depend on d.)  The database records are the oracle's own encoding,
+    uploaded to the device, so the oracle reads nothing the GPU wrote; for 4
+    sampled queries the GPU's id set must be the oracle's top-10 up to
+    near-ties at the 10th score."""
+    from vector_quantization_b200 import tq
+    cfg = synth.CONFIGS["vector_search_d1536"]
+    nq, k, seed = cfg["n_queries"], cfg["top_k"], cfg["seed"]
+    d, N = 256, 262_144
+    U = synth.haar_basis(d, seed)
+    db = synth.anisotropic(N, d, seed + 10, basis=U)
+    qs = synth.anisotropic(nq, d, seed + 11, basis=U)
+    g = _gpu_rot(d, bits, seed + bits)
+    o, _ = oracle_rotation(d, bits, seed + bits, kind="dense")
+    codes, signs, norms = _oracle_pack_chunked(o, db)
+    dev = cuda_device
+    sc, ids = tq.search_topk(g, torch.from_numpy(qs).to(dev),
+                             tuple(torch.from_numpy(a).to(dev) for a in (codes, signs, norms)), k)
+    torch.cuda.synchronize()
+    sc, ids = sc.cpu().numpy(), ids.cpu().numpy()
+    sample = np.random.default_rng(100 + bits).choice(nq, 4, replace=False)
+    ref = _oracle_scores_chunked(o, qs[sample], codes, signs, norms)
+    _check_topk(sc[sample], ids[sample], ref, k)
