@@ -50,7 +50,7 @@ UNIT = "tokens/s"
 SPLIT_TRAFFIC_PER_TOKEN = (235_454_464 + 6_769_152) / (16 * 8 * 16384)
 
 EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1",
-          "decode_llama8b_layer_window", "tiny_d128_t1024", "encode_esm2_33_layers")
+          "decode_llama8b_layer_window", "tiny_d128_t1024", "encode_esm2_33_layers", "memory_esm2")
 
 
 def parse():
@@ -87,7 +87,7 @@ def config_json(c, args, world):
             "kv_heads": c["kv_heads"], "head_dim": c["head_dim"], "context": c["tokens"],
             "bits": f"{args.bits}+1", "qjl_m": c["head_dim"], "kv_dtype_in": "bf16",
             "cache_bytes_per_step": c["layers"] * c["batch"] * c["kv_heads"] * c["tokens"] * 2 * rec_bytes(c, args),
-            "l2": "inputs larger than L2 (packed cache per layer >> 126 MB); no flush",
+            "l2": "inputs > L2, no flush",
             "parallelism": f"replicas x{world} (weak)" if world > 1 else "single GPU"}
 
 
@@ -188,8 +188,8 @@ def oracle_baseline(c, args, budget_s=12.0, max_steps=None):
     except AttributeError:
         cores = os.cpu_count()
     return {"value": T / per, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"1 layer x 1 sequence x 1 kv-head ({T} tokens, {G} query heads) per step, "
-                      f"{len(times)} steps, {per:.3f} s/step; float64 NumPy"}, len(times), per
+            "sample": f"1 layer x 1 seq x 1 kv-head ({T} tokens, {G} q-heads) per step, {len(times)} steps"}, \
+        len(times), per
 
 
 
@@ -384,9 +384,14 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, 
         try:
             for key, b in oracle_extra_baselines(select).items():
                 if key in out and "error" not in out[key]:
-                    out[key]["cpu_baseline"] = b
+                    out[key]["cpu"] = float(f"{b['value']:.4g}")   # the oracle, same unit as "value"
         except Exception as exc:
             out["cpu_baseline_error"] = f"{type(exc).__name__}: {exc}"
+    if "memory_esm2" in select:
+        try:
+            out["memory_esm2"] = memory_ratio_esm2()
+        except Exception as exc:
+            out["memory_esm2"] = {"error": f"{type(exc).__name__}: {exc}"}
     return out
 
 
@@ -407,10 +412,8 @@ def _extras_70b(dev, peak_gbs, select, Hkv, Hq, d, T, seed, c):
     nvec = 2 * Hkv * T
     byts = nvec * (2 * d + rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)))
     if "encode_70b_slice" in select:
-        out["encode_70b_slice"] = {"vectors": nvec, "ms": round(ms, 4), "vectors_per_s": nvec / ms * 1e3,
-                                   "GB_s": round(byts / ms / 1e6, 1),
-                                   "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4), "algorithmic_bytes": byts,
-                                   "note": "bf16 in (256 B) + packed record out (56 B) per vector"}
+        out["encode_70b_slice"] = {"value": nvec / ms * 1e3, "unit": "vectors/s", "ms": round(ms, 4),
+                                   "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4)}
     del k, v
     if "decode_70b_slice" not in select:
         return out
@@ -420,9 +423,8 @@ def _extras_70b(dev, peak_gbs, select, Hkv, Hq, d, T, seed, c):
     o = torch.empty((1, Hq, d), dtype=torch.float32, device=dev)
     ms = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws), reps=10)
     byts = Hkv * T * 2 * rec_bytes({"head_dim": d}, argparse.Namespace(bits=2))
-    out["decode_70b_slice"] = {"tokens_per_s": Hkv * T / ms * 1e3, "ms": round(ms, 4),
-                               "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
-                               "note": "G = 8 query heads per KV head; all three launches timed"}
+    out["decode_70b_slice"] = {"value": Hkv * T / ms * 1e3, "unit": "tokens/s", "ms": round(ms, 4),
+                               "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4)}
     return out
 
 
@@ -444,24 +446,44 @@ def _extra_encoder(dev, g):
     ws = tq.alloc_workspace(tq._lib.tq_encoder_workspace_size(rk.handle, B, H, T), dev)
     ms = _time_ms(lambda: tq.encoder_attention(rk, rv, q, kc, vc, T, out=o, workspace=ws))
     flops = 2 * B * H * T * T * 2 * (d + d)
-    out["encoder_esm2_layer"] = {"ms": round(ms, 4), "TFLOP_s": round(flops / ms / 1e9, 1), "algorithmic_flops": flops,
-                                 "note": "2 B H S T (d + m) MACs for scores and for values; tcgen05 tensor core (d = 64, 1-2 bit codes)"}
+    out["encoder_esm2_layer"] = {"value": round(flops / ms / 1e9, 1), "unit": "TFLOP/s", "ms": round(ms, 4)}
     return out
 
 
-def _extra_search(dev, g, rows=None):
+def _extra_search(dev, g, rows=None, recall_queries=100):
+    """1M x 1536 search at 1+1 and 3+1 bits: encode of the database, top-10
+    of 1000 queries, and recall@10 of the first `recall_queries` queries
+    against exact float64 brute-force inner-product search."""
     import torch
     import synth
     from vector_quantization_b200 import tq
     out = {}
-    # vector search: 1M x 1536 fp32, 1000 queries, top-10, 1+1 bits
+    # x = U (lambda^1/2 g), lambda_i = i^-0.8, U the workload's seeded Haar basis
     c = synth.CONFIGS["vector_search_d1536"]
     N, d, nq, kk, seed = c["n_db"], c["dim"], c["n_queries"], c["top_k"], c["seed"]
     N = rows or N
+    U = torch.from_numpy(synth.haar_basis(d, seed)).to(dev)
+    Uf = U.float()
     g.manual_seed(seed)
     lam = (torch.arange(1, d + 1, device=dev, dtype=torch.float32) ** -0.4)
-    db = torch.randn((N, d), generator=g, device=dev) * lam
-    qs = torch.randn((nq, d), generator=g, device=dev) * lam
+    db = torch.empty((N, d), dtype=torch.float32, device=dev)
+    for s0 in range(0, N, 131072):
+        n = min(N, s0 + 131072) - s0
+        db[s0:s0 + n] = (torch.randn((n, d), generator=g, device=dev) * lam) @ Uf.T
+    qs = (torch.randn((nq, d), generator=g, device=dev) * lam) @ Uf.T
+    # exact float64 top-10 of the recall subset
+    nr = min(recall_queries, nq)
+    qd = qs[:nr].double()
+    best_s = torch.full((nr, kk), -float("inf"), dtype=torch.float64, device=dev)
+    best_i = torch.zeros((nr, kk), dtype=torch.int64, device=dev)
+    for s0 in range(0, N, 131072):
+        sc = qd @ db[s0:s0 + 131072].double().T
+        cat_s = torch.cat([best_s, sc], 1)
+        cat_i = torch.cat([best_i, torch.arange(s0, s0 + sc.shape[1], device=dev).expand(nr, -1)], 1)
+        top = cat_s.topk(kk, dim=1)
+        best_s, best_i = top.values, cat_i.gather(1, top.indices)
+    exact = best_i.cpu().numpy()
+    del U, Uf
     wsd = None
     for bits, key in ((1, "search_1m_d1536"), (3, "search_1m_d1536_3p1")):
         rot = tq.Rotation(d, bits, synth.rotation_randomness(d, [seed, bits], dense=True), kind="dense")
@@ -471,13 +493,35 @@ def _extra_search(dev, g, rows=None):
         ms_enc = _time_ms(lambda: tq.quantize_dense(rot, db, out=packed, workspace=wsd), reps=1, warm=1)
         wss = tq.alloc_workspace(tq.search_workspace_size(rot, nq, N, kk), dev)
         ms = _time_ms(lambda: tq.search_topk(rot, qs, packed, kk, workspace=wss), reps=2, warm=1)
+        _, ids = tq.search_topk(rot, qs[:nr], packed, kk)
+        ids = ids.cpu().numpy()
+        recall = float(np.mean([len(set(ids[i].tolist()) & set(exact[i].tolist())) / kk for i in range(nr)]))
         flops = 2 * nq * N * (d + d)
-        gemm_flops = 2 * N * d * d * 2   # y = Pi x and S r, one fp32 product each
-        out[key] = {"queries_per_s": nq / ms * 1e3, "ms": round(ms, 3), "TFLOP_s": round(flops / ms / 1e9, 1),
-                    "encode_ms": round(ms_enc, 3), "encode_TFLOP_s": round(gemm_flops / ms_enc / 1e9, 1),
-                    "note": f"{bits}+1 bits, top-10; data isotropic-in-basis stand-in"}
+        out[key] = {"value": nq / ms * 1e3, "unit": "queries/s", "ms": round(ms, 3),
+                    "TFLOP_s": round(flops / ms / 1e9, 1), "recall10": round(recall, 4), "recall_q": nr,
+                    "enc_ms": round(ms_enc, 3)}
         del packed, wss
     return out
+
+
+def memory_ratio_esm2():
+    """Cache bytes of the ESM-2-650M-shaped encoder (33 layers, 20 heads,
+    d 64, 1024 tokens, batch 1) at 2+1 bits against float32 K and V, from the
+    library's record geometry (tq_rotation_dims), next to the page's quoted
+    330 MB -> 47 MB (7.1x)."""
+    import ctypes
+    import synth
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["esm2_650m_encoder"]
+    L, H, T, d = c["layers"], c["heads"], c["tokens"], c["head_dim"]
+    rot = tq.Rotation(d, 2, 0)
+    cb, sb = ctypes.c_int64(), ctypes.c_int64()
+    tq._lib.tq_rotation_dims(rot.handle, None, None, None, ctypes.byref(cb), ctypes.byref(sb))
+    rec = cb.value + sb.value + 8
+    vecs = 2 * L * H * T
+    fp32 = vecs * d * 4
+    return {"fp32_MiB": round(fp32 / 2**20, 2), "packed_MiB": round(vecs * rec / 2**20, 3),
+            "ratio": round(fp32 / (vecs * rec), 3), "page": "330 MB -> 47 MB, 7.1x"}
 
 
 def _extra_decode_3p1(dev, peak_gbs):
@@ -508,9 +552,9 @@ def _extra_decode_3p1(dev, peak_gbs):
     torch.cuda.synchronize()
     ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     byts = B * Hkv * T * 2 * rec_bytes({"head_dim": d}, argparse.Namespace(bits=3))
-    return {"decode_llama8b_layer_3p1": {"split_ms": round(ms, 4), "GB_s": round(byts / ms / 1e6, 1),
-                                         "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
-                                         "algorithmic_bytes": byts, "note": "one layer, 144 B per token pair"}}
+    return {"decode_llama8b_layer_3p1": {"value": B * Hkv * T / ms * 1e3, "unit": "tokens/s", "split_ms": round(ms, 4),
+                                         "GB_s": round(byts / ms / 1e6, 1),
+                                         "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4)}}
 
 def _extra_decode_window(dev, peak_gbs, R=128):
     """One layer of the Llama-3.1-8B-shaped decode (B16, Hq32, Hkv8, 2+1 bits)
@@ -543,12 +587,9 @@ def _extra_decode_window(dev, peak_gbs, R=128):
                                                        workspace=ws), reps=20, warm=3)
     ms_p = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws2), reps=20, warm=3)
     byts = B * Hkv * (T - R) * 2 * rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)) + 2 * kw.numel() * 2
-    return {"decode_llama8b_layer_window": {"ms": round(ms_w, 4), "ms_all_packed": round(ms_p, 4),
-                                            "GB_s": round(byts / ms_w / 1e6, 1),
-                                            "frac_hbm": round(byts / ms_w / 1e6 / peak_gbs, 4),
-                                            "algorithmic_bytes": byts,
-                                            "note": f"{T - R} packed tokens (112 B per pair) + {R}-token bf16 window "
-                                                    "(512 B per pair); whole call, 5 launches"}}
+    return {"decode_llama8b_layer_window": {"value": B * Hkv * T / ms_w * 1e3, "unit": "tokens/s",
+                                            "ms": round(ms_w, 4), "ms_all_packed": round(ms_p, 4),
+                                            "frac_hbm": round(byts / ms_w / 1e6 / peak_gbs, 4)}}
 
 def _extra_tiny(dev):
     """The tiny workload (1 head, d 128, 1024 fp32 tokens, heavy-tailed with
@@ -575,9 +616,7 @@ def _extra_tiny(dev):
     o = torch.empty((1, 1, d), dtype=torch.float32, device=dev)
     us_dec = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws),
                       reps=50, warm=5) * 1e3
-    return {"tiny_d128_t1024": {"encode_us": round(us_enc, 2), "decode_us": round(us_dec, 2),
-                                "note": "1024 keys (RoPE) + 1024 values encoded (two calls), then one decode of "
-                                        "one fp32 query; latency, inputs resident in L2"}}
+    return {"tiny_d128_t1024": {"value": round(us_dec, 2), "unit": "decode us", "encode_us": round(us_enc, 2)}}
 
 
 def _extra_encode_esm2(dev, peak_gbs, g):
@@ -604,10 +643,9 @@ def _extra_encode_esm2(dev, peak_gbs, g):
     ms = _time_ms(enc, reps=5, warm=2)
     nvec = 2 * n
     byts = nvec * (2 * d + rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)))
-    return {"encode_esm2_33_layers": {"vectors": nvec, "ms": round(ms, 4), "vectors_per_s": nvec / ms * 1e3,
+    return {"encode_esm2_33_layers": {"value": nvec / ms * 1e3, "unit": "vectors/s", "ms": round(ms, 4),
                                       "GB_s": round(byts / ms / 1e6, 1),
-                                      "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4), "algorithmic_bytes": byts,
-                                      "note": "bf16 in (128 B) + packed record out (32 B) per vector"}}
+                                      "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4)}}
 
 
 # --------------------------------------------------------------------------- reference arm

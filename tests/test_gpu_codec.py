@@ -71,8 +71,9 @@ def test_encode_parity(cuda_device, d, bits, dtype):
 @pytest.mark.parametrize("bits", [1, 2, 3])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_encode_parity_large_batch(cuda_device, d, bits, dtype):
-    """Batches of 16384 or more vectors take the thread-per-vector kernel:
-    several 128-row tiles per CTA group and a ragged last tile."""
+    """Batches of 16384 or more vectors take the 128-row tile kernels (the
+    tensor-core rotation kernel for d = 128, the row kernel for d = 64):
+    several tiles per CTA group and a ragged last tile."""
     _run_encode(d, bits, 16384 + 1031, dtype, rope=True, seed=200 + bits)
 
 
