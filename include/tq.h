@@ -302,7 +302,12 @@ size_t tq_search_workspace_size(const tq_rotation* h, int nq, int64_t N, int k);
  *   cache_stride  records between consecutive sequences (>= T, even)
  *   B, Hq, Hkv  batch, query heads, KV heads; Hq % Hkv == 0,
  *               Hq/Hkv in {1, 2, 4, 8} and B*Hkv <= 65535
- *   T           cached tokens per sequence (0 gives an all-zero output)
+ *   T           cached tokens per sequence, or with seq_lens the largest
+ *               length (0 gives an all-zero output)
+ *   seq_lens    device [B] int32 tokens of each sequence b (records 0 ..
+ *               seq_lens[b]-1 of its KV heads), each in 0..T; NULL: all T.
+ *               A length outside 0..T makes that sequence's outputs NaN
+ *               (device memory is not read on the host)
  *   scale       softmax scale (typically 1/sqrt(d))
  *   out         device [B, Hq, d] float32
  *   workspace   device scratch of at least tq_decode_workspace_size(...)
@@ -316,8 +321,8 @@ int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
                         const float* k_norms, const uint8_t* v_codes,
                         const uint8_t* v_signs, const float* v_norms,
                         int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
-                        float scale, float* out, void* workspace,
-                        size_t workspace_bytes, void* stream);
+                        const int32_t* seq_lens, float scale, float* out,
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes tq_decode_attention needs for these sizes (0 if invalid). */
 size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
@@ -330,8 +335,10 @@ size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
  * residual kept in full precision; when the residual is full the caller
  * flushes it (tq_quantize_kv / tq_quantize_kv_pair with positions T .. T+R-1
  * into records T .. T+R-1) and empties the window.
- *   hk ... cache_stride, B, Hq, Hkv, T, scale, out
- *               as in tq_decode_attention (T packed tokens, possibly 0)
+ *   hk ... cache_stride, B, Hq, Hkv, T, seq_lens, scale, out
+ *               as in tq_decode_attention (T packed tokens, possibly 0; with
+ *               seq_lens, sequence b has seq_lens[b] packed tokens and its
+ *               window tokens sit at positions seq_lens[b] + i)
  *   k_window, v_window
  *               device [B*Hkv, window_stride, d] elements of window_dtype:
  *               row (b*Hkv + j)*window_stride + i is token i of the window
@@ -357,9 +364,9 @@ int tq_decode_attention_window(const tq_rotation* hk, const tq_rotation* hv,
                                int64_t cache_stride, const void* k_window,
                                const void* v_window, int window_dtype,
                                int64_t window_stride, int R, int B, int Hq,
-                               int Hkv, int64_t T, float scale, float* out,
-                               void* workspace, size_t workspace_bytes,
-                               void* stream);
+                               int Hkv, int64_t T, const int32_t* seq_lens,
+                               float scale, float* out, void* workspace,
+                               size_t workspace_bytes, void* stream);
 
 /* Workspace bytes tq_decode_attention_window needs (0 if invalid). */
 size_t tq_decode_window_workspace_size(const tq_rotation* hk,
@@ -431,7 +438,8 @@ int tq_decode_attention_noalloc(const tq_rotation* hk, const tq_rotation* hv,
                                 const float* k_norms, const uint8_t* v_codes,
                                 const uint8_t* v_signs, const float* v_norms,
                                 int64_t cache_stride, int B, int Hq, int Hkv,
-                                int64_t T, float scale, float* out, void* stream);
+                                int64_t T, const int32_t* seq_lens, float scale,
+                                float* out, void* stream);
 
 /*
  * tq_profile_next_decode - instrumentation for benchmarks.  The next

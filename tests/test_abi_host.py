@@ -69,8 +69,10 @@ def test_bad_arguments_are_rejected_on_host():
     assert tq._lib.tq_quantize_kv(None, None, 0, 1, 64, None, 1, 0, 0, None, None, None, 1, None) == tq.TQ_EINVAL
     # window decode: null handles rejected on the host, before any device call
     assert tq._lib.tq_decode_attention_window(None, None, None, 0, None, None, None, None, None, None, None, 0,
-                                              None, None, 0, 0, 0, 1, 4, 1, 0, 0.125, None, None, 0,
+                                              None, None, 0, 0, 0, 1, 4, 1, 0, None, 0.125, None, None, 0,
                                               None) == tq.TQ_EINVAL
+    assert tq._lib.tq_decode_attention(None, None, None, 0, None, None, None, None, None, None, None, 0,
+                                       1, 4, 1, 0, None, 0.125, None, None, 0, None) == tq.TQ_EINVAL
 
 
 def test_window_binding_checks_shapes_before_any_call():

@@ -197,3 +197,60 @@ def test_decode_70b_slice_full_size_sampled(cuda_device):
     qq = q[:, j * G:(j + 1) * G].float().cpu().numpy()
     ref = at.decode_attention(rk_o, rv_o, qq, [T - 1], kk, vv, 1 / np.sqrt(D))
     assert_close(out[:, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"70B slice kv-head {j}")
+
+@pytest.mark.parametrize("bits,G", [(2, 4), (3, 8), (1, 1)])
+def test_decode_ragged_batch(cuda_device, bits, G):
+    """Per-sequence lengths (seq_lens, device int32): sequence b attends to its
+    own first seq_lens[b] records, with lengths 0, 1, 17, 300 and the maximum T
+    in one call.  Records past a sequence's length are poisoned (NaN norms,
+    0xFF bytes) so a read past it would show; an empty sequence gives zeros."""
+    from vector_quantization_b200 import tq
+    dev = cuda_device
+    lens = [0, 1, 17, 300, 1000]
+    B, Hkv, T = len(lens), 2, max(lens)
+    Hq, cap = G * Hkv, T + 4
+    seed = 40 + bits + G
+    rk_o, _ = oracle_rotation(D, bits, 500 + seed, rope=10000.0)
+    rv_o, _ = oracle_rotation(D, bits, 600 + seed)
+    rk, rv = _gpu_rot(bits, 500 + seed, 10000.0), _gpu_rot(bits, 600 + seed, 0.0)
+    k = synth.heavy_tailed((B, Hkv, T, D), 700 + seed)
+    v = synth.heavy_tailed((B, Hkv, T, D), 800 + seed)
+    kc = list(_packed_cache(rk_o, k, cap, np.arange(T)))
+    vc = list(_packed_cache(rv_o, v, cap))
+    for b, n in enumerate(lens):
+        for cache in (kc, vc):
+            cache[0][b, :, n:] = 0xFF
+            cache[1][b, :, n:] = 0xFF
+            cache[2][b, :, n:] = np.nan
+    q = torch.from_numpy(synth.heavy_tailed((B, Hq, D), 900 + seed)).to(dev)
+    qpos = [max(n - 1, 0) for n in lens]
+    out = tq.decode_attention(rk, rv, q, torch.tensor(qpos, dtype=torch.int64, device=dev), _to_dev(kc, dev),
+                              _to_dev(vc, dev), T, seq_lens=torch.tensor(lens, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    out = out.cpu().numpy()
+    for b, n in enumerate(lens):
+        ref = at.decode_attention(rk_o, rv_o, q[b:b + 1].cpu().numpy(), [qpos[b]],
+                                  tuple(a[b:b + 1, :, :n] for a in kc), tuple(a[b:b + 1, :, :n] for a in vc),
+                                  1 / np.sqrt(D))
+        assert_close(out[b:b + 1], ref, what=f"sequence {b} of length {n}")
+    assert np.all(out[0] == 0.0)
+
+
+def test_decode_length_outside_range_gives_nan(cuda_device):
+    """A seq_lens entry above T (or negative) cannot be checked on the host
+    (device memory); that sequence's outputs are NaN, the others unaffected."""
+    from vector_quantization_b200 import tq
+    dev = cuda_device
+    B, Hkv, G, T = 3, 1, 4, 64
+    rk_o, _ = oracle_rotation(D, 2, 71, rope=10000.0)
+    rv_o, _ = oracle_rotation(D, 2, 72)
+    rk, rv = _gpu_rot(2, 71, 10000.0), _gpu_rot(2, 72, 0.0)
+    kc = _packed_cache(rk_o, synth.heavy_tailed((B, Hkv, T, D), 73), T, np.arange(T))
+    vc = _packed_cache(rv_o, synth.heavy_tailed((B, Hkv, T, D), 74), T)
+    q = torch.from_numpy(synth.heavy_tailed((B, G * Hkv, D), 75)).to(dev)
+    qpos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    out = tq.decode_attention(rk, rv, q, qpos, _to_dev(kc, dev), _to_dev(vc, dev), T,
+                              seq_lens=torch.tensor([T, T + 1, -3], dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    out = out.cpu().numpy()
+    assert np.all(np.isfinite(out[0])) and np.all(np.isnan(out[1])) and np.all(np.isnan(out[2]))

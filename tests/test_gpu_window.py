@@ -235,3 +235,39 @@ def test_window_full_size_sampled(cuda_device):
                                          kw[b:b + 1, j:j + 1].double().cpu().numpy(),
                                          vw[b:b + 1, j:j + 1].double().cpu().numpy(), 1 / np.sqrt(D))
         assert_close(out[b:b + 1, j * G:(j + 1) * G].cpu().numpy(), ref, what=f"seq {b} kv-head {j}")
+
+
+def test_window_ragged_batch(cuda_device):
+    """Per-sequence packed lengths with a window of R tokens after each: the
+    window of sequence b sits at positions seq_lens[b] .. seq_lens[b] + R - 1,
+    lengths 0, 5 and 300 in one call."""
+    from vector_quantization_b200 import tq
+    dev = cuda_device
+    lens, R, G, Hkv, bits = [0, 5, 300], 40, 4, 2, 2
+    B, T = len(lens), max(lens)
+    cap = T + 6
+    rk_o, _ = oracle_rotation(D, bits, 1531, rope=10000.0)
+    rv_o, _ = oracle_rotation(D, bits, 1631)
+    rk, rv = _gpu_rot(bits, 1531, 10000.0), _gpu_rot(bits, 1631, 0.0)
+    kc = list(_packed_cache(rk_o, synth.heavy_tailed((B, Hkv, T, D), 1731), cap, np.arange(T)))
+    vc = list(_packed_cache(rv_o, synth.heavy_tailed((B, Hkv, T, D), 1831), cap))
+    for b, n in enumerate(lens):
+        for cache in (kc, vc):
+            cache[0][b, :, n:] = 0xFF
+            cache[1][b, :, n:] = 0xFF
+            cache[2][b, :, n:] = np.nan
+    kw, kw_ref = _window((B, Hkv, R, D), 1931, torch.float32, R + 2)
+    vw, vw_ref = _window((B, Hkv, R, D), 2031, torch.float32, R + 2)
+    q = torch.from_numpy(synth.heavy_tailed((B, G * Hkv, D), 2131)).to(dev)
+    qpos = [n + R - 1 for n in lens]
+    out = tq.decode_attention_window(rk, rv, q, torch.tensor(qpos, dtype=torch.int64, device=dev),
+                                     tuple(torch.from_numpy(a).to(dev) for a in kc),
+                                     tuple(torch.from_numpy(a).to(dev) for a in vc), T, kw.to(dev), vw.to(dev), R,
+                                     seq_lens=torch.tensor(lens, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    out = out.cpu().numpy()
+    for b, n in enumerate(lens):
+        ref = at.decode_attention_window(rk_o, rv_o, q[b:b + 1].double().cpu().numpy(), [qpos[b]],
+                                         tuple(a[b:b + 1, :, :n] for a in kc), tuple(a[b:b + 1, :, :n] for a in vc),
+                                         kw_ref[b:b + 1], vw_ref[b:b + 1], 1 / np.sqrt(D))
+        assert_close(out[b:b + 1], ref, what=f"sequence {b}: {n} packed + {R} window tokens")

@@ -26,7 +26,7 @@ def _bind():
     fn = tq._lib.tq_decode_attention_noalloc
     c_i, c_i64, c_p, c_f = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float
     fn.restype = c_i
-    fn.argtypes = [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i, c_i64, c_f, c_p, c_p]
+    fn.argtypes = [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p]
     return tq, fn
 
 
@@ -46,7 +46,7 @@ def _noalloc(fn, rk, rv, kc, vc, q, qpos, T, out):
     B, Hq, _ = q.shape
     Hkv, cap = kc[0].shape[1], kc[0].shape[2]
     st = fn(rk.handle, rv.handle, q.data_ptr(), 0, qpos.data_ptr(), kc[0].data_ptr(), kc[1].data_ptr(),
-            kc[2].data_ptr(), vc[0].data_ptr(), vc[1].data_ptr(), vc[2].data_ptr(), cap, B, Hq, Hkv, T,
+            kc[2].data_ptr(), vc[0].data_ptr(), vc[1].data_ptr(), vc[2].data_ptr(), cap, B, Hq, Hkv, T, None,
             1.0 / np.sqrt(D), out.data_ptr(), torch.cuda.current_stream().cuda_stream)
     return st
 
@@ -77,5 +77,5 @@ def test_noalloc_rejects_requests_beyond_its_scratch(cuda_device):
     B, Hkv, T = 512, 8, 1 << 20
     assert tq.decode_workspace_size(rk, rv, B, 4 * Hkv, Hkv, T) > (16 << 20)
     st = fn(rk.handle, rv.handle, q.data_ptr(), 0, qpos.data_ptr(), None, None, None, None, None, None,
-            T, B, 4 * Hkv, Hkv, T, 0.088, None, torch.cuda.current_stream().cuda_stream)
+            T, B, 4 * Hkv, Hkv, T, None, 0.088, None, torch.cuda.current_stream().cuda_stream)
     assert st == tq.TQ_EWORKSPACE

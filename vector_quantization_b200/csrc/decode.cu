@@ -36,6 +36,7 @@
 #include <mutex>
 
 #include "bitplane.cuh"
+#include "tcgen05.cuh"
 #include "tq_internal.h"
 
 namespace {
@@ -68,15 +69,20 @@ struct DecodeParams {
   float walsh_k[4];
   float walsh_v[4];
   uint32_t one_h, one_b;   // kOneH2 / kOneB2, passed at run time (see bit_select)
+  const int32_t* seq_lens; // [B] tokens of each sequence (<= T), or null: all T
+  int Hkv;
 };
 
-// Shared-memory position of the 16-byte chunk `part` of token `tok`'s codes.
-// With 2-bit codes (two chunks per token) the chunks of tokens 4..7 (mod 8)
-// are swapped so that the fragment reads below are free of bank conflicts.
+// Polls of a stage's mbarrier before the warp gives up on its copies (about a
+// second); the warp then reports NaN for its heads instead of hanging.
+constexpr int kCopyWaitPolls = 1 << 17;
+
+// Shared-memory position of the 16-byte chunk `part` (code plane) of token
+// `tok`'s codes: the records as they lie in the cache, one bulk copy per
+// array and tile.
 template <int BITS>
 __device__ __forceinline__ int code_chunk(int tok, int part) {
-  if constexpr (BITS == 2) return tok * 2 + (part ^ ((tok >> 2) & 1));
-  else return tok * BITS + part;
+  return tok * BITS + part;
 }
 
 template <int BITS, int G>
@@ -95,48 +101,64 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   const int bh = blockIdx.y;
   const int split = blockIdx.x;
   const uint32_t one_h = p.one_h, one_b = p.one_b;
+  // this sequence's length: T, or its own entry of seq_lens (a value outside
+  // 0..T makes every output of the sequence NaN)
+  int64_t T_seq = p.T;
+  bool bad_len = false;
+  if (p.seq_lens) {
+    const int64_t v = p.seq_lens[bh / p.Hkv];
+    bad_len = v < 0 || v > p.T;
+    T_seq = bad_len ? 0 : v;
+  }
   const int64_t t_begin = static_cast<int64_t>(split) * p.chunk;
-  const int64_t t_end = min(p.T, t_begin + p.chunk);
+  const int64_t t_end = min(T_seq, t_begin + p.chunk);
   const int n_tiles = t_end > t_begin ? static_cast<int>((t_end - t_begin + kTile - 1) / kTile) : 0;
   const int my_count = n_tiles > warp ? (n_tiles - warp + kWarps - 1) / kWarps : 0;
   const int64_t seq = static_cast<int64_t>(bh) * p.cache_stride;
   uint8_t* my_stages = smem + warp * kStages * STAGE;
 
-  const int sg_side = lane >> 4, sg_c = lane & 15;
-  const int nm_side = (lane >> 3) & 1, nm_c = lane & 7;
+  // One mbarrier per stage of this warp's ring.  Lane 0 issues a tile as six
+  // bulk copies - K codes, signs, norms and V codes, signs, norms, each one
+  // contiguous block of the cache - completing on the stage's mbarrier; the
+  // warp waits on it before reading the stage.  Rows past the tile's last
+  // token keep what the stage held before (the readers mask them).
+  __shared__ uint64_t s_mbar[kWarps][kStages];
+  if (lane == 0) {
+#pragma unroll
+    for (int st = 0; st < kStages; ++st) tqtc::mbar_init(&s_mbar[warp][st], 1);
+  }
+  __syncwarp();
+  auto tile_nv = [&](int i) {
+    const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
+    return static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
+  };
   auto issue = [&](int i) {
-    if (i < my_count) {
+    if (i < my_count && lane == 0) {
       const int64_t t0 = seq + t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
-      const int nv = static_cast<int>(t_end - (t0 - seq) < kTile ? t_end - (t0 - seq) : kTile);
+      const int nv = tile_nv(i);
+      const int nn = (nv + 1) & ~1;   // norms in pairs: 16-byte copies (record nv exists: cache_stride is even)
       uint8_t* stg = my_stages + (i % kStages) * STAGE;
-#pragma unroll
-      for (int side = 0; side < 2; ++side) {
-        const uint8_t* src = (side ? p.v_codes : p.k_codes) + t0 * CB;
-#pragma unroll
-        for (int c = lane; c < CCH; c += 32) {
-          const int tok = c / BITS, part = c % BITS;
-          cp_async16(stg + side * HALF + code_chunk<BITS>(tok, part) * 16, tok < nv ? src + c * 16 : src,
-                     tok < nv ? 16 : 0);
-        }
-      }
-      {
-        const uint8_t* src = (sg_side ? p.v_signs : p.k_signs) + t0 * SB;
-        cp_async16(stg + sg_side * HALF + kTile * CB + sg_c * 16, sg_c < nv ? src + sg_c * 16 : src, sg_c < nv ? 16 : 0);
-      }
-      if (lane < 16) {
-        const float2* src = (nm_side ? p.v_norms : p.k_norms) + t0;
-        const int bytes = max(0, min(16, (nv - 2 * nm_c) * 8));
-        cp_async16(stg + nm_side * HALF + kTile * (CB + SB) + nm_c * 16, bytes ? src + 2 * nm_c : src, bytes);
-      }
+      uint64_t* mb = &s_mbar[warp][i % kStages];
+      tqtc::mbar_arrive_expect_tx(mb, static_cast<uint32_t>(2 * (nv * (CB + SB) + nn * 8)));
+      tqtc::bulk_load(stg, p.k_codes + t0 * CB, nv * CB, mb);
+      tqtc::bulk_load(stg + kTile * CB, p.k_signs + t0 * SB, nv * SB, mb);
+      tqtc::bulk_load(stg + kTile * (CB + SB), p.k_norms + t0, nn * 8, mb);
+      tqtc::bulk_load(stg + HALF, p.v_codes + t0 * CB, nv * CB, mb);
+      tqtc::bulk_load(stg + HALF + kTile * CB, p.v_signs + t0 * SB, nv * SB, mb);
+      tqtc::bulk_load(stg + HALF + kTile * (CB + SB), p.v_norms + t0, nn * 8, mb);
     }
-    cp_async_commit();
+  };
+  // wait for tile i's copies; false if they did not complete in time
+  auto arrived = [&](int i) {
+    return tqtc::mbar_wait(&s_mbar[warp][i % kStages], static_cast<uint32_t>((i / kStages) & 1), kCopyWaitPolls);
   };
 
   // The first tiles of the cache do not depend on the q-prep launch: start
   // their copies, then wait for q-prep's outputs (programmatic dependent
   // launch; a no-op when launched without it).
+  int issued = my_count < kStages - 1 ? my_count : kStages - 1;
 #pragma unroll 1
-  for (int i = 0; i < kStages - 1; ++i) issue(i);
+  for (int i = 0; i < issued; ++i) issue(i);
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
   // The query B fragments: in registers for one n-tile (G <= 4); in shared
@@ -319,7 +341,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   };
 
   // ---- V side of one tile with its probabilities
-  auto v_side = [&](const uint8_t* stg, const float (&prob)[NT][2]) {
+  auto v_side = [&](const uint8_t* stg, const float (&prob)[NT][2], int nv) {
     const uint8_t* vcd = stg + HALF;
     const uint8_t* vs = vcd + kTile * CB;
     const float2* vn = reinterpret_cast<const float2*>(vcd + kTile * (CB + SB));
@@ -367,9 +389,9 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       uint32_t bc[P][2], bz[2];
       float wv[4], wr[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        wv[j] = pt[j] * vnorm[j].x;
-        wr[j] = pt[j] * vnorm[j].y;
+      for (int j = 0; j < 4; ++j) {   // rows past the tile's last token hold stale records
+        wv[j] = tk[j] < nv ? pt[j] * vnorm[j].x : 0.f;
+        wr[j] = tk[j] < nv ? pt[j] * vnorm[j].y : 0.f;
       }
       // B operand: lanes of even gid feed RN(w), odd gid RN(w - RN(w)), both
       // as bf16 pairs: one paired conversion, an FFMA by piece_m in {0, 1},
@@ -408,54 +430,60 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       }
     }
   };
-  auto tile_nv = [&](int i) {
-    const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
-    return static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
-  };
-
-  // Pipelined order (for G = 8 it fits the register file because the query
-  // fragments are in shared memory).
-  constexpr bool kPipe = true;
-  if constexpr (kPipe) {
+  // Pipelined order: the key side of tile i and the value side of tile i - 1
+  // share one loop body (for G = 8 this fits the register file because the
+  // query fragments are in shared memory).
+  bool failed = bad_len;
+  int consumed = 0;
+  {
     float prob_prev[NT][2];
     const uint8_t* stg_prev = my_stages;
-    if (my_count > 0) {
-      cp_async_wait<kStages - 2>();
-      __syncwarp();
-      float logit[NT][2];
-      k_side(my_stages, tile_nv(0), logit);
-      softmax(logit, prob_prev);
-      issue(kStages - 1);   // stage kStages-1 is still unused
+    int nv_prev = 0;
+    if (my_count > 0 && !failed) {
+      if (!arrived(0)) {
+        failed = true;
+      } else {
+        consumed = 1;
+        float logit[NT][2];
+        nv_prev = tile_nv(0);
+        k_side(my_stages, nv_prev, logit);
+        softmax(logit, prob_prev);
+        __syncwarp();
+        if (issued < my_count) issue(issued++);   // stage kStages-1 is still unused
+      }
     }
 #pragma unroll 1
-    for (int i = 1; i < my_count; ++i) {
-      cp_async_wait<kStages - 2>();
-      __syncwarp();
+    for (int i = 1; i < my_count && !failed; ++i) {
+      if (!arrived(i)) {
+        failed = true;
+        break;
+      }
+      consumed = i + 1;
       const uint8_t* stg = my_stages + (i % kStages) * STAGE;
+      const int nv = tile_nv(i);
       float logit[NT][2];
-      k_side(stg, tile_nv(i), logit);   // independent of the V side below
-      v_side(stg_prev, prob_prev);
+      k_side(stg, nv, logit);             // independent of the V side below
+      v_side(stg_prev, prob_prev, nv_prev);
       softmax(logit, prob_prev);
       stg_prev = stg;
+      nv_prev = nv;
       __syncwarp();
-      issue(i + kStages - 1);           // into the stage of tile i - 1
+      if (issued < my_count) issue(issued++);   // into the stage of tile i - 1
     }
-    if (my_count > 0) v_side(stg_prev, prob_prev);
-  } else {
+    if (consumed > 0 && !failed) v_side(stg_prev, prob_prev, nv_prev);
+  }
+  // copies still in flight into this warp's stages complete before the CTA
+  // leaves (bounded; after a timeout the CTA reports NaN)
 #pragma unroll 1
-    for (int i = 0; i < my_count; ++i) {
-      cp_async_wait<kStages - 2>();
-      __syncwarp();
-      const uint8_t* stg = my_stages + (i % kStages) * STAGE;
-      float logit[NT][2], prob[NT][2];
-      k_side(stg, tile_nv(i), logit);
-      softmax(logit, prob);
-      v_side(stg, prob);
-      __syncwarp();
-      issue(i + kStages - 1);           // into the stage of tile i - 1
+  for (int i = consumed; i < issued; ++i)
+    if (!arrived(i)) failed = true;
+  if (failed) {   // a finite max keeps the NaN sum from being dropped by the merges
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m_run[nt] = 0.f;
+      l_run[nt] = __int_as_float(0x7fc00000);
     }
   }
-  cp_async_wait<0>();
   __syncthreads();
 
   constexpr int REC = 2 + 2 * kD;
@@ -777,7 +805,8 @@ constexpr int kWinChunk = 32;      // window tokens per block, one partial recor
 template <typename TW, int G>
 __global__ void __launch_bounds__(kD) decode_window_kernel(
     const void* __restrict__ q, int q_f32, const int64_t* __restrict__ q_pos, int Hkv, const TW* __restrict__ k_win,
-    const TW* __restrict__ v_win, int64_t win_stride, int R, int64_t T, const float* __restrict__ v_dsigns,
+    const TW* __restrict__ v_win, int64_t win_stride, int R, int64_t T_all, const int32_t* __restrict__ seq_lens,
+    const float* __restrict__ v_dsigns,
     const float2* __restrict__ rope_hi, const float2* __restrict__ rope_lo, int64_t rope_max_pos, int rope,
     float score_scale, float* __restrict__ partial, int n_slots, int slot0) {
   constexpr int REC = 2 + 2 * kD;
@@ -789,6 +818,15 @@ __global__ void __launch_bounds__(kD) decode_window_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.y, b = bh / Hkv, chunk = blockIdx.x;
   const int t0 = chunk * kWinChunk;
+  // the window follows this sequence's packed tokens; a length outside
+  // 0..T_all makes the sequence's outputs NaN
+  int64_t T = T_all;
+  bool bad_len = false;
+  if (seq_lens) {
+    const int64_t v = seq_lens[b];
+    bad_len = v < 0 || v > T_all;
+    T = bad_len ? 0 : v;
+  }
   const int n = min(kWinChunk, R - t0);   // >= 1: the host launches ceil(R / kWinChunk) chunks
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   // The key and value rows of this warp's tokens do not depend on the query:
@@ -886,8 +924,8 @@ __global__ void __launch_bounds__(kD) decode_window_kernel(
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     if (lane == 0) {
-      stat[0][h] = mx;
-      stat[1][h] = l;
+      stat[0][h] = bad_len ? 0.f : mx;
+      stat[1][h] = bad_len ? __int_as_float(0x7fc00000) : l;
     }
   }
   __syncthreads();
@@ -1081,13 +1119,14 @@ namespace {
 
 int launch_window(int G, int win_dtype, int q_dtype, int BH, int Hkv, const void* q, const int64_t* q_pos,
                   const tq_rotation* hk, const tq_rotation* hv, int rope, const void* k_win, const void* v_win,
-                  int64_t win_stride, int R, int64_t T, float score_scale, float* partial, int n_slots, int slot,
-                  cudaStream_t s) {
+                  int64_t win_stride, int R, int64_t T, const int32_t* seq_lens, float score_scale, float* partial,
+                  int n_slots, int slot, cudaStream_t s) {
   const int q_f32 = q_dtype == TQ_F32 ? 1 : 0;
   const dim3 grid((R + kWinChunk - 1) / kWinChunk, BH);
 #define TQ_WINDOW(TW, GG)                                                                                            \
   return launch_pdl(decode_window_kernel<TW, GG>, grid, dim3(kD), 0, s, q, q_f32, q_pos, Hkv,                         \
-                    static_cast<const TW*>(k_win), static_cast<const TW*>(v_win), win_stride, R, T, hv->d_signs,   \
+                    static_cast<const TW*>(k_win), static_cast<const TW*>(v_win), win_stride, R, T, seq_lens,      \
+                    hv->d_signs,                                                                                   \
                     hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope, score_scale, partial, n_slots, slot)
   if (win_dtype == TQ_F32) {
     switch (G) {
@@ -1116,7 +1155,8 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
                 const uint8_t* k_codes, const uint8_t* k_signs, const float* k_norms, const uint8_t* v_codes,
                 const uint8_t* v_signs, const float* v_norms, int64_t cache_stride, const void* k_win,
                 const void* v_win, int win_dtype, int64_t win_stride, int R, int B, int Hq, int Hkv, int64_t T,
-                float scale, float* out, void* workspace, size_t workspace_bytes, cudaStream_t s,
+                const int32_t* seq_lens, float scale, float* out, void* workspace, size_t workspace_bytes,
+                cudaStream_t s,
                 cudaEvent_t prof_begin, cudaEvent_t prof_end) {
   {
     const int st = check_decode_sizes(hk, hv, B, Hq, Hkv, T);
@@ -1162,7 +1202,8 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   st = tq::launch_status();
   if (st != TQ_OK) return st;
   if (R > 0) {
-    st = launch_window(G, win_dtype, q_dtype, BH, Hkv, q, q_pos, hk, hv, rope, k_win, v_win, win_stride, R, T, score_scale,
+    st = launch_window(G, win_dtype, q_dtype, BH, Hkv, q, q_pos, hk, hv, rope, k_win, v_win, win_stride, R, T, seq_lens,
+                       score_scale,
                        partial, n_slots, sp.n_splits, s);
     if (st != TQ_OK) return st;
   }
@@ -1176,6 +1217,8 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   p.v_norms = reinterpret_cast<const float2*>(v_norms);
   p.cache_stride = cache_stride;
   p.T = T;
+  p.seq_lens = seq_lens;
+  p.Hkv = Hkv;
   p.chunk = sp.chunk;
   p.n_splits = sp.n_splits;
   p.n_slots = n_slots;
@@ -1220,11 +1263,12 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
                                    const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
                                    const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
                                    const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
-                                   float scale, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+                                   const int32_t* seq_lens, float scale, float* out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
   const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
   g_prof_begin = g_prof_end = nullptr;
   return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
-                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, scale, out, workspace, workspace_bytes,
+                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, workspace, workspace_bytes,
                      static_cast<cudaStream_t>(stream), prof_begin, prof_end);
 }
 
@@ -1233,12 +1277,12 @@ extern "C" int tq_decode_attention_window(const tq_rotation* hk, const tq_rotati
                                           const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
                                           const float* v_norms, int64_t cache_stride, const void* k_window,
                                           const void* v_window, int window_dtype, int64_t window_stride, int R,
-                                          int B, int Hq, int Hkv, int64_t T, float scale, float* out,
-                                          void* workspace, size_t workspace_bytes, void* stream) {
+                                          int B, int Hq, int Hkv, int64_t T, const int32_t* seq_lens, float scale,
+                                          float* out, void* workspace, size_t workspace_bytes, void* stream) {
   const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
   g_prof_begin = g_prof_end = nullptr;
   return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
-                     k_window, v_window, window_dtype, window_stride, R, B, Hq, Hkv, T, scale, out, workspace,
+                     k_window, v_window, window_dtype, window_stride, R, B, Hq, Hkv, T, seq_lens, scale, out, workspace,
                      workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end);
 }
 
@@ -1265,7 +1309,8 @@ extern "C" int tq_decode_attention_noalloc(const tq_rotation* hk, const tq_rotat
                                            const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
                                            const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
                                            const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv,
-                                           int64_t T, float scale, float* out, void* stream) {
+                                           int64_t T, const int32_t* seq_lens, float scale, float* out,
+                                           void* stream) {
   // the handle and size checks of tq_decode_attention come first, so a call
   // this library cannot serve at all reports that rather than the cap below
   {
@@ -1292,5 +1337,6 @@ extern "C" int tq_decode_attention_noalloc(const tq_rotation* hk, const tq_rotat
     scratch = g_noalloc_scratch_addr[dev];
   }
   return tq_decode_attention(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms,
-                             cache_stride, B, Hq, Hkv, T, scale, out, scratch, kNoAllocScratchBytes, stream);
+                             cache_stride, B, Hq, Hkv, T, seq_lens, scale, out, scratch, kNoAllocScratchBytes,
+                             stream);
 }

@@ -139,6 +139,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t b
                : "memory");
 }
 
+// Untiled bulk copy of `bytes` contiguous bytes (a multiple of 16, both
+// addresses 16-byte aligned) from global memory into this CTA's shared
+// memory, completing its bytes on `mbar`.  Issued by one thread.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(mbar))
+      : "memory");
+}
+
 // Tiled 2-D TMA load of one box at coordinates (c0 innermost, c1) of the
 // tensor map at `map` (a __grid_constant__ kernel parameter) into shared
 // memory, completing its bytes on `mbar`.  c0 times the element size must be a

@@ -47,10 +47,10 @@ def _load():
         "tq_quantize_kv_pair": (c_i, [c_p, c_p, c_p, c_p, c_i, c_i64, c_i64, c_p, c_i64, c_i64, c_i,
                                       c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_p]),
         "tq_decode_attention": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
-                                      c_i64, c_f, c_p, c_p, c_sz, c_p]),
+                                      c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
         "tq_decode_attention_window": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_p, c_p,
-                                             c_i, c_i64, c_i, c_i, c_i, c_i, c_i64, c_f, c_p, c_p, c_sz, c_p]),
+                                             c_i, c_i64, c_i, c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_window_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64, c_i]),
         "tq_profile_next_decode": (c_i, [c_p, c_p]),
         "tq_encoder_attention": (c_i, [c_p, c_p, c_p, c_i, c_i64, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i,
@@ -279,11 +279,23 @@ def alloc_workspace(nbytes: int, device):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
-def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, T: int, *, scale: float | None = None,
-                     out=None, workspace=None, stream=None):
+def _seq_lens(seq_lens, B, device):
+    """Per-sequence lengths as a contiguous int32 device tensor [B], or None."""
+    if seq_lens is None:
+        return None
+    import torch
+    t = torch.as_tensor(seq_lens, dtype=torch.int32, device=device).contiguous()
+    if t.shape != (B,):
+        raise ValueError(f"seq_lens must have shape ({B},)")
+    return t
+
+
+def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, T: int, *, seq_lens=None,
+                     scale: float | None = None, out=None, workspace=None, stream=None):
     """One decode step: q [B, Hq, d] against caches (codes, signs, norms) of
     shape [B, Hkv, cap, ...]; attends to the first T records of each
-    sequence.  Returns out [B, Hq, d] float32."""
+    sequence, or to the first seq_lens[b] (each <= T) of sequence b.
+    Returns out [B, Hq, d] float32."""
     import torch
     B, Hq, d = q.shape
     kc, ks, kn = k_cache
@@ -300,8 +312,9 @@ def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cach
     need = decode_workspace_size(rot_k, rot_v, B, Hq, Hkv, T)
     if workspace is None:
         workspace = alloc_workspace(need, q.device)
+    lens = _seq_lens(seq_lens, B, q.device)
     _check(_lib.tq_decode_attention(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos), _ptr(kc),
-                                    _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, T,
+                                    _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, T, _ptr(lens),
                                     float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream_ptr(stream)), "tq_decode_attention")
     return out
@@ -313,11 +326,13 @@ def decode_window_workspace_size(rot_k: Rotation, rot_v: Rotation, B: int, Hq: i
 
 
 def decode_attention_window(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, T: int, k_window,
-                            v_window, R: int, *, scale: float | None = None, out=None, workspace=None, stream=None):
-    """One decode step over the first T records of the packed caches plus the
-    first R tokens of the full-precision windows k_window, v_window
-    ([B, Hkv, cap_w, d], float32 or bfloat16, keys before RoPE); window token
-    i sits at position T + i.  Returns out [B, Hq, d] float32."""
+                            v_window, R: int, *, seq_lens=None, scale: float | None = None, out=None, workspace=None,
+                            stream=None):
+    """One decode step over the first T records of the packed caches (or
+    seq_lens[b] of sequence b) plus the first R tokens of the full-precision
+    windows k_window, v_window ([B, Hkv, cap_w, d], float32 or bfloat16, keys
+    before RoPE); window token i sits at position T + i (seq_lens[b] + i).
+    Returns out [B, Hq, d] float32."""
     import torch
     B, Hq, d = q.shape
     kc, ks, kn = k_cache
@@ -335,10 +350,11 @@ def decode_attention_window(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache,
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = alloc_workspace(decode_window_workspace_size(rot_k, rot_v, B, Hq, Hkv, T, R), q.device)
+    lens = _seq_lens(seq_lens, B, q.device)
     _check(_lib.tq_decode_attention_window(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos), _ptr(kc),
                                            _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, _ptr(k_window),
                                            _ptr(v_window), _dtype_code(k_window), k_window.shape[2], R, B, Hq, Hkv,
-                                           T, float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                           T, _ptr(lens), float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                            _stream_ptr(stream)), "tq_decode_attention_window")
     return out
 
