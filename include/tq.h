@@ -288,6 +288,23 @@ int tq_search_topk(const tq_rotation* h, const float* queries, int nq,
 size_t tq_search_workspace_size(const tq_rotation* h, int nq, int64_t N, int k);
 
 /*
+ * tq_search_merge_topk - the best k of n_lists candidate lists per query,
+ * e.g. the top-k lists of the database shards of a distributed search
+ * ([TurboQuant] "Performances en recherche vectorielle": brute-force top-k).
+ *   cand_scores, cand_ids  device [n_lists][nq][k] (float32, int64), each
+ *               list best first as tq_search_topk writes them (entries with
+ *               id -1 or score -inf are ignored)
+ *   id_offsets  device [n_lists] int64 added to the ids of each list (the
+ *               shard's first global row), or NULL
+ *   scores, ids device [nq][k] outputs: best first, ties to the lower id,
+ *               -inf / -1 when fewer than k candidates exist
+ * Returns TQ_OK, TQ_EINVAL or TQ_ECUDA.
+ */
+int tq_search_merge_topk(const float* cand_scores, const int64_t* cand_ids,
+                         int n_lists, int nq, int k, const int64_t* id_offsets,
+                         float* scores, int64_t* ids, void* stream);
+
+/*
  * tq_decode_attention - one decode step of attention over packed K/V caches.
  * [TurboESM] §2.E: dequantization, residual correction, inverse rotation
  * Pi^T and an online softmax fused in one pass over the cache;
@@ -372,6 +389,54 @@ int tq_decode_attention_window(const tq_rotation* hk, const tq_rotation* hv,
 size_t tq_decode_window_workspace_size(const tq_rotation* hk,
                                        const tq_rotation* hv, int B, int Hq,
                                        int Hkv, int64_t T, int R);
+
+/*
+ * tq_decode_partials - tq_decode_attention up to, but not including, the
+ * final normalisation: for every query head, the partial record of the
+ * softmax over this call's tokens, so that calls over disjoint token ranges
+ * of the same sequences (e.g. the shards of a long context on several GPUs)
+ * can be combined later by tq_decode_merge_partials.  [TurboESM] §2.E (the
+ * fused pass: online softmax, value accumulation in the rotated space,
+ * Pi^T at the end); the split into partials is the log-sum-exp rule of an
+ * online softmax, which the merge applies exactly.
+ *   hk ... seq_lens, scale  as in tq_decode_attention (the records are the
+ *               caller's shard; positions are those the keys were encoded
+ *               with, and q_pos is the query's own position)
+ *   partials    device out [B*Hq][2 + 2*d] float32: per query head (row
+ *               b*Hq + h) the log2-domain max m of its logits * scale *
+ *               log2(e), the sum l of 2^(logit - m), and the rotated-space
+ *               sums O_code[d] and O_z[d] (value codes and QJL signs, each
+ *               weighted by 2^(logit - m) and the record's norm).  A shard
+ *               without tokens gives m = -inf, l = 0, zeros.
+ *   workspace   as for tq_decode_attention with the same sizes
+ * Returns the statuses of tq_decode_attention.
+ */
+int tq_decode_partials(const tq_rotation* hk, const tq_rotation* hv,
+                       const void* q, int q_dtype, const int64_t* q_pos,
+                       const uint8_t* k_codes, const uint8_t* k_signs,
+                       const float* k_norms, const uint8_t* v_codes,
+                       const uint8_t* v_signs, const float* v_norms,
+                       int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
+                       const int32_t* seq_lens, float scale, float* partials,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * tq_decode_merge_partials - the attention output from n_parts partial
+ * records per query head (tq_decode_partials over disjoint token ranges):
+ * log-sum-exp combination, the QJL value correction sqrt(pi/2)/m S^T O_z and
+ * Pi^T of the value handle, divided by the combined sum.  [TurboESM] §2.E;
+ * [TurboQuant] "QJL".
+ *   hv          value handle (d = 128, Hadamard)
+ *   partials    device [n_parts][B*Hq][2 + 2*d] float32 (part-major, e.g.
+ *               the all-gather of every rank's tq_decode_partials output)
+ *   n_parts     1 .. 65536
+ *   B, Hq, Hkv  as in tq_decode_attention
+ *   out         device [B, Hq, d] float32
+ * Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED or TQ_ECUDA.
+ */
+int tq_decode_merge_partials(const tq_rotation* hv, const float* partials,
+                             int n_parts, int B, int Hq, int Hkv, float* out,
+                             void* stream);
 
 /*
  * tq_encoder_attention - bidirectional attention of S queries per head over

@@ -176,3 +176,71 @@ def decode_attention_window(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache,
             e = np.exp(score - np.max(score))
             out[b, h] = (e / np.sum(e)) @ V
     return out
+
+
+LOG2E = 1.4426950408889634
+
+
+def decode_partials(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, scale: float) -> np.ndarray:
+    """Per query head, the partial record of the softmax over this cache's
+    tokens (a shard of a longer context), [B, Hq, 2 + 2d]:
+      m    = max_t s_t, with s_t = score_t * log2(e) (scores as in
+             decode_attention, scale included),
+      l    = sum_t 2^(s_t - m),
+      A    = sum_t 2^(s_t - m) ||v_t|| c_V[idx^v_t]        (rotated space, d),
+      A_s  = sum_t 2^(s_t - m) ||r^v_t|| (2 z^v_t - 1)     (m entries).
+    An empty cache gives m = -inf, l = 0 and zeros.  The same definitions as
+    decode_attention before its normalisation and inverse rotation
+    ([TurboESM] §2.E)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    kc, kz, kn, kr = _unpack_cache(rot_k, *k_cache)
+    vc, vz, vn, vr = _unpack_cache(rot_v, *v_cache)
+    Hkv, T = kc.shape[1], kc.shape[2]
+    g = Hq // Hkv
+    out = np.zeros((B, Hq, 2 + 2 * rot_v.d))
+    for b in range(B):
+        qr = q[b]
+        if rot_k.rope_base:
+            qr = apply_rope(qr, np.full(Hq, q_pos[b]), rot_k.rope_base)
+        for h in range(Hq):
+            kv = h // g
+            if T == 0:
+                out[b, h, 0] = -np.inf
+                continue
+            qt = qr[h] @ rot_k.pi.T
+            sq = rot_k.s @ qt
+            score = (rot_k.levels[kc[b, kv]] @ qt) * kn[b, kv] \
+                + (np.where(kz[b, kv], 1.0, -1.0) @ sq) * (QJL_CONST / rot_k.m) * kr[b, kv]
+            s2 = score * scale * LOG2E
+            m = np.max(s2)
+            w = np.exp2(s2 - m)
+            out[b, h, 0] = m
+            out[b, h, 1] = np.sum(w)
+            out[b, h, 2:2 + rot_v.d] = (w * vn[b, kv]) @ rot_v.levels[vc[b, kv]]
+            out[b, h, 2 + rot_v.d:] = (w * vr[b, kv]) @ np.where(vz[b, kv], 1.0, -1.0)
+    return out
+
+
+def merge_partials(rot_v: Rotation, parts) -> np.ndarray:
+    """Attention output [B, Hq, d] from partial records [P, B, Hq, 2 + 2d] of
+    disjoint token ranges: with M = max_p m_p and f_p = 2^(m_p - M),
+      out = Pi_V^T (sum_p f_p A_p + sqrt(pi/2)/m S_V^T sum_p f_p A_s,p)
+            / sum_p f_p l_p,
+    zeros when every part is empty."""
+    parts = np.asarray(parts, dtype=np.float64)
+    P, B, Hq, rec = parts.shape
+    d = rot_v.d
+    out = np.zeros((B, Hq, d))
+    for b in range(B):
+        for h in range(Hq):
+            m = parts[:, b, h, 0]
+            if np.all(np.isneginf(m)):
+                continue
+            M = np.max(m)
+            f = np.where(np.isneginf(m), 0.0, np.exp2(m - M))
+            L = np.sum(f * parts[:, b, h, 1])
+            A = f @ parts[:, b, h, 2:2 + d]
+            As = f @ parts[:, b, h, 2 + d:]
+            out[b, h] = ((A + (QJL_CONST / rot_v.m) * (As @ rot_v.s)) / L) @ rot_v.pi
+    return out

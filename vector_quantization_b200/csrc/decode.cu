@@ -700,8 +700,17 @@ __global__ void __launch_bounds__(kD * G) decode_qprep_kernel(const T* __restric
 // shared memory.  The split weights f_s = 2^(m_s - M) of each head are formed
 // by the first warp of its group and staged in shared memory (dynamic,
 // n_splits * G floats), so each thread's sums over splits are plain loads.
-template <int G>
+//
+// Partial records of sequence bh, part s, head h sit at
+// partial + bh * bh_stride + s * part_stride + h * (2 + 2 kD): the split
+// partials of one call, or the partials several calls (e.g. the ranks of a
+// sequence-sharded decode) produced for the same heads.  With FINAL false the
+// kernel stops after the log-sum-exp combination and writes the combined
+// partial record (max, sum of weights, O_code, O_z) of each head to
+// out[(bh G + h) (2 + 2 kD)], for a later merge with other such records.
+template <int G, bool FINAL>
 __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __restrict__ partial, int n_splits,
+                                                             int64_t bh_stride, int64_t part_stride,
                                                              const float* __restrict__ s_mat,
                                                              const float* __restrict__ dsigns, float qjl,
                                                              float* __restrict__ out) {
@@ -710,23 +719,25 @@ __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __res
   __shared__ __align__(16) float oz[G][kD];
   __shared__ __align__(16) float part[G][G][kD];   // [row group][head][i]
   __shared__ __align__(16) float buf[G][kD];
-  __shared__ float Ls[G];
+  __shared__ float Ls[G], Ms[G];
   extern __shared__ float fs[];   // [n_splits][G]
   const int tid = threadIdx.x, h = tid / kD, i = tid % kD, lane = tid & 31;
   const int bh = blockIdx.x;
   float scol[KS];
+  if constexpr (FINAL) {
 #pragma unroll
-  for (int j = 0; j < KS; ++j) scol[j] = __ldg(s_mat + (h * KS + j) * kD + i);
+    for (int j = 0; j < KS; ++j) scol[j] = __ldg(s_mat + (h * KS + j) * kD + i);
+  }
   asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the split kernel's partials
-  const float* base = partial + static_cast<size_t>(bh) * n_splits * G * REC;
+  const float* base = partial + static_cast<size_t>(bh) * bh_stride + static_cast<size_t>(h) * REC;
   if (i < 32) {
     float M = -INFINITY;
-    for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, base[(static_cast<size_t>(s) * G + h) * REC]);
+    for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, base[static_cast<size_t>(s) * part_stride]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float l = 0.f;
     for (int s = lane; s < n_splits; s += 32) {
-      const float* rec = base + (static_cast<size_t>(s) * G + h) * REC;
+      const float* rec = base + static_cast<size_t>(s) * part_stride;
       const float ms = rec[0];
       const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
       fs[s * G + h] = f;
@@ -734,16 +745,29 @@ __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __res
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) Ls[h] = l;
+    if (lane == 0) {
+      Ls[h] = l;
+      Ms[h] = M;
+    }
   }
   __syncthreads();
   float c = 0.f, z = 0.f;
 #pragma unroll 4
   for (int s = 0; s < n_splits; ++s) {
     const float f = fs[s * G + h];
-    const float* rec = base + (static_cast<size_t>(s) * G + h) * REC;
+    const float* rec = base + static_cast<size_t>(s) * part_stride;
     c = fmaf(f, rec[2 + i], c);
     z = fmaf(f, rec[2 + kD + i], z);
+  }
+  if constexpr (!FINAL) {
+    float* dst = out + (static_cast<size_t>(bh) * G + h) * REC;
+    if (i == 0) {
+      dst[0] = Ms[h];
+      dst[1] = Ls[h];
+    }
+    dst[2 + i] = c;
+    dst[2 + kD + i] = z;
+    return;
   }
   oz[h][i] = z;
   __syncthreads();
@@ -760,7 +784,7 @@ __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __res
 #pragma unroll
   for (int g = 0; g < G; ++g) corr += part[g][h][i];
   // rotated-space value: O_code + sqrt(pi/2)/m S^T O_z, then Pi^T y = D H y / sqrt(d)
-  float y = Ls[h] > 0.f ? (c + qjl * corr) / Ls[h] : 0.f;
+  float y = Ls[h] != 0.f ? (c + qjl * corr) / Ls[h] : 0.f;   // a NaN sum (a failed part) stays NaN
   fwht_group(y, i, buf[h]);
   out[(static_cast<size_t>(bh) * G + h) * kD + i] = y * (dsigns[i] * rsqrtf(static_cast<float>(kD)));
 }
@@ -1082,17 +1106,26 @@ int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64
   return TQ_OK;
 }
 
-int launch_merge(int G, int BH, const float* partial, int n_splits, const tq_rotation* hv, float* out, cudaStream_t s) {
+// Merge of n_parts partial records per head (layout: see decode_merge_kernel).
+// final_out: the attention output [BH G][kD]; otherwise the combined partial
+// records [BH G][2 + 2 kD].
+int launch_merge(int G, int BH, const float* partial, int n_parts, int64_t bh_stride, int64_t part_stride,
+                 const tq_rotation* hv, float* out, bool final_out, cudaStream_t s) {
   const float qjl = static_cast<float>(kQjlConst / hv->m);
-  const size_t fsb = static_cast<size_t>(n_splits) * G * sizeof(float);   // <= (1184 + 32) * 8 * 4 bytes
+  const size_t fsb = static_cast<size_t>(n_parts) * G * sizeof(float);
+#define TQ_MERGE(GG)                                                                                                \
+  return final_out ? launch_pdl(decode_merge_kernel<GG, true>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts,  \
+                                bh_stride, part_stride, hv->d_s, hv->d_signs, qjl, out)                             \
+                   : launch_pdl(decode_merge_kernel<GG, false>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts, \
+                                bh_stride, part_stride, hv->d_s, hv->d_signs, qjl, out)
   switch (G) {
-    case 1: return launch_pdl(decode_merge_kernel<1>, dim3(BH), dim3(kD * 1), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
-    case 2: return launch_pdl(decode_merge_kernel<2>, dim3(BH), dim3(kD * 2), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
-    case 4: return launch_pdl(decode_merge_kernel<4>, dim3(BH), dim3(kD * 4), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
-    case 8: return launch_pdl(decode_merge_kernel<8>, dim3(BH), dim3(kD * 8), fsb, s, partial, n_splits, hv->d_s, hv->d_signs, qjl, out);
+    case 1: TQ_MERGE(1);
+    case 2: TQ_MERGE(2);
+    case 4: TQ_MERGE(4);
+    case 8: TQ_MERGE(8);
     default: return TQ_EUNSUPPORTED;
   }
-  return tq::launch_status();
+#undef TQ_MERGE
 }
 
 template <int BITS>
@@ -1155,14 +1188,14 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
                 const uint8_t* k_codes, const uint8_t* k_signs, const float* k_norms, const uint8_t* v_codes,
                 const uint8_t* v_signs, const float* v_norms, int64_t cache_stride, const void* k_win,
                 const void* v_win, int win_dtype, int64_t win_stride, int R, int B, int Hq, int Hkv, int64_t T,
-                const int32_t* seq_lens, float scale, float* out, void* workspace, size_t workspace_bytes,
-                cudaStream_t s,
+                const int32_t* seq_lens, float scale, float* out, float* partial_out, void* workspace,
+                size_t workspace_bytes, cudaStream_t s,
                 cudaEvent_t prof_begin, cudaEvent_t prof_end) {
   {
     const int st = check_decode_sizes(hk, hv, B, Hq, Hkv, T);
     if (st != TQ_OK) return st;
   }
-  if (!q || !out) return TQ_EINVAL;
+  if (!q || (!out && !partial_out)) return TQ_EINVAL;
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_EINVAL;
   if (!std::isfinite(scale)) return TQ_EINVAL;
   const int G = Hq / Hkv;
@@ -1242,7 +1275,9 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   }
   if (st != TQ_OK) return st;
   if (prof_end && cudaEventRecord(prof_end, s) != cudaSuccess) return TQ_ECUDA;
-  return launch_merge(G, BH, partial, n_slots, hv, out, s);
+  const int64_t rec = 2 + 2 * kD;
+  return launch_merge(G, BH, partial, n_slots, static_cast<int64_t>(n_slots) * G * rec, G * rec, hv,
+                      partial_out ? partial_out : out, partial_out == nullptr, s);
 }
 
 }  // namespace
@@ -1268,7 +1303,8 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
   const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
   g_prof_begin = g_prof_end = nullptr;
   return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
-                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, workspace, workspace_bytes,
+                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, nullptr, workspace,
+                     workspace_bytes,
                      static_cast<cudaStream_t>(stream), prof_begin, prof_end);
 }
 
@@ -1282,8 +1318,36 @@ extern "C" int tq_decode_attention_window(const tq_rotation* hk, const tq_rotati
   const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
   g_prof_begin = g_prof_end = nullptr;
   return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
-                     k_window, v_window, window_dtype, window_stride, R, B, Hq, Hkv, T, seq_lens, scale, out, workspace,
-                     workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end);
+                     k_window, v_window, window_dtype, window_stride, R, B, Hq, Hkv, T, seq_lens, scale, out, nullptr,
+                     workspace, workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end);
+}
+
+extern "C" int tq_decode_partials(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
+                                  const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
+                                  const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
+                                  const float* v_norms, int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
+                                  const int32_t* seq_lens, float scale, float* partials, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!partials) return TQ_EINVAL;
+  return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
+                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, nullptr, partials, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+extern "C" int tq_decode_merge_partials(const tq_rotation* hv, const float* partials, int n_parts, int B, int Hq,
+                                        int Hkv, float* out, void* stream) {
+  if (!hv || !partials || !out || n_parts < 1 || n_parts > (1 << 16)) return TQ_EINVAL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv) return TQ_EINVAL;
+  if (static_cast<int64_t>(B) * Hkv > kMaxSequences) return TQ_EUNSUPPORTED;
+  if (hv->d != kD || hv->m != kD || hv->kind != TQ_ROT_HADAMARD) return TQ_EUNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_EUNSUPPORTED;
+  if (!tq::on_handle_device(hv)) return TQ_EINVAL;
+  const int BH = B * Hkv;
+  const int64_t rec = 2 + 2 * kD;
+  const int st = launch_merge(G, BH, partials, n_parts, G * rec, static_cast<int64_t>(BH) * G * rec, hv, out, true,
+                              static_cast<cudaStream_t>(stream));
+  return st != TQ_OK ? st : tq::launch_status();
 }
 
 // ---------------------------------------------------------------------------

@@ -250,8 +250,12 @@ __global__ void __launch_bounds__(kSWarps * 32) search_score_kernel(SearchParams
 }
 
 // One warp per query: merge the candidate lists of all ranges.
+// One warp per query: the best k of n_ranges candidate lists [n_ranges][nq][k]
+// (descending score, ties to the lower id); list r's ids are shifted by
+// id_offsets[r] when id_offsets is given (lists of database shards).
 __global__ void search_merge_kernel(const float* __restrict__ cs, const int64_t* __restrict__ ci, int n_ranges, int nq,
-                                    int k, float* __restrict__ scores, int64_t* __restrict__ ids) {
+                                    int k, const int64_t* __restrict__ id_offsets, float* __restrict__ scores,
+                                    int64_t* __restrict__ ids) {
   const int lane = threadIdx.x & 31;
   const int q = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (q >= nq) return;
@@ -260,7 +264,8 @@ __global__ void search_merge_kernel(const float* __restrict__ cs, const int64_t*
   for (int r = 0; r < n_ranges; ++r) {
     const size_t base = (static_cast<size_t>(r) * nq + q) * k;
     const float s = lane < k ? cs[base + lane] : -INFINITY;
-    const int64_t id = lane < k ? ci[base + lane] : -1;
+    int64_t id = lane < k ? ci[base + lane] : -1;
+    if (id_offsets && id >= 0) id += id_offsets[r];
     unsigned cand = __ballot_sync(0xffffffffu, id >= 0 && s != -INFINITY);
     while (cand) {
       const int src = __ffs(cand) - 1;
@@ -444,6 +449,14 @@ extern "C" int tq_search_topk(const tq_rotation* h, const float* queries, int nq
     default: st = launch_score<3>(p, sp, s); break;
   }
   if (st != TQ_OK) return st;
-  search_merge_kernel<<<(nq + 7) / 8, 256, 0, s>>>(p.cand_score, p.cand_id, sp.n_ranges, nq, k, scores, ids);
+  search_merge_kernel<<<(nq + 7) / 8, 256, 0, s>>>(p.cand_score, p.cand_id, sp.n_ranges, nq, k, nullptr, scores, ids);
+  return tq::launch_status();
+}
+
+extern "C" int tq_search_merge_topk(const float* cand_scores, const int64_t* cand_ids, int n_lists, int nq, int k,
+                                    const int64_t* id_offsets, float* scores, int64_t* ids, void* stream) {
+  if (!cand_scores || !cand_ids || !scores || !ids || n_lists < 1 || nq < 1 || k < 1 || k > kMaxK) return TQ_EINVAL;
+  search_merge_kernel<<<(nq + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(cand_scores, cand_ids, n_lists, nq,
+                                                                                    k, id_offsets, scores, ids);
   return tq::launch_status();
 }

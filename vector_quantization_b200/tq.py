@@ -49,6 +49,10 @@ def _load():
         "tq_decode_attention": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
                                       c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
+        "tq_decode_partials": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
+                                     c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
+        "tq_decode_merge_partials": (c_i, [c_p, c_p, c_i, c_i, c_i, c_i, c_p, c_p]),
+        "tq_search_merge_topk": (c_i, [c_p, c_p, c_i, c_i, c_i, c_p, c_p, c_p, c_p]),
         "tq_decode_attention_window": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_p, c_p,
                                              c_i, c_i64, c_i, c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_window_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64, c_i]),
@@ -318,6 +322,65 @@ def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cach
                                     float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream_ptr(stream)), "tq_decode_attention")
     return out
+
+
+def decode_partials(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, T: int, *, seq_lens=None,
+                    scale: float | None = None, out=None, workspace=None, stream=None):
+    """Partial softmax records of one decode step over this call's tokens:
+    returns [B, Hq, 2 + 2 d] float32 (max, sum, O_code[d], O_z[d] per query
+    head), to be combined with other token ranges by decode_merge_partials."""
+    import torch
+    B, Hq, d = q.shape
+    kc, ks, kn = k_cache
+    vc, vs, vn = v_cache
+    Hkv, cap = kc.shape[1], kc.shape[2]
+    for t in (kc, ks, kn, vc, vs, vn):
+        if not t.is_contiguous():
+            raise ValueError("cache arrays must be contiguous")
+    q = q.contiguous()
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((B, Hq, 2 + 2 * d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_size(rot_k, rot_v, B, Hq, Hkv, T), q.device)
+    lens = _seq_lens(seq_lens, B, q.device)
+    _check(_lib.tq_decode_partials(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos), _ptr(kc),
+                                   _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, T, _ptr(lens),
+                                   float(scale), _ptr(out), _ptr(workspace), workspace.numel(), _stream_ptr(stream)),
+           "tq_decode_partials")
+    return out
+
+
+def decode_merge_partials(rot_v: Rotation, partials, Hkv: int, *, out=None, stream=None):
+    """Attention output [B, Hq, d] from partial records [P, B, Hq, 2 + 2 d]."""
+    import torch
+    P, B, Hq, rec = partials.shape
+    d = (rec - 2) // 2
+    partials = partials.contiguous()
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=partials.device)
+    _check(_lib.tq_decode_merge_partials(rot_v.handle, _ptr(partials), P, B, Hq, Hkv, _ptr(out), _stream_ptr(stream)),
+           "tq_decode_merge_partials")
+    return out
+
+
+def search_merge_topk(cand_scores, cand_ids, k: int, *, id_offsets=None, stream=None):
+    """Best k of L candidate lists per query: cand_scores [L, nq, k] float32,
+    cand_ids [L, nq, k] int64, id_offsets [L] int64 or None.  Returns
+    (scores [nq, k], ids [nq, k])."""
+    import torch
+    L, nq, kk = cand_scores.shape
+    if kk != k or cand_ids.shape != cand_scores.shape:
+        raise ValueError("candidate lists must be [L, nq, k]")
+    cs, ci = cand_scores.contiguous(), cand_ids.contiguous()
+    offs = None if id_offsets is None else torch.as_tensor(id_offsets, dtype=torch.int64,
+                                                          device=cs.device).contiguous()
+    scores = torch.empty((nq, k), dtype=torch.float32, device=cs.device)
+    ids = torch.empty((nq, k), dtype=torch.int64, device=cs.device)
+    _check(_lib.tq_search_merge_topk(_ptr(cs), _ptr(ci), L, nq, k, _ptr(offs), _ptr(scores), _ptr(ids),
+                                     _stream_ptr(stream)), "tq_search_merge_topk")
+    return scores, ids
 
 
 def decode_window_workspace_size(rot_k: Rotation, rot_v: Rotation, B: int, Hq: int, Hkv: int, T: int,
