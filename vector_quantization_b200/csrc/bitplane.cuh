@@ -42,6 +42,31 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], u
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D += A B, m16n8k32, A unsigned 8-bit, B signed 8-bit, int32 accumulate
+// (exact).  Fragments: a0/a1 rows g/g+8 at K 4t..4t+3, a2/a3 the same rows at
+// K 16+4t..; b0 K 4t.., b1 K 16+4t.. of column g; c0,c1 row g columns 2t,
+// 2t+1 and c2,c3 row g+8 (g = lane / 4, t = lane % 4).
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// An int32 of magnitude below 2^22 as float, exactly: adding it to the bit
+// pattern of 1.5 * 2^23 places it in the mantissa (integer add + one FADD).
+__device__ __forceinline__ float small_int_to_float(int x) {
+  return __int_as_float(x + 0x4B400000) - 12582912.0f;
+}
+
+// d0 + 2^8 d1 + 2^16 d2 + 2^24 d3 in fp32 for four digit sums below 2^22.
+__device__ __forceinline__ float digits_to_float(int d0, int d1, int d2, int d3) {
+  float f = small_int_to_float(d3);
+  f = fmaf(f, 256.f, small_int_to_float(d2));
+  f = fmaf(f, 256.f, small_int_to_float(d1));
+  return fmaf(f, 256.f, small_int_to_float(d0));
+}
+
 // Two bf16 values +-1 from bits x (low half) and x+16 (high half) of w:
 // bit = 1 -> +1.0, bit = 0 -> -1.0 (one shift and one LOP3).
 __device__ __forceinline__ uint32_t pm1_pair(uint32_t w, int x) {

@@ -61,8 +61,8 @@ struct DecodeParams {
   int64_t chunk;           // tokens per split (multiple of kTile)
   int n_splits;
   int n_slots;             // partial records per head: n_splits, then one per window chunk
-  const uint32_t* qfrag;   // [BH][2][NT][8][32][2]
-  const float2* kconst;    // [BH][2][8]: (sum_k mu_k B_k, 1 / fp16 range scale)
+  const uint32_t* qfrag;   // [BH][MG][2 NT][32][2]: int8 digits of the key-side B operand
+  const float4* kconst;    // [BH][8]: (2^-E code, code constant, 2^-E sign, sign constant) per head
   float* partial;          // [BH][n_slots][G][2 + 2 kD]
   float score_scale;       // softmax scale * log2(e)
   float qjl;               // sqrt(pi/2) / m
@@ -76,6 +76,25 @@ struct DecodeParams {
 // Polls of a stage's mbarrier before the warp gives up on its copies (about a
 // second); the warp then reports NaN for its heads instead of hanging.
 constexpr int kCopyWaitPolls = 1 << 17;
+
+// Key-side MMA groups of the split kernel (m16n8k32, u8 bits x s8 query
+// digits).  A group covers 32 K elements per 16 tokens: with two Walsh planes
+// a group takes byte position j (0..7) of one 32-coordinate word of each
+// plane (one AND each: bits j, j+8, j+16, j+24 at weight 2^j); a single
+// plane (1-bit codes, the sign plane) takes nibble position j (0..3) of the
+// word and of the word shifted right by four.  CODE groups for the code
+// planes, SIGN for the QJL signs.
+template <int BITS>
+struct KeyGroups {
+  static constexpr int P = Planes<BITS>::P;            // Walsh planes
+  static constexpr int CODE = BITS == 1 ? 4 : 8 * (P / 2);
+  static constexpr int SIGN = 4;
+  static constexpr int MG = CODE + SIGN;
+};
+
+struct WalshWeights {
+  float w[4];
+};
 
 // Shared-memory position of the 16-byte chunk `part` (code plane) of token
 // `tok`'s codes: the records as they lie in the cache, one bulk copy per
@@ -161,35 +180,22 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   for (int i = 0; i < issued; ++i) issue(i);
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
-  // The query B fragments: in registers for one n-tile (G <= 4); in shared
-  // memory for two (G = 8), read at each MMA, which frees the registers the
-  // pipelined loop needs there.
-  uint32_t qf[2][1][8][2];   // used for NT == 1 only (the compiler drops it otherwise)
-  __shared__ uint2 s_qf[2][NT][8][NT == 1 ? 1 : 32];   // a stub for NT == 1
-  float2 kc[2][NT];
+  // The key side's B operand (int8 digits of the query, one set of
+  // fragments per MMA group and n-tile) in shared memory, read at each MMA;
+  // the per-head scales and constants in registers.
+  constexpr int MG = KeyGroups<BITS>::MG;
+  constexpr int NTK = 2 * NT;
+  __shared__ uint2 s_qf[MG][NTK][32];
+  float4 kc[NT];
   {
-    const uint32_t* src = p.qfrag + static_cast<size_t>(bh) * (2 * NT * 8 * 32 * 2);
-    if constexpr (NT == 1) {
+    const uint2* src = reinterpret_cast<const uint2*>(p.qfrag) + static_cast<size_t>(bh) * (MG * NTK * 32);
+    for (int i = threadIdx.x; i < MG * NTK * 32; i += blockDim.x) (&s_qf[0][0][0])[i] = src[i];
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int kb = 0; kb < 8; ++kb) {
-          const uint2 v = *reinterpret_cast<const uint2*>(src + ((t * 8 + kb) * 32 + lane) * 2);
-          qf[t][0][kb][0] = v.x;
-          qf[t][0][kb][1] = v.y;
-        }
-    } else {
-      for (int i = threadIdx.x; i < 2 * NT * 8 * 32; i += blockDim.x)
-        (&s_qf[0][0][0][0])[i] = reinterpret_cast<const uint2*>(src)[i];
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h = tig + 4 * nt;
+      kc[nt] = h < G ? p.kconst[static_cast<size_t>(bh) * 8 + h] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-#pragma unroll
-    for (int t = 0; t < 2; ++t)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int h = tig + 4 * nt;
-        kc[t][nt] = h < G ? p.kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] : make_float2(0.f, 0.f);
-      }
-    if constexpr (NT != 1) __syncthreads();
+    __syncthreads();
   }
   float accC[NT][8][4], accZ[NT][8][4];
   float m_run[NT], l_run[NT];
@@ -206,12 +212,17 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   }
   const float piece_m = (gid & 1) ? 1.f : 0.f;   // this lane feeds the hi (0) or lo (1) piece
   const uint32_t half_sel = (gid & 1) ? 0x7632u : 0x5410u;
-  // ---- K side of one tile: logits of tokens gid, gid + 8 for head tig + 4 nt
+  // ---- K side of one tile: logits of tokens gid, gid + 8 for head tig + 4 nt.
+  // m16n8k32 u8 x s8 products into int32: rows are the 16 tokens, K runs over
+  // (plane, coordinate) slots, the columns are (head, digit); each A register
+  // is one AND of a plane word (see KeyGroups), so every product is exact and
+  // the four digit columns of a head recombine in fp32 (each column stays
+  // below 2^22 in magnitude, where the float conversion is exact).
   auto k_side = [&](const uint8_t* stg, int nv, float (&logit)[NT][2]) {
     const uint8_t* kcd = stg;
     const uint32_t* ks = reinterpret_cast<const uint32_t*>(stg + kTile * CB);
     const float2* kn = reinterpret_cast<const float2*>(stg + kTile * (CB + SB));
-    uint32_t wk[2][P + 1], ws[2][P + 1];
+    uint32_t wk[2][P], wz[2];
     float2 knorm[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -220,90 +231,67 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
 #pragma unroll
       for (int k = 0; k < BITS; ++k)
         raw[k] = reinterpret_cast<const uint32_t*>(kcd + code_chunk<BITS>(tok, k) * 16)[tig];
-      uint32_t pl[P];
-      Planes<BITS>::make(raw, pl);
-#pragma unroll
-      for (int q = 0; q < P; ++q) wk[e][q] = pl[q];
-      wk[e][P] = ks[tok * (SB / 4) + tig];
+      Planes<BITS>::make(raw, wk[e]);
+      wz[e] = ks[tok * (SB / 4) + tig];
       knorm[e] = kn[tok];
-#pragma unroll
-      for (int q = 0; q <= P; ++q) ws[e][q] = wk[e][q] << 8;
     }
-    float code[NT][2], zsc[NT][2];
-    if constexpr (NT == 1) {
-      // one accumulator per plane; planes interleaved per k-block (three
-      // independent tensor-core chains)
-      float c[P + 1][NT][4];
+    int accc[NTK][4], accs[NTK][4];
 #pragma unroll
-      for (int pl = 0; pl <= P; ++pl)
+    for (int n = 0; n < NTK; ++n)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) c[pl][nt][0] = c[pl][nt][1] = c[pl][nt][2] = c[pl][nt][3] = 0.f;
+      for (int r = 0; r < 4; ++r) accc[n][r] = accs[n][r] = 0;
+    if constexpr (BITS == 1) {
+      const uint32_t w4[2] = {wk[0][0] >> 4, wk[1][0] >> 4};
 #pragma unroll
-      for (int kb = 0; kb < 8; ++kb) {
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t M = 0x01010101u << j;
+        const uint32_t a[4] = {wk[0][0] & M, wk[1][0] & M, w4[0] & M, w4[1] & M};
 #pragma unroll
-        for (int pl = 0; pl <= P; ++pl) {
-          const int type = pl < P ? 0 : 1;
-          const uint32_t a[4] = {bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb, one_h),
-                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb, one_h),
-                                 bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb + 1, one_h),
-                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb + 1, one_h)};
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_f16(c[pl][nt], a, qf[type][nt][kb][0], qf[type][nt][kb][1]);
+        for (int n = 0; n < NTK; ++n) {
+          const uint2 b = s_qf[j][n][lane];
+          mma_u8s8(accc[n], a, b.x, b.y);
         }
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        code[nt][0] = code[nt][1] = 0.f;
-#pragma unroll
-        for (int pl = 0; pl < P; ++pl) {
-          code[nt][0] = fmaf(p.walsh_k[pl], (c[pl][nt][0] + c[pl][nt][1] - kc[0][nt].x) * kc[0][nt].y, code[nt][0]);
-          code[nt][1] = fmaf(p.walsh_k[pl], (c[pl][nt][2] + c[pl][nt][3] - kc[0][nt].x) * kc[0][nt].y, code[nt][1]);
-        }
-        zsc[nt][0] = (c[P][nt][0] + c[P][nt][1] - kc[1][nt].x) * kc[1][nt].y;
-        zsc[nt][1] = (c[P][nt][2] + c[P][nt][3] - kc[1][nt].x) * kc[1][nt].y;
       }
     } else {
-      // two n-tiles (G = 8): planes one after the other, one accumulator set
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) code[nt][0] = code[nt][1] = 0.f;
+      for (int pr = 0; pr < P / 2; ++pr)
 #pragma unroll
-      for (int pl = 0; pl <= P; ++pl) {
-        const int type = pl < P ? 0 : 1;
-        float c[NT][4];
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t M = 0x01010101u << j;
+          const uint32_t a[4] = {wk[0][2 * pr] & M, wk[1][2 * pr] & M, wk[0][2 * pr + 1] & M, wk[1][2 * pr + 1] & M};
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
-#pragma unroll
-        for (int kb = 0; kb < 8; ++kb) {
-          const uint32_t a[4] = {bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb, one_h),
-                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb, one_h),
-                                 bit_pair_h(wk[0][pl], ws[0][pl], 2 * kb + 1, one_h),
-                                 bit_pair_h(wk[1][pl], ws[1][pl], 2 * kb + 1, one_h)};
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint2 qb = s_qf[type][nt][kb][lane];
-            mma_f16(c[nt], a, qb.x, qb.y);
+          for (int n = 0; n < NTK; ++n) {
+            const uint2 b = s_qf[pr * 8 + j][n][lane];
+            mma_u8s8(accc[n], a, b.x, b.y);
           }
         }
+    }
+    {
+      const uint32_t z4[2] = {wz[0] >> 4, wz[1] >> 4};
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const float s0v = (c[nt][0] + c[nt][1] - kc[type][nt].x) * kc[type][nt].y;
-          const float s1v = (c[nt][2] + c[nt][3] - kc[type][nt].x) * kc[type][nt].y;
-          if (pl < P) {
-            code[nt][0] = fmaf(p.walsh_k[pl < P ? pl : 0], s0v, code[nt][0]);
-            code[nt][1] = fmaf(p.walsh_k[pl < P ? pl : 0], s1v, code[nt][1]);
-          } else {
-            zsc[nt][0] = s0v;
-            zsc[nt][1] = s1v;
-          }
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t M = 0x01010101u << j;
+        const uint32_t a[4] = {wz[0] & M, wz[1] & M, z4[0] & M, z4[1] & M};
+#pragma unroll
+        for (int n = 0; n < NTK; ++n) {
+          const uint2 b = s_qf[KeyGroups<BITS>::CODE + j][n][lane];
+          mma_u8s8(accs[n], a, b.x, b.y);
         }
       }
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const float l0 = fmaf(knorm[0].x, code[nt][0], knorm[0].y * p.qjl * zsc[nt][0]) * p.score_scale;
-      const float l1 = fmaf(knorm[1].x, code[nt][1], knorm[1].y * p.qjl * zsc[nt][1]) * p.score_scale;
-      logit[nt][0] = gid < nv ? l0 : -INFINITY;
-      logit[nt][1] = gid + 8 < nv ? l1 : -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float code = fmaf(digits_to_float(accc[2 * nt][2 * e], accc[2 * nt][2 * e + 1],
+                                                accc[2 * nt + 1][2 * e], accc[2 * nt + 1][2 * e + 1]),
+                                kc[nt].x, -kc[nt].y);
+        const float sgn = fmaf(digits_to_float(accs[2 * nt][2 * e], accs[2 * nt][2 * e + 1],
+                                               accs[2 * nt + 1][2 * e], accs[2 * nt + 1][2 * e + 1]),
+                               kc[nt].z, -kc[nt].w);
+        const float l = fmaf(knorm[e].x, code, knorm[e].y * p.qjl * sgn) * p.score_scale;
+        logit[nt][e] = gid + 8 * e < nv ? l : -INFINITY;
+      }
     }
   };
   // 2^x of the softmax: the hardware approximation for 1- and 2-bit codes; the
@@ -571,20 +559,20 @@ __device__ __forceinline__ void fwht_group(float& v, int i, float* buf) {
 
 // One block of G groups of kD threads per (sequence b, KV head); group h is
 // query head h of the group, thread i of it coordinate i: RoPE, q~ = Pi q,
-// s = S q~, then the fp16 B fragments of the split kernel.  The product S q~
+// s = S q~, then the int8 B fragments of the split kernel's key side.  The product S q~
 // is split by columns of S instead of by heads: group g holds columns
 // [g kD/G, (g + 1) kD/G) of row i of S in registers (loaded before the wait
 // for q, so the loads overlap the previous launch) and forms the partial sums
 // of all G heads over them; the G partials meet in shared memory.
-template <typename T, int G>
+template <typename T, int G, int BITS>
 __global__ void __launch_bounds__(kD * G) decode_qprep_kernel(const T* __restrict__ q, const int64_t* __restrict__ q_pos,
                                                              int Hkv, const float* __restrict__ dsigns,
                                                              const float* __restrict__ st,
                                                              const float2* __restrict__ rope_hi,
                                                              const float2* __restrict__ rope_lo, int64_t rope_max_pos,
-                                                             int rope, uint16_t* __restrict__ qfrag,
-                                                             float2* __restrict__ kconst) {
-  constexpr int NT = (2 * G + 7) / 8;
+                                                             int rope, WalshWeights walsh, uint32_t* __restrict__ qfrag,
+                                                             float4* __restrict__ kconst) {
+  constexpr int NT = (G + 3) / 4;
   constexpr int KS = kD / G;   // columns of S per group
   __shared__ __align__(16) float buf[G][kD];
   __shared__ __align__(16) float part[G][G][kD];   // [column group][head][i]
@@ -638,55 +626,84 @@ __global__ void __launch_bounds__(kD * G) decode_qprep_kernel(const T* __restric
 #pragma unroll
   for (int g = 0; g < G; ++g) sv += part[g][h][i];
 
-  // Scatter into the B-fragment layout of the split kernel.  Dim i sits in
-  // pair slot j = i & 15 of the word of lane-column tg = i / 32; that slot's
-  // half-word position fixes (mu_p, sigma_p) of the fp16 bit operand.  The
-  // value x / sigma_p is scaled by a per-head power of two into fp16 range
-  // and split into hi/lo fp16 pieces (columns n = 2 (head % 4) + piece of
-  // n-tile head / 4).  Columns of absent heads (G < 4) are zero.
-  const int tg = i >> 5, x = i & 31, e = x >> 4, j = x & 15, reg = j & 1, kb = j >> 1;
-  const int pp = slot_pos(j);
-  const float mu = 0.5f * (pos_v0_h(pp) + pos_v1_h(pp)), inv_sigma = 2.f / (pos_v1_h(pp) - pos_v0_h(pp));
-  auto frag_at = [&](int type, int nt, int n) {
-    return ((((static_cast<size_t>(bh) * 2 + type) * NT + nt) * 8 + kb) * 32 + 4 * n + tg) * 4 + reg * 2 + e;
-  };
-  const float val[2] = {v * inv_sigma, sv * inv_sigma};
+  // Scatter into the int8 B fragments of the split kernel's key side.  The
+  // key operand holds bit b of a plane at weight 2^j (j its position inside
+  // its byte, or inside its nibble for the single-plane groups), so the value
+  // that multiplies it is x 2^E / 2^j, x = 2 w_p q~_i for Walsh plane p and
+  // x = 2 (S q~)_i for the sign plane (a 0/1 bit b stands for 2b - 1); E puts
+  // max |x| just below 2^30, and the rounded value is cut into four balanced
+  // signed bytes (digits).  Digit d of head h is column 2 (h % 4) + (d % 2) of
+  // n-tile 2 (h / 4) + d / 2, so thread t of the split kernel holds all four
+  // digits of head t (+ 4 per head group).
+  constexpr int NTK = 2 * NT;
+  constexpr int MG = KeyGroups<BITS>::MG;
+  const int t = i >> 5, e = (i >> 3) & 3, j8 = i & 7;
+  float mx[2] = {fabsf(v), fabsf(sv)};
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    float mx = fabsf(val[t]);
+  for (int ty = 0; ty < 2; ++ty) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) red[0][h][t][wg] = mx;
+    for (int o = 16; o > 0; o >>= 1) mx[ty] = fmaxf(mx[ty], __shfl_xor_sync(0xffffffffu, mx[ty], o));
+    if (lane == 0) red[0][h][ty][wg] = mx[ty];
+  }
+  float csum = v, ssum = sv;   // sums over coordinates of q~ and S q~
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    csum += __shfl_xor_sync(0xffffffffu, csum, o);
+    ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+  }
+  if (lane == 0) {
+    red[1][h][0][wg] = csum;
+    red[1][h][1][wg] = ssum;
   }
   __syncthreads();
-  float lam[2];
+  float wmax = 0.f, wsum = 0.f;
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const float mx = fmaxf(fmaxf(red[0][h][t][0], red[0][h][t][1]), fmaxf(red[0][h][t][2], red[0][h][t][3]));
-    lam[t] = fp16_range_scale(mx);
-    const float x2 = val[t] * lam[t];
-    const __half hi = __float2half_rn(x2);
-    const __half lo = __float2half_rn(x2 - __half2float(hi));
-    const int n = 2 * (h & 3);
-    qfrag[frag_at(t, h >> 2, n)] = __half_as_ushort(hi);
-    qfrag[frag_at(t, h >> 2, n + 1)] = __half_as_ushort(lo);
-    float c = mu * (__half2float(hi) + __half2float(lo));   // sum over dims of mu_p (hi + lo)
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    if (lane == 0) red[1][h][t][wg] = c;
+  for (int pl = 0; pl < KeyGroups<BITS>::P; ++pl) {
+    wmax = fmaxf(wmax, fabsf(walsh.w[pl]));
+    wsum += walsh.w[pl];
   }
-  if constexpr (2 * G < 8) {
-    if (h == 0) {
+  int E[2];
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
-        for (int n = 2 * G; n < 8; ++n) qfrag[frag_at(t, 0, n)] = 0;
+  for (int ty = 0; ty < 2; ++ty) {
+    const float m = fmaxf(fmaxf(red[0][h][ty][0], red[0][h][ty][1]), fmaxf(red[0][h][ty][2], red[0][h][ty][3])) *
+                    (ty == 0 ? 2.f * wmax : 2.f);
+    int ex = 0;
+    if (m > 0.f && isfinite(m)) frexpf(m, &ex);   // m in [2^(ex-1), 2^ex)
+    E[ty] = m > 0.f && isfinite(m) ? 30 - ex : 0;
+  }
+  uint8_t* frag = reinterpret_cast<uint8_t*>(qfrag);
+  auto put = [&](int mg, int reg, int jj, float x, int ty) {
+    // round(x 2^E / 2^jj), then four balanced digits
+    int V = __float2int_rn(ldexpf(x, E[ty] - jj));
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+      const int dg = ((V + 128) & 0xFF) - 128;
+      V = (V - dg) >> 8;
+      const int ntk = 2 * (h >> 2) + (d >> 1), g = 2 * (h & 3) + (d & 1);
+      frag[((((static_cast<size_t>(bh) * MG + mg) * NTK + ntk) * 32 + 4 * g + t) * 2 + reg) * 4 + e] =
+          static_cast<uint8_t>(dg);
+    }
+  };
+  if constexpr (BITS == 1) {
+    put(j8 & 3, j8 >> 2, j8 & 3, 2.f * walsh.w[0] * v, 0);
+  } else {
+#pragma unroll
+    for (int pl = 0; pl < KeyGroups<BITS>::P; ++pl) put((pl >> 1) * 8 + j8, pl & 1, j8, 2.f * walsh.w[pl] * v, 0);
+  }
+  put(KeyGroups<BITS>::CODE + (j8 & 3), j8 >> 2, j8 & 3, 2.f * sv, 1);
+  if constexpr (G < 4) {
+    // columns of the absent heads of the first head group are zero
+    for (int idx = tid; idx < MG * 2 * 32 * 2 * 4; idx += blockDim.x) {
+      const int by = idx & 3, reg = (idx >> 2) & 1, ln = (idx >> 3) & 31, rest = idx >> 8;
+      const int ntk = rest & 1, mg = rest >> 1;
+      if ((ln >> 2) >= 2 * G)
+        frag[((((static_cast<size_t>(bh) * MG + mg) * NTK + ntk) * 32 + ln) * 2 + reg) * 4 + by] = 0;
     }
   }
-  __syncthreads();
-  if (i < 2) {
-    const int t = i;
-    const float c = (red[1][h][t][0] + red[1][h][t][1]) + (red[1][h][t][2] + red[1][h][t][3]);
-    kconst[(static_cast<size_t>(bh) * 2 + t) * 8 + h] = make_float2(c, 1.0f / lam[t]);
+  if (i == 0) {
+    const float cs = (red[1][h][0][0] + red[1][h][0][1]) + (red[1][h][0][2] + red[1][h][0][3]);
+    const float ss = (red[1][h][1][0] + red[1][h][1][1]) + (red[1][h][1][2] + red[1][h][1][3]);
+    kconst[static_cast<size_t>(bh) * 8 + h] = make_float4(ldexpf(1.f, -E[0]), wsum * cs, ldexpf(1.f, -E[1]), ss);
   }
 }
 
@@ -1012,13 +1029,15 @@ SplitPlan plan_splits(int BH, int64_t T) {
   return sp;
 }
 
-int num_tiles_n(int G) { return (2 * G + 7) / 8; }
-
-size_t frag_bytes(int BH, int G) { return static_cast<size_t>(BH) * 2 * num_tiles_n(G) * 8 * 32 * 2 * 4; }
+// Key-side B fragments: [BH][MG][2 NT][32][2] u32, MG for the largest code
+// (3 bits: 20 groups), NT = ceil(G / 4) head groups.
+size_t frag_bytes(int BH, int G) {
+  return static_cast<size_t>(BH) * KeyGroups<3>::MG * 2 * ((G + 3) / 4) * 32 * 2 * 4;
+}
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
-size_t kconst_bytes(int BH) { return static_cast<size_t>(BH) * 2 * 8 * sizeof(float2); }
+size_t kconst_bytes(int BH) { return static_cast<size_t>(BH) * 8 * sizeof(float4); }
 
 // Sequences (batch x KV heads) of one call: the split kernel's grid has one
 // row of blocks per sequence, and CUDA caps a grid's y extent at 65535.
@@ -1082,28 +1101,41 @@ int launch_split(const DecodeParams& p, int BH, cudaStream_t s) {
   return launch_pdl(kern, grid, dim3(kWarps * 32), smem, s, p);
 }
 
-template <typename T>
-void qprep_g(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope, uint16_t* qfrag,
-             float2* kconst, cudaStream_t s) {
+template <typename T, int BITS>
+int qprep_g(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
+            uint32_t* qfrag, float4* kconst, cudaStream_t s) {
+  WalshWeights w{};
+  for (int i = 0; i < 4; ++i) w.w[i] = static_cast<float>(hk->walsh[i]);
 #define TQ_QPREP(GG)                                                                                       \
-  launch_pdl(decode_qprep_kernel<T, GG>, dim3(BH), dim3(kD * GG), 0, s, q, q_pos, Hkv, hk->d_signs, hk->d_st,        \
-             hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope, qfrag, kconst)
+  return launch_pdl(decode_qprep_kernel<T, GG, BITS>, dim3(BH), dim3(kD * GG), 0, s, q, q_pos, Hkv,        \
+                    hk->d_signs, hk->d_st, hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope, w, qfrag, \
+                    kconst)
   switch (G) {
-    case 1: TQ_QPREP(1); break;
-    case 2: TQ_QPREP(2); break;
-    case 4: TQ_QPREP(4); break;
-    case 8: TQ_QPREP(8); break;
+    case 1: TQ_QPREP(1);
+    case 2: TQ_QPREP(2);
+    case 4: TQ_QPREP(4);
+    case 8: TQ_QPREP(8);
   }
 #undef TQ_QPREP
+  return TQ_EUNSUPPORTED;
+}
+
+template <typename T>
+int qprep_b(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
+            uint32_t* qfrag, float4* kconst, cudaStream_t s) {
+  switch (hk->bits) {
+    case 1: return qprep_g<T, 1>(G, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
+    case 2: return qprep_g<T, 2>(G, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
+    case 3: return qprep_g<T, 3>(G, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
+  }
+  return TQ_EUNSUPPORTED;
 }
 
 int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
-                 uint16_t* qfrag, float2* kconst, cudaStream_t s) {
+                 uint32_t* qfrag, float4* kconst, cudaStream_t s) {
   if (q_dtype == TQ_F32)
-    qprep_g<float>(G, BH, Hkv, static_cast<const float*>(q), q_pos, hk, rope, qfrag, kconst, s);
-  else
-    qprep_g<__nv_bfloat16>(G, BH, Hkv, static_cast<const __nv_bfloat16*>(q), q_pos, hk, rope, qfrag, kconst, s);
-  return TQ_OK;
+    return qprep_b<float>(G, BH, Hkv, static_cast<const float*>(q), q_pos, hk, rope, qfrag, kconst, s);
+  return qprep_b<__nv_bfloat16>(G, BH, Hkv, static_cast<const __nv_bfloat16*>(q), q_pos, hk, rope, qfrag, kconst, s);
 }
 
 // Merge of n_parts partial records per head (layout: see decode_merge_kernel).
@@ -1226,11 +1258,11 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   const int n_slots = sp.n_splits + (R + kWinChunk - 1) / kWinChunk;   // window chunks after the splits
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws);
-  float2* kconst = reinterpret_cast<float2*>(ws + align256(frag_bytes(BH, G)));
+  float4* kconst = reinterpret_cast<float4*>(ws + align256(frag_bytes(BH, G)));
   float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
   const float score_scale = scale * 1.4426950408889634f;
 
-  int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, reinterpret_cast<uint16_t*>(qfrag), kconst, s);
+  int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
   if (st != TQ_OK) return st;
   st = tq::launch_status();
   if (st != TQ_OK) return st;
