@@ -59,8 +59,7 @@ def test_partials_merge_equals_whole_decode(cuda_device, cuts, G):
                                          tuple(a[:, :, s:e] for a in vc), 1 / np.sqrt(D)))
     stacked = torch.stack(parts)
     out = tq.decode_merge_partials(rv, stacked, Hkv)
-    whole = tq.decode_attention(rk, rv, q, qpos, tuple(torch.from_numpy(a).to(dev) for a in kc),
-                                tuple(torch.from_numpy(a).to(dev) for a in vc), T)
+    whole = tq.decode_attention(rk, rv, q, qpos, shard(kc, 0, T), shard(vc, 0, T), T)
     torch.cuda.synchronize()
     ref = at.decode_attention(rk_o, rv_o, q.cpu().numpy(), [T - 1] * B, kc, vc, 1 / np.sqrt(D))
     assert_close(out.cpu().numpy(), ref, what="merged partials vs oracle")

@@ -211,7 +211,6 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       for (int r = 0; r < 4; ++r) accC[nt][rb][r] = accZ[nt][rb][r] = 0.f;
   }
   const float piece_m = (gid & 1) ? 1.f : 0.f;   // this lane feeds the hi (0) or lo (1) piece
-  const uint32_t half_sel = (gid & 1) ? 0x7632u : 0x5410u;
   // ---- K side of one tile: logits of tokens gid, gid + 8 for head tig + 4 nt.
   // m16n8k32 u8 x s8 products into int32: rows are the 16 tokens, K runs over
   // (plane, coordinate) slots, the columns are (head, digit); each A register
@@ -334,26 +333,31 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
     const uint8_t* vs = vcd + kTile * CB;
     const float2* vn = reinterpret_cast<const float2*>(vcd + kTile * (CB + SB));
     const int tk[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+    // Transposing matrix loads: an 8 x 8 matrix of 16-bit elements whose row r
+    // is the 16-byte plane (or sign) row of token r of a group of eight; the
+    // transposed load hands lane (g, t) half-word g (coordinates 16g..16g+15)
+    // of tokens 2t and 2t + 1 in one register, the pair a bit-select turns
+    // into the two K elements of the value operand.  Lane l addresses row
+    // l % 8 of matrix l / 8.
     uint32_t x01[P], x23[P], z01, z23;
     {
       uint32_t r01[BITS], r23[BITS];
-#pragma unroll
-      for (int k = 0; k < BITS; ++k) {
-        const uint32_t h0 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[0], k) * 16)[gid >> 1];
-        const uint32_t h1 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[1], k) * 16)[gid >> 1];
-        const uint32_t h2 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[2], k) * 16)[gid >> 1];
-        const uint32_t h3 = reinterpret_cast<const uint32_t*>(vcd + code_chunk<BITS>(tk[3], k) * 16)[gid >> 1];
-        r01[k] = __byte_perm(h0, h1, half_sel);
-        r23[k] = __byte_perm(h2, h3, half_sel);
+      const int mi = lane >> 3, rr = lane & 7;
+      const uint32_t vbase = tqtc::smem_u32(vcd), sbase = tqtc::smem_u32(vs);
+      const uint32_t code_row = vbase + static_cast<uint32_t>((rr + 8 * (mi & 1)) * CB + (mi >> 1) * 16);
+      const uint32_t sign_row = sbase + static_cast<uint32_t>((rr + 8 * (mi & 1)) * SB);
+      if constexpr (BITS == 1) {
+        ldsm_x4_trans(r01[0], r23[0], z01, z23, mi < 2 ? code_row : sign_row);
+      } else if constexpr (BITS == 2) {
+        ldsm_x4_trans(r01[0], r23[0], r01[1], r23[1], code_row);
+        ldsm_x2_trans(z01, z23, sign_row);
+      } else {
+        ldsm_x4_trans(r01[0], r23[0], r01[1], r23[1], code_row);
+        ldsm_x4_trans(r01[2], r23[2], z01, z23,
+                      mi < 2 ? vbase + static_cast<uint32_t>((rr + 8 * mi) * CB + 32) : sign_row);
       }
       Planes<BITS>::make(r01, x01);
       Planes<BITS>::make(r23, x23);
-      const uint32_t g0 = reinterpret_cast<const uint32_t*>(vs + tk[0] * SB)[gid >> 1];
-      const uint32_t g1 = reinterpret_cast<const uint32_t*>(vs + tk[1] * SB)[gid >> 1];
-      const uint32_t g2 = reinterpret_cast<const uint32_t*>(vs + tk[2] * SB)[gid >> 1];
-      const uint32_t g3 = reinterpret_cast<const uint32_t*>(vs + tk[3] * SB)[gid >> 1];
-      z01 = __byte_perm(g0, g1, half_sel);
-      z23 = __byte_perm(g2, g3, half_sel);
     }
     uint32_t xs01[P], xs23[P];
 #pragma unroll
