@@ -73,9 +73,6 @@ struct DecodeParams {
   int Hkv;
 };
 
-// Polls of a stage's mbarrier before the warp gives up on its copies (about a
-// second); the warp then reports NaN for its heads instead of hanging.
-constexpr int kCopyWaitPolls = 1 << 17;
 
 // Key-side MMA groups of the split kernel (m16n8k32, u8 bits x s8 query
 // digits).  A group covers 32 K elements per 16 tokens: with two Walsh planes
@@ -97,11 +94,13 @@ struct WalshWeights {
 };
 
 // Shared-memory position of the 16-byte chunk `part` (code plane) of token
-// `tok`'s codes: the records as they lie in the cache, one bulk copy per
-// array and tile.
+// `tok`'s codes.  With 2-bit codes (two chunks per token) the chunks of tokens
+// 4..7 (mod 8) are swapped so that the key side's word reads are free of bank
+// conflicts.
 template <int BITS>
 __device__ __forceinline__ int code_chunk(int tok, int part) {
-  return tok * BITS + part;
+  if constexpr (BITS == 2) return tok * 2 + (part ^ ((tok >> 2) & 1));
+  else return tok * BITS + part;
 }
 
 template <int BITS, int G>
@@ -136,48 +135,48 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   const int64_t seq = static_cast<int64_t>(bh) * p.cache_stride;
   uint8_t* my_stages = smem + warp * kStages * STAGE;
 
-  // One mbarrier per stage of this warp's ring.  Lane 0 issues a tile as six
-  // bulk copies - K codes, signs, norms and V codes, signs, norms, each one
-  // contiguous block of the cache - completing on the stage's mbarrier; the
-  // warp waits on it before reading the stage.  Rows past the tile's last
-  // token keep what the stage held before (the readers mask them).
-  __shared__ uint64_t s_mbar[kWarps][kStages];
-  if (lane == 0) {
-#pragma unroll
-    for (int st = 0; st < kStages; ++st) tqtc::mbar_init(&s_mbar[warp][st], 1);
-  }
-  __syncwarp();
+  // Each lane copies 16-byte chunks of the tile's K and V codes, signs and
+  // norms into the warp's stage (cp.async, a 4-stage ring per warp); rows past
+  // the tile's last token are zero-filled.
   auto tile_nv = [&](int i) {
     const int64_t t0 = t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
     return static_cast<int>(t_end - t0 < kTile ? t_end - t0 : kTile);
   };
+  const int sg_side = lane >> 4, sg_c = lane & 15;
+  const int nm_side = (lane >> 3) & 1, nm_c = lane & 7;
   auto issue = [&](int i) {
-    if (i < my_count && lane == 0) {
+    if (i < my_count) {
       const int64_t t0 = seq + t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
       const int nv = tile_nv(i);
-      const int nn = (nv + 1) & ~1;   // norms in pairs: 16-byte copies (record nv exists: cache_stride is even)
       uint8_t* stg = my_stages + (i % kStages) * STAGE;
-      uint64_t* mb = &s_mbar[warp][i % kStages];
-      tqtc::mbar_arrive_expect_tx(mb, static_cast<uint32_t>(2 * (nv * (CB + SB) + nn * 8)));
-      tqtc::bulk_load(stg, p.k_codes + t0 * CB, nv * CB, mb);
-      tqtc::bulk_load(stg + kTile * CB, p.k_signs + t0 * SB, nv * SB, mb);
-      tqtc::bulk_load(stg + kTile * (CB + SB), p.k_norms + t0, nn * 8, mb);
-      tqtc::bulk_load(stg + HALF, p.v_codes + t0 * CB, nv * CB, mb);
-      tqtc::bulk_load(stg + HALF + kTile * CB, p.v_signs + t0 * SB, nv * SB, mb);
-      tqtc::bulk_load(stg + HALF + kTile * (CB + SB), p.v_norms + t0, nn * 8, mb);
+#pragma unroll
+      for (int side = 0; side < 2; ++side) {
+        const uint8_t* src = (side ? p.v_codes : p.k_codes) + t0 * CB;
+#pragma unroll
+        for (int c = lane; c < CCH; c += 32) {
+          const int tok = c / BITS, part = c % BITS;
+          cp_async16(stg + side * HALF + code_chunk<BITS>(tok, part) * 16, tok < nv ? src + c * 16 : src,
+                     tok < nv ? 16 : 0);
+        }
+      }
+      {
+        const uint8_t* src = (sg_side ? p.v_signs : p.k_signs) + t0 * SB;
+        cp_async16(stg + sg_side * HALF + kTile * CB + sg_c * 16, sg_c < nv ? src + sg_c * 16 : src, sg_c < nv ? 16 : 0);
+      }
+      if (lane < 16) {
+        const float2* src = (nm_side ? p.v_norms : p.k_norms) + t0;
+        const int bytes = max(0, min(16, (nv - 2 * nm_c) * 8));
+        cp_async16(stg + nm_side * HALF + kTile * (CB + SB) + nm_c * 16, bytes ? src + 2 * nm_c : src, bytes);
+      }
     }
-  };
-  // wait for tile i's copies; false if they did not complete in time
-  auto arrived = [&](int i) {
-    return tqtc::mbar_wait(&s_mbar[warp][i % kStages], static_cast<uint32_t>((i / kStages) & 1), kCopyWaitPolls);
+    cp_async_commit();
   };
 
   // The first tiles of the cache do not depend on the q-prep launch: start
   // their copies, then wait for q-prep's outputs (programmatic dependent
   // launch; a no-op when launched without it).
-  int issued = my_count < kStages - 1 ? my_count : kStages - 1;
 #pragma unroll 1
-  for (int i = 0; i < issued; ++i) issue(i);
+  for (int i = 0; i < kStages - 1; ++i) issue(i);
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
   // The key side's B operand (int8 digits of the query, one set of
@@ -344,7 +343,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       uint32_t r01[BITS], r23[BITS];
       const int mi = lane >> 3, rr = lane & 7;
       const uint32_t vbase = tqtc::smem_u32(vcd), sbase = tqtc::smem_u32(vs);
-      const uint32_t code_row = vbase + static_cast<uint32_t>((rr + 8 * (mi & 1)) * CB + (mi >> 1) * 16);
+      const uint32_t code_row = vbase + static_cast<uint32_t>(code_chunk<BITS>(rr + 8 * (mi & 1), mi >> 1) * 16);
       const uint32_t sign_row = sbase + static_cast<uint32_t>((rr + 8 * (mi & 1)) * SB);
       if constexpr (BITS == 1) {
         ldsm_x4_trans(r01[0], r23[0], z01, z23, mi < 2 ? code_row : sign_row);
@@ -354,7 +353,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       } else {
         ldsm_x4_trans(r01[0], r23[0], r01[1], r23[1], code_row);
         ldsm_x4_trans(r01[2], r23[2], z01, z23,
-                      mi < 2 ? vbase + static_cast<uint32_t>((rr + 8 * mi) * CB + 32) : sign_row);
+                      mi < 2 ? vbase + static_cast<uint32_t>(code_chunk<BITS>(rr + 8 * mi, 2) * 16) : sign_row);
       }
       Planes<BITS>::make(r01, x01);
       Planes<BITS>::make(r23, x23);
@@ -425,32 +424,23 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   // Pipelined order: the key side of tile i and the value side of tile i - 1
   // share one loop body (for G = 8 this fits the register file because the
   // query fragments are in shared memory).
-  bool failed = bad_len;
-  int consumed = 0;
   {
     float prob_prev[NT][2];
     const uint8_t* stg_prev = my_stages;
     int nv_prev = 0;
-    if (my_count > 0 && !failed) {
-      if (!arrived(0)) {
-        failed = true;
-      } else {
-        consumed = 1;
-        float logit[NT][2];
-        nv_prev = tile_nv(0);
-        k_side(my_stages, nv_prev, logit);
-        softmax(logit, prob_prev);
-        __syncwarp();
-        if (issued < my_count) issue(issued++);   // stage kStages-1 is still unused
-      }
+    if (my_count > 0) {
+      cp_async_wait<kStages - 2>();
+      __syncwarp();
+      float logit[NT][2];
+      nv_prev = tile_nv(0);
+      k_side(my_stages, nv_prev, logit);
+      softmax(logit, prob_prev);
+      issue(kStages - 1);   // stage kStages-1 is still unused
     }
 #pragma unroll 1
-    for (int i = 1; i < my_count && !failed; ++i) {
-      if (!arrived(i)) {
-        failed = true;
-        break;
-      }
-      consumed = i + 1;
+    for (int i = 1; i < my_count; ++i) {
+      cp_async_wait<kStages - 2>();
+      __syncwarp();
       const uint8_t* stg = my_stages + (i % kStages) * STAGE;
       const int nv = tile_nv(i);
       float logit[NT][2];
@@ -460,16 +450,12 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       stg_prev = stg;
       nv_prev = nv;
       __syncwarp();
-      if (issued < my_count) issue(issued++);   // into the stage of tile i - 1
+      issue(i + kStages - 1);             // into the stage of tile i - 1
     }
-    if (consumed > 0 && !failed) v_side(stg_prev, prob_prev, nv_prev);
+    if (my_count > 0) v_side(stg_prev, prob_prev, nv_prev);
   }
-  // copies still in flight into this warp's stages complete before the CTA
-  // leaves (bounded; after a timeout the CTA reports NaN)
-#pragma unroll 1
-  for (int i = consumed; i < issued; ++i)
-    if (!arrived(i)) failed = true;
-  if (failed) {   // a finite max keeps the NaN sum from being dropped by the merges
+  cp_async_wait<0>();
+  if (bad_len) {   // a finite max keeps the NaN sum from being dropped by the merges
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       m_run[nt] = 0.f;
