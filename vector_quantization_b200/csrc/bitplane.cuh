@@ -70,18 +70,17 @@ __device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// An int32 of magnitude below 2^22 as float, exactly: adding it to the bit
-// pattern of 1.5 * 2^23 places it in the mantissa (integer add + one FADD).
-__device__ __forceinline__ float small_int_to_float(int x) {
-  return __int_as_float(x + 0x4B400000) - 12582912.0f;
-}
+// Integer accumulators started at kBiasedZero hold 1.5 * 2^23 + x as a float
+// bit pattern while |x| < 2^22, so the float value of x is one subtraction.
+constexpr int kBiasedZero = 0x4B400000;
+__device__ __forceinline__ float biased_to_float(int b) { return __int_as_float(b) - 12582912.0f; }
 
-// d0 + 2^8 d1 + 2^16 d2 + 2^24 d3 in fp32 for four digit sums below 2^22.
-__device__ __forceinline__ float digits_to_float(int d0, int d1, int d2, int d3) {
-  float f = small_int_to_float(d3);
-  f = fmaf(f, 256.f, small_int_to_float(d2));
-  f = fmaf(f, 256.f, small_int_to_float(d1));
-  return fmaf(f, 256.f, small_int_to_float(d0));
+// d0 + 2^8 d1 + 2^16 d2 + 2^24 d3 in fp32 from four biased digit sums.
+__device__ __forceinline__ float digits_to_float(int b0, int b1, int b2, int b3) {
+  float f = biased_to_float(b3);
+  f = fmaf(f, 256.f, biased_to_float(b2));
+  f = fmaf(f, 256.f, biased_to_float(b1));
+  return fmaf(f, 256.f, biased_to_float(b0));
 }
 
 // Two bf16 values +-1 from bits x (low half) and x+16 (high half) of w:

@@ -191,8 +191,12 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
     for (int i = threadIdx.x; i < MG * NTK * 32; i += blockDim.x) (&s_qf[0][0][0])[i] = src[i];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
+      // per-head scale and constant of the code sum and of the sign sum, with
+      // the softmax scale (and the QJL constant for the signs) folded in
       const int h = tig + 4 * nt;
-      kc[nt] = h < G ? p.kconst[static_cast<size_t>(bh) * 8 + h] : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 c = h < G ? p.kconst[static_cast<size_t>(bh) * 8 + h] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float zs = p.qjl * p.score_scale;
+      kc[nt] = make_float4(c.x * p.score_scale, c.y * p.score_scale, c.z * zs, c.w * zs);
     }
     __syncthreads();
   }
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
 #pragma unroll
     for (int n = 0; n < NTK; ++n)
 #pragma unroll
-      for (int r = 0; r < 4; ++r) accc[n][r] = accs[n][r] = 0;
+      for (int r = 0; r < 4; ++r) accc[n][r] = accs[n][r] = kBiasedZero;   // every column stays below 2^22
     if constexpr (BITS == 1) {
       const uint32_t w4[2] = {wk[0][0] >> 4, wk[1][0] >> 4};
 #pragma unroll
@@ -287,7 +291,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
         const float sgn = fmaf(digits_to_float(accs[2 * nt][2 * e], accs[2 * nt][2 * e + 1],
                                                accs[2 * nt + 1][2 * e], accs[2 * nt + 1][2 * e + 1]),
                                kc[nt].z, -kc[nt].w);
-        const float l = fmaf(knorm[e].x, code, knorm[e].y * p.qjl * sgn) * p.score_scale;
+        const float l = fmaf(knorm[e].x, code, knorm[e].y * sgn);
         logit[nt][e] = gid + 8 * e < nv ? l : -INFINITY;
       }
     }
@@ -380,9 +384,9 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       uint32_t bc[P][2], bz[2];
       float wv[4], wr[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {   // rows past the tile's last token hold stale records
-        wv[j] = tk[j] < nv ? pt[j] * vnorm[j].x : 0.f;
-        wr[j] = tk[j] < nv ? pt[j] * vnorm[j].y : 0.f;
+      for (int j = 0; j < 4; ++j) {
+        wv[j] = pt[j] * vnorm[j].x;   // rows past the tile's last token: p = 0, zero-filled norms
+        wr[j] = pt[j] * vnorm[j].y;
       }
       // B operand: lanes of even gid feed RN(w), odd gid RN(w - RN(w)), both
       // as bf16 pairs: one paired conversion, an FFMA by piece_m in {0, 1},
