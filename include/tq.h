@@ -243,6 +243,44 @@ int tq_quantize_kv_pair(const tq_rotation* hk, const void* xk, const tq_rotation
                         float* v_norms, int64_t out_stride, void* stream);
 
 /*
+ * tq_quantize_kv_scatter - tq_quantize_kv with an explicit destination record
+ * per row: row i is written to record out_rows[i] of the codes, signs and
+ * norms arrays.  One call writes rows bound for many sequences of a cache,
+ * e.g. the flush of every sequence's full-precision window ([NSNQuant] §4,
+ * "Résidus": the residual is quantized and appended when full) into records
+ * T_b .. T_b + R - 1 of each sequence b, with pos giving each row's position.
+ *   out_rows    device [n] int64 destination records; rows whose entry lies
+ *               outside [0, n_records) are skipped (nothing written)
+ *   n_records   records the codes, signs and norms arrays hold (>= 1)
+ *   other arguments as in tq_quantize_kv (out_stride is not used)
+ * Records are identical to tq_quantize_kv's for the same rows.  Returns the
+ * statuses of tq_quantize_kv.
+ */
+int tq_quantize_kv_scatter(const tq_rotation* h, const void* x, int dtype,
+                           int64_t n, int64_t ld, const int64_t* pos,
+                           int64_t pos_period, int64_t pos_offset,
+                           int apply_rope, uint8_t* codes, uint8_t* signs,
+                           float* norms, const int64_t* out_rows,
+                           int64_t n_records, void* stream);
+
+/*
+ * tq_quantize_kv_pair_scatter - tq_quantize_kv_pair with destination records
+ * out_rows[i] for row i of both sets (keys with RoPE at pos, values without),
+ * e.g. the new token of each sequence of a ragged batch appended at its own
+ * length.  One launch for n <= 256 with equal d and bits, else one launch per
+ * set.  Arguments as in tq_quantize_kv_pair and tq_quantize_kv_scatter.
+ */
+int tq_quantize_kv_pair_scatter(const tq_rotation* hk, const void* xk,
+                                const tq_rotation* hv, const void* xv, int dtype,
+                                int64_t n, int64_t ld, const int64_t* pos,
+                                int64_t pos_period, int64_t pos_offset,
+                                int apply_rope, uint8_t* k_codes,
+                                uint8_t* k_signs, float* k_norms,
+                                uint8_t* v_codes, uint8_t* v_signs,
+                                float* v_norms, const int64_t* out_rows,
+                                int64_t n_records, void* stream);
+
+/*
  * tq_quantize_dense - encode n vectors with a dense-rotation handle
  * (TQ_ROT_DENSE).  Same steps and record format as tq_quantize_kv, without
  * RoPE; y = Pi x and S r are dense contractions here, computed as fp32 GEMMs

@@ -252,3 +252,32 @@ def test_seeded_build_matches_oracle_from_its_own_generator(cuda_device, d, bits
         gpu = tq.quantize_kv(g, torch.from_numpy(x).to(cuda_device))
         codes, signs, norms, enc = oracle_records(o, x)
         compare_records(o, tuple(a.cpu().numpy() for a in gpu), enc)
+
+
+@pytest.mark.parametrize("n", [100, 300])
+def test_scatter_encode_places_rows_at_their_records(cuda_device, n):
+    """tq_quantize_kv_scatter: row i lands in record out_rows[i] (keys with
+    RoPE at their own positions), with the oracle's codes; rows whose target
+    lies outside the arrays are skipped and every other record is untouched."""
+    from vector_quantization_b200 import tq
+    d, bits, nrec = 128, 2, 1000
+    g = _gpu_rot(d, bits, 61, rope=10000.0)
+    o, _ = oracle_rotation(d, bits, 61, rope=10000.0)
+    rng = np.random.default_rng(62)
+    x = synth.heavy_tailed((n, d), 63)
+    pos = rng.integers(0, 5000, size=n).astype(np.int64)
+    rows = rng.permutation(nrec)[:n].astype(np.int64)
+    rows[3], rows[7] = -1, nrec + 5                      # skipped
+    dev = cuda_device
+    out = tuple(torch.full((nrec, w), 0xAB, dtype=torch.uint8, device=dev) for w in (g.code_bytes, g.sign_bytes))
+    out = out + (torch.full((nrec, 2), -7.0, dtype=torch.float32, device=dev),)
+    tq.quantize_kv_scatter(g, torch.from_numpy(x).to(dev), torch.from_numpy(rows).to(dev), out,
+                           pos=torch.from_numpy(pos).to(dev), apply_rope=True)
+    torch.cuda.synchronize()
+    got = tuple(a.cpu().numpy() for a in out)
+    keep = (rows >= 0) & (rows < nrec)
+    _, _, _, enc = oracle_records(o, x[keep], pos[keep])
+    compare_records(o, tuple(a[rows[keep]] for a in got), enc)
+    untouched = np.setdiff1d(np.arange(nrec), rows[keep])
+    assert np.all(got[0][untouched] == 0xAB) and np.all(got[1][untouched] == 0xAB)
+    assert np.all(got[2][untouched] == -7.0)

@@ -271,3 +271,34 @@ def test_window_ragged_batch(cuda_device):
                                          tuple(a[b:b + 1, :, :n] for a in kc), tuple(a[b:b + 1, :, :n] for a in vc),
                                          kw_ref[b:b + 1], vw_ref[b:b + 1], 1 / np.sqrt(D))
         assert_close(out[b:b + 1], ref, what=f"sequence {b}: {n} packed + {R} window tokens")
+
+
+def test_window_flush_in_one_call_matches_per_sequence_flushes(cuda_device):
+    """A ragged batch's windows flushed by one tq_quantize_kv_pair_scatter call
+    (row (b, j, i) -> record (b Hkv + j) cap + T_b + i, key position T_b + i)
+    give the same records, bit for bit, as one tq_quantize_kv_pair call per
+    (sequence, KV head)."""
+    from vector_quantization_b200 import tq
+    dev = cuda_device
+    lens, Hkv, R, bits = [100, 37, 0], 2, 16, 2
+    B, cap = len(lens), 140
+    rk, rv = _gpu_rot(bits, 1541, 10000.0), _gpu_rot(bits, 1641, 0.0)
+    kw = torch.from_numpy(synth.heavy_tailed((B, Hkv, R, D), 1741)).to(torch.bfloat16).to(dev)
+    vw = torch.from_numpy(synth.heavy_tailed((B, Hkv, R, D), 1841)).to(torch.bfloat16).to(dev)
+
+    def fresh():
+        return (tuple(torch.zeros((B, Hkv, cap, w), dtype=torch.uint8, device=dev) for w in (rk.code_bytes, rk.sign_bytes))
+                + (torch.zeros((B, Hkv, cap, 2), dtype=torch.float32, device=dev),))
+    ka, va, kb, vb = fresh(), fresh(), fresh(), fresh()
+    for b, n in enumerate(lens):
+        for j in range(Hkv):
+            tq.quantize_kv_pair(rk, kw[b, j], rv, vw[b, j], apply_rope=True, pos_period=R, pos_offset=n,
+                                out_k=tuple(a[b, j, n:n + R] for a in ka), out_v=tuple(a[b, j, n:n + R] for a in va))
+    rows = np.array([(b * Hkv + j) * cap + lens[b] + i for b in range(B) for j in range(Hkv) for i in range(R)],
+                    dtype=np.int64)
+    pos = np.array([lens[b] + i for b in range(B) for j in range(Hkv) for i in range(R)], dtype=np.int64)
+    tq.quantize_kv_pair_scatter(rk, kw, rv, vw, torch.from_numpy(rows).to(dev), kb, vb,
+                                pos=torch.from_numpy(pos).to(dev), apply_rope=True)
+    torch.cuda.synchronize()
+    for x, y in zip(ka + va, kb + vb):
+        assert torch.equal(x, y)

@@ -28,6 +28,8 @@ struct EncodeParams {
   uint32_t* signs;      // record = D / 32 words (m == D)
   float2* norms;        // record = (||x||, ||r||)
   int64_t out_stride;
+  const int64_t* out_rows;  // [n] record of each row (scatter calls), or null: row * out_stride
+  int64_t n_records;        // records in the output arrays (scatter calls: targets outside are skipped)
   const float* dsigns;  // [D]
   const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
   const uint16_t* hd_op; // tensor-core encode: H D in the same layout (fp16 bits when split, else bf16)
@@ -45,6 +47,15 @@ struct EncodeParams {
   float lpos[4];        // levels above 0, ascending (2^(b-1) of them)
   float2 theta[64];     // tensor-core encode: RoPE frequency i as (hi, lo) float pieces
 };
+
+// Output record of input row `row`: row * out_stride, or the row's entry of
+// out_rows for scatter calls (-1, not written, when that entry lies outside
+// the output arrays).
+__device__ __forceinline__ int64_t out_record(const EncodeParams& p, int64_t row) {
+  if (!p.out_rows) return row * p.out_stride;
+  const int64_t r = p.out_rows[row];
+  return r >= 0 && r < p.n_records ? r : -1;
+}
 
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
 constexpr int kTileVec = 128;
@@ -75,7 +86,8 @@ __device__ __forceinline__ void encode_vec_body(const EncodeParams& p) {
   float x;
   if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(xr) + i);
   else x = __bfloat162float(xr[i]);
-  const int64_t rec = row * p.out_stride;
+  const int64_t rec = out_record(p, row);
+  if (rec < 0) return;   // uniform over the block (one vector per block)
   if (p.rope) {
     const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
     if (pos < 0 || pos >= p.rope_max_pos) {   // uniform over the block
@@ -368,7 +380,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
       for (int c = 0; c < 2; ++c) {
         if (q0 + c >= RUN || warp * RUN + q0 + c >= R) break;
         if (valid[c]) {
-          const int64_t rec = row[c] * p.out_stride;
+          const int64_t rec = out_record(p, row[c]);
+          if (rec < 0) continue;
           if (pos_ok[c]) {
             uint32_t* crec = p.codes + rec * (BITS * NJ);
 #pragma unroll
@@ -431,12 +444,12 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
         for (int b = 0; b < 32; ++b) w |= (val[b] >= 0.f ? 1u : 0u) << b;
         words[c] = w;
       }
-      if (row < p.n) {
-        uint32_t* srec = p.signs + row * p.out_stride * NJ + half * (COLS / 32);
+      const int64_t rec = row < p.n ? out_record(p, row) : -1;
+      if (rec >= 0) {
+        uint32_t* srec = p.signs + rec * NJ + half * (COLS / 32);
 #pragma unroll
         for (int c = 0; c < COLS / 32; ++c) srec[c] = ok ? words[c] : 0u;
-        if (!ok && half == 0)
-          p.norms[row * p.out_stride] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+        if (!ok && half == 0) p.norms[rec] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
       }
     }
     tqtc::fence_before_sync();
@@ -1256,7 +1269,7 @@ int launch_encode(const EncodeParams& p, cudaStream_t stream) {
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, encode_vec_kernel<D, BITS, T>, p) == cudaSuccess ? TQ_OK : TQ_ECUDA;
   }
-  if (p.n < kRowsKernelMinN) return launch_encode_warp<D, BITS, T>(p, stream);
+  if (p.n < kRowsKernelMinN || p.out_rows) return launch_encode_warp<D, BITS, T>(p, stream);
   if constexpr (D == 128) return launch_encode_d128<BITS, T>(p, stream);
   return launch_encode_rows<D, BITS, T>(p, stream);
 }
@@ -1302,7 +1315,8 @@ namespace {
 // Checks of one tq_quantize_kv call and its kernel parameters.
 int make_encode_params(const tq_rotation* h, const void* x, int dtype, int64_t n, int64_t ld, const int64_t* pos,
                        int64_t pos_period, int64_t pos_offset, int apply_rope, uint8_t* codes, uint8_t* signs,
-                       float* norms, int64_t out_stride, EncodeParams* out) {
+                       float* norms, int64_t out_stride, EncodeParams* out, const int64_t* out_rows = nullptr,
+                       int64_t n_records = 0) {
   if (!h) return TQ_EINVAL;
   if (n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16)) return TQ_EINVAL;
   if (!x || !codes || !signs || !norms || out_stride < 1 || ld < h->d) return TQ_EINVAL;
@@ -1333,6 +1347,8 @@ int make_encode_params(const tq_rotation* h, const void* x, int dtype, int64_t n
   p.signs = reinterpret_cast<uint32_t*>(signs);
   p.norms = reinterpret_cast<float2*>(norms);
   p.out_stride = out_stride;
+  p.out_rows = out_rows;
+  p.n_records = n_records;
   p.dsigns = h->d_signs;
   p.s_op = h->d_s_op;
   // H D for the tensor-core encode: fp16 when the rows are split (RoPE or fp32 input), else bf16
@@ -1404,4 +1420,54 @@ extern "C" int tq_quantize_kv_pair(const tq_rotation* hk, const void* xk, const 
                       out_stride, stream);
   if (st != TQ_OK) return st;
   return tq_quantize_kv(hv, xv, dtype, n, ld, nullptr, 1, 0, 0, v_codes, v_signs, v_norms, out_stride, stream);
+}
+
+extern "C" int tq_quantize_kv_scatter(const tq_rotation* h, const void* x, int dtype, int64_t n, int64_t ld,
+                                      const int64_t* pos, int64_t pos_period, int64_t pos_offset, int apply_rope,
+                                      uint8_t* codes, uint8_t* signs, float* norms, const int64_t* out_rows,
+                                      int64_t n_records, void* stream) {
+  if (!h) return TQ_EINVAL;
+  if (n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16) || !out_rows || n_records < 1) return TQ_EINVAL;
+  if (n == 0) return TQ_OK;
+  EncodeParams p{};
+  const int st = make_encode_params(h, x, dtype, n, ld, pos, pos_period, pos_offset, apply_rope, codes, signs, norms,
+                                    1, &p, out_rows, n_records);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (h->d == 128)
+    return dtype == TQ_F32 ? dispatch_bits<128, float>(h->bits, p, s) : dispatch_bits<128, __nv_bfloat16>(h->bits, p, s);
+  if (h->d == 64)
+    return dtype == TQ_F32 ? dispatch_bits<64, float>(h->bits, p, s) : dispatch_bits<64, __nv_bfloat16>(h->bits, p, s);
+  return TQ_EUNSUPPORTED;
+}
+
+extern "C" int tq_quantize_kv_pair_scatter(const tq_rotation* hk, const void* xk, const tq_rotation* hv,
+                                           const void* xv, int dtype, int64_t n, int64_t ld, const int64_t* pos,
+                                           int64_t pos_period, int64_t pos_offset, int apply_rope, uint8_t* k_codes,
+                                           uint8_t* k_signs, float* k_norms, uint8_t* v_codes, uint8_t* v_signs,
+                                           float* v_norms, const int64_t* out_rows, int64_t n_records,
+                                           void* stream) {
+  if (!hk || !hv) return TQ_EINVAL;
+  if (n < 0 || (dtype != TQ_F32 && dtype != TQ_BF16) || !out_rows || n_records < 1) return TQ_EINVAL;
+  if (n == 0) return TQ_OK;
+  EncodeParams pk{}, pv{};
+  int st = make_encode_params(hk, xk, dtype, n, ld, pos, pos_period, pos_offset, apply_rope, k_codes, k_signs,
+                              k_norms, 1, &pk, out_rows, n_records);
+  if (st != TQ_OK) return st;
+  if ((st = make_encode_params(hv, xv, dtype, n, ld, nullptr, 1, 0, 0, v_codes, v_signs, v_norms, 1, &pv, out_rows,
+                               n_records)) != TQ_OK)
+    return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n <= kVecKernelMaxN && hk->d == hv->d && hk->bits == hv->bits && (hk->d == 128 || hk->d == 64)) {
+    if (hk->d == 128)
+      return dtype == TQ_F32 ? dispatch_vec_pair<128, float>(hk->bits, pk, pv, s)
+                             : dispatch_vec_pair<128, __nv_bfloat16>(hk->bits, pk, pv, s);
+    return dtype == TQ_F32 ? dispatch_vec_pair<64, float>(hk->bits, pk, pv, s)
+                           : dispatch_vec_pair<64, __nv_bfloat16>(hk->bits, pk, pv, s);
+  }
+  st = tq_quantize_kv_scatter(hk, xk, dtype, n, ld, pos, pos_period, pos_offset, apply_rope, k_codes, k_signs, k_norms,
+                              out_rows, n_records, stream);
+  if (st != TQ_OK) return st;
+  return tq_quantize_kv_scatter(hv, xv, dtype, n, ld, nullptr, 1, 0, 0, v_codes, v_signs, v_norms, out_rows,
+                                n_records, stream);
 }

@@ -61,6 +61,10 @@ def _load():
                                        c_i, c_i, c_i64, c_f, c_p, c_p, c_sz, c_p]),
         "tq_encoder_workspace_size": (c_sz, [c_p, c_i, c_i, c_i]),
         "tq_quantize_dense": (c_i, [c_p, c_p, c_i64, c_i64, c_p, c_p, c_p, c_p, c_sz, c_p]),
+        "tq_quantize_kv_scatter": (c_i, [c_p, c_p, c_i, c_i64, c_i64, c_p, c_i64, c_i64, c_i, c_p, c_p, c_p, c_p,
+                                         c_i64, c_p]),
+        "tq_quantize_kv_pair_scatter": (c_i, [c_p, c_p, c_p, c_p, c_i, c_i64, c_i64, c_p, c_i64, c_i64, c_i,
+                                              c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_p]),
         "tq_quantize_dense_workspace_size": (c_sz, [c_p, c_i64]),
         "tq_search_topk": (c_i, [c_p, c_p, c_i, c_p, c_p, c_p, c_i64, c_i, c_p, c_p, c_p, c_sz, c_p]),
         "tq_search_workspace_size": (c_sz, [c_p, c_i, c_i64, c_i]),
@@ -261,6 +265,69 @@ def quantize_kv_pair(rot_k: Rotation, xk, rot_v: Rotation, xv, *, pos=None, pos_
                                     period, pos_offset, 1 if apply_rope else 0, _ptr(out_k[0]), _ptr(out_k[1]),
                                     _ptr(out_k[2]), _ptr(out_v[0]), _ptr(out_v[1]), _ptr(out_v[2]), out_stride,
                                     _stream_ptr(stream)), "tq_quantize_kv_pair")
+    return out_k, out_v
+
+
+def _rows_of(x, d):
+    x2 = x.reshape(-1, d)
+    if x2.stride(-1) != 1:
+        raise ValueError("x rows must be contiguous")
+    return x2, (x2.stride(0) if x2.shape[0] > 1 else d)
+
+
+def _record_count(cache):
+    codes, signs, norms = cache
+    for t in cache:
+        if not t.is_contiguous():
+            raise ValueError("record arrays must be contiguous")
+    n = codes.numel() // codes.shape[-1]
+    if signs.numel() // signs.shape[-1] != n or norms.numel() // 2 != n:
+        raise ValueError("codes, signs and norms must hold the same number of records")
+    return n
+
+
+def quantize_kv_scatter(rot: Rotation, x, out_rows, out, *, pos=None, pos_period: int | None = None,
+                        pos_offset: int = 0, apply_rope: bool = False, stream=None):
+    """Encode the rows of ``x`` ([n, d] or [..., d]) into records
+    ``out_rows[i]`` (int64 device tensor [n]) of the arrays ``out`` (codes,
+    signs, norms of any shape [..., record]); rows whose target lies outside
+    the arrays are skipped.  Returns ``out``."""
+    d = x.shape[-1]
+    x2, ld = _rows_of(x, d)
+    n = x2.shape[0]
+    rows = out_rows.contiguous()
+    if rows.dtype != __import__("torch").int64 or rows.numel() != n:
+        raise ValueError("out_rows must be int64 with one entry per row")
+    period = pos_period if pos_period is not None else max(n, 1)
+    _check(_lib.tq_quantize_kv_scatter(rot.handle, _ptr(x2), _dtype_code(x2), n, ld, _ptr(pos), period, pos_offset,
+                                       1 if apply_rope else 0, _ptr(out[0]), _ptr(out[1]), _ptr(out[2]), _ptr(rows),
+                                       _record_count(out), _stream_ptr(stream)), "tq_quantize_kv_scatter")
+    return out
+
+
+def quantize_kv_pair_scatter(rot_k: Rotation, xk, rot_v: Rotation, xv, out_rows, out_k, out_v, *, pos=None,
+                             pos_period: int | None = None, pos_offset: int = 0, apply_rope: bool = False,
+                             stream=None):
+    """Keys (RoPE as in quantize_kv) and values into records ``out_rows[i]``
+    of ``out_k`` and ``out_v`` (one launch for up to 256 rows)."""
+    d = xk.shape[-1]
+    k2, ld = _rows_of(xk, d)
+    v2, ldv = _rows_of(xv, d)
+    if k2.shape != v2.shape or k2.dtype != v2.dtype or ld != ldv:
+        raise ValueError("keys and values must share shape, dtype and row stride")
+    n = k2.shape[0]
+    rows = out_rows.contiguous()
+    if rows.dtype != __import__("torch").int64 or rows.numel() != n:
+        raise ValueError("out_rows must be int64 with one entry per row")
+    nrec = _record_count(out_k)
+    if _record_count(out_v) != nrec:
+        raise ValueError("key and value arrays must hold the same number of records")
+    period = pos_period if pos_period is not None else max(n, 1)
+    _check(_lib.tq_quantize_kv_pair_scatter(rot_k.handle, _ptr(k2), rot_v.handle, _ptr(v2), _dtype_code(k2), n, ld,
+                                            _ptr(pos), period, pos_offset, 1 if apply_rope else 0, _ptr(out_k[0]),
+                                            _ptr(out_k[1]), _ptr(out_k[2]), _ptr(out_v[0]), _ptr(out_v[1]),
+                                            _ptr(out_v[2]), _ptr(rows), nrec, _stream_ptr(stream)),
+           "tq_quantize_kv_pair_scatter")
     return out_k, out_v
 
 
