@@ -65,6 +65,10 @@ extern "C" {
 #define TQ_F32           0   /* float32 elements */
 #define TQ_BF16          1   /* bfloat16 elements */
 
+/* Residual correction of a handle ([TurboQuant] Étape 2 / [TurboESM] §2.D). */
+#define TQ_RES_QJL       0   /* sign(S r) and ||r||; estimator sqrt(pi/2)/m   */
+#define TQ_RES_SIGN      1   /* sign(r) and mean |r_i|; x~ = x^ + e sign(r)   */
+
 typedef struct tq_rotation tq_rotation;
 
 /* Human-readable text for a status code (static storage). */
@@ -144,14 +148,32 @@ int tq_rotation_draws(int d, int kind, uint64_t seed, int m, int8_t* signs,
                       double* gauss_pi, float* gauss_s);
 
 /*
- * tq_build_rotation_seeded - tq_build_rotation from a 64-bit seed: the
+ * tq_build_rotation_seeded - tq_build_rotation_ex from a 64-bit seed: the
  * handle built from the draws tq_rotation_draws(d, kind, seed, m, ...)
- * returns, identical to passing those draws to tq_build_rotation.  The other
- * arguments and the statuses are those of tq_build_rotation.
+ * returns, identical to passing those draws to tq_build_rotation_ex with the
+ * same residual mode.  Other arguments and statuses as tq_build_rotation.
  */
-int tq_build_rotation_seeded(int d, int code_bits, int kind, uint64_t seed,
-                             int m, double rope_base, int64_t rope_max_pos,
-                             tq_rotation** out);
+int tq_build_rotation_seeded(int d, int code_bits, int kind, int residual,
+                             uint64_t seed, int m, double rope_base,
+                             int64_t rope_max_pos, tq_rotation** out);
+
+/*
+ * tq_build_rotation_ex - tq_build_rotation with a choice of residual
+ * correction.  residual = TQ_RES_QJL is tq_build_rotation.  residual =
+ * TQ_RES_SIGN keeps one sign bit per rotated residual coordinate and the mean
+ * residual magnitude e = ||r||_1 / d in place of ||r|| ([TurboESM] §2.D: the
+ * residual is corrected as x~ = x^ + e sign(r); the page calibrates e, here
+ * each vector's own mean magnitude is stored).  Such a handle holds S = I
+ * (gauss_s is ignored and may be NULL) and the estimator constant 1, so every
+ * entry point scores and accumulates sign(r) against q~ itself:
+ *   score = ||x|| <q~, c[idx]> + e <q~, 2z - 1>.
+ * Records keep the same layout (the signs array holds sign(r), norms[1] e).
+ * Other arguments and statuses as tq_build_rotation.
+ */
+int tq_build_rotation_ex(int d, int code_bits, int kind, int residual,
+                         const int8_t* signs, const double* gauss_pi,
+                         const float* gauss_s, int m, double rope_base,
+                         int64_t rope_max_pos, tq_rotation** out);
 
 /* Release a handle and its device memory (NULL is accepted). */
 int tq_free_rotation(tq_rotation* h);

@@ -1137,7 +1137,7 @@ int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64
 // records [BH G][2 + 2 kD].
 int launch_merge(int G, int BH, const float* partial, int n_parts, int64_t bh_stride, int64_t part_stride,
                  const tq_rotation* hv, float* out, bool final_out, cudaStream_t s) {
-  const float qjl = static_cast<float>(kQjlConst / hv->m);
+  const float qjl = static_cast<float>(hv->res_const);
   const size_t fsb = static_cast<size_t>(n_parts) * G * sizeof(float);
 #define TQ_MERGE(GG)                                                                                                \
   return final_out ? launch_pdl(decode_merge_kernel<GG, true>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts,  \
@@ -1287,7 +1287,7 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   p.score_scale = score_scale;
   p.one_h = kOneH2;
   p.one_b = kOneB2;
-  p.qjl = static_cast<float>(kQjlConst / hk->m);
+  p.qjl = static_cast<float>(hk->res_const);
   for (int i = 0; i < 4; ++i) {
     p.walsh_k[i] = static_cast<float>(hk->walsh[i]);
     p.walsh_v[i] = static_cast<float>(hv->walsh[i]);

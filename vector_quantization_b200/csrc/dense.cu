@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(256) dense_quantize_rows_kernel(const float* _
                                                                   __nv_bfloat16* __restrict__ rl,
                                                                   const float* __restrict__ thresholds,
                                                                   const float* __restrict__ levels,
-                                                                  uint32_t* __restrict__ codes, float2* __restrict__ norms) {
+                                                                  uint32_t* __restrict__ codes, float2* __restrict__ norms,
+                                                                  int sign_res) {
   constexpr int NT = (1 << BITS) - 1;
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(256) dense_quantize_rows_kernel(const float* _
     const __nv_bfloat16 h = __float2bfloat16_rn(r);
     rh[row * d + 32 * w + lane] = h;
     rl[row * d + 32 * w + lane] = __float2bfloat16_rn(r - __bfloat162float(h));
-    rr = fmaf(r, r, rr);
+    rr = sign_res ? rr + fabsf(r) : fmaf(r, r, rr);   // sign-residual handles keep mean |r_i|
 #pragma unroll
     for (int k = 0; k < BITS; ++k) {
       const uint32_t bits = __ballot_sync(0xffffffffu, (c >> k) & 1);
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(256) dense_quantize_rows_kernel(const float* _
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
-  if (lane == 0) norms[row] = make_float2(norm, sqrtf(rr));
+  if (lane == 0) norms[row] = make_float2(norm, sign_res ? rr / static_cast<float>(d) : sqrtf(rr));
 }
 
 // One warp per row: sign bits of P = R S^T.
@@ -226,10 +227,11 @@ extern "C" int tq_quantize_dense(const tq_rotation* h, const float* x, int64_t n
     float2* nw = reinterpret_cast<float2*>(norms) + r0;
     __nv_bfloat16* rh = reinterpret_cast<__nv_bfloat16*>(xh);
     __nv_bfloat16* rl = reinterpret_cast<__nv_bfloat16*>(xl);
+    const int sres = h->residual == TQ_RES_SIGN ? 1 : 0;
     switch (h->bits) {
-      case 1: dense_quantize_rows_kernel<1><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw); break;
-      case 2: dense_quantize_rows_kernel<2><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw); break;
-      default: dense_quantize_rows_kernel<3><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw); break;
+      case 1: dense_quantize_rows_kernel<1><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw, sres); break;
+      case 2: dense_quantize_rows_kernel<2><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw, sres); break;
+      default: dense_quantize_rows_kernel<3><<<blocks, 256, 0, s>>>(x + r0 * ld, ld, rows, d, yr, rh, rl, h->d_thresholds, h->d_levels, cw, nw, sres); break;
     }
     if ((st = tq::launch_status()) != TQ_OK) return st;
     if ((st = tq::tc_gemm_split(static_cast<int>(rows), m, d, xh, xl, d, h->d_s_bf16, nullptr, d, yr, m, s)) != TQ_OK)

@@ -30,6 +30,7 @@ struct EncodeParams {
   int64_t out_stride;
   const int64_t* out_rows;  // [n] record of each row (scatter calls), or null: row * out_stride
   int64_t n_records;        // records in the output arrays (scatter calls: targets outside are skipped)
+  int sign_res;             // sign-residual handle: norms[1] = mean |r_i| instead of ||r|| (S is the identity)
   const float* dsigns;  // [D]
   const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
   const uint16_t* hd_op; // tensor-core encode: H D in the same layout (fp16 bits when split, else bf16)
@@ -155,7 +156,7 @@ __device__ __forceinline__ void encode_vec_body(const EncodeParams& p) {
     const uint32_t word = __ballot_sync(0xffffffffu, bits[k]);
     if (lane == 0) crec[k * NW + w] = word;
   }
-  float rr = r * r;
+  float rr = p.sign_res ? fabsf(r) : r * r;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
   if (lane == 0) red[1][w] = rr;
@@ -178,7 +179,7 @@ __device__ __forceinline__ void encode_vec_body(const EncodeParams& p) {
     rr = 0.f;
 #pragma unroll
     for (int q = 0; q < NW; ++q) rr += red[1][q];
-    p.norms[rec] = make_float2(nrm, sqrtf(rr));
+    p.norms[rec] = make_float2(nrm, p.sign_res ? rr * (1.f / D) : sqrtf(rr));
   }
 }
 
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
           for (int t = 0; t < NT; ++t) ci += (y >= thr[t]) ? 1 : 0;
           idx[c][j] = ci;
           r[c][j] = keep ? nrm[c] * (y - lev_s[ci]) : 0.f;
-          rr[c] = fmaf(r[c][j], r[c][j], rr[c]);
+          rr[c] = p.sign_res ? rr[c] + fabsf(r[c][j]) : fmaf(r[c][j], r[c][j], rr[c]);
         }
       }
 #pragma unroll
@@ -392,7 +393,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_hadamard_kernel(EncodePara
                 if (lane == k * NJ + j) crec[k * NJ + j] = w;
               }
             }
-            if (lane == 0) p.norms[rec] = make_float2(nrm[c], sqrtf(rr[c]));
+            if (lane == 0) p.norms[rec] = make_float2(nrm[c], p.sign_res ? rr[c] * (1.f / D) : sqrtf(rr[c]));
           } else if (lane == 0) {
             p.norms[rec] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
           }
@@ -708,12 +709,20 @@ __global__ void __launch_bounds__(kRowThreads, 1) encode_rows_kernel(EncodeParam
 #pragma unroll
         for (int k = 0; k < BITS; ++k) words[k][j] = w[k];
       }
+      if (p.sign_res) {   // mean |r_i| in place of ||r||
+        float ra = 0.f;
+#pragma unroll
+        for (int i = 0; i < D; ++i) ra += fabsf(u[i]);
+        rr = ra * (1.f / D);
+      } else {
+        rr = sqrtf(rr);
+      }
       uint32_t* crec = p.codes + row * p.out_stride * (BITS * NJ);   // 4-byte aligned records
 #pragma unroll
       for (int k = 0; k < BITS; ++k)
 #pragma unroll
         for (int j = 0; j < NJ; ++j) crec[k * NJ + j] = words[k][j];
-      p.norms[row * p.out_stride] = make_float2(nrm, sqrtf(rr));
+      p.norms[row * p.out_stride] = make_float2(nrm, rr);
     } else {
 #pragma unroll
       for (int i = 0; i < D; ++i) u[i] = 0.f;
@@ -1125,6 +1134,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     uint32_t w0[BITS], w1[BITS];
     float rr = quantize32_x2<BITS>(u, tp, nl, nv, w0);        // coordinates 64 c4 .. + 31: word 2 c4
     rr += quantize32_x2<BITS>(u + 16, tp, nl, nv, w1);        // 64 c4 + 32 ..: word 2 c4 + 1
+    if (p.sign_res) {   // sum of |r_i| over this thread's 64 coordinates in place of sum r_i^2
+      float2 ra = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int m = 0; m < 32; ++m) ra = __fadd2_rn(ra, make_float2(fabsf(u[m].x), fabsf(u[m].y)));
+      rr = ra.x + ra.y;
+    }
     xrr[g][c4][r4] = rr;
     if (valid && ok_y) {
       constexpr int NJ = 4;
@@ -1171,7 +1186,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
                           tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), ids, true);
       tqtc::mma_commit(&mb_s[g]);
     }
-    if (valid && ok_y && c4 == 0) p.norms[row * p.out_stride] = make_float2(nrm, sqrtf(rr + xrr[g][1][r4]));
+    if (valid && ok_y && c4 == 0)
+      p.norms[row * p.out_stride] =
+          make_float2(nrm, p.sign_res ? (rr + xrr[g][1][r4]) * (1.f / D) : sqrtf(rr + xrr[g][1][r4]));
     const bool ok = ok_y && tqtc::mbar_wait(&mb_s[g], ph_s, kWaitLimit);
     ph_s ^= 1;
     tqtc::fence_after_sync();
@@ -1349,6 +1366,7 @@ int make_encode_params(const tq_rotation* h, const void* x, int dtype, int64_t n
   p.out_stride = out_stride;
   p.out_rows = out_rows;
   p.n_records = n_records;
+  p.sign_res = h->residual == TQ_RES_SIGN ? 1 : 0;
   p.dsigns = h->d_signs;
   p.s_op = h->d_s_op;
   // H D for the tensor-core encode: fp16 when the rows are split (RoPE or fp32 input), else bf16

@@ -1128,10 +1128,10 @@ extern "C" int tq_encoder_attention(const tq_rotation* hk, const tq_rotation* hv
   p.Hq = Hq;
   p.G = Hq / Hkv;
   p.score_scale = scale * 1.4426950408889634f;
-  p.qjl_k = static_cast<float>(kQjlConst / hk->m);
+  p.qjl_k = static_cast<float>(hk->res_const);
   p.one_h = kOneH2;
   p.one_b = kOneB2;
-  p.qjl_v = static_cast<float>(kQjlConst / hv->m);
+  p.qjl_v = static_cast<float>(hv->res_const);
   for (int i = 0; i < 4; ++i) {
     p.walsh_k[i] = static_cast<float>(hk->walsh[i]);
     p.walsh_v[i] = static_cast<float>(hv->walsh[i]);

@@ -438,7 +438,7 @@ extern "C" int tq_search_topk(const tq_rotation* h, const float* queries, int nq
   p.nblk = d / 128;
   p.qfrag = reinterpret_cast<const uint32_t*>(ws + L.frag);
   p.qconst = reinterpret_cast<const float4*>(ws + L.qconst);
-  p.qjl = static_cast<float>(kQjlConst / m);
+  p.qjl = static_cast<float>(h->res_const);
   for (int i = 0; i < 4; ++i) p.walsh[i] = static_cast<float>(h->walsh[i]);
   p.one_h = kOneH2;
   p.cand_score = reinterpret_cast<float*>(ws + L.cs);

@@ -338,12 +338,13 @@ int tq_lloyd_max(int d, int bits, double* levels, double* thresholds) {
   return TQ_OK;
 }
 
-int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
-                      const double* gauss_pi, const float* gauss_s, int m,
-                      double rope_base, int64_t rope_max_pos, tq_rotation** out) {
+int tq_build_rotation_ex(int d, int code_bits, int kind, int residual, const int8_t* signs,
+                         const double* gauss_pi, const float* gauss_s, int m, double rope_base,
+                         int64_t rope_max_pos, tq_rotation** out) {
   if (!out) return TQ_EINVAL;
   *out = nullptr;
-  if (code_bits < 1 || code_bits > 3 || m != d || !gauss_s) return TQ_EINVAL;
+  if (residual != TQ_RES_QJL && residual != TQ_RES_SIGN) return TQ_EINVAL;
+  if (code_bits < 1 || code_bits > 3 || m != d || (residual == TQ_RES_QJL && !gauss_s)) return TQ_EINVAL;
   if (kind == TQ_ROT_HADAMARD) {
     if (!signs) return TQ_EINVAL;
     if (d != 64 && d != 128) return TQ_EUNSUPPORTED;
@@ -365,6 +366,10 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
   h->m = m;
   h->bits = code_bits;
   h->kind = kind;
+  h->residual = residual;
+  // QJL: E[sign(s.r) s] = sqrt(2/pi) r/||r|| for Gaussian rows s, hence the
+  // sqrt(pi/2)/m estimator; the sign correction adds e_bar sign(r) as it is.
+  h->res_const = residual == TQ_RES_QJL ? kQjlConst / m : 1.0;
   h->rope_base = rope_base;
   h->rope_max_pos = rope_base > 0.0 ? rope_max_pos : 0;
 
@@ -420,7 +425,9 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
     std::vector<float> s(static_cast<size_t>(m) * d), stt(static_cast<size_t>(d) * m);
     for (int j = 0; j < m; ++j)
       for (int i = 0; i < d; ++i) {
-        const float v = round_to_bf16(gauss_s[static_cast<size_t>(j) * d + i]);
+        // the sign correction keeps the residual's own coordinates: S = I
+        const float v = residual == TQ_RES_SIGN ? (i == j ? 1.f : 0.f)
+                                                : round_to_bf16(gauss_s[static_cast<size_t>(j) * d + i]);
         s[static_cast<size_t>(j) * d + i] = v;
         stt[static_cast<size_t>(i) * m + j] = v;
       }
@@ -471,7 +478,7 @@ int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs,
         // coordinate, K = slot k standing for coordinate dim(k)
         auto slot_dim = [](int k) { return 32 * (k >> 5) + ((k >> 1) & 15) + 16 * (k & 1); };
         auto had = [](int i, int j) { return (__builtin_popcount(static_cast<unsigned>(i & j)) & 1) ? -1.0 : 1.0; };
-        const double qjl = kQjlConst / m;
+        const double qjl = h->res_const;
         std::vector<uint16_t> ep(static_cast<size_t>(3) * d * d);
         for (int i = 0; i < d; ++i)
           for (int k = 0; k < d; ++k) {
@@ -538,7 +545,13 @@ int tq_rotation_draws(int d, int kind, uint64_t seed, int m, int8_t* signs, doub
   return TQ_OK;
 }
 
-int tq_build_rotation_seeded(int d, int code_bits, int kind, uint64_t seed, int m, double rope_base,
+int tq_build_rotation(int d, int code_bits, int kind, const int8_t* signs, const double* gauss_pi,
+                      const float* gauss_s, int m, double rope_base, int64_t rope_max_pos, tq_rotation** out) {
+  return tq_build_rotation_ex(d, code_bits, kind, TQ_RES_QJL, signs, gauss_pi, gauss_s, m, rope_base, rope_max_pos,
+                              out);
+}
+
+int tq_build_rotation_seeded(int d, int code_bits, int kind, int residual, uint64_t seed, int m, double rope_base,
                              int64_t rope_max_pos, tq_rotation** out) {
   if (!out) return TQ_EINVAL;
   *out = nullptr;
@@ -549,8 +562,8 @@ int tq_build_rotation_seeded(int d, int code_bits, int kind, uint64_t seed, int 
   std::vector<double> gp(kind == TQ_ROT_DENSE ? static_cast<size_t>(d) * d : 0);
   const int st = tq_rotation_draws(d, kind, seed, m, sg.data(), gp.empty() ? nullptr : gp.data(), gs.data());
   if (st != TQ_OK) return st;
-  return tq_build_rotation(d, code_bits, kind, sg.data(), gp.empty() ? nullptr : gp.data(), gs.data(), m, rope_base,
-                           rope_max_pos, out);
+  return tq_build_rotation_ex(d, code_bits, kind, residual, sg.data(), gp.empty() ? nullptr : gp.data(), gs.data(), m,
+                              rope_base, rope_max_pos, out);
 }
 
 int tq_free_rotation(tq_rotation* h) {

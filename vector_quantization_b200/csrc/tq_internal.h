@@ -14,6 +14,10 @@
 struct tq_rotation {
   int device = 0;
   int d = 0, m = 0, bits = 0, kind = 0;
+  // Residual correction: TQ_RES_QJL (sign(S r), ||r||, constant sqrt(pi/2)/m)
+  // or TQ_RES_SIGN (sign(r), mean |r_i|, constant 1: S is the identity).
+  int residual = 0;
+  double res_const = 0.0;
   double rope_base = 0.0;
   int64_t rope_max_pos = 0;
   int rope_hi_rows = 0;                 // rows of the coarse RoPE table

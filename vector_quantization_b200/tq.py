@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libtq.so")
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EWORKSPACE, TQ_ECUDA, TQ_ENOMEM = 0, -1, -2, -3, -4, -5
 TQ_ROT_HADAMARD, TQ_ROT_DENSE = 0, 1
 TQ_F32, TQ_BF16 = 0, 1
+TQ_RES_QJL, TQ_RES_SIGN = 0, 1
 
 
 class TQError(RuntimeError):
@@ -38,7 +39,8 @@ def _load():
         "tq_version": (c_i, []),
         "tq_lloyd_max": (c_i, [c_i, c_i, c_p, c_p]),
         "tq_build_rotation": (c_i, [c_i, c_i, c_i, c_p, c_p, c_p, c_i, c_d, c_i64, ctypes.POINTER(c_p)]),
-        "tq_build_rotation_seeded": (c_i, [c_i, c_i, c_i, ctypes.c_uint64, c_i, c_d, c_i64, ctypes.POINTER(c_p)]),
+        "tq_build_rotation_seeded": (c_i, [c_i, c_i, c_i, c_i, ctypes.c_uint64, c_i, c_d, c_i64, ctypes.POINTER(c_p)]),
+        "tq_build_rotation_ex": (c_i, [c_i, c_i, c_i, c_i, c_p, c_p, c_p, c_i, c_d, c_i64, ctypes.POINTER(c_p)]),
         "tq_rotation_draws": (c_i, [c_i, c_i, ctypes.c_uint64, c_i, c_p, c_p, c_p]),
         "tq_free_rotation": (c_i, [c_p]),
         "tq_rotation_export": (c_i, [c_p, c_p, c_p, c_p, c_p]),
@@ -154,11 +156,12 @@ class Rotation:
     from which the library draws them itself (tq_build_rotation_seeded)."""
 
     def __init__(self, d: int, bits: int, randomness, kind: str = "hadamard",
-                 rope_base: float = 0.0, rope_max_pos: int = 1 << 21):
+                 rope_base: float = 0.0, rope_max_pos: int = 1 << 21, residual: str = "qjl"):
         kind_code = {"hadamard": TQ_ROT_HADAMARD, "dense": TQ_ROT_DENSE}[kind]
+        res_code = {"qjl": TQ_RES_QJL, "sign": TQ_RES_SIGN}[residual]
         h = ctypes.c_void_p()
         if isinstance(randomness, (int, np.integer)):
-            _check(_lib.tq_build_rotation_seeded(d, bits, kind_code, int(randomness) & (2**64 - 1), d,
+            _check(_lib.tq_build_rotation_seeded(d, bits, kind_code, res_code, int(randomness) & (2**64 - 1), d,
                                                  float(rope_base), int(rope_max_pos), ctypes.byref(h)),
                    "tq_build_rotation_seeded")
         else:
@@ -166,10 +169,10 @@ class Rotation:
             gs = np.ascontiguousarray(randomness["gauss_s"], dtype=np.float32)
             gp = randomness.get("gauss_pi")
             gp = None if gp is None else np.ascontiguousarray(gp, dtype=np.float64)
-            _check(_lib.tq_build_rotation(d, bits, kind_code, signs.ctypes.data,
-                                          None if gp is None else gp.ctypes.data, gs.ctypes.data, gs.shape[0],
-                                          float(rope_base), int(rope_max_pos), ctypes.byref(h)),
-                   "tq_build_rotation")
+            _check(_lib.tq_build_rotation_ex(d, bits, kind_code, res_code, signs.ctypes.data,
+                                             None if gp is None else gp.ctypes.data, gs.ctypes.data, gs.shape[0],
+                                             float(rope_base), int(rope_max_pos), ctypes.byref(h)),
+                   "tq_build_rotation_ex")
         self._h = h
         dd, mm, bb = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
         cb, sb = ctypes.c_int64(), ctypes.c_int64()
@@ -178,6 +181,7 @@ class Rotation:
         self.d, self.m, self.bits = dd.value, mm.value, bb.value
         self.code_bytes, self.sign_bytes = cb.value, sb.value
         self.kind = kind
+        self.residual = residual
         self.rope_base = rope_base
 
     @property
