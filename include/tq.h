@@ -401,6 +401,34 @@ int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
                         const int32_t* seq_lens, float scale, float* out,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * tq_decode_attention_append - one decode step with the new token's key and
+ * value appended to the caches first, in the same launch as the query
+ * preparation: [NSNQuant] §4 ("Résidus": quantize the new token and append
+ * it), then tq_decode_attention over caches that now hold it.
+ *   k_new, v_new  device [B*Hkv, d] rows in q_dtype, row b*Hkv + j the new
+ *               key / value of sequence b, KV head j; the key takes RoPE at
+ *               position q_pos[b] (when hk has RoPE)
+ *   k_codes .. v_norms  the caches (written: record len_b - 1 of each
+ *               sequence, len_b = seq_lens[b] or T, which counts the new
+ *               token; nothing is written where len_b is 0 or outside 0..T)
+ *   other arguments and the workspace as tq_decode_attention
+ * Same result as tq_quantize_kv_pair of the new rows into those records
+ * followed by tq_decode_attention.  Returns TQ_OK, TQ_EINVAL,
+ * TQ_EUNSUPPORTED, TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_decode_attention_append(const tq_rotation* hk, const tq_rotation* hv,
+                               const void* q, int q_dtype,
+                               const int64_t* q_pos, const void* k_new,
+                               const void* v_new, uint8_t* k_codes,
+                               uint8_t* k_signs, float* k_norms,
+                               uint8_t* v_codes, uint8_t* v_signs,
+                               float* v_norms, int64_t cache_stride, int B,
+                               int Hq, int Hkv, int64_t T,
+                               const int32_t* seq_lens, float scale,
+                               float* out, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Workspace bytes tq_decode_attention needs for these sizes (0 if invalid). */
 size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
                                 int B, int Hq, int Hkv, int64_t T);
@@ -489,7 +517,9 @@ int tq_decode_partials(const tq_rotation* hk, const tq_rotation* hv,
  *   hv          value handle (d = 128, Hadamard)
  *   partials    device [n_parts][B*Hq][2 + 2*d] float32 (part-major, e.g.
  *               the all-gather of every rank's tq_decode_partials output)
- *   n_parts     1 .. 65536
+ *   n_parts     1 .. 65536; the merge keeps n_parts * G floats of weights
+ *               in shared memory, so TQ_EUNSUPPORTED past the device's
+ *               per-block limit (about 5,900 parts at G = 8 on B200)
  *   B, Hq, Hkv  as in tq_decode_attention
  *   out         device [B, Hq, d] float32
  * Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED or TQ_ECUDA.

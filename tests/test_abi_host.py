@@ -73,6 +73,9 @@ def test_bad_arguments_are_rejected_on_host():
                                               None) == tq.TQ_EINVAL
     assert tq._lib.tq_decode_attention(None, None, None, 0, None, None, None, None, None, None, None, 0,
                                        1, 4, 1, 0, None, 0.125, None, None, 0, None) == tq.TQ_EINVAL
+    # fused append: missing new rows or handles rejected on the host
+    assert tq._lib.tq_decode_attention_append(None, None, None, 0, None, None, None, None, None, None, None, None,
+                                              None, 0, 1, 4, 1, 1, None, 0.125, None, None, 0, None) == tq.TQ_EINVAL
 
 
 def test_window_binding_checks_shapes_before_any_call():

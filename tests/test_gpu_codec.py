@@ -71,9 +71,9 @@ def test_encode_parity(cuda_device, d, bits, dtype):
 @pytest.mark.parametrize("bits", [1, 2, 3])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_encode_parity_large_batch(cuda_device, d, bits, dtype):
-    """Batches of 16384 or more vectors take the 128-row tile kernels (the
-    tensor-core rotation kernel for d = 128, the row kernel for d = 64):
-    several tiles per CTA group and a ragged last tile."""
+    """Batches of 16384 or more vectors take the tensor-core rotation kernel
+    (128-row tiles, d = 64 and 128): several tiles per CTA group and a ragged
+    last tile."""
     _run_encode(d, bits, 16384 + 1031, dtype, rope=True, seed=200 + bits)
 
 
@@ -90,31 +90,35 @@ def test_encode_small_batch_positions_array_strided(cuda_device):
     _run_encode(128, 3, 128, torch.bfloat16, rope=True, seed=230, offset=77, pos_array=True, out_stride=5)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("bits", [1, 2, 3])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_encode_parity_large_batch_no_rope(cuda_device, bits, dtype):
+def test_encode_parity_large_batch_no_rope(cuda_device, d, bits, dtype):
     """Large batches without RoPE: bf16 rows go to the tensor core as they
     are staged, fp32 rows through the fp16 hi/lo split."""
-    _run_encode(128, bits, 2 * 16384 + 389, dtype, rope=False, seed=250 + bits)
+    _run_encode(d, bits, 2 * 16384 + 389, dtype, rope=False, seed=250 + bits)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_encode_large_batch_far_positions(cuda_device, dtype):
-    """Two-thread kernel at the top of its RoPE range: positions up to
+def test_encode_large_batch_far_positions(cuda_device, d, dtype):
+    """Tensor-core kernel at the top of its RoPE range: positions up to
     2^22 - 1, where pos * theta_0 needs the widest reduction by 2 pi."""
     n = 16384 + 259
-    _run_encode(128, 2, n, dtype, rope=True, seed=240, offset=(1 << 22) - n, max_pos=1 << 22)
+    _run_encode(d, 2, n, dtype, rope=True, seed=240, offset=(1 << 22) - n, max_pos=1 << 22)
 
 
-def test_encode_large_batch_positions_past_reduction_range(cuda_device):
+@pytest.mark.parametrize("d", [64, 128])
+def test_encode_large_batch_positions_past_reduction_range(cuda_device, d):
     """A handle whose positions may pass 2^22 takes the table-driven kernel."""
     n = 16384 + 3
-    _run_encode(128, 3, n, torch.bfloat16, rope=True, seed=241, offset=(1 << 22) + 100,
+    _run_encode(d, 3, n, torch.bfloat16, rope=True, seed=241, offset=(1 << 22) + 100,
                 max_pos=(1 << 22) + 100 + n)
 
 
-def test_encode_large_batch_positions_array_strided(cuda_device):
-    _run_encode(128, 2, 16384 + 77, torch.bfloat16, rope=True, seed=210, period=5000, offset=3,
+@pytest.mark.parametrize("d", [64, 128])
+def test_encode_large_batch_positions_array_strided(cuda_device, d):
+    _run_encode(d, 2, 16384 + 77, torch.bfloat16, rope=True, seed=210, period=5000, offset=3,
                 pos_array=True, out_stride=2)
 
 

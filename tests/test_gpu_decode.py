@@ -71,6 +71,14 @@ def test_decode_parity_lengths(cuda_device, T):
     assert_close(gpu, ref, what=f"T={T}")
 
 
+def test_decode_one_sequence_many_splits(cuda_device):
+    """One sequence with one KV head and 8 query heads over 80000 tokens:
+    313 splits, whose merge weights (10 KB) take the merge kernel past the
+    default 48 KB of shared memory."""
+    out, ref = run_decode(2, 8, 80000, B=1, Hkv=1, seed=7)
+    assert_close(out, ref, what="G 8, 313 splits")
+
+
 def test_decode_bf16_query(cuda_device):
     gpu, ref = run_decode(2, 4, 777, q_dtype=torch.bfloat16, seed=3)
     assert_close(gpu, ref)

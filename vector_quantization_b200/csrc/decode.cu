@@ -36,6 +36,7 @@
 #include <mutex>
 
 #include "bitplane.cuh"
+#include "encode_vec.cuh"
 #include "tcgen05.cuh"
 #include "tq_internal.h"
 
@@ -71,6 +72,7 @@ struct DecodeParams {
   uint32_t one_h, one_b;   // kOneH2 / kOneB2, passed at run time (see bit_select)
   const int32_t* seq_lens; // [B] tokens of each sequence (<= T), or null: all T
   int Hkv;
+  int append;              // the preceding launch writes each sequence's last record: no copy before its end
 };
 
 
@@ -101,6 +103,27 @@ template <int BITS>
 __device__ __forceinline__ int code_chunk(int tok, int part) {
   if constexpr (BITS == 2) return tok * 2 + (part ^ ((tok >> 2) & 1));
   else return tok * BITS + part;
+}
+
+// Fast Walsh-Hadamard transform (Sylvester order, unnormalised) of one kD
+// vector per group of kD threads, thread i of the group holding coordinate i:
+// five stages by warp shuffles, the two across warps through the group's row
+// of shared memory `buf`.  All groups of the block run it together.
+__device__ __forceinline__ void fwht_group(float& v, int i, float* buf) {
+  const int lane = i & 31;
+#pragma unroll
+  for (int bit = 1; bit < 32; bit <<= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, bit);
+    v = (lane & bit) ? o - v : v + o;
+  }
+#pragma unroll
+  for (int bit = 32; bit < kD; bit <<= 1) {
+    __syncthreads();
+    buf[i] = v;
+    __syncthreads();
+    const float o = buf[i ^ bit];
+    v = (i & bit) ? o - v : v + o;
+  }
 }
 
 template <int BITS, int G>
@@ -144,8 +167,40 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   };
   const int sg_side = lane >> 4, sg_c = lane & 15;
   const int nm_side = (lane >> 3) & 1, nm_c = lane & 7;
+  // Per-lane copy plan of a full tile: sources advance by kWarps tiles per
+  // issue, destinations are fixed offsets within a stage.
+  constexpr int CIT = (CCH + 31) / 32;
+  const int64_t tok0 = seq + t_begin + static_cast<int64_t>(warp) * kTile;
+  const uint8_t* src_code[2][CIT];
+  uint32_t dst_code[2][CIT];
+#pragma unroll
+  for (int side = 0; side < 2; ++side)
+#pragma unroll
+    for (int k = 0; k < CIT; ++k) {
+      const int c = lane + 32 * k;
+      const int cc = c < CCH ? c : 0;
+      src_code[side][k] = (side ? p.v_codes : p.k_codes) + tok0 * CB + cc * 16;
+      dst_code[side][k] = side * HALF + code_chunk<BITS>(cc / BITS, cc % BITS) * 16;
+    }
+  const uint8_t* src_sign = (sg_side ? p.v_signs : p.k_signs) + tok0 * SB + sg_c * 16;
+  const uint32_t dst_sign = sg_side * HALF + kTile * CB + sg_c * 16;
+  const uint8_t* src_norm = reinterpret_cast<const uint8_t*>((nm_side ? p.v_norms : p.k_norms) + tok0) + nm_c * 16;
+  const uint32_t dst_norm = nm_side * HALF + kTile * (CB + SB) + nm_c * 16;
+  constexpr int64_t kStepTok = static_cast<int64_t>(kWarps) * kTile;
+  const int64_t n_full = (t_end - t_begin) / kTile;   // full tiles of the split (t_end >= t_begin or none)
+  const int my_full = t_end > t_begin && n_full > warp ? static_cast<int>((n_full - warp + kWarps - 1) / kWarps) : 0;
   auto issue = [&](int i) {
-    if (i < my_count) {
+    if (i < my_full) {
+      uint8_t* stg = my_stages + (i % kStages) * STAGE;
+      const int64_t adv = kStepTok * i;
+#pragma unroll
+      for (int side = 0; side < 2; ++side)
+#pragma unroll
+        for (int k = 0; k < CIT; ++k)
+          if (lane + 32 * k < CCH) cp_async16(stg + dst_code[side][k], src_code[side][k] + adv * CB, 16);
+      cp_async16(stg + dst_sign, src_sign + adv * SB, 16);
+      if (lane < 16) cp_async16(stg + dst_norm, src_norm + adv * 8, 16);
+    } else if (i < my_count) {
       const int64_t t0 = seq + t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
       const int nv = tile_nv(i);
       uint8_t* stg = my_stages + (i % kStages) * STAGE;
@@ -175,9 +230,15 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   // The first tiles of the cache do not depend on the q-prep launch: start
   // their copies, then wait for q-prep's outputs (programmatic dependent
   // launch; a no-op when launched without it).
+  if (!p.append) {
 #pragma unroll 1
-  for (int i = 0; i < kStages - 1; ++i) issue(i);
+    for (int i = 0; i < kStages - 1; ++i) issue(i);
+  }
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
+  if (p.append) {
+#pragma unroll 1
+    for (int i = 0; i < kStages - 1; ++i) issue(i);
+  }
 
   // The key side's B operand (int8 digits of the query, one set of
   // fragments per MMA group and n-tile) in shared memory, read at each MMA;
@@ -530,26 +591,6 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   }
 }
 
-// Fast Walsh-Hadamard transform (Sylvester order, unnormalised) of one kD
-// vector per group of kD threads, thread i of the group holding coordinate i:
-// five stages by warp shuffles, the two across warps through the group's row
-// of shared memory `buf`.  All groups of the block run it together.
-__device__ __forceinline__ void fwht_group(float& v, int i, float* buf) {
-  const int lane = i & 31;
-#pragma unroll
-  for (int bit = 1; bit < 32; bit <<= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, v, bit);
-    v = (lane & bit) ? o - v : v + o;
-  }
-#pragma unroll
-  for (int bit = 32; bit < kD; bit <<= 1) {
-    __syncthreads();
-    buf[i] = v;
-    __syncthreads();
-    const float o = buf[i ^ bit];
-    v = (i & bit) ? o - v : v + o;
-  }
-}
 
 // One block of G groups of kD threads per (sequence b, KV head); group h is
 // query head h of the group, thread i of it coordinate i: RoPE, q~ = Pi q,
@@ -558,21 +599,44 @@ __device__ __forceinline__ void fwht_group(float& v, int i, float* buf) {
 // [g kD/G, (g + 1) kD/G) of row i of S in registers (loaded before the wait
 // for q, so the loads overlap the previous launch) and forms the partial sums
 // of all G heads over them; the G partials meet in shared memory.
+// Arguments of the query preparation (one block of G x kD threads per
+// sequence bh = b * Hkv + kv).
+template <typename T>
+struct QPrepArgs {
+  const T* q;              // [B Hq][kD]; query head h of the group is row bh * G + h
+  const int64_t* q_pos;    // [B]
+  int Hkv;
+  const float* dsigns;
+  const float* st;
+  const float2* rope_hi;
+  const float2* rope_lo;
+  int64_t rope_max_pos;
+  int rope;
+  WalshWeights walsh;
+  uint32_t* qfrag;
+  float4* kconst;
+};
+
 template <typename T, int G, int BITS>
-__global__ void __launch_bounds__(kD * G) decode_qprep_kernel(const T* __restrict__ q, const int64_t* __restrict__ q_pos,
-                                                             int Hkv, const float* __restrict__ dsigns,
-                                                             const float* __restrict__ st,
-                                                             const float2* __restrict__ rope_hi,
-                                                             const float2* __restrict__ rope_lo, int64_t rope_max_pos,
-                                                             int rope, WalshWeights walsh, uint32_t* __restrict__ qfrag,
-                                                             float4* __restrict__ kconst) {
+__device__ __forceinline__ void qprep_body(const QPrepArgs<T>& a, int bh) {
+  const T* __restrict__ q = a.q;
+  const int64_t* __restrict__ q_pos = a.q_pos;
+  const int Hkv = a.Hkv;
+  const float* __restrict__ dsigns = a.dsigns;
+  const float* __restrict__ st = a.st;
+  const float2* __restrict__ rope_hi = a.rope_hi;
+  const float2* __restrict__ rope_lo = a.rope_lo;
+  const int64_t rope_max_pos = a.rope_max_pos;
+  const int rope = a.rope;
+  const WalshWeights& walsh = a.walsh;
+  uint32_t* __restrict__ qfrag = a.qfrag;
+  float4* __restrict__ kconst = a.kconst;
   constexpr int NT = (G + 3) / 4;
   constexpr int KS = kD / G;   // columns of S per group
   __shared__ __align__(16) float buf[G][kD];
   __shared__ __align__(16) float part[G][G][kD];   // [column group][head][i]
   __shared__ float red[2][G][2][kD / 32];
   const int tid = threadIdx.x, h = tid / kD, i = tid % kD, lane = tid & 31, wg = i >> 5;
-  const int bh = blockIdx.x;   // b * Hkv + kv; query head h of the group is row bh * G + h of q
   const int b = bh / Hkv;
   float scol[KS];
 #pragma unroll
@@ -699,6 +763,52 @@ __global__ void __launch_bounds__(kD * G) decode_qprep_kernel(const T* __restric
     const float ss = (red[1][h][1][0] + red[1][h][1][1]) + (red[1][h][1][2] + red[1][h][1][3]);
     kconst[static_cast<size_t>(bh) * 8 + h] = make_float4(ldexpf(1.f, -E[0]), wsum * cs, ldexpf(1.f, -E[1]), ss);
   }
+}
+
+template <typename T, int G, int BITS>
+__global__ void __launch_bounds__(kD * G) decode_qprep_kernel(const __grid_constant__ QPrepArgs<T> a) {
+  qprep_body<T, G, BITS>(a, blockIdx.x);
+}
+
+// The decode step's append and query preparation in one launch: blocks
+// 0..BH-1 prepare the queries (qprep_body); the others hold G groups of kD
+// threads, each encoding one new row (encode_vec_core) into the record
+// before the end of its sequence: keys (RoPE at the query's position) for
+// vectors e < BH, values after.  [NSNQuant] §4 ("Résidus": quantize and
+// append); [TurboESM] §3 (the record format).
+struct AppendArgs {
+  int BH;
+  int64_t T;
+  const int32_t* seq_lens;   // [B] or null: every sequence holds T tokens (the new one included)
+  int64_t cache_stride;
+};
+
+template <typename T, int G, int BITS>
+__global__ void __launch_bounds__(kD * G) decode_prep_kernel(const __grid_constant__ QPrepArgs<T> a,
+                                                            const __grid_constant__ AppendArgs ap,
+                                                            const __grid_constant__ EncodeParams pk,
+                                                            const __grid_constant__ EncodeParams pv) {
+  if (static_cast<int>(blockIdx.x) < ap.BH) {
+    qprep_body<T, G, BITS>(a, blockIdx.x);
+    return;
+  }
+  __shared__ __align__(16) float gbuf[G][kD];
+  __shared__ float gred[G][2][kD / 32];
+  const int gi = threadIdx.x / kD, i = threadIdx.x % kD;
+  const int64_t e = static_cast<int64_t>(blockIdx.x - ap.BH) * G + gi;
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");   // the cache may be read by the previous launch
+  if (e >= 2 * static_cast<int64_t>(ap.BH)) return;       // uniform over the group
+  const bool is_v = e >= ap.BH;
+  const int64_t sq = is_v ? e - ap.BH : e;                 // sequence b * Hkv + kv
+  const int b = static_cast<int>(sq / a.Hkv);
+  const int64_t len = ap.seq_lens ? ap.seq_lens[b] : ap.T;
+  if (len < 1 || len > ap.T) return;                       // nothing to append to (the decode gives NaN or zeros)
+  const EncodeParams& p = is_v ? pv : pk;
+  const int64_t rec = sq * ap.cache_stride + len - 1;
+  const int64_t pos = p.rope ? a.q_pos[b] : 0;
+  encode_vec_core<kD, BITS, T>(p, i, static_cast<const T*>(p.x) + sq * p.ld, rec, pos, gbuf[gi], gred[gi],
+                               [gi] { asm volatile("bar.sync %0, %1;\n" ::"r"(1 + gi), "r"(kD) : "memory"); },
+                               [&](int k) { return __ldg(p.st + k * kD + i); });
 }
 
 // One block of G groups of kD threads per (sequence b, KV head); group h is
@@ -1095,41 +1205,115 @@ int launch_split(const DecodeParams& p, int BH, cudaStream_t s) {
   return launch_pdl(kern, grid, dim3(kWarps * 32), smem, s, p);
 }
 
+// The decode step's new rows, for the fused append (decode_prep_kernel).
+struct AppendIn {
+  const void* k_new;   // [B Hkv][kD] in the query's dtype, row b * Hkv + kv
+  const void* v_new;
+  const tq_rotation* hv;
+  uint8_t* k_codes;
+  uint8_t* k_signs;
+  float* k_norms;
+  uint8_t* v_codes;
+  uint8_t* v_signs;
+  float* v_norms;
+  int64_t cache_stride;
+  int64_t T;
+  const int32_t* seq_lens;
+};
+
+EncodeParams append_params(const tq_rotation* h, const void* x, int BH, int rope, uint8_t* codes, uint8_t* signs,
+                           float* norms) {
+  EncodeParams p{};
+  p.x = x;
+  p.n = BH;
+  p.ld = kD;
+  p.pos_period = 1;
+  p.rope = rope;
+  p.codes = reinterpret_cast<uint32_t*>(codes);
+  p.signs = reinterpret_cast<uint32_t*>(signs);
+  p.norms = reinterpret_cast<float2*>(norms);
+  p.out_stride = 1;
+  fill_handle_fields(p, h);
+  return p;
+}
+
 template <typename T, int BITS>
-int qprep_g(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
-            uint32_t* qfrag, float4* kconst, cudaStream_t s) {
-  WalshWeights w{};
-  for (int i = 0; i < 4; ++i) w.w[i] = static_cast<float>(hk->walsh[i]);
-#define TQ_QPREP(GG)                                                                                       \
-  return launch_pdl(decode_qprep_kernel<T, GG, BITS>, dim3(BH), dim3(kD * GG), 0, s, q, q_pos, Hkv,        \
-                    hk->d_signs, hk->d_st, hk->d_rope_hi, hk->d_rope_lo, hk->rope_max_pos, rope, w, qfrag, \
-                    kconst)
-  switch (G) {
-    case 1: TQ_QPREP(1);
-    case 2: TQ_QPREP(2);
-    case 4: TQ_QPREP(4);
-    case 8: TQ_QPREP(8);
-  }
+int qprep_g(int G, int BH, const QPrepArgs<T>& a, const AppendIn* app, const tq_rotation* hk, cudaStream_t s) {
+  if (!app) {
+#define TQ_QPREP(GG) return launch_pdl(decode_qprep_kernel<T, GG, BITS>, dim3(BH), dim3(kD * GG), 0, s, a)
+    switch (G) {
+      case 1: TQ_QPREP(1);
+      case 2: TQ_QPREP(2);
+      case 4: TQ_QPREP(4);
+      case 8: TQ_QPREP(8);
+    }
 #undef TQ_QPREP
+    return TQ_EUNSUPPORTED;
+  }
+  const EncodeParams pk = append_params(hk, app->k_new, BH, a.rope, app->k_codes, app->k_signs, app->k_norms);
+  const EncodeParams pv = append_params(app->hv, app->v_new, BH, 0, app->v_codes, app->v_signs, app->v_norms);
+  const AppendArgs ap{BH, app->T, app->seq_lens, app->cache_stride};
+  const unsigned blocks = static_cast<unsigned>(BH + (2 * BH + G - 1) / G);
+#define TQ_PREP(GG) return launch_pdl(decode_prep_kernel<T, GG, BITS>, dim3(blocks), dim3(kD * GG), 0, s, a, ap, pk, pv)
+  switch (G) {
+    case 1: TQ_PREP(1);
+    case 2: TQ_PREP(2);
+    case 4: TQ_PREP(4);
+    case 8: TQ_PREP(8);
+  }
+#undef TQ_PREP
   return TQ_EUNSUPPORTED;
 }
 
 template <typename T>
 int qprep_b(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
-            uint32_t* qfrag, float4* kconst, cudaStream_t s) {
+            uint32_t* qfrag, float4* kconst, const AppendIn* app, cudaStream_t s) {
+  QPrepArgs<T> a{};
+  a.q = q;
+  a.q_pos = q_pos;
+  a.Hkv = Hkv;
+  a.dsigns = hk->d_signs;
+  a.st = hk->d_st;
+  a.rope_hi = hk->d_rope_hi;
+  a.rope_lo = hk->d_rope_lo;
+  a.rope_max_pos = hk->rope_max_pos;
+  a.rope = rope;
+  for (int i = 0; i < 4; ++i) a.walsh.w[i] = static_cast<float>(hk->walsh[i]);
+  a.qfrag = qfrag;
+  a.kconst = kconst;
   switch (hk->bits) {
-    case 1: return qprep_g<T, 1>(G, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
-    case 2: return qprep_g<T, 2>(G, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
-    case 3: return qprep_g<T, 3>(G, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
+    case 1: return qprep_g<T, 1>(G, BH, a, app, hk, s);
+    case 2: return qprep_g<T, 2>(G, BH, a, app, hk, s);
+    case 3: return qprep_g<T, 3>(G, BH, a, app, hk, s);
   }
   return TQ_EUNSUPPORTED;
 }
 
 int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
-                 uint32_t* qfrag, float4* kconst, cudaStream_t s) {
+                 uint32_t* qfrag, float4* kconst, const AppendIn* app, cudaStream_t s) {
   if (q_dtype == TQ_F32)
-    return qprep_b<float>(G, BH, Hkv, static_cast<const float*>(q), q_pos, hk, rope, qfrag, kconst, s);
-  return qprep_b<__nv_bfloat16>(G, BH, Hkv, static_cast<const __nv_bfloat16*>(q), q_pos, hk, rope, qfrag, kconst, s);
+    return qprep_b<float>(G, BH, Hkv, static_cast<const float*>(q), q_pos, hk, rope, qfrag, kconst, app, s);
+  return qprep_b<__nv_bfloat16>(G, BH, Hkv, static_cast<const __nv_bfloat16*>(q), q_pos, hk, rope, qfrag, kconst,
+                                app, s);
+}
+
+// Lets `kern` take `bytes` of dynamic shared memory: past the default 48 KB
+// (with its static arrays) the kernel must opt in; TQ_EUNSUPPORTED beyond
+// the device's per-block maximum.
+template <typename K>
+int allow_dyn_smem(K kern, size_t bytes) {
+  if (bytes <= 4096) return TQ_OK;   // inside the default limit for every merge instance
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return TQ_ECUDA;
+  if (bytes <= static_cast<size_t>(fa.maxDynamicSharedSizeBytes)) return TQ_OK;
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (fa.sharedSizeBytes + bytes > static_cast<size_t>(optin)) return TQ_EUNSUPPORTED;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
+                 cudaSuccess
+             ? TQ_OK
+             : TQ_ECUDA;
 }
 
 // Merge of n_parts partial records per head (layout: see decode_merge_kernel).
@@ -1138,8 +1322,15 @@ int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64
 int launch_merge(int G, int BH, const float* partial, int n_parts, int64_t bh_stride, int64_t part_stride,
                  const tq_rotation* hv, float* out, bool final_out, cudaStream_t s) {
   const float qjl = static_cast<float>(hv->res_const);
+  // weights of the parts, [n_parts][G] floats: 37 KB at G = 8 with the most
+  // splits a single sequence gets (1184)
   const size_t fsb = static_cast<size_t>(n_parts) * G * sizeof(float);
 #define TQ_MERGE(GG)                                                                                                \
+  {                                                                                                                 \
+    const int st = final_out ? allow_dyn_smem(decode_merge_kernel<GG, true>, fsb)                                  \
+                             : allow_dyn_smem(decode_merge_kernel<GG, false>, fsb);                                \
+    if (st != TQ_OK) return st;                                                                                     \
+  }                                                                                                                 \
   return final_out ? launch_pdl(decode_merge_kernel<GG, true>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts,  \
                                 bh_stride, part_stride, hv->d_s, hv->d_signs, qjl, out)                             \
                    : launch_pdl(decode_merge_kernel<GG, false>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts, \
@@ -1216,7 +1407,7 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
                 const void* v_win, int win_dtype, int64_t win_stride, int R, int B, int Hq, int Hkv, int64_t T,
                 const int32_t* seq_lens, float scale, float* out, float* partial_out, void* workspace,
                 size_t workspace_bytes, cudaStream_t s,
-                cudaEvent_t prof_begin, cudaEvent_t prof_end) {
+                cudaEvent_t prof_begin, cudaEvent_t prof_end, const AppendIn* app = nullptr) {
   {
     const int st = check_decode_sizes(hk, hv, B, Hq, Hkv, T);
     if (st != TQ_OK) return st;
@@ -1256,7 +1447,7 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
   const float score_scale = scale * 1.4426950408889634f;
 
-  int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, s);
+  int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, app, s);
   if (st != TQ_OK) return st;
   st = tq::launch_status();
   if (st != TQ_OK) return st;
@@ -1288,6 +1479,7 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   p.one_h = kOneH2;
   p.one_b = kOneB2;
   p.qjl = static_cast<float>(hk->res_const);
+  p.append = app ? 1 : 0;
   for (int i = 0; i < 4; ++i) {
     p.walsh_k[i] = static_cast<float>(hk->walsh[i]);
     p.walsh_v[i] = static_cast<float>(hv->walsh[i]);
@@ -1332,6 +1524,21 @@ extern "C" int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
                      nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, nullptr, workspace,
                      workspace_bytes,
                      static_cast<cudaStream_t>(stream), prof_begin, prof_end);
+}
+
+extern "C" int tq_decode_attention_append(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
+                                          const int64_t* q_pos, const void* k_new, const void* v_new,
+                                          uint8_t* k_codes, uint8_t* k_signs, float* k_norms, uint8_t* v_codes,
+                                          uint8_t* v_signs, float* v_norms, int64_t cache_stride, int B, int Hq,
+                                          int Hkv, int64_t T, const int32_t* seq_lens, float scale, float* out,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (!k_new || !v_new) return TQ_EINVAL;
+  const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
+  g_prof_begin = g_prof_end = nullptr;
+  AppendIn app{k_new, v_new, hv, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride, T, seq_lens};
+  return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
+                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, nullptr, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end, &app);
 }
 
 extern "C" int tq_decode_attention_window(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,

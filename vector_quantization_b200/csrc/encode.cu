@@ -13,69 +13,27 @@
 #include <cuda_bf16.h>
 
 #include "bitplane.cuh"
+#include "encode_vec.cuh"
 #include "tcgen05.cuh"
 #include "tq_internal.h"
 
 namespace {
-
-struct EncodeParams {
-  const void* x;
-  int64_t n, ld;
-  const int64_t* pos;
-  int64_t pos_period, pos_offset;
-  int rope;
-  uint32_t* codes;      // record = BITS * D / 32 words
-  uint32_t* signs;      // record = D / 32 words (m == D)
-  float2* norms;        // record = (||x||, ||r||)
-  int64_t out_stride;
-  const int64_t* out_rows;  // [n] record of each row (scatter calls), or null: row * out_stride
-  int64_t n_records;        // records in the output arrays (scatter calls: targets outside are skipped)
-  int sign_res;             // sign-residual handle: norms[1] = mean |r_i| instead of ||r|| (S is the identity)
-  const float* dsigns;  // [D]
-  const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
-  const uint16_t* hd_op; // tensor-core encode: H D in the same layout (fp16 bits when split, else bf16)
-  const float* st;      // S transposed, fp32: st[k * d + j] = S[j][k]
-  int rows;             // warp-per-vector kernel: vectors per tile, R in {8, 16, ..., 128}
-  const float* thresholds;
-  const float* levels;
-  const float2* rope_hi;
-  const float2* rope_lo;
-  int64_t rope_max_pos;
-  // thread-per-vector kernel: sign diagonal and the positive half of the
-  // (symmetric) codebook, read straight from the parameter space
-  float dsg[128];
-  float tpos[4];        // thresholds above 0, ascending (2^(b-1) - 1 of them)
-  float lpos[4];        // levels above 0, ascending (2^(b-1) of them)
-  float2 theta[64];     // tensor-core encode: RoPE frequency i as (hi, lo) float pieces
-};
-
-// Output record of input row `row`: row * out_stride, or the row's entry of
-// out_rows for scatter calls (-1, not written, when that entry lies outside
-// the output arrays).
-__device__ __forceinline__ int64_t out_record(const EncodeParams& p, int64_t row) {
-  if (!p.out_rows) return row * p.out_stride;
-  const int64_t r = p.out_rows[row];
-  return r >= 0 && r < p.n_records ? r : -1;
-}
 
 // Tile of 128 vectors per CTA iteration (the M of one tensor-core product).
 constexpr int kTileVec = 128;
 constexpr int kWaitLimit = 1 << 17;   // polls of about 9 us each: a wait gives up after about a second
 
 // ===========================================================================
-// Block-per-vector encode, for the few vectors a decode step appends: thread
-// i owns coordinate i; RoPE pairs meet through shared memory, the norm and
-// ||r|| are block reductions, the Walsh-Hadamard transform takes five
-// shuffle stages and log2(d/32) shared-memory stages, a warp ballot yields a
-// plane word, and S r is a matrix-vector product on the CUDA cores with row i
-// of S loaded into registers at the start (so its loads overlap the rest).
+// Block-per-vector encode, for the few vectors a decode step appends: one
+// vector per block of D threads (encode_vec_core), with row i of S loaded
+// into registers before the wait on the previous launch, so its loads
+// overlap that launch's tail.
 // ===========================================================================
 template <int D, int BITS, typename T>
 __device__ __forceinline__ void encode_vec_body(const EncodeParams& p) {
-  constexpr int NW = D / 32;
   __shared__ __align__(16) float buf[D];
-  __shared__ float red[2][NW];
-  const int i = threadIdx.x, lane = i & 31, w = i >> 5;
+  __shared__ float red[2][D / 32];
+  const int i = threadIdx.x;
   const int64_t row = blockIdx.x;
   float scol[D];   // row i of S
 #pragma unroll
@@ -83,104 +41,11 @@ __device__ __forceinline__ void encode_vec_body(const EncodeParams& p) {
   // S belongs to the handle; everything below may depend on the previous
   // launch on the stream (programmatic dependent launch)
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  const T* xr = static_cast<const T*>(p.x) + row * p.ld;
-  float x;
-  if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(xr) + i);
-  else x = __bfloat162float(xr[i]);
   const int64_t rec = out_record(p, row);
   if (rec < 0) return;   // uniform over the block (one vector per block)
-  if (p.rope) {
-    const int64_t pos = p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period;
-    if (pos < 0 || pos >= p.rope_max_pos) {   // uniform over the block
-      if (i == 0) p.norms[rec] = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-      return;
-    }
-    buf[i] = x;
-    __syncthreads();
-    const int j = i & (D / 2 - 1);
-    const float2 a = p.rope_hi[(pos >> kRopeLoBits) * (D / 2) + j];
-    const float2 b = p.rope_lo[(pos & (kRopeLoRows - 1)) * (D / 2) + j];
-    const float cs = a.x * b.x - a.y * b.y, sn = a.y * b.x + a.x * b.y;
-    const float x1 = buf[j], x2 = buf[j + D / 2];
-    x = i < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
-  }
-  // ||x|| and u = H D x (unnormalised, Sylvester order)
-  float ss = x * x;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  float u = x * p.dsg[i];
-#pragma unroll
-  for (int bit = 1; bit < 32; bit <<= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, u, bit);
-    u = (lane & bit) ? o - u : u + o;
-  }
-  if (lane == 0) red[0][w] = ss;
-#pragma unroll
-  for (int bit = 32; bit < D; bit <<= 1) {
-    __syncthreads();
-    buf[i] = u;
-    __syncthreads();
-    const float o = buf[i ^ bit];
-    u = (i & bit) ? o - u : u + o;
-  }
-  __syncthreads();
-  ss = 0.f;
-#pragma unroll
-  for (int q = 0; q < NW; ++q) ss += red[0][q];
-  const float nrm = sqrtf(ss);
-  const float y = fmaf(u, (nrm > 0.f ? 1.0f / nrm : 0.f) * rsqrtf(static_cast<float>(D)), 0.f);   // -0 -> +0
-  // symmetric codebook: sign picks the half, |y| against the positive thresholds the level
-  const bool pos = y >= 0.f;
-  const float a = fabsf(y);
-  uint32_t bits[BITS];
-  float mag;
-  if constexpr (BITS == 1) {
-    bits[0] = pos;
-    mag = p.lpos[0];
-  } else if constexpr (BITS == 2) {
-    const bool o = a >= p.tpos[0];
-    bits[1] = pos;
-    bits[0] = pos == o;
-    mag = o ? p.lpos[1] : p.lpos[0];
-  } else {
-    const bool m1 = a >= p.tpos[0], m2 = a >= p.tpos[1], m3 = a >= p.tpos[2];
-    bits[2] = pos;
-    bits[1] = pos == m2;
-    bits[0] = pos == (m1 != (m2 != m3));
-    mag = m3 ? p.lpos[3] : (m2 ? p.lpos[2] : (m1 ? p.lpos[1] : p.lpos[0]));
-  }
-  const float r = nrm * (y - copysignf(mag, y));
-  uint32_t* crec = p.codes + rec * (BITS * NW);
-#pragma unroll
-  for (int k = 0; k < BITS; ++k) {
-    const uint32_t word = __ballot_sync(0xffffffffu, bits[k]);
-    if (lane == 0) crec[k * NW + w] = word;
-  }
-  float rr = p.sign_res ? fabsf(r) : r * r;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
-  if (lane == 0) red[1][w] = rr;
-  buf[i] = r;
-  __syncthreads();
-  // (S r)_i
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int k = 0; k < D; k += 4) {
-    const float4 rv = *reinterpret_cast<const float4*>(buf + k);
-    acc[0] = fmaf(scol[k], rv.x, acc[0]);
-    acc[1] = fmaf(scol[k + 1], rv.y, acc[1]);
-    acc[2] = fmaf(scol[k + 2], rv.z, acc[2]);
-    acc[3] = fmaf(scol[k + 3], rv.w, acc[3]);
-  }
-  const float proj = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  const uint32_t sword = __ballot_sync(0xffffffffu, proj >= 0.f);
-  if (lane == 0) p.signs[rec * NW + w] = sword;
-  if (i == 0) {
-    rr = 0.f;
-#pragma unroll
-    for (int q = 0; q < NW; ++q) rr += red[1][q];
-    p.norms[rec] = make_float2(nrm, p.sign_res ? rr * (1.f / D) : sqrtf(rr));
-  }
+  const int64_t pos = p.rope ? (p.pos ? p.pos[row] : p.pos_offset + row % p.pos_period) : 0;
+  encode_vec_core<D, BITS, T>(p, i, static_cast<const T*>(p.x) + row * p.ld, rec, pos, buf, red,
+                              [] { __syncthreads(); }, [&](int k) { return scol[k]; });
 }
 
 template <int D, int BITS, typename T>
@@ -848,8 +713,8 @@ constexpr float kInvTwoPi = 0.15915494309189533577f;
 constexpr int64_t kPairsMaxRopePos = int64_t(1) << 22;
 
 // ===========================================================================
-// Rotation on the tensor core (d = 128, large batches).  y = H D x is a
-// dense 128 x 128 contraction with exact +-1 entries, so each 128-row tile
+// Rotation on the tensor core (d = 64 or 128, large batches).  y = H D x is
+// a dense d x d contraction with exact +-1 entries, so each 128-row tile
 // is rotated by tcgen05 MMAs against H D resident in shared memory, and the
 // CUDA cores keep only RoPE, the codes, the residual and the sign bits.
 //
@@ -873,12 +738,15 @@ constexpr int64_t kPairsMaxRopePos = int64_t(1) << 22;
 // ===========================================================================
 constexpr int kTcThreads = 512;   // two groups of 8 warps
 
-template <int BITS, typename T, bool SPLIT>
+template <int D, int BITS, typename T, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                  EncodeParams p) {
   static_assert(SPLIT || sizeof(T) == 2, "fp32 input needs the split path");
-  constexpr int D = 128;
-  constexpr int OPB = kTileVec * D * 2;           // 32 KB: one 16-bit [128 x 128] operand
+  static_assert(D == 64 || D == 128, "tensor-core encode: d = 64 or 128");
+  constexpr int OPB = kTileVec * D * 2;           // one 16-bit [128 x d] operand (32 KB at d = 128)
+  constexpr int SOPB = D * D * 2;                 // S or H D: one 16-bit [d x d] operand
+  constexpr int HC = D / 4;                       // phase 2: coordinates per thread in each half of a row
+  constexpr int NJ = D / 32;                      // 32-bit words per plane
   constexpr int kBoxCols = 128 / static_cast<int>(sizeof(T));
   constexpr int kBoxes = D / kBoxCols;
   constexpr uint32_t kXBytes = kTileVec * D * sizeof(T);
@@ -892,10 +760,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
   __shared__ float xrr[2][2][kTileVec];           // per group: partial sums of squared residuals
   uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
   uint8_t* s_op = base;
-  uint8_t* hd_op = base + OPB;
+  uint8_t* hd_op = base + SOPB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = warp >> 3, gw = warp & 7, gt = tid & 255;
-  uint8_t* a_hi = base + 2 * OPB + g * 2 * OPB;
+  uint8_t* a_hi = base + 2 * SOPB + g * 2 * OPB;
   uint8_t* a_lo = a_hi + OPB;
   uint8_t* xs = a_hi;   // staged input tile (bf16: a_hi; fp32: a_hi and a_lo)
   const int64_t n_tiles = (p.n + kTileVec - 1) / kTileVec;
@@ -907,8 +775,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     for (int b = 0; b < kBoxes; ++b)
       tqtc::tma_load_2d(xs + b * (kTileVec * 128), &xmap, b * kBoxCols, static_cast<int>(tl * kTileVec), &mb_x[g]);
   };
-  for (int c = tid; c < 2 * OPB / 16; c += blockDim.x)
-    tqdev::cp_async16(base + 16 * c, c < OPB / 16 ? p.s_op + 8 * c : p.hd_op + 8 * (c - OPB / 16), 16);
+  for (int c = tid; c < 2 * SOPB / 16; c += blockDim.x)
+    tqdev::cp_async16(base + 16 * c, c < SOPB / 16 ? p.s_op + 8 * c : p.hd_op + 8 * (c - SOPB / 16), 16);
   tqdev::cp_async_commit();
   if (tid < D / 4) {
     thh_s[tid] = make_float2(p.theta[2 * tid].x, p.theta[2 * tid + 1].x);
@@ -922,7 +790,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
       tqtc::mbar_init(&mb_s[i], 1);
     }
   }
-  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, 256);
+  if (warp == 0) tqtc::tmem_alloc(&tmem_slot, 2 * D);
   tqdev::cp_async_wait<0>();
   tqtc::fence_smem_to_async();
   tqtc::fence_before_sync();
@@ -930,7 +798,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
   tqtc::fence_after_sync();
   int64_t tile = 2 * static_cast<int64_t>(blockIdx.x) + g;
   if (gt == 0 && tile < n_tiles) issue_x(tile);
-  const uint32_t tm = tmem_slot + 128 * g;                  // y, then S r: 128 columns per group
+  const uint32_t tm = tmem_slot + D * g;                    // y, then S r: d columns per group
   const uint32_t tm_lane = static_cast<uint32_t>(32 * (gw & 3)) << 16;
   constexpr uint32_t idy = SPLIT ? tqtc::idesc_f16_f32(kTileVec, D) : tqtc::idesc_bf16_f32(kTileVec, D);
   constexpr uint32_t ids = tqtc::idesc_bf16_f32(kTileVec, D);
@@ -939,10 +807,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
   float tp[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) tp[k] = p.tpos[k];
-  // phase-2 mapping (SPLIT): row t2 of the tile, coordinates {32 h2 + i, 64 + 32 h2 + i}
+  // phase-2 mapping (SPLIT): row t2 of the tile, coordinates {HC h2 + i, d/2 + HC h2 + i}, i < HC
   const int t2 = 32 * (gw & 3) + 16 * (gw >> 2) + (lane & 15), h2 = lane >> 4;
   const uint32_t rowbase2 = static_cast<uint32_t>((t2 >> 3) * 1024 + (t2 & 7) * 128);
-  // phase-4 mapping: row r4 = tensor-memory lane, coordinates 64 c4 .. 64 c4 + 63
+  // phase-4 mapping: row r4 = tensor-memory lane, coordinates d/2 c4 .. d/2 c4 + d/2 - 1
   const int r4 = 32 * (gw & 3) + lane, c4 = gw >> 2;
   const uint32_t rowbase4 = static_cast<uint32_t>((r4 >> 3) * 1024 + (r4 & 7) * 128);
   uint32_t ph_x = 0, ph_y = 0, ph_s = 0;
@@ -956,35 +824,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
       // ---- 2. row t2 into registers, ||x||, RoPE, fp16 hi + lo A operand
       const int64_t row = tile * kTileVec + t2;
       bool valid = row < p.n && ok_x;
-      float2 v[32];   // v[16 s + m] = coordinates (64 s + 32 h2 + 2m, + 1)
+      // v[HC/2 s + m] = coordinates (d/2 s + HC h2 + 2m, + 1); a staged row is
+      // 128-byte boxes of 16-byte chunks, chunk c of a box at c ^ (row % 8)
+      constexpr int NV = HC;   // float2 per thread
+      float2 v[NV];
       if constexpr (sizeof(T) == 2) {
 #pragma unroll
         for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int j = 4 * h2 + q;
-            const uint4 w4 = *reinterpret_cast<const uint4*>(xs + sh * (kTileVec * 128) + t2 * 128 + ((j ^ (t2 & 7)) << 4));
+          for (int q = 0; q < HC / 8; ++q) {
+            // chunk of 8 coordinates: box, chunk within the box
+            const int box = D == 128 ? sh : 0, cb = D == 128 ? 4 * h2 + q : 4 * sh + 2 * h2 + q;
+            const uint4 w4 = *reinterpret_cast<const uint4*>(xs + box * (kTileVec * 128) + t2 * 128 +
+                                                             ((cb ^ (t2 & 7)) << 4));
             const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              v[16 * sh + 4 * q + e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+              v[(HC / 2) * sh + 4 * q + e] =
+                  make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
           }
       } else {
 #pragma unroll
         for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int b = 2 * sh + h2;
-            const float4 f = *reinterpret_cast<const float4*>(xs + b * (kTileVec * 128) + t2 * 128 + ((q ^ (t2 & 7)) << 4));
-            v[16 * sh + 2 * q] = make_float2(f.x, f.y);
-            v[16 * sh + 2 * q + 1] = make_float2(f.z, f.w);
+          for (int q = 0; q < HC / 4; ++q) {
+            // chunk of 4 coordinates: box, chunk within the box
+            const int box = D == 128 ? 2 * sh + h2 : sh, cb = D == 128 ? q : 4 * h2 + q;
+            const float4 f = *reinterpret_cast<const float4*>(xs + box * (kTileVec * 128) + t2 * 128 +
+                                                              ((cb ^ (t2 & 7)) << 4));
+            v[(HC / 2) * sh + 2 * q] = make_float2(f.x, f.y);
+            v[(HC / 2) * sh + 2 * q + 1] = make_float2(f.z, f.w);
           }
       }
       float ss;
       {
         float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) a2 = __ffma2_rn(v[m], v[m], a2);
+        for (int m = 0; m < NV; ++m) a2 = __ffma2_rn(v[m], v[m], a2);
         ss = a2.x + a2.y;
       }
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);
@@ -993,7 +869,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
         if (pos < 0 || pos >= p.rope_max_pos) {
           valid = false;
         } else {
-          // pairs (v[m], v[16 + m]) turn by pos * theta_j, j = 32 h2 + 2m (+1):
+          // pairs (v[m], v[HC/2 + m]) turn by pos * theta_j, j = HC h2 + 2m (+1):
           // angle pos theta_hi + pos theta_lo, reduced by 2 pi in three terms
           // (k negated: rint is odd), then sin / cos on [-pi, pi]
           const float pf = static_cast<float>(pos);   // exact: pos < 2^22
@@ -1001,9 +877,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
           const float2 q2c = make_float2(-kInvTwoPi, -kInvTwoPi), six2 = make_float2(6.f, 6.f);
           const float2 c2c = make_float2(kC2, kC2), c3c = make_float2(kC3, kC3);
 #pragma unroll
-          for (int m = 0; m < 16; ++m) {
+          for (int m = 0; m < HC / 2; ++m) {
             if ((m & 3) == 0) asm volatile("" ::: "memory");   // bound the loads in flight (registers)
-            const float2 thh = thh_s[16 * h2 + m], thl = thl_s[16 * h2 + m];
+            const float2 thh = thh_s[(HC / 2) * h2 + m], thl = thl_s[(HC / 2) * h2 + m];
             const float2 ah = __fmul2_rn(pf2, thh);
             const float2 e = __ffma2_rn(npf2, thh, ah);
             const float2 nal = __ffma2_rn(npf2, thl, e);
@@ -1017,9 +893,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
             __sincosf(r.x, &s0, &c0);
             __sincosf(r.y, &s1, &c1);
             const float2 sn = make_float2(s0, s1), cs = make_float2(c0, c1);
-            const float2 x = v[m], y = v[16 + m];
+            const float2 x = v[m], y = v[HC / 2 + m];
             v[m] = __ffma2_rn(y, __fmul2_rn(sn, m1), __fmul2_rn(x, cs));
-            v[16 + m] = __ffma2_rn(x, sn, __fmul2_rn(y, cs));
+            v[HC / 2 + m] = __ffma2_rn(x, sn, __fmul2_rn(y, cs));
           }
         }
       }
@@ -1038,19 +914,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
 #pragma unroll
       for (int sh = 0; sh < 2; ++sh)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < HC / 8; ++q) {
           uint32_t hv[4], lv[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 x = __fmul2_rn(v[16 * sh + 4 * q + e], sc2);
+            const float2 x = __fmul2_rn(v[(HC / 2) * sh + 4 * q + e], sc2);
             const __half2 hh = __floats2half2_rn(x.x, x.y);
             const float2 lo = __ffma2_rn(__half22float2(hh), m1, x);
             const __half2 lh = __floats2half2_rn(lo.x, lo.y);
             hv[e] = *reinterpret_cast<const uint32_t*>(&hh);
             lv[e] = *reinterpret_cast<const uint32_t*>(&lh);
           }
-          const int c = 8 * sh + 4 * h2 + q;
-          const uint32_t off = (c >> 3) * (kTileVec * 128) + rowbase2 + ((((c & 7) ^ (t2 & 7))) << 4);
+          // 16-byte chunk of the K-major operand row: K block, chunk within it
+          const int kb = D == 128 ? sh : 0, cb = D == 128 ? 4 * h2 + q : 4 * sh + 2 * h2 + q;
+          const uint32_t off = kb * (kTileVec * 128) + rowbase2 + ((cb ^ (t2 & 7)) << 4);
           *reinterpret_cast<uint4*>(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
           *reinterpret_cast<uint4*>(a_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
         }
@@ -1058,11 +935,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     }
     const int64_t row = tile * kTileVec + r4;
     if constexpr (!SPLIT) {
-      // ||x||^2 of row r4, this thread's 64 coordinates (box c4 of the staged bf16 tile)
+      // ||x||^2 of row r4, this thread's d/2 coordinates of the staged bf16 tile
       float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 w4 = *reinterpret_cast<const uint4*>(xs + c4 * (kTileVec * 128) + rowbase4 + ((j ^ (r4 & 7)) << 4));
+      for (int j = 0; j < D / 16; ++j) {
+        const int box = D == 128 ? c4 : 0, cb = D == 128 ? j : 4 * c4 + j;
+        const uint4 w4 = *reinterpret_cast<const uint4*>(xs + box * (kTileVec * 128) + rowbase4 +
+                                                         ((cb ^ (r4 & 7)) << 4));
         const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -1112,48 +991,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     const bool ok_y = !failed && tqtc::mbar_wait(&mb_y[g], ph_y, kWaitLimit);
     ph_y ^= 1;
     tqtc::fence_after_sync();
-    float2 u[32];   // u[m] = coordinates (64 c4 + 2m, + 1)
-    {
+    constexpr int NU = D / 4;   // float2 per thread
+    float2 u[NU];   // u[m] = coordinates (d/2 c4 + 2m, + 1)
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) {
       float y[32];
-      tqtc::tmem_ld32(tm + tm_lane + 64 * c4, y);
+      tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * h, y);
 #pragma unroll
-      for (int m = 0; m < 16; ++m) u[m] = make_float2(y[2 * m], y[2 * m + 1]);
-      tqtc::tmem_ld32(tm + tm_lane + 64 * c4 + 32, y);
-#pragma unroll
-      for (int m = 0; m < 16; ++m) u[16 + m] = make_float2(y[2 * m], y[2 * m + 1]);
+      for (int m = 0; m < 16; ++m) u[16 * h + m] = make_float2(y[2 * m], y[2 * m + 1]);
     }
     {
       const float2 sc2 = make_float2(scale, scale), z2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int m = 0; m < 32; ++m) u[m] = __ffma2_rn(u[m], sc2, z2);   // unit-vector coordinates, -0 -> +0
+      for (int m = 0; m < NU; ++m) u[m] = __ffma2_rn(u[m], sc2, z2);   // unit-vector coordinates, -0 -> +0
     }
     const float nv = valid ? nrm : 0.f;
     float nl[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) nl[k] = nv * p.lpos[k];
-    uint32_t w0[BITS], w1[BITS];
-    float rr = quantize32_x2<BITS>(u, tp, nl, nv, w0);        // coordinates 64 c4 .. + 31: word 2 c4
-    rr += quantize32_x2<BITS>(u + 16, tp, nl, nv, w1);        // 64 c4 + 32 ..: word 2 c4 + 1
-    if (p.sign_res) {   // sum of |r_i| over this thread's 64 coordinates in place of sum r_i^2
+    uint32_t wq[D / 64][BITS];   // words (d/64) c4 + h of each plane
+    float rr = 0.f;
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) rr += quantize32_x2<BITS>(u + 16 * h, tp, nl, nv, wq[h]);
+    if (p.sign_res) {   // sum of |r_i| over this thread's d/2 coordinates in place of sum r_i^2
       float2 ra = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int m = 0; m < 32; ++m) ra = __fadd2_rn(ra, make_float2(fabsf(u[m].x), fabsf(u[m].y)));
+      for (int m = 0; m < NU; ++m) ra = __fadd2_rn(ra, make_float2(fabsf(u[m].x), fabsf(u[m].y)));
       rr = ra.x + ra.y;
     }
     xrr[g][c4][r4] = rr;
     if (valid && ok_y) {
-      constexpr int NJ = 4;
       uint32_t* crec = p.codes + row * p.out_stride * (BITS * NJ);   // 4-byte aligned records
 #pragma unroll
-      for (int k = 0; k < BITS; ++k) {
-        crec[k * NJ + 2 * c4] = w0[k];
-        crec[k * NJ + 2 * c4 + 1] = w1[k];
-      }
+      for (int k = 0; k < BITS; ++k)
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) crec[k * NJ + (D / 64) * c4 + h] = wq[h][k];
     }
     // residual (zero on absent rows) as bf16 hi + lo over the A operand, row r4
     // (the staged tile was read before the barrier ahead of the products)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < D / 16; ++j) {
       uint32_t hv[4], lv[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -1166,7 +1043,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
         hv[e] = hbits;
         lv[e] = *reinterpret_cast<uint32_t*>(&lb);
       }
-      const uint32_t off = c4 * (kTileVec * 128) + rowbase4 + ((j ^ (r4 & 7)) << 4);
+      const int kb = D == 128 ? c4 : 0, cb = D == 128 ? j : 4 * c4 + j;
+      const uint32_t off = kb * (kTileVec * 128) + rowbase4 + ((cb ^ (r4 & 7)) << 4);
       *reinterpret_cast<uint4*>(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
       *reinterpret_cast<uint4*>(a_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
     }
@@ -1198,15 +1076,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     // sign bits of S r: complemented fp32 sign bits, one funnel shift each
     // (an exact -0 projection reads as negative, within the sign tolerance)
     {
-      constexpr int NJ = 4;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         float val[32];
-        tqtc::tmem_ld32(tm + tm_lane + 64 * c4 + 32 * c, val);
+        tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * c, val);
         uint32_t w = 0;
 #pragma unroll
         for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[b]), w, 1);
-        if (row < p.n) p.signs[row * p.out_stride * NJ + 2 * c4 + c] = ok ? ~w : 0u;
+        if (row < p.n) p.signs[row * p.out_stride * NJ + (D / 64) * c4 + c] = ok ? ~w : 0u;
       }
       if (!ok && c4 == 0 && row < p.n) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
     }
@@ -1215,7 +1092,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
   }
   tqtc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tqtc::tmem_free(tmem_slot, 256);
+  if (warp == 0) tqtc::tmem_free(tmem_slot, 2 * D);
 }
 
 template <int D, int BITS, typename T>
@@ -1240,10 +1117,11 @@ int launch_encode_rows(const EncodeParams& p, cudaStream_t stream) {
 // Batches below this many vectors take the low-latency warp-per-vector kernel.
 constexpr int64_t kRowsKernelMinN = 16384;
 
-template <int BITS, typename T, bool SPLIT>
+template <int D, int BITS, typename T, bool SPLIT>
 int launch_encode_tc(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_t stream) {
-  const size_t smem = 6 * static_cast<size_t>(kTileVec) * 128 * 2 + 1024;   // S, H D, 2 x (hi, lo): 193 KB
-  auto kern = encode_tc_kernel<BITS, T, SPLIT>;
+  // S, H D, 2 groups x (hi, lo): 193 KB at d = 128, 81 KB at d = 64
+  const size_t smem = 2 * static_cast<size_t>(D) * D * 2 + 4 * static_cast<size_t>(kTileVec) * D * 2 + 1024;
+  auto kern = encode_tc_kernel<D, BITS, T, SPLIT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return TQ_ECUDA;
   int dev = 0, sms = 148;
@@ -1256,20 +1134,20 @@ int launch_encode_tc(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_
   return tq::launch_status();
 }
 
-template <int BITS, typename T>
-int launch_encode_d128(const EncodeParams& p, cudaStream_t stream) {
+template <int D, int BITS, typename T>
+int launch_encode_tcd(const EncodeParams& p, cudaStream_t stream) {
   // Positions past 2^22 (the in-kernel angle reduction's range) or more rows
   // than a TMA coordinate holds go to the table-driven one-thread kernel.
   if ((p.rope && p.rope_max_pos > kPairsMaxRopePos) || p.n >= (int64_t(1) << 31) || !p.hd_op)
-    return launch_encode_rows<128, BITS, T>(p, stream);
+    return launch_encode_rows<D, BITS, T>(p, stream);
   CUtensorMap xmap;
-  if (!tq::make_tmap_2d(&xmap, p.x, static_cast<int>(sizeof(T)), p.n, 128, p.ld, 128 / static_cast<int>(sizeof(T)),
+  if (!tq::make_tmap_2d(&xmap, p.x, static_cast<int>(sizeof(T)), p.n, D, p.ld, 128 / static_cast<int>(sizeof(T)),
                         kTileVec))
-    return launch_encode_rows<128, BITS, T>(p, stream);
+    return launch_encode_rows<D, BITS, T>(p, stream);
   if constexpr (sizeof(T) == 2) {
-    if (!p.rope) return launch_encode_tc<BITS, T, false>(p, xmap, stream);
+    if (!p.rope) return launch_encode_tc<D, BITS, T, false>(p, xmap, stream);
   }
-  return launch_encode_tc<BITS, T, true>(p, xmap, stream);
+  return launch_encode_tc<D, BITS, T, true>(p, xmap, stream);
 }
 
 template <int D, int BITS, typename T>
@@ -1287,8 +1165,7 @@ int launch_encode(const EncodeParams& p, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, encode_vec_kernel<D, BITS, T>, p) == cudaSuccess ? TQ_OK : TQ_ECUDA;
   }
   if (p.n < kRowsKernelMinN || p.out_rows) return launch_encode_warp<D, BITS, T>(p, stream);
-  if constexpr (D == 128) return launch_encode_d128<BITS, T>(p, stream);
-  return launch_encode_rows<D, BITS, T>(p, stream);
+  return launch_encode_tcd<D, BITS, T>(p, stream);
 }
 
 template <int D, int BITS, typename T>
@@ -1366,26 +1243,9 @@ int make_encode_params(const tq_rotation* h, const void* x, int dtype, int64_t n
   p.out_stride = out_stride;
   p.out_rows = out_rows;
   p.n_records = n_records;
-  p.sign_res = h->residual == TQ_RES_SIGN ? 1 : 0;
-  p.dsigns = h->d_signs;
-  p.s_op = h->d_s_op;
+  fill_handle_fields(p, h);
   // H D for the tensor-core encode: fp16 when the rows are split (RoPE or fp32 input), else bf16
   p.hd_op = (apply_rope || dtype == TQ_F32) ? h->d_hd_f16 : h->d_hd_bf16;
-  p.st = h->d_st;
-  {
-    const int half = 1 << (h->bits - 1);
-    for (int i = 0; i < h->d && i < 128; ++i) p.dsg[i] = h->signs[i];
-    for (int k = 0; k < 4; ++k) {
-      p.lpos[k] = k < half ? static_cast<float>(h->levels[half + k]) : 0.f;
-      p.tpos[k] = k < half - 1 ? static_cast<float>(h->thresholds[half + k]) : 0.f;
-    }
-  }
-  p.thresholds = h->d_thresholds;
-  p.levels = h->d_levels;
-  p.rope_hi = h->d_rope_hi;
-  p.rope_lo = h->d_rope_lo;
-  p.rope_max_pos = h->rope_max_pos;
-  for (int i = 0; i < 64; ++i) p.theta[i] = make_float2(h->rope_th_hi[i], h->rope_th_lo[i]);
   *out = p;
   return TQ_OK;
 }

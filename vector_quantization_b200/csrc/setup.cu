@@ -457,7 +457,7 @@ int tq_build_rotation_ex(int d, int code_bits, int kind, int residual, const int
           op[off / 2] = static_cast<uint16_t>(bits >> 16);
         }
       if ((st = upload(&h->d_s_op, op.data(), op.size())) != TQ_OK) { release(h); return st; }
-      if (d == 128) {
+      if (d == 128 || d == 64) {
         // H D with H[j][k] = (-1)^popcount(j & k): rows j (output coordinate),
         // K = k, entries +-1 exact in fp16 (0x3C00) and bf16 (0x3F80)
         std::vector<uint16_t> hf(static_cast<size_t>(d) * d), hb(static_cast<size_t>(d) * d);

@@ -45,7 +45,7 @@ struct tq_rotation {
   uint16_t* d_s_op = nullptr;
   // H D (the unnormalised Hadamard times the sign diagonal, entries +-1) in
   // the same operand layout, rows = output coordinate, as fp16 and as bf16
-  // bits; Hadamard kind, d = 128 only.
+  // bits; Hadamard kind, d = 64 and 128.
   uint16_t* d_hd_f16 = nullptr;
   uint16_t* d_hd_bf16 = nullptr;
   // Hadamard kind, d = 64: the output transform of the tensor-core encoder

@@ -50,6 +50,8 @@ def _load():
                                       c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_p]),
         "tq_decode_attention": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
                                       c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
+        "tq_decode_attention_append": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64,
+                                             c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
         "tq_decode_partials": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
                                      c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
@@ -392,6 +394,43 @@ def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cach
                                     _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), cap, B, Hq, Hkv, T, _ptr(lens),
                                     float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream_ptr(stream)), "tq_decode_attention")
+    return out
+
+
+def decode_attention_append(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_new, v_new, k_cache, v_cache, T: int, *,
+                            seq_lens=None, scale: float | None = None, out=None, workspace=None, stream=None):
+    """One decode step that first appends the new token: k_new, v_new
+    [B, Hkv, d] (or [B*Hkv, d]) in q's dtype are encoded into record T - 1
+    (seq_lens[b] - 1 for sequence b) of each sequence, the key with RoPE at
+    q_pos[b]; then q [B, Hq, d] attends to the first T (seq_lens[b]) records.
+    One launch does the append and the query preparation.  Returns out
+    [B, Hq, d] float32."""
+    import torch
+    B, Hq, d = q.shape
+    kc, ks, kn = k_cache
+    vc, vs, vn = v_cache
+    Hkv, cap = kc.shape[1], kc.shape[2]
+    for t in (kc, ks, kn, vc, vs, vn):
+        if not t.is_contiguous():
+            raise ValueError("cache arrays must be contiguous")
+    if k_new.dtype != q.dtype or v_new.dtype != q.dtype:
+        raise ValueError("k_new and v_new must have the query's dtype")
+    if k_new.numel() != B * Hkv * d or v_new.numel() != B * Hkv * d:
+        raise ValueError("k_new and v_new must hold B * Hkv rows of d")
+    q, k_new, v_new = q.contiguous(), k_new.contiguous(), v_new.contiguous()
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(rot_k, rot_v, B, Hq, Hkv, T)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    lens = _seq_lens(seq_lens, B, q.device)
+    _check(_lib.tq_decode_attention_append(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos),
+                                           _ptr(k_new), _ptr(v_new), _ptr(kc), _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs),
+                                           _ptr(vn), cap, B, Hq, Hkv, T, _ptr(lens), float(scale), _ptr(out),
+                                           _ptr(workspace), workspace.numel(), _stream_ptr(stream)),
+           "tq_decode_attention_append")
     return out
 
 
