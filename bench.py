@@ -7,10 +7,9 @@ sequence, bf16 heavy-tailed K/V (N(0,1) + 4 outlier channels x20 per
 (layer, kv-head)), 2-bit Lloyd-Max codes + 1-bit QJL (m = 128).
 
 One step = one decode step of the whole model's attention: for every layer,
-quantize the new token's K and V into slot T-1 of each sequence
-(tq_quantize_kv_pair: keys and values in one launch) and score the query
-against all T cached tokens (tq_decode_attention: q-prep, split-KV kernel,
-merge).  The packed cache (15 GB) is far larger than L2, so no flush is
+one tq_decode_attention_append call quantizes the new token's K and V into
+record T-1 of each sequence in the same launch as the query preparation,
+then scores the query against all T cached tokens (split-KV kernel, merge).  The packed cache (15 GB) is far larger than L2, so no flush is
 needed between steps.
 
 Metric: cached tokens scored per second, one unit = one (layer, sequence,
@@ -45,9 +44,9 @@ UNIT = "tokens/s"
 
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of decode_split_kernel<2,4>
-# per cached token (235,717,120 + 5,504,512 B over 16*8*16384 tokens), or None
+# per cached token (235,722,240 + 5,576,448 B over 16*8*16384 tokens), or None
 # when the kernel has changed since that capture.
-SPLIT_TRAFFIC_PER_TOKEN = (235_717_120 + 5_504_512) / (16 * 8 * 16384)
+SPLIT_TRAFFIC_PER_TOKEN = (235_722_240 + 5_576_448) / (16 * 8 * 16384)
 
 EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1",
           "decode_llama8b_layer_window", "tiny_d128_t1024", "encode_esm2_33_layers", "memory_esm2")
@@ -587,9 +586,18 @@ def _extra_decode_window(dev, peak_gbs, R=128):
                                                        workspace=ws), reps=20, warm=3)
     ms_p = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws2), reps=20, warm=3)
     byts = B * Hkv * (T - R) * 2 * rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)) + 2 * kw.numel() * 2
+    # the flush when the window is full: its R tokens of every sequence into
+    # records T - R .. T - 1 (keys with RoPE at those positions), one launch
+    rows = torch.arange(B * Hkv, device=dev, dtype=torch.int64).repeat_interleave(R) * T + \
+        torch.arange(T - R, T, device=dev, dtype=torch.int64).repeat(B * Hkv)
+    fpos = torch.arange(T - R, T, device=dev, dtype=torch.int64).repeat(B * Hkv)
+    flat = lambda cache: tuple(a.view(B * Hkv * T, -1) for a in cache)
+    ms_f = _time_ms(lambda: tq.quantize_kv_pair_scatter(rk, kw.view(-1, d), rv, vw.view(-1, d), rows, flat(kc),
+                                                        flat(vc), pos=fpos, apply_rope=True), reps=20, warm=3)
     return {"decode_llama8b_layer_window": {"value": B * Hkv * T / ms_w * 1e3, "unit": "tokens/s",
                                             "ms": round(ms_w, 4), "ms_all_packed": round(ms_p, 4),
-                                            "frac_hbm": round(byts / ms_w / 1e6 / peak_gbs, 4)}}
+                                            "frac_hbm": round(byts / ms_w / 1e6 / peak_gbs, 4),
+                                            "flush_ms": round(ms_f, 4), "flush_rows": 2 * B * Hkv * R}}
 
 def _extra_tiny(dev):
     """The tiny workload (1 head, d 128, 1024 fp32 tokens, heavy-tailed with
@@ -719,22 +727,20 @@ def run_ours(args, rank, world, local_rank):
     outs = [torch.empty((B, Hq, d), dtype=torch.float32, device=dev) for _ in range(L)]
     torch.cuda.synchronize()
 
-    def slot(cache):
-        return tuple(a[:, :, T - 1] for a in cache)
-
     def step(prof=None, src=None):
+        # per layer: the new token's K and V appended at record T - 1 (RoPE at
+        # position T - 1) in the same launch as the query preparation, then
+        # attention over all T records
         for layer in range(L):
             nk = nks[layer] if src is None else src[0][layer]
             nv = nvs[layer] if src is None else src[1][layer]
             q = qs[layer] if src is None else src[2][layer]
-            tq.quantize_kv_pair(rks[layer], nk, rvs[layer], nv, apply_rope=True, pos_period=1, pos_offset=T - 1,
-                                out_k=slot(kcs[layer]), out_v=slot(vcs[layer]), out_stride=T)
             if prof is not None:
                 tq.profile_next_decode(*prof[layer])
-            tq.decode_attention(rks[layer], rvs[layer], q, qpos, kcs[layer], vcs[layer], T, out=outs[layer],
-                                workspace=ws)
+            tq.decode_attention_append(rks[layer], rvs[layer], q, qpos, nk, nv, kcs[layer], vcs[layer], T,
+                                       out=outs[layer], workspace=ws)
 
-    launches_per_step = L * (1 + 3)
+    launches_per_step = L * 3
     dist = None
     if world > 1:
         import torch.distributed as dist
