@@ -739,7 +739,7 @@ constexpr int64_t kPairsMaxRopePos = int64_t(1) << 22;
 constexpr int kTcThreads = 512;   // two groups of 8 warps
 
 template <int D, int BITS, typename T, bool SPLIT>
-__global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+__global__ void __launch_bounds__(kTcThreads, D == 64 ? 2 : 1) encode_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                  EncodeParams p) {
   static_assert(SPLIT || sizeof(T) == 2, "fp32 input needs the split path");
   static_assert(D == 64 || D == 128, "tensor-core encode: d = 64 or 128");
@@ -1129,7 +1129,8 @@ int launch_encode_tc(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = (p.n + kTileVec - 1) / kTileVec;
   const int64_t pairs = (tiles + 1) / 2;
-  const int blocks = static_cast<int>(pairs < sms ? pairs : sms);
+  const int64_t slots = static_cast<int64_t>(sms) * (D == 64 ? 2 : 1);   // CTAs resident per SM
+  const int blocks = static_cast<int>(pairs < slots ? pairs : slots);
   kern<<<blocks, kTcThreads, smem, stream>>>(xmap, p);
   return tq::launch_status();
 }
