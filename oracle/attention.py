@@ -96,6 +96,49 @@ def decode_attention(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cach
     return out
 
 
+def decode_attention_nsn(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, k_s1, k_o, v_s1, v_o,
+                         scale: float) -> np.ndarray:
+    """decode_attention over NSN records ([NSNQuant] §1, §4; codec.nsn_encode):
+    key t of sequence (b, j) is k'^_t + s1k_t o_k[b, j] and value t is
+    v'^_t + s1v_t o_v[b, j], so
+
+      score_t = scale * ( <q', k'^_t> + s1k_t <q', o_k> )
+      out     = sum_t p_t v'^_t + o_v sum_t p_t s1v_t
+
+    with q' = RoPE(q) and k'^, v'^ the codec's estimates of the shifted
+    records (scored as in decode_attention).  k_s1, v_s1 [B, Hkv, T];
+    k_o, v_o [B, Hkv, d].  Returns out [B, Hq, d] float64."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, d = q.shape
+    kc, kz, kn, kr = _unpack_cache(rot_k, *k_cache)
+    vc, vz, vn, vr = _unpack_cache(rot_v, *v_cache)
+    k_s1, k_o = np.asarray(k_s1, dtype=np.float64), np.asarray(k_o, dtype=np.float64)
+    v_s1, v_o = np.asarray(v_s1, dtype=np.float64), np.asarray(v_o, dtype=np.float64)
+    Hkv, T = kc.shape[1], kc.shape[2]
+    g = Hq // Hkv
+    out = np.zeros((B, Hq, rot_v.d))
+    if T == 0:
+        return out
+    for b in range(B):
+        qr = q[b]
+        if rot_k.rope_base:
+            qr = apply_rope(qr, np.full(Hq, q_pos[b]), rot_k.rope_base)
+        for h in range(Hq):
+            j = h // g
+            qt = qr[h] @ rot_k.pi.T
+            sq = rot_k.s @ qt
+            kzs = np.where(kz[b, j], 1.0, -1.0)
+            score = (rot_k.levels[kc[b, j]] @ qt) * kn[b, j] + (kzs @ sq) * (QJL_CONST / rot_k.m) * kr[b, j]
+            score = scale * (score + k_s1[b, j] * (qr[h] @ k_o[b, j]))
+            p = np.exp(score - np.max(score))
+            p = p / np.sum(p)
+            vzs = np.where(vz[b, j], 1.0, -1.0)
+            rotated = (p * vn[b, j]) @ rot_v.levels[vc[b, j]] + \
+                (QJL_CONST / rot_v.m) * (((p * vr[b, j]) @ vzs) @ rot_v.s)
+            out[b, h] = rotated @ rot_v.pi + v_o[b, j] * (p @ v_s1[b, j])
+    return out
+
+
 def encoder_attention(rot_k: Rotation, rot_v: Rotation, q, k_cache, v_cache, scale: float,
                       q_pos_offset: int = 0) -> np.ndarray:
     """Bidirectional attention of S queries per head over the whole cache.

@@ -177,8 +177,7 @@ def dequantize_mse_only(rot: Rotation, codes, norm, rotated: bool = False) -> np
 
 
 # ---------------------------------------------------------------------------
-# Normalize-Shift-Normalize pre-transform ([NSNQuant] §1), for comparison
-# (test infrastructure; the CUDA path has no NSN step).  For a block of l
+# Normalize-Shift-Normalize pre-transform ([NSNQuant] §1).  For a block of l
 # tokens x [l, d]:
 #   x1 = x sqrt(d) / ||x||           per token, s1 = ||x|| / sqrt(d)
 #   o  = mean over the block's tokens of x1, per channel
@@ -201,3 +200,38 @@ def nsn_forward(x):
 def nsn_inverse(x3, s1, o, s2):
     """x = s1 (s2 x3 + o)."""
     return np.asarray(s1)[:, None] * (np.asarray(s2)[:, None] * np.asarray(x3) + np.asarray(o)[None, :])
+
+
+# ---------------------------------------------------------------------------
+# NSN as a record mode of the codec ([NSNQuant] §1 and §4).  For one block of
+# tokens (one sequence and head), RoPE first (the codec's codes live in the
+# space after RoPE, [TurboESM] §2.A), then (x3, s1, o, s2) = nsn_forward(x~).
+# The codec encodes x' = s1 s2 x3 = x~ - s1 o without RoPE, so its record
+# holds the direction of x3 and the norms ||x'|| = s1 s2 sqrt(d) and
+# ||r'|| = s1 s2 ||r3||; s1 per token and o per block are kept beside it.
+# Dequantization: x^ = x'^ + s1 o, the inverse of the page's transform with
+# x3 replaced by its reconstruction.  (NSNQuant applies NSN before RoPE; with
+# the shift after RoPE the score term s1 <q', o> needs one dot product per
+# query and block instead of one per token.)
+# ---------------------------------------------------------------------------
+def nsn_encode(rot: Rotation, x, pos=None) -> dict:
+    """Encode one block x [l, d] with NSN: the codec dict of x' plus the
+    per-token s1 [l] and the block shift o [d] (both in the space after
+    RoPE)."""
+    x = np.asarray(x, dtype=np.float64)
+    if rot.rope_base and pos is not None:
+        x = apply_rope(x, np.asarray(pos), rot.rope_base)
+    x3, s1, o, s2 = nsn_forward(x)
+    xp = (s1 * s2)[:, None] * x3
+    e = encode(rot, xp, None)
+    e["s1"] = s1
+    e["o"] = o
+    e["x_nsn"] = x
+    e["x_shift"] = xp
+    return e
+
+
+def dequantize_nsn(rot: Rotation, codes, signs, norm, rnorm, s1, o) -> np.ndarray:
+    """x^ [n, d] = dequantize(record of x') + s1 o (space after RoPE)."""
+    xp = dequantize(rot, codes, signs, norm, rnorm)
+    return xp + np.asarray(s1, dtype=np.float64)[:, None] * np.asarray(o, dtype=np.float64)[None, :]
