@@ -49,7 +49,8 @@ UNIT = "tokens/s"
 SPLIT_TRAFFIC_PER_TOKEN = (235_722_240 + 5_576_448) / (16 * 8 * 16384)
 
 EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1",
-          "decode_llama8b_layer_window", "tiny_d128_t1024", "encode_esm2_33_layers", "memory_esm2")
+          "decode_llama8b_layer_window", "tiny_d128_t1024", "encode_esm2_33_layers", "memory_esm2",
+          "decode_llama8b_layer_nsn")
 
 
 def parse():
@@ -370,7 +371,8 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, 
             ({"decode_llama8b_layer_3p1"}, lambda: _extra_decode_3p1(dev, peak_gbs)),
             ({"decode_llama8b_layer_window"}, lambda: _extra_decode_window(dev, peak_gbs)),
             ({"tiny_d128_t1024"}, lambda: _extra_tiny(dev)),
-            ({"encode_esm2_33_layers"}, lambda: _extra_encode_esm2(dev, peak_gbs, g))]
+            ({"encode_esm2_33_layers"}, lambda: _extra_encode_esm2(dev, peak_gbs, g)),
+            ({"decode_llama8b_layer_nsn"}, lambda: _extra_decode_nsn(dev, peak_gbs))]
     for names, run in runs:
         if not names & select:
             continue
@@ -598,6 +600,41 @@ def _extra_decode_window(dev, peak_gbs, R=128):
                                             "ms": round(ms_w, 4), "ms_all_packed": round(ms_p, 4),
                                             "frac_hbm": round(byts / ms_w / 1e6 / peak_gbs, 4),
                                             "flush_ms": round(ms_f, 4), "flush_rows": 2 * B * Hkv * R}}
+
+def _extra_decode_nsn(dev, peak_gbs):
+    """One layer of the Llama-3.1-8B-shaped decode (B16, Hq32, Hkv8, 2+1
+    bits, T 32768) over NSN records ([NSNQuant] §1): the NSN encode of the
+    layer's keys (RoPE) and values (tq_nsn_shift, then the codec on the
+    shifted rows) and the decode with the s1 and o terms, against the plain
+    decode of the same records.  The s1 arrays add 4 B per record to the
+    112 B of the record pair."""
+    import torch
+    import synth
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["llama31_8b_gqa_decode"]
+    B, Hq, Hkv, d, T, seed = c["batch"], c["q_heads"], c["kv_heads"], c["head_dim"], c["tokens"], c["seed"]
+    rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 11, 1]), rope_base=c["rope_base"], rope_max_pos=T)
+    rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 11, 2]))
+    xk = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, 11, 3], dev)
+    kc, ks1, ko = tq.quantize_kv_nsn(rk, xk, apply_rope=True)
+    enc_k = _time_ms(lambda: tq.quantize_kv_nsn(rk, xk, apply_rope=True, out=kc), reps=3, warm=1)
+    del xk
+    xv = synth.heavy_tailed_torch((B, Hkv, T, d), [seed, 11, 4], dev)
+    vc, vs1, vo = tq.quantize_kv_nsn(rv, xv)
+    enc_v = _time_ms(lambda: tq.quantize_kv_nsn(rv, xv, out=vc), reps=3, warm=1)
+    del xv
+    q = synth.heavy_tailed_torch((B, Hq, d), [seed, 11, 5], dev)
+    qpos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    o = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ws = tq.alloc_workspace(tq.decode_workspace_size(rk, rv, B, Hq, Hkv, T), dev)
+    ms = _time_ms(lambda: tq.decode_attention_nsn(rk, rv, q, qpos, kc, vc, ks1, ko, vs1, vo, T, out=o, workspace=ws),
+                  reps=20, warm=3)
+    ms_p = _time_ms(lambda: tq.decode_attention(rk, rv, q, qpos, kc, vc, T, out=o, workspace=ws), reps=20, warm=3)
+    byts = B * Hkv * T * 2 * (rec_bytes({"head_dim": d}, argparse.Namespace(bits=2)) + 4)
+    return {"decode_llama8b_layer_nsn": {"value": B * Hkv * T / ms * 1e3, "unit": "tokens/s", "ms": round(ms, 4),
+                                         "ms_plain": round(ms_p, 4), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4),
+                                         "encode_ms": round(enc_k + enc_v, 4)}}
+
 
 def _extra_tiny(dev):
     """The tiny workload (1 head, d 128, 1024 fp32 tokens, heavy-tailed with

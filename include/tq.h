@@ -303,6 +303,29 @@ int tq_quantize_kv_pair_scatter(const tq_rotation* hk, const void* xk,
                                 int64_t n_records, void* stream);
 
 /*
+ * tq_nsn_shift - the Normalize-Shift-Normalize transform of [NSNQuant] §1
+ * as a shift ahead of the codec (the NSN record mode).  For each of n_blocks
+ * blocks of L rows (a sequence and head), after RoPE at positions
+ * pos_offset + t when apply_rope (the handle's base; [TurboESM] §2.A):
+ *   s1_t = ||x~_t|| / sqrt(d),  o = mean_t x~_t / s1_t (per channel),
+ *   x'_t = x~_t - s1_t o  (= s1 s2 x3 of the page: x3's direction, norm
+ *          s1 s2 sqrt(d))
+ * tq_quantize_kv of x' without RoPE then writes the records; s1 and o are
+ * kept beside them for tq_decode_attention_nsn.
+ *   h           handle (d = 64 or 128; its RoPE tables when apply_rope)
+ *   x           device rows in dtype, row b*L + t at x + (b*L + t)*ld
+ *   x_shift     device [n_blocks*L, d] float32 output x'
+ *   s1          device [n_blocks*L] float32 output
+ *   o           device [n_blocks, d] float32 output
+ * Zero rows have s1 = 0 and add nothing to o.  Returns TQ_OK, TQ_EINVAL,
+ * TQ_EUNSUPPORTED or TQ_ECUDA.
+ */
+int tq_nsn_shift(const tq_rotation* h, const void* x, int dtype,
+                 int64_t n_blocks, int64_t L, int64_t ld, int64_t pos_offset,
+                 int apply_rope, float* x_shift, float* s1, float* o,
+                 void* stream);
+
+/*
  * tq_quantize_dense - encode n vectors with a dense-rotation handle
  * (TQ_ROT_DENSE).  Same steps and record format as tq_quantize_kv, without
  * RoPE; y = Pi x and S r are dense contractions here, computed as fp32 GEMMs
@@ -400,6 +423,33 @@ int tq_decode_attention(const tq_rotation* hk, const tq_rotation* hv,
                         int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
                         const int32_t* seq_lens, float scale, float* out,
                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * tq_decode_attention_nsn - tq_decode_attention over records written in the
+ * NSN mode (tq_nsn_shift, then tq_quantize_kv of the shifted rows):
+ * [NSNQuant] §1 and §4, "the attention score uses s1, s2, o directly".  Key t
+ * of a sequence stands for k'_t + s1k_t o_k and value t for v'_t + s1v_t o_v
+ * (k', v' the records' vectors), so
+ *   score_t = scale (<q', k'^_t> + s1k_t <q', o_k>),
+ *   out     = sum_t p_t v'^_t + o_v sum_t p_t s1v_t.
+ *   k_s1, v_s1  device float32 s1 of every record, indexed as the norms
+ *               ((b*Hkv + j)*cache_stride + t); 16-byte aligned
+ *   k_o, v_o    device [B*Hkv, d] float32 shifts (keys: after RoPE)
+ *   cache_stride  as tq_decode_attention, and a multiple of 4
+ *   other arguments and the workspace as tq_decode_attention
+ * Returns TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_decode_attention_nsn(const tq_rotation* hk, const tq_rotation* hv,
+                            const void* q, int q_dtype, const int64_t* q_pos,
+                            const uint8_t* k_codes, const uint8_t* k_signs,
+                            const float* k_norms, const uint8_t* v_codes,
+                            const uint8_t* v_signs, const float* v_norms,
+                            const float* k_s1, const float* k_o,
+                            const float* v_s1, const float* v_o,
+                            int64_t cache_stride, int B, int Hq, int Hkv,
+                            int64_t T, const int32_t* seq_lens, float scale,
+                            float* out, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /*
  * tq_decode_attention_append - one decode step with the new token's key and

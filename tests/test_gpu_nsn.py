@@ -1,0 +1,154 @@
+"""GPU parity of the NSN record mode ([NSNQuant] §1, §4) against the oracle:
+tq_nsn_shift + the codec (s1, o and the records of the shifted rows), and
+tq_decode_attention_nsn over NSN records (oracle-packed, and end to end)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from helpers import assert_close, compare_records, oracle_rotation
+from oracle import attention as at
+from oracle import codec
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_rot(d, bits, seed, rope):
+    from vector_quantization_b200 import tq
+    return tq.Rotation(d, bits, synth.rotation_randomness(d, seed), "hadamard", rope_base=rope,
+                       rope_max_pos=(1 << 16) if rope else 0)
+
+
+def _offset_rows(shape, seed, offset=4.0):
+    """Heavy-tailed rows plus 8 channels offset by +-offset in every token of
+    a block (the case NSN's shift removes)."""
+    x = synth.heavy_tailed(shape, seed).astype(np.float64)
+    g = np.random.default_rng(seed)
+    *lead, L, d = shape
+    for idx in np.ndindex(*lead):
+        ch = g.choice(d, 8, replace=False)
+        x[idx][:, ch] += offset * np.where(g.random(8) < 0.5, -1.0, 1.0)
+    return x.astype(np.float32)
+
+
+@pytest.mark.parametrize("d,bits,rope,dtype", [(128, 2, 10000.0, torch.float32), (128, 3, 0.0, torch.bfloat16),
+                                               (64, 2, 10000.0, torch.bfloat16), (64, 1, 0.0, torch.float32)])
+@pytest.mark.parametrize("L", [300, 20000])
+def test_nsn_encode_parity(cuda_device, d, bits, rope, dtype, L):
+    """s1, o and the records of the shifted rows against nsn_encode; L = 20000
+    takes the tensor-core encode for the shifted rows."""
+    from vector_quantization_b200 import tq
+    nb = 2
+    x = _offset_rows((nb, L, d), 30 + d + bits)
+    xt = torch.from_numpy(x).to(cuda_device).to(dtype)
+    xin = xt.float().cpu().numpy().astype(np.float64)   # the rows as the GPU sees them
+    g = _gpu_rot(d, bits, 40 + bits, rope)
+    o_rot, _ = oracle_rotation(d, bits, 40 + bits, rope=rope)
+    rec, s1, o = tq.quantize_kv_nsn(g, xt, apply_rope=bool(rope), pos_offset=5)
+    torch.cuda.synchronize()
+    for b in range(nb):
+        e = codec.nsn_encode(o_rot, xin[b], np.arange(L) + 5 if rope else None)
+        np.testing.assert_allclose(s1[b].cpu().numpy(), e["s1"], rtol=2e-6, atol=0)
+        np.testing.assert_allclose(o[b].cpu().numpy(), e["o"], rtol=0, atol=2e-6 * math.sqrt(d))
+        compare_records(o_rot, tuple(a[b].cpu().numpy() for a in rec), e)
+
+
+def _nsn_caches(rot, x, pos, cap):
+    """Oracle NSN records of blocks x [B, H, T, d] in caches of capacity cap
+    (records past T poisoned), s1 [B, H, cap] (NaN past T), o [B, H, d]."""
+    B, H, T, d = x.shape
+    codes = np.full((B, H, cap, rot.bits * d // 8), 0xFF, np.uint8)
+    signs = np.full((B, H, cap, rot.m // 8), 0xFF, np.uint8)
+    norms = np.full((B, H, cap, 2), np.nan, np.float32)
+    s1 = np.full((B, H, cap), np.nan, np.float32)
+    o = np.zeros((B, H, d), np.float32)
+    for b in range(B):
+        for h in range(H):
+            e = codec.nsn_encode(rot, x[b, h], pos)
+            codes[b, h, :T] = codec.pack_planes(e["codes"], rot.bits)
+            signs[b, h, :T] = codec.pack_bits(e["signs"])
+            norms[b, h, :T] = np.stack([e["norm"], e["rnorm"]], axis=1)
+            s1[b, h, :T] = e["s1"]
+            o[b, h] = e["o"]
+    return (codes, signs, norms), s1, o
+
+
+@pytest.mark.parametrize("G,bits,T", [(4, 2, 300), (1, 3, 17), (8, 1, 1000), (2, 2, 1)])
+def test_nsn_decode_parity(cuda_device, G, bits, T):
+    from vector_quantization_b200 import tq
+    d, B, Hkv = 128, 2, 2
+    Hq, cap = G * Hkv, T + 8 - (T % 4)
+    rk, rv = _gpu_rot(d, bits, 60 + bits, 10000.0), _gpu_rot(d, bits, 70 + bits, 0.0)
+    ork, _ = oracle_rotation(d, bits, 60 + bits, rope=10000.0)
+    orv, _ = oracle_rotation(d, bits, 70 + bits)
+    k = _offset_rows((B, Hkv, T, d), 80 + G).astype(np.float64)
+    v = _offset_rows((B, Hkv, T, d), 90 + G).astype(np.float64)
+    kc, ks1, ko = _nsn_caches(ork, k, np.arange(T), cap)
+    vc, vs1, vo = _nsn_caches(orv, v, None, cap)
+    dev = cuda_device
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    q = synth.heavy_tailed((B, Hq, d), 7 + G)
+    q_pos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    out = tq.decode_attention_nsn(rk, rv, to(q), q_pos, tuple(map(to, kc)), tuple(map(to, vc)), to(ks1), to(ko),
+                                  to(vs1), to(vo), T)
+    torch.cuda.synchronize()
+    ref = at.decode_attention_nsn(ork, orv, q, [T - 1] * B, tuple(a[:, :, :T] for a in kc),
+                                  tuple(a[:, :, :T] for a in vc), ks1[:, :, :T], ko, vs1[:, :, :T], vo,
+                                  1 / math.sqrt(d))
+    assert_close(out.cpu().numpy(), ref, what=f"NSN decode G {G} bits {bits} T {T}")
+
+
+def test_nsn_decode_ragged_lengths(cuda_device):
+    from vector_quantization_b200 import tq
+    d, B, Hkv, G, T, bits = 128, 3, 2, 4, 500, 2
+    Hq, cap = G * Hkv, 504
+    rk, rv = _gpu_rot(d, bits, 61, 10000.0), _gpu_rot(d, bits, 71, 0.0)
+    ork, _ = oracle_rotation(d, bits, 61, rope=10000.0)
+    orv, _ = oracle_rotation(d, bits, 71)
+    k = _offset_rows((B, Hkv, T, d), 81).astype(np.float64)
+    v = _offset_rows((B, Hkv, T, d), 91).astype(np.float64)
+    kc, ks1, ko = _nsn_caches(ork, k, np.arange(T), cap)
+    vc, vs1, vo = _nsn_caches(orv, v, None, cap)
+    dev = cuda_device
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    lens = [500, 1, 0]
+    q = synth.heavy_tailed((B, Hq, d), 5)
+    q_pos = torch.tensor([max(n - 1, 0) for n in lens], dtype=torch.int64, device=dev)
+    out = tq.decode_attention_nsn(rk, rv, to(q), q_pos, tuple(map(to, kc)), tuple(map(to, vc)), to(ks1), to(ko),
+                                  to(vs1), to(vo), T, seq_lens=torch.tensor(lens, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    out = out.cpu().numpy()
+    assert np.all(out[2] == 0)
+    for b in range(2):
+        # the shift o of a block covers all T tokens; attention reads the first lens[b]
+        n = lens[b]
+        ref = at.decode_attention_nsn(ork, orv, q[b:b + 1], [n - 1], tuple(a[b:b + 1, :, :n] for a in kc),
+                                      tuple(a[b:b + 1, :, :n] for a in vc), ks1[b:b + 1, :, :n], ko[b:b + 1],
+                                      vs1[b:b + 1, :, :n], vo[b:b + 1], 1 / math.sqrt(d))
+        assert_close(out[b:b + 1], ref, what=f"NSN ragged seq {b}")
+
+
+def test_nsn_end_to_end(cuda_device):
+    """GPU NSN encode of keys (RoPE) and values, then GPU NSN decode, against
+    the oracle's encode and decode of the same rows."""
+    from vector_quantization_b200 import tq
+    d, B, Hkv, G, T, bits = 128, 2, 2, 4, 1500, 2
+    Hq, cap = G * Hkv, 1500
+    dev = cuda_device
+    rk, rv = _gpu_rot(d, bits, 62, 10000.0), _gpu_rot(d, bits, 72, 0.0)
+    ork, _ = oracle_rotation(d, bits, 62, rope=10000.0)
+    orv, _ = oracle_rotation(d, bits, 72)
+    k = _offset_rows((B, Hkv, T, d), 83)
+    v = _offset_rows((B, Hkv, T, d), 93)
+    kr, ks1, ko = tq.quantize_kv_nsn(rk, torch.from_numpy(k).to(dev), apply_rope=True)
+    vr, vs1, vo = tq.quantize_kv_nsn(rv, torch.from_numpy(v).to(dev))
+    q = synth.heavy_tailed((B, Hq, d), 9)
+    q_pos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    out = tq.decode_attention_nsn(rk, rv, torch.from_numpy(q).to(dev), q_pos, kr, vr, ks1, ko, vs1, vo, T)
+    torch.cuda.synchronize()
+    okc, oks1, oko = _nsn_caches(ork, k.astype(np.float64), np.arange(T), cap)
+    ovc, ovs1, ovo = _nsn_caches(orv, v.astype(np.float64), None, cap)
+    ref = at.decode_attention_nsn(ork, orv, q, [T - 1] * B, okc, ovc, oks1, oko, ovs1, ovo, 1 / math.sqrt(d))
+    assert_close(out.cpu().numpy(), ref, what="NSN end to end")

@@ -73,7 +73,17 @@ struct DecodeParams {
   const int32_t* seq_lens; // [B] tokens of each sequence (<= T), or null: all T
   int Hkv;
   int append;              // the preceding launch writes each sequence's last record: no copy before its end
+  // NSN record mode ([NSNQuant] §1): s1 of every record (same indexing as the
+  // norms) and <q', o_k> per query head ([BH][8], from q-prep)
+  const float* k_s1;
+  const float* v_s1;
+  const float* qo;
 };
+
+// Floats of one partial record: m, l, O_code [kD], O_z [kD], and for the NSN
+// mode sum_t p_t s1v_t and a pad.
+template <bool NSN>
+constexpr int partial_rec() { return 2 + 2 * kD + (NSN ? 2 : 0); }
 
 
 // Key-side MMA groups of the split kernel (m16n8k32, u8 bits x s8 query
@@ -126,14 +136,15 @@ __device__ __forceinline__ void fwht_group(float& v, int i, float* buf) {
   }
 }
 
-template <int BITS, int G>
+template <int BITS, int G, bool NSN>
 __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kernel(DecodeParams p) {
   constexpr int NT = (2 * G + 7) / 8;
   constexpr int P = Planes<BITS>::P;
   constexpr int CB = BITS * kD / 8;
   constexpr int SB = kD / 8;
-  constexpr int HALF = kTile * (CB + SB + 8);
+  constexpr int HALF = kTile * (CB + SB + 8 + (NSN ? 4 : 0));   // codes, signs, norms (, s1) of one side
   constexpr int STAGE = 2 * HALF;
+  constexpr int S1OFF = kTile * (CB + SB + 8);
   constexpr int CCH = kTile * CB / 16;
   extern __shared__ __align__(16) uint8_t smem[];
 
@@ -186,6 +197,11 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   const uint32_t dst_sign = sg_side * HALF + kTile * CB + sg_c * 16;
   const uint8_t* src_norm = reinterpret_cast<const uint8_t*>((nm_side ? p.v_norms : p.k_norms) + tok0) + nm_c * 16;
   const uint32_t dst_norm = nm_side * HALF + kTile * (CB + SB) + nm_c * 16;
+  // NSN: lanes 16..23 copy the tile's s1 (four tokens per lane; keys, then values)
+  const int s1_side = (lane >> 2) & 1, s1_c = lane & 3;
+  const uint8_t* src_s1 = nullptr;
+  if constexpr (NSN) src_s1 = reinterpret_cast<const uint8_t*>((s1_side ? p.v_s1 : p.k_s1) + tok0) + s1_c * 16;
+  const uint32_t dst_s1 = s1_side * HALF + S1OFF + s1_c * 16;
   constexpr int64_t kStepTok = static_cast<int64_t>(kWarps) * kTile;
   const int64_t n_full = (t_end - t_begin) / kTile;   // full tiles of the split (t_end >= t_begin or none)
   const int my_full = t_end > t_begin && n_full > warp ? static_cast<int>((n_full - warp + kWarps - 1) / kWarps) : 0;
@@ -200,6 +216,9 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
           if (lane + 32 * k < CCH) cp_async16(stg + dst_code[side][k], src_code[side][k] + adv * CB, 16);
       cp_async16(stg + dst_sign, src_sign + adv * SB, 16);
       if (lane < 16) cp_async16(stg + dst_norm, src_norm + adv * 8, 16);
+      if constexpr (NSN) {
+        if (lane >= 16 && lane < 24) cp_async16(stg + dst_s1, src_s1 + adv * 4, 16);
+      }
     } else if (i < my_count) {
       const int64_t t0 = seq + t_begin + static_cast<int64_t>(warp + kWarps * i) * kTile;
       const int nv = tile_nv(i);
@@ -222,6 +241,13 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
         const float2* src = (nm_side ? p.v_norms : p.k_norms) + t0;
         const int bytes = max(0, min(16, (nv - 2 * nm_c) * 8));
         cp_async16(stg + nm_side * HALF + kTile * (CB + SB) + nm_c * 16, bytes ? src + 2 * nm_c : src, bytes);
+      }
+      if constexpr (NSN) {
+        if (lane >= 16 && lane < 24) {
+          const float* src = (s1_side ? p.v_s1 : p.k_s1) + t0;
+          const int bytes = max(0, min(16, (nv - 4 * s1_c) * 4));
+          cp_async16(stg + s1_side * HALF + S1OFF + s1_c * 16, bytes ? src + 4 * s1_c : src, bytes);
+        }
       }
     }
     cp_async_commit();
@@ -247,6 +273,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   constexpr int NTK = 2 * NT;
   __shared__ uint2 s_qf[MG][NTK][32];
   float4 kc[NT];
+  float qo[NT];   // NSN: score_scale <q', o_k> of head tig + 4 nt
   {
     const uint2* src = reinterpret_cast<const uint2*>(p.qfrag) + static_cast<size_t>(bh) * (MG * NTK * 32);
     for (int i = threadIdx.x; i < MG * NTK * 32; i += blockDim.x) (&s_qf[0][0][0])[i] = src[i];
@@ -258,17 +285,18 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       float4 c = h < G ? p.kconst[static_cast<size_t>(bh) * 8 + h] : make_float4(0.f, 0.f, 0.f, 0.f);
       const float zs = p.qjl * p.score_scale;
       kc[nt] = make_float4(c.x * p.score_scale, c.y * p.score_scale, c.z * zs, c.w * zs);
+      if constexpr (NSN) qo[nt] = h < G ? p.qo[static_cast<size_t>(bh) * 8 + h] * p.score_scale : 0.f;
     }
     __syncthreads();
   }
   float accC[NT][8][4], accZ[NT][8][4];
   float m_run[NT], l_run[NT];
-  float sbc[NT], sbz[NT];
+  float sbc[NT], sbz[NT], s1sum[NT];   // s1sum: NSN, sum_t p_t s1v_t of this lane's tokens
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     m_run[nt] = -INFINITY;
     l_run[nt] = 0.f;
-    sbc[nt] = sbz[nt] = 0.f;
+    sbc[nt] = sbz[nt] = s1sum[nt] = 0.f;
 #pragma unroll
     for (int rb = 0; rb < 8; ++rb)
 #pragma unroll
@@ -352,7 +380,8 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
         const float sgn = fmaf(digits_to_float(accs[2 * nt][2 * e], accs[2 * nt][2 * e + 1],
                                                accs[2 * nt + 1][2 * e], accs[2 * nt + 1][2 * e + 1]),
                                kc[nt].z, -kc[nt].w);
-        const float l = fmaf(knorm[e].x, code, knorm[e].y * sgn);
+        float l = fmaf(knorm[e].x, code, knorm[e].y * sgn);
+        if constexpr (NSN) l = fmaf(reinterpret_cast<const float*>(stg + S1OFF)[gid + 8 * e], qo[nt], l);
         logit[nt][e] = gid + 8 * e < nv ? l : -INFINITY;
       }
     }
@@ -376,6 +405,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
         l_run[nt] *= alpha;
         sbc[nt] *= alpha_b;
         sbz[nt] *= alpha_b;
+        if constexpr (NSN) s1sum[nt] *= alpha_b;
 #pragma unroll
         for (int rb = 0; rb < 8; ++rb)
 #pragma unroll
@@ -470,6 +500,11 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       // w by at most 2^-17 |w|, far inside the output tolerance)
       sbc[nt] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
       sbz[nt] += (wr[0] + wr[1]) + (wr[2] + wr[3]);
+      if constexpr (NSN) {
+        const float* vs1 = reinterpret_cast<const float*>(vcd + S1OFF);   // zero-filled past the tile's end
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s1sum[nt] = fmaf(pt[j], vs1[tk[j]], s1sum[nt]);
+      }
 #pragma unroll
       for (int rb = 0; rb < 8; ++rb) {
 #pragma unroll
@@ -529,7 +564,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   }
   __syncthreads();
 
-  constexpr int REC = 2 + 2 * kD;
+  constexpr int REC = partial_rec<NSN>();
   float* mbuf = reinterpret_cast<float*>(smem);
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -551,11 +586,22 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
     for (int pl = 0; pl < P; ++pl) wsum += p.walsh_v[pl];
     const float SBc = __shfl_sync(0xffffffffu, bc_sum, 8 * tig) * wsum;
     const float SBz = __shfl_sync(0xffffffffu, bz_sum, 8 * tig);
+    float S1v = 0.f;
+    if constexpr (NSN) {   // the same reduction as the weight sums
+      float v = s1sum[nt];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      S1v = __shfl_sync(0xffffffffu, v, 8 * tig);
+    }
     if (h < G) {
       float* dst = mbuf + (warp * G + h) * REC;
       if (gid == 0) {
         dst[0] = m_run[nt];
         dst[1] = l;
+        if constexpr (NSN) {
+          dst[2 + 2 * kD] = S1v;
+          dst[3 + 2 * kD] = 0.f;
+        }
       }
 #pragma unroll
       for (int rb = 0; rb < 8; ++rb) {
@@ -615,6 +661,8 @@ struct QPrepArgs {
   WalshWeights walsh;
   uint32_t* qfrag;
   float4* kconst;
+  const float* o_k;        // NSN: the key shift o of each sequence [BH][kD] (or null)
+  float* qo;               // NSN: <q', o_k> per query head [BH][8]
 };
 
 template <typename T, int G, int BITS>
@@ -663,6 +711,14 @@ __device__ __forceinline__ void qprep_body(const QPrepArgs<T>& a, int bh) {
       const float x1 = buf[h][j], x2 = buf[h][j + kD / 2];
       v = i < kD / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
     }
+  }
+  // NSN: <q', o_k> of this head (q' after RoPE), summed over the group
+  __shared__ float qsum[G][kD / 32];
+  if (a.o_k) {
+    float t = v * a.o_k[static_cast<size_t>(bh) * kD + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) qsum[h][wg] = t;
   }
   // q~ = H (D q) / sqrt(d)
   v *= dsigns[i];
@@ -762,6 +818,7 @@ __device__ __forceinline__ void qprep_body(const QPrepArgs<T>& a, int bh) {
     const float cs = (red[1][h][0][0] + red[1][h][0][1]) + (red[1][h][0][2] + red[1][h][0][3]);
     const float ss = (red[1][h][1][0] + red[1][h][1][1]) + (red[1][h][1][2] + red[1][h][1][3]);
     kconst[static_cast<size_t>(bh) * 8 + h] = make_float4(ldexpf(1.f, -E[0]), wsum * cs, ldexpf(1.f, -E[1]), ss);
+    if (a.o_k) a.qo[static_cast<size_t>(bh) * 8 + h] = (qsum[h][0] + qsum[h][1]) + (qsum[h][2] + qsum[h][3]);
   }
 }
 
@@ -829,18 +886,20 @@ __global__ void __launch_bounds__(kD * G) decode_prep_kernel(const __grid_consta
 // kernel stops after the log-sum-exp combination and writes the combined
 // partial record (max, sum of weights, O_code, O_z) of each head to
 // out[(bh G + h) (2 + 2 kD)], for a later merge with other such records.
-template <int G, bool FINAL>
+template <int G, bool FINAL, bool NSN = false>
 __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __restrict__ partial, int n_splits,
                                                              int64_t bh_stride, int64_t part_stride,
                                                              const float* __restrict__ s_mat,
                                                              const float* __restrict__ dsigns, float qjl,
-                                                             float* __restrict__ out) {
-  constexpr int REC = 2 + 2 * kD;
+                                                             float* __restrict__ out,
+                                                             const float* __restrict__ v_o = nullptr) {
+  static_assert(FINAL || !NSN, "NSN records merge into the output only");
+  constexpr int REC = partial_rec<NSN>();
   constexpr int KS = kD / G;   // rows of S per group
   __shared__ __align__(16) float oz[G][kD];
   __shared__ __align__(16) float part[G][G][kD];   // [row group][head][i]
   __shared__ __align__(16) float buf[G][kD];
-  __shared__ float Ls[G], Ms[G];
+  __shared__ float Ls[G], Ms[G], S1s[G];
   extern __shared__ float fs[];   // [n_splits][G]
   const int tid = threadIdx.x, h = tid / kD, i = tid % kD, lane = tid & 31;
   const int bh = blockIdx.x;
@@ -856,19 +915,24 @@ __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __res
     for (int s = lane; s < n_splits; s += 32) M = fmaxf(M, base[static_cast<size_t>(s) * part_stride]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float l = 0.f;
+    float l = 0.f, s1 = 0.f;
     for (int s = lane; s < n_splits; s += 32) {
       const float* rec = base + static_cast<size_t>(s) * part_stride;
       const float ms = rec[0];
       const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
       fs[s * G + h] = f;
       l = fmaf(f, rec[1], l);
+      if constexpr (NSN) s1 = fmaf(f, rec[2 + 2 * kD], s1);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, o);
+      if constexpr (NSN) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    }
     if (lane == 0) {
       Ls[h] = l;
       Ms[h] = M;
+      S1s[h] = s1;
     }
   }
   __syncthreads();
@@ -907,7 +971,10 @@ __global__ void __launch_bounds__(kD * G) decode_merge_kernel(const float* __res
   // rotated-space value: O_code + sqrt(pi/2)/m S^T O_z, then Pi^T y = D H y / sqrt(d)
   float y = Ls[h] != 0.f ? (c + qjl * corr) / Ls[h] : 0.f;   // a NaN sum (a failed part) stays NaN
   fwht_group(y, i, buf[h]);
-  out[(static_cast<size_t>(bh) * G + h) * kD + i] = y * (dsigns[i] * rsqrtf(static_cast<float>(kD)));
+  float r = y * (dsigns[i] * rsqrtf(static_cast<float>(kD)));
+  // NSN values: v_t = v'_t + s1v_t o_v, so the output gains o_v sum p s1v / l
+  if constexpr (NSN) r = Ls[h] != 0.f ? fmaf(v_o[static_cast<size_t>(bh) * kD + i], S1s[h] / Ls[h], r) : r;
+  out[(static_cast<size_t>(bh) * G + h) * kD + i] = r;
 }
 
 // (cos, sin) of pos * theta_j from the two RoPE tables: the angle of the
@@ -1170,7 +1237,8 @@ size_t workspace_for(int B, int Hq, int Hkv, int64_t T, int R = 0) {
   const SplitPlan sp = plan_splits(BH, T);
   const int slots = sp.n_splits + (R + kWinChunk - 1) / kWinChunk;
   return align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)) +
-         align256(static_cast<size_t>(BH) * slots * G * (2 + 2 * kD) * sizeof(float));
+         align256(static_cast<size_t>(BH) * slots * G * partial_rec<true>() * sizeof(float)) +
+         align256(static_cast<size_t>(BH) * 8 * sizeof(float));
 }
 
 // Launch that may overlap the tail of the previous kernel on the stream
@@ -1191,14 +1259,14 @@ int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaS
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? TQ_OK : TQ_ECUDA;
 }
 
-template <int BITS, int G>
+template <int BITS, int G, bool NSN>
 int launch_split(const DecodeParams& p, int BH, cudaStream_t s) {
   constexpr int CB = BITS * kD / 8, SB = kD / 8;
-  constexpr int STAGE = 2 * kTile * (CB + SB + 8);
+  constexpr int STAGE = 2 * kTile * (CB + SB + 8 + (NSN ? 4 : 0));
   const size_t stage_bytes = static_cast<size_t>(kWarps) * kStages * STAGE;
-  const size_t merge_bytes = static_cast<size_t>(kWarps) * G * (2 + 2 * kD) * sizeof(float);
+  const size_t merge_bytes = static_cast<size_t>(kWarps) * G * partial_rec<NSN>() * sizeof(float);
   const size_t smem = stage_bytes > merge_bytes ? stage_bytes : merge_bytes;
-  auto kern = decode_split_kernel<BITS, G>;
+  auto kern = decode_split_kernel<BITS, G, NSN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return TQ_ECUDA;
   dim3 grid(p.n_splits, BH);
@@ -1267,8 +1335,10 @@ int qprep_g(int G, int BH, const QPrepArgs<T>& a, const AppendIn* app, const tq_
 
 template <typename T>
 int qprep_b(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
-            uint32_t* qfrag, float4* kconst, const AppendIn* app, cudaStream_t s) {
+            uint32_t* qfrag, float4* kconst, const AppendIn* app, const float* o_k, float* qo, cudaStream_t s) {
   QPrepArgs<T> a{};
+  a.o_k = o_k;
+  a.qo = qo;
   a.q = q;
   a.q_pos = q_pos;
   a.Hkv = Hkv;
@@ -1290,11 +1360,11 @@ int qprep_b(int G, int BH, int Hkv, const T* q, const int64_t* q_pos, const tq_r
 }
 
 int launch_qprep(int G, int q_dtype, int BH, int Hkv, const void* q, const int64_t* q_pos, const tq_rotation* hk, int rope,
-                 uint32_t* qfrag, float4* kconst, const AppendIn* app, cudaStream_t s) {
+                 uint32_t* qfrag, float4* kconst, const AppendIn* app, const float* o_k, float* qo, cudaStream_t s) {
   if (q_dtype == TQ_F32)
-    return qprep_b<float>(G, BH, Hkv, static_cast<const float*>(q), q_pos, hk, rope, qfrag, kconst, app, s);
+    return qprep_b<float>(G, BH, Hkv, static_cast<const float*>(q), q_pos, hk, rope, qfrag, kconst, app, o_k, qo, s);
   return qprep_b<__nv_bfloat16>(G, BH, Hkv, static_cast<const __nv_bfloat16*>(q), q_pos, hk, rope, qfrag, kconst,
-                                app, s);
+                                app, o_k, qo, s);
 }
 
 // Lets `kern` take `bytes` of dynamic shared memory: past the default 48 KB
@@ -1320,21 +1390,23 @@ int allow_dyn_smem(K kern, size_t bytes) {
 // final_out: the attention output [BH G][kD]; otherwise the combined partial
 // records [BH G][2 + 2 kD].
 int launch_merge(int G, int BH, const float* partial, int n_parts, int64_t bh_stride, int64_t part_stride,
-                 const tq_rotation* hv, float* out, bool final_out, cudaStream_t s) {
+                 const tq_rotation* hv, float* out, bool final_out, cudaStream_t s, const float* v_o = nullptr) {
   const float qjl = static_cast<float>(hv->res_const);
   // weights of the parts, [n_parts][G] floats: 37 KB at G = 8 with the most
   // splits a single sequence gets (1184)
   const size_t fsb = static_cast<size_t>(n_parts) * G * sizeof(float);
-#define TQ_MERGE(GG)                                                                                                \
-  {                                                                                                                 \
-    const int st = final_out ? allow_dyn_smem(decode_merge_kernel<GG, true>, fsb)                                  \
-                             : allow_dyn_smem(decode_merge_kernel<GG, false>, fsb);                                \
-    if (st != TQ_OK) return st;                                                                                     \
-  }                                                                                                                 \
-  return final_out ? launch_pdl(decode_merge_kernel<GG, true>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts,  \
-                                bh_stride, part_stride, hv->d_s, hv->d_signs, qjl, out)                             \
-                   : launch_pdl(decode_merge_kernel<GG, false>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts, \
-                                bh_stride, part_stride, hv->d_s, hv->d_signs, qjl, out)
+  const float* no_o = nullptr;
+#define TQ_MERGE_ONE(GG, FIN, NSN, VO)                                                                         \
+  {                                                                                                            \
+    const int st = allow_dyn_smem(decode_merge_kernel<GG, FIN, NSN>, fsb);                                    \
+    if (st != TQ_OK) return st;                                                                                \
+    return launch_pdl(decode_merge_kernel<GG, FIN, NSN>, dim3(BH), dim3(kD * GG), fsb, s, partial, n_parts,   \
+                      bh_stride, part_stride, hv->d_s, hv->d_signs, qjl, out, VO);                             \
+  }
+#define TQ_MERGE(GG)                                         \
+  if (v_o) TQ_MERGE_ONE(GG, true, true, v_o)                 \
+  else if (final_out) TQ_MERGE_ONE(GG, true, false, no_o)    \
+  else TQ_MERGE_ONE(GG, false, false, no_o)
   switch (G) {
     case 1: TQ_MERGE(1);
     case 2: TQ_MERGE(2);
@@ -1343,15 +1415,16 @@ int launch_merge(int G, int BH, const float* partial, int n_parts, int64_t bh_st
     default: return TQ_EUNSUPPORTED;
   }
 #undef TQ_MERGE
+#undef TQ_MERGE_ONE
 }
 
-template <int BITS>
+template <int BITS, bool NSN>
 int dispatch_g(int G, const DecodeParams& p, int BH, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_split<BITS, 1>(p, BH, s);
-    case 2: return launch_split<BITS, 2>(p, BH, s);
-    case 4: return launch_split<BITS, 4>(p, BH, s);
-    case 8: return launch_split<BITS, 8>(p, BH, s);
+    case 1: return launch_split<BITS, 1, NSN>(p, BH, s);
+    case 2: return launch_split<BITS, 2, NSN>(p, BH, s);
+    case 4: return launch_split<BITS, 4, NSN>(p, BH, s);
+    case 8: return launch_split<BITS, 8, NSN>(p, BH, s);
   }
   return TQ_EUNSUPPORTED;
 }
@@ -1407,7 +1480,9 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
                 const void* v_win, int win_dtype, int64_t win_stride, int R, int B, int Hq, int Hkv, int64_t T,
                 const int32_t* seq_lens, float scale, float* out, float* partial_out, void* workspace,
                 size_t workspace_bytes, cudaStream_t s,
-                cudaEvent_t prof_begin, cudaEvent_t prof_end, const AppendIn* app = nullptr) {
+                cudaEvent_t prof_begin, cudaEvent_t prof_end, const AppendIn* app = nullptr,
+                const float* k_s1 = nullptr, const float* k_o = nullptr, const float* v_s1 = nullptr,
+                const float* v_o = nullptr) {
   {
     const int st = check_decode_sizes(hk, hv, B, Hq, Hkv, T);
     if (st != TQ_OK) return st;
@@ -1445,9 +1520,16 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(ws);
   float4* kconst = reinterpret_cast<float4*>(ws + align256(frag_bytes(BH, G)));
   float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
+  // NSN record mode: all four side arrays, decode over the packed cache only
+  const bool nsn = k_s1 != nullptr;
+  if (nsn && (!k_o || !v_s1 || !v_o || R > 0 || partial_out || app)) return TQ_EINVAL;
+  float* qo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(partial) +
+                                       align256(static_cast<size_t>(BH) * n_slots * G * partial_rec<true>() *
+                                                sizeof(float)));
   const float score_scale = scale * 1.4426950408889634f;
 
-  int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, app, s);
+  int st = launch_qprep(G, q_dtype, BH, Hkv, q, q_pos, hk, rope, qfrag, kconst, app, nsn ? k_o : nullptr,
+                        nsn ? qo : nullptr, s);
   if (st != TQ_OK) return st;
   st = tq::launch_status();
   if (st != TQ_OK) return st;
@@ -1480,22 +1562,25 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   p.one_b = kOneB2;
   p.qjl = static_cast<float>(hk->res_const);
   p.append = app ? 1 : 0;
+  p.k_s1 = k_s1;
+  p.v_s1 = v_s1;
+  p.qo = qo;
   for (int i = 0; i < 4; ++i) {
     p.walsh_k[i] = static_cast<float>(hk->walsh[i]);
     p.walsh_v[i] = static_cast<float>(hv->walsh[i]);
   }
   if (prof_begin && cudaEventRecord(prof_begin, s) != cudaSuccess) return TQ_ECUDA;
   switch (hk->bits) {
-    case 1: st = dispatch_g<1>(G, p, BH, s); break;
-    case 2: st = dispatch_g<2>(G, p, BH, s); break;
-    case 3: st = dispatch_g<3>(G, p, BH, s); break;
+    case 1: st = nsn ? dispatch_g<1, true>(G, p, BH, s) : dispatch_g<1, false>(G, p, BH, s); break;
+    case 2: st = nsn ? dispatch_g<2, true>(G, p, BH, s) : dispatch_g<2, false>(G, p, BH, s); break;
+    case 3: st = nsn ? dispatch_g<3, true>(G, p, BH, s) : dispatch_g<3, false>(G, p, BH, s); break;
     default: st = TQ_EUNSUPPORTED;
   }
   if (st != TQ_OK) return st;
   if (prof_end && cudaEventRecord(prof_end, s) != cudaSuccess) return TQ_ECUDA;
-  const int64_t rec = 2 + 2 * kD;
+  const int64_t rec = nsn ? partial_rec<true>() : partial_rec<false>();
   return launch_merge(G, BH, partial, n_slots, static_cast<int64_t>(n_slots) * G * rec, G * rec, hv,
-                      partial_out ? partial_out : out, partial_out == nullptr, s);
+                      partial_out ? partial_out : out, partial_out == nullptr, s, nsn ? v_o : nullptr);
 }
 
 }  // namespace
@@ -1539,6 +1624,24 @@ extern "C" int tq_decode_attention_append(const tq_rotation* hk, const tq_rotati
   return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
                      nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, nullptr, workspace,
                      workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end, &app);
+}
+
+extern "C" int tq_decode_attention_nsn(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,
+                                       const int64_t* q_pos, const uint8_t* k_codes, const uint8_t* k_signs,
+                                       const float* k_norms, const uint8_t* v_codes, const uint8_t* v_signs,
+                                       const float* v_norms, const float* k_s1, const float* k_o, const float* v_s1,
+                                       const float* v_o, int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
+                                       const int32_t* seq_lens, float scale, float* out, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (!k_s1 || !k_o || !v_s1 || !v_o) return TQ_EINVAL;
+  if (T > 0 && (!tq::aligned16(k_s1) || !tq::aligned16(v_s1))) return TQ_EINVAL;   // copied 16 bytes at a time
+  if (cache_stride % 4) return TQ_EINVAL;   // each sequence's s1 row starts 16-byte aligned
+  const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
+  g_prof_begin = g_prof_end = nullptr;
+  return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
+                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, nullptr, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end, nullptr, k_s1, k_o,
+                     v_s1, v_o);
 }
 
 extern "C" int tq_decode_attention_window(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,

@@ -52,6 +52,9 @@ def _load():
                                       c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_attention_append": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64,
                                              c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
+        "tq_nsn_shift": (c_i, [c_p, c_p, c_i, c_i64, c_i64, c_i64, c_i64, c_i, c_p, c_p, c_p, c_p]),
+        "tq_decode_attention_nsn": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
+                                          c_i64, c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
         "tq_decode_partials": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
                                      c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
@@ -311,6 +314,40 @@ def quantize_kv_scatter(rot: Rotation, x, out_rows, out, *, pos=None, pos_period
     return out
 
 
+def quantize_kv_nsn(rot: Rotation, x, *, apply_rope: bool = False, pos_offset: int = 0, out=None, stream=None):
+    """NSN record mode ([NSNQuant] §1): x [..., L, d] (float32/bfloat16) as
+    blocks of L tokens (row t of a block at position pos_offset + t).  Each
+    block is shifted by tq_nsn_shift and the shifted rows x' are encoded by
+    the codec without RoPE.  Returns ((codes, signs, norms), s1, o) with the
+    records and s1 shaped [..., L] and o [..., d].  With ``out`` (record arrays
+    [..., cap, ...], cap >= L) the records land in the first L slots of each
+    block."""
+    import torch
+    *lead, L, d = x.shape
+    nb = int(np.prod(lead)) if lead else 1
+    x3 = x.reshape(nb * L, d)
+    if x3.stride(-1) != 1 or (nb * L > 1 and x3.stride(0) != d):
+        x3 = x3.contiguous()
+    xs = torch.empty((nb * L, d), dtype=torch.float32, device=x.device)
+    s1 = torch.empty((nb * L,), dtype=torch.float32, device=x.device)
+    o = torch.empty((nb, d), dtype=torch.float32, device=x.device)
+    _check(_lib.tq_nsn_shift(rot.handle, _ptr(x3), _dtype_code(x3), nb, L, d, pos_offset, 1 if apply_rope else 0,
+                             _ptr(xs), _ptr(s1), _ptr(o), _stream_ptr(stream)), "tq_nsn_shift")
+    if out is None:
+        rec = quantize_kv(rot, xs, stream=stream)
+        rec = tuple(a.view(*lead, L, -1) for a in rec)
+    else:
+        cap = out[0].shape[-2]
+        if cap == L:
+            quantize_kv(rot, xs, out=tuple(a.view(nb * L, -1) for a in out), stream=stream)
+        else:
+            rows = (torch.arange(nb, device=x.device, dtype=torch.int64).repeat_interleave(L) * cap +
+                    torch.arange(L, device=x.device, dtype=torch.int64).repeat(nb))
+            quantize_kv_scatter(rot, xs, rows, tuple(a.view(nb * cap, -1) for a in out), stream=stream)
+        rec = out
+    return rec, s1.view(*lead, L), o.view(*lead, d)
+
+
 def quantize_kv_pair_scatter(rot_k: Rotation, xk, rot_v: Rotation, xv, out_rows, out_k, out_v, *, pos=None,
                              pos_period: int | None = None, pos_offset: int = 0, apply_rope: bool = False,
                              stream=None):
@@ -431,6 +468,39 @@ def decode_attention_append(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_new, v
                                            _ptr(vn), cap, B, Hq, Hkv, T, _ptr(lens), float(scale), _ptr(out),
                                            _ptr(workspace), workspace.numel(), _stream_ptr(stream)),
            "tq_decode_attention_append")
+    return out
+
+
+def decode_attention_nsn(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_cache, k_s1, k_o, v_s1, v_o,
+                         T: int, *, seq_lens=None, scale: float | None = None, out=None, workspace=None, stream=None):
+    """decode_attention over NSN records (quantize_kv_nsn): k_s1, v_s1
+    [B, Hkv, cap] float32 beside the caches, k_o, v_o [B, Hkv, d] float32.
+    Returns out [B, Hq, d] float32."""
+    import torch
+    B, Hq, d = q.shape
+    kc, ks, kn = k_cache
+    vc, vs, vn = v_cache
+    Hkv, cap = kc.shape[1], kc.shape[2]
+    side = (k_s1, k_o, v_s1, v_o)
+    for t in (kc, ks, kn, vc, vs, vn) + side:
+        if not t.is_contiguous():
+            raise ValueError("cache and NSN arrays must be contiguous")
+    if k_s1.shape[-1] != cap or v_s1.shape[-1] != cap or k_o.numel() != B * Hkv * d or v_o.numel() != B * Hkv * d:
+        raise ValueError("s1 arrays must be [B, Hkv, cap] and shifts [B, Hkv, d]")
+    q = q.contiguous()
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(rot_k, rot_v, B, Hq, Hkv, T)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    lens = _seq_lens(seq_lens, B, q.device)
+    _check(_lib.tq_decode_attention_nsn(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos), _ptr(kc),
+                                        _ptr(ks), _ptr(kn), _ptr(vc), _ptr(vs), _ptr(vn), _ptr(k_s1), _ptr(k_o),
+                                        _ptr(v_s1), _ptr(v_o), cap, B, Hq, Hkv, T, _ptr(lens), float(scale), _ptr(out),
+                                        _ptr(workspace), workspace.numel(), _stream_ptr(stream)),
+           "tq_decode_attention_nsn")
     return out
 
 
