@@ -70,6 +70,8 @@ def parse():
                     help="context of the 70B-shaped slice for --extra runs (default 2^20)")
     ap.add_argument("--search-rows", type=int, default=None,
                     help="database rows of the search workload for --extra runs (default 10^6)")
+    ap.add_argument("--esm-layers", type=int, default=None,
+                    help="layers of the ESM-2-shaped cache encode for --extra runs (default 33)")
     return ap.parse_args()
 
 
@@ -348,7 +350,7 @@ def _time_ms(fn, reps=3, warm=2):
     return a.elapsed_time(b) / reps
 
 
-def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, cpu=True):
+def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, cpu=True, esm_layers=None):
     """Device-timed measurements of the other rows of the path, each on its
     own workload: encode and decode on the Llama-3.1-70B-shaped 1M-token
     slice, one ESM-2-650M encoder layer, and 1M-vector d=1536 search.
@@ -371,7 +373,7 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, 
             ({"decode_llama8b_layer_3p1"}, lambda: _extra_decode_3p1(dev, peak_gbs)),
             ({"decode_llama8b_layer_window"}, lambda: _extra_decode_window(dev, peak_gbs)),
             ({"tiny_d128_t1024"}, lambda: _extra_tiny(dev)),
-            ({"encode_esm2_33_layers"}, lambda: _extra_encode_esm2(dev, peak_gbs, g)),
+            ({"encode_esm2_33_layers"}, lambda: _extra_encode_esm2(dev, peak_gbs, g, esm_layers)),
             ({"decode_llama8b_layer_nsn"}, lambda: _extra_decode_nsn(dev, peak_gbs))]
     for names, run in runs:
         if not names & select:
@@ -381,7 +383,7 @@ def run_extras(dev, peak_gbs, select=None, slice_tokens=None, search_rows=None, 
         except Exception as exc:
             out[sorted(names & select)[0]] = {"error": f"{type(exc).__name__}: {exc}"}
         torch.cuda.empty_cache()
-    if cpu and not slice_tokens:
+    if cpu and not slice_tokens and not esm_layers:
         try:
             for key, b in oracle_extra_baselines(select).items():
                 if key in out and "error" not in out[key]:
@@ -664,7 +666,7 @@ def _extra_tiny(dev):
     return {"tiny_d128_t1024": {"value": round(us_dec, 2), "unit": "decode us", "encode_us": round(us_enc, 2)}}
 
 
-def _extra_encode_esm2(dev, peak_gbs, g):
+def _extra_encode_esm2(dev, peak_gbs, g, layers=None):
     """Encode of the whole ESM-2-650M-shaped cache: 33 layers x [8, 20, 1024,
     64] bf16 keys (RoPE at positions 0..1023) and values, 2+1 bits, one call
     each: 2 x 5.4M vectors.  N(0, 1) bf16 rows stand in for the log-normal
@@ -674,6 +676,7 @@ def _extra_encode_esm2(dev, peak_gbs, g):
     from vector_quantization_b200 import tq
     c = synth.CONFIGS["esm2_650m_encoder"]
     L, B, H, T, d, seed = c["layers"], c["batch"], c["heads"], c["tokens"], c["head_dim"], c["seed"]
+    L = layers or L
     n = L * B * H * T
     rk = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 1]), rope_base=c["rope_base"], rope_max_pos=T)
     rv = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 9, 2]))
@@ -887,7 +890,8 @@ def main():
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
         print(json.dumps({"extras": run_extras(dev, measured_peaks()[0], args.extra, args.slice_tokens,
-                                               args.search_rows, cpu=not args.no_cpu_baseline)}), flush=True)
+                                               args.search_rows, cpu=not args.no_cpu_baseline,
+                                               esm_layers=args.esm_layers)}), flush=True)
         return
     if world > 1:
         import datetime

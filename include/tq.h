@@ -314,11 +314,14 @@ int tq_quantize_kv_pair_scatter(const tq_rotation* hk, const void* xk,
  * kept beside them for tq_decode_attention_nsn.
  *   h           handle (d = 64 or 128; its RoPE tables when apply_rope)
  *   x           device rows in dtype, row b*L + t at x + (b*L + t)*ld
- *   x_shift     device [n_blocks*L, d] float32 output x'
+ *   n_blocks    0 .. 65535
+ *   x_shift     device [n_blocks*L, d] float32 output x' (8-byte aligned:
+ *               it holds the blocks' partial sums before x')
  *   s1          device [n_blocks*L] float32 output
  *   o           device [n_blocks, d] float32 output
- * Zero rows have s1 = 0 and add nothing to o.  Returns TQ_OK, TQ_EINVAL,
- * TQ_EUNSUPPORTED or TQ_ECUDA.
+ * Zero rows have s1 = 0 and add nothing to o.  The block sums run in double
+ * in a fixed order, so the outputs do not depend on scheduling.  Returns
+ * TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED or TQ_ECUDA.
  */
 int tq_nsn_shift(const tq_rotation* h, const void* x, int dtype,
                  int64_t n_blocks, int64_t L, int64_t ld, int64_t pos_offset,
