@@ -310,6 +310,25 @@ def oracle_extra_baselines(select):
         r, calls, per = _oracle_rate(lambda: (codec.encode(rk, x[0, 0], pos), codec.encode(rv, x[0, 1])), 2 * ne)
         out["encode_esm2_33_layers"] = base(r, "vectors/s", f"{ne} keys (RoPE) + {ne} values, d {de}, 2+1 bits; "
                                                             f"{calls} calls, {per:.2f} s each")
+    if "decode_llama8b_layer_nsn" in select:
+        c = synth.CONFIGS["llama31_8b_gqa_decode"]
+        T, G = 8192, c["q_heads"] // c["kv_heads"]
+        rk = ro.build_rotation(d, 2, synth.rotation_randomness(d, [c["seed"], 11, 1]), rope_base=c["rope_base"])
+        rv = ro.build_rotation(d, 2, synth.rotation_randomness(d, [c["seed"], 11, 2]))
+        k = synth.heavy_tailed((1, 1, T, d), [c["seed"], 11, 3]).reshape(T, d)
+        v = synth.heavy_tailed((1, 1, T, d), [c["seed"], 11, 4]).reshape(T, d)
+        q = synth.heavy_tailed((1, G, d), [c["seed"], 11, 5])
+        ek, ev = codec.nsn_encode(rk, k, np.arange(T)), codec.nsn_encode(rv, v)
+        rec = lambda e, rot: (codec.pack_planes(e["codes"], rot.bits)[None, None],
+                              codec.pack_bits(e["signs"])[None, None],
+                              np.stack([e["norm"], e["rnorm"]], 1).astype(np.float32)[None, None])
+        kc, vc = rec(ek, rk), rec(ev, rv)
+        fn = lambda: at.decode_attention_nsn(rk, rv, q, [T - 1], kc, vc, ek["s1"][None, None], ek["o"][None, None],
+                                             ev["s1"][None, None], ev["o"][None, None], 1 / np.sqrt(d))
+        r, calls, per = _oracle_rate(fn, T)
+        out["decode_llama8b_layer_nsn"] = base(r, "tokens/s", f"one (sequence, KV head), {T} of the layer's "
+                                                              f"{c['tokens']} NSN records, {G} query heads, 2+1 bits; "
+                                                              f"{calls} calls, {per:.2f} s each")
     if select & {"decode_llama8b_layer_3p1", "decode_llama8b_layer_window"}:
         c = synth.CONFIGS["llama31_8b_gqa_decode"]
         T, G = 8192, c["q_heads"] // c["kv_heads"]

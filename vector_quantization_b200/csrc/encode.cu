@@ -664,6 +664,10 @@ __device__ __forceinline__ float quantize32_x2(float2* y, const float (&tp)[4], 
 #pragma unroll
   for (int k = 0; k < BITS; ++k) w[k] = 0;
   const float2 norm2 = make_float2(norm, norm);
+  // 2 bits: level = sign(v) (mid + sign(|v| - t_0) half), both signs taken
+  // from sign bits the plane words already use (mid + half = nl[1] and
+  // mid - half = nl[0] within an ulp)
+  const uint32_t mid_b = __float_as_uint(0.5f * (nl[0] + nl[1])), half_b = __float_as_uint(0.5f * (nl[1] - nl[0]));
   float2 rr = make_float2(0.f, 0.f);
 #pragma unroll
   for (int m = 15; m >= 0; --m) {
@@ -673,24 +677,24 @@ __device__ __forceinline__ float quantize32_x2(float2* y, const float (&tp)[4], 
       const float v = e ? y[m].y : y[m].x;
       const uint32_t sy = __float_as_uint(v);
       const float a = fabsf(v);
-      float nmag;
       if constexpr (BITS == 1) {
         w[0] = __funnelshift_l(sy, w[0], 1);
-        nmag = nl[0];
+        c[e] = -copysignf(nl[0], v);
       } else if constexpr (BITS == 2) {
         const uint32_t s0 = __float_as_uint(a - tp[0]);
+        const uint32_t x = sy ^ s0;
         w[1] = __funnelshift_l(sy, w[1], 1);
-        w[0] = __funnelshift_l(sy ^ s0, w[0], 1);
-        nmag = a >= tp[0] ? nl[1] : nl[0];
+        w[0] = __funnelshift_l(x, w[0], 1);
+        c[e] = -(__uint_as_float((sy & 0x80000000u) | mid_b) + __uint_as_float((x & 0x80000000u) | half_b));
       } else {
         const uint32_t s0 = __float_as_uint(a - tp[0]), s1 = __float_as_uint(a - tp[1]),
                        s2 = __float_as_uint(a - tp[2]);
         w[2] = __funnelshift_l(sy, w[2], 1);
         w[1] = __funnelshift_l(sy ^ s1, w[1], 1);
         w[0] = __funnelshift_l(sy ^ s0 ^ s1 ^ s2, w[0], 1);
-        nmag = a >= tp[2] ? nl[3] : (a >= tp[1] ? nl[2] : (a >= tp[0] ? nl[1] : nl[0]));
+        const float nmag = a >= tp[2] ? nl[3] : (a >= tp[1] ? nl[2] : (a >= tp[0] ? nl[1] : nl[0]));
+        c[e] = -copysignf(nmag, v);
       }
-      c[e] = -copysignf(nmag, v);
     }
     const float2 r = __ffma2_rn(norm2, y[m], make_float2(c[0], c[1]));
     y[m] = r;
