@@ -73,6 +73,10 @@ def test_bad_arguments_are_rejected_on_host():
                                               None) == tq.TQ_EINVAL
     assert tq._lib.tq_decode_attention(None, None, None, 0, None, None, None, None, None, None, None, 0,
                                        1, 4, 1, 0, None, 0.125, None, None, 0, None) == tq.TQ_EINVAL
+    # NSN: null handle or buffers rejected on the host
+    assert tq._lib.tq_nsn_shift(None, None, 0, 1, 4, 128, 0, 0, None, None, None, None) == tq.TQ_EINVAL
+    assert tq._lib.tq_decode_attention_nsn(None, None, None, 0, None, None, None, None, None, None, None, None, None,
+                                           None, None, 0, 1, 4, 1, 1, None, 0.125, None, None, 0, None) == tq.TQ_EINVAL
     # fused append: missing new rows or handles rejected on the host
     assert tq._lib.tq_decode_attention_append(None, None, None, 0, None, None, None, None, None, None, None, None,
                                               None, 0, 1, 4, 1, 1, None, 0.125, None, None, 0, None) == tq.TQ_EINVAL

@@ -152,3 +152,44 @@ def test_nsn_end_to_end(cuda_device):
     ovc, ovs1, ovo = _nsn_caches(orv, v.astype(np.float64), None, cap)
     ref = at.decode_attention_nsn(ork, orv, q, [T - 1] * B, okc, ovc, oks1, oko, ovs1, ovo, 1 / math.sqrt(d))
     assert_close(out.cpu().numpy(), ref, what="NSN end to end")
+
+
+def test_nsn_shift_small_blocks_and_zero_rows(cuda_device):
+    """Blocks of one, two and 257 rows (one chunk, o written directly; two
+    chunks) with an all-zero row (s1 = 0, nothing added to o; its record is
+    the zero vector's) against nsn_encode."""
+    from vector_quantization_b200 import tq
+    d = 128
+    g = _gpu_rot(d, 2, 44, 10000.0)
+    o_rot, _ = oracle_rotation(d, 2, 44, rope=10000.0)
+    for L in (1, 2, 257):
+        x = _offset_rows((3, L, d), 50 + L)
+        x[1, 0] = 0.0
+        xt = torch.from_numpy(x).to(cuda_device)
+        rec, s1, o = tq.quantize_kv_nsn(g, xt, apply_rope=True)
+        torch.cuda.synchronize()
+        for b in range(3):
+            e = codec.nsn_encode(o_rot, x[b].astype(np.float64), np.arange(L))
+            np.testing.assert_allclose(s1[b].cpu().numpy(), e["s1"], rtol=2e-6, atol=0)
+            np.testing.assert_allclose(o[b].cpu().numpy(), e["o"], rtol=0, atol=2e-6 * math.sqrt(d))
+            # a one-row block shifts its row to x' = 0 up to rounding, whose
+            # direction is noise: its records are not compared
+            if L > 1:
+                compare_records(o_rot, tuple(a[b].cpu().numpy() for a in rec), e)
+
+
+def test_nsn_decode_empty_cache(cuda_device):
+    from vector_quantization_b200 import tq
+    d, B, Hkv, G = 128, 1, 2, 4
+    rk, rv = _gpu_rot(d, 2, 63, 10000.0), _gpu_rot(d, 2, 73, 0.0)
+    dev = cuda_device
+    cap = 8
+    kc = tq.empty_records(rk, (B, Hkv, cap), dev)
+    vc = tq.empty_records(rv, (B, Hkv, cap), dev)
+    z1 = torch.zeros((B, Hkv, cap), dtype=torch.float32, device=dev)
+    zo = torch.zeros((B, Hkv, d), dtype=torch.float32, device=dev)
+    q = torch.ones((B, G * Hkv, d), dtype=torch.float32, device=dev)
+    out = tq.decode_attention_nsn(rk, rv, q, torch.zeros((B,), dtype=torch.int64, device=dev), kc, vc, z1, zo, z1,
+                                  zo, 0)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
