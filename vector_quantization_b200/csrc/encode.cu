@@ -997,12 +997,22 @@ __global__ void __launch_bounds__(kTcThreads, D == 64 ? 2 : 1) encode_tc_kernel(
     tqtc::fence_after_sync();
     constexpr int NU = D / 4;   // float2 per thread
     float2 u[NU];   // u[m] = coordinates (d/2 c4 + 2m, + 1)
+    if constexpr (D == 128 && SPLIT) {   // both 32-column loads under one wait (the key launches)
+      float y0[32], y1[32];
+      tqtc::tmem_ld32x2(tm + tm_lane + 64 * c4, tm + tm_lane + 64 * c4 + 32, y0, y1);
 #pragma unroll
-    for (int h = 0; h < D / 64; ++h) {
-      float y[32];
-      tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * h, y);
+      for (int m = 0; m < 16; ++m) {
+        u[m] = make_float2(y0[2 * m], y0[2 * m + 1]);
+        u[16 + m] = make_float2(y1[2 * m], y1[2 * m + 1]);
+      }
+    } else {
 #pragma unroll
-      for (int m = 0; m < 16; ++m) u[16 * h + m] = make_float2(y[2 * m], y[2 * m + 1]);
+      for (int h = 0; h < D / 64; ++h) {
+        float y[32];
+        tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * h, y);
+#pragma unroll
+        for (int m = 0; m < 16; ++m) u[16 * h + m] = make_float2(y[2 * m], y[2 * m + 1]);
+      }
     }
     {
       const float2 sc2 = make_float2(scale, scale), z2 = make_float2(0.f, 0.f);
@@ -1080,14 +1090,26 @@ __global__ void __launch_bounds__(kTcThreads, D == 64 ? 2 : 1) encode_tc_kernel(
     // sign bits of S r: complemented fp32 sign bits, one funnel shift each
     // (an exact -0 projection reads as negative, within the sign tolerance)
     {
+      if constexpr (D == 128 && SPLIT) {   // both loads under one wait (the key launches)
+        float val[2][32];
+        tqtc::tmem_ld32x2(tm + tm_lane + 64 * c4, tm + tm_lane + 64 * c4 + 32, val[0], val[1]);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        float val[32];
-        tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * c, val);
-        uint32_t w = 0;
+        for (int c = 0; c < 2; ++c) {
+          uint32_t w = 0;
 #pragma unroll
-        for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[b]), w, 1);
-        if (row < p.n) p.signs[row * p.out_stride * NJ + (D / 64) * c4 + c] = ok ? ~w : 0u;
+          for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[c][b]), w, 1);
+          if (row < p.n) p.signs[row * p.out_stride * NJ + 2 * c4 + c] = ok ? ~w : 0u;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          float val[32];
+          tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * c, val);
+          uint32_t w = 0;
+#pragma unroll
+          for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[b]), w, 1);
+          if (row < p.n) p.signs[row * p.out_stride * NJ + (D / 64) * c4 + c] = ok ? ~w : 0u;
+        }
       }
       if (!ok && c4 == 0 && row < p.n) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
     }
