@@ -436,6 +436,15 @@ def _extras_70b(dev, peak_gbs, select, Hkv, Hq, d, T, seed, c):
     if "encode_70b_slice" in select:
         out["encode_70b_slice"] = {"value": nvec / ms * 1e3, "unit": "vectors/s", "ms": round(ms, 4),
                                    "GB_s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / peak_gbs, 4)}
+        # the same slice in sign-residual records (same record sizes)
+        rks = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 1]), rope_base=c["rope_base"], rope_max_pos=T,
+                          residual="sign")
+        rvs = tq.Rotation(d, 2, synth.rotation_randomness(d, [seed, 2]), residual="sign")
+        def enc_sign():
+            tq.quantize_kv(rks, k, apply_rope=True, pos_period=T, out=kc)
+            tq.quantize_kv(rvs, v, out=vc)
+        out["encode_70b_slice"]["ms_sign"] = round(_time_ms(enc_sign), 4)
+        enc()   # the QJL records again for the decode line
     del k, v
     if "decode_70b_slice" not in select:
         return out

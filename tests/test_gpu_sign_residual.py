@@ -68,6 +68,21 @@ def test_sign_mode_encode_parity(cuda_device, d, n):
     _check_records(o, tuple(a.cpu().numpy() for a in gpu), xb, pos)
 
 
+@pytest.mark.parametrize("d,bits,dtype", [(128, 2, torch.bfloat16), (128, 3, torch.float32), (64, 1, torch.bfloat16),
+                                           (64, 2, torch.float32)])
+def test_sign_mode_encode_parity_no_rope(cuda_device, d, bits, dtype):
+    """The 128-row tile kernels in sign mode without RoPE (the value
+    launches: a bf16 input enters the rotation product as one operand, fp32
+    as a hi + lo pair), 17000 rows: 132 full tiles and a ragged one."""
+    from vector_quantization_b200 import tq
+    g, o = _rots(d, bits, 407 + d + bits)
+    x = synth.heavy_tailed((17000, d), 408 + bits)
+    xt = torch.from_numpy(x).to(cuda_device).to(dtype)
+    gpu = tq.quantize_kv(g, xt)
+    torch.cuda.synchronize()
+    _check_records(o, tuple(a.cpu().numpy() for a in gpu), xt.float().cpu().numpy().astype(np.float64))
+
+
 def _oracle_cache(o, x, pos=None, cap=None):
     """The oracle's sign-mode records of x [B, H, T, d] packed as a cache
     [B, H, cap, ...] (so both sides read the same bytes), and the encodings."""

@@ -739,10 +739,13 @@ constexpr int64_t kPairsMaxRopePos = int64_t(1) << 22;
 //     coordinates y / (||x|| sqrt d), the codes and the residual (fp32x2),
 //     and write the residual as bf16 hi + lo over the A operand;
 //  5. S r into the same tensor-memory columns; the sign bits are read back.
+// SGN (sign-residual records, S = I): steps 4-5 keep no residual operand and
+// no S r product; the sign bits of r come straight from the registers and the
+// group's next tile is requested as soon as y has been read.
 // ===========================================================================
 constexpr int kTcThreads = 512;   // two groups of 8 warps
 
-template <int D, int BITS, typename T, bool SPLIT>
+template <int D, int BITS, typename T, bool SPLIT, bool SGN>
 __global__ void __launch_bounds__(kTcThreads, D == 64 ? 2 : 1) encode_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                  EncodeParams p) {
   static_assert(SPLIT || sizeof(T) == 2, "fp32 input needs the split path");
@@ -1041,77 +1044,105 @@ __global__ void __launch_bounds__(kTcThreads, D == 64 ? 2 : 1) encode_tc_kernel(
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) crec[k * NJ + (D / 64) * c4 + h] = wq[h][k];
     }
-    // residual (zero on absent rows) as bf16 hi + lo over the A operand, row r4
-    // (the staged tile was read before the barrier ahead of the products)
+    if constexpr (SGN) {
+      // sign-residual records: S is the identity, so the sign bits are those
+      // of r itself, taken from the registers (no S r product, no residual
+      // operand); the staged tile and y are consumed, so the group's next
+      // tile is requested at once
+      uint32_t ws[D / 64];
 #pragma unroll
-    for (int j = 0; j < D / 16; ++j) {
-      uint32_t hv[4], lv[4];
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t w = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 r = u[4 * j + e];
-        __nv_bfloat162 hb2 = __floats2bfloat162_rn(r.x, r.y);
-        const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb2);
-        const float2 lo =
-            __ffma2_rn(make_float2(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u)), m1, r);
-        __nv_bfloat162 lb = __floats2bfloat162_rn(lo.x, lo.y);
-        hv[e] = hbits;
-        lv[e] = *reinterpret_cast<uint32_t*>(&lb);
+        for (int b = 31; b >= 0; --b) {
+          const float2 r = u[16 * c + (b >> 1)];
+          w = __funnelshift_l(__float_as_uint((b & 1) ? r.y : r.x), w, 1);
+        }
+        ws[c] = ~w;
       }
-      const int kb = D == 128 ? c4 : 0, cb = D == 128 ? j : 4 * c4 + j;
-      const uint32_t off = kb * (kTileVec * 128) + rowbase4 + ((cb ^ (r4 & 7)) << 4);
-      *reinterpret_cast<uint4*>(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      *reinterpret_cast<uint4*>(a_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
-    }
-    // ---- 5. S r of the tile, into the columns y has left
-    tqtc::fence_smem_to_async();
-    tqtc::fence_before_sync();
-    gsync();
-    if (gt == 0 && !failed) {
+      tqtc::fence_before_sync();
+      gsync();   // the partner half's sum of |r_i| (xrr) is visible
+      if (valid && ok_y && c4 == 0) p.norms[row * p.out_stride] = make_float2(nrm, (rr + xrr[g][1][r4]) * (1.f / D));
+      if (!ok_y || !ok_x) s_fail[g] = 1;
+      if (gt == 0 && ok_y && tile + tstep < n_tiles) issue_x(tile + tstep);
+      if (row < p.n) {
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) p.signs[row * p.out_stride * NJ + (D / 64) * c4 + c] = ok_y ? ws[c] : 0u;
+        if (!ok_y && c4 == 0) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
+      }
+    } else {
+      // residual (zero on absent rows) as bf16 hi + lo over the A operand, row r4
+      // (the staged tile was read before the barrier ahead of the products)
+  #pragma unroll
+      for (int j = 0; j < D / 16; ++j) {
+        uint32_t hv[4], lv[4];
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 r = u[4 * j + e];
+          __nv_bfloat162 hb2 = __floats2bfloat162_rn(r.x, r.y);
+          const uint32_t hbits = *reinterpret_cast<uint32_t*>(&hb2);
+          const float2 lo =
+              __ffma2_rn(make_float2(__uint_as_float(hbits << 16), __uint_as_float(hbits & 0xFFFF0000u)), m1, r);
+          __nv_bfloat162 lb = __floats2bfloat162_rn(lo.x, lo.y);
+          hv[e] = hbits;
+          lv[e] = *reinterpret_cast<uint32_t*>(&lb);
+        }
+        const int kb = D == 128 ? c4 : 0, cb = D == 128 ? j : 4 * c4 + j;
+        const uint32_t off = kb * (kTileVec * 128) + rowbase4 + ((cb ^ (r4 & 7)) << 4);
+        *reinterpret_cast<uint4*>(a_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4*>(a_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+      }
+      // ---- 5. S r of the tile, into the columns y has left
+      tqtc::fence_smem_to_async();
+      tqtc::fence_before_sync();
+      gsync();
+      if (gt == 0 && !failed) {
+        tqtc::fence_after_sync();
+  #pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_hi), ks, kTileVec),
+                            tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), ids, ks > 0);
+  #pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks)
+          tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_lo), ks, kTileVec),
+                            tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), ids, true);
+        tqtc::mma_commit(&mb_s[g]);
+      }
+      if (valid && ok_y && c4 == 0)
+        p.norms[row * p.out_stride] =
+            make_float2(nrm, p.sign_res ? (rr + xrr[g][1][r4]) * (1.f / D) : sqrtf(rr + xrr[g][1][r4]));
+      const bool ok = ok_y && tqtc::mbar_wait(&mb_s[g], ph_s, kWaitLimit);
+      ph_s ^= 1;
       tqtc::fence_after_sync();
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_hi), ks, kTileVec),
-                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), ids, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-        tqtc::mma_bf16_ss(tm, tqtc::sw128_desc_kstep(tqtc::smem_u32(a_lo), ks, kTileVec),
-                          tqtc::sw128_desc_kstep(tqtc::smem_u32(s_op), ks, D), ids, true);
-      tqtc::mma_commit(&mb_s[g]);
-    }
-    if (valid && ok_y && c4 == 0)
-      p.norms[row * p.out_stride] =
-          make_float2(nrm, p.sign_res ? (rr + xrr[g][1][r4]) * (1.f / D) : sqrtf(rr + xrr[g][1][r4]));
-    const bool ok = ok_y && tqtc::mbar_wait(&mb_s[g], ph_s, kWaitLimit);
-    ph_s ^= 1;
-    tqtc::fence_after_sync();
-    if (!ok || !ok_x) s_fail[g] = 1;
-    // the products have read the operand buffer: it takes the group's next tile
-    if (gt == 0 && ok && tile + tstep < n_tiles) issue_x(tile + tstep);
-    // sign bits of S r: complemented fp32 sign bits, one funnel shift each
-    // (an exact -0 projection reads as negative, within the sign tolerance)
-    {
-      if constexpr (D == 128 && SPLIT) {   // both loads under one wait (the key launches)
-        float val[2][32];
-        tqtc::tmem_ld32x2(tm + tm_lane + 64 * c4, tm + tm_lane + 64 * c4 + 32, val[0], val[1]);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t w = 0;
-#pragma unroll
-          for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[c][b]), w, 1);
-          if (row < p.n) p.signs[row * p.out_stride * NJ + 2 * c4 + c] = ok ? ~w : 0u;
+      if (!ok || !ok_x) s_fail[g] = 1;
+      // the products have read the operand buffer: it takes the group's next tile
+      if (gt == 0 && ok && tile + tstep < n_tiles) issue_x(tile + tstep);
+      // sign bits of S r: complemented fp32 sign bits, one funnel shift each
+      // (an exact -0 projection reads as negative, within the sign tolerance)
+      {
+        if constexpr (D == 128 && SPLIT) {   // both loads under one wait (the key launches)
+          float val[2][32];
+          tqtc::tmem_ld32x2(tm + tm_lane + 64 * c4, tm + tm_lane + 64 * c4 + 32, val[0], val[1]);
+  #pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t w = 0;
+  #pragma unroll
+            for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[c][b]), w, 1);
+            if (row < p.n) p.signs[row * p.out_stride * NJ + 2 * c4 + c] = ok ? ~w : 0u;
+          }
+        } else {
+  #pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            float val[32];
+            tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * c, val);
+            uint32_t w = 0;
+  #pragma unroll
+            for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[b]), w, 1);
+            if (row < p.n) p.signs[row * p.out_stride * NJ + (D / 64) * c4 + c] = ok ? ~w : 0u;
+          }
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          float val[32];
-          tqtc::tmem_ld32(tm + tm_lane + (D / 2) * c4 + 32 * c, val);
-          uint32_t w = 0;
-#pragma unroll
-          for (int b = 31; b >= 0; --b) w = __funnelshift_l(__float_as_uint(val[b]), w, 1);
-          if (row < p.n) p.signs[row * p.out_stride * NJ + (D / 64) * c4 + c] = ok ? ~w : 0u;
-        }
+        if (!ok && c4 == 0 && row < p.n) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
       }
-      if (!ok && c4 == 0 && row < p.n) p.norms[row * p.out_stride] = make_float2(qnan, qnan);
     }
     tqtc::fence_before_sync();
     gsync();
@@ -1143,11 +1174,11 @@ int launch_encode_rows(const EncodeParams& p, cudaStream_t stream) {
 // Batches below this many vectors take the low-latency warp-per-vector kernel.
 constexpr int64_t kRowsKernelMinN = 16384;
 
-template <int D, int BITS, typename T, bool SPLIT>
-int launch_encode_tc(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_t stream) {
+template <int D, int BITS, typename T, bool SPLIT, bool SGN>
+int launch_encode_tc_mode(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_t stream) {
   // S, H D, 2 groups x (hi, lo): 193 KB at d = 128, 81 KB at d = 64
   const size_t smem = 2 * static_cast<size_t>(D) * D * 2 + 4 * static_cast<size_t>(kTileVec) * D * 2 + 1024;
-  auto kern = encode_tc_kernel<D, BITS, T, SPLIT>;
+  auto kern = encode_tc_kernel<D, BITS, T, SPLIT, SGN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return TQ_ECUDA;
   int dev = 0, sms = 148;
@@ -1159,6 +1190,12 @@ int launch_encode_tc(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_
   const int blocks = static_cast<int>(pairs < slots ? pairs : slots);
   kern<<<blocks, kTcThreads, smem, stream>>>(xmap, p);
   return tq::launch_status();
+}
+
+template <int D, int BITS, typename T, bool SPLIT>
+int launch_encode_tc(const EncodeParams& p, const CUtensorMap& xmap, cudaStream_t stream) {
+  if (p.sign_res) return launch_encode_tc_mode<D, BITS, T, SPLIT, true>(p, xmap, stream);
+  return launch_encode_tc_mode<D, BITS, T, SPLIT, false>(p, xmap, stream);
 }
 
 template <int D, int BITS, typename T>
