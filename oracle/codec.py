@@ -231,6 +231,23 @@ def nsn_encode(rot: Rotation, x, pos=None) -> dict:
     return e
 
 
+def nsn_append(rot: Rotation, x, pos, o) -> dict:
+    """Encode tokens x [n, d] appended to a block whose shift o [d] is already
+    fixed ([NSNQuant] §4: tokens after the block keep its statistics): RoPE
+    at pos when the handle has it, s1 = ||x~|| / sqrt(d), x' = x~ - s1 o, and
+    the codec's record of x'.  Returns the codec dict of x' plus s1 [n]."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[1]
+    if rot.rope_base and pos is not None:
+        x = apply_rope(x, np.asarray(pos), rot.rope_base)
+    s1 = np.sqrt(np.sum(x * x, axis=1)) / math.sqrt(d)
+    xp = x - s1[:, None] * np.asarray(o, dtype=np.float64)[None, :]
+    e = encode(rot, xp, None)
+    e["s1"] = s1
+    e["x_shift"] = xp
+    return e
+
+
 def dequantize_nsn(rot: Rotation, codes, signs, norm, rnorm, s1, o) -> np.ndarray:
     """x^ [n, d] = dequantize(record of x') + s1 o (space after RoPE)."""
     xp = dequantize(rot, codes, signs, norm, rnorm)

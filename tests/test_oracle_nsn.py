@@ -122,3 +122,36 @@ def test_nsn_decode_with_zero_shift_is_decode_attention():
     a = at.decode_attention_nsn(rk, rv, q, [T - 1], kc, vc, s1, zero, s1, zero, 1 / math.sqrt(d))
     b = at.decode_attention(rk, rv, q, [T - 1], kc, vc, 1 / math.sqrt(d))
     np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-11)
+
+
+def test_nsn_append_matches_block_encode():
+    """A token appended to a block with the block's own shift o is encoded as
+    the block encode does for it: appending block token t (its raw row and
+    position) reproduces token t's record and s1 exactly, and x' + s1 o
+    gives back the token after RoPE."""
+    d, l = 128, 257
+    rot, _ = oracle_rotation(d, 2, 7, rope=10000.0)
+    x = _block(l, d, 3)
+    pos = np.arange(l) + 11
+    e = codec.nsn_encode(rot, x, pos)
+    pick = np.array([0, 100, l - 1])
+    a = codec.nsn_append(rot, x[pick], pos[pick], e["o"])
+    for key in ("codes", "signs"):
+        assert np.array_equal(a[key], e[key][pick])
+    for key in ("norm", "rnorm", "s1"):
+        np.testing.assert_allclose(a[key], e[key][pick], rtol=1e-12, atol=0)
+    np.testing.assert_allclose(a["x_shift"] + a["s1"][:, None] * e["o"][None, :],
+                               apply_rope(x[pick], pos[pick], 10000.0), rtol=1e-12, atol=1e-12)
+
+
+def test_nsn_append_zero_shift_is_plain_encode():
+    """With o = 0 the appended record is the plain codec's record of x~."""
+    d = 64
+    rot, _ = oracle_rotation(d, 3, 8, rope=10000.0)
+    x = _block(5, d, 4)
+    pos = np.array([0, 3, 9, 1000, 65535])
+    a = codec.nsn_append(rot, x, pos, np.zeros(d))
+    p = codec.encode(rot, x, pos)
+    assert np.array_equal(a["codes"], p["codes"]) and np.array_equal(a["signs"], p["signs"])
+    np.testing.assert_allclose(a["norm"], p["norm"], rtol=1e-12)
+    np.testing.assert_allclose(a["s1"], np.linalg.norm(x, axis=1) / math.sqrt(d), rtol=1e-12)
