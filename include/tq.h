@@ -482,6 +482,36 @@ int tq_decode_attention_append(const tq_rotation* hk, const tq_rotation* hv,
                                float* out, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/*
+ * tq_decode_attention_nsn_append - tq_decode_attention_append over NSN
+ * records: [NSNQuant] §1 and §4 (a token after the block keeps the block's
+ * statistics).  The new key takes RoPE at q_pos[b]; each new row x~ then
+ * gets s1 = ||x~|| / sqrt(d), written to k_s1 / v_s1 at record len_b - 1,
+ * and its record is that of x' = x~ - s1 o with its sequence's o (k_o / v_o,
+ * not changed).  Then tq_decode_attention_nsn over the caches that now hold
+ * the token.
+ *   k_s1, v_s1  device float32 s1 arrays as tq_decode_attention_nsn (written
+ *               at the new records); 16-byte aligned
+ *   k_o, v_o    device [B*Hkv, d] float32 shifts (keys: after RoPE)
+ *   cache_stride  a multiple of 4 (and even)
+ *   other arguments as tq_decode_attention_append
+ * Returns TQ_OK, TQ_EINVAL (also for any of the four side arrays missing),
+ * TQ_EUNSUPPORTED, TQ_EWORKSPACE or TQ_ECUDA.
+ */
+int tq_decode_attention_nsn_append(const tq_rotation* hk, const tq_rotation* hv,
+                                   const void* q, int q_dtype,
+                                   const int64_t* q_pos, const void* k_new,
+                                   const void* v_new, uint8_t* k_codes,
+                                   uint8_t* k_signs, float* k_norms,
+                                   uint8_t* v_codes, uint8_t* v_signs,
+                                   float* v_norms, float* k_s1,
+                                   const float* k_o, float* v_s1,
+                                   const float* v_o, int64_t cache_stride,
+                                   int B, int Hq, int Hkv, int64_t T,
+                                   const int32_t* seq_lens, float scale,
+                                   float* out, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* Workspace bytes tq_decode_attention needs for these sizes (0 if invalid). */
 size_t tq_decode_workspace_size(const tq_rotation* hk, const tq_rotation* hv,
                                 int B, int Hq, int Hkv, int64_t T);

@@ -80,6 +80,10 @@ def test_bad_arguments_are_rejected_on_host():
     # fused append: missing new rows or handles rejected on the host
     assert tq._lib.tq_decode_attention_append(None, None, None, 0, None, None, None, None, None, None, None, None,
                                               None, 0, 1, 4, 1, 1, None, 0.125, None, None, 0, None) == tq.TQ_EINVAL
+    # fused NSN append: missing new rows, side arrays or handles rejected on the host
+    assert tq._lib.tq_decode_attention_nsn_append(None, None, None, 0, None, None, None, None, None, None, None, None,
+                                                  None, None, None, None, None, 4, 1, 4, 1, 1, None, 0.125, None,
+                                                  None, 0, None) == tq.TQ_EINVAL
 
 
 def test_window_binding_checks_shapes_before_any_call():

@@ -193,3 +193,91 @@ def test_nsn_decode_empty_cache(cuda_device):
                                   zo, 0)
     torch.cuda.synchronize()
     assert torch.all(out == 0)
+
+
+def _append_case(G, bits, dtype, T, seed, dev):
+    """Oracle NSN caches of the first T - 1 tokens of each block (o from
+    those tokens; token T - 1 and its s1 poisoned) and the raw rows of token
+    T - 1, in the dtype the GPU reads."""
+    from vector_quantization_b200 import tq
+    d, B, Hkv = 128, 2, 2
+    Hq, cap = G * Hkv, T + 4 - T % 4
+    rk, rv = _gpu_rot(d, bits, seed, 10000.0), _gpu_rot(d, bits, seed + 10, 0.0)
+    ork, _ = oracle_rotation(d, bits, seed, rope=10000.0)
+    orv, _ = oracle_rotation(d, bits, seed + 10)
+    kt = torch.from_numpy(_offset_rows((B, Hkv, T, d), seed + 20)).to(dtype)
+    vt = torch.from_numpy(_offset_rows((B, Hkv, T, d), seed + 30)).to(dtype)
+    k64, v64 = (a.float().numpy().astype(np.float64) for a in (kt, vt))
+    kc, ks1, ko = _nsn_caches(ork, k64[:, :, :T - 1], np.arange(T - 1), cap)
+    vc, vs1, vo = _nsn_caches(orv, v64[:, :, :T - 1], None, cap)
+    qt = torch.from_numpy(synth.heavy_tailed((B, Hq, d), seed + 40)).to(dtype)
+    return dict(rk=rk, rv=rv, ork=ork, orv=orv, k64=k64, v64=v64, kc=kc, ks1=ks1, ko=ko, vc=vc, vs1=vs1, vo=vo,
+                k_new=kt[:, :, T - 1].contiguous().to(dev), v_new=vt[:, :, T - 1].contiguous().to(dev),
+                q=qt.to(dev), q64=qt.float().numpy().astype(np.float64), B=B, Hkv=Hkv, cap=cap)
+
+
+@pytest.mark.parametrize("G,bits,dtype", [(4, 2, torch.float32), (8, 3, torch.bfloat16), (1, 1, torch.float32)])
+def test_nsn_append_against_oracle(cuda_device, G, bits, dtype):
+    """The fused NSN append writes token T - 1 from the raw rows (key after
+    RoPE, both shifted by their block's o): records and s1 against the
+    oracle's nsn_append with the same o; the output against the oracle's NSN
+    attention over all T records, the last ones the oracle's own."""
+    from vector_quantization_b200 import tq
+    T, dev, d = 600, cuda_device, 128
+    c = _append_case(G, bits, dtype, T, 100 + 3 * G + bits, dev)
+    B, Hkv = c["B"], c["Hkv"]
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    kcd, vcd = tuple(map(to, c["kc"])), tuple(map(to, c["vc"]))
+    ks1d, vs1d = to(c["ks1"]), to(c["vs1"])
+    q_pos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    out = tq.decode_attention_nsn_append(c["rk"], c["rv"], c["q"], q_pos, c["k_new"], c["v_new"], kcd, vcd, ks1d,
+                                         to(c["ko"]), vs1d, to(c["vo"]), T)
+    torch.cuda.synchronize()
+    kc, vc = tuple(np.array(a) for a in c["kc"]), tuple(np.array(a) for a in c["vc"])
+    ks1, vs1 = c["ks1"].copy(), c["vs1"].copy()
+    for side, (ot, x64, o, cache, s1, gcache, gs1, pos) in enumerate(
+            ((c["ork"], c["k64"], c["ko"], kc, ks1, kcd, ks1d, [T - 1]),
+             (c["orv"], c["v64"], c["vo"], vc, vs1, vcd, vs1d, None))):
+        for b in range(B):
+            for j in range(Hkv):
+                e = codec.nsn_append(ot, x64[b, j, T - 1:T], pos, o[b, j])
+                compare_records(ot, tuple(a[b, j, T - 1:T].cpu().numpy() for a in gcache), e)
+                np.testing.assert_allclose(gs1[b, j, T - 1].item(), e["s1"][0], rtol=2e-6, atol=0)
+                cache[0][b, j, T - 1] = codec.pack_planes(e["codes"], ot.bits)[0]
+                cache[1][b, j, T - 1] = codec.pack_bits(e["signs"])[0]
+                cache[2][b, j, T - 1] = (e["norm"][0], e["rnorm"][0])
+                s1[b, j, T - 1] = e["s1"][0]
+    ref = at.decode_attention_nsn(c["ork"], c["orv"], c["q64"], [T - 1] * B, tuple(a[:, :, :T] for a in kc),
+                                  tuple(a[:, :, :T] for a in vc), ks1[:, :, :T], c["ko"], vs1[:, :, :T], c["vo"],
+                                  1 / math.sqrt(d))
+    assert_close(out.cpu().numpy(), ref, what=f"NSN append G {G} bits {bits}")
+
+
+def test_nsn_append_equals_append_then_decode(cuda_device):
+    """Ragged lengths (T, 1, 0): the fused call's output equals
+    decode_attention_nsn over the caches it wrote, bit for bit; the empty
+    sequence's records stay as they were and its output is zero."""
+    from vector_quantization_b200 import tq
+    T, dev = 333, cuda_device
+    c = _append_case(4, 2, torch.bfloat16, T, 150, dev)
+    B = c["B"]
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    # a third sequence of length 0 next to lengths T and 1
+    pad = lambda a: np.concatenate([a, a[:1]], axis=0)
+    kcd, vcd = tuple(to(pad(a)) for a in c["kc"]), tuple(to(pad(a)) for a in c["vc"])
+    ks1d, vs1d, kod, vod = (to(pad(a)) for a in (c["ks1"], c["vs1"], c["ko"], c["vo"]))
+    before = tuple(a[2].clone() for a in kcd + vcd)
+    k_new = torch.cat([c["k_new"], c["k_new"][:1]])
+    v_new = torch.cat([c["v_new"], c["v_new"][:1]])
+    q = torch.cat([c["q"], c["q"][:1]])
+    lens = torch.tensor([T, 1, 0], dtype=torch.int32, device=dev)
+    q_pos = torch.tensor([T - 1, 0, 0], dtype=torch.int64, device=dev)
+    out_a = tq.decode_attention_nsn_append(c["rk"], c["rv"], q, q_pos, k_new, v_new, kcd, vcd, ks1d, kod, vs1d, vod,
+                                           T, seq_lens=lens)
+    out_b = tq.decode_attention_nsn(c["rk"], c["rv"], q, q_pos, kcd, vcd, ks1d, kod, vs1d, vod, T, seq_lens=lens)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, out_b)
+    assert torch.all(out_a[2] == 0)
+    for x, y in zip(before, tuple(a[2] for a in kcd + vcd)):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))   # bytes: the poisoned norms are NaN
+    assert torch.isfinite(ks1d[1, :, 0]).all() and torch.isfinite(vs1d[1, :, 0]).all()

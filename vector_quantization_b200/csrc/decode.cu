@@ -838,6 +838,8 @@ struct AppendArgs {
   int64_t T;
   const int32_t* seq_lens;   // [B] or null: every sequence holds T tokens (the new one included)
   int64_t cache_stride;
+  const float* k_o;          // NSN records: [BH][kD] shift of each sequence's keys (values: v_o), else null
+  const float* v_o;
 };
 
 template <typename T, int G, int BITS>
@@ -863,9 +865,10 @@ __global__ void __launch_bounds__(kD * G) decode_prep_kernel(const __grid_consta
   const EncodeParams& p = is_v ? pv : pk;
   const int64_t rec = sq * ap.cache_stride + len - 1;
   const int64_t pos = p.rope ? a.q_pos[b] : 0;
+  const float* o = is_v ? ap.v_o : ap.k_o;
   encode_vec_core<kD, BITS, T>(p, i, static_cast<const T*>(p.x) + sq * p.ld, rec, pos, gbuf[gi], gred[gi],
                                [gi] { asm volatile("bar.sync %0, %1;\n" ::"r"(1 + gi), "r"(kD) : "memory"); },
-                               [&](int k) { return __ldg(p.st + k * kD + i); });
+                               [&](int k) { return __ldg(p.st + k * kD + i); }, o ? o + sq * kD : nullptr);
 }
 
 // One block of G groups of kD threads per (sequence b, KV head); group h is
@@ -1287,10 +1290,14 @@ struct AppendIn {
   int64_t cache_stride;
   int64_t T;
   const int32_t* seq_lens;
+  float* k_s1;        // NSN records (all four set, or all null): s1 of the new tokens go here,
+  float* v_s1;        // and the new rows are shifted by their sequence's o before encoding
+  const float* k_o;
+  const float* v_o;
 };
 
 EncodeParams append_params(const tq_rotation* h, const void* x, int BH, int rope, uint8_t* codes, uint8_t* signs,
-                           float* norms) {
+                           float* norms, float* s1) {
   EncodeParams p{};
   p.x = x;
   p.n = BH;
@@ -1301,6 +1308,7 @@ EncodeParams append_params(const tq_rotation* h, const void* x, int BH, int rope
   p.signs = reinterpret_cast<uint32_t*>(signs);
   p.norms = reinterpret_cast<float2*>(norms);
   p.out_stride = 1;
+  p.nsn_s1 = s1;
   fill_handle_fields(p, h);
   return p;
 }
@@ -1318,9 +1326,11 @@ int qprep_g(int G, int BH, const QPrepArgs<T>& a, const AppendIn* app, const tq_
 #undef TQ_QPREP
     return TQ_EUNSUPPORTED;
   }
-  const EncodeParams pk = append_params(hk, app->k_new, BH, a.rope, app->k_codes, app->k_signs, app->k_norms);
-  const EncodeParams pv = append_params(app->hv, app->v_new, BH, 0, app->v_codes, app->v_signs, app->v_norms);
-  const AppendArgs ap{BH, app->T, app->seq_lens, app->cache_stride};
+  const EncodeParams pk =
+      append_params(hk, app->k_new, BH, a.rope, app->k_codes, app->k_signs, app->k_norms, app->k_s1);
+  const EncodeParams pv =
+      append_params(app->hv, app->v_new, BH, 0, app->v_codes, app->v_signs, app->v_norms, app->v_s1);
+  const AppendArgs ap{BH, app->T, app->seq_lens, app->cache_stride, app->k_o, app->v_o};
   const unsigned blocks = static_cast<unsigned>(BH + (2 * BH + G - 1) / G);
 #define TQ_PREP(GG) return launch_pdl(decode_prep_kernel<T, GG, BITS>, dim3(blocks), dim3(kD * GG), 0, s, a, ap, pk, pv)
   switch (G) {
@@ -1522,7 +1532,10 @@ int decode_impl(const tq_rotation* hk, const tq_rotation* hv, const void* q, int
   float* partial = reinterpret_cast<float*>(ws + align256(frag_bytes(BH, G)) + align256(kconst_bytes(BH)));
   // NSN record mode: all four side arrays, decode over the packed cache only
   const bool nsn = k_s1 != nullptr;
-  if (nsn && (!k_o || !v_s1 || !v_o || R > 0 || partial_out || app)) return TQ_EINVAL;
+  if (nsn && (!k_o || !v_s1 || !v_o || R > 0 || partial_out)) return TQ_EINVAL;
+  if (app && (app->k_s1 != (nsn ? k_s1 : nullptr) || app->v_s1 != (nsn ? v_s1 : nullptr) ||
+              app->k_o != (nsn ? k_o : nullptr) || app->v_o != (nsn ? v_o : nullptr)))
+    return TQ_EINVAL;   // the appended records take the same side arrays as the decode
   float* qo = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(partial) +
                                        align256(static_cast<size_t>(BH) * n_slots * G * partial_rec<true>() *
                                                 sizeof(float)));
@@ -1642,6 +1655,27 @@ extern "C" int tq_decode_attention_nsn(const tq_rotation* hk, const tq_rotation*
                      nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, nullptr, workspace,
                      workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end, nullptr, k_s1, k_o,
                      v_s1, v_o);
+}
+
+extern "C" int tq_decode_attention_nsn_append(const tq_rotation* hk, const tq_rotation* hv, const void* q,
+                                              int q_dtype, const int64_t* q_pos, const void* k_new,
+                                              const void* v_new, uint8_t* k_codes, uint8_t* k_signs, float* k_norms,
+                                              uint8_t* v_codes, uint8_t* v_signs, float* v_norms, float* k_s1,
+                                              const float* k_o, float* v_s1, const float* v_o,
+                                              int64_t cache_stride, int B, int Hq, int Hkv, int64_t T,
+                                              const int32_t* seq_lens, float scale, float* out, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  if (!k_new || !v_new || !k_s1 || !k_o || !v_s1 || !v_o) return TQ_EINVAL;
+  if (T > 0 && (!tq::aligned16(k_s1) || !tq::aligned16(v_s1))) return TQ_EINVAL;   // copied 16 bytes at a time
+  if (cache_stride % 4) return TQ_EINVAL;   // each sequence's s1 row starts 16-byte aligned
+  const cudaEvent_t prof_begin = g_prof_begin, prof_end = g_prof_end;
+  g_prof_begin = g_prof_end = nullptr;
+  AppendIn app{k_new, v_new, hv, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride, T, seq_lens,
+               k_s1, v_s1, k_o, v_o};
+  return decode_impl(hk, hv, q, q_dtype, q_pos, k_codes, k_signs, k_norms, v_codes, v_signs, v_norms, cache_stride,
+                     nullptr, nullptr, TQ_F32, 0, 0, B, Hq, Hkv, T, seq_lens, scale, out, nullptr, workspace,
+                     workspace_bytes, static_cast<cudaStream_t>(stream), prof_begin, prof_end, &app, k_s1, k_o, v_s1,
+                     v_o);
 }
 
 extern "C" int tq_decode_attention_window(const tq_rotation* hk, const tq_rotation* hv, const void* q, int q_dtype,

@@ -26,6 +26,7 @@ struct EncodeParams {
   const int64_t* out_rows;  // [n] record of each row (scatter calls), or null: row * out_stride
   int64_t n_records;        // records in the output arrays (scatter calls: targets outside are skipped)
   int sign_res;             // sign-residual handle: norms[1] = mean |r_i| instead of ||r|| (S is the identity)
+  float* nsn_s1;            // one-vector encode with an NSN shift: s1 of each record (indexed as the norms)
   const float* dsigns;  // [D]
   const uint16_t* s_op; // S, bf16 bits in the swizzled K-major operand layout
   const uint16_t* hd_op; // tensor-core encode: H D in the same layout (fp16 bits when split, else bf16)
@@ -82,10 +83,14 @@ inline void fill_handle_fields(EncodeParams& p, const tq_rotation* h) {
 //   xr     the input row; rec its record (>= 0); pos its RoPE position
 //   buf    D floats of the group's shared memory, red 2 x D/32 floats
 //   sync   the group's barrier; scol(k) = S[i][k]
+//   nsn_o  null, or the shift o [D] of the NSN block the row is appended to
+//          ([NSNQuant] §1, §4): after RoPE, s1 = ||x~|| / sqrt(d) goes to
+//          p.nsn_s1[rec] and the codec encodes x' = x~ - s1 o
 // Every early return depends on the row alone (uniform over the group).
 template <int D, int BITS, typename T, typename Sync, typename SCol>
 __device__ __forceinline__ void encode_vec_core(const EncodeParams& p, int i, const T* xr, int64_t rec, int64_t pos,
-                                                float* buf, float (*red)[D / 32], Sync sync, SCol scol) {
+                                                float* buf, float (*red)[D / 32], Sync sync, SCol scol,
+                                                const float* nsn_o = nullptr) {
   constexpr int NW = D / 32;
   const int lane = i & 31, w = i >> 5;
   float x;
@@ -104,6 +109,21 @@ __device__ __forceinline__ void encode_vec_core(const EncodeParams& p, int i, co
     const float cs = a.x * b.x - a.y * b.y, sn = a.y * b.x + a.x * b.y;
     const float x1 = buf[j], x2 = buf[j + D / 2];
     x = i < D / 2 ? x1 * cs - x2 * sn : x2 * cs + x1 * sn;
+  }
+  if (nsn_o) {
+    // s1 from a group reduction (red[1] is free until the residual sums,
+    // several barriers later)
+    float s = x * x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) red[1][w] = s;
+    sync();
+    s = 0.f;
+#pragma unroll
+    for (int q = 0; q < NW; ++q) s += red[1][q];
+    const float s1 = sqrtf(s) * rsqrtf(static_cast<float>(D));
+    x = fmaf(-s1, __ldg(nsn_o + i), x);
+    if (i == 0) p.nsn_s1[rec] = s1;
   }
   // ||x|| and u = H D x (unnormalised, Sylvester order)
   float ss = x * x;

@@ -55,6 +55,8 @@ def _load():
         "tq_nsn_shift": (c_i, [c_p, c_p, c_i, c_i64, c_i64, c_i64, c_i64, c_i, c_p, c_p, c_p, c_p]),
         "tq_decode_attention_nsn": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
                                           c_i64, c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
+        "tq_decode_attention_nsn_append": (c_i, [c_p, c_p, c_p, c_i] + [c_p] * 13 +
+                                           [c_i64, c_i, c_i, c_i, c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
         "tq_decode_workspace_size": (c_sz, [c_p, c_p, c_i, c_i, c_i, c_i64]),
         "tq_decode_partials": (c_i, [c_p, c_p, c_p, c_i, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i64, c_i, c_i, c_i,
                                      c_i64, c_p, c_f, c_p, c_p, c_sz, c_p]),
@@ -501,6 +503,46 @@ def decode_attention_nsn(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_cache, v_
                                         _ptr(v_s1), _ptr(v_o), cap, B, Hq, Hkv, T, _ptr(lens), float(scale), _ptr(out),
                                         _ptr(workspace), workspace.numel(), _stream_ptr(stream)),
            "tq_decode_attention_nsn")
+    return out
+
+
+def decode_attention_nsn_append(rot_k: Rotation, rot_v: Rotation, q, q_pos, k_new, v_new, k_cache, v_cache, k_s1, k_o,
+                                v_s1, v_o, T: int, *, seq_lens=None, scale: float | None = None, out=None,
+                                workspace=None, stream=None):
+    """decode_attention_append over NSN records: each new row (the key after
+    RoPE at q_pos[b]) is shifted by its sequence's o (k_o, v_o [B, Hkv, d],
+    not changed) and its s1 written into k_s1 / v_s1 [B, Hkv, cap] next to
+    its record; then decode_attention_nsn over the first T (seq_lens[b])
+    records.  Returns out [B, Hq, d] float32."""
+    import torch
+    B, Hq, d = q.shape
+    kc, ks, kn = k_cache
+    vc, vs, vn = v_cache
+    Hkv, cap = kc.shape[1], kc.shape[2]
+    for t in (kc, ks, kn, vc, vs, vn, k_s1, k_o, v_s1, v_o):
+        if not t.is_contiguous():
+            raise ValueError("cache and NSN arrays must be contiguous")
+    if k_s1.shape[-1] != cap or v_s1.shape[-1] != cap or k_o.numel() != B * Hkv * d or v_o.numel() != B * Hkv * d:
+        raise ValueError("s1 arrays must be [B, Hkv, cap] and shifts [B, Hkv, d]")
+    if k_new.dtype != q.dtype or v_new.dtype != q.dtype:
+        raise ValueError("k_new and v_new must have the query's dtype")
+    if k_new.numel() != B * Hkv * d or v_new.numel() != B * Hkv * d:
+        raise ValueError("k_new and v_new must hold B * Hkv rows of d")
+    q, k_new, v_new = q.contiguous(), k_new.contiguous(), v_new.contiguous()
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(d))
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(rot_k, rot_v, B, Hq, Hkv, T)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    lens = _seq_lens(seq_lens, B, q.device)
+    _check(_lib.tq_decode_attention_nsn_append(rot_k.handle, rot_v.handle, _ptr(q), _dtype_code(q), _ptr(q_pos),
+                                               _ptr(k_new), _ptr(v_new), _ptr(kc), _ptr(ks), _ptr(kn), _ptr(vc),
+                                               _ptr(vs), _ptr(vn), _ptr(k_s1), _ptr(k_o), _ptr(v_s1), _ptr(v_o), cap,
+                                               B, Hq, Hkv, T, _ptr(lens), float(scale), _ptr(out), _ptr(workspace),
+                                               workspace.numel(), _stream_ptr(stream)),
+           "tq_decode_attention_nsn_append")
     return out
 
 
