@@ -168,3 +168,28 @@ def heavy_tailed_torch(shape, seed, device, n_outliers: int = 4,
         y = torch.randn((e - s, T, d), generator=gen, device=device, dtype=torch.float32)
         x[s:e] = (y * scale[s:e]).to(dtype)
     return x.view(*lead, T, d) if lead else x.view(T, d)
+
+
+def lognormal_channels_torch(shape, seed, device, sigma: float = 0.5, p_outlier: float = 0.02,
+                             outlier_scale: float = 15.0, dtype=None):
+    """Device version of :func:`lognormal_channels` (different random stream):
+    per-(group, channel) LogNormal(0, sigma) scales, x outlier_scale with
+    probability ``p_outlier``, drawn on the host; the N(0, 1) rows are drawn
+    on ``device`` with a seeded ``torch.Generator``."""
+    import torch
+    dtype = torch.bfloat16 if dtype is None else dtype
+    *lead, T, d = tuple(shape)
+    n_groups = int(np.prod(lead)) if lead else 1
+    g = _rng([*np.atleast_1d(seed).tolist(), 0x109B])
+    scale = np.exp(sigma * g.standard_normal((n_groups, 1, d)))
+    scale = scale * np.where(g.random((n_groups, 1, d)) < p_outlier, outlier_scale, 1.0)
+    scale = torch.as_tensor(scale.astype(np.float32), device=device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(np.random.SeedSequence([*np.atleast_1d(seed).tolist(), 0x7012]).generate_state(1)[0]))
+    x = torch.empty((n_groups, T, d), dtype=dtype, device=device)
+    chunk = max(1, (1 << 28) // max(1, T * d))
+    for s in range(0, n_groups, chunk):
+        e = min(n_groups, s + chunk)
+        y = torch.randn((e - s, T, d), generator=gen, device=device, dtype=torch.float32)
+        x[s:e] = (y * scale[s:e]).to(dtype)
+    return x.view(*lead, T, d) if lead else x.view(T, d)

@@ -210,6 +210,39 @@ def test_encode_70b_slice_full_size_sampled(cuda_device):
         del x, out
 
 
+def test_encode_esm2_cache_full_size_sampled(cuda_device):
+    """The bench's ESM-2-650M-shaped cache encode at full size: 33 layers x
+    [8, 20, 1024, 64] bf16 keys (RoPE at the token's position) and values,
+    2+1 bits, each as one launch like the bench (5.4M vectors, the d = 64
+    tensor-core encode at two CTAs per SM), with the config's log-normal
+    channel law.  Sampled rows (tile edges, the last rows, a seeded random
+    set) against the oracle over the same bf16 inputs."""
+    from vector_quantization_b200 import tq
+    c = synth.CONFIGS["esm2_650m_encoder"]
+    L, B, H, T, d, seed = c["layers"], c["batch"], c["heads"], c["tokens"], c["head_dim"], c["seed"]
+    dev = cuda_device_of()
+    n = L * B * H * T
+    rng = np.random.default_rng([seed, 78])
+    rows = np.unique(np.concatenate([
+        np.array([0, 1, 127, 128, 129, 255, 256, T - 1, T, T + 1, n - 129, n - 128, n - 2, n - 1]),
+        rng.integers(0, n, size=1500)]))
+    for apply_rope, tag in ((True, 1), (False, 2)):
+        rnd = synth.rotation_randomness(d, [seed, 9, tag])
+        g = tq.Rotation(d, 2, rnd, rope_base=c["rope_base"] if apply_rope else 0.0, rope_max_pos=T)
+        o = ro.build_rotation(d, 2, rnd, rope_base=c["rope_base"] if apply_rope else 0.0)
+        x = synth.lognormal_channels_torch((L * B * H, T, d), [seed, 9, tag + 2], dev).reshape(n, d)
+        out = tq.empty_records(g, (n,), dev)
+        kw = dict(apply_rope=True, pos_period=T) if apply_rope else {}
+        tq.quantize_kv(g, x, out=out, **kw)
+        torch.cuda.synchronize()
+        idx = torch.from_numpy(rows).to(dev)
+        xs = x.index_select(0, idx).float().cpu().numpy()
+        gpu = tuple(t.reshape(n, -1).index_select(0, idx).cpu().numpy() for t in out)
+        _, _, _, enc = oracle_records(o, xs, (rows % T).astype(np.int64) if apply_rope else None)
+        compare_records(o, gpu, enc)
+        del x, out
+
+
 @pytest.mark.parametrize("n", [1, 128, 256, 300])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_quantize_kv_pair_equals_two_calls(cuda_device, n, dtype):
