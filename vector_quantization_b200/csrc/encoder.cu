@@ -591,8 +591,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
   __shared__ int s_fail;
   __shared__ float s_inv_lam[2][kTcQ];        // per query row: 1 / range scale of q~ (0) and S q~ (1)
   __shared__ float s_mx[4][kTcQ];             // per key quarter, query row: tile maximum of the logits
-  __shared__ float2 s_kf[2][kTcKeys];         // per tile buffer, key: (||k||, ||r_k|| qjl_k) x score scale
-  __shared__ float4 s_vf[2][kTcKeys];         // per tile buffer, key: (||v|| w_0, ||v|| w_1, ||r_v||, 0)
+  __shared__ __align__(16) float2 s_kf[2][kTcKeys];   // per tile buffer, key: (||k||, ||r_k|| qjl_k) x score scale
+  __shared__ __align__(16) float s_vf[3][2][kTcKeys];  // per factor, tile buffer, key: ||v|| w_0, ||v|| w_1, ||r_v||
   uint8_t* base = raw + ((1024 - (tqtc::smem_u32(raw) & 1023)) & 1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kq = warp >> 2;                   // key quarter of this thread in the softmax
@@ -738,7 +738,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
       const float2 kn = reinterpret_cast<const float2*>(s0 + kTcKeys * (CB + SB))[tid];
       const float2 vn = reinterpret_cast<const float2*>(s0 + HALF + kTcKeys * (CB + SB))[tid];
       s_kf[t & 1][tid] = make_float2(kn.x * p.score_scale, kn.y * p.qjl_k * p.score_scale);
-      s_vf[t & 1][tid] = make_float4(vn.x * p.walsh_v[0], vn.x * p.walsh_v[1], vn.y, 0.f);
+      s_vf[0][t & 1][tid] = vn.x * p.walsh_v[0];
+      s_vf[1][t & 1][tid] = vn.x * p.walsh_v[1];
+      s_vf[2][t & 1][tid] = vn.y;
     }
   };
 
@@ -863,12 +865,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
       tqtc::tmem_ld8x3(dcol, dcol + 32 * (P - 1), dcol + 32 * P, d0, d1, dzv);
       const float iq = s_inv_lam[0][row], iz = s_inv_lam[1][row];
       const float wq0 = p.walsh_k[0] * iq, wq1 = p.walsh_k[1] * iq;
+      const float2 wq0_2 = make_float2(wq0, wq0), wq1_2 = make_float2(wq1, wq1), iz_2 = make_float2(iz, iz);
+      // two keys per fp32x2 instruction (the same roundings as one key at a time)
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float2 kf = s_kf[it & 1][8 * kq + k];
-        float c = wq0 * d0[k];
-        if constexpr (P == 2) c = fmaf(wq1, d1[k], c);
-        lg[k] = fmaf(kf.x, c, kf.y * iz * dzv[k]);
+      for (int k = 0; k < 8; k += 2) {
+        const float4 kf = *reinterpret_cast<const float4*>(&s_kf[it & 1][8 * kq + k]);   // keys k, k + 1
+        float2 c = __fmul2_rn(wq0_2, make_float2(d0[k], d0[k + 1]));
+        if constexpr (P == 2) c = __ffma2_rn(wq1_2, make_float2(d1[k], d1[k + 1]), c);
+        const float2 zt = __fmul2_rn(__fmul2_rn(make_float2(kf.y, kf.w), iz_2), make_float2(dzv[k], dzv[k + 1]));
+        const float2 l2 = __ffma2_rn(make_float2(kf.x, kf.z), c, zt);
+        lg[k] = l2.x;
+        lg[k + 1] = l2.y;
       }
     }
     if (nv < kTcKeys) {
@@ -909,15 +916,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) encoder_tc_kernel(const __grid_
     }
     // ---- probabilities -> value-product operands (row `row`, keys 8 kq .. + 7)
     {
-      float xc[P][8], xz[8];
+      float xc[P][8], xz[8], pk[8];
+      const float2 nm = make_float2(-m_run, -m_run);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float pk = lg[k] == -INFINITY ? 0.f : exp2_approx(lg[k] - m_run);
-        l_run += pk;
-        const float4 vf = s_vf[it & 1][8 * kq + k];
-        xc[0][k] = pk * vf.x;
-        if constexpr (P == 2) xc[P - 1][k] = pk * vf.y;
-        xz[k] = pk * vf.z;
+      for (int k = 0; k < 8; k += 2) {   // two keys per fp32x2 instruction
+        const float2 e = __fadd2_rn(make_float2(lg[k], lg[k + 1]), nm);
+        pk[k] = lg[k] == -INFINITY ? 0.f : exp2_approx(e.x);
+        pk[k + 1] = lg[k + 1] == -INFINITY ? 0.f : exp2_approx(e.y);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) l_run += pk[k];
+#pragma unroll
+      for (int f = 0; f < 3; ++f) {
+        if (P == 1 && f == 1) continue;
+        float* dst = f == 2 ? xz : xc[f < P ? f : 0];
+#pragma unroll
+        for (int k = 0; k < 8; k += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(&s_vf[f][it & 1][8 * kq + k]);
+          const float2 a = __fmul2_rn(make_float2(pk[k], pk[k + 1]), make_float2(v.x, v.y));
+          const float2 b = __fmul2_rn(make_float2(pk[k + 2], pk[k + 3]), make_float2(v.z, v.w));
+          dst[k] = a.x;
+          dst[k + 1] = a.y;
+          dst[k + 2] = b.x;
+          dst[k + 3] = b.y;
+        }
       }
       uint4 hi, lo;
 #pragma unroll
