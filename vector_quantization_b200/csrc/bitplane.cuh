@@ -75,6 +75,20 @@ __device__ __forceinline__ void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], ui
 constexpr int kBiasedZero = 0x4B400000;
 __device__ __forceinline__ float biased_to_float(int b) { return __int_as_float(b) - 12582912.0f; }
 
+// Two biased digit sums at once (fp32x2: the same rounding as two calls).
+__device__ __forceinline__ float2 biased_to_float2(int a, int b) {
+  return __fadd2_rn(make_float2(__int_as_float(a), __int_as_float(b)), make_float2(-12582912.0f, -12582912.0f));
+}
+
+// digits_to_float of two rows at once: digit k of row 0 in a[k], of row 1 in b[k].
+__device__ __forceinline__ float2 digits_to_float2(const int (&a)[4], const int (&b)[4]) {
+  const float2 s = make_float2(256.f, 256.f);
+  float2 f = biased_to_float2(a[3], b[3]);
+  f = __ffma2_rn(f, s, biased_to_float2(a[2], b[2]));
+  f = __ffma2_rn(f, s, biased_to_float2(a[1], b[1]));
+  return __ffma2_rn(f, s, biased_to_float2(a[0], b[0]));
+}
+
 // d0 + 2^8 d1 + 2^16 d2 + 2^24 d3 in fp32 from four biased digit sums.
 __device__ __forceinline__ float digits_to_float(int b0, int b1, int b2, int b3) {
   float f = biased_to_float(b3);

@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   const int gid = lane >> 2, tig = lane & 3;
   const int bh = blockIdx.y;
   const int split = blockIdx.x;
-  const uint32_t one_h = p.one_h, one_b = p.one_b;
+  const uint32_t one_b = p.one_b;
   // this sequence's length: T, or its own entry of seq_lens (a value outside
   // 0..T makes every output of the sequence NaN)
   int64_t T_seq = p.T;
@@ -271,6 +271,15 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
   // the per-head scales and constants in registers.
   constexpr int MG = KeyGroups<BITS>::MG;
   constexpr int NTK = 2 * NT;
+  // fp32x2 (two rows or two tokens per instruction, the same roundings) for
+  // the key-side recombination and the softmax, and for the value weights:
+  // chosen per instance by measurement of the split launch (Llama-8B-shaped
+  // layer at G = 4, the 70B-shaped slice at G = 8): 2 bits G 4 the same with
+  // the first, 4 % slower with the second; 3 bits G 4 3.6 % faster with the
+  // second alone, slower with the first; 2 bits G 8 2.6 % faster with both;
+  // 1 bit G 4 1 % slower with the first
+  constexpr bool kPackKS = BITS == 2;
+  constexpr bool kPackV = BITS == 3 || G == 8;
   __shared__ uint2 s_qf[MG][NTK][32];
   float4 kc[NT];
   float qo[NT];   // NSN: score_scale <q', o_k> of head tig + 4 nt
@@ -370,19 +379,42 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
         }
       }
     }
+    if constexpr (kPackKS) {
+      // both rows (tokens gid, gid + 8) at once on fp32x2 instructions
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+      for (int nt = 0; nt < NT; ++nt) {
+        const int c0[4] = {accc[2 * nt][0], accc[2 * nt][1], accc[2 * nt + 1][0], accc[2 * nt + 1][1]};
+        const int c1[4] = {accc[2 * nt][2], accc[2 * nt][3], accc[2 * nt + 1][2], accc[2 * nt + 1][3]};
+        const int z0[4] = {accs[2 * nt][0], accs[2 * nt][1], accs[2 * nt + 1][0], accs[2 * nt + 1][1]};
+        const int z1[4] = {accs[2 * nt][2], accs[2 * nt][3], accs[2 * nt + 1][2], accs[2 * nt + 1][3]};
+        const float2 code = __ffma2_rn(digits_to_float2(c0, c1), make_float2(kc[nt].x, kc[nt].x),
+                                       make_float2(-kc[nt].y, -kc[nt].y));
+        const float2 sgn = __ffma2_rn(digits_to_float2(z0, z1), make_float2(kc[nt].z, kc[nt].z),
+                                      make_float2(-kc[nt].w, -kc[nt].w));
+        float2 l = __ffma2_rn(make_float2(knorm[0].x, knorm[1].x), code,
+                              __fmul2_rn(make_float2(knorm[0].y, knorm[1].y), sgn));
+        if constexpr (NSN) {
+          const float* s1 = reinterpret_cast<const float*>(stg + S1OFF);
+          l = __ffma2_rn(make_float2(s1[gid], s1[gid + 8]), make_float2(qo[nt], qo[nt]), l);
+        }
+        logit[nt][0] = gid < nv ? l.x : -INFINITY;
+        logit[nt][1] = gid + 8 < nv ? l.y : -INFINITY;
+      }
+    } else {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float code = fmaf(digits_to_float(accc[2 * nt][2 * e], accc[2 * nt][2 * e + 1],
-                                                accc[2 * nt + 1][2 * e], accc[2 * nt + 1][2 * e + 1]),
-                                kc[nt].x, -kc[nt].y);
-        const float sgn = fmaf(digits_to_float(accs[2 * nt][2 * e], accs[2 * nt][2 * e + 1],
-                                               accs[2 * nt + 1][2 * e], accs[2 * nt + 1][2 * e + 1]),
-                               kc[nt].z, -kc[nt].w);
-        float l = fmaf(knorm[e].x, code, knorm[e].y * sgn);
-        if constexpr (NSN) l = fmaf(reinterpret_cast<const float*>(stg + S1OFF)[gid + 8 * e], qo[nt], l);
-        logit[nt][e] = gid + 8 * e < nv ? l : -INFINITY;
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float code = fmaf(digits_to_float(accc[2 * nt][2 * e], accc[2 * nt][2 * e + 1],
+                                                  accc[2 * nt + 1][2 * e], accc[2 * nt + 1][2 * e + 1]),
+                                  kc[nt].x, -kc[nt].y);
+          const float sgn = fmaf(digits_to_float(accs[2 * nt][2 * e], accs[2 * nt][2 * e + 1],
+                                                 accs[2 * nt + 1][2 * e], accs[2 * nt + 1][2 * e + 1]),
+                                 kc[nt].z, -kc[nt].w);
+          float l = fmaf(knorm[e].x, code, knorm[e].y * sgn);
+          if constexpr (NSN) l = fmaf(reinterpret_cast<const float*>(stg + S1OFF)[gid + 8 * e], qo[nt], l);
+          logit[nt][e] = gid + 8 * e < nv ? l : -INFINITY;
+        }
       }
     }
   };
@@ -415,9 +447,16 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
           }
         if (need) m_run[nt] = mx;
       }
+      if constexpr (kPackKS) {
+        const float2 x = __fadd2_rn(make_float2(logit[nt][0], logit[nt][1]), make_float2(-m_run[nt], -m_run[nt]));
+        prob[nt][0] = softmax_exp2(x.x);
+        prob[nt][1] = softmax_exp2(x.y);
+        l_run[nt] += prob[nt][0] + prob[nt][1];
+      } else {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) prob[nt][e] = softmax_exp2(logit[nt][e] - m_run[nt]);
-      l_run[nt] += prob[nt][0] + prob[nt][1];
+        for (int e = 0; e < 2; ++e) prob[nt][e] = softmax_exp2(logit[nt][e] - m_run[nt]);
+        l_run[nt] += prob[nt][0] + prob[nt][1];
+      }
     }
   };
 
@@ -474,28 +513,60 @@ __global__ void __launch_bounds__(kWarps * 32, G <= 4 ? 3 : 1) decode_split_kern
       pt[3] = __shfl_sync(0xffffffffu, prob[nt][1], srcB);
       uint32_t bc[P][2], bz[2];
       float wv[4], wr[4];
+      if constexpr (kPackV) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        wv[j] = pt[j] * vnorm[j].x;   // rows past the tile's last token: p = 0, zero-filled norms
-        wr[j] = pt[j] * vnorm[j].y;
-      }
-      // B operand: lanes of even gid feed RN(w), odd gid RN(w - RN(w)), both
-      // as bf16 pairs: one paired conversion, an FFMA by piece_m in {0, 1},
-      // one paired conversion out (|w - hi - lo| <= 2^-17 |w|).
-      auto pair2 = [&](float a, float b) -> uint32_t {
-        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-        const uint32_t hb = *reinterpret_cast<uint32_t*>(&h);
-        const float ha = __uint_as_float(hb << 16), hbf = __uint_as_float(hb & 0xFFFF0000u);
-        __nv_bfloat162 r = __floats2bfloat162_rn(fmaf(-piece_m, ha, a), fmaf(-piece_m, hbf, b));
-        return *reinterpret_cast<uint32_t*>(&r);
-      };
+        for (int j = 0; j < 4; j += 2) {   // rows past the tile's last token: p = 0, zero-filled norms
+          const float2 pp = make_float2(pt[j], pt[j + 1]);
+          const float2 a = __fmul2_rn(pp, make_float2(vnorm[j].x, vnorm[j + 1].x));
+          const float2 b = __fmul2_rn(pp, make_float2(vnorm[j].y, vnorm[j + 1].y));
+          wv[j] = a.x;
+          wv[j + 1] = a.y;
+          wr[j] = b.x;
+          wr[j + 1] = b.y;
+        }
+        // B operand: lanes of even gid feed RN(w), odd gid RN(w - RN(w)), both
+        // as bf16 pairs: one paired conversion, an FFMA by piece_m in {0, 1},
+        // one paired conversion out (|w - hi - lo| <= 2^-17 |w|).
+        const float2 npm = make_float2(-piece_m, -piece_m);
+        auto pair2 = [&](float2 w) -> uint32_t {
+          __nv_bfloat162 h = __floats2bfloat162_rn(w.x, w.y);
+          const uint32_t hb = *reinterpret_cast<uint32_t*>(&h);
+          const float2 r = __ffma2_rn(npm, make_float2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u)), w);
+          __nv_bfloat162 rb = __floats2bfloat162_rn(r.x, r.y);
+          return *reinterpret_cast<uint32_t*>(&rb);
+        };
 #pragma unroll
-      for (int pl = 0; pl < P; ++pl) {
-        bc[pl][0] = pair2(p.walsh_v[pl] * wv[0], p.walsh_v[pl] * wv[1]);
-        bc[pl][1] = pair2(p.walsh_v[pl] * wv[2], p.walsh_v[pl] * wv[3]);
+        for (int pl = 0; pl < P; ++pl) {
+          const float2 wp = make_float2(p.walsh_v[pl], p.walsh_v[pl]);
+          bc[pl][0] = pair2(__fmul2_rn(wp, make_float2(wv[0], wv[1])));
+          bc[pl][1] = pair2(__fmul2_rn(wp, make_float2(wv[2], wv[3])));
+        }
+        bz[0] = pair2(make_float2(wr[0], wr[1]));
+        bz[1] = pair2(make_float2(wr[2], wr[3]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          wv[j] = pt[j] * vnorm[j].x;   // rows past the tile's last token: p = 0, zero-filled norms
+          wr[j] = pt[j] * vnorm[j].y;
+        }
+        // B operand: lanes of even gid feed RN(w), odd gid RN(w - RN(w)), both
+        // as bf16 pairs: one paired conversion, an FFMA by piece_m in {0, 1},
+        // one paired conversion out (|w - hi - lo| <= 2^-17 |w|).
+        auto pair2 = [&](float a, float b) -> uint32_t {
+          __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+          const uint32_t hb = *reinterpret_cast<uint32_t*>(&h);
+          const float ha = __uint_as_float(hb << 16), hbf = __uint_as_float(hb & 0xFFFF0000u);
+          __nv_bfloat162 r = __floats2bfloat162_rn(fmaf(-piece_m, ha, a), fmaf(-piece_m, hbf, b));
+          return *reinterpret_cast<uint32_t*>(&r);
+        };
+#pragma unroll
+        for (int pl = 0; pl < P; ++pl) {
+          bc[pl][0] = pair2(p.walsh_v[pl] * wv[0], p.walsh_v[pl] * wv[1]);
+          bc[pl][1] = pair2(p.walsh_v[pl] * wv[2], p.walsh_v[pl] * wv[3]);
+        }
+        bz[0] = pair2(wr[0], wr[1]);
+        bz[1] = pair2(wr[2], wr[3]);
       }
-      bz[0] = pair2(wr[0], wr[1]);
-      bz[1] = pair2(wr[2], wr[3]);
       // unrounded weight sums for the offset mu_p sum B (hi + lo differ from
       // w by at most 2^-17 |w|, far inside the output tolerance)
       sbc[nt] += (wv[0] + wv[1]) + (wv[2] + wv[3]);
