@@ -44,9 +44,9 @@ UNIT = "tokens/s"
 
 
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of decode_split_kernel<2,4>
-# per cached token (235,722,240 + 5,576,448 B over 16*8*16384 tokens), or None
+# per cached token (235,720,704 + 5,453,056 B over 16*8*16384 tokens), or None
 # when the kernel has changed since that capture.
-SPLIT_TRAFFIC_PER_TOKEN = (235_722_240 + 5_576_448) / (16 * 8 * 16384)
+SPLIT_TRAFFIC_PER_TOKEN = (235_720_704 + 5_453_056) / (16 * 8 * 16384)
 
 EXTRAS = ("encode_70b_slice", "decode_70b_slice", "encoder_esm2_layer", "search_1m_d1536", "decode_llama8b_layer_3p1",
           "decode_llama8b_layer_window", "tiny_d128_t1024", "encode_esm2_33_layers", "memory_esm2",
