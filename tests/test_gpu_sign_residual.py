@@ -134,6 +134,73 @@ def test_sign_mode_decode_parity(cuda_device, bits, G):
             assert_close(out[b, h:h + 1], ref, what=f"b={b} h={h}")
 
 
+def test_sign_mode_window_decode_parity(cuda_device):
+    """The packed part in sign-residual records plus a full-precision window
+    (fp32 keys before RoPE, token i at position T + i): against textbook
+    attention over the oracle's dequantized rows followed by the window's."""
+    from vector_quantization_b200 import tq
+    dev = cuda_device
+    d, B, Hkv, G, T, R, W = 128, 2, 2, 4, 500, 37, 64
+    gk, ok = _rots(d, 2, 431, rope=10000.0)
+    gv, ov = _rots(d, 2, 432)
+    xk = synth.heavy_tailed((B, Hkv, T, d), 433)
+    xv = synth.heavy_tailed((B, Hkv, T, d), 434)
+    kc, ek = _oracle_cache(ok, xk, np.arange(T))
+    vc, ev = _oracle_cache(ov, xv)
+    kw = synth.heavy_tailed((B, Hkv, W, d), 435).astype(np.float32)
+    vw = synth.heavy_tailed((B, Hkv, W, d), 436).astype(np.float32)
+    q = synth.heavy_tailed((B, Hkv * G, d), 437)
+    qpos = T + R - 1
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    out = tq.decode_attention_window(gk, gv, to(q), torch.full((B,), qpos, dtype=torch.int64, device=dev),
+                                     tuple(map(to, kc)), tuple(map(to, vc)), T, to(kw), to(vw), R)
+    torch.cuda.synchronize()
+    out = out.cpu().numpy()
+    for b in range(B):
+        for h in range(Hkv * G):
+            j = h // G
+            qr = ro.apply_rope(q[b, h:h + 1], np.array([qpos]), ok.rope_base)
+            keys = np.concatenate([_dequant(ok, ek[b, j]),
+                                   ro.apply_rope(kw[b, j, :R].astype(np.float64), T + np.arange(R), ok.rope_base)])
+            vals = np.concatenate([_dequant(ov, ev[b, j]), vw[b, j, :R].astype(np.float64)])
+            ref = at.exact_attention(qr, keys, vals, 1 / np.sqrt(d))
+            assert_close(out[b, h:h + 1], ref, what=f"window b={b} h={h}")
+
+
+def test_sign_mode_fused_append_equals_separate(cuda_device):
+    """The fused decode-step append with sign-residual handles writes the
+    same records as the scatter encode of the new rows, and the decode that
+    follows gives the same output, bit for bit."""
+    from vector_quantization_b200 import tq
+    dev = cuda_device
+    d, B, Hkv, G, T = 128, 2, 2, 4, 400
+    cap = T + 4
+    gk, _ = _rots(d, 2, 441, rope=10000.0)
+    gv, _ = _rots(d, 2, 442)
+    kc = tq.quantize_kv(gk, synth.heavy_tailed_torch((B, Hkv, cap, d), [443, 1], dev), apply_rope=True,
+                        pos_period=cap)
+    vc = tq.quantize_kv(gv, synth.heavy_tailed_torch((B, Hkv, cap, d), [443, 2], dev))
+    kc = tuple(a.view(B, Hkv, cap, -1) for a in kc)
+    vc = tuple(a.view(B, Hkv, cap, -1) for a in vc)
+    q = synth.heavy_tailed_torch((B, Hkv * G, d), [443, 3], dev)
+    k_new = synth.heavy_tailed_torch((B, Hkv, d), [443, 4], dev)
+    v_new = synth.heavy_tailed_torch((B, Hkv, d), [443, 5], dev)
+    q_pos = torch.full((B,), T - 1, dtype=torch.int64, device=dev)
+    ka, va = tuple(a.clone() for a in kc), tuple(a.clone() for a in vc)
+    seqs = torch.arange(B * Hkv, dtype=torch.int64, device=dev)
+    flat = lambda c: tuple(a.view(B * Hkv * cap, -1) for a in c)
+    tq.quantize_kv_pair_scatter(gk, k_new.view(B * Hkv, d), gv, v_new.view(B * Hkv, d), seqs * cap + T - 1,
+                                flat(ka), flat(va), pos=torch.full((B * Hkv,), T - 1, dtype=torch.int64, device=dev),
+                                apply_rope=True)
+    out_a = tq.decode_attention(gk, gv, q, q_pos, ka, va, T)
+    kb, vb = tuple(a.clone() for a in kc), tuple(a.clone() for a in vc)
+    out_b = tq.decode_attention_append(gk, gv, q, q_pos, k_new, v_new, kb, vb, T)
+    torch.cuda.synchronize()
+    for x, y in zip(ka + va, kb + vb):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+    assert torch.equal(out_a, out_b)
+
+
 @pytest.mark.parametrize("d,bits", [(64, 2), (64, 1), (128, 3)])
 def test_sign_mode_encoder_parity(cuda_device, d, bits):
     """Encoder attention (the tensor-core kernel for d = 64 and 1-2 bit codes,
