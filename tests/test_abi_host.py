@@ -130,3 +130,26 @@ def test_library_seeded_draws_reject_bad_sizes():
     assert tq._lib.tq_rotation_draws(0, 0, 1, 128, None, None, None) == tq.TQ_EINVAL
     assert tq._lib.tq_rotation_draws(128, 7, 1, 128, None, None, None) == tq.TQ_EINVAL
     assert tq._lib.tq_rotation_draws(128, 0, 1, 128, None, None, None) == tq.TQ_OK
+
+
+def test_binding_without_the_library_raises_on_import(tmp_path):
+    """A copy of the package without libtq.so: importing the binding raises
+    ImportError naming the missing library (no fallback path exists)."""
+    import os
+    import shutil
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = tmp_path / "vector_quantization_b200"
+    pkg.mkdir()
+    for name in ("__init__.py", "tq.py", "sharded.py", "build.py"):
+        shutil.copy(os.path.join(root, "vector_quantization_b200", name), pkg / name)
+    code = ("import sys; sys.path.insert(0, sys.argv[1])\n"
+            "try:\n"
+            "    import vector_quantization_b200.tq\n"
+            "except ImportError as e:\n"
+            "    print('raised', 'libtq.so' in str(e))\n"
+            "else:\n"
+            "    print('imported')\n")
+    run = subprocess.run([sys.executable, "-c", code, str(tmp_path)], capture_output=True, text=True, timeout=300)
+    assert run.stdout.strip() == "raised True", run.stdout + run.stderr
