@@ -89,6 +89,21 @@ def test_decode_no_rope(cuda_device):
     assert_close(gpu, ref)
 
 
+def test_decode_sequence_limit(cuda_device):
+    """B * Hkv sequences fill the split kernel's grid rows, which CUDA caps at
+    65535: at the cap the workspace query answers, one past it the query
+    gives 0 and the call returns TQ_EUNSUPPORTED on the host, before any
+    pointer is looked at or anything is launched."""
+    from vector_quantization_b200 import tq
+    rk, rv = _gpu_rot(2, 1, 10000.0), _gpu_rot(2, 2, 0.0)
+    assert tq.decode_workspace_size(rk, rv, 65535, 4, 1, 16) > 0
+    assert tq.decode_workspace_size(rk, rv, 65536, 4, 1, 16) == 0
+    assert tq.decode_workspace_size(rk, rv, 32768, 8, 2, 16) == 0
+    st = tq._lib.tq_decode_attention(rk.handle, rv.handle, None, 0, None, None, None, None, None, None, None, 16,
+                                     65536, 4, 1, 16, None, 0.125, None, None, 0, None)
+    assert st == tq.TQ_EUNSUPPORTED
+
+
 def test_decode_empty_cache(cuda_device):
     from vector_quantization_b200 import tq
     dev = torch.device("cuda:0")
