@@ -65,3 +65,33 @@ def test_packed_layout_ratio():
     g = {r[0]: float(r[1]) for r in read_golden("turboesm_memory.txt")}
     # the printed MB figures are rounded (47 MB: 46.5..47.5 -> 6.95..7.10x)
     assert g["baseline_MB"] / g["packed_MB"] == pytest.approx(g["ratio"], abs=0.1)
+
+
+def test_search_scores_equal_inner_products_with_dequantized_rows():
+    """The packed-record score route equals <q, x_hat> with x_hat the
+    dequantized row (the QJL estimator written as a reconstruction), for
+    the dense rotation with m = d and with m != d, at 1 and 3 bits."""
+    d, N, nq = 64, 200, 7
+    rng = np.random.default_rng(91)
+    for bits, m in ((1, 64), (3, 64), (1, 96)):
+        rot = ro.build_rotation(d, bits, synth.rotation_randomness(d, 92 + bits + m, dense=True, m=m), "dense")
+        db = rng.standard_normal((N, d))
+        qs = rng.standard_normal((nq, d))
+        e = codec.encode(rot, db)
+        codes = codec.pack_planes(e["codes"], bits)
+        signs = codec.pack_bits(e["signs"])
+        norms = np.stack([e["norm"], e["rnorm"]], 1)
+        sc = search.search_scores(rot, qs, codes, signs, norms)
+        xh = codec.dequantize(rot, e["codes"], e["signs"], e["norm"], e["rnorm"])
+        np.testing.assert_allclose(sc, qs @ xh.T, rtol=1e-10, atol=1e-10)
+
+
+def test_exact_mips_topk_matches_a_loop():
+    rng = np.random.default_rng(93)
+    db, qs = rng.standard_normal((300, 16)), rng.standard_normal((5, 16))
+    vals, ids = search.exact_mips_topk(qs, db, 10)
+    for i, q in enumerate(qs):
+        s = [float(np.dot(q, x)) for x in db]
+        order = sorted(range(len(s)), key=lambda j: (-s[j], j))[:10]
+        assert list(ids[i]) == order
+        np.testing.assert_allclose(vals[i], [s[j] for j in order], rtol=1e-12)
